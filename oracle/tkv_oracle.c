@@ -1,0 +1,464 @@
+/*
+ * tkv_oracle.c -- plain, slow CPU oracle of the thought-adaptive compressed
+ * KV-cache decode step (ThinKV-style).  TEST INFRASTRUCTURE ONLY: it is used by
+ * the test-suite, by the smoke check and by the benchmark's CPU-baseline leg; the
+ * product path never links, loads or calls it.  It shares no code with the CUDA
+ * library (its own structs, its own fp16 conversion, its own packing).
+ *
+ * What it computes, and where the pages define it:
+ *
+ *  - Thought-adaptive group quantisation ("ThinKV", section Metodologia, TBQ
+ *    paragraph: precision chosen by thought type, importance R > E > T,
+ *    tokens group-quantised per category).  Reading used here: asymmetric
+ *    integer codes of 8/4/2 bits for R/E/T, groups of 32 consecutive head_dim
+ *    elements, one fp16 scale and one fp16 zero (an offset value) per group,
+ *    for K and for V of every token; zero = min rounded down to fp16, scale =
+ *    (max - zero)/(2^b - 1) rounded up to fp16; code = round-half-even of
+ *    (x - zero)/scale in fp32, clamped to [0, 2^b-1].  Tokens whose position is
+ *    below n_protect (attention sinks / question window: "DYNTS", section 2.3,
+ *    question window never evicted) are stored as bf16.
+ *  - Paged per-precision pools with in-place slot reuse ("ThinKV", section
+ *    Implementacao do Sistema, Continuous Thinking: a block table tracks
+ *    thought type and eviction, and new tokens of the same type overwrite
+ *    evicted slots without gather-based compaction).
+ *  - Decode attention over the dequantised cache, in fp64, and accumulation of
+ *    each token's attention mass as its importance score (H2O-style cumulative
+ *    attention; "Back from the Future", problem statement; "ThinKV",
+ *    Resultados names H2O/R-KV as the baselines).
+ *  - Budgeted top-k eviction ("DYNTS", section 2.3, selection window: keep
+ *    the k highest-scoring tokens, evict the rest) followed by a stable
+ *    compaction of the block table; evicted slots go to a per-class free stack.
+ *
+ * Floating point: quantisation is done in IEEE fp32 with round-to-nearest-even
+ * and no contraction (build with -ffp-contract=off, no fast-math).  The
+ * fp32 -> fp16 directed conversions are written here from the IEEE-754
+ * definition (largest fp16 <= x, smallest fp16 >= x).  Attention, softmax and
+ * scores are fp64; output is rounded to fp32 and the score is stored as fp32.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORC_OK 0
+#define ORC_ERR_INVALID 1
+#define ORC_ERR_CAPACITY 2
+
+typedef struct {
+    int32_t B, Hkv, G, D, group, n_protect;
+    int32_t bits[4];   /* 16 (bf16), 8, 4, 2 for classes 0..3 */
+    int32_t cap[4];    /* slots per stream per class */
+    uint8_t *pool[4];  /* [S][cap[c]][rec_bytes(c)] */
+    int32_t *n, *ft, *hw;          /* [S][4] */
+    int32_t *handle[4], *pos[4], *fs[4];  /* [S][cap[c]] */
+    float *score[4];               /* [S][cap[c]] */
+} orc_state;
+
+/* ------------------------------------------------------------------ */
+/* bf16 / fp16 scalar helpers (IEEE-754 definitions)                   */
+/* ------------------------------------------------------------------ */
+static float bf16_to_f32(uint16_t h) {
+    uint32_t u = ((uint32_t)h) << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+double orc_f16_to_f64(uint16_t h) {
+    int sign = (h >> 15) & 1;
+    int e = (h >> 10) & 0x1F;
+    int m = h & 0x3FF;
+    double v;
+    if (e == 0)
+        v = ldexp((double)m, -24);
+    else if (e == 31)
+        v = m ? NAN : INFINITY;
+    else
+        v = ldexp((double)(1024 + m), e - 25);
+    return sign ? -v : v;
+}
+
+/* fp16 bit pattern of a double that is exactly representable in fp16
+ * (or +-inf). */
+static uint16_t exact_to_f16_bits(double v) {
+    uint16_t sign = (v < 0 || (v == 0 && signbit(v))) ? 0x8000 : 0;
+    double a = fabs(v);
+    if (isinf(a)) return sign | 0x7C00;
+    if (a == 0) return sign;
+    if (a < ldexp(1.0, -14)) return sign | (uint16_t)(a / ldexp(1.0, -24));
+    int E;
+    frexp(a, &E);          /* a = f * 2^E, f in [0.5, 1) */
+    int e = E - 1;         /* a in [2^e, 2^(e+1)) */
+    double mant = a / ldexp(1.0, e) - 1.0;  /* [0, 1) */
+    return sign | (uint16_t)((e + 15) << 10) | (uint16_t)(mant * 1024.0);
+}
+
+/* spacing of fp16 values at magnitude a (a finite, >= 0) */
+static double f16_quantum(double a) {
+    if (a < ldexp(1.0, -14)) return ldexp(1.0, -24);
+    int E;
+    frexp(a, &E);
+    int e = E - 1;
+    if (e > 15) e = 15;
+    return ldexp(1.0, e - 10);
+}
+
+/* largest fp16 value <= x (round toward -inf) */
+uint16_t orc_f32_to_f16_rd(float xf) {
+    double x = xf;
+    if (isnan(x)) return 0x7FFF;
+    if (isinf(x)) return x > 0 ? 0x7C00 : 0xFC00;
+    if (x == 0) return signbit(x) ? 0x8000 : 0;
+    double q = f16_quantum(fabs(x));
+    double v = floor(x / q) * q;
+    if (v > 65504.0) v = 65504.0;
+    if (v < -65504.0) v = -INFINITY;
+    if (v == 0) v = 0.0; /* floor of a tiny positive value is +0 */
+    return exact_to_f16_bits(v);
+}
+
+/* smallest fp16 value >= x (round toward +inf) */
+uint16_t orc_f32_to_f16_ru(float xf) {
+    double x = xf;
+    if (isnan(x)) return 0x7FFF;
+    if (isinf(x)) return x > 0 ? 0x7C00 : 0xFC00;
+    if (x == 0) return signbit(x) ? 0x8000 : 0;
+    double q = f16_quantum(fabs(x));
+    double v = ceil(x / q) * q;
+    if (v < -65504.0) v = -65504.0;
+    if (v > 65504.0) v = INFINITY;
+    if (v == 0) v = -0.0; /* ceil of a tiny negative value is -0 */
+    return exact_to_f16_bits(v);
+}
+
+/* ------------------------------------------------------------------ */
+/* Group quantisation and record packing                               */
+/* ------------------------------------------------------------------ */
+int orc_record_bytes(int bits, int D, int group) {
+    if (bits == 16) return 2 * D * 2;
+    int ngroups = D / group;
+    return 2 * (D * bits / 8) + 4 * ngroups * 2;
+}
+
+/* Quantise one group of n fp32 values (exact bf16 values) at `bits`. */
+void orc_quantize_group(const float *x, int n, int bits, uint16_t *scale_h,
+                        uint16_t *zero_h, uint8_t *codes) {
+    float mn = x[0], mx = x[0];
+    for (int i = 1; i < n; ++i) {
+        if (x[i] < mn) mn = x[i];
+        if (x[i] > mx) mx = x[i];
+    }
+    const int qmax = (1 << bits) - 1;
+    uint16_t z = orc_f32_to_f16_rd(mn);
+    float zf = (float)orc_f16_to_f64(z);
+    float range = mx - zf;                 /* fp32, round to nearest even */
+    float step = range / (float)qmax;      /* fp32 IEEE division */
+    uint16_t s = orc_f32_to_f16_ru(step);
+    float sf = (float)orc_f16_to_f64(s);
+    *zero_h = z;
+    *scale_h = s;
+    for (int i = 0; i < n; ++i) {
+        if (sf == 0.0f) {
+            codes[i] = 0;
+            continue;
+        }
+        float d = x[i] - zf;
+        float r = d / sf;
+        float q = nearbyintf(r);           /* round half to even (default mode) */
+        if (q < 0) q = 0;
+        if (q > (float)qmax) q = (float)qmax;
+        codes[i] = (uint8_t)q;
+    }
+}
+
+/* Pack codes little-endian within each byte: element i at bit bits*(i % (8/bits))
+ * of byte i*bits/8. */
+static void pack_codes(const uint8_t *codes, int n, int bits, uint8_t *out) {
+    int per = 8 / bits;
+    memset(out, 0, (size_t)n * bits / 8);
+    for (int i = 0; i < n; ++i)
+        out[i / per] |= (uint8_t)(codes[i] << (bits * (i % per)));
+}
+
+static void unpack_codes(const uint8_t *in, int n, int bits, uint8_t *codes) {
+    int per = 8 / bits;
+    int mask = (1 << bits) - 1;
+    for (int i = 0; i < n; ++i) codes[i] = (in[i / per] >> (bits * (i % per))) & mask;
+}
+
+static void put_u16(uint8_t *p, uint16_t v) {
+    p[0] = (uint8_t)(v & 0xFF);
+    p[1] = (uint8_t)(v >> 8);
+}
+
+static uint16_t get_u16(const uint8_t *p) { return (uint16_t)(p[0] | (p[1] << 8)); }
+
+/* Record layout (all little-endian):
+ *   bf16:  [K: D x bf16][V: D x bf16]
+ *   b-bit: [K codes: D*b/8 bytes][V codes: D*b/8 bytes]
+ *          [K scale x ngroups][K zero x ngroups][V scale x ngroups][V zero x ngroups] (fp16)
+ */
+void orc_pack_record(int bits, int D, int group, const uint16_t *k, const uint16_t *v,
+                     uint8_t *rec) {
+    if (bits == 16) {
+        for (int d = 0; d < D; ++d) put_u16(rec + 2 * d, k[d]);
+        for (int d = 0; d < D; ++d) put_u16(rec + 2 * D + 2 * d, v[d]);
+        return;
+    }
+    int ng = D / group;
+    int cb = D * bits / 8;
+    uint8_t *meta = rec + 2 * cb;
+    uint8_t codes[512];
+    float x[512];
+    for (int which = 0; which < 2; ++which) {
+        const uint16_t *src = which == 0 ? k : v;
+        uint8_t allc[512];
+        for (int g = 0; g < ng; ++g) {
+            uint16_t s, z;
+            for (int i = 0; i < group; ++i) x[i] = bf16_to_f32(src[g * group + i]);
+            orc_quantize_group(x, group, bits, &s, &z, codes);
+            memcpy(allc + g * group, codes, group);
+            put_u16(meta + (which * 2 * ng + g) * 2, s);
+            put_u16(meta + (which * 2 * ng + ng + g) * 2, z);
+        }
+        pack_codes(allc, D, bits, rec + which * cb);
+    }
+}
+
+/* Dequantise a record: x_hat = code * scale + zero, evaluated in fp64. */
+void orc_unpack_record(int bits, int D, int group, const uint8_t *rec, double *k_hat,
+                       double *v_hat) {
+    if (bits == 16) {
+        for (int d = 0; d < D; ++d) k_hat[d] = bf16_to_f32(get_u16(rec + 2 * d));
+        for (int d = 0; d < D; ++d) v_hat[d] = bf16_to_f32(get_u16(rec + 2 * D + 2 * d));
+        return;
+    }
+    int ng = D / group;
+    int cb = D * bits / 8;
+    const uint8_t *meta = rec + 2 * cb;
+    uint8_t codes[512];
+    for (int which = 0; which < 2; ++which) {
+        double *dst = which == 0 ? k_hat : v_hat;
+        unpack_codes(rec + which * cb, D, bits, codes);
+        for (int d = 0; d < D; ++d) {
+            int g = d / group;
+            double s = orc_f16_to_f64(get_u16(meta + (which * 2 * ng + g) * 2));
+            double z = orc_f16_to_f64(get_u16(meta + (which * 2 * ng + ng + g) * 2));
+            dst[d] = (double)codes[d] * s + z;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* Cache operations                                                    */
+/* ------------------------------------------------------------------ */
+static int n_streams(const orc_state *st) { return st->B * st->Hkv; }
+
+static uint8_t *record_ptr(const orc_state *st, int s, int c, int slot) {
+    size_t rb = (size_t)orc_record_bytes(st->bits[c], st->D, st->group);
+    return st->pool[c] + ((size_t)s * st->cap[c] + slot) * rb;
+}
+
+/* Append T tokens per stream.  k, v: bf16 [B][Hkv][T][D]; cls, pos: [B][T].
+ * Tokens are processed in order; a token at position < n_protect is stored in
+ * class 0 (bf16).  Slot: pop the stream's free stack for that class if it is
+ * non-empty, else take the next never-used slot; if neither exists the token
+ * is dropped and CAPACITY is reported.  A class id > 3 drops the token and
+ * reports INVALID.  New table entries start with score 0. */
+int orc_append(orc_state *st, const uint16_t *k, const uint16_t *v, const uint8_t *cls,
+               const int32_t *pos, int T) {
+    int status = ORC_OK;
+    const int D = st->D;
+    for (int b = 0; b < st->B; ++b)
+        for (int h = 0; h < st->Hkv; ++h) {
+            int s = b * st->Hkv + h;
+            for (int t = 0; t < T; ++t) {
+                int32_t p = pos[(size_t)b * T + t];
+                int c = p < st->n_protect ? 0 : cls[(size_t)b * T + t];
+                if (c < 0 || c > 3) {
+                    if (status == ORC_OK) status = ORC_ERR_INVALID;
+                    continue;
+                }
+                int32_t slot;
+                int32_t *ft = &st->ft[s * 4 + c], *hw = &st->hw[s * 4 + c];
+                if (*ft > 0) {
+                    *ft -= 1;
+                    slot = st->fs[c][(size_t)s * st->cap[c] + *ft];
+                } else if (*hw < st->cap[c]) {
+                    slot = *hw;
+                    *hw += 1;
+                } else {
+                    if (status == ORC_OK) status = ORC_ERR_CAPACITY;
+                    continue;
+                }
+                int32_t i = st->n[s * 4 + c]++;
+                size_t e = (size_t)s * st->cap[c] + i;
+                st->handle[c][e] = slot;
+                st->pos[c][e] = p;
+                st->score[c][e] = 0.0f;
+                size_t off = (((size_t)b * st->Hkv + h) * T + t) * D;
+                orc_pack_record(st->bits[c], D, st->group, k + off, v + off,
+                                record_ptr(st, s, c, slot));
+            }
+        }
+    return status;
+}
+
+/* One decode step of attention for every stream s = (b, kv head):
+ *   logit[j][t] = softmax_scale * sum_d q[b][kvh*G + j][d] * k_hat[t][d]
+ *   p = softmax over all live tokens of the stream (every class);
+ *   out[b][kvh*G + j][:] = sum_t p[j][t] * v_hat[t][:]   (fp64, stored fp32)
+ *   score[t] += sum_j p[j][t]                          (fp64 add, stored fp32)
+ * q: bf16 [B][Hkv*G][D]; out: fp32 [B][Hkv*G][D].  An empty stream gives a zero
+ * output.  If p_out is non-NULL it receives p for stream s_dbg in entry order
+ * (class 0 entries, then class 1, ...), [G][N]. */
+void orc_attend(orc_state *st, const uint16_t *q, float softmax_scale, float *out,
+                int s_dbg, double *p_out) {
+    const int D = st->D, G = st->G, S = n_streams(st);
+    const int Hq = st->Hkv * G;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int s = 0; s < S; ++s) {
+        int b = s / st->Hkv, kvh = s % st->Hkv;
+        int N = 0;
+        for (int c = 0; c < 4; ++c) N += st->n[s * 4 + c];
+        double *qd = malloc(sizeof(double) * G * D);
+        double *logit = malloc(sizeof(double) * G * (N > 0 ? N : 1));
+        double *vh = malloc(sizeof(double) * (size_t)(N > 0 ? N : 1) * D);
+        double *kh = malloc(sizeof(double) * D);
+        float **sc = malloc(sizeof(float *) * (N > 0 ? N : 1));
+        for (int j = 0; j < G; ++j)
+            for (int d = 0; d < D; ++d)
+                qd[j * D + d] = bf16_to_f32(q[((size_t)b * Hq + kvh * G + j) * D + d]);
+        int t = 0;
+        for (int c = 0; c < 4; ++c)
+            for (int i = 0; i < st->n[s * 4 + c]; ++i, ++t) {
+                size_t e = (size_t)s * st->cap[c] + i;
+                orc_unpack_record(st->bits[c], D, st->group,
+                                  record_ptr(st, s, c, st->handle[c][e]), kh, vh + (size_t)t * D);
+                sc[t] = &st->score[c][e];
+                for (int j = 0; j < G; ++j) {
+                    double acc = 0;
+                    for (int d = 0; d < D; ++d) acc += qd[j * D + d] * kh[d];
+                    logit[(size_t)j * N + t] = acc * (double)softmax_scale;
+                }
+            }
+        double *incr = calloc((size_t)(N > 0 ? N : 1), sizeof(double));
+        for (int j = 0; j < G; ++j) {
+            double *o = calloc(D, sizeof(double));
+            if (N > 0) {
+                double m = -INFINITY;
+                for (t = 0; t < N; ++t) m = fmax(m, logit[(size_t)j * N + t]);
+                double l = 0;
+                for (t = 0; t < N; ++t) l += exp(logit[(size_t)j * N + t] - m);
+                for (t = 0; t < N; ++t) {
+                    double p = exp(logit[(size_t)j * N + t] - m) / l;
+                    incr[t] += p;
+                    if (p_out && s == s_dbg) p_out[(size_t)j * N + t] = p;
+                    for (int d = 0; d < D; ++d) o[d] += p * vh[(size_t)t * D + d];
+                }
+            }
+            for (int d = 0; d < D; ++d)
+                out[((size_t)b * Hq + kvh * G + j) * D + d] = (float)o[d];
+            free(o);
+        }
+        for (t = 0; t < N; ++t) *sc[t] = (float)((double)*sc[t] + incr[t]);
+        free(incr);
+        free(qd); free(logit); free(vh); free(kh); free(sc);
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* Budgeted top-k eviction + table compaction                          */
+/* ------------------------------------------------------------------ */
+typedef struct {
+    uint32_t skey;  /* order-preserving image of the fp32 score bits */
+    int32_t pos;
+    int32_t c, i;
+} cand_t;
+
+/* Monotone map of fp32 bit patterns onto uint32: a < b as floats (with -0 < +0)
+ * iff key(a) < key(b). */
+static uint32_t score_key(float f) {
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+/* Total order: higher score first, then lower position, then lower class,
+ * then lower table index. */
+static int cand_cmp(const void *pa, const void *pb) {
+    const cand_t *a = pa, *b = pb;
+    if (a->skey != b->skey) return a->skey > b->skey ? -1 : 1;
+    if (a->pos != b->pos) return a->pos < b->pos ? -1 : 1;
+    if (a->c != b->c) return a->c < b->c ? -1 : 1;
+    if (a->i != b->i) return a->i < b->i ? -1 : 1;
+    return 0;
+}
+
+/* For every stream: entries with pos < n_protect are always kept; among the
+ * others keep the `budget` first under the total order above and evict the
+ * rest.  Each class list keeps its surviving entries in their previous order
+ * (scores carried over).  The slots of evicted entries are pushed on the
+ * class's free stack in reverse table order, so the earliest evicted entry
+ * ends on top and is reused first.  budget >= candidates is a no-op. */
+int orc_evict(orc_state *st, int budget) {
+    if (budget < 0) return ORC_ERR_INVALID;
+    const int S = n_streams(st);
+    for (int s = 0; s < S; ++s) {
+        int N = 0;
+        for (int c = 0; c < 4; ++c) N += st->n[s * 4 + c];
+        cand_t *cand = malloc(sizeof(cand_t) * (N > 0 ? N : 1));
+        int nc = 0;
+        for (int c = 0; c < 4; ++c)
+            for (int i = 0; i < st->n[s * 4 + c]; ++i) {
+                size_t e = (size_t)s * st->cap[c] + i;
+                if (st->pos[c][e] < st->n_protect) continue;
+                cand[nc].skey = score_key(st->score[c][e]);
+                cand[nc].pos = st->pos[c][e];
+                cand[nc].c = c;
+                cand[nc].i = i;
+                ++nc;
+            }
+        if (nc > budget) {
+            qsort(cand, nc, sizeof(cand_t), cand_cmp);
+            uint8_t *evict[4];
+            for (int c = 0; c < 4; ++c) evict[c] = calloc(st->n[s * 4 + c] + 1, 1);
+            for (int r = budget; r < nc; ++r) evict[cand[r].c][cand[r].i] = 1;
+            for (int c = 0; c < 4; ++c) {
+                int n = st->n[s * 4 + c];
+                size_t base = (size_t)s * st->cap[c];
+                int m = 0;
+                for (int i = 0; i < n; ++i) m += evict[c][i];
+                int ft0 = st->ft[s * 4 + c];
+                int w = 0, r = 0;
+                for (int i = 0; i < n; ++i) {
+                    if (evict[c][i]) {
+                        st->fs[c][base + ft0 + (m - 1 - r)] = st->handle[c][base + i];
+                        ++r;
+                    } else {
+                        st->handle[c][base + w] = st->handle[c][base + i];
+                        st->pos[c][base + w] = st->pos[c][base + i];
+                        st->score[c][base + w] = st->score[c][base + i];
+                        ++w;
+                    }
+                }
+                st->n[s * 4 + c] = w;
+                st->ft[s * 4 + c] = ft0 + m;
+                free(evict[c]);
+            }
+        }
+        free(cand);
+    }
+    return ORC_OK;
+}
+
+int orc_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
