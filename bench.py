@@ -1,0 +1,397 @@
+"""Benchmark of the compressed-KV decode step on B200.
+
+Workload (default): batch 64 x 32 query / 8 kv heads, head_dim 128, 32k-token
+context with x10 K outlier channels, R/E/T = 0.35/0.35/0.30 segments, a 128-token
+bf16 question window, eviction to 1638 tokens, then the timed step: quantize-append
+of the new token + decode attention with score accumulation.
+
+One timed step = tkv_quantize_append + tkv_decode_attention on every stream.  The
+cache counters are restored (untimed) before each step so every step sees the same
+post-eviction cache, and the L2 is flushed (untimed) before each step.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl tkv|reference]
+
+N > 1 runs under torchrun: every rank runs an independent replica (weak scaling,
+no data-path collective); rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+WORKLOAD = "b64_ctx32k_evict5pct"
+METRIC = "decode-attn tokens/s & effective HBM GB/s on packed KV (fraction of 8 TB/s)"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+SCALE = 128 ** -0.5
+REC_BYTES = (512, 288, 160, 96)
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["tkv", "reference"], default="tkv")
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=None)
+    return ap.parse_args()
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
+    return FALLBACK_HBM_GBS, "fallback 6.65 TB/s (MEASURED_PEAKS.json absent)"
+
+
+def stored_traffic():
+    """DRAM bytes per attention launch from the committed ncu summary, if it was taken
+    on the current kernel source (null otherwise)."""
+    p = os.path.join(ROOT, "profiles", "attention_traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    src = os.path.join(ROOT, "reasoning_model_kv_b200", "csrc", "attention.cu")
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    if d.get("attention_cu_sha256_16") != h:
+        return None
+    return d
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed loop runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append((float(f[1]), float(f[2]), float(f[3]), f[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no nvidia-smi samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[3]) if v.lower() == "active"})
+        loaded = [r for r in rows if r[2] > 200.0] or rows
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows), "samples_under_load": len(loaded),
+                "power_w_max": max(r[2] for r in rows)}
+
+
+def gpu_smi_id(dev) -> str:
+    """PCI bus id of the device, as nvidia-smi -i accepts it."""
+    pr = torch.cuda.get_device_properties(dev)
+    try:
+        return f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
+    except AttributeError:
+        return str(torch.cuda.current_device())
+
+
+def packed_bytes(n: np.ndarray) -> int:
+    return int(sum(int(n[:, c].sum()) * REC_BYTES[c] for c in range(4)))
+
+
+# ----------------------------------------------------------------------------
+def setup_cache(w, dev, seed):
+    from reasoning_model_kv_b200 import TkvCache
+    gpu = TkvCache(w["B"], w["Hkv"], w["G"], w["cap"], w["n_protect"], max_append=w["ctx"])
+    cls = w["cls"][:, :w["ctx"]].contiguous().to(dev)
+    gpu.quantize_append(w["k"], w["v"], cls, w["pos"].to(dev))
+    k, v, c, p, q = synth.decode_inputs(w, 0, device=dev)        # untimed scoring step
+    gpu.quantize_append(k, v, c, p)
+    gpu.decode_attention(q, SCALE)
+    gpu.evict_compact(w["budget"])
+    torch.cuda.synchronize()
+    assert gpu.poll_error() == 0
+    return gpu
+
+
+def run_tkv(args, rank, world, dev):
+    w = synth.prefill_inputs(args.workload, seed=rank, device=dev, steps=2)
+    gpu = setup_cache(w, dev, rank)
+    del w["k"], w["v"]
+    torch.cuda.empty_cache()
+    views = gpu.state_views()
+    saved = {k: views[k].clone() for k in ("n", "ft", "hw")}
+    k, v, c, p, q = synth.decode_inputs(w, 1, device=dev)
+    out = torch.empty((w["B"], w["Hq"], 128), dtype=torch.float32, device=dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
+
+    def restore():
+        for key in ("n", "ft", "hw"):
+            views[key].copy_(saved[key])
+
+    def step():
+        gpu.quantize_append(k, v, c, p)
+        gpu.decode_attention(q, SCALE, out)
+
+    # packed bytes read by the timed attention: every live entry after the append
+    restore()
+    step()
+    torch.cuda.synchronize()
+    n_after = views["n"].cpu().numpy()
+    pk = packed_bytes(n_after)
+    kv_tokens = int(n_after.sum())
+
+    for _ in range(args.warmup):
+        restore()
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    st = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    launches0 = gpu.launch_count()
+    torch.cuda.synchronize()
+    with ClockSampler(gpu_smi_id(dev)) as cs:
+        for i in range(args.steps):
+            restore()
+            flush.zero_()
+            ev[i][0].record(st)
+            gpu.quantize_append(k, v, c, p)
+            ev[i][1].record(st)
+            gpu.decode_attention(q, SCALE, out)
+            ev[i][2].record(st)
+        torch.cuda.synchronize()
+    launches = gpu.launch_count() - launches0
+    step_ms = [a.elapsed_time(b2) for a, _, b2 in ev]
+    attn_ms = [m.elapsed_time(b2) for _, m, b2 in ev]
+    t_step = sum(step_ms) / len(step_ms)
+    t_attn = sum(attn_ms) / len(attn_ms)
+    if world > 1:
+        t = torch.tensor([t_step, t_attn], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        t_step, t_attn = t.tolist()
+    assert gpu.poll_error() == 0
+
+    # ---- end to end through the public API with host buffers
+    e2e_steps = args.e2e_steps or max(20, min(500, args.steps // 4))
+    hk, hv, hc, hp, hq = (x.cpu().pin_memory() for x in (k, v, c, p, q))
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dk, dv, dc, dp, dq = (torch.empty_like(x) for x in (k, v, c, p, q))
+    e2e_ms = []
+    for i in range(args.warmup + e2e_steps):
+        restore()
+        flush.zero_()
+        a, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        for d_, h_ in ((dk, hk), (dv, hv), (dc, hc), (dp, hp), (dq, hq)):
+            d_.copy_(h_, non_blocking=True)
+        gpu.quantize_append(dk, dv, dc, dp)
+        gpu.decode_attention(dq, SCALE, out)
+        hout.copy_(out, non_blocking=True)
+        b2.record(st)
+        b2.synchronize()
+        if i >= args.warmup:
+            e2e_ms.append(a.elapsed_time(b2))
+    t_e2e = sum(e2e_ms) / len(e2e_ms)
+    if world > 1:
+        t = torch.tensor([t_e2e], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        t_e2e = t.item()
+    h2d = sum(x.numel() * x.element_size() for x in (hk, hv, hc, hp, hq))
+    d2h = hout.numel() * hout.element_size()
+
+    peak, peak_src = measured_peaks()
+    gbs = pk / (t_attn * 1e-3) / 1e9
+    B = w["B"]
+    res = {
+        "metric": METRIC,
+        "value": world * B / (t_step * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": t_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int8/int4/int2 codes + bf16 -> fp32",
+        "data": "synthetic (seeded counter-hash N(0,1) bf16, K x10 outlier channels)",
+        "config": {"workload": args.workload, "batch": B, "q_heads": w["Hq"], "kv_heads": w["Hkv"],
+                   "head_dim": 128, "context": w["ctx"], "budget": w["budget"],
+                   "bf16_window": w["n_protect"], "p_RET": [w["p_r"], w["p_e"], 1 - w["p_r"] - w["p_e"]],
+                   "live_kv_tokens": kv_tokens, "packed_kv_bytes": pk,
+                   "l2": "flushed (write of %d MB) before every timed step" % (flush.numel() >> 20),
+                   "parallelism": f"{world} independent replicas" if world > 1 else "single GPU"},
+        "hbm_gbs_packed": gbs,
+        "frac_of_8tbs": gbs / NOMINAL_HBM_GBS,
+        "attention_ms": t_attn,
+        "kv_tokens_per_s": world * kv_tokens / (t_attn * 1e-3),
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
+                     "frac": gbs / peak, "traffic": None, "peak_source": peak_src,
+                     "kernel": "tkv_decode_attention (all its launches, CUDA events)"},
+        "e2e": {"value": world * B / (t_e2e * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": t_e2e},
+        "gpu_launches": int(launches),
+        "clocks": cs.summary(),
+    }
+    tr = stored_traffic()
+    if tr is not None:
+        res["roofline"]["traffic"] = tr["dram_bytes_per_launch"]
+    return res, gpu, w
+
+
+def cpu_baseline(gpu, w, rows, reps_budget_s=12.0):
+    """The oracle (as it stands) on a bounded sample: the same timed step for batch
+    rows `rows`, starting from the GPU's post-eviction state of those rows."""
+    from oracle import oracle as orc
+    sub = [b * w["Hkv"] + h for b in rows for h in range(w["Hkv"])]
+    st = gpu.export_state(sub)
+    o = orc.OracleCache(len(rows), w["Hkv"], w["G"], cap=w["cap"], n_protect=w["n_protect"])
+    k, v, c, p, q = synth.decode_inputs(w, 1)
+
+    def bits(t):
+        return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+    kb, vb, qb = bits(k[rows]), bits(v[rows]), bits(q[rows])
+    cb, pb = c[rows].numpy(), p[rows].numpy()
+    times = []
+    t_all = time.perf_counter()
+    while True:
+        o.load_state(st)
+        t0 = time.perf_counter()
+        o.append(kb, vb, cb, pb)
+        o.attend(qb, SCALE)
+        times.append(time.perf_counter() - t0)
+        if time.perf_counter() - t_all > reps_budget_s or len(times) >= 50:
+            break
+    t = statistics.median(times)
+    frac = len(sub) / (w["B"] * w["Hkv"])
+    t_full = t / frac
+    return {"value": w["B"] / t_full, "unit": "tokens/s", "cores": orc.num_threads(), "kind": "oracle",
+            "sample": f"{len(rows)} of {w['B']} batch rows ({len(sub)} of {w['B'] * w['Hkv']} streams), "
+                      f"append+attend of the timed step, median of {len(times)} reps, scaled by "
+                      f"{1 / frac:.0f}x to the full batch",
+            "ms_per_step_full_batch_est": t_full * 1e3}
+
+
+def run_reference(args, rank, world):
+    """The oracle as the reference arm: CPU only, on rank 0."""
+    if rank != 0:
+        return None
+    from oracle import oracle as orc
+    w = synth.prefill_inputs(args.workload, seed=0, steps=2, B=1)
+    # one batch row (8 streams) per step sample: prefill, scoring step, eviction, then time
+    o = orc.OracleCache(w["B"], w["Hkv"], w["G"], cap=w["cap"], n_protect=w["n_protect"])
+
+    def bits(t):
+        return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+    o.append(bits(w["k"]), bits(w["v"]), w["cls"][:, :w["ctx"]].numpy(), w["pos"].numpy())
+    k, v, c, p, q = synth.decode_inputs(w, 0)
+    o.append(bits(k), bits(v), c.numpy(), p.numpy())
+    o.attend(bits(q), SCALE)
+    o.evict(w["budget"])
+    st = o.copy_state()
+    k, v, c, p, q = synth.decode_inputs(w, 1)
+    kb, vb, qb, cb, pb = bits(k), bits(v), bits(q), c.numpy(), p.numpy()
+    full_B = synth.WORKLOADS[args.workload]["B"]
+    times = []
+    for i in range(args.warmup + args.steps):
+        o.load_state(st)
+        t0 = time.perf_counter()
+        o.append(kb, vb, cb, pb)
+        o.attend(qb, SCALE)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(dt)
+    t_row = sum(times) / len(times)
+    t_step = t_row * full_B
+    val = full_B / t_step
+    sample = (f"1 of {full_B} batch rows per step (8 streams), append+attend of the timed step, "
+              f"scaled x{full_B} to the full batch")
+    return {"impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_step * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded counter-hash N(0,1) bf16, K x10 outlier channels)",
+            "config": {"workload": args.workload, "batch": full_B, "q_heads": w["Hq"],
+                       "kv_heads": w["Hkv"], "head_dim": 128, "context": w["ctx"],
+                       "budget": w["budget"], "bf16_window": w["n_protect"]},
+            "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": orc.num_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = f"cuda:{local}"
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device(dev))
+    from reasoning_model_kv_b200 import build as b
+    b.build()
+    res, gpu, w = run_tkv(args, rank, world, dev)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(gpu, w, rows=list(range(8)))
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

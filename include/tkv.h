@@ -1,0 +1,188 @@
+/*
+ * tkv.h -- C ABI of libtkv: one decode step of attention over a thought-adaptive
+ * compressed KV cache (ThinKV-style), for NVIDIA B200 (sm_100a).
+ *
+ * The method (from the ThinKV page, sections "Metodologia" and
+ * "Implementacao do Sistema"):
+ *   - every token's K/V is group-quantised at a bit-width set by the thought
+ *     type of its segment: Reasoning 8-bit, Execution 4-bit, Transition 2-bit
+ *     (TBQ, "Think Before you Quantize"); tokens at positions below n_protect
+ *     (attention sinks and the question window -- the DYNTS page, section 2.3,
+ *     gives the question window infinite importance) stay bf16;
+ *   - records live in paged per-precision pools and evicted slots are reused in
+ *     place by new tokens of the same type, with no gather-based compaction
+ *     (Continuous Thinking block table);
+ *   - decode attention dequantises on the fly, and every token accumulates the
+ *     attention mass it receives as its importance score (cumulative,
+ *     H2O-style -- "Back from the Future", problem statement);
+ *   - eviction keeps, per (batch, kv head) stream, the `budget` highest-scoring
+ *     unprotected tokens (DYNTS page, section 2.3, selection window: keep the
+ *     top-k, evict the rest), then compacts the block table.
+ *
+ * Conventions for every call:
+ *   - Device pointers are plain CUDA device addresses; `stream` is a
+ *     cudaStream_t passed as void* (NULL = the legacy default stream).
+ *   - Calls are asynchronous on `stream` and never synchronise, except
+ *     tkv_poll_error, tkv_export_state and tkv_import_state, which do.
+ *   - The library never allocates device memory: the caller owns the workspace
+ *     and every input/output buffer, and keeps them alive while work that uses
+ *     them is in flight.  A tkv_cache is a small host object.
+ *   - Argument errors are detected on the host, return TKV_ERR_INVALID and
+ *     launch nothing.  Conditions only the device can see (a full pool, an
+ *     invalid class id in device memory) skip the offending write, latch a
+ *     device error word, and are reported by the next tkv_poll_error.
+ *     Launch failures return TKV_ERR_CUDA.  tkv_last_error_string() describes
+ *     the last non-OK status of the calling thread.
+ *   - One cache may be used from one stream at a time; calls on one cache that
+ *     overlap on the GPU race.
+ */
+#ifndef TKV_H
+#define TKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TKV_API __attribute__((visibility("default")))
+#else
+#define TKV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    TKV_OK = 0,
+    TKV_ERR_INVALID = 1,   /* bad argument (host) or bad class id (device) */
+    TKV_ERR_CAPACITY = 2,  /* a pool had no free slot: token dropped       */
+    TKV_ERR_CUDA = 3,      /* a CUDA runtime call or launch failed         */
+    TKV_ERR_TIMEOUT = 4    /* reserved: a bounded device wait gave up      */
+} tkv_status;
+
+/* Thought classes.  Class 0 holds bf16 records (protected positions, or tokens
+ * the caller labels 0); classes 1..3 hold Reasoning / Execution / Transition
+ * tokens at bits[1..3]. */
+enum { TKV_CLASS_BF16 = 0, TKV_CLASS_R = 1, TKV_CLASS_E = 2, TKV_CLASS_T = 3 };
+
+typedef struct {
+    int32_t B;           /* batch rows                                        */
+    int32_t Hkv;         /* kv heads; a stream is s = b * Hkv + kv_head       */
+    int32_t G;           /* query heads per kv head (1, 2, 4 or 8)            */
+    int32_t D;           /* head dim: must be 128                              */
+    int32_t group;       /* quantisation group along head dim: must be 32      */
+    int32_t bits[4];     /* must be {16, 8, 4, 2}                              */
+    int32_t n_protect;   /* positions [0, n_protect) are bf16, never evicted   */
+    int32_t cap[4];      /* slots per stream for each class (>= 0)             */
+    int32_t max_append;  /* largest T accepted by tkv_quantize_append (>= 1)   */
+} tkv_config;
+
+typedef struct tkv_cache tkv_cache;
+
+/* Byte offsets of the state arrays inside the workspace (all 256-byte aligned),
+ * so a caller can inspect or checkpoint the cache with plain copies.
+ * Per stream s and class c:
+ *   n[s*4+c], ft[s*4+c], hw[s*4+c]  int32: live entries, free-stack top, next never-used slot
+ *   handle_c[s*cap_c + i]           int32: slot of table entry i (i < n), entries in append order
+ *   pos_c[s*cap_c + i]              int32: token position of entry i
+ *   score_c[s*cap_c + i]            float: accumulated attention mass of entry i
+ *   fs_c[s*cap_c + j]               int32: free stack of slots (j < ft; top = j = ft-1)
+ *   pool_c[(s*cap_c + slot)*rec_bytes_c]  packed record of a slot:
+ *     bf16 class: [K: D bf16][V: D bf16]                                 (512 bytes)
+ *     b-bit class: [K codes D*b/8][V codes D*b/8][K scale x4][K zero x4]
+ *                  [V scale x4][V zero x4]  (fp16, little-endian)        (288/160/96 bytes)
+ *     element i of a code block sits at bit b*(i % (8/b)) of byte i*b/8.
+ * The state region [0, state_bytes) holds all of the above; the rest of the
+ * workspace is scratch. */
+typedef struct {
+    size_t n, ft, hw, err;
+    size_t handle[4], pos[4], score[4], fs[4], pool[4];
+    int32_t rec_bytes[4];
+    size_t state_bytes;
+    size_t total_bytes;
+} tkv_layout;
+
+/* Bytes of device workspace a cache with this configuration needs (0 if the
+ * configuration is invalid). */
+TKV_API size_t tkv_workspace_bytes(const tkv_config *cfg);
+
+/* Create a cache over a caller-owned device workspace of at least
+ * tkv_workspace_bytes(cfg) bytes, 256-byte aligned.  The cache starts empty
+ * once tkv_reset has run on a stream (tkv_create does not touch the device). */
+TKV_API tkv_status tkv_create(const tkv_config *cfg, void *d_workspace, size_t workspace_bytes,
+                      tkv_cache **out);
+
+/* Free the host object.  The workspace stays the caller's. */
+TKV_API tkv_status tkv_destroy(tkv_cache *cache);
+
+/* Empty the cache: zero every counter (n, ft, hw) and the device error word. */
+TKV_API tkv_status tkv_reset(tkv_cache *cache, void *stream);
+
+/* Workspace offsets of the state arrays (see tkv_layout). */
+TKV_API tkv_status tkv_get_layout(const tkv_cache *cache, tkv_layout *out);
+
+/*
+ * Quantise and append T new tokens per stream (ThinKV, TBQ; Continuous
+ * Thinking slot reuse).
+ *   k, v   device bf16 [B][Hkv][T][D]  keys / values of the new tokens
+ *   cls    device uint8 [B][T]          thought class 1 (R), 2 (E), 3 (T) or 0 (bf16)
+ *   pos    device int32 [B][T]          absolute positions
+ *   T      1 <= T <= max_append
+ * Per stream, tokens are taken in t order.  A token at pos < n_protect is
+ * stored in class 0.  For b-bit classes each group of 32 elements gets
+ * zero = fp16 round-down(min), scale = fp16 round-up((max - zero)/(2^b-1)),
+ * code = round-half-even((x - zero)/scale) in fp32 clamped to [0, 2^b-1]
+ * (all codes 0 when scale == 0).  Its slot is popped from the stream's free
+ * stack of that class if non-empty, else the next never-used slot; a token that
+ * finds neither is dropped (device error TKV_ERR_CAPACITY), and a class id > 3
+ * drops the token (device error TKV_ERR_INVALID).  New entries start with
+ * score 0.
+ */
+TKV_API tkv_status tkv_quantize_append(tkv_cache *cache, const void *k, const void *v,
+                               const uint8_t *cls, const int32_t *pos, int32_t T, void *stream);
+
+/*
+ * One decode step of GQA attention over every live token of every stream
+ * (dequantised on the fly), plus score accumulation.
+ *   q              device bf16 [B][Hkv*G][D]; query head h reads kv head h / G
+ *   softmax_scale  logit = softmax_scale * (q . k_hat)   (typically D^-1/2)
+ *   out            device fp32 [B][Hkv*G][D]: sum_t softmax_t(logit) * v_hat_t
+ * Every live token t of stream s then gets score_t += sum over the G query
+ * heads of s of its softmax weight.  An empty stream yields a zero output.
+ */
+TKV_API tkv_status tkv_decode_attention(tkv_cache *cache, const void *q, float softmax_scale,
+                                float *out, void *stream);
+
+/*
+ * Budgeted top-k eviction and table compaction, per stream.
+ *   budget  >= 0: unprotected tokens kept per stream.
+ * Entries with pos < n_protect are always kept.  Among the others the `budget`
+ * first under the order (score descending, then position ascending, then
+ * class, then table index) are kept; the rest are evicted.  Each class table
+ * keeps its survivors in their previous order with their scores; evicted
+ * slots are pushed on the class's free stack in reverse table order, so the
+ * earliest evicted entry is reused first.  A stream with <= budget
+ * unprotected tokens is untouched.
+ */
+TKV_API tkv_status tkv_evict_compact(tkv_cache *cache, int32_t budget, void *stream);
+
+/* Synchronise `stream`, read and clear the device error word; returns the
+ * first device-side status latched since the last poll (TKV_OK if none). */
+TKV_API tkv_status tkv_poll_error(tkv_cache *cache, void *stream);
+
+/* Copy the state region (see tkv_layout) to / from a host buffer of
+ * state_bytes bytes.  Both synchronise `stream`. */
+TKV_API tkv_status tkv_export_state(tkv_cache *cache, void *host_dst, void *stream);
+TKV_API tkv_status tkv_import_state(tkv_cache *cache, const void *host_src, void *stream);
+
+/* Launch counters since tkv_create (kernels this cache has launched). */
+TKV_API int64_t tkv_launch_count(const tkv_cache *cache);
+
+/* Human-readable description of the calling thread's last non-OK status. */
+TKV_API const char *tkv_last_error_string(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TKV_H */

@@ -1,0 +1,230 @@
+// append.cu -- tkv_quantize_append: thought-adaptive group quantisation of new
+// tokens (ThinKV, Metodologia / TBQ) into paged per-precision pools with
+// in-place reuse of evicted slots (ThinKV, Implementacao do Sistema /
+// Continuous Thinking).
+//
+// One warp packs one (stream, token): lane l owns head-dim elements
+// [4l, 4l+4), so a 32-element group is 8 lanes and its min/max is a 3-step
+// xor-shuffle reduction.  The quantiser uses only correctly rounded fp32
+// operations (__fsub_rn, __fdiv_rn, __float2int_rn) and the hardware's
+// directed fp32->fp16 conversions, so codes, scales and zeros are bit-exact
+// with any IEEE implementation of the same definition.
+//
+// Slot allocation needs, per (stream, class), the rank of each new token among
+// the new tokens of its class.  For T == 1 that rank is 0 and the packing warp
+// also updates the stream's counters (one kernel).  For T > 1 a scan kernel per
+// batch row computes the ranks (they are shared by all kv heads of the row), the
+// pack kernel runs on every (stream, token) in parallel against the pre-call
+// counters, and a finalize kernel advances the counters.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "tkv_internal.cuh"
+
+namespace tkv {
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+// Class a new token is stored in; -1 for an invalid class id.
+__device__ __forceinline__ int token_class(const Dev &d, uint8_t c, int32_t p) {
+    if (p < d.n_protect) return 0;
+    return c <= 3 ? static_cast<int>(c) : -1;
+}
+
+__global__ void append_rank_kernel(Dev d, const uint8_t *__restrict__ cls,
+                                   const int32_t *__restrict__ pos, int T) {
+    const int b = blockIdx.x;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    __shared__ int carry[4];
+    __shared__ int wtot[32][4];
+    if (threadIdx.x < 4) carry[threadIdx.x] = 0;
+    __syncthreads();
+    for (int t0 = 0; t0 < T; t0 += blockDim.x) {
+        const int t = t0 + threadIdx.x;
+        int c = -2;
+        if (t < T) c = token_class(d, cls[(size_t)b * T + t], pos[(size_t)b * T + t]);
+        int myrank = 0;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+            const unsigned m = __ballot_sync(kFull, c == cc);
+            if (lane == 0) wtot[warp][cc] = __popc(m);
+            if (c == cc) myrank = __popc(m & ((1u << lane) - 1u));
+        }
+        __syncthreads();
+        if (c >= 0) {
+            int pre = carry[c];
+            for (int w = 0; w < warp; ++w) pre += wtot[w][c];
+            d.rank[(size_t)b * d.max_append + t] = pre + myrank;
+        } else if (t < T) {
+            d.rank[(size_t)b * d.max_append + t] = -1;
+        }
+        __syncthreads();
+        if (threadIdx.x < 4) {
+            int sum = 0;
+            for (int w = 0; w < nwarps; ++w) sum += wtot[w][threadIdx.x];
+            carry[threadIdx.x] += sum;
+        }
+        __syncthreads();
+    }
+    if (threadIdx.x < 4) d.totals[b * 4 + threadIdx.x] = carry[threadIdx.x];
+}
+
+// Quantise one 128-element bf16 row held as 4 elements per lane and write its
+// packed codes and its (scale, zero) pairs.
+template <int BITS>
+__device__ __forceinline__ void quantize_row(const float (&x)[4], int lane, uint8_t *codes,
+                                             __half *meta /* [scale x4][zero x4] */) {
+    constexpr int kQmax = (1 << BITS) - 1;
+    float mn = fminf(fminf(x[0], x[1]), fminf(x[2], x[3]));
+    float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) {
+        mn = fminf(mn, __shfl_xor_sync(kFull, mn, o));
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
+    }
+    const __half zh = __float2half_rd(mn);
+    const float zf = __half2float(zh);
+    const float step = __fdiv_rn(__fsub_rn(mx, zf), static_cast<float>(kQmax));
+    const __half sh = __float2half_ru(step);
+    const float sf = __half2float(sh);
+    uint32_t q[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        int v = 0;
+        if (sf != 0.0f) {
+            v = __float2int_rn(__fdiv_rn(__fsub_rn(x[i], zf), sf));
+            v = v < 0 ? 0 : (v > kQmax ? kQmax : v);
+        }
+        q[i] = static_cast<uint32_t>(v);
+    }
+    if constexpr (BITS == 8) {
+        reinterpret_cast<uint32_t *>(codes)[lane] = q[0] | (q[1] << 8) | (q[2] << 16) | (q[3] << 24);
+    } else if constexpr (BITS == 4) {
+        reinterpret_cast<uint16_t *>(codes)[lane] =
+            static_cast<uint16_t>(q[0] | (q[1] << 4) | (q[2] << 8) | (q[3] << 12));
+    } else {
+        codes[lane] = static_cast<uint8_t>(q[0] | (q[1] << 2) | (q[2] << 4) | (q[3] << 6));
+    }
+    if ((lane & 7) == 0) {
+        const int g = lane >> 3;
+        meta[g] = sh;
+        meta[kNG + g] = zh;
+    }
+}
+
+__device__ __forceinline__ void load_row(const __nv_bfloat16 *src, int lane, float (&x)[4],
+                                         uint2 &raw) {
+    raw = reinterpret_cast<const uint2 *>(src)[lane];
+    x[0] = __uint_as_float(raw.x << 16);
+    x[1] = __uint_as_float(raw.x & 0xffff0000u);
+    x[2] = __uint_as_float(raw.y << 16);
+    x[3] = __uint_as_float(raw.y & 0xffff0000u);
+}
+
+template <int BITS>
+__device__ __forceinline__ void pack_record(const __nv_bfloat16 *k, const __nv_bfloat16 *v,
+                                            uint8_t *rec, int lane) {
+    float x[4];
+    uint2 raw;
+    if constexpr (BITS == 16) {
+        load_row(k, lane, x, raw);
+        reinterpret_cast<uint2 *>(rec)[lane] = raw;
+        load_row(v, lane, x, raw);
+        reinterpret_cast<uint2 *>(rec + 2 * kD)[lane] = raw;
+    } else {
+        constexpr int cb = kD * BITS / 8;
+        __half *meta = reinterpret_cast<__half *>(rec + 2 * cb);
+        load_row(k, lane, x, raw);
+        quantize_row<BITS>(x, lane, rec, meta);
+        load_row(v, lane, x, raw);
+        quantize_row<BITS>(x, lane, rec + cb, meta + 2 * kNG);
+    }
+}
+
+template <bool kSingle>
+__global__ void __launch_bounds__(256) append_pack_kernel(
+    Dev d, const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ v,
+    const uint8_t *__restrict__ cls, const int32_t *__restrict__ pos, int T) {
+    const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (gw >= d.S * T) return;
+    const int s = gw / T, t = gw - s * T;
+    const int b = s / d.Hkv;
+    const int32_t p = pos[(size_t)b * T + t];
+    const int c = token_class(d, cls[(size_t)b * T + t], p);
+    if (c < 0) {
+        if (lane == 0) raise_error(d.err, kErrInvalid, (uint32_t)gw);
+        return;
+    }
+    const int r = kSingle ? 0 : d.rank[(size_t)b * d.max_append + t];
+    const int sc = s * 4 + c;
+    const int cap = d.cap[c];
+    const int ft = d.ft[sc], hw = d.hw[sc], n = d.n[sc];
+    int slot;
+    if (r < ft) {
+        slot = d.fs[c][(size_t)s * cap + ft - 1 - r];
+    } else {
+        slot = hw + (r - ft);
+        if (slot >= cap) {
+            if (lane == 0) raise_error(d.err, kErrCapacity, (uint32_t)sc);
+            return;
+        }
+    }
+    const size_t e = (size_t)s * cap + n + r;
+    if (lane == 0) {
+        d.handle[c][e] = slot;
+        d.pos[c][e] = p;
+        d.score[c][e] = 0.0f;
+    }
+    uint8_t *rec = d.pool[c] + ((size_t)s * cap + slot) * d.rec[c];
+    const size_t row = ((size_t)s * T + t) * kD;
+    switch (c) {
+        case 0: pack_record<16>(k + row, v + row, rec, lane); break;
+        case 1: pack_record<8>(k + row, v + row, rec, lane); break;
+        case 2: pack_record<4>(k + row, v + row, rec, lane); break;
+        default: pack_record<2>(k + row, v + row, rec, lane); break;
+    }
+    __syncwarp();  // every lane has read the pre-call counters
+    if (kSingle && lane == 0) {
+        if (r < ft) d.ft[sc] = ft - 1; else d.hw[sc] = hw + 1;
+        d.n[sc] = n + 1;
+    }
+}
+
+__global__ void append_finalize_kernel(Dev d) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= d.S * 4) return;
+    const int s = i >> 2, c = i & 3, b = s / d.Hkv;
+    const int tot = d.totals[b * 4 + c];
+    const int ft = d.ft[i], hw = d.hw[i];
+    const int pops = tot < ft ? tot : ft;
+    int fresh = tot - pops;
+    if (fresh > d.cap[c] - hw) fresh = d.cap[c] - hw;
+    d.ft[i] = ft - pops;
+    d.hw[i] = hw + fresh;
+    d.n[i] += pops + fresh;
+}
+
+}  // namespace
+
+cudaError_t launch_append(const Dev &d, const void *k, const void *v, const uint8_t *cls,
+                          const int32_t *pos, int T, cudaStream_t st, int64_t *launches) {
+    const auto *kk = static_cast<const __nv_bfloat16 *>(k);
+    const auto *vv = static_cast<const __nv_bfloat16 *>(v);
+    const long long warps = (long long)d.S * T;
+    const int threads = 256;
+    const unsigned blocks = (unsigned)((warps * 32 + threads - 1) / threads);
+    if (T == 1) {
+        append_pack_kernel<true><<<blocks, threads, 0, st>>>(d, kk, vv, cls, pos, T);
+        *launches += 1;
+        return cudaGetLastError();
+    }
+    append_rank_kernel<<<d.B, 1024, 0, st>>>(d, cls, pos, T);
+    append_pack_kernel<false><<<blocks, threads, 0, st>>>(d, kk, vv, cls, pos, T);
+    append_finalize_kernel<<<(d.S * 4 + 255) / 256, 256, 0, st>>>(d);
+    *launches += 3;
+    return cudaGetLastError();
+}
+
+}  // namespace tkv

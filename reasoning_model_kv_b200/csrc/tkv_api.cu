@@ -1,0 +1,245 @@
+// tkv_api.cu -- host side of the C ABI in include/tkv.h: configuration checks,
+// the workspace layout, argument validation and kernel launches.  No device
+// memory is allocated here; nothing synchronises except poll/export/import.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+
+#include "tkv.h"
+#include "tkv_internal.cuh"
+
+struct tkv_cache {
+    tkv_config cfg;
+    tkv_layout lay;
+    tkv::Dev dev;
+    uint8_t *base;
+    long long live_ub;   // host-side upper bound of live entries in any stream
+    int64_t launches;
+};
+
+namespace {
+
+thread_local std::string g_last_error;
+
+tkv_status fail(tkv_status st, const std::string &msg) {
+    g_last_error = msg;
+    return st;
+}
+
+constexpr size_t kAlign = 256;
+constexpr int kMaxSplits = 64;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool valid_config(const tkv_config *c, std::string *why) {
+    if (!c) { *why = "config is NULL"; return false; }
+    if (c->B < 1 || c->Hkv < 1) { *why = "B and Hkv must be >= 1"; return false; }
+    if (!(c->G == 1 || c->G == 2 || c->G == 4 || c->G == 8)) { *why = "G must be 1, 2, 4 or 8"; return false; }
+    if (c->D != tkv::kD) { *why = "D must be 128"; return false; }
+    if (c->group != tkv::kGroup) { *why = "group must be 32"; return false; }
+    const int want[4] = {16, 8, 4, 2};
+    for (int i = 0; i < 4; ++i)
+        if (c->bits[i] != want[i]) { *why = "bits must be {16, 8, 4, 2}"; return false; }
+    if (c->n_protect < 0) { *why = "n_protect must be >= 0"; return false; }
+    long long ncap = 0;
+    for (int i = 0; i < 4; ++i) {
+        if (c->cap[i] < 0) { *why = "cap[c] must be >= 0"; return false; }
+        ncap += c->cap[i];
+    }
+    if (ncap > (1ll << 30)) { *why = "sum of cap too large"; return false; }
+    if (c->max_append < 1 || c->max_append > (1 << 24)) { *why = "max_append must be in [1, 2^24]"; return false; }
+    if ((long long)c->B * c->Hkv > (1 << 20)) { *why = "too many streams"; return false; }
+    return true;
+}
+
+// Lays the workspace out; fills *lay and, if base != NULL, the device view.
+void make_layout(const tkv_config &c, tkv_layout *lay, tkv::Dev *dev, uint8_t *base) {
+    const size_t S = (size_t)c.B * c.Hkv;
+    size_t off = 0;
+    auto take = [&](size_t bytes) { const size_t o = off; off = align_up(off + bytes); return o; };
+    lay->n = take(S * 4 * sizeof(int32_t));
+    lay->ft = take(S * 4 * sizeof(int32_t));
+    lay->hw = take(S * 4 * sizeof(int32_t));
+    lay->err = take(16 * sizeof(uint32_t));
+    for (int k = 0; k < 4; ++k) {
+        const size_t e = S * (size_t)c.cap[k];
+        lay->handle[k] = take(e * sizeof(int32_t));
+        lay->pos[k] = take(e * sizeof(int32_t));
+        lay->score[k] = take(e * sizeof(float));
+        lay->fs[k] = take(e * sizeof(int32_t));
+    }
+    for (int k = 0; k < 4; ++k) {
+        lay->rec_bytes[k] = tkv::record_bytes(c.bits[k]);
+        lay->pool[k] = take(S * (size_t)c.cap[k] * lay->rec_bytes[k]);
+    }
+    lay->state_bytes = off;
+    const int ncap = c.cap[0] + c.cap[1] + c.cap[2] + c.cap[3];
+    const size_t o_rank = take((size_t)c.B * c.max_append * sizeof(int32_t));
+    const size_t o_tot = take((size_t)c.B * 4 * sizeof(int32_t));
+    const size_t o_part = take(S * kMaxSplits * c.G * (tkv::kD + 2) * sizeof(float));
+    const size_t o_lg = take(S * (size_t)ncap * c.G * sizeof(float));
+    lay->total_bytes = off;
+    if (!dev) return;
+    dev->B = c.B; dev->Hkv = c.Hkv; dev->G = c.G; dev->S = (int)S;
+    dev->n_protect = c.n_protect; dev->max_append = c.max_append;
+    dev->n = reinterpret_cast<int32_t *>(base + lay->n);
+    dev->ft = reinterpret_cast<int32_t *>(base + lay->ft);
+    dev->hw = reinterpret_cast<int32_t *>(base + lay->hw);
+    dev->err = reinterpret_cast<uint32_t *>(base + lay->err);
+    for (int k = 0; k < 4; ++k) {
+        dev->cap[k] = c.cap[k];
+        dev->rec[k] = lay->rec_bytes[k];
+        dev->handle[k] = reinterpret_cast<int32_t *>(base + lay->handle[k]);
+        dev->pos[k] = reinterpret_cast<int32_t *>(base + lay->pos[k]);
+        dev->score[k] = reinterpret_cast<float *>(base + lay->score[k]);
+        dev->fs[k] = reinterpret_cast<int32_t *>(base + lay->fs[k]);
+        dev->pool[k] = base + lay->pool[k];
+    }
+    dev->rank = reinterpret_cast<int32_t *>(base + o_rank);
+    dev->totals = reinterpret_cast<int32_t *>(base + o_tot);
+    dev->part = reinterpret_cast<float *>(base + o_part);
+    dev->logits = reinterpret_cast<float *>(base + o_lg);
+    dev->max_splits = kMaxSplits;
+    dev->ncap = ncap;
+}
+
+tkv_status cuda_status(cudaError_t e, const char *what) {
+    if (e == cudaSuccess) return TKV_OK;
+    return fail(TKV_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+size_t tkv_workspace_bytes(const tkv_config *cfg) {
+    std::string why;
+    if (!valid_config(cfg, &why)) { g_last_error = why; return 0; }
+    tkv_layout lay;
+    make_layout(*cfg, &lay, nullptr, nullptr);
+    return lay.total_bytes;
+}
+
+tkv_status tkv_create(const tkv_config *cfg, void *d_workspace, size_t workspace_bytes,
+                      tkv_cache **out) {
+    std::string why;
+    if (!out) return fail(TKV_ERR_INVALID, "out is NULL");
+    *out = nullptr;
+    if (!valid_config(cfg, &why)) return fail(TKV_ERR_INVALID, why);
+    if (!d_workspace) return fail(TKV_ERR_INVALID, "workspace is NULL");
+    if (reinterpret_cast<uintptr_t>(d_workspace) % kAlign)
+        return fail(TKV_ERR_INVALID, "workspace must be 256-byte aligned");
+    tkv_layout lay;
+    make_layout(*cfg, &lay, nullptr, nullptr);
+    if (workspace_bytes < lay.total_bytes) return fail(TKV_ERR_INVALID, "workspace too small");
+    auto *c = new (std::nothrow) tkv_cache();
+    if (!c) return fail(TKV_ERR_INVALID, "out of host memory");
+    c->cfg = *cfg;
+    c->base = static_cast<uint8_t *>(d_workspace);
+    make_layout(*cfg, &c->lay, &c->dev, c->base);
+    c->live_ub = 0;
+    c->launches = 0;
+    *out = c;
+    return TKV_OK;
+}
+
+tkv_status tkv_destroy(tkv_cache *cache) {
+    delete cache;
+    return TKV_OK;
+}
+
+tkv_status tkv_reset(tkv_cache *c, void *stream) {
+    if (!c) return fail(TKV_ERR_INVALID, "cache is NULL");
+    auto st = static_cast<cudaStream_t>(stream);
+    // n, ft, hw and err are contiguous at the start of the workspace
+    cudaError_t e = cudaMemsetAsync(c->base, 0, c->lay.err + 16 * sizeof(uint32_t), st);
+    if (e != cudaSuccess) return cuda_status(e, "tkv_reset");
+    c->live_ub = 0;
+    return TKV_OK;
+}
+
+tkv_status tkv_get_layout(const tkv_cache *c, tkv_layout *out) {
+    if (!c || !out) return fail(TKV_ERR_INVALID, "NULL argument");
+    *out = c->lay;
+    return TKV_OK;
+}
+
+tkv_status tkv_quantize_append(tkv_cache *c, const void *k, const void *v, const uint8_t *cls,
+                               const int32_t *pos, int32_t T, void *stream) {
+    if (!c) return fail(TKV_ERR_INVALID, "cache is NULL");
+    if (!k || !v || !cls || !pos) return fail(TKV_ERR_INVALID, "NULL input pointer");
+    if (T < 1 || T > c->cfg.max_append) return fail(TKV_ERR_INVALID, "T out of [1, max_append]");
+    if (!aligned16(k) || !aligned16(v)) return fail(TKV_ERR_INVALID, "k and v must be 16-byte aligned");
+    if (!aligned16(pos)) return fail(TKV_ERR_INVALID, "pos must be 16-byte aligned");
+    cudaError_t e = tkv::launch_append(c->dev, k, v, cls, pos, T, static_cast<cudaStream_t>(stream),
+                                       &c->launches);
+    const long long ncap = c->dev.ncap;
+    c->live_ub = std::min(ncap, c->live_ub + T);
+    return cuda_status(e, "tkv_quantize_append");
+}
+
+tkv_status tkv_decode_attention(tkv_cache *c, const void *q, float softmax_scale, float *out,
+                                void *stream) {
+    if (!c) return fail(TKV_ERR_INVALID, "cache is NULL");
+    if (!q || !out) return fail(TKV_ERR_INVALID, "NULL q or out");
+    if (!aligned16(q) || !aligned16(out)) return fail(TKV_ERR_INVALID, "q and out must be 16-byte aligned");
+    const long long ub = std::max(1ll, c->live_ub);
+    int splits = (int)std::min<long long>(kMaxSplits, (ub + 255) / 256);
+    splits = std::max(1, splits);
+    cudaError_t e = tkv::launch_attention(c->dev, q, softmax_scale, out, splits,
+                                          static_cast<cudaStream_t>(stream), &c->launches);
+    return cuda_status(e, "tkv_decode_attention");
+}
+
+tkv_status tkv_evict_compact(tkv_cache *c, int32_t budget, void *stream) {
+    if (!c) return fail(TKV_ERR_INVALID, "cache is NULL");
+    if (budget < 0) return fail(TKV_ERR_INVALID, "budget must be >= 0");
+    cudaError_t e = tkv::launch_evict(c->dev, budget, static_cast<cudaStream_t>(stream), &c->launches);
+    const long long bound = (long long)budget + c->cfg.cap[0];
+    c->live_ub = std::min(c->live_ub, bound);
+    return cuda_status(e, "tkv_evict_compact");
+}
+
+tkv_status tkv_poll_error(tkv_cache *c, void *stream) {
+    if (!c) return fail(TKV_ERR_INVALID, "cache is NULL");
+    auto st = static_cast<cudaStream_t>(stream);
+    uint32_t w[4] = {0, 0, 0, 0};
+    cudaError_t e = cudaMemcpyAsync(w, c->dev.err, sizeof(w), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(c->dev.err, 0, sizeof(w), st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_status(e, "tkv_poll_error");
+    if (w[0] == 0) return TKV_OK;
+    char msg[160];
+    std::snprintf(msg, sizeof(msg), "device error %u (%u occurrences, detail %u)", w[0], w[1], w[2]);
+    return fail(static_cast<tkv_status>(w[0]), msg);
+}
+
+tkv_status tkv_export_state(tkv_cache *c, void *host_dst, void *stream) {
+    if (!c || !host_dst) return fail(TKV_ERR_INVALID, "NULL argument");
+    auto st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(host_dst, c->base, c->lay.state_bytes, cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    return cuda_status(e, "tkv_export_state");
+}
+
+tkv_status tkv_import_state(tkv_cache *c, const void *host_src, void *stream) {
+    if (!c || !host_src) return fail(TKV_ERR_INVALID, "NULL argument");
+    auto st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(c->base, host_src, c->lay.state_bytes, cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    c->live_ub = c->dev.ncap;
+    return cuda_status(e, "tkv_import_state");
+}
+
+int64_t tkv_launch_count(const tkv_cache *c) { return c ? c->launches : 0; }
+
+const char *tkv_last_error_string(void) { return g_last_error.c_str(); }
+
+}  // extern "C"

@@ -1,0 +1,55 @@
+// tkv_internal.cuh -- device-side view of a cache workspace and the launchers
+// of the sm_100a kernels.  Internal to libtkv (the C ABI is include/tkv.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+namespace tkv {
+
+constexpr int kD = 128;       // head dim
+constexpr int kGroup = 32;    // quantisation group along head dim
+constexpr int kNG = kD / kGroup;
+constexpr int kMaxG = 8;      // query heads per kv head supported
+
+// Record bytes of a class with `bits` bits per element (bits == 16: bf16).
+__host__ __device__ constexpr int record_bytes(int bits) {
+    return bits == 16 ? 4 * kD : 2 * (kD * bits / 8) + 4 * kNG * 2;
+}
+
+// Everything a kernel needs to address one cache.  Passed by value.
+struct Dev {
+    int B, Hkv, G, S, n_protect, max_append;
+    int cap[4];
+    int rec[4];
+    int32_t *n, *ft, *hw;   // [S][4]
+    uint32_t *err;          // [0] first status, [1] count, [2] detail
+    int32_t *handle[4], *pos[4], *fs[4];
+    float *score[4];
+    uint8_t *pool[4];
+    // scratch
+    int32_t *rank;     // [B][max_append] rank of a new token within its class
+    int32_t *totals;   // [B][4] tokens per class in the current append
+    float *part;       // [S][max_splits][G][kD + 2] split partials (m, l, O)
+    float *logits;     // [S][ncap][G] raw logits of the current step
+    int max_splits;
+    int ncap;          // sum of cap[c]
+};
+
+enum : uint32_t { kErrInvalid = 1, kErrCapacity = 2, kErrTimeout = 4 };
+
+__device__ __forceinline__ void raise_error(uint32_t *err, uint32_t code, uint32_t detail) {
+    if (atomicCAS(err, 0u, code) == 0u) err[2] = detail;
+    atomicAdd(err + 1, 1u);
+}
+
+// Launchers (each returns the CUDA error of its launches and adds the number
+// of kernels it launched to *launches).
+cudaError_t launch_append(const Dev &d, const void *k, const void *v, const uint8_t *cls,
+                          const int32_t *pos, int T, cudaStream_t st, int64_t *launches);
+cudaError_t launch_attention(const Dev &d, const void *q, float scale, float *out, int splits,
+                             cudaStream_t st, int64_t *launches);
+cudaError_t launch_evict(const Dev &d, int budget, cudaStream_t st, int64_t *launches);
+
+}  // namespace tkv

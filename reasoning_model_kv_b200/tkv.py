@@ -1,0 +1,241 @@
+"""Thin ctypes binding of libtkv (include/tkv.h).
+
+Argument marshalling only: torch tensors provide device memory and the current
+CUDA stream; every step of the decode path runs in the library's kernels.
+There is no fallback: if libtkv.so is missing or no CUDA device is present,
+the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+from pathlib import Path
+
+import torch
+
+LIB_PATH = Path(__file__).resolve().parent / "libtkv.so"
+
+TKV_OK, TKV_ERR_INVALID, TKV_ERR_CAPACITY, TKV_ERR_CUDA, TKV_ERR_TIMEOUT = range(5)
+STATUS_NAMES = {0: "TKV_OK", 1: "TKV_ERR_INVALID", 2: "TKV_ERR_CAPACITY", 3: "TKV_ERR_CUDA",
+                4: "TKV_ERR_TIMEOUT"}
+BITS = (16, 8, 4, 2)
+
+
+class TkvError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+class TkvConfig(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("Hkv", ctypes.c_int32), ("G", ctypes.c_int32),
+                ("D", ctypes.c_int32), ("group", ctypes.c_int32), ("bits", ctypes.c_int32 * 4),
+                ("n_protect", ctypes.c_int32), ("cap", ctypes.c_int32 * 4),
+                ("max_append", ctypes.c_int32)]
+
+
+class TkvLayout(ctypes.Structure):
+    _fields_ = [("n", ctypes.c_size_t), ("ft", ctypes.c_size_t), ("hw", ctypes.c_size_t),
+                ("err", ctypes.c_size_t), ("handle", ctypes.c_size_t * 4),
+                ("pos", ctypes.c_size_t * 4), ("score", ctypes.c_size_t * 4),
+                ("fs", ctypes.c_size_t * 4), ("pool", ctypes.c_size_t * 4),
+                ("rec_bytes", ctypes.c_int32 * 4), ("state_bytes", ctypes.c_size_t),
+                ("total_bytes", ctypes.c_size_t)]
+
+
+EXPORTS = ["tkv_workspace_bytes", "tkv_create", "tkv_destroy", "tkv_reset", "tkv_get_layout",
+           "tkv_quantize_append", "tkv_decode_attention", "tkv_evict_compact", "tkv_poll_error",
+           "tkv_export_state", "tkv_import_state", "tkv_launch_count", "tkv_last_error_string"]
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libtkv.so (built by reasoning_model_kv_b200.build); raises if absent."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not LIB_PATH.exists():
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m reasoning_model_kv_b200.build`")
+    L = ctypes.CDLL(str(LIB_PATH))
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+    P = ctypes.POINTER
+    L.tkv_workspace_bytes.argtypes = [P(TkvConfig)]
+    L.tkv_workspace_bytes.restype = sz
+    L.tkv_create.argtypes = [P(TkvConfig), vp, sz, P(vp)]
+    L.tkv_destroy.argtypes = [vp]
+    L.tkv_reset.argtypes = [vp, vp]
+    L.tkv_get_layout.argtypes = [vp, P(TkvLayout)]
+    L.tkv_quantize_append.argtypes = [vp, vp, vp, vp, vp, i32, vp]
+    L.tkv_decode_attention.argtypes = [vp, vp, ctypes.c_float, vp, vp]
+    L.tkv_evict_compact.argtypes = [vp, i32, vp]
+    L.tkv_poll_error.argtypes = [vp, vp]
+    L.tkv_export_state.argtypes = [vp, vp, vp]
+    L.tkv_import_state.argtypes = [vp, vp, vp]
+    L.tkv_launch_count.argtypes = [vp]
+    L.tkv_launch_count.restype = ctypes.c_int64
+    L.tkv_last_error_string.restype = ctypes.c_char_p
+    for name in ("tkv_create", "tkv_destroy", "tkv_reset", "tkv_get_layout", "tkv_quantize_append",
+                 "tkv_decode_attention", "tkv_evict_compact", "tkv_poll_error", "tkv_export_state",
+                 "tkv_import_state"):
+        getattr(L, name).restype = ctypes.c_int
+    _lib = L
+    return L
+
+
+def _check(status: int):
+    if status != TKV_OK:
+        raise TkvError(status, lib().tkv_last_error_string().decode())
+
+
+def make_config(B, Hkv, G, cap, n_protect, max_append=1, D=128, group=32) -> TkvConfig:
+    cfg = TkvConfig()
+    cfg.B, cfg.Hkv, cfg.G, cfg.D, cfg.group = B, Hkv, G, D, group
+    for i in range(4):
+        cfg.bits[i] = BITS[i]
+        cfg.cap[i] = int(cap[i])
+    cfg.n_protect = n_protect
+    cfg.max_append = max_append
+    return cfg
+
+
+def tkv_workspace_bytes(cfg: TkvConfig) -> int:
+    return lib().tkv_workspace_bytes(ctypes.byref(cfg))
+
+
+def _stream(stream=None) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _dptr(t: torch.Tensor, dtype, name: str) -> int:
+    if not t.is_cuda:
+        raise TkvError(TKV_ERR_INVALID, f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TkvError(TKV_ERR_INVALID, f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise TkvError(TKV_ERR_INVALID, f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+class TkvCache:
+    """One layer's compressed KV cache: a device workspace owned by torch plus the
+    library's cache object.  Methods mirror the C ABI names."""
+
+    def __init__(self, B, Hkv, G, cap, n_protect, max_append=1, device="cuda"):
+        self.cfg = make_config(B, Hkv, G, cap, n_protect, max_append)
+        self.B, self.Hkv, self.G, self.S = B, Hkv, G, B * Hkv
+        self.cap = tuple(int(c) for c in cap)
+        self.n_protect, self.max_append = n_protect, max_append
+        nbytes = tkv_workspace_bytes(self.cfg)
+        if nbytes == 0:
+            raise TkvError(TKV_ERR_INVALID, lib().tkv_last_error_string().decode())
+        self.workspace = torch.empty(nbytes + 256, dtype=torch.uint8, device=device)
+        base = self.workspace.data_ptr()
+        self._pad = (-base) % 256
+        h = ctypes.c_void_p()
+        _check(lib().tkv_create(ctypes.byref(self.cfg), base + self._pad, nbytes, ctypes.byref(h)))
+        self._h = h
+        self.layout = TkvLayout()
+        _check(lib().tkv_get_layout(self._h, ctypes.byref(self.layout)))
+        self.reset()
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and _lib is not None:
+            _lib.tkv_destroy(h)
+            self._h = None
+
+    # -- the three calls of the decode path
+    def quantize_append(self, k: torch.Tensor, v: torch.Tensor, cls: torch.Tensor,
+                        pos: torch.Tensor, stream=None):
+        T = k.shape[2]
+        if k.shape != (self.B, self.Hkv, T, 128) or v.shape != k.shape:
+            raise TkvError(TKV_ERR_INVALID, f"k/v must be [B, Hkv, T, 128], got {tuple(k.shape)}")
+        if cls.shape != (self.B, T) or pos.shape != (self.B, T):
+            raise TkvError(TKV_ERR_INVALID, "cls/pos must be [B, T]")
+        _check(lib().tkv_quantize_append(self._h, _dptr(k, torch.bfloat16, "k"),
+                                         _dptr(v, torch.bfloat16, "v"),
+                                         _dptr(cls, torch.uint8, "cls"),
+                                         _dptr(pos, torch.int32, "pos"), T, _stream(stream)))
+
+    def decode_attention(self, q: torch.Tensor, softmax_scale: float, out: torch.Tensor | None = None,
+                         stream=None) -> torch.Tensor:
+        if q.shape != (self.B, self.Hkv * self.G, 128):
+            raise TkvError(TKV_ERR_INVALID, f"q must be [B, Hkv*G, 128], got {tuple(q.shape)}")
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+        _check(lib().tkv_decode_attention(self._h, _dptr(q, torch.bfloat16, "q"),
+                                          float(softmax_scale), _dptr(out, torch.float32, "out"),
+                                          _stream(stream)))
+        return out
+
+    def evict_compact(self, budget: int, stream=None):
+        _check(lib().tkv_evict_compact(self._h, int(budget), _stream(stream)))
+
+    # -- housekeeping
+    def reset(self, stream=None):
+        _check(lib().tkv_reset(self._h, _stream(stream)))
+
+    def poll_error(self, stream=None) -> int:
+        """Synchronise and return (and clear) the first device-side status."""
+        st = lib().tkv_poll_error(self._h, _stream(stream))
+        if st == TKV_ERR_CUDA:
+            _check(st)
+        return st
+
+    def launch_count(self) -> int:
+        return lib().tkv_launch_count(self._h)
+
+    def state_views(self) -> dict:
+        """Zero-copy torch views of the state arrays inside the workspace."""
+        L = self.layout
+        ws = self.workspace[self._pad:]
+        S = self.S
+
+        def view(off, count, dtype, shape):
+            nbytes = count * torch.empty((), dtype=dtype).element_size()
+            return ws[off:off + nbytes].view(dtype).view(*shape)
+
+        out = {"n": view(L.n, S * 4, torch.int32, (S, 4)),
+               "ft": view(L.ft, S * 4, torch.int32, (S, 4)),
+               "hw": view(L.hw, S * 4, torch.int32, (S, 4))}
+        for c in range(4):
+            cc = self.cap[c]
+            out[f"handle{c}"] = view(L.handle[c], S * cc, torch.int32, (S, cc))
+            out[f"pos{c}"] = view(L.pos[c], S * cc, torch.int32, (S, cc))
+            out[f"score{c}"] = view(L.score[c], S * cc, torch.float32, (S, cc))
+            out[f"fs{c}"] = view(L.fs[c], S * cc, torch.int32, (S, cc))
+            rb = L.rec_bytes[c]
+            out[f"pool{c}"] = ws[L.pool[c]:L.pool[c] + S * cc * rb].view(S, cc, rb)
+        return out
+
+    def export_state(self, streams=None) -> dict:
+        """Host (numpy) copy of the state, optionally of a subset of streams."""
+        torch.cuda.current_stream().synchronize()
+        v = self.state_views()
+        if streams is None:
+            return {k: t.cpu().numpy() for k, t in v.items()}
+        idx = torch.as_tensor(list(streams), device=self.workspace.device)
+        return {k: t.index_select(0, idx).cpu().numpy() for k, t in v.items()}
+
+    def import_state(self, state: dict):
+        v = self.state_views()
+        for k, arr in state.items():
+            if k in v:
+                v[k].copy_(torch.as_tensor(arr).view(v[k].dtype).reshape(v[k].shape))
+        torch.cuda.current_stream().synchronize()
+
+
+# Module-level aliases with the C ABI's names.
+def tkv_quantize_append(cache: TkvCache, k, v, cls, pos, stream=None):
+    return cache.quantize_append(k, v, cls, pos, stream)
+
+
+def tkv_decode_attention(cache: TkvCache, q, softmax_scale, out=None, stream=None):
+    return cache.decode_attention(q, softmax_scale, out, stream)
+
+
+def tkv_evict_compact(cache: TkvCache, budget, stream=None):
+    return cache.evict_compact(budget, stream)

@@ -105,12 +105,14 @@ def normal_bf16(seed: int, layer: int, tid: int, B: int, H: int, pos0: int, T: i
     return _normal_from_counters(stream_base(seed, layer, tid), ctr)
 
 
-def normal_bf16_chunked(seed, layer, tid, B, H, pos0, T, D, device="cpu", chunk_T=4096):
+def normal_bf16_chunked(seed, layer, tid, B, H, pos0, T, D, device="cpu", b0: int = 0,
+                        chunk_elems: int = 1 << 26):
     """Same values as ``normal_bf16``; generated in position chunks to bound temporaries."""
     out = torch.empty((B, H, T, D), dtype=torch.bfloat16, device=device)
+    chunk_T = max(1, chunk_elems // max(1, B * H * D))
     for t0 in range(0, T, chunk_T):
         tt = min(chunk_T, T - t0)
-        out[:, :, t0:t0 + tt] = normal_bf16(seed, layer, tid, B, H, pos0 + t0, tt, D, device)
+        out[:, :, t0:t0 + tt] = normal_bf16(seed, layer, tid, B, H, pos0 + t0, tt, D, device, b0)
     return out
 
 
@@ -203,3 +205,49 @@ WORKLOADS = {
                                      p_r=0.4, p_e=0.4, outliers=True, budget=1638, steps=1024,
                                      evict_every=64, layers=32),
 }
+
+
+def class_counts(cls: torch.Tensor, n_protect: int, pos0: int = 0) -> list[int]:
+    """Max over batch rows of the number of positions stored in each class
+    (positions below n_protect count as class 0).  Used to size pools."""
+    B, T = cls.shape
+    pos = torch.arange(pos0, pos0 + T).view(1, T).expand(B, T)
+    eff = torch.where(pos < n_protect, torch.zeros_like(cls), cls)
+    return [int((eff == c).sum(dim=1).max().item()) for c in range(4)]
+
+
+def prefill_inputs(name: str, seed: int = 0, layer: int = 0, device="cpu", b0: int = 0,
+                   B: int | None = None, **over):
+    """Inputs of a named workload: dict with the workload parameters plus
+    k, v (bf16 [B, Hkv, ctx, D]), cls (uint8 [B, ctx + steps]), pos (int32 [B, ctx]),
+    and cap (slots per class sized for the whole run)."""
+    w = dict(WORKLOADS[name])
+    w.update(over)
+    if B is not None:
+        w["B"] = B
+    Bn, Hkv, D, ctx = w["B"], w["Hkv"], w["D"], w["ctx"]
+    k = normal_bf16_chunked(seed, layer, TID_K, Bn, Hkv, 0, ctx, D, device, b0)
+    v = normal_bf16_chunked(seed, layer, TID_V, Bn, Hkv, 0, ctx, D, device, b0)
+    if w["outliers"]:
+        k = apply_k_outliers(k, seed, layer)
+    total = ctx + w["steps"]
+    cls_all = class_ids(seed, b0 + Bn, total, w["p_r"], w["p_e"])[b0:]
+    w.update(k=k, v=v, cls=cls_all, pos=positions(Bn, 0, ctx),
+             cap=[c + 1 for c in class_counts(cls_all, w["n_protect"])],
+             G=w["Hq"] // Hkv, seed=seed, layer=layer, b0=b0)
+    return w
+
+
+def decode_inputs(w: dict, step: int, device="cpu"):
+    """Inputs of decode step `step` (position ctx + step): k, v [B, Hkv, 1, D],
+    cls/pos [B, 1], q [B, Hq, D]."""
+    B, Hkv, Hq, D, p = w["B"], w["Hkv"], w["Hq"], w["D"], w["ctx"] + step
+    seed, layer, b0 = w["seed"], w["layer"], w.get("b0", 0)
+    k = normal_bf16(seed, layer, TID_K, B, Hkv, p, 1, D, device, b0)
+    if w["outliers"]:
+        k = apply_k_outliers(k, seed, layer)
+    v = normal_bf16(seed, layer, TID_V, B, Hkv, p, 1, D, device, b0)
+    q = normal_bf16(seed, layer, TID_Q, B, Hq, p, 1, D, device, b0)[:, :, 0].contiguous()
+    cls = w["cls"][:, p:p + 1].contiguous().to(device)
+    pos = torch.full((B, 1), p, dtype=torch.int32, device=device)
+    return k, v, cls, pos, q

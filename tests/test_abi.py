@@ -1,0 +1,96 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports every
+function include/tkv.h declares, sizes workspaces and rejects bad arguments on the
+host without launching anything."""
+import ctypes
+import re
+from pathlib import Path
+
+import pytest
+
+from reasoning_model_kv_b200 import tkv
+
+ROOT = Path(__file__).resolve().parents[1]
+
+
+def declared_functions():
+    text = (ROOT / "include" / "tkv.h").read_text()
+    return sorted(set(re.findall(r"TKV_API\s+[\w\s\*]*?\b(tkv_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_exports():
+    assert declared_functions() == sorted(tkv.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    L = tkv.lib()
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def _cfg(**kw):
+    args = dict(B=2, Hkv=2, G=4, cap=[8, 16, 16, 16], n_protect=4, max_append=64)
+    args.update(kw)
+    return tkv.make_config(**args)
+
+
+def test_workspace_bytes_valid_and_invalid():
+    n = tkv.tkv_workspace_bytes(_cfg())
+    assert n > 0 and n % 256 == 0
+    bigger = tkv.tkv_workspace_bytes(_cfg(cap=[8, 32, 16, 16]))
+    assert bigger > n
+    for bad in (dict(G=3), dict(B=0), dict(cap=[1, -1, 0, 0]), dict(max_append=0)):
+        assert tkv.tkv_workspace_bytes(_cfg(**bad)) == 0
+    cfg = _cfg()
+    cfg.D = 64
+    assert tkv.tkv_workspace_bytes(cfg) == 0
+    cfg = _cfg()
+    cfg.bits[1] = 6
+    assert tkv.tkv_workspace_bytes(cfg) == 0
+
+
+def test_layout_is_aligned_and_inside_workspace():
+    L = tkv.lib()
+    cfg = _cfg()
+    n = L.tkv_workspace_bytes(ctypes.byref(cfg))
+    h = ctypes.c_void_p()
+    # tkv_create only records the pointer: a fake aligned address is fine on the host
+    assert L.tkv_create(ctypes.byref(cfg), ctypes.c_void_p(1 << 20), n, ctypes.byref(h)) == 0
+    lay = tkv.TkvLayout()
+    assert L.tkv_get_layout(h, ctypes.byref(lay)) == 0
+    offs = [lay.n, lay.ft, lay.hw, lay.err] + [getattr(lay, f)[c] for f in
+                                               ("handle", "pos", "score", "fs", "pool") for c in range(4)]
+    assert all(o % 256 == 0 for o in offs)
+    assert lay.state_bytes <= lay.total_bytes == n
+    assert list(lay.rec_bytes) == [512, 288, 160, 96]
+    assert L.tkv_destroy(h) == 0
+
+
+def test_create_rejects_bad_workspace():
+    L = tkv.lib()
+    cfg = _cfg()
+    n = L.tkv_workspace_bytes(ctypes.byref(cfg))
+    h = ctypes.c_void_p()
+    assert L.tkv_create(ctypes.byref(cfg), None, n, ctypes.byref(h)) == tkv.TKV_ERR_INVALID
+    assert L.tkv_create(ctypes.byref(cfg), ctypes.c_void_p(4096 + 16), n, ctypes.byref(h)) == tkv.TKV_ERR_INVALID
+    assert L.tkv_create(ctypes.byref(cfg), ctypes.c_void_p(4096), n - 1, ctypes.byref(h)) == tkv.TKV_ERR_INVALID
+    assert b"small" in L.tkv_last_error_string()
+
+
+def test_calls_reject_bad_arguments_without_launching():
+    L = tkv.lib()
+    cfg = _cfg()
+    n = L.tkv_workspace_bytes(ctypes.byref(cfg))
+    h = ctypes.c_void_p()
+    assert L.tkv_create(ctypes.byref(cfg), ctypes.c_void_p(1 << 20), n, ctypes.byref(h)) == 0
+    p = ctypes.c_void_p(1 << 24)
+    INV = tkv.TKV_ERR_INVALID
+    assert L.tkv_quantize_append(h, None, p, p, p, 1, None) == INV
+    assert L.tkv_quantize_append(h, p, p, p, p, 0, None) == INV
+    assert L.tkv_quantize_append(h, p, p, p, p, 65, None) == INV          # > max_append
+    assert L.tkv_quantize_append(h, ctypes.c_void_p((1 << 24) + 8), p, p, p, 1, None) == INV
+    assert L.tkv_decode_attention(h, None, 0.1, p, None) == INV
+    assert L.tkv_decode_attention(h, p, 0.1, ctypes.c_void_p((1 << 24) + 4), None) == INV
+    assert L.tkv_evict_compact(h, -1, None) == INV
+    assert L.tkv_evict_compact(None, 3, None) == INV
+    assert L.tkv_launch_count(h) == 0
+    assert L.tkv_destroy(h) == 0

@@ -1,0 +1,282 @@
+"""Parity of the CUDA path (called through the C ABI) with the CPU oracle.
+
+Every comparison hands the oracle the GPU's pre-call state, so a difference is
+always attributable to one call: codes/scales/zeros/tables/free stacks are
+compared bit for bit, attention output within max-abs 2e-3, scores within the
+fp32 dot-product bound stated in tests/gpu_harness.py.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import oracle as orc
+from reasoning_model_kv_b200 import TkvCache, TkvError, tkv
+from tests.conftest import gpu_available
+from tests.gpu_harness import (OUT_ATOL, build_pair, compare_states, np_bits, oracle_for,
+                               rows_streams, score_error)
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not gpu_available(), reason="needs a CUDA device")]
+
+DEV = "cuda"
+SCALE = 128 ** -0.5
+
+
+def _decode_step(w, gpu, o, rows, step, check=True):
+    """Lock-step append + attention on GPU and oracle (oracle first loads the GPU state)."""
+    k, v, cls, pos, q = synth.decode_inputs(w, step)
+    sub = rows_streams(gpu, rows)
+    pre = gpu.export_state(sub)
+    o.load_state(pre)
+    gpu.quantize_append(k.to(DEV), v.to(DEV), cls.to(DEV), pos.to(DEV))
+    assert o.append(np_bits(k[rows]), np_bits(v[rows]), cls[rows].numpy(), pos[rows].numpy()) == 0
+    if check:
+        compare_states(gpu.export_state(sub), o.state, what=f"append step {step}")
+    out = gpu.decode_attention(q.to(DEV), SCALE)
+    ref = o.attend(np_bits(q[rows]), SCALE)
+    got = out[rows].cpu().numpy()
+    err = float(np.max(np.abs(got - ref)))
+    assert err <= OUT_ATOL, f"step {step}: max-abs {err}"
+    if check:
+        compare_states(gpu.export_state(sub), o.state, scores="tol", what=f"attention step {step}")
+    assert gpu.poll_error() == tkv.TKV_OK
+    return err
+
+
+def _evict_lockstep(gpu, o, rows, budget):
+    sub = rows_streams(gpu, rows)
+    o.load_state(gpu.export_state(sub))
+    gpu.evict_compact(budget)
+    assert o.evict(budget) == 0
+    compare_states(gpu.export_state(sub), o.state, what=f"evict {budget}")
+
+
+# ----------------------------------------------------------------------------
+def test_tiny_prefill_decode_evict_reuse():
+    """2k-token single-layer workload: prefill, decode step, eviction to 512, and
+    a second step that reuses evicted slots."""
+    w, gpu, o, rows = build_pair("tiny_b1_ctx2k")
+    compare_states(gpu.export_state(), o.state, what="prefill")
+    _decode_step(w, gpu, o, rows, 0)
+    _evict_lockstep(gpu, o, rows, w["budget"])
+    n = gpu.export_state()["n"]
+    assert (n[:, 1:].sum(axis=1) == w["budget"]).all()
+    w2 = dict(w, steps=2)
+    w2["cls"] = synth.class_ids(0, w["B"], w["ctx"] + 2, w["p_r"], w["p_e"])
+    _decode_step(w2, gpu, o, rows, 1)
+    assert gpu.launch_count() > 0
+
+
+def test_kept_sets_free_running_match_up_to_near_ties():
+    """GPU and oracle each evict on their own accumulated scores; kept sets agree
+    except for entries whose oracle scores tie the threshold within the score
+    tolerance."""
+    w, gpu, o, rows = build_pair("tiny_b1_ctx2k")
+    for step in range(3):
+        k, v, cls, pos, q = synth.decode_inputs(dict(w, cls=synth.class_ids(0, 1, w["ctx"] + 3, 0.4, 0.4)), step)
+        gpu.quantize_append(k.to(DEV), v.to(DEV), cls.to(DEV), pos.to(DEV))
+        o.append(np_bits(k), np_bits(v), cls.numpy(), pos.numpy())
+        gpu.decode_attention(q.to(DEV), SCALE)
+        o.attend(np_bits(q), SCALE)
+    g_before = gpu.export_state()
+    gpu.evict_compact(w["budget"])
+    o_before = o.copy_state()
+    o.evict(w["budget"])
+    g = gpu.export_state()
+    for s in range(gpu.S):
+        kept_g = set(np.concatenate([g[f"pos{c}"][s, :g["n"][s, c]] for c in range(4)]).tolist())
+        kept_o = set(np.concatenate([o.state[f"pos{c}"][s, :o.state["n"][s, c]] for c in range(4)]).tolist())
+        diff = kept_g ^ kept_o
+        if diff:
+            sc = {}
+            for c in range(4):
+                n = o_before["n"][s, c]
+                sc.update(zip(o_before[f"pos{c}"][s, :n].tolist(), o_before[f"score{c}"][s, :n].tolist()))
+            thr = sorted((v for p, v in sc.items() if p >= w["n_protect"]), reverse=True)[w["budget"] - 1]
+            for p in diff:
+                assert abs(sc[p] - thr) <= 1e-4 * thr, (p, sc[p], thr)
+
+
+@pytest.mark.parametrize("G,n_protect,outliers", [(1, 4, False), (2, 128, True), (4, 4, True),
+                                                  (8, 128, False)])
+def test_gqa_widths_and_windows(G, n_protect, outliers):
+    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", B=2, Hq=2 * G, Hkv=2, ctx=709,
+                                 n_protect=n_protect, outliers=outliers, steps=2)
+    compare_states(gpu.export_state(), o.state, what="prefill")
+    _decode_step(w, gpu, o, rows, 0)
+    _evict_lockstep(gpu, o, rows, 300)
+    _decode_step(w, gpu, o, rows, 1)
+
+
+def test_multi_token_append_after_eviction_reuses_slots_in_order():
+    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", ctx=600, steps=80)
+    gpu.decode_attention(synth.decode_inputs(w, 0)[4].to(DEV), SCALE)
+    _evict_lockstep(gpu, o, rows, 100)
+    T = 77
+    p0 = w["ctx"]
+    k = synth.normal_bf16(0, 0, synth.TID_K, 1, 2, p0, T, 128)
+    v = synth.normal_bf16(0, 0, synth.TID_V, 1, 2, p0, T, 128)
+    cls = w["cls"][:, p0:p0 + T].contiguous()
+    pos = synth.positions(1, p0, T)
+    o.load_state(gpu.export_state())
+    gpu.quantize_append(k.to(DEV), v.to(DEV), cls.to(DEV), pos.to(DEV))
+    assert o.append(np_bits(k), np_bits(v), cls.numpy(), pos.numpy()) == 0
+    compare_states(gpu.export_state(), o.state, what="append T=77 after eviction")
+
+
+def test_empty_cache_and_single_token():
+    gpu = TkvCache(1, 2, 4, cap=[4, 4, 4, 4], n_protect=0)
+    q = synth.normal_bf16(0, 0, synth.TID_Q, 1, 8, 0, 1, 128)[:, :, 0].contiguous()
+    out = gpu.decode_attention(q.to(DEV), SCALE)
+    assert not out.any()
+    k = synth.normal_bf16(0, 0, synth.TID_K, 1, 2, 0, 1, 128)
+    cls = torch.tensor([[3]], dtype=torch.uint8)
+    pos = torch.zeros((1, 1), dtype=torch.int32)
+    gpu.quantize_append(k.to(DEV), k.to(DEV), cls.to(DEV), pos.to(DEV))
+    o = orc.OracleCache(1, 2, 4, cap=[4, 4, 4, 4], n_protect=0)
+    o.append(np_bits(k), np_bits(k), cls.numpy(), pos.numpy())
+    out = gpu.decode_attention(q.to(DEV), SCALE).cpu().numpy()
+    ref = o.attend(np_bits(q), SCALE)
+    assert np.max(np.abs(out - ref)) <= OUT_ATOL
+    g = gpu.export_state()
+    assert abs(g["score3"][0, 0] - 4.0) < 1e-6 and abs(g["score3"][1, 0] - 4.0) < 1e-6
+
+
+def test_budget_edge_cases():
+    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", ctx=300, n_protect=17)
+    gpu.decode_attention(synth.decode_inputs(w, 0)[4].to(DEV), SCALE)
+    before = gpu.export_state()
+    gpu.evict_compact(300)                     # budget >= candidates: untouched
+    after = gpu.export_state()
+    for key in before:
+        assert np.array_equal(before[key], after[key]), key
+    _evict_lockstep(gpu, o, rows, 0)           # evict every unprotected token
+    g = gpu.export_state()
+    assert (g["n"].sum(axis=1) == 17).all()
+
+
+def test_all_scores_equal_keep_lowest_positions():
+    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", ctx=500)
+    views = gpu.state_views()
+    for c in range(4):
+        views[f"score{c}"].fill_(0.5)
+    _evict_lockstep(gpu, o, rows, 40)
+    g = gpu.export_state()
+    for s in range(gpu.S):
+        kept = sorted(np.concatenate([g[f"pos{c}"][s, :g["n"][s, c]] for c in range(4)]).tolist())
+        assert kept == list(range(44))
+
+
+def test_exact_key_ties_resolved_by_class_then_index():
+    """Duplicate positions with equal scores: the 64-bit key ties, so class then table
+    index decide (same rule on both sides)."""
+    B, Hkv, T = 1, 1, 40
+    gpu = TkvCache(B, Hkv, 4, cap=[4, 40, 40, 40], n_protect=0, max_append=T)
+    o = orc.OracleCache(B, Hkv, 4, cap=[4, 40, 40, 40], n_protect=0)
+    k = synth.normal_bf16(3, 0, synth.TID_K, B, Hkv, 0, T, 128)
+    cls = torch.tensor([[1 + (t % 3) for t in range(T)]], dtype=torch.uint8)
+    pos = torch.tensor([[t // 4 for t in range(T)]], dtype=torch.int32)   # duplicates
+    gpu.quantize_append(k.to(DEV), k.to(DEV), cls.to(DEV), pos.to(DEV))
+    views = gpu.state_views()
+    for c in range(4):
+        views[f"score{c}"].copy_((views[f"pos{c}"] % 3).float() * 0.25)
+    o.load_state(gpu.export_state())
+    for budget in (13, 7, 1):
+        gpu.evict_compact(budget)
+        o.evict(budget)
+        compare_states(gpu.export_state(), o.state, what=f"tie budget {budget}")
+
+
+def test_device_errors_capacity_and_invalid_class():
+    gpu = TkvCache(1, 2, 4, cap=[1, 2, 2, 2], n_protect=1, max_append=8)
+    k = synth.normal_bf16(0, 0, synth.TID_K, 1, 2, 0, 5, 128).to(DEV)
+    cls = torch.tensor([[1, 1, 1, 1, 2]], dtype=torch.uint8, device=DEV)
+    pos = torch.arange(5, dtype=torch.int32, device=DEV).view(1, 5)
+    gpu.quantize_append(k, k, cls, pos)        # class 1 gets 4 tokens but has 2 slots
+    assert gpu.poll_error() == tkv.TKV_ERR_CAPACITY
+    assert gpu.poll_error() == tkv.TKV_OK      # cleared by the poll
+    g = gpu.export_state()
+    assert g["n"][0].tolist() == [1, 2, 1, 0] and g["hw"][0].tolist() == [1, 2, 1, 0]
+    gpu2 = TkvCache(1, 1, 4, cap=[4, 4, 4, 4], n_protect=0)
+    gpu2.quantize_append(k[:, :1, :1].contiguous(), k[:, :1, :1].contiguous(),
+                         torch.tensor([[9]], dtype=torch.uint8, device=DEV),
+                         torch.zeros((1, 1), dtype=torch.int32, device=DEV))
+    assert gpu2.poll_error() == tkv.TKV_ERR_INVALID
+    assert gpu2.export_state()["n"].sum() == 0
+
+
+def test_binding_rejects_wrong_tensors():
+    gpu = TkvCache(1, 2, 4, cap=[4, 4, 4, 4], n_protect=0)
+    q = torch.zeros((1, 8, 128), dtype=torch.float32, device=DEV)
+    with pytest.raises(TkvError):
+        gpu.decode_attention(q, SCALE)
+    with pytest.raises(TkvError):
+        gpu.decode_attention(q.to(torch.bfloat16)[:, :4], SCALE)
+
+
+# ----------------------------------------------------------------------------
+# The workload shapes of the decode configurations, lock-step on sampled rows/steps
+# ----------------------------------------------------------------------------
+def test_b64_ctx32k_timed_step_sampled_rows():
+    """Batch 64 x 32/8 heads, 32k context, K outliers, 5 % budget + 128-token bf16
+    window: prefill, scoring step, eviction to 1638, then the timed step
+    (append + attention), compared on three sampled batch rows."""
+    rows = [0, 37, 63]
+    w = synth.prefill_inputs("b64_ctx32k_evict5pct", device=DEV, steps=2)
+    w["cls"] = synth.class_ids(0, w["B"], w["ctx"] + 2, w["p_r"], w["p_e"])
+    gpu = TkvCache(w["B"], w["Hkv"], w["G"], w["cap"], w["n_protect"], max_append=w["ctx"])
+    gpu.quantize_append(w["k"], w["v"], w["cls"][:, :w["ctx"]].contiguous().to(DEV), w["pos"].to(DEV))
+    del w["k"], w["v"]
+    torch.cuda.empty_cache()
+    o = oracle_for(gpu, gpu.export_state(rows_streams(gpu, rows)), B=len(rows))
+    _decode_step(w, gpu, o, rows, 0)                 # scoring step
+    _evict_lockstep(gpu, o, rows, w["budget"])
+    err = _decode_step(w, gpu, o, rows, 1)           # the timed step's work
+    assert err <= OUT_ATOL
+
+
+def test_b8_ctx16k_decode_loop_sampled_steps():
+    """Batch 8 x 32/8 heads, 16k context, 256 decode steps with eviction to 1638
+    every 128 steps; lock-step checks on one row at steps 0, 127, 128, 255."""
+    rows = [5]
+    w = synth.prefill_inputs("b8_ctx16k_256steps", device=DEV)
+    gpu = TkvCache(w["B"], w["Hkv"], w["G"], w["cap"], w["n_protect"], max_append=w["ctx"])
+    gpu.quantize_append(w["k"], w["v"], w["cls"][:, :w["ctx"]].contiguous().to(DEV), w["pos"].to(DEV))
+    o = oracle_for(gpu, gpu.export_state(rows_streams(gpu, rows)), B=1)
+    for step in range(w["steps"]):
+        if step in (0, 127, 128, 255):
+            _decode_step(w, gpu, o, rows, step)
+        else:
+            k, v, cls, pos, q = synth.decode_inputs(w, step, device=DEV)
+            gpu.quantize_append(k, v, cls, pos)
+            gpu.decode_attention(q, SCALE)
+        if (step + 1) % w["evict_every"] == 0:
+            if step == 127:
+                _evict_lockstep(gpu, o, rows, w["budget"])
+            else:
+                gpu.evict_compact(w["budget"])
+    assert gpu.poll_error() == tkv.TKV_OK
+
+
+def test_b1_ctx131k_long_decode_sampled_steps():
+    """Batch 1 x 64/8 heads (G = 8), 131k context, transition-heavy segments,
+    eviction to 4096 every 64 steps; lock-step at steps 0, 63, 64 and 200."""
+    rows = [0]
+    w = synth.prefill_inputs("b1_ctx131k_512steps", device=DEV, steps=201)
+    gpu = TkvCache(w["B"], w["Hkv"], w["G"], w["cap"], w["n_protect"], max_append=w["ctx"])
+    gpu.quantize_append(w["k"], w["v"], w["cls"][:, :w["ctx"]].contiguous().to(DEV), w["pos"].to(DEV))
+    o = oracle_for(gpu, gpu.export_state(), B=1)
+    for step in range(201):
+        if step in (0, 63, 64, 200):
+            _decode_step(w, gpu, o, rows, step)
+        else:
+            k, v, cls, pos, q = synth.decode_inputs(w, step, device=DEV)
+            gpu.quantize_append(k, v, cls, pos)
+            gpu.decode_attention(q, SCALE)
+        if (step + 1) % w["evict_every"] == 0:
+            if step == 63:
+                _evict_lockstep(gpu, o, rows, w["budget"])
+            else:
+                gpu.evict_compact(w["budget"])
+    assert gpu.poll_error() == tkv.TKV_OK
