@@ -142,6 +142,26 @@ TKV_API tkv_status tkv_quantize_append(tkv_cache *cache, const void *k, const vo
                                const uint8_t *cls, const int32_t *pos, int32_t T, void *stream);
 
 /*
+ * tkv_quantize_append without any scratch memory of the caller's (the paper has
+ * no counterpart: this is a deployment variant).  Same arguments, semantics and
+ * results as tkv_quantize_append, for callers that cannot allocate device memory
+ * and so cannot size a workspace scratch for their largest append -- e.g. code
+ * running where cudaMalloc is not allowed or an allocator must not grow.  The
+ * per-token class ranks of a multi-token append live in a fixed 2 MiB device
+ * array inside the library instead (held by every GPU that loads the library
+ * until the process exits); it calls no allocating function.
+ *   Limit: B * (T + 4) <= 524288 when T > 1 (T == 1 needs no scratch);
+ *          larger appends return TKV_ERR_INVALID and launch nothing.
+ *   The first call on each device looks up the array's device address (with
+ *   that device current); make that first call before any stream capture.
+ *   All calls share the one array and each call rewrites what it uses, so calls
+ *   that overlap on the GPU (two streams, or two caches at once) race.
+ */
+TKV_API tkv_status tkv_quantize_append_noalloc(tkv_cache *cache, const void *k, const void *v,
+                                       const uint8_t *cls, const int32_t *pos, int32_t T,
+                                       void *stream);
+
+/*
  * One decode step of GQA attention over every live token of every stream
  * (dequantised on the fly), plus score accumulation.
  *   q              device bf16 [B][Hkv*G][D]; query head h reads kv head h / G

@@ -116,6 +116,19 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 }  // namespace
 
+// Hooks for entry points defined in other translation units.
+namespace tkv {
+const Dev *cache_dev(const tkv_cache *c, int *max_append) {
+    *max_append = c->cfg.max_append;
+    return &c->dev;
+}
+void note_append(tkv_cache *c, int64_t launches, int T) {
+    c->launches += launches;
+    c->live_ub = std::min<long long>(c->dev.ncap, c->live_ub + T);
+}
+tkv_status api_fail(tkv_status st, const std::string &msg) { return fail(st, msg); }
+}  // namespace tkv
+
 extern "C" {
 
 size_t tkv_workspace_bytes(const tkv_config *cfg) {

@@ -43,7 +43,7 @@ class TkvLayout(ctypes.Structure):
 
 
 EXPORTS = ["tkv_workspace_bytes", "tkv_create", "tkv_destroy", "tkv_reset", "tkv_get_layout",
-           "tkv_quantize_append", "tkv_decode_attention", "tkv_evict_compact", "tkv_poll_error",
+           "tkv_quantize_append", "tkv_quantize_append_noalloc", "tkv_decode_attention", "tkv_evict_compact", "tkv_poll_error",
            "tkv_export_state", "tkv_import_state", "tkv_launch_count", "tkv_last_error_string"]
 
 _lib = None
@@ -67,6 +67,7 @@ def lib() -> ctypes.CDLL:
     L.tkv_reset.argtypes = [vp, vp]
     L.tkv_get_layout.argtypes = [vp, P(TkvLayout)]
     L.tkv_quantize_append.argtypes = [vp, vp, vp, vp, vp, i32, vp]
+    L.tkv_quantize_append_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, vp]
     L.tkv_decode_attention.argtypes = [vp, vp, ctypes.c_float, vp, vp]
     L.tkv_evict_compact.argtypes = [vp, i32, vp]
     L.tkv_poll_error.argtypes = [vp, vp]
@@ -76,6 +77,7 @@ def lib() -> ctypes.CDLL:
     L.tkv_launch_count.restype = ctypes.c_int64
     L.tkv_last_error_string.restype = ctypes.c_char_p
     for name in ("tkv_create", "tkv_destroy", "tkv_reset", "tkv_get_layout", "tkv_quantize_append",
+                 "tkv_quantize_append_noalloc",
                  "tkv_decode_attention", "tkv_evict_compact", "tkv_poll_error", "tkv_export_state",
                  "tkv_import_state"):
         getattr(L, name).restype = ctypes.c_int
@@ -159,6 +161,20 @@ class TkvCache:
                                          _dptr(v, torch.bfloat16, "v"),
                                          _dptr(cls, torch.uint8, "cls"),
                                          _dptr(pos, torch.int32, "pos"), T, _stream(stream)))
+
+    def quantize_append_noalloc(self, k: torch.Tensor, v: torch.Tensor, cls: torch.Tensor,
+                                pos: torch.Tensor, stream=None):
+        """Same as quantize_append, using the library's fixed device scratch instead of
+        the workspace's (for callers that cannot allocate; B*(T+4) <= 524288)."""
+        T = k.shape[2]
+        if k.shape != (self.B, self.Hkv, T, 128) or v.shape != k.shape:
+            raise TkvError(TKV_ERR_INVALID, f"k/v must be [B, Hkv, T, 128], got {tuple(k.shape)}")
+        if cls.shape != (self.B, T) or pos.shape != (self.B, T):
+            raise TkvError(TKV_ERR_INVALID, "cls/pos must be [B, T]")
+        _check(lib().tkv_quantize_append_noalloc(self._h, _dptr(k, torch.bfloat16, "k"),
+                                                 _dptr(v, torch.bfloat16, "v"),
+                                                 _dptr(cls, torch.uint8, "cls"),
+                                                 _dptr(pos, torch.int32, "pos"), T, _stream(stream)))
 
     def decode_attention(self, q: torch.Tensor, softmax_scale: float, out: torch.Tensor | None = None,
                          stream=None) -> torch.Tensor:
