@@ -50,6 +50,9 @@ def parse():
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=None)
+    ap.add_argument("--ctx", type=int, default=None,
+                    help="prefill context before the eviction (default: the workload's); the "
+                         "timed step is the same post-eviction step, with smaller pools")
     return ap.parse_args()
 
 
@@ -156,7 +159,8 @@ def setup_cache(w, dev, seed):
 
 
 def run_tkv(args, rank, world, dev):
-    w = synth.prefill_inputs(args.workload, seed=rank, device=dev, steps=2)
+    over = {"ctx": args.ctx} if args.ctx else {}
+    w = synth.prefill_inputs(args.workload, seed=rank, device=dev, steps=2, **over)
     gpu = setup_cache(w, dev, rank)
     del w["k"], w["v"]
     torch.cuda.empty_cache()
@@ -258,7 +262,8 @@ def run_tkv(args, rank, world, dev):
         "vs_baseline": None,
         "dtype": "int8/int4/int2 codes + bf16 -> fp32",
         "data": "synthetic (seeded counter-hash N(0,1) bf16, K x10 outlier channels)",
-        "config": {"workload": args.workload, "batch": B, "q_heads": w["Hq"], "kv_heads": w["Hkv"],
+        "config": {"workload": args.workload + (f" (prefill ctx {args.ctx})" if args.ctx else ""),
+                   "batch": B, "q_heads": w["Hq"], "kv_heads": w["Hkv"],
                    "head_dim": 128, "context": w["ctx"], "budget": w["budget"],
                    "bf16_window": w["n_protect"], "p_RET": [w["p_r"], w["p_e"], 1 - w["p_r"] - w["p_e"]],
                    "live_kv_tokens": kv_tokens, "packed_kv_bytes": pk,

@@ -174,19 +174,38 @@ void orc_quantize_group(const float *x, int n, int bits, uint16_t *scale_h,
     }
 }
 
-/* Pack codes little-endian within each byte: element i at bit bits*(i % (8/bits))
- * of byte i*bits/8. */
-static void pack_codes(const uint8_t *codes, int n, int bits, uint8_t *out) {
+/* Storage order of a 128-element code block (K or V).  The block is four
+ * quarters of 32 elements; quarter q holds 16 pairs of head-dim indices:
+ *   K pair p: dims 32*(p/4) + 8*q + 2*(p%4) + {0, 1}
+ *   V pair p: dims  8*p     + 2*q           + {0, 1}
+ * Each 32-bit word of the quarter holds 32/b elements (b bits each, element e
+ * at bits b*e) and 16/b pairs: pair p = w*(16/b) + s of word w puts its lower
+ * dim at element s and its upper dim at element s + 16/b (16 bits higher).
+ * Returns the head-dim index stored at element i (0..127) of the block. */
+static int storage_dim(int is_v, int bits, int i) {
+    int q = i / 32, u = i % 32;
+    int per_word = 32 / bits, pairs_per_word = 16 / bits;
+    int w = u / per_word, e = u % per_word;
+    int p = w * pairs_per_word + e % pairs_per_word;
+    int hi = e / pairs_per_word;
+    if (is_v) return 8 * p + 2 * q + hi;
+    return 32 * (p / 4) + 8 * q + 2 * (p % 4) + hi;
+}
+
+/* Pack codes (indexed by head dim) in storage order, little-endian within each
+ * byte: storage element i at bit bits*(i % (8/bits)) of byte i*bits/8. */
+static void pack_codes(const uint8_t *codes, int n, int bits, int is_v, uint8_t *out) {
     int per = 8 / bits;
     memset(out, 0, (size_t)n * bits / 8);
     for (int i = 0; i < n; ++i)
-        out[i / per] |= (uint8_t)(codes[i] << (bits * (i % per)));
+        out[i / per] |= (uint8_t)(codes[storage_dim(is_v, bits, i)] << (bits * (i % per)));
 }
 
-static void unpack_codes(const uint8_t *in, int n, int bits, uint8_t *codes) {
+static void unpack_codes(const uint8_t *in, int n, int bits, int is_v, uint8_t *codes) {
     int per = 8 / bits;
     int mask = (1 << bits) - 1;
-    for (int i = 0; i < n; ++i) codes[i] = (in[i / per] >> (bits * (i % per))) & mask;
+    for (int i = 0; i < n; ++i)
+        codes[storage_dim(is_v, bits, i)] = (in[i / per] >> (bits * (i % per))) & mask;
 }
 
 static void put_u16(uint8_t *p, uint16_t v) {
@@ -197,15 +216,16 @@ static void put_u16(uint8_t *p, uint16_t v) {
 static uint16_t get_u16(const uint8_t *p) { return (uint16_t)(p[0] | (p[1] << 8)); }
 
 /* Record layout (all little-endian):
- *   bf16:  [K: D x bf16][V: D x bf16]
- *   b-bit: [K codes: D*b/8 bytes][V codes: D*b/8 bytes]
+ *   bf16:  [K: D x bf16][V: D x bf16], each block in the storage order above (b = 16)
+ *   b-bit: [K codes: D*b/8 bytes][V codes: D*b/8 bytes]  (storage order above)
  *          [K scale x ngroups][K zero x ngroups][V scale x ngroups][V zero x ngroups] (fp16)
+ * Groups are 32 consecutive head dims; only the placement of codes is permuted.
  */
 void orc_pack_record(int bits, int D, int group, const uint16_t *k, const uint16_t *v,
                      uint8_t *rec) {
     if (bits == 16) {
-        for (int d = 0; d < D; ++d) put_u16(rec + 2 * d, k[d]);
-        for (int d = 0; d < D; ++d) put_u16(rec + 2 * D + 2 * d, v[d]);
+        for (int i = 0; i < D; ++i) put_u16(rec + 2 * i, k[storage_dim(0, 16, i)]);
+        for (int i = 0; i < D; ++i) put_u16(rec + 2 * D + 2 * i, v[storage_dim(1, 16, i)]);
         return;
     }
     int ng = D / group;
@@ -224,7 +244,7 @@ void orc_pack_record(int bits, int D, int group, const uint16_t *k, const uint16
             put_u16(meta + (which * 2 * ng + g) * 2, s);
             put_u16(meta + (which * 2 * ng + ng + g) * 2, z);
         }
-        pack_codes(allc, D, bits, rec + which * cb);
+        pack_codes(allc, D, bits, which, rec + which * cb);
     }
 }
 
@@ -232,8 +252,9 @@ void orc_pack_record(int bits, int D, int group, const uint16_t *k, const uint16
 void orc_unpack_record(int bits, int D, int group, const uint8_t *rec, double *k_hat,
                        double *v_hat) {
     if (bits == 16) {
-        for (int d = 0; d < D; ++d) k_hat[d] = bf16_to_f32(get_u16(rec + 2 * d));
-        for (int d = 0; d < D; ++d) v_hat[d] = bf16_to_f32(get_u16(rec + 2 * D + 2 * d));
+        for (int i = 0; i < D; ++i) k_hat[storage_dim(0, 16, i)] = bf16_to_f32(get_u16(rec + 2 * i));
+        for (int i = 0; i < D; ++i)
+            v_hat[storage_dim(1, 16, i)] = bf16_to_f32(get_u16(rec + 2 * D + 2 * i));
         return;
     }
     int ng = D / group;
@@ -242,7 +263,7 @@ void orc_unpack_record(int bits, int D, int group, const uint8_t *rec, double *k
     uint8_t codes[512];
     for (int which = 0; which < 2; ++which) {
         double *dst = which == 0 ? k_hat : v_hat;
-        unpack_codes(rec + which * cb, D, bits, codes);
+        unpack_codes(rec + which * cb, D, bits, which, codes);
         for (int d = 0; d < D; ++d) {
             int g = d / group;
             double s = orc_f16_to_f64(get_u16(meta + (which * 2 * ng + g) * 2));

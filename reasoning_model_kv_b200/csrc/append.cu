@@ -5,7 +5,9 @@
 //
 // One warp packs one (stream, token): lane l owns head-dim elements
 // [4l, 4l+4), so a 32-element group is 8 lanes and its min/max is a 3-step
-// xor-shuffle reduction.  The quantiser uses only correctly rounded fp32
+// xor-shuffle reduction.  Codes are then re-gathered through shared memory into
+// the record's storage order (see stored_dim), which the decode kernel reads
+// with wide loads straight into tensor-core operand registers.  The quantiser uses only correctly rounded fp32
 // operations (__fsub_rn, __fdiv_rn, __float2int_rn) and the hardware's
 // directed fp32->fp16 conversions, so codes, scales and zeros are bit-exact
 // with any IEEE implementation of the same definition.
@@ -70,11 +72,39 @@ __global__ void append_rank_kernel(Dev d, const uint8_t *__restrict__ cls,
     if (threadIdx.x < 4) d.totals[b * 4 + threadIdx.x] = carry[threadIdx.x];
 }
 
-// Quantise one 128-element bf16 row held as 4 elements per lane and write its
-// packed codes and its (scale, zero) pairs.
-template <int BITS>
-__device__ __forceinline__ void quantize_row(const float (&x)[4], int lane, uint8_t *codes,
-                                             __half *meta /* [scale x4][zero x4] */) {
+// Head-dim index held by storage element e of word w in quarter q of a code
+// block (K or V) with BITS-bit elements.  Quarter q holds 16 dim pairs:
+//   K pair p: 32*(p/4) + 8*q + 2*(p%4) + {0,1}   (the lane-quad operand of one
+//             m16n8k16 k-step per group half),
+//   V pair p: 8*p + 2*q + {0,1}                   (one column pair of an 8x8 block);
+// a word holds 16/BITS pairs, pair s at elements s and s + 16/BITS, so the two
+// members of a pair are always 16 bits apart.
+template <int BITS, bool IS_V>
+__device__ __forceinline__ int stored_dim(int q, int w, int e) {
+    constexpr int ppw = 16 / BITS;
+    const int p = w * ppw + e % ppw, hi = e / ppw;
+    return IS_V ? 8 * p + 2 * q + hi : 32 * (p / 4) + 8 * q + 2 * (p % 4) + hi;
+}
+
+// Word `word` (0 .. 4*BITS-1) of a code block whose codes, indexed by head dim,
+// are in shared memory.
+template <int BITS, bool IS_V>
+__device__ __forceinline__ uint32_t code_word(const uint8_t *codes, int word) {
+    const int q = word / BITS, w = word % BITS;
+    uint32_t r = 0;
+#pragma unroll
+    for (int e = 0; e < 32 / BITS; ++e)
+        r |= static_cast<uint32_t>(codes[stored_dim<BITS, IS_V>(q, w, e)]) << (BITS * e);
+    return r;
+}
+
+// Quantise one 128-element bf16 row held as 4 elements per lane (lane l owns dims
+// 4l..4l+3, so a group is 8 lanes); write the codes in storage order and the
+// group's (scale, zero).
+template <int BITS, bool IS_V>
+__device__ __forceinline__ void quantize_row(const float (&x)[4], int lane, uint8_t *codes_out,
+                                             __half *meta /* [scale x4][zero x4] */,
+                                             uint8_t *stage /* 128 bytes of this warp */) {
     constexpr int kQmax = (1 << BITS) - 1;
     float mn = fminf(fminf(x[0], x[1]), fminf(x[2], x[3]));
     float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
@@ -88,7 +118,7 @@ __device__ __forceinline__ void quantize_row(const float (&x)[4], int lane, uint
     const float step = __fdiv_rn(__fsub_rn(mx, zf), static_cast<float>(kQmax));
     const __half sh = __float2half_ru(step);
     const float sf = __half2float(sh);
-    uint32_t q[4];
+    uint32_t packed = 0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         int v = 0;
@@ -96,16 +126,13 @@ __device__ __forceinline__ void quantize_row(const float (&x)[4], int lane, uint
             v = __float2int_rn(__fdiv_rn(__fsub_rn(x[i], zf), sf));
             v = v < 0 ? 0 : (v > kQmax ? kQmax : v);
         }
-        q[i] = static_cast<uint32_t>(v);
+        packed |= static_cast<uint32_t>(v) << (8 * i);
     }
-    if constexpr (BITS == 8) {
-        reinterpret_cast<uint32_t *>(codes)[lane] = q[0] | (q[1] << 8) | (q[2] << 16) | (q[3] << 24);
-    } else if constexpr (BITS == 4) {
-        reinterpret_cast<uint16_t *>(codes)[lane] =
-            static_cast<uint16_t>(q[0] | (q[1] << 4) | (q[2] << 8) | (q[3] << 12));
-    } else {
-        codes[lane] = static_cast<uint8_t>(q[0] | (q[1] << 2) | (q[2] << 4) | (q[3] << 6));
-    }
+    __syncwarp();
+    reinterpret_cast<uint32_t *>(stage)[lane] = packed;   // codes by head dim
+    __syncwarp();
+    if (lane < 4 * BITS)
+        reinterpret_cast<uint32_t *>(codes_out)[lane] = code_word<BITS, IS_V>(stage, lane);
     if ((lane & 7) == 0) {
         const int g = lane >> 3;
         meta[g] = sh;
@@ -122,23 +149,40 @@ __device__ __forceinline__ void load_row(const __nv_bfloat16 *src, int lane, flo
     x[3] = __uint_as_float(raw.y & 0xffff0000u);
 }
 
+// bf16 row -> storage order: word w of quarter q holds the pair (p = w) of 16-bit values.
+template <bool IS_V>
+__device__ __forceinline__ void store_bf16_row(const uint2 &raw, int lane, uint8_t *dst,
+                                               uint16_t *stage /* 128 halves */) {
+    __syncwarp();
+    reinterpret_cast<uint2 *>(stage)[lane] = raw;          // values by head dim
+    __syncwarp();
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const int word = lane + 32 * k, q = word / 16, w = word % 16;
+        const uint32_t lo = stage[stored_dim<16, IS_V>(q, w, 0)];
+        const uint32_t hi = stage[stored_dim<16, IS_V>(q, w, 1)];
+        reinterpret_cast<uint32_t *>(dst)[word] = lo | (hi << 16);
+    }
+}
+
 template <int BITS>
 __device__ __forceinline__ void pack_record(const __nv_bfloat16 *k, const __nv_bfloat16 *v,
-                                            uint8_t *rec, int lane) {
+                                            uint8_t *rec, int lane, uint8_t *stage) {
     float x[4];
     uint2 raw;
     if constexpr (BITS == 16) {
+        uint16_t *st16 = reinterpret_cast<uint16_t *>(stage);
         load_row(k, lane, x, raw);
-        reinterpret_cast<uint2 *>(rec)[lane] = raw;
+        store_bf16_row<false>(raw, lane, rec, st16);
         load_row(v, lane, x, raw);
-        reinterpret_cast<uint2 *>(rec + 2 * kD)[lane] = raw;
+        store_bf16_row<true>(raw, lane, rec + 2 * kD, st16);
     } else {
         constexpr int cb = kD * BITS / 8;
         __half *meta = reinterpret_cast<__half *>(rec + 2 * cb);
         load_row(k, lane, x, raw);
-        quantize_row<BITS>(x, lane, rec, meta);
+        quantize_row<BITS, false>(x, lane, rec, meta, stage);
         load_row(v, lane, x, raw);
-        quantize_row<BITS>(x, lane, rec + cb, meta + 2 * kNG);
+        quantize_row<BITS, true>(x, lane, rec + cb, meta + 2 * kNG, stage);
     }
 }
 
@@ -146,6 +190,7 @@ template <bool kSingle>
 __global__ void __launch_bounds__(256) append_pack_kernel(
     Dev d, const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ v,
     const uint8_t *__restrict__ cls, const int32_t *__restrict__ pos, int T) {
+    __shared__ __align__(16) uint8_t stage_all[8 * 2 * kD];   // per warp: a row by head dim
     const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (gw >= d.S * T) return;
@@ -179,11 +224,12 @@ __global__ void __launch_bounds__(256) append_pack_kernel(
     }
     uint8_t *rec = d.pool[c] + ((size_t)s * cap + slot) * d.rec[c];
     const size_t row = ((size_t)s * T + t) * kD;
+    uint8_t *stage = stage_all + (threadIdx.x >> 5) * 2 * kD;
     switch (c) {
-        case 0: pack_record<16>(k + row, v + row, rec, lane); break;
-        case 1: pack_record<8>(k + row, v + row, rec, lane); break;
-        case 2: pack_record<4>(k + row, v + row, rec, lane); break;
-        default: pack_record<2>(k + row, v + row, rec, lane); break;
+        case 0: pack_record<16>(k + row, v + row, rec, lane, stage); break;
+        case 1: pack_record<8>(k + row, v + row, rec, lane, stage); break;
+        case 2: pack_record<4>(k + row, v + row, rec, lane, stage); break;
+        default: pack_record<2>(k + row, v + row, rec, lane, stage); break;
     }
     __syncwarp();  // every lane has read the pre-call counters
     if (kSingle && lane == 0) {

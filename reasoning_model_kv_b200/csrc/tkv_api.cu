@@ -31,7 +31,6 @@ tkv_status fail(tkv_status st, const std::string &msg) {
 }
 
 constexpr size_t kAlign = 256;
-constexpr int kMaxSplits = 64;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
@@ -52,7 +51,7 @@ bool valid_config(const tkv_config *c, std::string *why) {
     }
     if (ncap > (1ll << 30)) { *why = "sum of cap too large"; return false; }
     if (c->max_append < 1 || c->max_append > (1 << 24)) { *why = "max_append must be in [1, 2^24]"; return false; }
-    if ((long long)c->B * c->Hkv > (1 << 20)) { *why = "too many streams"; return false; }
+    if ((long long)c->B * c->Hkv > 65535) { *why = "B * Hkv must be <= 65535"; return false; }
     return true;
 }
 
@@ -77,10 +76,10 @@ void make_layout(const tkv_config &c, tkv_layout *lay, tkv::Dev *dev, uint8_t *b
         lay->pool[k] = take(S * (size_t)c.cap[k] * lay->rec_bytes[k]);
     }
     lay->state_bytes = off;
-    const int ncap = c.cap[0] + c.cap[1] + c.cap[2] + c.cap[3];
+    // logits rows padded to 32 entries so every CTA's slice starts on a 128-byte line
+    const int ncap = (c.cap[0] + c.cap[1] + c.cap[2] + c.cap[3] + 31) & ~31;
     const size_t o_rank = take((size_t)c.B * c.max_append * sizeof(int32_t));
     const size_t o_tot = take((size_t)c.B * 4 * sizeof(int32_t));
-    const size_t o_part = take(S * kMaxSplits * c.G * (tkv::kD + 2) * sizeof(float));
     const size_t o_lg = take(S * (size_t)ncap * c.G * sizeof(float));
     lay->total_bytes = off;
     if (!dev) return;
@@ -101,9 +100,7 @@ void make_layout(const tkv_config &c, tkv_layout *lay, tkv::Dev *dev, uint8_t *b
     }
     dev->rank = reinterpret_cast<int32_t *>(base + o_rank);
     dev->totals = reinterpret_cast<int32_t *>(base + o_tot);
-    dev->part = reinterpret_cast<float *>(base + o_part);
     dev->logits = reinterpret_cast<float *>(base + o_lg);
-    dev->max_splits = kMaxSplits;
     dev->ncap = ncap;
 }
 
@@ -203,9 +200,7 @@ tkv_status tkv_decode_attention(tkv_cache *c, const void *q, float softmax_scale
     if (!q || !out) return fail(TKV_ERR_INVALID, "NULL q or out");
     if (!aligned16(q) || !aligned16(out)) return fail(TKV_ERR_INVALID, "q and out must be 16-byte aligned");
     const long long ub = std::max(1ll, c->live_ub);
-    int splits = (int)std::min<long long>(kMaxSplits, (ub + 255) / 256);
-    splits = std::max(1, splits);
-    cudaError_t e = tkv::launch_attention(c->dev, q, softmax_scale, out, splits,
+    cudaError_t e = tkv::launch_attention(c->dev, q, softmax_scale, out, ub,
                                           static_cast<cudaStream_t>(stream), &c->launches);
     return cuda_status(e, "tkv_decode_attention");
 }

@@ -31,10 +31,8 @@ struct Dev {
     // scratch
     int32_t *rank;     // [B][max_append] rank of a new token within its class
     int32_t *totals;   // [B][4] tokens per class in the current append
-    float *part;       // [S][max_splits][G][kD + 2] split partials (m, l, O)
-    float *logits;     // [S][ncap][G] raw logits of the current step
-    int max_splits;
-    int ncap;          // sum of cap[c]
+    float *logits;     // [S][ncap][G] raw logits (log2 domain) of the current step
+    int ncap;          // sum of cap[c], rounded up to a multiple of 32
 };
 
 enum : uint32_t { kErrInvalid = 1, kErrCapacity = 2, kErrTimeout = 4 };
@@ -48,8 +46,8 @@ __device__ __forceinline__ void raise_error(uint32_t *err, uint32_t code, uint32
 // of kernels it launched to *launches).
 cudaError_t launch_append(const Dev &d, const void *k, const void *v, const uint8_t *cls,
                           const int32_t *pos, int T, cudaStream_t st, int64_t *launches);
-cudaError_t launch_attention(const Dev &d, const void *q, float scale, float *out, int splits,
-                             cudaStream_t st, int64_t *launches);
+cudaError_t launch_attention(const Dev &d, const void *q, float scale, float *out,
+                             long long live_ub, cudaStream_t st, int64_t *launches);
 cudaError_t launch_evict(const Dev &d, int budget, cudaStream_t st, int64_t *launches);
 
 }  // namespace tkv

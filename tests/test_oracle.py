@@ -168,44 +168,69 @@ def test_error_bound_every_element_tiny_workload():
 
 
 # --------------------------------------------------------------------------
-# record packing (layout: K codes | V codes | K scales | K zeros | V scales | V zeros)
+# record packing.  Layout: K codes | V codes | K scales | K zeros | V scales | V zeros.
+# A code block is four 32-element quarters; quarter q holds 16 pairs of dims,
+#   K pair p: 32*(p//4) + 8q + 2*(p%4) + {0,1};   V pair p: 8p + 2q + {0,1},
+# and a 32-bit word holds 16/b pairs, pair s of the word at elements s and s + 16/b.
 # --------------------------------------------------------------------------
 def test_pack_hand_built_q2():
-    # K[d] = d % 4: every group has min 0, max 3 -> zero 0.0, scale 1.0 (fp16 0x3C00),
-    # codes = d % 4; byte j holds elements 4j..4j+3 at bits 0,2,4,6: 0|1<<2|2<<4|3<<6 = 0xE4.
+    # K[d] = d % 4: zero 0.0, scale 1.0 (fp16 0x3C00), code = d % 4.  In a word (16 elements)
+    # element e holds pair s = e % 8 (dims 2*(s%4) + e//8 above a multiple of 8 + 8q), so
+    # code = 2*(e % 2) + e // 8: elements 0-7 -> 0,2,0,2,... (bytes 0x88, 0x88),
+    # elements 8-15 -> 1,3,1,3,... (bytes 0xDD, 0xDD).
     k = bf16_bits(np.arange(D) % 4)
-    # V[d] = -1 + 0.5 * ((d // 4) % 4): min -1, max 0.5 -> zero -1.0 (0xBC00),
-    # scale 0.5 (0x3800); byte j holds four copies of code j % 4: 0x00,0x55,0xAA,0xFF.
+    # V[d] = -1 + 0.5 * ((d // 4) % 4): zero -1.0 (0xBC00), scale 0.5 (0x3800),
+    # code = (d // 4) % 4.  V pair p of quarter q is dims 8p + 2q + {0,1}, so its code is
+    # (2p + q // 2) % 4 = (2s + q // 2) % 4: quarters 0, 1 -> 0,2,0,2 (0x88);
+    # quarters 2, 3 -> 1,3,1,3 (0xDD).
     v = bf16_bits(-1 + 0.5 * ((np.arange(D) // 4) % 4))
     rec = orc.pack_record(2, k, v)
     assert rec.size == 96
-    assert np.all(rec[:32] == 0xE4)
-    assert list(rec[32:64]) == [0x00, 0x55, 0xAA, 0xFF] * 8
+    assert list(rec[:32]) == [0x88, 0x88, 0xDD, 0xDD] * 8
+    assert list(rec[32:64]) == [0x88] * 16 + [0xDD] * 16
     meta = rec[64:].view(np.uint16)
     assert list(meta) == [0x3C00] * 4 + [0x0000] * 4 + [0x3800] * 4 + [0xBC00] * 4
 
 
 def test_pack_hand_built_q4_q8():
-    # 4 bits: K[d] = d % 16 -> zero 0, scale 1, byte j = (2j % 16) | ((2j+1) % 16) << 4
+    # 4 bits, K[d] = V[d] = d % 16: zero 0, scale 1.  A word holds 8 nibbles = 4 pairs.
+    # K: element e is dim 8q + 2*(e%4) + e//4 (mod 16): q even -> 0,2,4,6,1,3,5,7
+    #    (bytes 20 64 31 75), q odd -> +8 (bytes A8 EC B9 FD); 4 equal words per quarter.
+    # V: element e is dim 8*blk + 2q + e//4 with blk % 2 = e % 2: 8*(e%2) + 2q + e//4,
+    #    q = 0..3 -> bytes (80 80 91 91), (A2 A2 B3 B3), (C4 C4 D5 D5), (E6 E6 F7 F7).
     k = bf16_bits(np.arange(D) % 16)
     rec = orc.pack_record(4, k, k)
-    exp = [(2 * j % 16) | (((2 * j + 1) % 16) << 4) for j in range(64)]
-    assert list(rec[:64]) == exp and list(rec[64:128]) == exp
+    kq = {0: [0x20, 0x64, 0x31, 0x75], 1: [0xA8, 0xEC, 0xB9, 0xFD]}
+    assert list(rec[:64]) == sum((kq[q % 2] * 4 for q in range(4)), [])
+    vq = [[0x80, 0x80, 0x91, 0x91], [0xA2, 0xA2, 0xB3, 0xB3], [0xC4, 0xC4, 0xD5, 0xD5],
+          [0xE6, 0xE6, 0xF7, 0xF7]]
+    assert list(rec[64:128]) == sum((vq[q] * 4 for q in range(4)), [])
     assert list(rec[128:].view(np.uint16)[:8]) == [0x3C00] * 4 + [0] * 4
-    # 8 bits: group values 0, 8, ..., 240, 255 -> zero 0, scale 1, codes = values
+    # 8 bits: K[d] = 8 * (d % 32), except 255 where d % 32 == 31: zero 0, scale 1,
+    # codes = values.  Element e of word w in quarter q is dim 8q + 4*(w%2) + [0,2,1,3][e]
+    # (mod 32), so a word holds 8*[m, m+2, m+1, m+3] with m = 8q + 4*(w%2).
     g = np.array([8 * i for i in range(31)] + [255], dtype=np.float32)
     k = bf16_bits(np.tile(g, 4))
     rec = orc.pack_record(8, k, k)
-    assert list(rec[:128]) == list(np.tile(g, 4).astype(np.uint8))
+    exp = []
+    for q in range(4):
+        for w in range(8):
+            m = 8 * q + 4 * (w % 2)
+            exp += [min(255, 8 * x) if x != 31 else 255 for x in (m, m + 2, m + 1, m + 3)]
+    assert list(rec[:128]) == exp
     assert rec.size == 288
 
 
-def test_pack_bf16_is_raw_bits():
-    rng = np.random.default_rng(3)
-    k = bf16_bits(rng.standard_normal(D))
-    v = bf16_bits(rng.standard_normal(D))
-    rec = orc.pack_record(16, k, v)
-    assert np.array_equal(rec.view(np.uint16), np.concatenate([k, v]))
+def test_pack_bf16_storage_order():
+    """bf16 records store raw bits in the same order (b = 16: one pair per word)."""
+    d = np.arange(D)
+    rec = orc.pack_record(16, bf16_bits(d), bf16_bits(d - 64))
+    u = bf16_value(rec.view(np.uint16)).astype(int)
+    # K quarter q: for each group g the dims 32g + 8q .. 32g + 8q + 7 in order
+    k_exp = [32 * g + 8 * q + j for q in range(4) for g in range(4) for j in range(8)]
+    # V quarter q: for each 8-dim block the dims 8blk + 2q, 8blk + 2q + 1
+    v_exp = [8 * b + 2 * q + j - 64 for q in range(4) for b in range(16) for j in range(2)]
+    assert list(u[:D]) == k_exp and list(u[D:]) == v_exp
 
 
 @pytest.mark.parametrize("bits", [2, 4, 8, 16])
@@ -218,24 +243,51 @@ def test_unpack_of_pack_matches_numpy_dequant(bits):
     kh, vh = orc.unpack_record(bits, rec)
     ref_k, ref_v = _np_dequant(rec, bits)
     assert np.array_equal(kh, ref_k) and np.array_equal(vh, ref_v)
+    if bits == 16:
+        assert np.array_equal(kh, bf16_value(k)) and np.array_equal(vh, bf16_value(v))
+
+
+def _np_dims(is_v, bits):
+    """Head-dim index of every storage element of a code block (from the layout rule)."""
+    dims = []
+    ppw = 16 // bits
+    for q in range(4):
+        for w in range(bits):                       # 32 elements of b bits = b words
+            for e in range(32 // bits):
+                p, hi = w * ppw + e % ppw, e // ppw
+                dims.append(8 * p + 2 * q + hi if is_v else 32 * (p // 4) + 8 * q + 2 * (p % 4) + hi)
+    return np.array(dims)
 
 
 def _np_dequant(rec, bits):
     if bits == 16:
         u = rec.view(np.uint16)
-        return bf16_value(u[:D]).astype(np.float64), bf16_value(u[D:]).astype(np.float64)
+        out = []
+        for w in range(2):
+            x = np.zeros(D)
+            x[_np_dims(w, 16)] = bf16_value(u[w * D:(w + 1) * D])
+            out.append(x)
+        return out[0], out[1]
     cb = D * bits // 8
     per = 8 // bits
     meta = rec[2 * cb:].view(np.uint16).view(np.float16).astype(np.float64)
     out = []
     for w in range(2):
         by = rec[w * cb:(w + 1) * cb]
-        codes = np.array([(by[i // per] >> (bits * (i % per))) & ((1 << bits) - 1)
-                          for i in range(D)], dtype=np.float64)
+        stored = np.array([(by[i // per] >> (bits * (i % per))) & ((1 << bits) - 1)
+                           for i in range(D)], dtype=np.float64)
+        codes = np.zeros(D)
+        codes[_np_dims(w, bits)] = stored
         sc = np.repeat(meta[w * 8:w * 8 + 4], GROUP)
         zr = np.repeat(meta[w * 8 + 4:w * 8 + 8], GROUP)
         out.append(codes * sc + zr)
     return out[0], out[1]
+
+
+def test_storage_order_is_a_permutation():
+    for bits in (2, 4, 8, 16):
+        for is_v in (0, 1):
+            assert sorted(_np_dims(is_v, bits)) == list(range(D))
 
 
 # --------------------------------------------------------------------------
