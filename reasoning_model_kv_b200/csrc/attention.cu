@@ -1,38 +1,41 @@
 // attention.cu -- tkv_decode_attention: one GQA decode step over the
-// mixed-precision pools with fused dequantisation, online softmax split over a
-// thread-block cluster, and accumulation of each token's attention mass into its
-// score (ThinKV decode over the Continuous Thinking block table; cumulative
-// attention scores as described on the "Back from the Future" page, problem
-// statement).
+// mixed-precision pools with fused dequantisation, online softmax, and
+// accumulation of each token's attention mass into its score (ThinKV decode over
+// the Continuous Thinking block table; cumulative attention scores as described
+// on the "Back from the Future" page, problem statement).
 //
-// Work decomposition.  Stream s = (b, kv head) is processed by one cluster of C
-// one-warp CTAs (grid (C, S), cluster (C, 1, 1)); CTA r takes a contiguous range
-// of the stream's entries (class 0, 1, 2, 3 tables concatenated).  C is chosen
-// on the host so that the whole grid is resident at once.
+// Work decomposition.  Stream s = (b, kv head) is processed by a cluster of C
+// CTAs of 3 warps (grid (C, S), cluster (C, 1, 1)); CTA r takes a contiguous
+// range of the stream's entries (class 0, 1, 2, 3 tables concatenated) and cuts
+// it into class-homogeneous tiles (16 records; 8 for bf16).  Warp w computes
+// tiles w, w+3, w+6, ... with its own online-softmax state.  C is picked on the
+// host so that the whole grid is resident (C = 1 for many streams).
 //
-// Memory path.  A CTA walks its range in class-homogeneous tiles (16 records;
-// 8 for bf16).  For each tile, the lanes of the warp issue one TMA bulk copy per
-// record (cp.async.bulk, L2 evict_first) into a 3-stage shared-memory ring, so
-// two tiles are in flight while one is computed; an mbarrier per stage tracks
-// the bytes.  Handles are prefetched one tile further ahead.
+// Memory path.  Each warp stages its tiles in a 3-deep shared-memory ring with
+// 16-byte cp.async copies (L2 evict_first), eight lanes per record so every
+// instruction reads whole 128-byte lines; two tiles are in flight while one is
+// computed.  Tile descriptors and the record handles are read three
+// tiles ahead into a small register ring, off the critical path.
 //
 // Math path (tensor cores, mma.sync m16n8k16, f16 x f16 -> f32):
-//   S[t][h] = K[t][:] . Q[h][:]   M = 16 tokens, N = 8 heads (G used), per 32-dim
-//            group, so the group's scale multiplies the fp32 accumulator and
-//            its zero adds zero * sum_g(q);
-//   O[d][h] += V^T[d][t] . (P * vscale)[t][h]   M = 16 dims, N = 8 heads, K = 16 tokens,
-//            plus sum_t p * vzero per group.
+//   S[t][h] = K[t][:] . Q[h][:]      M = 16 tokens, N = 8 heads (G used), one fp32
+//            accumulator per 32-dim group; the group's scale multiplies it and its
+//            zero adds zero * sum_group(q);
+//   O[d][h] += V^T[d][t] . (P * vscale)[t][h]   M = 16 dims, N = 8 heads, K = 16
+//            tokens, plus sum_t p * vzero per group (fp32, outside the MMA).
 // Integer codes are exact in f16 (magic-number conversion, 1-2 ALU ops per pair);
 // bf16 keys/values and queries convert exactly to f16 in its normal range.  The
 // record storage order puts each lane's operand pairs 16 bits apart in one word,
-// so fragments load with one or two 16-byte shared-memory reads per row; the V
-// operand and P are transposed with movmatrix.
+// so a row's quarter loads with one or two 16-byte shared-memory reads; the V
+// operand and P are transposed in registers with movmatrix.  The running max is
+// only moved (and O, l rescaled) when a tile exceeds it by more than 2^8.
 //
-// Epilogue.  Each CTA leaves (m, l, O) in shared memory; after a cluster barrier
-// every CTA reads its peers' (m, l) over DSMEM, rank r merges its slice of the
-// output, and every CTA adds p = exp2(x - M) / L, summed over the G heads, to
-// the scores of its own tokens.  Raw logits (log2 domain) go through a global
-// scratch that stays in L2 and is discarded (no write-back) after use.
+// Epilogue.  The CTA merges its warps in shared memory; with C > 1 every CTA
+// then reads its peers' (m, l) over DSMEM after a cluster barrier and rank r
+// merges its slice of the output.  Finally every CTA adds p = exp2(x - M) / L,
+// summed over the G heads, to the scores of its own tokens.  Raw logits (log2
+// domain) go through a global scratch that stays in L2 and is discarded (no
+// write-back) once read.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -43,47 +46,19 @@ namespace tkv {
 namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
+constexpr int kWarps = 3;
+constexpr int kThreads = 32 * kWarps;
 constexpr int kStages = 3;
-constexpr int kStageBytes = 16 * 304;   // the largest tile: 16 int8 records at a 304-byte stride
-constexpr long long kSpinLimit = 1ll << 24;  // bounded mbarrier waits (seconds, never reached)
-
-// Per class: bits per element, record bytes, shared-memory row stride (padded so
-// the fragment loads of 2-4 rows per phase hit distinct banks) and tile rows.
-__device__ __forceinline__ int class_rec(int c) { return c == 0 ? 512 : c == 1 ? 288 : c == 2 ? 160 : 96; }
-__device__ __forceinline__ int class_stride(int c) { return c == 0 ? 528 : c == 1 ? 304 : c == 2 ? 192 : 96; }
-__device__ __forceinline__ int class_rows(int c) { return c == 0 ? 8 : 16; }
+constexpr int kStageBytes = 16 * 288;   // the largest tile: 16 int8 records (rows unpadded, swizzled)
+constexpr int kRingBytes = kWarps * kStages * kStageBytes;
+constexpr int kMaxCluster = 8;
+constexpr float kRescaleSlack = 8.f;    // log2 units the running max may lag behind
+constexpr float kNoMax = -1e30f;        // reference max before any token: finite, so that
+                                        // exp2(-inf - kNoMax) = 0 and exp2(kNoMax - kNoMax) = 1
 
 // ----------------------------------------------------------------- PTX helpers
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_addr(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// Bounded wait: false if the phase did not complete within kSpinLimit polls.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
-    for (long long i = 0; i < kSpinLimit; ++i)
-        if (mbar_try_wait(bar, parity)) return true;
-    return false;
 }
 
 __device__ __forceinline__ uint64_t policy_evict_first() {
@@ -92,23 +67,17 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
     return p;
 }
 
-// One record: global -> this CTA's shared memory, completion counted on `bar`.
-__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar,
-                                          uint64_t policy) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
-        "[%0], [%1], %2, [%3], %4;" ::"r"(smem_addr(dst)),
-        "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
-        : "memory");
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint64_t policy) {
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+                 "l"(policy)
+                 : "memory");
 }
 
-__device__ __forceinline__ void fence_proxy_async() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 
-__device__ __forceinline__ void fence_mbarrier_init() {
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
+__device__ __forceinline__ void cp_async_wait_2() { asm volatile("cp.async.wait_group 2;" ::: "memory"); }
+
+__device__ __forceinline__ void cp_async_wait_0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
@@ -158,28 +127,40 @@ __device__ __forceinline__ uint32_t f32x2_to_f16x2(float lo, float hi) {
     return h2_as_u32(__floats2half2_rn(lo, hi));
 }
 
+__device__ __forceinline__ int sel4(int c, int a0, int a1, int a2, int a3) {
+    return c == 0 ? a0 : c == 1 ? a1 : c == 2 ? a2 : a3;
+}
+
 // ------------------------------------------------- code pair -> f16x2 operand
 // A 32-bit word of a BITS-bit code block holds 16/BITS dim pairs; pair s has its
 // members at bits BITS*s and BITS*s + 16.  OR-ing the masked word into 0x6400
 // (f16 1024) gives 1024 + m*code in each half (m = 2^(BITS*s') after an optional
 // 8-bit shift); one f16x2 FMA, exact, turns that into the code.
+// 0x64006400 held in a register (opaque to constant folding), so that
+// (w & mask) | magic compiles to a single three-input LOP3.
+__device__ __forceinline__ uint32_t magic_f16() {
+    uint32_t m;
+    asm volatile("mov.b32 %0, 0x64006400;" : "=r"(m));
+    return m;
+}
+
 template <int BITS, int S>
-__device__ __forceinline__ uint32_t code_pair(uint32_t word) {
+__device__ __forceinline__ uint32_t code_pair(uint32_t word, uint32_t magic) {
     if constexpr (BITS == 16) {
         return f32x2_to_f16x2(__uint_as_float(word << 16), __uint_as_float(word & 0xffff0000u));
     } else if constexpr (BITS == 8) {
         const uint32_t x = __byte_perm(word, 0x64646464u, S == 0 ? 0x4240 : 0x4341);
         return h2_as_u32(__hsub2(u32_as_h2(x), u32_as_h2(0x64006400u)));
     } else {
-        constexpr int kPerShift = BITS == 4 ? 2 : 4;        // pairs reachable without a shift
+        constexpr int kPerShift = BITS == 4 ? 2 : 4;   // pairs reachable without a shift
         constexpr int ss = S % kPerShift;
         const uint32_t w = (S >= kPerShift) ? (word >> 8) : word;
         constexpr uint32_t mask = ((1u << BITS) - 1u) * 0x00010001u;
-        const uint32_t x = (w & (mask << (BITS * ss))) | 0x64006400u;
+        const uint32_t x = (w & (mask << (BITS * ss))) | magic;
         if constexpr (ss == 0) {
             return h2_as_u32(__hsub2(u32_as_h2(x), u32_as_h2(0x64006400u)));
         } else {
-            // x = 1024 + 2^(BITS*ss) * code: multiply by 2^-(BITS*ss), subtract 1024 * 2^-(BITS*ss)
+            // x = 1024 + 2^e * code: multiply by 2^-e, add -1024 * 2^-e (exact in f16)
             constexpr int e = BITS * ss;   // 2, 4 or 6
             constexpr uint32_t mul = e == 2 ? 0x34003400u : e == 4 ? 0x2C002C00u : 0x24002400u;
             constexpr uint32_t add = e == 2 ? 0xDC00DC00u : e == 4 ? 0xD400D400u : 0xCC00CC00u;
@@ -190,13 +171,24 @@ __device__ __forceinline__ uint32_t code_pair(uint32_t word) {
 
 // Pair P (0..15) of a quarter held as BITS words.
 template <int BITS, int P>
-__device__ __forceinline__ uint32_t quarter_pair(const uint32_t (&w)[BITS]) {
+__device__ __forceinline__ uint32_t quarter_pair(const uint32_t (&w)[BITS], uint32_t magic) {
     constexpr int ppw = 16 / BITS;
-    return code_pair<BITS, P % ppw>(w[P / ppw]);
+    return code_pair<BITS, P % ppw>(w[P / ppw], magic);
 }
 
+// One row's quarter (4*BITS bytes at byte offset `off` of the record).  Int8 tiles keep
+// rows unpadded (288 bytes) and store odd rows with 16-byte chunks k and k ^ 1
+// swapped, which spreads the two rows a load phase touches over all 32 banks.
 template <int BITS>
-__device__ __forceinline__ void load_quarter(const uint8_t *src, uint32_t (&w)[BITS]) {
+__device__ __forceinline__ void load_quarter(const uint8_t *row, int off, int odd, uint32_t (&w)[BITS]) {
+    if constexpr (BITS == 8) {
+        const uint4 a = *reinterpret_cast<const uint4 *>(row + off + 16 * odd);
+        const uint4 b = *reinterpret_cast<const uint4 *>(row + off + 16 - 16 * odd);
+        w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+        w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+        return;
+    }
+    const uint8_t *src = row + off;
     if constexpr (BITS == 2) {
         const uint2 v = *reinterpret_cast<const uint2 *>(src);
         w[0] = v.x; w[1] = v.y;
@@ -216,77 +208,86 @@ __device__ __forceinline__ void load_quarter(const uint8_t *src, uint32_t (&w)[B
 template <int BITS, int GRP>
 __device__ __forceinline__ void qk_group(float (&x)[4], const uint32_t (&k0)[BITS],
                                          const uint32_t (&k1)[BITS], const uint32_t (&qb)[4][2][2],
-                                         const float (&qs)[2][4], const float (&ks)[2][4],
-                                         const float (&kz)[2][4]) {
+                                         const float (&qs)[2][4], const float2 (&km0)[4],
+                                         const float2 (&km1)[4], uint32_t magic) {
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    mma16816(acc, quarter_pair<BITS, 4 * GRP>(k0), quarter_pair<BITS, 4 * GRP>(k1),
-             quarter_pair<BITS, 4 * GRP + 1>(k0), quarter_pair<BITS, 4 * GRP + 1>(k1),
+    mma16816(acc, quarter_pair<BITS, 4 * GRP>(k0, magic), quarter_pair<BITS, 4 * GRP>(k1, magic),
+             quarter_pair<BITS, 4 * GRP + 1>(k0, magic), quarter_pair<BITS, 4 * GRP + 1>(k1, magic),
              qb[GRP][0][0], qb[GRP][0][1]);
-    mma16816(acc, quarter_pair<BITS, 4 * GRP + 2>(k0), quarter_pair<BITS, 4 * GRP + 2>(k1),
-             quarter_pair<BITS, 4 * GRP + 3>(k0), quarter_pair<BITS, 4 * GRP + 3>(k1),
+    mma16816(acc, quarter_pair<BITS, 4 * GRP + 2>(k0, magic), quarter_pair<BITS, 4 * GRP + 2>(k1, magic),
+             quarter_pair<BITS, 4 * GRP + 3>(k0, magic), quarter_pair<BITS, 4 * GRP + 3>(k1, magic),
              qb[GRP][1][0], qb[GRP][1][1]);
     if constexpr (BITS == 16) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) x[i] += acc[i];
     } else {
-        x[0] = fmaf(ks[0][GRP], acc[0], fmaf(kz[0][GRP], qs[0][GRP], x[0]));
-        x[1] = fmaf(ks[0][GRP], acc[1], fmaf(kz[0][GRP], qs[1][GRP], x[1]));
-        x[2] = fmaf(ks[1][GRP], acc[2], fmaf(kz[1][GRP], qs[0][GRP], x[2]));
-        x[3] = fmaf(ks[1][GRP], acc[3], fmaf(kz[1][GRP], qs[1][GRP], x[3]));
+        // km = (scale, zero) of the group for row g (0) and row g + 8 (1)
+        x[0] = fmaf(km0[GRP].x, acc[0], fmaf(km0[GRP].y, qs[0][GRP], x[0]));
+        x[1] = fmaf(km0[GRP].x, acc[1], fmaf(km0[GRP].y, qs[1][GRP], x[1]));
+        x[2] = fmaf(km1[GRP].x, acc[2], fmaf(km1[GRP].y, qs[0][GRP], x[2]));
+        x[3] = fmaf(km1[GRP].x, acc[3], fmaf(km1[GRP].y, qs[1][GRP], x[3]));
     }
 }
 
-struct Softmax {
-    float m[2], l[2];       // running max / sum for heads 2*tig, 2*tig+1 (partial over this lane's rows)
-    float o[8][4];          // O^T fragments: dims 16*mt + g (+8), heads 2*tig, 2*tig+1
-    float z[2][4];          // sum_t p * vzero per (head, group)
+// (scale, zero) pairs of the 4 groups from half of a record's meta block.
+__device__ __forceinline__ void load_meta(const uint8_t *meta, float2 (&out)[4]) {
+    const uint4 m = *reinterpret_cast<const uint4 *>(meta);   // scale x4 then zero x4 (fp16)
+    const float2 s01 = __half22float2(u32_as_h2(m.x)), s23 = __half22float2(u32_as_h2(m.y));
+    const float2 z01 = __half22float2(u32_as_h2(m.z)), z23 = __half22float2(u32_as_h2(m.w));
+    out[0] = make_float2(s01.x, z01.x);
+    out[1] = make_float2(s01.y, z01.y);
+    out[2] = make_float2(s23.x, z23.x);
+    out[3] = make_float2(s23.y, z23.y);
+}
+
+struct WarpState {
+    float m[2], l[2];   // reference max / (lane-partial) sum for heads 2*tig, 2*tig+1
+    float o[8][4];      // O^T fragments: dims 16*mt + g (+8), heads 2*tig, 2*tig+1
+    float z[2][4];      // lane-partial sum_t p * vzero per (head, group)
 };
 
-// One tile: up to 16 (ROWS) records of one class, resident in shared memory.
-template <int BITS, int ROWS, int G>
-__device__ __forceinline__ void tile_compute(const uint8_t *st, int stride, int nr, int lane,
+// One tile: up to ROWS records of one class, resident in shared memory (row stride
+// STRIDE).  Lane (g, tig) owns rows g and g + 8.  Rows at or beyond nr read the
+// last valid row instead (finite data, no divergent loads); their logits are
+// masked to -inf, so they contribute p = 0 everywhere.
+template <int BITS, int ROWS, int STRIDE, int G>
+__device__ __forceinline__ void tile_compute(const uint8_t *st, int nr, int lane,
                                              const uint32_t (&qb)[4][2][2], const float (&qs)[2][4],
-                                             float xscale, Softmax &sm, float *lg) {
+                                             float xscale, WarpState &ws, float *lg, uint32_t magic) {
     const int g = lane >> 2, tig = lane & 3;
     constexpr int QB = 4 * BITS;     // bytes of one quarter of a code block
     constexpr int CB = 16 * BITS;    // bytes of a code block
     const bool v0 = g < nr;
     const bool v1 = ROWS == 16 && g + 8 < nr;
-    uint32_t k0[BITS], k1[BITS], w0[BITS], w1[BITS];
-#pragma unroll
-    for (int i = 0; i < BITS; ++i) k0[i] = k1[i] = w0[i] = w1[i] = 0u;
-    float ks[2][4], kz[2][4], vs[2][4], vz[2][4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) ks[0][i] = ks[1][i] = kz[0][i] = kz[1][i] = vs[0][i] = vs[1][i] = vz[0][i] = vz[1][i] = 0.f;
-    auto load_row = [&](const uint8_t *row, uint32_t (&kw)[BITS], uint32_t (&vw)[BITS], int ri) {
-        load_quarter<BITS>(row + QB * tig, kw);
-        load_quarter<BITS>(row + CB + QB * tig, vw);
-        if constexpr (BITS < 16) {
-            const uint4 ma = *reinterpret_cast<const uint4 *>(row + 2 * CB);
-            const uint4 mb = *reinterpret_cast<const uint4 *>(row + 2 * CB + 16);
-            const uint32_t mw[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const float2 a = __half22float2(u32_as_h2(mw[j]));       // K scales
-                const float2 bz = __half22float2(u32_as_h2(mw[2 + j]));  // K zeros
-                const float2 c = __half22float2(u32_as_h2(mw[4 + j]));   // V scales
-                const float2 e = __half22float2(u32_as_h2(mw[6 + j]));   // V zeros
-                ks[ri][2 * j] = a.x; ks[ri][2 * j + 1] = a.y;
-                kz[ri][2 * j] = bz.x; kz[ri][2 * j + 1] = bz.y;
-                vs[ri][2 * j] = c.x; vs[ri][2 * j + 1] = c.y;
-                vz[ri][2 * j] = e.x; vz[ri][2 * j + 1] = e.y;
-            }
-        }
-    };
-    if (v0) load_row(st + g * stride, k0, w0, 0);
-    if (v1) load_row(st + (g + 8) * stride, k1, w1, 1);
+    const int i0 = min(g, nr - 1), i1 = min(g + 8, nr - 1);
+    const uint8_t *r0 = st + i0 * STRIDE;
+    const uint8_t *r1 = st + i1 * STRIDE;
+    const int odd0 = BITS == 8 ? (i0 & 1) : 0, odd1 = BITS == 8 ? (i1 & 1) : 0;
+    // meta chunk positions (int8 rows: chunks 16 and 17 swap on odd rows)
+    const int km_off0 = 2 * CB + 16 * odd0, vm_off0 = 2 * CB + 16 - 16 * odd0;
+    const int km_off1 = 2 * CB + 16 * odd1, vm_off1 = 2 * CB + 16 - 16 * odd1;
 
-    // ---- S = K . Q^T, one fp32 accumulator per 32-dim group
+    // ---- phase 1: S = K . Q^T
     float x[4] = {0.f, 0.f, 0.f, 0.f};   // (row g, head 2tig), (g, 2tig+1), (g+8, 2tig), (g+8, 2tig+1)
-    qk_group<BITS, 0>(x, k0, k1, qb, qs, ks, kz);
-    qk_group<BITS, 1>(x, k0, k1, qb, qs, ks, kz);
-    qk_group<BITS, 2>(x, k0, k1, qb, qs, ks, kz);
-    qk_group<BITS, 3>(x, k0, k1, qb, qs, ks, kz);
+    {
+        uint32_t k0[BITS], k1[BITS];
+        float2 km0[4], km1[4];
+        load_quarter<BITS>(r0, QB * tig, odd0, k0);
+        if constexpr (ROWS == 16) {
+            load_quarter<BITS>(r1, QB * tig, odd1, k1);
+        } else {
+#pragma unroll
+            for (int i = 0; i < BITS; ++i) k1[i] = 0u;
+        }
+        if constexpr (BITS < 16) {
+            load_meta(r0 + km_off0, km0);
+            load_meta(r1 + km_off1, km1);
+        }
+        qk_group<BITS, 0>(x, k0, k1, qb, qs, km0, km1, magic);
+        qk_group<BITS, 1>(x, k0, k1, qb, qs, km0, km1, magic);
+        qk_group<BITS, 2>(x, k0, k1, qb, qs, km0, km1, magic);
+        qk_group<BITS, 3>(x, k0, k1, qb, qs, km0, km1, magic);
+    }
     const bool h0 = 2 * tig < G, h1 = 2 * tig + 1 < G;
     x[0] = (v0 && h0) ? x[0] * xscale : -INFINITY;
     x[1] = (v0 && h1) ? x[1] * xscale : -INFINITY;
@@ -294,44 +295,45 @@ __device__ __forceinline__ void tile_compute(const uint8_t *st, int stride, int 
     x[3] = (v1 && h1) ? x[3] * xscale : -INFINITY;
     // raw logits (log2 domain) for the score pass
     if constexpr (G >= 2) {
-        if (h0) {
-            if (v0) *reinterpret_cast<float2 *>(lg + g * G + 2 * tig) = make_float2(x[0], x[1]);
-            if (v1) *reinterpret_cast<float2 *>(lg + (g + 8) * G + 2 * tig) = make_float2(x[2], x[3]);
-        }
+        if (h0 && v0) *reinterpret_cast<float2 *>(lg + g * G + 2 * tig) = make_float2(x[0], x[1]);
+        if (h0 && v1) *reinterpret_cast<float2 *>(lg + (g + 8) * G + 2 * tig) = make_float2(x[2], x[3]);
     } else {
-        if (tig == 0) {
-            if (v0) lg[g] = x[0];
-            if (v1) lg[g + 8] = x[2];
-        }
+        if (tig == 0 && v0) lg[g] = x[0];
+        if (tig == 0 && v1) lg[g + 8] = x[2];
     }
 
-    // ---- online softmax (heads are columns: reduce over the 8 row lanes)
+    // ---- online softmax; heads are columns, so reduce over the 8 row lanes
     float t0 = fmaxf(x[0], x[2]), t1 = fmaxf(x[1], x[3]);
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) {
         t0 = fmaxf(t0, __shfl_xor_sync(kFull, t0, o));
         t1 = fmaxf(t1, __shfl_xor_sync(kFull, t1, o));
     }
-    const float mn0 = fmaxf(sm.m[0], t0), mn1 = fmaxf(sm.m[1], t1);
-    const float a0 = mn0 == -INFINITY ? 1.f : ex2(sm.m[0] - mn0);
-    const float a1 = mn1 == -INFINITY ? 1.f : ex2(sm.m[1] - mn1);
-    float p[4];
-    p[0] = mn0 == -INFINITY ? 0.f : ex2(x[0] - mn0);
-    p[2] = mn0 == -INFINITY ? 0.f : ex2(x[2] - mn0);
-    p[1] = mn1 == -INFINITY ? 0.f : ex2(x[1] - mn1);
-    p[3] = mn1 == -INFINITY ? 0.f : ex2(x[3] - mn1);
-    sm.l[0] = sm.l[0] * a0 + p[0] + p[2];
-    sm.l[1] = sm.l[1] * a1 + p[1] + p[3];
-    sm.m[0] = mn0;
-    sm.m[1] = mn1;
+    // move the reference max only when a tile exceeds it by more than the slack;
+    // the reference starts at a finite sentinel, so p needs no -inf guard
+    if (__any_sync(kFull, t0 > ws.m[0] + kRescaleSlack || t1 > ws.m[1] + kRescaleSlack)) {
+        const float mn0 = fmaxf(ws.m[0], t0), mn1 = fmaxf(ws.m[1], t1);
+        const float a0 = ex2(ws.m[0] - mn0), a1 = ex2(ws.m[1] - mn1);
+        ws.m[0] = mn0;
+        ws.m[1] = mn1;
+        ws.l[0] *= a0;
+        ws.l[1] *= a1;
 #pragma unroll
-    for (int mt = 0; mt < 8; ++mt) {
-        sm.o[mt][0] *= a0; sm.o[mt][1] *= a1; sm.o[mt][2] *= a0; sm.o[mt][3] *= a1;
+        for (int mt = 0; mt < 8; ++mt) {
+            ws.o[mt][0] *= a0; ws.o[mt][1] *= a1; ws.o[mt][2] *= a0; ws.o[mt][3] *= a1;
+        }
+#pragma unroll
+        for (int grp = 0; grp < 4; ++grp) { ws.z[0][grp] *= a0; ws.z[1][grp] *= a1; }
     }
-#pragma unroll
-    for (int grp = 0; grp < 4; ++grp) { sm.z[0][grp] *= a0; sm.z[1][grp] *= a1; }
+    float p[4];
+    p[0] = ex2(x[0] - ws.m[0]);
+    p[2] = ex2(x[2] - ws.m[0]);
+    p[1] = ex2(x[1] - ws.m[1]);
+    p[3] = ex2(x[3] - ws.m[1]);
+    ws.l[0] += p[0] + p[2];
+    ws.l[1] += p[1] + p[3];
 
-    // ---- O += V^T . (P * vscale) per group; zero term accumulated separately
+    // ---- phase 2: O += V^T . (P * vscale) per group; zero term accumulated apart
     uint32_t bfr[4][2];
     if constexpr (BITS == 16) {
         const uint32_t b0 = transpose8x8(f32x2_to_f16x2(p[0], p[1]));
@@ -339,74 +341,103 @@ __device__ __forceinline__ void tile_compute(const uint8_t *st, int stride, int 
 #pragma unroll
         for (int grp = 0; grp < 4; ++grp) { bfr[grp][0] = b0; bfr[grp][1] = b1; }
     } else {
+        float2 vm0[4], vm1[4];
+        load_meta(r0 + vm_off0, vm0);
+        load_meta(r1 + vm_off1, vm1);
 #pragma unroll
         for (int grp = 0; grp < 4; ++grp) {
-            sm.z[0][grp] += p[0] * vz[0][grp] + p[2] * vz[1][grp];
-            sm.z[1][grp] += p[1] * vz[0][grp] + p[3] * vz[1][grp];
-            bfr[grp][0] = transpose8x8(f32x2_to_f16x2(p[0] * vs[0][grp], p[1] * vs[0][grp]));
-            bfr[grp][1] = transpose8x8(f32x2_to_f16x2(p[2] * vs[1][grp], p[3] * vs[1][grp]));
+            ws.z[0][grp] = fmaf(p[2], vm1[grp].y, fmaf(p[0], vm0[grp].y, ws.z[0][grp]));
+            ws.z[1][grp] = fmaf(p[3], vm1[grp].y, fmaf(p[1], vm0[grp].y, ws.z[1][grp]));
+            bfr[grp][0] = transpose8x8(f32x2_to_f16x2(p[0] * vm0[grp].x, p[1] * vm0[grp].x));
+            bfr[grp][1] = transpose8x8(f32x2_to_f16x2(p[2] * vm1[grp].x, p[3] * vm1[grp].x));
         }
     }
-#define TKV_VMMA(MT)                                                                          \
-    {                                                                                         \
-        const uint32_t e0 = transpose8x8(quarter_pair<BITS, 2 * (MT)>(w0));                   \
-        const uint32_t e1 = transpose8x8(quarter_pair<BITS, 2 * (MT) + 1>(w0));               \
-        const uint32_t e2 = ROWS == 16 ? transpose8x8(quarter_pair<BITS, 2 * (MT)>(w1)) : 0u; \
-        const uint32_t e3 = ROWS == 16 ? transpose8x8(quarter_pair<BITS, 2 * (MT) + 1>(w1)) : 0u; \
-        mma16816(sm.o[MT], e0, e1, e2, e3, bfr[(MT) >> 1][0], bfr[(MT) >> 1][1]);             \
+    uint32_t w0[BITS], w1[BITS];
+    load_quarter<BITS>(r0, CB + QB * tig, odd0, w0);
+    if constexpr (ROWS == 16) {
+        load_quarter<BITS>(r1, CB + QB * tig, odd1, w1);
+    } else {
+#pragma unroll
+        for (int i = 0; i < BITS; ++i) w1[i] = 0u;
+    }
+#define TKV_VMMA(MT)                                                                              \
+    {                                                                                             \
+        const uint32_t e0 = transpose8x8(quarter_pair<BITS, 2 * (MT)>(w0, magic));                       \
+        const uint32_t e1 = transpose8x8(quarter_pair<BITS, 2 * (MT) + 1>(w0, magic));                   \
+        const uint32_t e2 = ROWS == 16 ? transpose8x8(quarter_pair<BITS, 2 * (MT)>(w1, magic)) : 0u;     \
+        const uint32_t e3 = ROWS == 16 ? transpose8x8(quarter_pair<BITS, 2 * (MT) + 1>(w1, magic)) : 0u; \
+        mma16816(ws.o[MT], e0, e1, e2, e3, bfr[(MT) >> 1][0], bfr[(MT) >> 1][1]);                 \
     }
     TKV_VMMA(0) TKV_VMMA(1) TKV_VMMA(2) TKV_VMMA(3) TKV_VMMA(4) TKV_VMMA(5) TKV_VMMA(6) TKV_VMMA(7)
 #undef TKV_VMMA
 }
 
-// Tile cursor over the CTA's entry range, class by class.
-struct Cursor {
-    int c, e;
-    __device__ __forceinline__ void skip_empty(const int (&lo)[4], const int (&hi)[4]) {
-        while (c < 4 && e >= hi[c]) { ++c; if (c < 4) e = lo[c]; }
+// Copy a tile of class C_ into a stage with coalesced 16-byte cp.async: eight
+// consecutive lanes cover 128 contiguous bytes of one record, so one instruction
+// reads four whole 128-byte lines (records r = lane/8 + 4i).  `hd` holds, in lane
+// j < 16, the slot of the tile's record j.  Int8 rows are unpadded and odd rows
+// store 16-byte chunk k at k ^ 1.
+template <int C_>
+__device__ __forceinline__ void issue_tile(uint32_t stage, const uint8_t *pool, int hd, int nr,
+                                           int lane, uint64_t pol) {
+    constexpr int REC = C_ == 0 ? 512 : C_ == 1 ? 288 : C_ == 2 ? 160 : 96;
+    constexpr int STRIDE = C_ == 0 ? 528 : C_ == 1 ? 288 : C_ == 2 ? 192 : 96;
+    constexpr int ROWS = C_ == 0 ? 8 : 16;
+    constexpr int NCH = REC / 16;                  // 16-byte chunks per record
+    constexpr int NBLK = (NCH + 7) / 8;            // 8-chunk blocks per record
+    const int sub = lane & 7;
+#pragma unroll
+    for (int i = 0; i < ROWS / 4; ++i) {
+        const int r = (lane >> 3) + 4 * i;
+        const int slot = __shfl_sync(kFull, hd, r);
+        if (r < nr) {
+            const uint8_t *src = pool + (size_t)slot * REC + 16 * sub;
+            int dpos = 16 * sub;
+            if constexpr (C_ == 1) dpos += (r & 1) ? ((sub & 1) ? -16 : 16) : 0;   // k ^ 1 on odd rows
+            const uint32_t dst = stage + r * STRIDE + dpos;
+#pragma unroll
+            for (int j = 0; j < NBLK; ++j)
+                if (8 * j + sub < NCH) cp_async16(dst + 128 * j, src + 128 * j, pol);
+        }
     }
-    __device__ __forceinline__ void advance(const int (&lo)[4], const int (&hi)[4]) {
-        e += class_rows(c);
-        skip_empty(lo, hi);
-    }
-    __device__ __forceinline__ int rows(const int (&hi)[4]) const {
-        return min(class_rows(c), hi[c] - e);
-    }
-};
+}
 
 template <int G>
-__global__ void __launch_bounds__(32) attn_kernel(Dev d, const __nv_bfloat16 *__restrict__ q,
-                                                  float xscale, float *__restrict__ out, int C) {
-    __shared__ __align__(128) uint8_t ring[kStages * kStageBytes];
-    __shared__ __align__(8) uint64_t bars[kStages];
-    __shared__ float fac[16][kMaxG];     // exp2(m_j - M) per peer rank and head
+__global__ void __launch_bounds__(kThreads, 4) attn_kernel(const __grid_constant__ Dev d,
+                                                           const __nv_bfloat16 *__restrict__ q,
+                                                           float xscale, float *__restrict__ out,
+                                                           int C) {
+    extern __shared__ __align__(128) uint8_t ring[];   // kRingBytes, dynamic
+    __shared__ float cta_m[kMaxG], cta_l[kMaxG];
+    __shared__ float fac[kMaxCluster][kMaxG];     // exp2(m_j - M) per warp / peer rank and head
     __shared__ float gM[kMaxG], gInvL[kMaxG];
 
-    const int lane = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, tig = lane & 3;
     const int rank = blockIdx.x;
     const int s = blockIdx.y;
     const int b = s / d.Hkv, kvh = s - b * d.Hkv;
 
-    int n[4], off[5];
-    off[0] = 0;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) { n[c] = d.n[s * 4 + c]; off[c + 1] = off[c] + n[c]; }
-    const int N = off[4];
+    // ---- this CTA's entry range and its tiles (class by class)
+    const int n0 = d.n[s * 4 + 0], n1 = d.n[s * 4 + 1], n2 = d.n[s * 4 + 2], n3 = d.n[s * 4 + 3];
+    const int o1 = n0, o2 = o1 + n1, o3 = o2 + n2, N = o3 + n3;
     const int chunk = ((N + C - 1) / C + 31) & ~31;
     const int t0 = min(N, rank * chunk), t1 = min(N, t0 + chunk);
-    int lo[4], hi[4];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        lo[c] = min(max(t0 - off[c], 0), n[c]);
-        hi[c] = min(max(t1 - off[c], 0), n[c]);
-    }
+    const int lo0 = min(t0, o1), hi0 = min(t1, o1);
+    const int lo1 = min(max(t0 - o1, 0), n1), hi1 = min(max(t1 - o1, 0), n1);
+    const int lo2 = min(max(t0 - o2, 0), n2), hi2 = min(max(t1 - o2, 0), n2);
+    const int lo3 = min(max(t0 - o3, 0), n3), hi3 = min(max(t1 - o3, 0), n3);
+    const int p1 = (hi0 - lo0 + 7) / 8;                 // tile prefix counts
+    const int p2 = p1 + (hi1 - lo1 + 15) / 16;
+    const int p3 = p2 + (hi2 - lo2 + 15) / 16;
+    const int p4 = p3 + (hi3 - lo3 + 15) / 16;
     float *lgs = d.logits + (size_t)s * d.ncap * G;   // this stream's logits, by entry order
 
     // ---- query operand (B of S = K Q^T): head g, dims 32grp + 8tig + 4hh + 0..3
     uint32_t qb[4][2][2];
-    float qsg[4];
+    float qs[2][4];
     {
+        float qsg[4];
         const __nv_bfloat16 *qr = q + ((size_t)b * d.Hkv * G + (size_t)kvh * G + (g < G ? g : 0)) * kD;
 #pragma unroll
         for (int grp = 0; grp < 4; ++grp) {
@@ -425,177 +456,203 @@ __global__ void __launch_bounds__(32) attn_kernel(Dev d, const __nv_bfloat16 *__
             sum += __shfl_xor_sync(kFull, sum, 2);
             qsg[grp] = sum;                              // sum over group grp of q[head g]
         }
-    }
-    float qs[2][4];
-#pragma unroll
-    for (int grp = 0; grp < 4; ++grp) {
-        qs[0][grp] = __shfl_sync(kFull, qsg[grp], (2 * tig) * 4);
-        qs[1][grp] = __shfl_sync(kFull, qsg[grp], (2 * tig + 1) * 4);
-    }
-
-    Softmax sm;
-    sm.m[0] = sm.m[1] = -INFINITY;
-    sm.l[0] = sm.l[1] = 0.f;
-#pragma unroll
-    for (int mt = 0; mt < 8; ++mt) sm.o[mt][0] = sm.o[mt][1] = sm.o[mt][2] = sm.o[mt][3] = 0.f;
-#pragma unroll
-    for (int grp = 0; grp < 4; ++grp) sm.z[0][grp] = sm.z[1][grp] = 0.f;
-
-    if (lane == 0) {
-#pragma unroll
-        for (int i = 0; i < kStages; ++i) mbar_init(&bars[i], 1);
-        fence_mbarrier_init();
-    }
-    __syncwarp();
-    const uint64_t pol = policy_evict_first();
-
-    // cursors: consumer, producer (2 tiles ahead), handle prefetch (3 ahead)
-    Cursor cc{0, lo[0]}, cp{0, lo[0]}, ch{0, lo[0]};
-    cc.skip_empty(lo, hi);
-    cp.skip_empty(lo, hi);
-    ch.skip_empty(lo, hi);
-    auto handle_of = [&](const Cursor &cu) -> int {
-        if (cu.c >= 4 || lane >= cu.rows(hi)) return 0;
-        return d.handle[cu.c][(size_t)s * d.cap[cu.c] + cu.e + lane];
-    };
-    auto issue = [&](const Cursor &cu, int stage, int hd) {
-        const int c = cu.c, nr = cu.rows(hi), rb = class_rec(c);
-        fence_proxy_async();
-        if (lane == 0) mbar_arrive_expect_tx(&bars[stage], (uint32_t)(nr * rb));
-        __syncwarp();
-        if (lane < nr)
-            bulk_load(ring + stage * kStageBytes + lane * class_stride(c),
-                      d.pool[c] + ((size_t)s * d.cap[c] + hd) * rb, (uint32_t)rb, &bars[stage], pol);
-    };
-
-    int issued = 0;
-    int h_next = 0;
-    for (int k = 0; k < 2 && cp.c < 4; ++k) {
-        issue(cp, issued % kStages, handle_of(cp));
-        ++issued;
-        cp.advance(lo, hi);
-    }
-    ch = cp;
-    h_next = handle_of(ch);
-    if (ch.c < 4) ch.advance(lo, hi);
-
-    bool ok = true;
-    int consumed = 0;
-    while (cc.c < 4) {
-        if (cp.c < 4) {
-            issue(cp, issued % kStages, h_next);
-            ++issued;
-            cp.advance(lo, hi);
-            h_next = handle_of(ch);
-            if (ch.c < 4) ch.advance(lo, hi);
-        }
-        const int stage = consumed % kStages;
-        // every lane waits (acquire of the TMA writes); the outcome is made warp-uniform
-        const bool arrived = mbar_wait(&bars[stage], (uint32_t)((consumed / kStages) & 1));
-        if (!__all_sync(kFull, arrived)) {
-            ok = false;
-            break;
-        }
-        const uint8_t *st = ring + stage * kStageBytes;
-        const int nr = cc.rows(hi);
-        float *lg = lgs + (size_t)(off[cc.c] + cc.e) * G;
-        switch (cc.c) {
-            case 0: tile_compute<16, 8, G>(st, 528, nr, lane, qb, qs, xscale, sm, lg); break;
-            case 1: tile_compute<8, 16, G>(st, 304, nr, lane, qb, qs, xscale, sm, lg); break;
-            case 2: tile_compute<4, 16, G>(st, 192, nr, lane, qb, qs, xscale, sm, lg); break;
-            default: tile_compute<2, 16, G>(st, 96, nr, lane, qb, qs, xscale, sm, lg); break;
-        }
-        __syncwarp();
-        ++consumed;
-        cc.advance(lo, hi);
-    }
-    if (!ok) {
-        if (lane == 0) raise_error(d.err, kErrTimeout, (uint32_t)s);
-        // let every copy still in flight land before the ring is reused (bounded)
-        for (int i = consumed; i < issued; ++i) mbar_wait(&bars[i % kStages], (uint32_t)((i / kStages) & 1));
-    }
-
-    // ---- finish this CTA's partial: reduce over the 8 row lanes, fold the zero term
-#pragma unroll
-    for (int o = 4; o < 32; o <<= 1) {
-        sm.l[0] += __shfl_xor_sync(kFull, sm.l[0], o);
-        sm.l[1] += __shfl_xor_sync(kFull, sm.l[1], o);
 #pragma unroll
         for (int grp = 0; grp < 4; ++grp) {
-            sm.z[0][grp] += __shfl_xor_sync(kFull, sm.z[0][grp], o);
-            sm.z[1][grp] += __shfl_xor_sync(kFull, sm.z[1][grp], o);
+            qs[0][grp] = __shfl_sync(kFull, qsg[grp], (2 * tig) * 4);
+            qs[1][grp] = __shfl_sync(kFull, qsg[grp], (2 * tig + 1) * 4);
         }
     }
-    float *ep_m = reinterpret_cast<float *>(ring);    // [kMaxG]
-    float *ep_l = ep_m + kMaxG;                        // [kMaxG]
-    float *ep_o = ep_m + 2 * kMaxG;                    // [G][kD]
-    __syncwarp();
-    if (g == 0) {
-        if (2 * tig < G) { ep_m[2 * tig] = sm.m[0]; ep_l[2 * tig] = sm.l[0]; }
-        if (2 * tig + 1 < G) { ep_m[2 * tig + 1] = sm.m[1]; ep_l[2 * tig + 1] = sm.l[1]; }
-    }
-#pragma unroll
-    for (int mt = 0; mt < 8; ++mt) {
-        const int d0 = 16 * mt + g, grp = mt >> 1;
-        if (2 * tig < G) {
-            ep_o[(2 * tig) * kD + d0] = sm.o[mt][0] + sm.z[0][grp];
-            ep_o[(2 * tig) * kD + d0 + 8] = sm.o[mt][2] + sm.z[0][grp];
-        }
-        if (2 * tig + 1 < G) {
-            ep_o[(2 * tig + 1) * kD + d0] = sm.o[mt][1] + sm.z[1][grp];
-            ep_o[(2 * tig + 1) * kD + d0 + 8] = sm.o[mt][3] + sm.z[1][grp];
-        }
-    }
-    cluster_sync();
 
-    // ---- merge the cluster: global (M, L) per head, then this rank's output slice
-    if (lane < G) {
-        float M = -INFINITY;
-        for (int j = 0; j < C; ++j) M = fmaxf(M, dsmem_ld(dsmem_addr(ep_m + lane, (uint32_t)j)));
-        float L = 0.f;
-        for (int j = 0; j < C; ++j) {
-            const float mj = dsmem_ld(dsmem_addr(ep_m + lane, (uint32_t)j));
-            const float f = M == -INFINITY ? 0.f : ex2(mj - M);
-            fac[j][lane] = f;
-            L += f * dsmem_ld(dsmem_addr(ep_l + lane, (uint32_t)j));
+    WarpState ws;
+    ws.m[0] = ws.m[1] = kNoMax;
+    ws.l[0] = ws.l[1] = 0.f;
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) ws.o[mt][0] = ws.o[mt][1] = ws.o[mt][2] = ws.o[mt][3] = 0.f;
+#pragma unroll
+    for (int grp = 0; grp < 4; ++grp) ws.z[0][grp] = ws.z[1][grp] = 0.f;
+
+    const uint64_t pol = policy_evict_first();
+    const uint32_t ring0 = smem_addr(ring) + warp * kStages * kStageBytes;
+
+    // tile T -> packed descriptor: entry e (bits 0-23), rows nr (24-28), class c (29-30)
+    auto tile_of = [&](int T) -> int {
+        if (T >= p4) return -1;
+        const int c = (T >= p1) + (T >= p2) + (T >= p3);
+        const int rows = c == 0 ? 8 : 16;
+        const int e = sel4(c, lo0, lo1, lo2, lo3) + (T - sel4(c, 0, p1, p2, p3)) * rows;
+        const int nr = min(rows, sel4(c, hi0, hi1, hi2, hi3) - e);
+        return e | (nr << 24) | (c << 29);
+    };
+    // lane j holds the slot of record min(j, nr - 1) of a tile
+    auto handle_of = [&](int dsc) -> int {
+        if (dsc < 0) return 0;
+        const int e = dsc & 0xffffff, nr = (dsc >> 24) & 31, c = dsc >> 29;
+        return d.handle[c][(size_t)s * d.cap[c] + e + min(lane, nr - 1)];
+    };
+    auto issue = [&](int dsc, int stage, int hd) {
+        const int nr = (dsc >> 24) & 31, c = dsc >> 29;
+        const uint32_t st = ring0 + stage * kStageBytes;
+        const uint8_t *pool = d.pool[c] + (size_t)s * d.cap[c] * d.rec[c];
+        switch (c) {
+            case 0: issue_tile<0>(st, pool, hd, nr, lane, pol); break;
+            case 1: issue_tile<1>(st, pool, hd, nr, lane, pol); break;
+            case 2: issue_tile<2>(st, pool, hd, nr, lane, pol); break;
+            default: issue_tile<3>(st, pool, hd, nr, lane, pol); break;
         }
-        gM[lane] = M;
-        gInvL[lane] = L > 0.f ? 1.f / L : 0.f;
+    };
+    const uint32_t magic = magic_f16();
+
+    // Warp tiles t_k = warp + 4k.  Iteration k computes t_k (stage k % 3) after
+    // issuing t_{k+2}; descriptors and handles of t_{k+2..k+4} sit in a register ring
+    // and t_{k+5}'s are loaded each iteration, three iterations before use.
+    int dc0 = tile_of(warp), dc1 = tile_of(warp + kWarps);
+    if (dc0 >= 0) issue(dc0, 0, handle_of(dc0));
+    cp_async_commit();
+    if (dc1 >= 0) issue(dc1, 1, handle_of(dc1));
+    cp_async_commit();
+    int dr0 = tile_of(warp + 2 * kWarps), dr1 = tile_of(warp + 3 * kWarps), dr2 = tile_of(warp + 4 * kWarps);
+    int hr0 = handle_of(dr0), hr1 = handle_of(dr1), hr2 = handle_of(dr2);
+    int stage = 0;
+    for (int T = warp; dc0 >= 0; T += kWarps) {
+        if (dr0 >= 0) issue(dr0, stage == 0 ? 2 : stage - 1, hr0);
+        cp_async_commit();
+        const int dc2 = dr0;
+        dr0 = dr1; dr1 = dr2; hr0 = hr1; hr1 = hr2;
+        dr2 = tile_of(T + 5 * kWarps);
+        hr2 = handle_of(dr2);
+        cp_async_wait_2();
+        __syncwarp();
+        const int ec = dc0 & 0xffffff, nc = (dc0 >> 24) & 31, cc = dc0 >> 29;
+        const uint8_t *st = ring + (warp * kStages + stage) * kStageBytes;
+        float *lg = lgs + (size_t)(sel4(cc, 0, o1, o2, o3) + ec) * G;
+        switch (cc) {
+            case 0: tile_compute<16, 8, 528, G>(st, nc, lane, qb, qs, xscale, ws, lg, magic); break;
+            case 1: tile_compute<8, 16, 288, G>(st, nc, lane, qb, qs, xscale, ws, lg, magic); break;
+            case 2: tile_compute<4, 16, 192, G>(st, nc, lane, qb, qs, xscale, ws, lg, magic); break;
+            default: tile_compute<2, 16, 96, G>(st, nc, lane, qb, qs, xscale, ws, lg, magic); break;
+        }
+        __syncwarp();
+        dc0 = dc1; dc1 = dc2;
+        stage = stage == 2 ? 0 : stage + 1;
     }
-    __syncwarp();
+    cp_async_wait_0();
+
+    // ---- warp partials: reduce the lane partials over the 8 row lanes, fold z into O
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+        ws.l[0] += __shfl_xor_sync(kFull, ws.l[0], o);
+        ws.l[1] += __shfl_xor_sync(kFull, ws.l[1], o);
+#pragma unroll
+        for (int grp = 0; grp < 4; ++grp) {
+            ws.z[0][grp] += __shfl_xor_sync(kFull, ws.z[0][grp], o);
+            ws.z[1][grp] += __shfl_xor_sync(kFull, ws.z[1][grp], o);
+        }
+    }
+    __syncthreads();                                   // every warp is done with the ring
+    float *wm = reinterpret_cast<float *>(ring);       // [kWarps][kMaxG]
+    float *wl = wm + kWarps * kMaxG;                   // [kWarps][kMaxG]
+    float *wo = wl + kWarps * kMaxG;                   // [kWarps][G][kD]
+    float *co = wo + kWarps * G * kD;                  // [G][kD] the CTA's merged O
+    if (g == 0) {
+        if (2 * tig < G) { wm[warp * kMaxG + 2 * tig] = ws.m[0]; wl[warp * kMaxG + 2 * tig] = ws.l[0]; }
+        if (2 * tig + 1 < G) { wm[warp * kMaxG + 2 * tig + 1] = ws.m[1]; wl[warp * kMaxG + 2 * tig + 1] = ws.l[1]; }
+    }
     {
+        float *w = wo + warp * G * kD;
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+            const int d0 = 16 * mt + g, grp = mt >> 1;
+            if (2 * tig < G) {
+                w[(2 * tig) * kD + d0] = ws.o[mt][0] + ws.z[0][grp];
+                w[(2 * tig) * kD + d0 + 8] = ws.o[mt][2] + ws.z[0][grp];
+            }
+            if (2 * tig + 1 < G) {
+                w[(2 * tig + 1) * kD + d0] = ws.o[mt][1] + ws.z[1][grp];
+                w[(2 * tig + 1) * kD + d0 + 8] = ws.o[mt][3] + ws.z[1][grp];
+            }
+        }
+    }
+    __syncthreads();
+    // ---- CTA merge of the warps
+    if (tid < G) {
+        float M = kNoMax;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) M = fmaxf(M, wm[w * kMaxG + tid]);
+        float L = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+            const float f = ex2(wm[w * kMaxG + tid] - M);   // warps without tokens carry l = 0
+            fac[w][tid] = f;
+            L += f * wl[w * kMaxG + tid];
+        }
+        cta_m[tid] = M;
+        cta_l[tid] = L;
+    }
+    __syncthreads();
+    for (int idx = tid; idx < G * kD; idx += kThreads) {
+        const int h = idx / kD;
+        float acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) acc += fac[w][h] * wo[w * G * kD + idx];
+        co[idx] = acc;
+    }
+    __syncthreads();
+
+    // ---- cluster merge: global (M, L) per head; this rank writes its output slice
+    float *orow = out + ((size_t)b * d.Hkv * G + (size_t)kvh * G) * kD;
+    if (C == 1) {
+        if (tid < G) {
+            gM[tid] = cta_m[tid];
+            gInvL[tid] = cta_l[tid] > 0.f ? 1.f / cta_l[tid] : 0.f;
+        }
+        __syncthreads();
+        for (int idx = tid; idx < G * kD; idx += kThreads) orow[idx] = co[idx] * gInvL[idx / kD];
+    } else {
+        cluster_sync();
+        if (tid < G) {
+            float M = kNoMax;
+            for (int j = 0; j < C; ++j) M = fmaxf(M, dsmem_ld(dsmem_addr(cta_m + tid, (uint32_t)j)));
+            float L = 0.f;
+            for (int j = 0; j < C; ++j) {
+                const float mj = dsmem_ld(dsmem_addr(cta_m + tid, (uint32_t)j));
+                const float f = ex2(mj - M);
+                fac[j][tid] = f;
+                L += f * dsmem_ld(dsmem_addr(cta_l + tid, (uint32_t)j));
+            }
+            gM[tid] = M;
+            gInvL[tid] = L > 0.f ? 1.f / L : 0.f;
+        }
+        __syncthreads();
         const int E = G * kD;
         const int per = (E + C - 1) / C;
         const int e0 = rank * per, e1 = min(E, e0 + per);
-        float *orow = out + ((size_t)b * d.Hkv * G + (size_t)kvh * G) * kD;
-        for (int idx = e0 + lane; idx < e1; idx += 32) {
+        for (int idx = e0 + tid; idx < e1; idx += kThreads) {
             const int h = idx / kD;
             float acc = 0.f;
-            for (int j = 0; j < C; ++j) acc += fac[j][h] * dsmem_ld(dsmem_addr(ep_o + idx, (uint32_t)j));
+            for (int j = 0; j < C; ++j) acc += fac[j][h] * dsmem_ld(dsmem_addr(co + idx, (uint32_t)j));
             orow[idx] = acc * gInvL[h];
         }
     }
 
-    // ---- scores of this CTA's tokens: += sum_h exp2(x - M_h) / L_h
-    if (ok && gM[0] != -INFINITY) {
+    // ---- scores of this CTA's tokens: += sum_h exp2(x - M_h) / L_h (none if the stream is empty)
+    if (N > 0) {
         float Mh[kMaxG], Ih[kMaxG];
 #pragma unroll
         for (int h = 0; h < G; ++h) { Mh[h] = gM[h]; Ih[h] = gInvL[h]; }
-        for (int t = t0 + lane; t < t1; t += 32) {
+        for (int t = t0 + tid; t < t1; t += kThreads) {
             const float *xt = lgs + (size_t)t * G;
             float inc = 0.f;
 #pragma unroll
             for (int h = 0; h < G; ++h) inc += ex2(xt[h] - Mh[h]) * Ih[h];
-            int c = 0;
-            while (t >= off[c + 1]) ++c;
-            d.score[c][(size_t)s * d.cap[c] + (t - off[c])] += inc;
+            const int c = (t >= o1) + (t >= o2) + (t >= o3);
+            d.score[c][(size_t)s * d.cap[c] + (t - sel4(c, 0, o1, o2, o3))] += inc;
         }
-        __syncwarp();
+        __syncthreads();
         const char *base = reinterpret_cast<const char *>(lgs + (size_t)t0 * G);
         const int nlines = (int)(((size_t)(t1 - t0) * G * sizeof(float) + 127) / 128);
-        for (int i = lane; i < nlines; i += 32) discard_l2_line(base + (size_t)i * 128);
+        for (int i = tid; i < nlines; i += kThreads) discard_l2_line(base + (size_t)i * 128);
     }
-    cluster_sync();   // peers may still be reading this CTA's shared memory
+    if (C > 1) cluster_sync();   // peers may still be reading this CTA's shared memory
 }
 
 int g_blocks_per_sm[kMaxG + 1] = {0};
@@ -610,20 +667,25 @@ cudaError_t launch_g(const Dev &d, const void *q, float scale, float *out, long 
         cudaDeviceGetAttribute(&g_sms, cudaDevAttrMultiProcessorCount, dev);
     }
     if (g_blocks_per_sm[G] == 0) {
+        cudaError_t e = cudaFuncSetAttribute(attn_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kRingBytes);
+        if (e != cudaSuccess) return e;
         int nb = 0;
-        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, attn_kernel<G>, 32, 0);
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, attn_kernel<G>, kThreads, kRingBytes);
         if (e != cudaSuccess) return e;
         g_blocks_per_sm[G] = nb > 0 ? nb : 1;
     }
+    // Largest cluster (<= 8) whose grid is fully resident, never splitting a stream
+    // below ~128 tokens per CTA; one CTA per stream when the streams fill the GPU.
     const long long slots = (long long)g_blocks_per_sm[G] * g_sms;
     long long C = slots / d.S;
-    C = C < 1 ? 1 : (C > 8 ? 8 : C);
-    const long long by_tokens = live_ub / 64;
-    if (C > by_tokens) C = by_tokens < 1 ? 1 : by_tokens;
+    if (C > kMaxCluster) C = kMaxCluster;
+    if (C > live_ub / 128) C = live_ub / 128;
+    if (C < 1) C = 1;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)C, (unsigned)d.S, 1);
-    cfg.blockDim = dim3(32, 1, 1);
-    cfg.dynamicSmemBytes = 0;
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = kRingBytes;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
