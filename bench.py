@@ -283,7 +283,9 @@ def run_tkv(args, rank, world, dev):
     }
     tr = stored_traffic()
     if tr is not None:
-        res["roofline"]["traffic"] = tr["dram_bytes_per_launch"]
+        # DRAM bytes of one launch, from the committed capture, scaled to this launch's packed bytes
+        res["roofline"]["traffic"] = int(tr["traffic_per_packed_byte"] * pk)
+        res["roofline"]["traffic_source"] = tr["capture"] + " (scaled by packed bytes)"
     return res, gpu, w
 
 
