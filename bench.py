@@ -139,6 +139,15 @@ def gpu_smi_id(dev) -> str:
         return str(torch.cuda.current_device())
 
 
+def reduce_max(vals, world: int, device) -> list:
+    """Max over ranks of per-rank timings (every rank makes the same call)."""
+    if world <= 1:
+        return list(vals)
+    t = torch.tensor(list(vals), dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
+
+
 def packed_bytes(n: np.ndarray) -> int:
     return int(sum(int(n[:, c].sum()) * REC_BYTES[c] for c in range(4)))
 
@@ -214,10 +223,7 @@ def run_tkv(args, rank, world, dev):
     attn_ms = [m.elapsed_time(b2) for _, m, b2 in ev]
     t_step = sum(step_ms) / len(step_ms)
     t_attn = sum(attn_ms) / len(attn_ms)
-    if world > 1:
-        t = torch.tensor([t_step, t_attn], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        t_step, t_attn = t.tolist()
+    t_step, t_attn = reduce_max([t_step, t_attn], world, dev)
     assert gpu.poll_error() == 0
 
     # ---- end to end through the public API with host buffers
@@ -241,10 +247,7 @@ def run_tkv(args, rank, world, dev):
         if i >= args.warmup:
             e2e_ms.append(a.elapsed_time(b2))
     t_e2e = sum(e2e_ms) / len(e2e_ms)
-    if world > 1:
-        t = torch.tensor([t_e2e], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        t_e2e = t.item()
+    t_e2e, = reduce_max([t_e2e], world, dev)
     h2d = sum(x.numel() * x.element_size() for x in (hk, hv, hc, hp, hq))
     d2h = hout.numel() * hout.element_size()
 
