@@ -73,6 +73,14 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint64
                  : "memory");
 }
 
+// 16-byte copy that reads only `src_size` bytes (0 or 16) and zero-fills the rest.
+__device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void *src, uint32_t src_size,
+                                                 uint64_t policy) {
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;" ::"r"(dst), "l"(src),
+                 "r"(src_size), "l"(policy)
+                 : "memory");
+}
+
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 
 __device__ __forceinline__ void cp_async_wait_2() { asm volatile("cp.async.wait_group 2;" ::: "memory"); }
@@ -247,9 +255,9 @@ struct WarpState {
 };
 
 // One tile: up to ROWS records of one class, resident in shared memory (row stride
-// STRIDE).  Lane (g, tig) owns rows g and g + 8.  Rows at or beyond nr read the
-// last valid row instead (finite data, no divergent loads); their logits are
-// masked to -inf, so they contribute p = 0 everywhere.
+// STRIDE).  Lane (g, tig) owns rows g and g + 8.  Rows at or beyond nr hold zeros
+// (the copy zero-fills them); their logits are masked to -inf, so they contribute
+// p = 0 everywhere.
 template <int BITS, int ROWS, int STRIDE, int G>
 __device__ __forceinline__ void tile_compute(const uint8_t *st, int nr, int lane,
                                              const uint32_t (&qb)[4][2][2], const float (&qs)[2][4],
@@ -259,7 +267,7 @@ __device__ __forceinline__ void tile_compute(const uint8_t *st, int nr, int lane
     constexpr int CB = 16 * BITS;    // bytes of a code block
     const bool v0 = g < nr;
     const bool v1 = ROWS == 16 && g + 8 < nr;
-    const int i0 = min(g, nr - 1), i1 = min(g + 8, nr - 1);
+    const int i0 = g, i1 = g + 8;
     const uint8_t *r0 = st + i0 * STRIDE;
     const uint8_t *r1 = st + i1 * STRIDE;
     const int odd0 = BITS == 8 ? (i0 & 1) : 0, odd1 = BITS == 8 ? (i1 & 1) : 0;
@@ -375,8 +383,10 @@ __device__ __forceinline__ void tile_compute(const uint8_t *st, int nr, int lane
 // Copy a tile of class C_ into a stage with coalesced 16-byte cp.async: eight
 // consecutive lanes cover 128 contiguous bytes of one record, so one instruction
 // reads four whole 128-byte lines (records r = lane/8 + 4i).  `hd` holds, in lane
-// j < 16, the slot of the tile's record j.  Int8 rows are unpadded and odd rows
-// store 16-byte chunk k at k ^ 1.
+// j < 16, the slot of the tile's record j (any valid slot past the tile).  Rows at
+// or beyond nr are zero-filled without reading memory, so the copy has no
+// branches and the compute reads zeros (finite) there.  Int8 rows are unpadded and
+// odd rows store 16-byte chunk k at k ^ 1.
 template <int C_>
 __device__ __forceinline__ void issue_tile(uint32_t stage, const uint8_t *pool, int hd, int nr,
                                            int lane, uint64_t pol) {
@@ -390,15 +400,14 @@ __device__ __forceinline__ void issue_tile(uint32_t stage, const uint8_t *pool, 
     for (int i = 0; i < ROWS / 4; ++i) {
         const int r = (lane >> 3) + 4 * i;
         const int slot = __shfl_sync(kFull, hd, r);
-        if (r < nr) {
-            const uint8_t *src = pool + (size_t)slot * REC + 16 * sub;
-            int dpos = 16 * sub;
-            if constexpr (C_ == 1) dpos += (r & 1) ? ((sub & 1) ? -16 : 16) : 0;   // k ^ 1 on odd rows
-            const uint32_t dst = stage + r * STRIDE + dpos;
+        const uint32_t bytes = r < nr ? 16u : 0u;
+        const uint8_t *src = pool + (size_t)slot * REC + 16 * sub;
+        int dpos = 16 * sub;
+        if constexpr (C_ == 1) dpos += (r & 1) ? ((sub & 1) ? -16 : 16) : 0;   // k ^ 1 on odd rows
+        const uint32_t dst = stage + r * STRIDE + dpos;
 #pragma unroll
-            for (int j = 0; j < NBLK; ++j)
-                if (8 * j + sub < NCH) cp_async16(dst + 128 * j, src + 128 * j, pol);
-        }
+        for (int j = 0; j < NBLK; ++j)
+            if (8 * j + sub < NCH) cp_async16_zfill(dst + 128 * j, src + 128 * j, bytes, pol);
     }
 }
 
@@ -502,39 +511,46 @@ __global__ void __launch_bounds__(kThreads, 4) attn_kernel(const __grid_constant
     };
     const uint32_t magic = magic_f16();
 
-    // Warp tiles t_k = warp + 4k.  Iteration k computes t_k (stage k % 3) after
-    // issuing t_{k+2}; descriptors and handles of t_{k+2..k+4} sit in a register ring
-    // and t_{k+5}'s are loaded each iteration, three iterations before use.
-    int dc0 = tile_of(warp), dc1 = tile_of(warp + kWarps);
-    if (dc0 >= 0) issue(dc0, 0, handle_of(dc0));
-    cp_async_commit();
-    if (dc1 >= 0) issue(dc1, 1, handle_of(dc1));
-    cp_async_commit();
+    // Warp tiles t_k = warp + kWarps * k.  Iteration k computes t_k (stage k % 3)
+    // after issuing t_{k+2}; descriptors and handles of t_{k+2..k+4} sit in a
+    // register ring and t_{k+5}'s are loaded each iteration, three iterations
+    // before use.  The consumer runs one loop per class (compile-time class).
+    {
+        const int d0 = tile_of(warp), d1 = tile_of(warp + kWarps);
+        if (d0 >= 0) issue(d0, 0, handle_of(d0));
+        cp_async_commit();
+        if (d1 >= 0) issue(d1, 1, handle_of(d1));
+        cp_async_commit();
+    }
     int dr0 = tile_of(warp + 2 * kWarps), dr1 = tile_of(warp + 3 * kWarps), dr2 = tile_of(warp + 4 * kWarps);
     int hr0 = handle_of(dr0), hr1 = handle_of(dr1), hr2 = handle_of(dr2);
     int stage = 0;
-    for (int T = warp; dc0 >= 0; T += kWarps) {
+    int T = warp;
+    auto produce = [&]() {
         if (dr0 >= 0) issue(dr0, stage == 0 ? 2 : stage - 1, hr0);
         cp_async_commit();
-        const int dc2 = dr0;
         dr0 = dr1; dr1 = dr2; hr0 = hr1; hr1 = hr2;
         dr2 = tile_of(T + 5 * kWarps);
         hr2 = handle_of(dr2);
         cp_async_wait_2();
         __syncwarp();
-        const int ec = dc0 & 0xffffff, nc = (dc0 >> 24) & 31, cc = dc0 >> 29;
-        const uint8_t *st = ring + (warp * kStages + stage) * kStageBytes;
-        float *lg = lgs + (size_t)(sel4(cc, 0, o1, o2, o3) + ec) * G;
-        switch (cc) {
-            case 0: tile_compute<16, 8, 528, G>(st, nc, lane, qb, qs, xscale, ws, lg, magic); break;
-            case 1: tile_compute<8, 16, 288, G>(st, nc, lane, qb, qs, xscale, ws, lg, magic); break;
-            case 2: tile_compute<4, 16, 192, G>(st, nc, lane, qb, qs, xscale, ws, lg, magic); break;
-            default: tile_compute<2, 16, 96, G>(st, nc, lane, qb, qs, xscale, ws, lg, magic); break;
-        }
-        __syncwarp();
-        dc0 = dc1; dc1 = dc2;
-        stage = stage == 2 ? 0 : stage + 1;
+    };
+#define TKV_CONSUME(CLS, BITS, ROWS, STRIDE, PLO, PHI, LO, HI, OFF)                               \
+    for (; T < (PHI); T += kWarps) {                                                          \
+        produce();                                                                            \
+        const int e = (LO) + (T - (PLO)) * (ROWS);                                            \
+        const int nr = min((ROWS), (HI) - e);                                                 \
+        tile_compute<BITS, ROWS, STRIDE, G>(ring + (warp * kStages + stage) * kStageBytes, nr, \
+                                            lane, qb, qs, xscale, ws,                         \
+                                            lgs + (size_t)((OFF) + e) * G, magic);            \
+        __syncwarp();                                                                         \
+        stage = stage == 2 ? 0 : stage + 1;                                                   \
     }
+    TKV_CONSUME(0, 16, 8, 528, 0, p1, lo0, hi0, 0)
+    TKV_CONSUME(1, 8, 16, 288, p1, p2, lo1, hi1, o1)
+    TKV_CONSUME(2, 4, 16, 192, p2, p3, lo2, hi2, o2)
+    TKV_CONSUME(3, 2, 16, 96, p3, p4, lo3, hi3, o3)
+#undef TKV_CONSUME
     cp_async_wait_0();
 
     // ---- warp partials: reduce the lane partials over the 8 row lanes, fold z into O

@@ -280,3 +280,57 @@ def test_b1_ctx131k_long_decode_sampled_steps():
             else:
                 gpu.evict_compact(w["budget"])
     assert gpu.poll_error() == tkv.TKV_OK
+
+
+def test_l32_b32_ctx32k_decode_loop_sampled_layers_and_steps():
+    """32 layers x batch 32 x 32/8 heads, 32k context with K outliers and a 128-token
+    bf16 window, 1024 decode steps with eviction to 1638 every 64 steps.  Every layer
+    runs every step; lock-step oracle checks on one batch row of layers 0 and 31 at
+    steps 0, 63 (and the eviction after it), 64 and 1023."""
+    name = "l32_b32_ctx32k_1024steps"
+    spec = synth.WORKLOADS[name]
+    L, steps, E = spec["layers"], spec["steps"], spec["evict_every"]
+    rows, check_layers, check_steps = [3], (0, L - 1), (0, 63, 64, steps - 1)
+    caches, ws, oracles = [], [], {}
+    for layer in range(L):
+        w = synth.prefill_inputs(name, layer=layer, device=DEV)
+        cache = TkvCache(w["B"], w["Hkv"], w["G"], w["cap"], w["n_protect"], max_append=w["ctx"])
+        cache.quantize_append(w["k"], w["v"], w["cls"][:, :w["ctx"]].contiguous().to(DEV),
+                              w["pos"].to(DEV))
+        del w["k"], w["v"]
+        caches.append(cache)
+        ws.append(w)
+        if layer in check_layers:
+            oracles[layer] = oracle_for(cache, cache.export_state(rows_streams(cache, rows)), B=1)
+    torch.cuda.synchronize()
+    B, Hkv, Hq, D, ctx = spec["B"], spec["Hkv"], spec["Hq"], spec["D"], spec["ctx"]
+    cls_dev = ws[0]["cls"][:, ctx:ctx + steps].contiguous().to(DEV)
+    for c0 in range(0, steps, 64):
+        chunk = []
+        for layer in range(L):
+            seed = ws[layer]["seed"]
+            k = synth.normal_bf16(seed, layer, synth.TID_K, B, Hkv, ctx + c0, 64, D, DEV)
+            k = synth.apply_k_outliers(k, seed, layer)
+            v = synth.normal_bf16(seed, layer, synth.TID_V, B, Hkv, ctx + c0, 64, D, DEV)
+            q = synth.normal_bf16(seed, layer, synth.TID_Q, B, Hq, ctx + c0, 64, D, DEV)
+            chunk.append((k, v, q))
+        for j in range(64):
+            step = c0 + j
+            pos = torch.full((B, 1), ctx + step, dtype=torch.int32, device=DEV)
+            cls = cls_dev[:, step:step + 1].contiguous()
+            for layer in range(L):
+                if layer in check_layers and step in check_steps:
+                    _decode_step(ws[layer], caches[layer], oracles[layer], rows, step)
+                    continue
+                k, v, q = chunk[layer]
+                caches[layer].quantize_append(k[:, :, j:j + 1].contiguous(), v[:, :, j:j + 1].contiguous(),
+                                              cls, pos)
+                caches[layer].decode_attention(q[:, :, j].contiguous(), SCALE)
+            if (step + 1) % E == 0:
+                for layer in range(L):
+                    if layer in check_layers and step == 63:
+                        _evict_lockstep(caches[layer], oracles[layer], rows, spec["budget"])
+                    else:
+                        caches[layer].evict_compact(spec["budget"])
+    for cache in caches:
+        assert cache.poll_error() == tkv.TKV_OK
