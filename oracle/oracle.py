@@ -46,7 +46,7 @@ class _State(ctypes.Structure):
     _fields_ = [
         ("B", ctypes.c_int32), ("Hkv", ctypes.c_int32), ("G", ctypes.c_int32),
         ("D", ctypes.c_int32), ("group", ctypes.c_int32), ("n_protect", ctypes.c_int32),
-        ("bits", ctypes.c_int32 * 4), ("cap", ctypes.c_int32 * 4),
+        ("bits", ctypes.c_int32 * 4), ("cap", ctypes.c_int32 * 4), ("dense", ctypes.c_int32),
         ("pool", ctypes.c_void_p * 4),
         ("n", ctypes.c_void_p), ("ft", ctypes.c_void_p), ("hw", ctypes.c_void_p),
         ("handle", ctypes.c_void_p * 4), ("pos", ctypes.c_void_p * 4),
@@ -144,8 +144,9 @@ def num_threads() -> int:
 class OracleCache:
     """Host-side model of one layer's compressed cache."""
 
-    def __init__(self, B, Hkv, G, cap, n_protect, D=128, group=32, bits=BITS):
+    def __init__(self, B, Hkv, G, cap, n_protect, D=128, group=32, bits=BITS, dense=False):
         self.B, self.Hkv, self.G, self.D, self.group = B, Hkv, G, D, group
+        self.dense = bool(dense)
         self.n_protect = n_protect
         self.bits = tuple(bits)
         self.cap = tuple(int(c) for c in cap)
@@ -170,6 +171,7 @@ class OracleCache:
         st = _State()
         st.B, st.Hkv, st.G, st.D, st.group = self.B, self.Hkv, self.G, self.D, self.group
         st.n_protect = self.n_protect
+        st.dense = int(self.dense)
         for c in range(4):
             st.bits[c] = self.bits[c]
             st.cap[c] = self.cap[c]

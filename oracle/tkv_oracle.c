@@ -51,6 +51,7 @@ typedef struct {
     int32_t B, Hkv, G, D, group, n_protect;
     int32_t bits[4];   /* 16 (bf16), 8, 4, 2 for classes 0..3 */
     int32_t cap[4];    /* slots per stream per class */
+    int32_t dense;     /* 0: evicted slots reused in place; 1: dense placement */
     uint8_t *pool[4];  /* [S][cap[c]][rec_bytes(c)] */
     int32_t *n, *ft, *hw;          /* [S][4] */
     int32_t *handle[4], *pos[4], *fs[4];  /* [S][cap[c]] */
@@ -287,7 +288,8 @@ static uint8_t *record_ptr(const orc_state *st, int s, int c, int slot) {
  * Tokens are processed in order; a token at position < n_protect is stored in
  * class 0 (bf16).  Slot: pop the stream's free stack for that class if it is
  * non-empty, else take the next never-used slot; if neither exists the token
- * is dropped and CAPACITY is reported.  A class id > 3 drops the token and
+ * is dropped and CAPACITY is reported.  (In dense placement the free stack is
+ * always empty, so the slot is always the next never-used one.)  A class id > 3 drops the token and
  * reports INVALID.  New table entries start with score 0. */
 int orc_append(orc_state *st, const uint16_t *k, const uint16_t *v, const uint8_t *cls,
                const int32_t *pos, int T) {
@@ -424,7 +426,11 @@ static int cand_cmp(const void *pa, const void *pb) {
  * rest.  Each class list keeps its surviving entries in their previous order
  * (scores carried over).  The slots of evicted entries are pushed on the
  * class's free stack in reverse table order, so the earliest evicted entry
- * ends on top and is reused first.  budget >= candidates is a no-op. */
+ * ends on top and is reused first.  budget >= candidates is a no-op.
+ * Dense placement instead moves the record of the entry that ends at table
+ * index i to slot i, empties the free stack and sets the next never-used slot
+ * to the new entry count: a class's live records stay contiguous, in table
+ * order. */
 int orc_evict(orc_state *st, int budget) {
     if (budget < 0) return ORC_ERR_INVALID;
     const int S = n_streams(st);
@@ -455,11 +461,15 @@ int orc_evict(orc_state *st, int budget) {
                 for (int i = 0; i < n; ++i) m += evict[c][i];
                 int ft0 = st->ft[s * 4 + c];
                 int w = 0, r = 0;
+                size_t rb = (size_t)orc_record_bytes(st->bits[c], st->D, st->group);
+                uint8_t *moved = st->dense ? malloc(rb * (n - m > 0 ? n - m : 1)) : NULL;
                 for (int i = 0; i < n; ++i) {
                     if (evict[c][i]) {
-                        st->fs[c][base + ft0 + (m - 1 - r)] = st->handle[c][base + i];
+                        if (!st->dense) st->fs[c][base + ft0 + (m - 1 - r)] = st->handle[c][base + i];
                         ++r;
                     } else {
+                        if (st->dense)
+                            memcpy(moved + (size_t)w * rb, record_ptr(st, s, c, st->handle[c][base + i]), rb);
                         st->handle[c][base + w] = st->handle[c][base + i];
                         st->pos[c][base + w] = st->pos[c][base + i];
                         st->score[c][base + w] = st->score[c][base + i];
@@ -467,7 +477,17 @@ int orc_evict(orc_state *st, int budget) {
                     }
                 }
                 st->n[s * 4 + c] = w;
-                st->ft[s * 4 + c] = ft0 + m;
+                if (st->dense) {
+                    for (int i = 0; i < w; ++i) {
+                        memcpy(record_ptr(st, s, c, i), moved + (size_t)i * rb, rb);
+                        st->handle[c][base + i] = i;
+                    }
+                    st->hw[s * 4 + c] = w;
+                    st->ft[s * 4 + c] = 0;
+                    free(moved);
+                } else {
+                    st->ft[s * 4 + c] = ft0 + m;
+                }
                 free(evict[c]);
             }
         }

@@ -544,3 +544,40 @@ def test_scores_accumulate_over_steps():
         total += p.sum(axis=0)
     got = np.concatenate([cache.live(1, c)[2] for c in range(4)]).astype(np.float64)
     assert np.max(np.abs(got - total) / total) < 2e-7
+
+
+# --------------------------------------------------------------------------
+# dense placement: same results as in-place reuse, records kept contiguous
+# --------------------------------------------------------------------------
+def test_dense_placement_matches_in_place_reuse():
+    B, Hkv, G, ctx = 1, 2, 4, 900
+    cls = synth.class_ids(4, B, ctx + 40, 0.4, 0.4)
+    caps = class_capacities(cls, 4, extra=40)
+    ct = orc.OracleCache(B, Hkv, G, cap=caps, n_protect=4)
+    dn = orc.OracleCache(B, Hkv, G, cap=caps, n_protect=4, dense=True)
+    k = synth.normal_bf16(4, 0, synth.TID_K, B, Hkv, 0, ctx + 40, D)
+    v = synth.normal_bf16(4, 0, synth.TID_V, B, Hkv, 0, ctx + 40, D)
+    pos = synth.positions(B, 0, ctx + 40).numpy()
+    kb, vb, c = bits_of(k), bits_of(v), cls.numpy()
+    for cache in (ct, dn):
+        assert cache.append(kb[:, :, :ctx], vb[:, :, :ctx], c[:, :ctx], pos[:, :ctx]) == 0
+    for step in range(3):
+        q = bits_of(synth.normal_bf16(4, 0, synth.TID_Q, B, Hkv * G, ctx + step, 1, D)[:, :, 0])
+        o1, o2 = ct.attend(q, 0.09), dn.attend(q, 0.09)
+        assert np.array_equal(o1, o2)
+        for cache in (ct, dn):
+            t = ctx + step
+            cache.append(kb[:, :, t:t + 1], vb[:, :, t:t + 1], c[:, t:t + 1], pos[:, t:t + 1])
+        for cache in (ct, dn):
+            cache.evict(150 - 30 * step)
+        for s in range(ct.S):
+            for cc in range(4):
+                n = ct.state["n"][s, cc]
+                assert dn.state["n"][s, cc] == n
+                assert np.array_equal(ct.state[f"pos{cc}"][s, :n], dn.state[f"pos{cc}"][s, :n])
+                assert np.array_equal(ct.state[f"score{cc}"][s, :n], dn.state[f"score{cc}"][s, :n])
+                # dense: entry i lives in slot i, holding the record the in-place cache has
+                assert np.array_equal(dn.state[f"handle{cc}"][s, :n], np.arange(n))
+                assert dn.state["hw"][s, cc] == n and dn.state["ft"][s, cc] == 0
+                hs = ct.state[f"handle{cc}"][s, :n]
+                assert np.array_equal(dn.state[f"pool{cc}"][s, :n], ct.state[f"pool{cc}"][s, hs])
