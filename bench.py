@@ -50,6 +50,11 @@ def parse():
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=None)
+    ap.add_argument("--placement", choices=["dense", "reuse"], default="dense",
+                    help="record placement: dense (eviction moves kept records together, appends "
+                         "go after them) or reuse (records stay put, evicted slots are reused)")
+    ap.add_argument("--evict-reps", type=int, default=5,
+                    help="timed repetitions of the eviction that precedes the timed step")
     ap.add_argument("--ctx", type=int, default=None,
                     help="prefill context before the eviction (default: the workload's); the "
                          "timed step is the same post-eviction step, with smaller pools")
@@ -153,32 +158,49 @@ def packed_bytes(n: np.ndarray) -> int:
 
 
 # ----------------------------------------------------------------------------
-def setup_cache(w, dev, seed):
+def setup_cache(w, dev, dense, evict_reps, flush):
+    """Prefill, one scoring step, then the eviction to the budget.  The eviction is
+    timed (CUDA events, L2 flushed) over `evict_reps` repetitions, each from a copy
+    of the pre-eviction workspace; it is not part of the timed decode step."""
     from reasoning_model_kv_b200 import TkvCache
-    gpu = TkvCache(w["B"], w["Hkv"], w["G"], w["cap"], w["n_protect"], max_append=w["ctx"])
+    gpu = TkvCache(w["B"], w["Hkv"], w["G"], w["cap"], w["n_protect"], max_append=w["ctx"], dense=dense)
     cls = w["cls"][:, :w["ctx"]].contiguous().to(dev)
     gpu.quantize_append(w["k"], w["v"], cls, w["pos"].to(dev))
     k, v, c, p, q = synth.decode_inputs(w, 0, device=dev)        # untimed scoring step
     gpu.quantize_append(k, v, c, p)
     gpu.decode_attention(q, SCALE)
-    gpu.evict_compact(w["budget"])
+    evict_ms = []
+    snap = gpu.workspace.clone() if evict_reps > 0 else None
+    st = torch.cuda.current_stream()
+    for i in range(evict_reps + 1 if evict_reps > 0 else 1):
+        if snap is not None:
+            gpu.workspace.copy_(snap)
+        flush.zero_()
+        a, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        gpu.evict_compact(w["budget"])
+        b2.record(st)
+        b2.synchronize()
+        if i > 0:
+            evict_ms.append(a.elapsed_time(b2))
+    del snap
     torch.cuda.synchronize()
     assert gpu.poll_error() == 0
-    return gpu
+    return gpu, (statistics.median(evict_ms) if evict_ms else None)
 
 
 def run_tkv(args, rank, world, dev):
     over = {"ctx": args.ctx} if args.ctx else {}
     w = synth.prefill_inputs(args.workload, seed=rank, device=dev, steps=2, **over)
-    gpu = setup_cache(w, dev, rank)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
+    gpu, evict_ms = setup_cache(w, dev, args.placement == "dense", args.evict_reps, flush)
     del w["k"], w["v"]
     torch.cuda.empty_cache()
     views = gpu.state_views()
     saved = {k: views[k].clone() for k in ("n", "ft", "hw")}
     k, v, c, p, q = synth.decode_inputs(w, 1, device=dev)
     out = torch.empty((w["B"], w["Hq"], 128), dtype=torch.float32, device=dev)
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
 
     def restore():
         for key in ("n", "ft", "hw"):
@@ -270,11 +292,14 @@ def run_tkv(args, rank, world, dev):
                    "head_dim": 128, "context": w["ctx"], "budget": w["budget"],
                    "bf16_window": w["n_protect"], "p_RET": [w["p_r"], w["p_e"], 1 - w["p_r"] - w["p_e"]],
                    "live_kv_tokens": kv_tokens, "packed_kv_bytes": pk,
+                   "placement": args.placement,
                    "l2": "flushed (write of %d MB) before every timed step" % (flush.numel() >> 20),
                    "parallelism": f"{world} independent replicas" if world > 1 else "single GPU"},
         "hbm_gbs_packed": gbs,
         "frac_of_8tbs": gbs / NOMINAL_HBM_GBS,
         "attention_ms": t_attn,
+        "append_ms": t_step - t_attn,
+        "evict_ms_untimed_step": evict_ms,
         "kv_tokens_per_s": world * kv_tokens / (t_attn * 1e-3),
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
                      "frac": gbs / peak, "traffic": None, "peak_source": peak_src,
@@ -298,7 +323,8 @@ def cpu_baseline(gpu, w, rows, reps_budget_s=12.0):
     from oracle import oracle as orc
     sub = [b * w["Hkv"] + h for b in rows for h in range(w["Hkv"])]
     st = gpu.export_state(sub)
-    o = orc.OracleCache(len(rows), w["Hkv"], w["G"], cap=w["cap"], n_protect=w["n_protect"])
+    o = orc.OracleCache(len(rows), w["Hkv"], w["G"], cap=w["cap"], n_protect=w["n_protect"],
+                        dense=gpu.dense)
     k, v, c, p, q = synth.decode_inputs(w, 1)
 
     def bits(t):

@@ -75,6 +75,14 @@ typedef struct {
     int32_t n_protect;   /* positions [0, n_protect) are bf16, never evicted   */
     int32_t cap[4];      /* slots per stream for each class (>= 0)             */
     int32_t max_append;  /* largest T accepted by tkv_quantize_append (>= 1)   */
+    int32_t dense;       /* placement: 0 = evicted slots are reused in place
+                            (free stacks, the pages' Continuous Thinking);
+                            1 = dense: eviction moves each kept record to the
+                            slot equal to its table index and appends always
+                            take the next never-used slot, so a class's live
+                            records are contiguous in table order (handle[i] ==
+                            i) and decode reads them as whole blocks.  Results
+                            are identical in both modes.                      */
 } tkv_config;
 
 typedef struct tkv_cache tkv_cache;
@@ -182,7 +190,10 @@ TKV_API tkv_status tkv_decode_attention(tkv_cache *cache, const void *q, float s
  * keeps its survivors in their previous order with their scores; evicted
  * slots are pushed on the class's free stack in reverse table order, so the
  * earliest evicted entry is reused first.  A stream with <= budget
- * unprotected tokens is untouched.
+ * unprotected tokens is untouched.  In dense placement (cfg.dense = 1) the kept
+ * records are instead moved to the slots equal to their new table indices, the
+ * free stack stays empty and the next never-used slot becomes the entry count;
+ * dense placement requires handle[i] == i on entry (which it maintains).
  */
 TKV_API tkv_status tkv_evict_compact(tkv_cache *cache, int32_t budget, void *stream);
 

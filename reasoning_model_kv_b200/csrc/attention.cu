@@ -67,12 +67,6 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
     return p;
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint64_t policy) {
-    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
-                 "l"(policy)
-                 : "memory");
-}
-
 // 16-byte copy that reads only `src_size` bytes (0 or 16) and zero-fills the rest.
 __device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void *src, uint32_t src_size,
                                                  uint64_t policy) {
@@ -86,6 +80,53 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 __device__ __forceinline__ void cp_async_wait_2() { asm volatile("cp.async.wait_group 2;" ::: "memory"); }
 
 __device__ __forceinline__ void cp_async_wait_0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// ---- dense placement: one bulk copy per tile, completion tracked by an mbarrier
+__device__ __forceinline__ void mbar_init(uint32_t bar) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_init_fence() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ uint32_t mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return done;
+}
+
+// Bounded wait for phase `parity` of the barrier: false after ~1 s without it.
+constexpr long long kWaitCycles = 1ll << 31;
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity))
+        if (clock64() - t0 > kWaitCycles) return false;
+    return true;
+}
+
+__device__ __forceinline__ void bulk_copy(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar,
+                                          uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, "
+        "[%3], %4;" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
 
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
@@ -255,10 +296,10 @@ struct WarpState {
 };
 
 // One tile: up to ROWS records of one class, resident in shared memory (row stride
-// STRIDE).  Lane (g, tig) owns rows g and g + 8.  Rows at or beyond nr hold zeros
-// (the copy zero-fills them); their logits are masked to -inf, so they contribute
-// p = 0 everywhere.
-template <int BITS, int ROWS, int STRIDE, int G>
+// STRIDE; int8 odd rows chunk-swizzled when SWZ).  Lane (g, tig) owns rows g and
+// g + 8.  Rows at or beyond nr hold zeros (the copy zero-fills them); their logits
+// are masked to -inf, so they contribute p = 0 everywhere.
+template <int BITS, int ROWS, int STRIDE, int G, bool SWZ>
 __device__ __forceinline__ void tile_compute(const uint8_t *st, int nr, int lane,
                                              const uint32_t (&qb)[4][2][2], const float (&qs)[2][4],
                                              float xscale, WarpState &ws, float *lg, uint32_t magic) {
@@ -270,7 +311,7 @@ __device__ __forceinline__ void tile_compute(const uint8_t *st, int nr, int lane
     const int i0 = g, i1 = g + 8;
     const uint8_t *r0 = st + i0 * STRIDE;
     const uint8_t *r1 = st + i1 * STRIDE;
-    const int odd0 = BITS == 8 ? (i0 & 1) : 0, odd1 = BITS == 8 ? (i1 & 1) : 0;
+    const int odd0 = (BITS == 8 && SWZ) ? (i0 & 1) : 0, odd1 = (BITS == 8 && SWZ) ? (i1 & 1) : 0;
     // meta chunk positions (int8 rows: chunks 16 and 17 swap on odd rows)
     const int km_off0 = 2 * CB + 16 * odd0, vm_off0 = 2 * CB + 16 - 16 * odd0;
     const int km_off1 = 2 * CB + 16 * odd1, vm_off1 = 2 * CB + 16 - 16 * odd1;
@@ -411,7 +452,30 @@ __device__ __forceinline__ void issue_tile(uint32_t stage, const uint8_t *pool, 
     }
 }
 
-template <int G>
+// Dense placement: the tile's nr records are nr * REC contiguous bytes of the pool,
+// copied by one bulk copy into an unpadded stage (row stride REC).  Rows nr..ROWS-1
+// of the stage are zeroed first by the warp (generic stores, then a proxy fence so
+// they are ordered before later bulk writes of the stage).
+template <int C_>
+__device__ __forceinline__ void issue_tile_dense(uint8_t *stage_ptr, uint32_t stage, const uint8_t *src,
+                                                 int nr, int lane, uint32_t bar, uint64_t pol) {
+    constexpr int REC = C_ == 0 ? 512 : C_ == 1 ? 288 : C_ == 2 ? 160 : 96;
+    constexpr int ROWS = C_ == 0 ? 8 : 16;
+    if (nr < ROWS) {
+        uint4 *z = reinterpret_cast<uint4 *>(stage_ptr + nr * REC);
+        const int nz = (ROWS - nr) * (REC / 16);
+        for (int i = lane; i < nz; i += 32) z[i] = make_uint4(0u, 0u, 0u, 0u);
+        fence_proxy_async_smem();
+        __syncwarp();
+    }
+    if (lane == 0) {
+        const uint32_t bytes = (uint32_t)(nr * REC);
+        mbar_expect_tx(bar, bytes);
+        bulk_copy(stage, src, bytes, bar, pol);
+    }
+}
+
+template <int G, bool DENSE>
 __global__ void __launch_bounds__(kThreads, 4) attn_kernel(const __grid_constant__ Dev d,
                                                            const __nv_bfloat16 *__restrict__ q,
                                                            float xscale, float *__restrict__ out,
@@ -420,6 +484,7 @@ __global__ void __launch_bounds__(kThreads, 4) attn_kernel(const __grid_constant
     __shared__ float cta_m[kMaxG], cta_l[kMaxG];
     __shared__ float fac[kMaxCluster][kMaxG];     // exp2(m_j - M) per warp / peer rank and head
     __shared__ float gM[kMaxG], gInvL[kMaxG];
+    __shared__ __align__(8) uint64_t bars[kWarps][kStages];   // dense placement only
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, tig = lane & 3;
@@ -482,6 +547,17 @@ __global__ void __launch_bounds__(kThreads, 4) attn_kernel(const __grid_constant
 
     const uint64_t pol = policy_evict_first();
     const uint32_t ring0 = smem_addr(ring) + warp * kStages * kStageBytes;
+    uint8_t *ring_w = ring + warp * kStages * kStageBytes;
+    const uint32_t bar0 = smem_addr(&bars[warp][0]);   // stage i: bar0 + 8 i
+    uint32_t phase = 0;                                // dense: parity bit per stage
+    if constexpr (DENSE) {
+        if (lane == 0) {
+#pragma unroll
+            for (int i = 0; i < kStages; ++i) mbar_init(bar0 + 8 * i);
+            mbar_init_fence();
+        }
+        __syncwarp();
+    }
 
     // tile T -> packed descriptor: entry e (bits 0-23), rows nr (24-28), class c (29-30)
     auto tile_of = [&](int T) -> int {
@@ -492,35 +568,63 @@ __global__ void __launch_bounds__(kThreads, 4) attn_kernel(const __grid_constant
         const int nr = min(rows, sel4(c, hi0, hi1, hi2, hi3) - e);
         return e | (nr << 24) | (c << 29);
     };
-    // lane j holds the slot of record min(j, nr - 1) of a tile
+    // lane j holds the slot of record min(j, nr - 1) of a tile (slot = entry when dense)
     auto handle_of = [&](int dsc) -> int {
-        if (dsc < 0) return 0;
-        const int e = dsc & 0xffffff, nr = (dsc >> 24) & 31, c = dsc >> 29;
-        return d.handle[c][(size_t)s * d.cap[c] + e + min(lane, nr - 1)];
+        if constexpr (DENSE) {
+            return 0;
+        } else {
+            if (dsc < 0) return 0;
+            const int e = dsc & 0xffffff, nr = (dsc >> 24) & 31, c = dsc >> 29;
+            return d.handle[c][(size_t)s * d.cap[c] + e + min(lane, nr - 1)];
+        }
     };
     auto issue = [&](int dsc, int stage, int hd) {
         const int nr = (dsc >> 24) & 31, c = dsc >> 29;
         const uint32_t st = ring0 + stage * kStageBytes;
         const uint8_t *pool = d.pool[c] + (size_t)s * d.cap[c] * d.rec[c];
-        switch (c) {
-            case 0: issue_tile<0>(st, pool, hd, nr, lane, pol); break;
-            case 1: issue_tile<1>(st, pool, hd, nr, lane, pol); break;
-            case 2: issue_tile<2>(st, pool, hd, nr, lane, pol); break;
-            default: issue_tile<3>(st, pool, hd, nr, lane, pol); break;
+        if constexpr (DENSE) {
+            const int e = dsc & 0xffffff;
+            uint8_t *sp = ring_w + stage * kStageBytes;
+            const uint32_t bar = bar0 + 8 * stage;
+            switch (c) {
+                case 0: issue_tile_dense<0>(sp, st, pool + (size_t)e * 512, nr, lane, bar, pol); break;
+                case 1: issue_tile_dense<1>(sp, st, pool + (size_t)e * 288, nr, lane, bar, pol); break;
+                case 2: issue_tile_dense<2>(sp, st, pool + (size_t)e * 160, nr, lane, bar, pol); break;
+                default: issue_tile_dense<3>(sp, st, pool + (size_t)e * 96, nr, lane, bar, pol); break;
+            }
+        } else {
+            switch (c) {
+                case 0: issue_tile<0>(st, pool, hd, nr, lane, pol); break;
+                case 1: issue_tile<1>(st, pool, hd, nr, lane, pol); break;
+                case 2: issue_tile<2>(st, pool, hd, nr, lane, pol); break;
+                default: issue_tile<3>(st, pool, hd, nr, lane, pol); break;
+            }
         }
+    };
+    // wait until the tile in `stage` has landed (dense: its barrier phase; otherwise
+    // the cp.async groups, two of which may stay in flight)
+    auto arrive_wait = [&](int stage) {
+        if constexpr (DENSE) {
+            const bool ok = mbar_wait(bar0 + 8 * stage, (phase >> stage) & 1u);
+            phase ^= 1u << stage;
+            if (!__all_sync(kFull, ok) && lane == 0) raise_error(d.err, kErrTimeout, (uint32_t)s);
+        } else {
+            cp_async_wait_2();
+        }
+        __syncwarp();
     };
     const uint32_t magic = magic_f16();
 
     // Warp tiles t_k = warp + kWarps * k.  Iteration k computes t_k (stage k % 3)
-    // after issuing t_{k+2}; descriptors and handles of t_{k+2..k+4} sit in a
+    // after issuing t_{k+2}; descriptors (and handles) of t_{k+2..k+4} sit in a
     // register ring and t_{k+5}'s are loaded each iteration, three iterations
     // before use.  The consumer runs one loop per class (compile-time class).
     {
         const int d0 = tile_of(warp), d1 = tile_of(warp + kWarps);
         if (d0 >= 0) issue(d0, 0, handle_of(d0));
-        cp_async_commit();
+        if constexpr (!DENSE) cp_async_commit();
         if (d1 >= 0) issue(d1, 1, handle_of(d1));
-        cp_async_commit();
+        if constexpr (!DENSE) cp_async_commit();
     }
     int dr0 = tile_of(warp + 2 * kWarps), dr1 = tile_of(warp + 3 * kWarps), dr2 = tile_of(warp + 4 * kWarps);
     int hr0 = handle_of(dr0), hr1 = handle_of(dr1), hr2 = handle_of(dr2);
@@ -528,30 +632,36 @@ __global__ void __launch_bounds__(kThreads, 4) attn_kernel(const __grid_constant
     int T = warp;
     auto produce = [&]() {
         if (dr0 >= 0) issue(dr0, stage == 0 ? 2 : stage - 1, hr0);
-        cp_async_commit();
+        if constexpr (!DENSE) cp_async_commit();
         dr0 = dr1; dr1 = dr2; hr0 = hr1; hr1 = hr2;
         dr2 = tile_of(T + 5 * kWarps);
         hr2 = handle_of(dr2);
-        cp_async_wait_2();
-        __syncwarp();
+        arrive_wait(stage);
     };
 #define TKV_CONSUME(CLS, BITS, ROWS, STRIDE, PLO, PHI, LO, HI, OFF)                               \
     for (; T < (PHI); T += kWarps) {                                                          \
         produce();                                                                            \
         const int e = (LO) + (T - (PLO)) * (ROWS);                                            \
         const int nr = min((ROWS), (HI) - e);                                                 \
-        tile_compute<BITS, ROWS, STRIDE, G>(ring + (warp * kStages + stage) * kStageBytes, nr, \
-                                            lane, qb, qs, xscale, ws,                         \
-                                            lgs + (size_t)((OFF) + e) * G, magic);            \
+        tile_compute<BITS, ROWS, STRIDE, G, !DENSE>(ring + (warp * kStages + stage) * kStageBytes, \
+                                                    nr, lane, qb, qs, xscale, ws,             \
+                                                    lgs + (size_t)((OFF) + e) * G, magic);    \
         __syncwarp();                                                                         \
         stage = stage == 2 ? 0 : stage + 1;                                                   \
     }
-    TKV_CONSUME(0, 16, 8, 528, 0, p1, lo0, hi0, 0)
-    TKV_CONSUME(1, 8, 16, 288, p1, p2, lo1, hi1, o1)
-    TKV_CONSUME(2, 4, 16, 192, p2, p3, lo2, hi2, o2)
-    TKV_CONSUME(3, 2, 16, 96, p3, p4, lo3, hi3, o3)
+    if constexpr (DENSE) {
+        TKV_CONSUME(0, 16, 8, 512, 0, p1, lo0, hi0, 0)
+        TKV_CONSUME(1, 8, 16, 288, p1, p2, lo1, hi1, o1)
+        TKV_CONSUME(2, 4, 16, 160, p2, p3, lo2, hi2, o2)
+        TKV_CONSUME(3, 2, 16, 96, p3, p4, lo3, hi3, o3)
+    } else {
+        TKV_CONSUME(0, 16, 8, 528, 0, p1, lo0, hi0, 0)
+        TKV_CONSUME(1, 8, 16, 288, p1, p2, lo1, hi1, o1)
+        TKV_CONSUME(2, 4, 16, 192, p2, p3, lo2, hi2, o2)
+        TKV_CONSUME(3, 2, 16, 96, p3, p4, lo3, hi3, o3)
+    }
 #undef TKV_CONSUME
-    cp_async_wait_0();
+    if constexpr (!DENSE) cp_async_wait_0();
 
     // ---- warp partials: reduce the lane partials over the 8 row lanes, fold z into O
 #pragma unroll
@@ -671,10 +781,10 @@ __global__ void __launch_bounds__(kThreads, 4) attn_kernel(const __grid_constant
     if (C > 1) cluster_sync();   // peers may still be reading this CTA's shared memory
 }
 
-int g_blocks_per_sm[kMaxG + 1] = {0};
+int g_blocks_per_sm[2][kMaxG + 1] = {};
 int g_sms = 0;
 
-template <int G>
+template <int G, bool DENSE>
 cudaError_t launch_g(const Dev &d, const void *q, float scale, float *out, long long live_ub,
                      cudaStream_t st, int64_t *launches) {
     if (g_sms == 0) {
@@ -682,18 +792,19 @@ cudaError_t launch_g(const Dev &d, const void *q, float scale, float *out, long 
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&g_sms, cudaDevAttrMultiProcessorCount, dev);
     }
-    if (g_blocks_per_sm[G] == 0) {
-        cudaError_t e = cudaFuncSetAttribute(attn_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             kRingBytes);
+    int &bps = g_blocks_per_sm[DENSE][G];
+    if (bps == 0) {
+        cudaError_t e = cudaFuncSetAttribute(attn_kernel<G, DENSE>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, kRingBytes);
         if (e != cudaSuccess) return e;
         int nb = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, attn_kernel<G>, kThreads, kRingBytes);
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, attn_kernel<G, DENSE>, kThreads, kRingBytes);
         if (e != cudaSuccess) return e;
-        g_blocks_per_sm[G] = nb > 0 ? nb : 1;
+        bps = nb > 0 ? nb : 1;
     }
     // Largest cluster (<= 8) whose grid is fully resident, never splitting a stream
     // below ~128 tokens per CTA; one CTA per stream when the streams fill the GPU.
-    const long long slots = (long long)g_blocks_per_sm[G] * g_sms;
+    const long long slots = (long long)bps * g_sms;
     long long C = slots / d.S;
     if (C > kMaxCluster) C = kMaxCluster;
     if (C > live_ub / 128) C = live_ub / 128;
@@ -711,7 +822,7 @@ cudaError_t launch_g(const Dev &d, const void *q, float scale, float *out, long 
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     const float xscale = scale * 1.4426950408889634f;   // logits in the log2 domain
-    cudaError_t e = cudaLaunchKernelEx(&cfg, attn_kernel<G>, d, static_cast<const __nv_bfloat16 *>(q),
+    cudaError_t e = cudaLaunchKernelEx(&cfg, attn_kernel<G, DENSE>, d, static_cast<const __nv_bfloat16 *>(q),
                                        xscale, out, (int)C);
     *launches += 1;
     return e;
@@ -721,11 +832,20 @@ cudaError_t launch_g(const Dev &d, const void *q, float scale, float *out, long 
 
 cudaError_t launch_attention(const Dev &d, const void *q, float scale, float *out, long long live_ub,
                              cudaStream_t st, int64_t *launches) {
+    if (d.dense) {
+        switch (d.G) {
+            case 1: return launch_g<1, true>(d, q, scale, out, live_ub, st, launches);
+            case 2: return launch_g<2, true>(d, q, scale, out, live_ub, st, launches);
+            case 4: return launch_g<4, true>(d, q, scale, out, live_ub, st, launches);
+            case 8: return launch_g<8, true>(d, q, scale, out, live_ub, st, launches);
+            default: return cudaErrorInvalidValue;
+        }
+    }
     switch (d.G) {
-        case 1: return launch_g<1>(d, q, scale, out, live_ub, st, launches);
-        case 2: return launch_g<2>(d, q, scale, out, live_ub, st, launches);
-        case 4: return launch_g<4>(d, q, scale, out, live_ub, st, launches);
-        case 8: return launch_g<8>(d, q, scale, out, live_ub, st, launches);
+        case 1: return launch_g<1, false>(d, q, scale, out, live_ub, st, launches);
+        case 2: return launch_g<2, false>(d, q, scale, out, live_ub, st, launches);
+        case 4: return launch_g<4, false>(d, q, scale, out, live_ub, st, launches);
+        case 8: return launch_g<8, false>(d, q, scale, out, live_ub, st, launches);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -15,13 +15,16 @@
 // index order, resolved by a block scan during compaction.  Compaction runs
 // each class table chunk by chunk; a chunk is read into registers before any
 // thread writes, and every write goes to an index no larger than its source,
-// so the table compacts in place.
+// so the table compacts in place.  In dense placement (handle[i] == i) the kept
+// records move the same way, from slot i to slot = new index, staged through
+// shared memory in batches.
 #include "tkv_internal.cuh"
 
 namespace tkv {
 namespace {
 
 constexpr int kThreads = 512;
+constexpr int kMoveBytes = 16384;   // dense placement: records staged per move batch
 constexpr int kWarpsE = kThreads / 32;
 constexpr unsigned kFull = 0xffffffffu;
 
@@ -76,6 +79,8 @@ __global__ void __launch_bounds__(kThreads) evict_kernel(Dev d, int budget) {
     const int s = blockIdx.x;
     __shared__ unsigned hist[256];
     __shared__ int scratch[33];
+    __shared__ int move_src[kThreads];                       // dense: source slot per kept entry
+    __shared__ uint4 move_buf[kMoveBytes / sizeof(uint4)];
     __shared__ unsigned long long sh_prefix;
     __shared__ int sh_bits, sh_rem, sh_done;
 
@@ -177,6 +182,8 @@ __global__ void __launch_bounds__(kThreads) evict_kernel(Dev d, int budget) {
         int32_t *fsc = d.fs[c] + base_e;
         const int ft0 = d.ft[s * 4 + c];
         const int m = evicted[c];
+        const int rec = d.rec[c];
+        uint8_t *pool = d.pool[c] + base_e * rec;
         int kept_carry = 0, ev_carry = 0;
         for (int base = 0; base < n[c]; base += kThreads) {
             const int i = base + threadIdx.x;
@@ -208,11 +215,36 @@ __global__ void __launch_bounds__(kThreads) evict_kernel(Dev d, int budget) {
             // block_scan ends with a barrier: the whole chunk has been read
             if (valid) {
                 if (keep) {
-                    hc[wk] = hd;
+                    hc[wk] = d.dense ? wk : hd;
                     pc[wk] = p;
                     sc[wk] = scv;
-                } else {
+                    if (d.dense) move_src[wk - kept_carry] = i;
+                } else if (!d.dense) {
                     fsc[ft0 + (m - 1 - r)] = hd;
+                }
+            }
+            if (d.dense) {
+                // move this chunk's kept records from slot i to slot wk (wk <= i), in
+                // batches staged through shared memory: a batch is read completely before
+                // any of it is written, and later batches only read slots above this one's
+                __syncthreads();
+                const int per_rec = rec / 16;
+                const int batch = kMoveBytes / rec;
+                for (int b0 = 0; b0 < nkeep; b0 += batch) {
+                    const int nb_rec = min(batch, nkeep - b0);
+                    const int pieces = nb_rec * per_rec;
+                    for (int q = threadIdx.x; q < pieces; q += kThreads) {
+                        const int k = q / per_rec, part = q - k * per_rec;
+                        move_buf[k * per_rec + part] =
+                            reinterpret_cast<const uint4 *>(pool + (size_t)move_src[b0 + k] * rec)[part];
+                    }
+                    __syncthreads();
+                    for (int q = threadIdx.x; q < pieces; q += kThreads) {
+                        const int k = q / per_rec, part = q - k * per_rec;
+                        reinterpret_cast<uint4 *>(pool + (size_t)(kept_carry + b0 + k) * rec)[part] =
+                            move_buf[k * per_rec + part];
+                    }
+                    __syncthreads();
                 }
             }
             kept_carry += nkeep;
@@ -221,7 +253,12 @@ __global__ void __launch_bounds__(kThreads) evict_kernel(Dev d, int budget) {
         }
         if (threadIdx.x == 0) {
             d.n[s * 4 + c] = n[c] - m;
-            d.ft[s * 4 + c] = ft0 + m;
+            if (d.dense) {
+                d.ft[s * 4 + c] = 0;
+                d.hw[s * 4 + c] = n[c] - m;
+            } else {
+                d.ft[s * 4 + c] = ft0 + m;
+            }
         }
     }
 }

@@ -21,6 +21,7 @@ __host__ __device__ constexpr int record_bytes(int bits) {
 // Everything a kernel needs to address one cache.  Passed by value.
 struct Dev {
     int B, Hkv, G, S, n_protect, max_append;
+    int dense;              // 1: live records contiguous in table order (handle[i] == i)
     int cap[4];
     int rec[4];
     int32_t *n, *ft, *hw;   // [S][4]

@@ -30,7 +30,7 @@ class TkvConfig(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("Hkv", ctypes.c_int32), ("G", ctypes.c_int32),
                 ("D", ctypes.c_int32), ("group", ctypes.c_int32), ("bits", ctypes.c_int32 * 4),
                 ("n_protect", ctypes.c_int32), ("cap", ctypes.c_int32 * 4),
-                ("max_append", ctypes.c_int32)]
+                ("max_append", ctypes.c_int32), ("dense", ctypes.c_int32)]
 
 
 class TkvLayout(ctypes.Structure):
@@ -90,7 +90,7 @@ def _check(status: int):
         raise TkvError(status, lib().tkv_last_error_string().decode())
 
 
-def make_config(B, Hkv, G, cap, n_protect, max_append=1, D=128, group=32) -> TkvConfig:
+def make_config(B, Hkv, G, cap, n_protect, max_append=1, D=128, group=32, dense=False) -> TkvConfig:
     cfg = TkvConfig()
     cfg.B, cfg.Hkv, cfg.G, cfg.D, cfg.group = B, Hkv, G, D, group
     for i in range(4):
@@ -98,6 +98,7 @@ def make_config(B, Hkv, G, cap, n_protect, max_append=1, D=128, group=32) -> Tkv
         cfg.cap[i] = int(cap[i])
     cfg.n_protect = n_protect
     cfg.max_append = max_append
+    cfg.dense = int(bool(dense))
     return cfg
 
 
@@ -125,8 +126,9 @@ class TkvCache:
     """One layer's compressed KV cache: a device workspace owned by torch plus the
     library's cache object.  Methods mirror the C ABI names."""
 
-    def __init__(self, B, Hkv, G, cap, n_protect, max_append=1, device="cuda"):
-        self.cfg = make_config(B, Hkv, G, cap, n_protect, max_append)
+    def __init__(self, B, Hkv, G, cap, n_protect, max_append=1, device="cuda", dense=False):
+        self.cfg = make_config(B, Hkv, G, cap, n_protect, max_append, dense=dense)
+        self.dense = bool(dense)
         self.B, self.Hkv, self.G, self.S = B, Hkv, G, B * Hkv
         self.cap = tuple(int(c) for c in cap)
         self.n_protect, self.max_append = n_protect, max_append

@@ -52,11 +52,23 @@ def _evict_lockstep(gpu, o, rows, budget):
     compare_states(gpu.export_state(sub), o.state, what=f"evict {budget}")
 
 
+def _assert_dense(gpu):
+    """Dense placement invariant: entry i of every class table lives in slot i."""
+    g = gpu.export_state()
+    assert (g["ft"] == 0).all() and np.array_equal(g["hw"], g["n"])
+    for c in range(4):
+        for s in range(gpu.S):
+            n = g["n"][s, c]
+            assert np.array_equal(g[f"handle{c}"][s, :n], np.arange(n)), (c, s)
+
+
 # ----------------------------------------------------------------------------
-def test_tiny_prefill_decode_evict_reuse():
+@pytest.mark.parametrize("dense", [False, True], ids=["reuse", "dense"])
+def test_tiny_prefill_decode_evict_reuse(dense):
     """2k-token single-layer workload: prefill, decode step, eviction to 512, and
-    a second step that reuses evicted slots."""
-    w, gpu, o, rows = build_pair("tiny_b1_ctx2k")
+    a second step that reuses evicted slots (dense placement: appends after the
+    moved records)."""
+    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", dense=dense)
     compare_states(gpu.export_state(), o.state, what="prefill")
     _decode_step(w, gpu, o, rows, 0)
     _evict_lockstep(gpu, o, rows, w["budget"])
@@ -66,6 +78,8 @@ def test_tiny_prefill_decode_evict_reuse():
     w2["cls"] = synth.class_ids(0, w["B"], w["ctx"] + 2, w["p_r"], w["p_e"])
     _decode_step(w2, gpu, o, rows, 1)
     assert gpu.launch_count() > 0
+    if dense:
+        _assert_dense(gpu)
 
 
 def test_kept_sets_free_running_match_up_to_near_ties():
@@ -98,19 +112,21 @@ def test_kept_sets_free_running_match_up_to_near_ties():
                 assert abs(sc[p] - thr) <= 1e-4 * thr, (p, sc[p], thr)
 
 
+@pytest.mark.parametrize("dense", [False, True], ids=["reuse", "dense"])
 @pytest.mark.parametrize("G,n_protect,outliers", [(1, 4, False), (2, 128, True), (4, 4, True),
                                                   (8, 128, False)])
-def test_gqa_widths_and_windows(G, n_protect, outliers):
+def test_gqa_widths_and_windows(G, n_protect, outliers, dense):
     w, gpu, o, rows = build_pair("tiny_b1_ctx2k", B=2, Hq=2 * G, Hkv=2, ctx=709,
-                                 n_protect=n_protect, outliers=outliers, steps=2)
+                                 n_protect=n_protect, outliers=outliers, steps=2, dense=dense)
     compare_states(gpu.export_state(), o.state, what="prefill")
     _decode_step(w, gpu, o, rows, 0)
     _evict_lockstep(gpu, o, rows, 300)
     _decode_step(w, gpu, o, rows, 1)
 
 
-def test_multi_token_append_after_eviction_reuses_slots_in_order():
-    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", ctx=600, steps=80)
+@pytest.mark.parametrize("dense", [False, True], ids=["reuse", "dense"])
+def test_multi_token_append_after_eviction_reuses_slots_in_order(dense):
+    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", ctx=600, steps=80, dense=dense)
     gpu.decode_attention(synth.decode_inputs(w, 0)[4].to(DEV), SCALE)
     _evict_lockstep(gpu, o, rows, 100)
     T = 77
@@ -143,8 +159,9 @@ def test_empty_cache_and_single_token():
     assert abs(g["score3"][0, 0] - 4.0) < 1e-6 and abs(g["score3"][1, 0] - 4.0) < 1e-6
 
 
-def test_budget_edge_cases():
-    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", ctx=300, n_protect=17)
+@pytest.mark.parametrize("dense", [False, True], ids=["reuse", "dense"])
+def test_budget_edge_cases(dense):
+    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", ctx=300, n_protect=17, dense=dense)
     gpu.decode_attention(synth.decode_inputs(w, 0)[4].to(DEV), SCALE)
     before = gpu.export_state()
     gpu.evict_compact(300)                     # budget >= candidates: untouched
@@ -168,12 +185,13 @@ def test_all_scores_equal_keep_lowest_positions():
         assert kept == list(range(44))
 
 
-def test_exact_key_ties_resolved_by_class_then_index():
+@pytest.mark.parametrize("dense", [False, True], ids=["reuse", "dense"])
+def test_exact_key_ties_resolved_by_class_then_index(dense):
     """Duplicate positions with equal scores: the 64-bit key ties, so class then table
     index decide (same rule on both sides)."""
     B, Hkv, T = 1, 1, 40
-    gpu = TkvCache(B, Hkv, 4, cap=[4, 40, 40, 40], n_protect=0, max_append=T)
-    o = orc.OracleCache(B, Hkv, 4, cap=[4, 40, 40, 40], n_protect=0)
+    gpu = TkvCache(B, Hkv, 4, cap=[4, 40, 40, 40], n_protect=0, max_append=T, dense=dense)
+    o = orc.OracleCache(B, Hkv, 4, cap=[4, 40, 40, 40], n_protect=0, dense=dense)
     k = synth.normal_bf16(3, 0, synth.TID_K, B, Hkv, 0, T, 128)
     cls = torch.tensor([[1 + (t % 3) for t in range(T)]], dtype=torch.uint8)
     pos = torch.tensor([[t // 4 for t in range(T)]], dtype=torch.int32)   # duplicates
@@ -218,14 +236,15 @@ def test_binding_rejects_wrong_tensors():
 # ----------------------------------------------------------------------------
 # The workload shapes of the decode configurations, lock-step on sampled rows/steps
 # ----------------------------------------------------------------------------
-def test_b64_ctx32k_timed_step_sampled_rows():
+@pytest.mark.parametrize("dense", [False, True], ids=["reuse", "dense"])
+def test_b64_ctx32k_timed_step_sampled_rows(dense):
     """Batch 64 x 32/8 heads, 32k context, K outliers, 5 % budget + 128-token bf16
     window: prefill, scoring step, eviction to 1638, then the timed step
     (append + attention), compared on three sampled batch rows."""
     rows = [0, 37, 63]
     w = synth.prefill_inputs("b64_ctx32k_evict5pct", device=DEV, steps=2)
     w["cls"] = synth.class_ids(0, w["B"], w["ctx"] + 2, w["p_r"], w["p_e"])
-    gpu = TkvCache(w["B"], w["Hkv"], w["G"], w["cap"], w["n_protect"], max_append=w["ctx"])
+    gpu = TkvCache(w["B"], w["Hkv"], w["G"], w["cap"], w["n_protect"], max_append=w["ctx"], dense=dense)
     gpu.quantize_append(w["k"], w["v"], w["cls"][:, :w["ctx"]].contiguous().to(DEV), w["pos"].to(DEV))
     del w["k"], w["v"]
     torch.cuda.empty_cache()
@@ -234,14 +253,17 @@ def test_b64_ctx32k_timed_step_sampled_rows():
     _evict_lockstep(gpu, o, rows, w["budget"])
     err = _decode_step(w, gpu, o, rows, 1)           # the timed step's work
     assert err <= OUT_ATOL
+    if dense:
+        _assert_dense(gpu)
 
 
-def test_b8_ctx16k_decode_loop_sampled_steps():
+@pytest.mark.parametrize("dense", [False, True], ids=["reuse", "dense"])
+def test_b8_ctx16k_decode_loop_sampled_steps(dense):
     """Batch 8 x 32/8 heads, 16k context, 256 decode steps with eviction to 1638
     every 128 steps; lock-step checks on one row at steps 0, 127, 128, 255."""
     rows = [5]
     w = synth.prefill_inputs("b8_ctx16k_256steps", device=DEV)
-    gpu = TkvCache(w["B"], w["Hkv"], w["G"], w["cap"], w["n_protect"], max_append=w["ctx"])
+    gpu = TkvCache(w["B"], w["Hkv"], w["G"], w["cap"], w["n_protect"], max_append=w["ctx"], dense=dense)
     gpu.quantize_append(w["k"], w["v"], w["cls"][:, :w["ctx"]].contiguous().to(DEV), w["pos"].to(DEV))
     o = oracle_for(gpu, gpu.export_state(rows_streams(gpu, rows)), B=1)
     for step in range(w["steps"]):
