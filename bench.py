@@ -53,6 +53,9 @@ def parse():
     ap.add_argument("--placement", choices=["dense", "reuse"], default="dense",
                     help="record placement: dense (eviction moves kept records together, appends "
                          "go after them) or reuse (records stay put, evicted slots are reused)")
+    ap.add_argument("--attn-kernel", choices=["warp", "tc"], default="warp",
+                    help="decode-attention kernel: warp-tile mma.sync (default) or the tcgen05 "
+                         "tensor-memory kernel (dense placement only)")
     ap.add_argument("--evict-reps", type=int, default=5,
                     help="timed repetitions of the eviction that precedes the timed step")
     ap.add_argument("--ctx", type=int, default=None,
@@ -158,12 +161,13 @@ def packed_bytes(n: np.ndarray) -> int:
 
 
 # ----------------------------------------------------------------------------
-def setup_cache(w, dev, dense, evict_reps, flush):
+def setup_cache(w, dev, dense, evict_reps, flush, attn_kernel=0):
     """Prefill, one scoring step, then the eviction to the budget.  The eviction is
     timed (CUDA events, L2 flushed) over `evict_reps` repetitions, each from a copy
     of the pre-eviction workspace; it is not part of the timed decode step."""
     from reasoning_model_kv_b200 import TkvCache
-    gpu = TkvCache(w["B"], w["Hkv"], w["G"], w["cap"], w["n_protect"], max_append=w["ctx"], dense=dense)
+    gpu = TkvCache(w["B"], w["Hkv"], w["G"], w["cap"], w["n_protect"], max_append=w["ctx"], dense=dense,
+                   attn_kernel=attn_kernel)
     cls = w["cls"][:, :w["ctx"]].contiguous().to(dev)
     gpu.quantize_append(w["k"], w["v"], cls, w["pos"].to(dev))
     k, v, c, p, q = synth.decode_inputs(w, 0, device=dev)        # untimed scoring step
@@ -194,7 +198,8 @@ def run_tkv(args, rank, world, dev):
     w = synth.prefill_inputs(args.workload, seed=rank, device=dev, steps=2, **over)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
-    gpu, evict_ms = setup_cache(w, dev, args.placement == "dense", args.evict_reps, flush)
+    gpu, evict_ms = setup_cache(w, dev, args.placement == "dense", args.evict_reps, flush,
+                                attn_kernel=1 if args.attn_kernel == "tc" else 0)
     del w["k"], w["v"]
     torch.cuda.empty_cache()
     views = gpu.state_views()
@@ -292,7 +297,7 @@ def run_tkv(args, rank, world, dev):
                    "head_dim": 128, "context": w["ctx"], "budget": w["budget"],
                    "bf16_window": w["n_protect"], "p_RET": [w["p_r"], w["p_e"], 1 - w["p_r"] - w["p_e"]],
                    "live_kv_tokens": kv_tokens, "packed_kv_bytes": pk,
-                   "placement": args.placement,
+                   "placement": args.placement, "attn_kernel": args.attn_kernel,
                    "l2": "flushed (write of %d MB) before every timed step" % (flush.numel() >> 20),
                    "parallelism": f"{world} independent replicas" if world > 1 else "single GPU"},
         "hbm_gbs_packed": gbs,

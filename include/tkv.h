@@ -83,6 +83,12 @@ typedef struct {
                             records are contiguous in table order (handle[i] ==
                             i) and decode reads them as whole blocks.  Results
                             are identical in both modes.                      */
+    int32_t attn_kernel; /* decode-attention kernel: 0 = warp-tile kernel
+                            (mma.sync fragments, either placement; the
+                            default); 1 = tensor-memory kernel (tcgen05 MMAs
+                            with accumulators in tensor memory, one thread per
+                            token row; dense placement only).  Both compute the
+                            same result within the stated tolerances.         */
 } tkv_config;
 
 typedef struct tkv_cache tkv_cache;

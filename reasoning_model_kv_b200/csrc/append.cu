@@ -140,9 +140,7 @@ __device__ __forceinline__ void quantize_row(const float (&x)[4], int lane, uint
     }
 }
 
-__device__ __forceinline__ void load_row(const __nv_bfloat16 *src, int lane, float (&x)[4],
-                                         uint2 &raw) {
-    raw = reinterpret_cast<const uint2 *>(src)[lane];
+__device__ __forceinline__ void row_floats(const uint2 &raw, float (&x)[4]) {
     x[0] = __uint_as_float(raw.x << 16);
     x[1] = __uint_as_float(raw.x & 0xffff0000u);
     x[2] = __uint_as_float(raw.y << 16);
@@ -165,25 +163,27 @@ __device__ __forceinline__ void store_bf16_row(const uint2 &raw, int lane, uint8
     }
 }
 
+// Packs one record from this lane's 4 elements of the K and V rows (raw bf16 pairs).
 template <int BITS>
-__device__ __forceinline__ void pack_record(const __nv_bfloat16 *k, const __nv_bfloat16 *v,
-                                            uint8_t *rec, int lane, uint8_t *stage) {
-    float x[4];
-    uint2 raw;
+__device__ __forceinline__ void pack_record(const uint2 &rk, const uint2 &rv, uint8_t *rec, int lane,
+                                            uint8_t *stage) {
     if constexpr (BITS == 16) {
         uint16_t *st16 = reinterpret_cast<uint16_t *>(stage);
-        load_row(k, lane, x, raw);
-        store_bf16_row<false>(raw, lane, rec, st16);
-        load_row(v, lane, x, raw);
-        store_bf16_row<true>(raw, lane, rec + 2 * kD, st16);
+        store_bf16_row<false>(rk, lane, rec, st16);
+        store_bf16_row<true>(rv, lane, rec + 2 * kD, st16);
     } else {
         constexpr int cb = kD * BITS / 8;
         __half *meta = reinterpret_cast<__half *>(rec + 2 * cb);
-        load_row(k, lane, x, raw);
+        float x[4];
+        row_floats(rk, x);
         quantize_row<BITS, false>(x, lane, rec, meta, stage);
-        load_row(v, lane, x, raw);
+        row_floats(rv, x);
         quantize_row<BITS, true>(x, lane, rec + cb, meta + 2 * kNG, stage);
     }
+}
+
+__device__ __forceinline__ int pick4(const int4 &v, int c) {
+    return c == 0 ? v.x : c == 1 ? v.y : c == 2 ? v.z : v.w;
 }
 
 template <bool kSingle>
@@ -196,8 +196,17 @@ __global__ void __launch_bounds__(256) append_pack_kernel(
     if (gw >= d.S * T) return;
     const int s = gw / T, t = gw - s * T;
     const int b = s / d.Hkv;
+    // every independent load first (one round trip): the K/V rows, the token's
+    // position and class, and the stream's counters of all four classes
+    const size_t row = ((size_t)s * T + t) * kD;
+    const uint2 rk = reinterpret_cast<const uint2 *>(k + row)[lane];
+    const uint2 rv = reinterpret_cast<const uint2 *>(v + row)[lane];
     const int32_t p = pos[(size_t)b * T + t];
-    const int c = token_class(d, cls[(size_t)b * T + t], p);
+    const uint8_t craw = cls[(size_t)b * T + t];
+    const int4 n4 = *reinterpret_cast<const int4 *>(d.n + s * 4);
+    const int4 ft4 = *reinterpret_cast<const int4 *>(d.ft + s * 4);
+    const int4 hw4 = *reinterpret_cast<const int4 *>(d.hw + s * 4);
+    const int c = token_class(d, craw, p);
     if (c < 0) {
         if (lane == 0) raise_error(d.err, kErrInvalid, (uint32_t)gw);
         return;
@@ -205,7 +214,7 @@ __global__ void __launch_bounds__(256) append_pack_kernel(
     const int r = kSingle ? 0 : d.rank[(size_t)b * d.max_append + t];
     const int sc = s * 4 + c;
     const int cap = d.cap[c];
-    const int ft = d.ft[sc], hw = d.hw[sc], n = d.n[sc];
+    const int ft = pick4(ft4, c), hw = pick4(hw4, c), n = pick4(n4, c);
     int slot;
     if (r < ft) {
         slot = d.fs[c][(size_t)s * cap + ft - 1 - r];
@@ -223,13 +232,12 @@ __global__ void __launch_bounds__(256) append_pack_kernel(
         d.score[c][e] = 0.0f;
     }
     uint8_t *rec = d.pool[c] + ((size_t)s * cap + slot) * d.rec[c];
-    const size_t row = ((size_t)s * T + t) * kD;
     uint8_t *stage = stage_all + (threadIdx.x >> 5) * 2 * kD;
     switch (c) {
-        case 0: pack_record<16>(k + row, v + row, rec, lane, stage); break;
-        case 1: pack_record<8>(k + row, v + row, rec, lane, stage); break;
-        case 2: pack_record<4>(k + row, v + row, rec, lane, stage); break;
-        default: pack_record<2>(k + row, v + row, rec, lane, stage); break;
+        case 0: pack_record<16>(rk, rv, rec, lane, stage); break;
+        case 1: pack_record<8>(rk, rv, rec, lane, stage); break;
+        case 2: pack_record<4>(rk, rv, rec, lane, stage); break;
+        default: pack_record<2>(rk, rv, rec, lane, stage); break;
     }
     __syncwarp();  // every lane has read the pre-call counters
     if (kSingle && lane == 0) {

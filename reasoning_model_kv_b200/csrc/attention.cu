@@ -40,254 +40,25 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
-#include "tkv_internal.cuh"
+#include "attn_common.cuh"
 
 namespace tkv {
 namespace {
 
-constexpr unsigned kFull = 0xffffffffu;
-constexpr int kWarps = 3;
+using namespace attn;
+
+// Warps per CTA and the minimum resident CTAs per SM the register budget is fitted to.
+#ifndef TKV_ATTN_WARPS
+#define TKV_ATTN_WARPS 4
+#endif
+#ifndef TKV_ATTN_MIN_BLOCKS
+#define TKV_ATTN_MIN_BLOCKS 4
+#endif
+constexpr int kWarps = TKV_ATTN_WARPS;
 constexpr int kThreads = 32 * kWarps;
 constexpr int kStages = 3;
 constexpr int kStageBytes = 16 * 288;   // the largest tile: 16 int8 records (rows unpadded, swizzled)
 constexpr int kRingBytes = kWarps * kStages * kStageBytes;
-constexpr int kMaxCluster = 8;
-constexpr float kRescaleSlack = 8.f;    // log2 units the running max may lag behind
-constexpr float kNoMax = -1e30f;        // reference max before any token: finite, so that
-                                        // exp2(-inf - kNoMax) = 0 and exp2(kNoMax - kNoMax) = 1
-
-// ----------------------------------------------------------------- PTX helpers
-__device__ __forceinline__ uint32_t smem_addr(const void *p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ uint64_t policy_evict_first() {
-    uint64_t p;
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-    return p;
-}
-
-// 16-byte copy that reads only `src_size` bytes (0 or 16) and zero-fills the rest.
-__device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void *src, uint32_t src_size,
-                                                 uint64_t policy) {
-    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;" ::"r"(dst), "l"(src),
-                 "r"(src_size), "l"(policy)
-                 : "memory");
-}
-
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-
-__device__ __forceinline__ void cp_async_wait_2() { asm volatile("cp.async.wait_group 2;" ::: "memory"); }
-
-__device__ __forceinline__ void cp_async_wait_0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-
-// ---- dense placement: one bulk copy per tile, completion tracked by an mbarrier
-__device__ __forceinline__ void mbar_init(uint32_t bar) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar) : "memory");
-}
-
-__device__ __forceinline__ void mbar_init_fence() {
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-
-__device__ __forceinline__ uint32_t mbar_try_wait(uint32_t bar, uint32_t parity) {
-    uint32_t done;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(done)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return done;
-}
-
-// Bounded wait for phase `parity` of the barrier: false after ~1 s without it.
-constexpr long long kWaitCycles = 1ll << 31;
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity))
-        if (clock64() - t0 > kWaitCycles) return false;
-    return true;
-}
-
-__device__ __forceinline__ void bulk_copy(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar,
-                                          uint64_t policy) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, "
-        "[%3], %4;" ::"r"(dst),
-        "l"(src), "r"(bytes), "r"(bar), "l"(policy)
-        : "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ void cluster_sync() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ uint32_t dsmem_addr(const void *p, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
-    return r;
-}
-
-__device__ __forceinline__ float dsmem_ld(uint32_t addr) {
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-    return v;
-}
-
-__device__ __forceinline__ void discard_l2_line(const void *p) {
-    asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
-}
-
-__device__ __forceinline__ float ex2(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-__device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                         uint32_t a3, uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-        "{%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ uint32_t transpose8x8(uint32_t x) {
-    uint32_t y;
-    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
-    return y;
-}
-
-__device__ __forceinline__ uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
-__device__ __forceinline__ __half2 u32_as_h2(uint32_t u) { return *reinterpret_cast<__half2 *>(&u); }
-
-__device__ __forceinline__ uint32_t f32x2_to_f16x2(float lo, float hi) {
-    return h2_as_u32(__floats2half2_rn(lo, hi));
-}
-
-__device__ __forceinline__ int sel4(int c, int a0, int a1, int a2, int a3) {
-    return c == 0 ? a0 : c == 1 ? a1 : c == 2 ? a2 : a3;
-}
-
-// ------------------------------------------------- code pair -> f16x2 operand
-// A 32-bit word of a BITS-bit code block holds 16/BITS dim pairs; pair s has its
-// members at bits BITS*s and BITS*s + 16.  OR-ing the masked word into 0x6400
-// (f16 1024) gives 1024 + m*code in each half (m = 2^(BITS*s') after an optional
-// 8-bit shift); one f16x2 FMA, exact, turns that into the code.
-// 0x64006400 held in a register (opaque to constant folding), so that
-// (w & mask) | magic compiles to a single three-input LOP3.
-__device__ __forceinline__ uint32_t magic_f16() {
-    uint32_t m;
-    asm volatile("mov.b32 %0, 0x64006400;" : "=r"(m));
-    return m;
-}
-
-template <int BITS, int S>
-__device__ __forceinline__ uint32_t code_pair(uint32_t word, uint32_t magic) {
-    if constexpr (BITS == 16) {
-        return f32x2_to_f16x2(__uint_as_float(word << 16), __uint_as_float(word & 0xffff0000u));
-    } else if constexpr (BITS == 8) {
-        const uint32_t x = __byte_perm(word, 0x64646464u, S == 0 ? 0x4240 : 0x4341);
-        return h2_as_u32(__hsub2(u32_as_h2(x), u32_as_h2(0x64006400u)));
-    } else {
-        constexpr int kPerShift = BITS == 4 ? 2 : 4;   // pairs reachable without a shift
-        constexpr int ss = S % kPerShift;
-        const uint32_t w = (S >= kPerShift) ? (word >> 8) : word;
-        constexpr uint32_t mask = ((1u << BITS) - 1u) * 0x00010001u;
-        const uint32_t x = (w & (mask << (BITS * ss))) | magic;
-        if constexpr (ss == 0) {
-            return h2_as_u32(__hsub2(u32_as_h2(x), u32_as_h2(0x64006400u)));
-        } else {
-            // x = 1024 + 2^e * code: multiply by 2^-e, add -1024 * 2^-e (exact in f16)
-            constexpr int e = BITS * ss;   // 2, 4 or 6
-            constexpr uint32_t mul = e == 2 ? 0x34003400u : e == 4 ? 0x2C002C00u : 0x24002400u;
-            constexpr uint32_t add = e == 2 ? 0xDC00DC00u : e == 4 ? 0xD400D400u : 0xCC00CC00u;
-            return h2_as_u32(__hfma2(u32_as_h2(x), u32_as_h2(mul), u32_as_h2(add)));
-        }
-    }
-}
-
-// Pair P (0..15) of a quarter held as BITS words.
-template <int BITS, int P>
-__device__ __forceinline__ uint32_t quarter_pair(const uint32_t (&w)[BITS], uint32_t magic) {
-    constexpr int ppw = 16 / BITS;
-    return code_pair<BITS, P % ppw>(w[P / ppw], magic);
-}
-
-// One row's quarter (4*BITS bytes at byte offset `off` of the record).  Int8 tiles keep
-// rows unpadded (288 bytes) and store odd rows with 16-byte chunks k and k ^ 1
-// swapped, which spreads the two rows a load phase touches over all 32 banks.
-template <int BITS>
-__device__ __forceinline__ void load_quarter(const uint8_t *row, int off, int odd, uint32_t (&w)[BITS]) {
-    if constexpr (BITS == 8) {
-        const uint4 a = *reinterpret_cast<const uint4 *>(row + off + 16 * odd);
-        const uint4 b = *reinterpret_cast<const uint4 *>(row + off + 16 - 16 * odd);
-        w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
-        w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
-        return;
-    }
-    const uint8_t *src = row + off;
-    if constexpr (BITS == 2) {
-        const uint2 v = *reinterpret_cast<const uint2 *>(src);
-        w[0] = v.x; w[1] = v.y;
-    } else {
-#pragma unroll
-        for (int i = 0; i < BITS / 4; ++i) {
-            const uint4 v = reinterpret_cast<const uint4 *>(src)[i];
-            w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
-        }
-    }
-}
-
-// S += K . Q^T over head-dim group GRP (32 dims = 2 k-steps).  Pair p = 4*GRP + 2*hh
-// of a quarter carries k-indices 2tig, 2tig+1 of k-step hh; pair p + 1 carries
-// 2tig+8, 2tig+9.  The group's K scale multiplies the fp32 result and its zero adds
-// zero * sum_group(q).
-template <int BITS, int GRP>
-__device__ __forceinline__ void qk_group(float (&x)[4], const uint32_t (&k0)[BITS],
-                                         const uint32_t (&k1)[BITS], const uint32_t (&qb)[4][2][2],
-                                         const float (&qs)[2][4], const float2 (&km0)[4],
-                                         const float2 (&km1)[4], uint32_t magic) {
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    mma16816(acc, quarter_pair<BITS, 4 * GRP>(k0, magic), quarter_pair<BITS, 4 * GRP>(k1, magic),
-             quarter_pair<BITS, 4 * GRP + 1>(k0, magic), quarter_pair<BITS, 4 * GRP + 1>(k1, magic),
-             qb[GRP][0][0], qb[GRP][0][1]);
-    mma16816(acc, quarter_pair<BITS, 4 * GRP + 2>(k0, magic), quarter_pair<BITS, 4 * GRP + 2>(k1, magic),
-             quarter_pair<BITS, 4 * GRP + 3>(k0, magic), quarter_pair<BITS, 4 * GRP + 3>(k1, magic),
-             qb[GRP][1][0], qb[GRP][1][1]);
-    if constexpr (BITS == 16) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) x[i] += acc[i];
-    } else {
-        // km = (scale, zero) of the group for row g (0) and row g + 8 (1)
-        x[0] = fmaf(km0[GRP].x, acc[0], fmaf(km0[GRP].y, qs[0][GRP], x[0]));
-        x[1] = fmaf(km0[GRP].x, acc[1], fmaf(km0[GRP].y, qs[1][GRP], x[1]));
-        x[2] = fmaf(km1[GRP].x, acc[2], fmaf(km1[GRP].y, qs[0][GRP], x[2]));
-        x[3] = fmaf(km1[GRP].x, acc[3], fmaf(km1[GRP].y, qs[1][GRP], x[3]));
-    }
-}
-
-// (scale, zero) pairs of the 4 groups from half of a record's meta block.
-__device__ __forceinline__ void load_meta(const uint8_t *meta, float2 (&out)[4]) {
-    const uint4 m = *reinterpret_cast<const uint4 *>(meta);   // scale x4 then zero x4 (fp16)
-    const float2 s01 = __half22float2(u32_as_h2(m.x)), s23 = __half22float2(u32_as_h2(m.y));
-    const float2 z01 = __half22float2(u32_as_h2(m.z)), z23 = __half22float2(u32_as_h2(m.w));
-    out[0] = make_float2(s01.x, z01.x);
-    out[1] = make_float2(s01.y, z01.y);
-    out[2] = make_float2(s23.x, z23.x);
-    out[3] = make_float2(s23.y, z23.y);
-}
 
 struct WarpState {
     float m[2], l[2];   // reference max / (lane-partial) sum for heads 2*tig, 2*tig+1
@@ -476,7 +247,7 @@ __device__ __forceinline__ void issue_tile_dense(uint8_t *stage_ptr, uint32_t st
 }
 
 template <int G, bool DENSE>
-__global__ void __launch_bounds__(kThreads, 4) attn_kernel(const __grid_constant__ Dev d,
+__global__ void __launch_bounds__(kThreads, TKV_ATTN_MIN_BLOCKS) attn_kernel(const __grid_constant__ Dev d,
                                                            const __nv_bfloat16 *__restrict__ q,
                                                            float xscale, float *__restrict__ out,
                                                            int C) {
@@ -832,6 +603,7 @@ cudaError_t launch_g(const Dev &d, const void *q, float scale, float *out, long 
 
 cudaError_t launch_attention(const Dev &d, const void *q, float scale, float *out, long long live_ub,
                              cudaStream_t st, int64_t *launches) {
+    if (d.dense && d.attn_kernel == 1) return launch_attention_tc(d, q, scale, out, live_ub, st, launches);
     if (d.dense) {
         switch (d.G) {
             case 1: return launch_g<1, true>(d, q, scale, out, live_ub, st, launches);

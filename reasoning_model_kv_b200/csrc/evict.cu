@@ -115,11 +115,22 @@ __global__ void __launch_bounds__(kThreads) evict_kernel(Dev d, int budget) {
         for (int c = 0; c < 4; ++c) {
             const int32_t *pc = d.pos[c] + (size_t)s * d.cap[c];
             const float *sc = d.score[c] + (size_t)s * d.cap[c];
-            for (int i = threadIdx.x; i < n[c]; i += kThreads) {
-                const int32_t p = pc[i];
-                if (p < d.n_protect) continue;
-                const uint64_t key = entry_key(sc[i], p);
-                if (top_bits(key, 8 * pass) == want) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+            // whole warps iterate together so equal digits can be counted with one
+            // atomic per warp (scores cluster in a few exponents: per-lane atomics on
+            // one bin would serialise)
+            for (int base = 0; base < n[c]; base += kThreads) {
+                const int i = base + threadIdx.x;
+                unsigned digit = 256u;                     // 256: lane adds nothing
+                if (i < n[c]) {
+                    const int32_t p = pc[i];
+                    if (p >= d.n_protect) {
+                        const uint64_t key = entry_key(sc[i], p);
+                        if (top_bits(key, 8 * pass) == want) digit = (unsigned)(key >> shift) & 255u;
+                    }
+                }
+                const unsigned peers = __match_any_sync(kFull, digit);
+                if (digit < 256u && (threadIdx.x & 31) == __ffs(peers) - 1)
+                    atomicAdd(&hist[digit], (unsigned)__popc(peers));
             }
         }
         __syncthreads();

@@ -53,6 +53,8 @@ bool valid_config(const tkv_config *c, std::string *why) {
     if (c->max_append < 1 || c->max_append > (1 << 24)) { *why = "max_append must be in [1, 2^24]"; return false; }
     if ((long long)c->B * c->Hkv > 65535) { *why = "B * Hkv must be <= 65535"; return false; }
     if (c->dense != 0 && c->dense != 1) { *why = "dense must be 0 or 1"; return false; }
+    if (c->attn_kernel != 0 && c->attn_kernel != 1) { *why = "attn_kernel must be 0 or 1"; return false; }
+    if (c->attn_kernel == 1 && c->dense != 1) { *why = "attn_kernel 1 needs dense placement"; return false; }
     for (int i = 0; i < 4; ++i)
         if (c->cap[i] >= (1 << 24)) { *why = "cap[c] must be < 2^24"; return false; }
     return true;
@@ -89,6 +91,7 @@ void make_layout(const tkv_config &c, tkv_layout *lay, tkv::Dev *dev, uint8_t *b
     dev->B = c.B; dev->Hkv = c.Hkv; dev->G = c.G; dev->S = (int)S;
     dev->n_protect = c.n_protect; dev->max_append = c.max_append;
     dev->dense = c.dense;
+    dev->attn_kernel = c.attn_kernel;
     dev->n = reinterpret_cast<int32_t *>(base + lay->n);
     dev->ft = reinterpret_cast<int32_t *>(base + lay->ft);
     dev->hw = reinterpret_cast<int32_t *>(base + lay->hw);

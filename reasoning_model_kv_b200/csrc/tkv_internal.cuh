@@ -22,6 +22,7 @@ __host__ __device__ constexpr int record_bytes(int bits) {
 struct Dev {
     int B, Hkv, G, S, n_protect, max_append;
     int dense;              // 1: live records contiguous in table order (handle[i] == i)
+    int attn_kernel;        // 0: warp-tile (mma.sync) kernel, 1: tensor-memory (tcgen05) kernel
     int cap[4];
     int rec[4];
     int32_t *n, *ft, *hw;   // [S][4]
@@ -49,6 +50,9 @@ cudaError_t launch_append(const Dev &d, const void *k, const void *v, const uint
                           const int32_t *pos, int T, cudaStream_t st, int64_t *launches);
 cudaError_t launch_attention(const Dev &d, const void *q, float scale, float *out,
                              long long live_ub, cudaStream_t st, int64_t *launches);
+// Dense placement: the tcgen05 kernel (attention_tc.cu).
+cudaError_t launch_attention_tc(const Dev &d, const void *q, float scale, float *out, long long live_ub,
+                                cudaStream_t st, int64_t *launches);
 cudaError_t launch_evict(const Dev &d, int budget, cudaStream_t st, int64_t *launches);
 
 }  // namespace tkv

@@ -30,7 +30,8 @@ class TkvConfig(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("Hkv", ctypes.c_int32), ("G", ctypes.c_int32),
                 ("D", ctypes.c_int32), ("group", ctypes.c_int32), ("bits", ctypes.c_int32 * 4),
                 ("n_protect", ctypes.c_int32), ("cap", ctypes.c_int32 * 4),
-                ("max_append", ctypes.c_int32), ("dense", ctypes.c_int32)]
+                ("max_append", ctypes.c_int32), ("dense", ctypes.c_int32),
+                ("attn_kernel", ctypes.c_int32)]
 
 
 class TkvLayout(ctypes.Structure):
@@ -90,7 +91,8 @@ def _check(status: int):
         raise TkvError(status, lib().tkv_last_error_string().decode())
 
 
-def make_config(B, Hkv, G, cap, n_protect, max_append=1, D=128, group=32, dense=False) -> TkvConfig:
+def make_config(B, Hkv, G, cap, n_protect, max_append=1, D=128, group=32, dense=False,
+                attn_kernel=0) -> TkvConfig:
     cfg = TkvConfig()
     cfg.B, cfg.Hkv, cfg.G, cfg.D, cfg.group = B, Hkv, G, D, group
     for i in range(4):
@@ -99,6 +101,7 @@ def make_config(B, Hkv, G, cap, n_protect, max_append=1, D=128, group=32, dense=
     cfg.n_protect = n_protect
     cfg.max_append = max_append
     cfg.dense = int(bool(dense))
+    cfg.attn_kernel = int(attn_kernel)
     return cfg
 
 
@@ -126,9 +129,10 @@ class TkvCache:
     """One layer's compressed KV cache: a device workspace owned by torch plus the
     library's cache object.  Methods mirror the C ABI names."""
 
-    def __init__(self, B, Hkv, G, cap, n_protect, max_append=1, device="cuda", dense=False):
-        self.cfg = make_config(B, Hkv, G, cap, n_protect, max_append, dense=dense)
+    def __init__(self, B, Hkv, G, cap, n_protect, max_append=1, device="cuda", dense=False, attn_kernel=0):
+        self.cfg = make_config(B, Hkv, G, cap, n_protect, max_append, dense=dense, attn_kernel=attn_kernel)
         self.dense = bool(dense)
+        self.attn_kernel = int(attn_kernel)
         self.B, self.Hkv, self.G, self.S = B, Hkv, G, B * Hkv
         self.cap = tuple(int(c) for c in cap)
         self.n_protect, self.max_append = n_protect, max_append

@@ -79,12 +79,19 @@ def np_bits(t: torch.Tensor) -> np.ndarray:
     return bits_of(t)
 
 
-def build_pair(name: str, device="cuda", rows=None, dense=False, **over):
+# Cache modes the parity tests run in: placement and decode-attention kernel.
+MODES = {"reuse": dict(dense=False), "dense": dict(dense=True),
+         "dense_tc": dict(dense=True, attn_kernel=1)}
+
+
+def build_pair(name: str, device="cuda", rows=None, dense=False, attn_kernel=0, **over):
     """Prefill a GPU cache with a workload, and an oracle cache with the same
     inputs for batch rows `rows` (default: all); `dense` selects dense placement
-    on both sides.  Returns (w, gpu, oracle, rows)."""
+    on both sides, `attn_kernel` the GPU's decode-attention kernel.  Returns
+    (w, gpu, oracle, rows)."""
     w = synth.prefill_inputs(name, **over)
-    gpu = TkvCache(w["B"], w["Hkv"], w["G"], w["cap"], w["n_protect"], max_append=w["ctx"], dense=dense)
+    gpu = TkvCache(w["B"], w["Hkv"], w["G"], w["cap"], w["n_protect"], max_append=w["ctx"], dense=dense,
+                   attn_kernel=attn_kernel)
     k, v = w["k"].to(device), w["v"].to(device)
     cls = w["cls"][:, :w["ctx"]].contiguous().to(device)
     pos = w["pos"].to(device)

@@ -13,7 +13,7 @@ import synth
 from oracle import oracle as orc
 from reasoning_model_kv_b200 import TkvCache, TkvError, tkv
 from tests.conftest import gpu_available
-from tests.gpu_harness import (OUT_ATOL, build_pair, compare_states, np_bits, oracle_for,
+from tests.gpu_harness import (MODES, OUT_ATOL, build_pair, compare_states, np_bits, oracle_for,
                                rows_streams, score_error)
 
 pytestmark = [pytest.mark.gpu,
@@ -63,12 +63,13 @@ def _assert_dense(gpu):
 
 
 # ----------------------------------------------------------------------------
-@pytest.mark.parametrize("dense", [False, True], ids=["reuse", "dense"])
-def test_tiny_prefill_decode_evict_reuse(dense):
+@pytest.mark.parametrize("mode", list(MODES))
+def test_tiny_prefill_decode_evict_reuse(mode):
     """2k-token single-layer workload: prefill, decode step, eviction to 512, and
     a second step that reuses evicted slots (dense placement: appends after the
     moved records)."""
-    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", dense=dense)
+    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", **MODES[mode])
+    dense = gpu.dense
     compare_states(gpu.export_state(), o.state, what="prefill")
     _decode_step(w, gpu, o, rows, 0)
     _evict_lockstep(gpu, o, rows, w["budget"])
@@ -112,12 +113,12 @@ def test_kept_sets_free_running_match_up_to_near_ties():
                 assert abs(sc[p] - thr) <= 1e-4 * thr, (p, sc[p], thr)
 
 
-@pytest.mark.parametrize("dense", [False, True], ids=["reuse", "dense"])
+@pytest.mark.parametrize("mode", list(MODES))
 @pytest.mark.parametrize("G,n_protect,outliers", [(1, 4, False), (2, 128, True), (4, 4, True),
                                                   (8, 128, False)])
-def test_gqa_widths_and_windows(G, n_protect, outliers, dense):
+def test_gqa_widths_and_windows(G, n_protect, outliers, mode):
     w, gpu, o, rows = build_pair("tiny_b1_ctx2k", B=2, Hq=2 * G, Hkv=2, ctx=709,
-                                 n_protect=n_protect, outliers=outliers, steps=2, dense=dense)
+                                 n_protect=n_protect, outliers=outliers, steps=2, **MODES[mode])
     compare_states(gpu.export_state(), o.state, what="prefill")
     _decode_step(w, gpu, o, rows, 0)
     _evict_lockstep(gpu, o, rows, 300)
@@ -236,15 +237,16 @@ def test_binding_rejects_wrong_tensors():
 # ----------------------------------------------------------------------------
 # The workload shapes of the decode configurations, lock-step on sampled rows/steps
 # ----------------------------------------------------------------------------
-@pytest.mark.parametrize("dense", [False, True], ids=["reuse", "dense"])
-def test_b64_ctx32k_timed_step_sampled_rows(dense):
+@pytest.mark.parametrize("mode", list(MODES))
+def test_b64_ctx32k_timed_step_sampled_rows(mode):
     """Batch 64 x 32/8 heads, 32k context, K outliers, 5 % budget + 128-token bf16
     window: prefill, scoring step, eviction to 1638, then the timed step
     (append + attention), compared on three sampled batch rows."""
     rows = [0, 37, 63]
     w = synth.prefill_inputs("b64_ctx32k_evict5pct", device=DEV, steps=2)
     w["cls"] = synth.class_ids(0, w["B"], w["ctx"] + 2, w["p_r"], w["p_e"])
-    gpu = TkvCache(w["B"], w["Hkv"], w["G"], w["cap"], w["n_protect"], max_append=w["ctx"], dense=dense)
+    gpu = TkvCache(w["B"], w["Hkv"], w["G"], w["cap"], w["n_protect"], max_append=w["ctx"], **MODES[mode])
+    dense = gpu.dense
     gpu.quantize_append(w["k"], w["v"], w["cls"][:, :w["ctx"]].contiguous().to(DEV), w["pos"].to(DEV))
     del w["k"], w["v"]
     torch.cuda.empty_cache()
@@ -257,13 +259,13 @@ def test_b64_ctx32k_timed_step_sampled_rows(dense):
         _assert_dense(gpu)
 
 
-@pytest.mark.parametrize("dense", [False, True], ids=["reuse", "dense"])
-def test_b8_ctx16k_decode_loop_sampled_steps(dense):
+@pytest.mark.parametrize("mode", list(MODES))
+def test_b8_ctx16k_decode_loop_sampled_steps(mode):
     """Batch 8 x 32/8 heads, 16k context, 256 decode steps with eviction to 1638
     every 128 steps; lock-step checks on one row at steps 0, 127, 128, 255."""
     rows = [5]
     w = synth.prefill_inputs("b8_ctx16k_256steps", device=DEV)
-    gpu = TkvCache(w["B"], w["Hkv"], w["G"], w["cap"], w["n_protect"], max_append=w["ctx"], dense=dense)
+    gpu = TkvCache(w["B"], w["Hkv"], w["G"], w["cap"], w["n_protect"], max_append=w["ctx"], **MODES[mode])
     gpu.quantize_append(w["k"], w["v"], w["cls"][:, :w["ctx"]].contiguous().to(DEV), w["pos"].to(DEV))
     o = oracle_for(gpu, gpu.export_state(rows_streams(gpu, rows)), B=1)
     for step in range(w["steps"]):
