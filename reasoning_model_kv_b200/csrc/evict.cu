@@ -18,6 +18,8 @@
 // so the table compacts in place.  In dense placement (handle[i] == i) the kept
 // records move the same way, from slot i to slot = new index, staged through
 // shared memory in batches.
+#include <climits>
+
 #include "tkv_internal.cuh"
 
 namespace tkv {
@@ -25,6 +27,7 @@ namespace {
 
 constexpr int kThreads = 512;
 constexpr int kMoveBytes = 16384;   // dense placement: records staged per move batch
+constexpr int kPer = 4;             // entries per thread in flight (passes) / per chunk (compaction)
 constexpr int kWarpsE = kThreads / 32;
 constexpr unsigned kFull = 0xffffffffu;
 
@@ -79,38 +82,32 @@ __global__ void __launch_bounds__(kThreads) evict_kernel(Dev d, int budget) {
     const int s = blockIdx.x;
     __shared__ unsigned hist[256];
     __shared__ int scratch[33];
-    __shared__ int move_src[kThreads];                       // dense: source slot per kept entry
+    __shared__ int move_src[kPer * kThreads];                // dense: source slot per kept entry
     __shared__ uint4 move_buf[kMoveBytes / sizeof(uint4)];
     __shared__ unsigned long long sh_prefix;
-    __shared__ int sh_bits, sh_rem, sh_done;
+    __shared__ int sh_bits, sh_rem, sh_done, sh_cand;
 
     int n[4];
 #pragma unroll
     for (int c = 0; c < 4; ++c) n[c] = d.n[s * 4 + c];
 
-    // 1. number of unprotected entries
-    int cnt = 0;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        const int32_t *pc = d.pos[c] + (size_t)s * d.cap[c];
-        for (int i = threadIdx.x; i < n[c]; i += kThreads) cnt += pc[i] >= d.n_protect;
-    }
-    const int cand = block_sum(cnt, scratch);
-    if (cand <= budget) return;
-
-    // 2. radix select of the budget-th largest key (budget == 0: nothing kept)
+    // 1+2. radix select of the budget-th largest key (budget == 0: nothing kept);
+    //      pass 0 also counts the unprotected entries
     if (threadIdx.x == 0) {
         sh_prefix = 0ull;
         sh_bits = 0;
         sh_rem = budget;
         sh_done = budget == 0;
+        sh_cand = 0;
     }
     __syncthreads();
-    for (int pass = 0; pass < 8 && !sh_done; ++pass) {
+    for (int pass = 0; pass < 8; ++pass) {
+        if (pass > 0 && sh_done) break;
         const int shift = 56 - 8 * pass;
         for (int i = threadIdx.x; i < 256; i += kThreads) hist[i] = 0u;
         __syncthreads();
         const uint64_t want = top_bits(sh_prefix, 8 * pass);
+        int cnt = 0;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
             const int32_t *pc = d.pos[c] + (size_t)s * d.cap[c];
@@ -118,32 +115,68 @@ __global__ void __launch_bounds__(kThreads) evict_kernel(Dev d, int budget) {
             // whole warps iterate together so equal digits can be counted with one
             // atomic per warp (scores cluster in a few exponents: per-lane atomics on
             // one bin would serialise)
-            for (int base = 0; base < n[c]; base += kThreads) {
-                const int i = base + threadIdx.x;
-                unsigned digit = 256u;                     // 256: lane adds nothing
-                if (i < n[c]) {
-                    const int32_t p = pc[i];
-                    if (p >= d.n_protect) {
-                        const uint64_t key = entry_key(sc[i], p);
+            for (int base = 0; base < n[c]; base += kPer * kThreads) {
+                int32_t pv[kPer];
+                float sv[kPer];
+#pragma unroll
+                for (int j = 0; j < kPer; ++j) {             // all loads first: kPer in flight
+                    const int i = base + j * kThreads + threadIdx.x;
+                    pv[j] = i < n[c] ? pc[i] : INT_MIN;
+                    sv[j] = i < n[c] ? sc[i] : 0.f;
+                }
+#pragma unroll
+                for (int j = 0; j < kPer; ++j) {
+                    unsigned digit = 256u;                     // 256: lane adds nothing
+                    if (pv[j] >= d.n_protect) {
+                        ++cnt;
+                        const uint64_t key = entry_key(sv[j], pv[j]);
                         if (top_bits(key, 8 * pass) == want) digit = (unsigned)(key >> shift) & 255u;
                     }
+                    const unsigned peers = __match_any_sync(kFull, digit);
+                    if (digit < 256u && (threadIdx.x & 31) == __ffs(peers) - 1)
+                        atomicAdd(&hist[digit], (unsigned)__popc(peers));
                 }
-                const unsigned peers = __match_any_sync(kFull, digit);
-                if (digit < 256u && (threadIdx.x & 31) == __ffs(peers) - 1)
-                    atomicAdd(&hist[digit], (unsigned)__popc(peers));
             }
         }
+        if (pass == 0) {
+            cnt = __reduce_add_sync(kFull, cnt);
+            if ((threadIdx.x & 31) == 0) atomicAdd(&sh_cand, cnt);
+        }
         __syncthreads();
-        if (threadIdx.x == 0) {
-            int acc = 0, dg = 255;
-            for (; dg > 0; --dg) {
-                if (acc + (int)hist[dg] >= sh_rem) break;
-                acc += hist[dg];
+        if (sh_cand <= budget) return;   // nothing to evict (uniform: read after the barrier)
+        if (sh_done) break;              // budget 0: every unprotected entry goes
+        // warp 0 picks the digit: the first bin, from the top, where the count of
+        // keys at or above it reaches the remaining rank (bin 0 if none does)
+        if (threadIdx.x < 32) {
+            const int lane = threadIdx.x;
+            unsigned h[8];
+            int sum = 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                h[j] = hist[255 - 8 * lane - j];
+                sum += (int)h[j];
             }
-            sh_rem -= acc;
-            sh_prefix |= static_cast<unsigned long long>(dg) << shift;
-            sh_bits = 64 - shift;
-            if ((int)hist[dg] == sh_rem) sh_done = 1;
+            int incl = sum;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(kFull, incl, o);
+                if (lane >= o) incl += y;
+            }
+            const int rem = sh_rem;
+            const unsigned hit = __ballot_sync(kFull, incl >= rem);
+            const int owner = hit ? __ffs(hit) - 1 : 31;
+            if (lane == owner) {
+                int acc = incl - sum, j = 0;
+                for (; j < 7; ++j) {
+                    if (acc + (int)h[j] >= rem) break;
+                    acc += (int)h[j];
+                }
+                const int dg = 255 - 8 * lane - j;
+                sh_rem = rem - acc;
+                sh_prefix |= static_cast<unsigned long long>(dg) << shift;
+                sh_bits = 64 - shift;
+                if ((int)h[j] == rem - acc) sh_done = 1;
+            }
         }
         __syncthreads();
     }
@@ -152,7 +185,20 @@ __global__ void __launch_bounds__(kThreads) evict_kernel(Dev d, int budget) {
     const bool keep_none = budget == 0;
 
     // 3. keep flags -> per-class evicted counts (first sweep), then the writes
-    //    (second sweep).  Both sweeps replay the same tie order.
+    //    (second sweep).  Without exact key ties (`done`, or nothing kept) the keep
+    //    flag is a function of the key alone: the first sweep needs one block
+    //    reduction per class and the second one scan per chunk (an evicted entry's
+    //    rank in its class is its index minus the kept entries before it).  With
+    //    ties, both sweeps replay the same tie order with block scans.
+    const bool no_ties = done || keep_none;
+    auto keep_of = [&](int32_t p, float scv, int &tie) -> int {
+        tie = 0;
+        if (p < d.n_protect) return 1;
+        if (keep_none) return 0;
+        const uint64_t tb = top_bits(entry_key(scv, p), nb);
+        tie = tb == pref && !done;
+        return tb > pref || (tb == pref && done);
+    };
     int evicted[4];
     int tie_carry = 0;
 #pragma unroll
@@ -160,21 +206,29 @@ __global__ void __launch_bounds__(kThreads) evict_kernel(Dev d, int budget) {
         const int32_t *pc = d.pos[c] + (size_t)s * d.cap[c];
         const float *sc = d.score[c] + (size_t)s * d.cap[c];
         int ev = 0;
+        if (no_ties) {
+            for (int base = 0; base < n[c]; base += kPer * kThreads) {
+                int32_t pv[kPer];
+                float sv[kPer];
+#pragma unroll
+                for (int j = 0; j < kPer; ++j) {
+                    const int i = base + j * kThreads + threadIdx.x;
+                    pv[j] = i < n[c] ? pc[i] : INT_MIN;
+                    sv[j] = i < n[c] ? sc[i] : 0.f;
+                }
+#pragma unroll
+                for (int j = 0; j < kPer; ++j) {
+                    int tie;
+                    if (pv[j] != INT_MIN) ev += !keep_of(pv[j], sv[j], tie);
+                }
+            }
+            evicted[c] = block_sum(ev, scratch);
+            continue;
+        }
         for (int base = 0; base < n[c]; base += kThreads) {
             const int i = base + threadIdx.x;
             int keep = 1, tie = 0;
-            if (i < n[c]) {
-                const int32_t p = pc[i];
-                if (p >= d.n_protect) {
-                    if (keep_none) {
-                        keep = 0;
-                    } else {
-                        const uint64_t tb = top_bits(entry_key(sc[i], p), nb);
-                        keep = tb > pref || (tb == pref && done);
-                        tie = tb == pref && !done;
-                    }
-                }
-            }
+            if (i < n[c]) keep = keep_of(pc[i], sc[i], tie);
             int ntie;
             const int tr = block_scan(tie, &ntie, scratch) + tie_carry;
             tie_carry += ntie;
@@ -196,42 +250,60 @@ __global__ void __launch_bounds__(kThreads) evict_kernel(Dev d, int budget) {
         const int rec = d.rec[c];
         uint8_t *pool = d.pool[c] + base_e * rec;
         int kept_carry = 0, ev_carry = 0;
-        for (int base = 0; base < n[c]; base += kThreads) {
-            const int i = base + threadIdx.x;
-            int keep = 1, tie = 0;
-            int32_t hd = 0, p = 0;
-            float scv = 0.f;
-            if (i < n[c]) {
-                hd = hc[i];
-                p = pc[i];
-                scv = sc[i];
-                if (p >= d.n_protect) {
-                    if (keep_none) {
-                        keep = 0;
-                    } else {
-                        const uint64_t tb = top_bits(entry_key(scv, p), nb);
-                        keep = tb > pref || (tb == pref && done);
-                        tie = tb == pref && !done;
-                    }
-                }
+        // chunks of kPer * kThreads entries; thread t owns kPer consecutive entries, so
+        // an exclusive block scan of per-thread counts plus a running count inside the
+        // thread gives every entry its rank in table order
+        for (int base = 0; base < n[c]; base += kPer * kThreads) {
+            const int i0 = base + kPer * threadIdx.x;
+            int32_t hd[kPer], pv[kPer];
+            float sv[kPer];
+            int keep[kPer], tie[kPer];
+#pragma unroll
+            for (int j = 0; j < kPer; ++j) {
+                const int i = i0 + j;
+                const bool valid = i < n[c];
+                hd[j] = valid ? hc[i] : 0;
+                pv[j] = valid ? pc[i] : 0;
+                sv[j] = valid ? sc[i] : 0.f;
             }
-            int ntie;
-            const int tr = block_scan(tie, &ntie, scratch) + tie_carry;
-            tie_carry += ntie;
-            if (tie) keep = tr < rem0;
-            const int valid = i < n[c];
-            int nkeep, nev;
-            const int wk = block_scan(valid && keep, &nkeep, scratch) + kept_carry;
-            const int r = block_scan(valid && !keep, &nev, scratch) + ev_carry;
+            int nt = 0, nk = 0, nv = 0;
+#pragma unroll
+            for (int j = 0; j < kPer; ++j) {
+                const bool valid = i0 + j < n[c];
+                keep[j] = valid ? keep_of(pv[j], sv[j], tie[j]) : 0;
+                if (!valid) tie[j] = 0;
+                nt += tie[j];
+                nv += valid;
+            }
+            if (!no_ties) {
+                int ntie;
+                int tr = block_scan(nt, &ntie, scratch) + tie_carry;
+                tie_carry += ntie;
+#pragma unroll
+                for (int j = 0; j < kPer; ++j)
+                    if (tie[j]) keep[j] = tr++ < rem0;
+            }
+#pragma unroll
+            for (int j = 0; j < kPer; ++j) nk += keep[j];
+            int nkeep;
+            int wk = block_scan(nk, &nkeep, scratch) + kept_carry;
+            int er = 0, nev = 0;
+            if (!no_ties) er = block_scan(nv - nk, &nev, scratch) + ev_carry;
+            else nev = min(kPer * kThreads, n[c] - base) - nkeep;
             // block_scan ends with a barrier: the whole chunk has been read
-            if (valid) {
-                if (keep) {
-                    hc[wk] = d.dense ? wk : hd;
-                    pc[wk] = p;
-                    sc[wk] = scv;
+#pragma unroll
+            for (int j = 0; j < kPer; ++j) {
+                const int i = i0 + j;
+                if (i >= n[c]) continue;
+                if (keep[j]) {
+                    hc[wk] = d.dense ? wk : hd[j];
+                    pc[wk] = pv[j];
+                    sc[wk] = sv[j];
                     if (d.dense) move_src[wk - kept_carry] = i;
-                } else if (!d.dense) {
-                    fsc[ft0 + (m - 1 - r)] = hd;
+                    ++wk;
+                } else {
+                    const int r = no_ties ? i - wk : er++;   // evicted entries of this class before i
+                    if (!d.dense) fsc[ft0 + (m - 1 - r)] = hd[j];
                 }
             }
             if (d.dense) {
@@ -260,7 +332,8 @@ __global__ void __launch_bounds__(kThreads) evict_kernel(Dev d, int budget) {
             }
             kept_carry += nkeep;
             ev_carry += nev;
-            __syncthreads();
+            // writes of this chunk go to indices below the next chunk's reads; the
+            // scan scratch and the move staging are protected by their own barriers
         }
         if (threadIdx.x == 0) {
             d.n[s * 4 + c] = n[c] - m;
