@@ -278,36 +278,6 @@ __global__ void __launch_bounds__(kThreads, TKV_ATTN_MIN_BLOCKS) attn_kernel(con
     const int p4 = p3 + (hi3 - lo3 + 15) / 16;
     float *lgs = d.logits + (size_t)s * d.ncap * G;   // this stream's logits, by entry order
 
-    // ---- query operand (B of S = K Q^T): head g, dims 32grp + 8tig + 4hh + 0..3
-    uint32_t qb[4][2][2];
-    float qs[2][4];
-    {
-        float qsg[4];
-        const __nv_bfloat16 *qr = q + ((size_t)b * d.Hkv * G + (size_t)kvh * G + (g < G ? g : 0)) * kD;
-#pragma unroll
-        for (int grp = 0; grp < 4; ++grp) {
-            float sum = 0.f;
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                uint2 raw = make_uint2(0u, 0u);
-                if (g < G) raw = *reinterpret_cast<const uint2 *>(qr + 32 * grp + 8 * tig + 4 * hh);
-                const float f0 = __uint_as_float(raw.x << 16), f1 = __uint_as_float(raw.x & 0xffff0000u);
-                const float f2 = __uint_as_float(raw.y << 16), f3 = __uint_as_float(raw.y & 0xffff0000u);
-                qb[grp][hh][0] = f32x2_to_f16x2(f0, f1);
-                qb[grp][hh][1] = f32x2_to_f16x2(f2, f3);
-                sum += (f0 + f1) + (f2 + f3);
-            }
-            sum += __shfl_xor_sync(kFull, sum, 1);
-            sum += __shfl_xor_sync(kFull, sum, 2);
-            qsg[grp] = sum;                              // sum over group grp of q[head g]
-        }
-#pragma unroll
-        for (int grp = 0; grp < 4; ++grp) {
-            qs[0][grp] = __shfl_sync(kFull, qsg[grp], (2 * tig) * 4);
-            qs[1][grp] = __shfl_sync(kFull, qsg[grp], (2 * tig + 1) * 4);
-        }
-    }
-
     WarpState ws;
     ws.m[0] = ws.m[1] = kNoMax;
     ws.l[0] = ws.l[1] = 0.f;
@@ -397,6 +367,37 @@ __global__ void __launch_bounds__(kThreads, TKV_ATTN_MIN_BLOCKS) attn_kernel(con
         if (d1 >= 0) issue(d1, 1, handle_of(d1));
         if constexpr (!DENSE) cp_async_commit();
     }
+    // ---- query operand (loaded after the first two tiles are in flight)
+    //      B of S = K Q^T: head g, dims 32grp + 8tig + 4hh + 0..3
+    uint32_t qb[4][2][2];
+    float qs[2][4];
+    {
+        float qsg[4];
+        const __nv_bfloat16 *qr = q + ((size_t)b * d.Hkv * G + (size_t)kvh * G + (g < G ? g : 0)) * kD;
+#pragma unroll
+        for (int grp = 0; grp < 4; ++grp) {
+            float sum = 0.f;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                uint2 raw = make_uint2(0u, 0u);
+                if (g < G) raw = *reinterpret_cast<const uint2 *>(qr + 32 * grp + 8 * tig + 4 * hh);
+                const float f0 = __uint_as_float(raw.x << 16), f1 = __uint_as_float(raw.x & 0xffff0000u);
+                const float f2 = __uint_as_float(raw.y << 16), f3 = __uint_as_float(raw.y & 0xffff0000u);
+                qb[grp][hh][0] = f32x2_to_f16x2(f0, f1);
+                qb[grp][hh][1] = f32x2_to_f16x2(f2, f3);
+                sum += (f0 + f1) + (f2 + f3);
+            }
+            sum += __shfl_xor_sync(kFull, sum, 1);
+            sum += __shfl_xor_sync(kFull, sum, 2);
+            qsg[grp] = sum;                              // sum over group grp of q[head g]
+        }
+#pragma unroll
+        for (int grp = 0; grp < 4; ++grp) {
+            qs[0][grp] = __shfl_sync(kFull, qsg[grp], (2 * tig) * 4);
+            qs[1][grp] = __shfl_sync(kFull, qsg[grp], (2 * tig + 1) * 4);
+        }
+    }
+
     int dr0 = tile_of(warp + 2 * kWarps), dr1 = tile_of(warp + 3 * kWarps), dr2 = tile_of(warp + 4 * kWarps);
     int hr0 = handle_of(dr0), hr1 = handle_of(dr1), hr2 = handle_of(dr2);
     int stage = 0;
@@ -533,17 +534,7 @@ __global__ void __launch_bounds__(kThreads, TKV_ATTN_MIN_BLOCKS) attn_kernel(con
 
     // ---- scores of this CTA's tokens: += sum_h exp2(x - M_h) / L_h (none if the stream is empty)
     if (N > 0) {
-        float Mh[kMaxG], Ih[kMaxG];
-#pragma unroll
-        for (int h = 0; h < G; ++h) { Mh[h] = gM[h]; Ih[h] = gInvL[h]; }
-        for (int t = t0 + tid; t < t1; t += kThreads) {
-            const float *xt = lgs + (size_t)t * G;
-            float inc = 0.f;
-#pragma unroll
-            for (int h = 0; h < G; ++h) inc += ex2(xt[h] - Mh[h]) * Ih[h];
-            const int c = (t >= o1) + (t >= o2) + (t >= o3);
-            d.score[c][(size_t)s * d.cap[c] + (t - sel4(c, 0, o1, o2, o3))] += inc;
-        }
+        add_scores<G, kThreads>(d, s, lgs, t0, t1, o1, o2, o3, gM, gInvL, tid);
         __syncthreads();
         const char *base = reinterpret_cast<const char *>(lgs + (size_t)t0 * G);
         const int nlines = (int)(((size_t)(t1 - t0) * G * sizeof(float) + 127) / 128);

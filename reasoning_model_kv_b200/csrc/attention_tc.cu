@@ -568,17 +568,7 @@ __global__ void __launch_bounds__(kTT, 1)
 
     // ---- scores of this CTA's tokens: += sum_h exp2(x - M_h) / L_h
     if (N > 0) {
-        float Mh[kMaxG], Ih[kMaxG];
-#pragma unroll
-        for (int h = 0; h < G; ++h) { Mh[h] = gM[h]; Ih[h] = gInvL[h]; }
-        for (int t = t0 + tid; t < t1; t += kTT) {
-            const float *xt = lgs + (size_t)t * G;
-            float inc = 0.f;
-#pragma unroll
-            for (int h = 0; h < G; ++h) inc += ex2(xt[h] - Mh[h]) * Ih[h];
-            const int c = (t >= o1) + (t >= o2) + (t >= o3);
-            d.score[c][(size_t)s * d.cap[c] + (t - sel4(c, 0, o1, o2, o3))] += inc;
-        }
+        add_scores<G, kTT>(d, s, lgs, t0, t1, o1, o2, o3, gM, gInvL, tid);
         __syncthreads();
         const char *base = reinterpret_cast<const char *>(lgs + (size_t)t0 * G);
         const int nlines = (int)(((size_t)(t1 - t0) * G * sizeof(float) + 127) / 128);

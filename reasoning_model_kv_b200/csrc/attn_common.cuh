@@ -262,5 +262,51 @@ __device__ __forceinline__ void load_meta(const uint8_t *meta, float2 (&out)[4])
     out[3] = make_float2(s23.y, z23.y);
 }
 
+// Scores of this CTA's entries [t0, t1) of stream s: score += sum_h exp2(x_h - M_h) *
+// invL_h, x the step's raw logits (log2 domain, entry order).  Four entries per
+// thread are in flight (every load issued before any use): the score loads come
+// from DRAM and would otherwise serialise one round trip per entry.
+template <int G, int NT>
+__device__ __forceinline__ void add_scores(const Dev &d, int s, const float *lgs, int t0, int t1, int o1, int o2,
+                                           int o3, const float *gM, const float *gInvL, int tid) {
+    float Mh[G], Ih[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) { Mh[h] = gM[h]; Ih[h] = gInvL[h]; }
+    for (int t = t0 + tid; t < t1; t += 4 * NT) {
+        float x[4][G], sv[4];
+        float *sp[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int tt = t + u * NT;
+            sp[u] = nullptr;
+            sv[u] = 0.f;
+            if (tt < t1) {
+                const float *xt = lgs + (size_t)tt * G;
+                if constexpr (G % 4 == 0) {
+#pragma unroll
+                    for (int h = 0; h < G; h += 4) {
+                        const float4 v = *reinterpret_cast<const float4 *>(xt + h);
+                        x[u][h] = v.x; x[u][h + 1] = v.y; x[u][h + 2] = v.z; x[u][h + 3] = v.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int h = 0; h < G; ++h) x[u][h] = xt[h];
+                }
+                const int c = (tt >= o1) + (tt >= o2) + (tt >= o3);
+                sp[u] = d.score[c] + (size_t)s * d.cap[c] + (tt - sel4(c, 0, o1, o2, o3));
+                sv[u] = *sp[u];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (sp[u] == nullptr) continue;
+            float inc = 0.f;
+#pragma unroll
+            for (int h = 0; h < G; ++h) inc += ex2(x[u][h] - Mh[h]) * Ih[h];
+            *sp[u] = sv[u] + inc;
+        }
+    }
+}
+
 }  // namespace attn
 }  // namespace tkv
