@@ -72,16 +72,19 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, "fallback 6.65 TB/s (MEASURED_PEAKS.json absent)"
 
 
-def stored_traffic():
-    """DRAM bytes per attention launch from the committed ncu summary, if it was taken
-    on the current kernel source (null otherwise)."""
+def stored_traffic(placement: str, attn_kernel: str):
+    """DRAM bytes per attention launch from the committed ncu summary of this kernel,
+    if it was taken on the current kernel sources (null otherwise)."""
     p = os.path.join(ROOT, "profiles", "attention_traffic.json")
     if not os.path.exists(p):
         return None
-    d = json.load(open(p))
-    src = os.path.join(ROOT, "reasoning_model_kv_b200", "csrc", "attention.cu")
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    if d.get("attention_cu_sha256_16") != h:
+    d = json.load(open(p)).get(f"placement={placement},attn_kernel={attn_kernel}")
+    if not d:
+        return None
+    m = hashlib.sha256()
+    for f in d["sources"]:
+        m.update(open(os.path.join(ROOT, "reasoning_model_kv_b200", "csrc", f), "rb").read())
+    if d.get("sources_sha256_16") != m.hexdigest()[:16]:
         return None
     return d
 
@@ -314,7 +317,7 @@ def run_tkv(args, rank, world, dev):
         "gpu_launches": int(launches),
         "clocks": cs.summary(),
     }
-    tr = stored_traffic()
+    tr = stored_traffic(args.placement, args.attn_kernel)
     if tr is not None:
         # DRAM bytes of one launch, from the committed capture, scaled to this launch's packed bytes
         res["roofline"]["traffic"] = int(tr["traffic_per_packed_byte"] * pk)
