@@ -191,6 +191,9 @@ __global__ void __launch_bounds__(256) append_pack_kernel(
     Dev d, const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ v,
     const uint8_t *__restrict__ cls, const int32_t *__restrict__ pos, int T) {
     __shared__ __align__(16) uint8_t stage_all[8 * 2 * kD];   // per warp: a row by head dim
+    // let the next kernel in the stream (decode attention) launch now; it waits for
+    // this grid's completion before it reads the cache
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (gw >= d.S * T) return;

@@ -263,6 +263,39 @@ __global__ void __launch_bounds__(kThreads, TKV_ATTN_MIN_BLOCKS) attn_kernel(con
     const int s = blockIdx.y;
     const int b = s / d.Hkv, kvh = s - b * d.Hkv;
 
+    // ---- query operand (B of S = K Q^T; independent of the previous kernel, so it is
+    //      loaded before the dependency wait): head g, dims 32grp + 8tig + 4hh + 0..3
+    uint32_t qb[4][2][2];
+    float qs[2][4];
+    {
+        float qsg[4];
+        const __nv_bfloat16 *qr = q + ((size_t)b * d.Hkv * G + (size_t)kvh * G + (g < G ? g : 0)) * kD;
+#pragma unroll
+        for (int grp = 0; grp < 4; ++grp) {
+            float sum = 0.f;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                uint2 raw = make_uint2(0u, 0u);
+                if (g < G) raw = *reinterpret_cast<const uint2 *>(qr + 32 * grp + 8 * tig + 4 * hh);
+                const float f0 = __uint_as_float(raw.x << 16), f1 = __uint_as_float(raw.x & 0xffff0000u);
+                const float f2 = __uint_as_float(raw.y << 16), f3 = __uint_as_float(raw.y & 0xffff0000u);
+                qb[grp][hh][0] = f32x2_to_f16x2(f0, f1);
+                qb[grp][hh][1] = f32x2_to_f16x2(f2, f3);
+                sum += (f0 + f1) + (f2 + f3);
+            }
+            sum += __shfl_xor_sync(kFull, sum, 1);
+            sum += __shfl_xor_sync(kFull, sum, 2);
+            qsg[grp] = sum;                              // sum over group grp of q[head g]
+        }
+#pragma unroll
+        for (int grp = 0; grp < 4; ++grp) {
+            qs[0][grp] = __shfl_sync(kFull, qsg[grp], (2 * tig) * 4);
+            qs[1][grp] = __shfl_sync(kFull, qsg[grp], (2 * tig + 1) * 4);
+        }
+    }
+
+    grid_dependency_wait();   // the append's counters and records are visible from here
+
     // ---- this CTA's entry range and its tiles (class by class)
     const int n0 = d.n[s * 4 + 0], n1 = d.n[s * 4 + 1], n2 = d.n[s * 4 + 2], n3 = d.n[s * 4 + 3];
     const int o1 = n0, o2 = o1 + n1, o3 = o2 + n2, N = o3 + n3;
@@ -367,37 +400,6 @@ __global__ void __launch_bounds__(kThreads, TKV_ATTN_MIN_BLOCKS) attn_kernel(con
         if (d1 >= 0) issue(d1, 1, handle_of(d1));
         if constexpr (!DENSE) cp_async_commit();
     }
-    // ---- query operand (loaded after the first two tiles are in flight)
-    //      B of S = K Q^T: head g, dims 32grp + 8tig + 4hh + 0..3
-    uint32_t qb[4][2][2];
-    float qs[2][4];
-    {
-        float qsg[4];
-        const __nv_bfloat16 *qr = q + ((size_t)b * d.Hkv * G + (size_t)kvh * G + (g < G ? g : 0)) * kD;
-#pragma unroll
-        for (int grp = 0; grp < 4; ++grp) {
-            float sum = 0.f;
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                uint2 raw = make_uint2(0u, 0u);
-                if (g < G) raw = *reinterpret_cast<const uint2 *>(qr + 32 * grp + 8 * tig + 4 * hh);
-                const float f0 = __uint_as_float(raw.x << 16), f1 = __uint_as_float(raw.x & 0xffff0000u);
-                const float f2 = __uint_as_float(raw.y << 16), f3 = __uint_as_float(raw.y & 0xffff0000u);
-                qb[grp][hh][0] = f32x2_to_f16x2(f0, f1);
-                qb[grp][hh][1] = f32x2_to_f16x2(f2, f3);
-                sum += (f0 + f1) + (f2 + f3);
-            }
-            sum += __shfl_xor_sync(kFull, sum, 1);
-            sum += __shfl_xor_sync(kFull, sum, 2);
-            qsg[grp] = sum;                              // sum over group grp of q[head g]
-        }
-#pragma unroll
-        for (int grp = 0; grp < 4; ++grp) {
-            qs[0][grp] = __shfl_sync(kFull, qsg[grp], (2 * tig) * 4);
-            qs[1][grp] = __shfl_sync(kFull, qsg[grp], (2 * tig + 1) * 4);
-        }
-    }
-
     int dr0 = tile_of(warp + 2 * kWarps), dr1 = tile_of(warp + 3 * kWarps), dr2 = tile_of(warp + 4 * kWarps);
     int hr0 = handle_of(dr0), hr1 = handle_of(dr1), hr2 = handle_of(dr2);
     int stage = 0;
@@ -576,13 +578,15 @@ cudaError_t launch_g(const Dev &d, const void *q, float scale, float *out, long 
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = kRingBytes;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)C;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // overlap the launch with the append
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     const float xscale = scale * 1.4426950408889634f;   // logits in the log2 domain
     cudaError_t e = cudaLaunchKernelEx(&cfg, attn_kernel<G, DENSE>, d, static_cast<const __nv_bfloat16 *>(q),
                                        xscale, out, (int)C);

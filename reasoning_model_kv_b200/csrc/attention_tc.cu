@@ -196,25 +196,6 @@ __global__ void __launch_bounds__(kTT, 1)
     const int b = s / d.Hkv, kvh = s - b * d.Hkv;
     const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
 
-    // ---- this CTA's entry range and its tiles (class by class)
-    const int n0 = d.n[s * 4 + 0], n1 = d.n[s * 4 + 1], n2 = d.n[s * 4 + 2], n3 = d.n[s * 4 + 3];
-    const int o1 = n0, o2 = o1 + n1, o3 = o2 + n2, N = o3 + n3;
-    const int chunk = ((N + C - 1) / C + 31) & ~31;
-    const int t0 = min(N, rank * chunk), t1 = min(N, t0 + chunk);
-    const int lo0 = min(t0, o1), hi0 = min(t1, o1);
-    const int lo1 = min(max(t0 - o1, 0), n1), hi1 = min(max(t1 - o1, 0), n1);
-    const int lo2 = min(max(t0 - o2, 0), n2), hi2 = min(max(t1 - o2, 0), n2);
-    const int lo3 = min(max(t0 - o3, 0), n3), hi3 = min(max(t1 - o3, 0), n3);
-    const int p1 = (hi0 - lo0 + tc_rows(0) - 1) / tc_rows(0);
-    const int p2 = p1 + (hi1 - lo1 + tc_rows(1) - 1) / tc_rows(1);
-    const int p3 = p2 + (hi2 - lo2 + tc_rows(2) - 1) / tc_rows(2);
-    const int P = p3 + (hi3 - lo3 + tc_rows(3) - 1) / tc_rows(3);
-    float *lgs = d.logits + (size_t)s * d.ncap * G;
-    // tile T -> packed descriptor: entry e (bits 0-23), class c (bits 29-30); rows via nr_of
-    auto tile_c = [&](int T) { return (T >= p1) + (T >= p2) + (T >= p3); };
-    auto tile_e = [&](int T, int c) { return sel4(c, lo0, lo1, lo2, lo3) + (T - sel4(c, 0, p1, p2, p3)) * tc_rows(c); };
-    auto tile_nr = [&](int c, int e) { return min(tc_rows(c), sel4(c, hi0, hi1, hi2, hi3) - e); };
-
     // ---- set-up: tensor memory, barriers, the stacked q operand
     if (warp == 0) tmem_alloc(smem_addr(&tmem_base), kTmemCols);
     if (tid == 0) {
@@ -251,6 +232,26 @@ __global__ void __launch_bounds__(kTT, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    grid_dependency_wait();   // the append's counters and records are visible from here
+    // ---- this CTA's entry range and its tiles (class by class)
+    const int n0 = d.n[s * 4 + 0], n1 = d.n[s * 4 + 1], n2 = d.n[s * 4 + 2], n3 = d.n[s * 4 + 3];
+    const int o1 = n0, o2 = o1 + n1, o3 = o2 + n2, N = o3 + n3;
+    const int chunk = ((N + C - 1) / C + 31) & ~31;
+    const int t0 = min(N, rank * chunk), t1 = min(N, t0 + chunk);
+    const int lo0 = min(t0, o1), hi0 = min(t1, o1);
+    const int lo1 = min(max(t0 - o1, 0), n1), hi1 = min(max(t1 - o1, 0), n1);
+    const int lo2 = min(max(t0 - o2, 0), n2), hi2 = min(max(t1 - o2, 0), n2);
+    const int lo3 = min(max(t0 - o3, 0), n3), hi3 = min(max(t1 - o3, 0), n3);
+    const int p1 = (hi0 - lo0 + tc_rows(0) - 1) / tc_rows(0);
+    const int p2 = p1 + (hi1 - lo1 + tc_rows(1) - 1) / tc_rows(1);
+    const int p3 = p2 + (hi2 - lo2 + tc_rows(2) - 1) / tc_rows(2);
+    const int P = p3 + (hi3 - lo3 + tc_rows(3) - 1) / tc_rows(3);
+    float *lgs = d.logits + (size_t)s * d.ncap * G;
+    // tile T -> packed descriptor: entry e (bits 0-23), class c (bits 29-30); rows via nr_of
+    auto tile_c = [&](int T) { return (T >= p1) + (T >= p2) + (T >= p3); };
+    auto tile_e = [&](int T, int c) { return sel4(c, lo0, lo1, lo2, lo3) + (T - sel4(c, 0, p1, p2, p3)) * tc_rows(c); };
+    auto tile_nr = [&](int c, int e) { return min(tc_rows(c), sel4(c, hi0, hi1, hi2, hi3) - e); };
+
     const uint32_t tb = tmem_base;
     const uint64_t pol = policy_evict_first();
     const uint32_t magic = magic_f16();
@@ -608,13 +609,15 @@ cudaError_t launch_tc_g(const Dev &d, const void *q, float scale, float *out, lo
     cfg.blockDim = dim3(kTT, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)C;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // overlap the launch with the append
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     const float xscale = scale * 1.4426950408889634f;   // logits in the log2 domain
     cudaError_t e = cudaLaunchKernelEx(&cfg, attn_tc_kernel<G>, d, static_cast<const __nv_bfloat16 *>(q), xscale,
                                        out, (int)C);
