@@ -283,12 +283,13 @@ def test_b8_ctx16k_decode_loop_sampled_steps(mode):
     assert gpu.poll_error() == tkv.TKV_OK
 
 
-def test_b1_ctx131k_long_decode_sampled_steps():
+@pytest.mark.parametrize("mode", ["reuse", "dense"])
+def test_b1_ctx131k_long_decode_sampled_steps(mode):
     """Batch 1 x 64/8 heads (G = 8), 131k context, transition-heavy segments,
     eviction to 4096 every 64 steps; lock-step at steps 0, 63, 64 and 200."""
     rows = [0]
     w = synth.prefill_inputs("b1_ctx131k_512steps", device=DEV, steps=201)
-    gpu = TkvCache(w["B"], w["Hkv"], w["G"], w["cap"], w["n_protect"], max_append=w["ctx"])
+    gpu = TkvCache(w["B"], w["Hkv"], w["G"], w["cap"], w["n_protect"], max_append=w["ctx"], **MODES[mode])
     gpu.quantize_append(w["k"], w["v"], w["cls"][:, :w["ctx"]].contiguous().to(DEV), w["pos"].to(DEV))
     o = oracle_for(gpu, gpu.export_state(), B=1)
     for step in range(201):
@@ -306,7 +307,8 @@ def test_b1_ctx131k_long_decode_sampled_steps():
     assert gpu.poll_error() == tkv.TKV_OK
 
 
-def test_l32_b32_ctx32k_decode_loop_sampled_layers_and_steps():
+@pytest.mark.parametrize("mode", ["reuse", "dense"])
+def test_l32_b32_ctx32k_decode_loop_sampled_layers_and_steps(mode):
     """32 layers x batch 32 x 32/8 heads, 32k context with K outliers and a 128-token
     bf16 window, 1024 decode steps with eviction to 1638 every 64 steps.  Every layer
     runs every step; lock-step oracle checks on one batch row of layers 0 and 31 at
@@ -318,7 +320,8 @@ def test_l32_b32_ctx32k_decode_loop_sampled_layers_and_steps():
     caches, ws, oracles = [], [], {}
     for layer in range(L):
         w = synth.prefill_inputs(name, layer=layer, device=DEV)
-        cache = TkvCache(w["B"], w["Hkv"], w["G"], w["cap"], w["n_protect"], max_append=w["ctx"])
+        cache = TkvCache(w["B"], w["Hkv"], w["G"], w["cap"], w["n_protect"], max_append=w["ctx"],
+                         **MODES[mode])
         cache.quantize_append(w["k"], w["v"], w["cls"][:, :w["ctx"]].contiguous().to(DEV),
                               w["pos"].to(DEV))
         del w["k"], w["v"]
