@@ -570,10 +570,7 @@ __global__ void __launch_bounds__(kTT, 1)
     // ---- scores of this CTA's tokens: += sum_h exp2(x - M_h) / L_h
     if (N > 0) {
         add_scores<G, kTT>(d, s, lgs, t0, t1, o1, o2, o3, gM, gInvL, tid);
-        __syncthreads();
-        const char *base = reinterpret_cast<const char *>(lgs + (size_t)t0 * G);
-        const int nlines = (int)(((size_t)(t1 - t0) * G * sizeof(float) + 127) / 128);
-        for (int i = tid; i < nlines; i += kTT) discard_l2_line(base + (size_t)i * 128);
+
     }
     if (C > 1) cluster_sync();   // peers may still be reading this CTA's shared memory
 }

@@ -268,47 +268,61 @@ __device__ __forceinline__ void load_meta(const uint8_t *meta, float2 (&out)[4])
 }
 
 // Scores of this CTA's entries [t0, t1) of stream s: score += sum_h exp2(x_h - M_h) *
-// invL_h, x the step's raw logits (log2 domain, entry order).  Four entries per
-// thread are in flight (every load issued before any use): the score loads come
-// from DRAM and would otherwise serialise one round trip per entry.
+// invL_h, x the step's raw logits (log2 domain, entry order, from the L2 scratch).
+// Entry t0 + k*NT + tid belongs to thread tid (coalesced), kPer of them per round
+// with every load issued before any use (one round covers NT*kPer entries).  A
+// warp's 32 consecutive entries fill exactly G whole 128-byte scratch lines (a CTA's
+// range starts on a 32-entry boundary), so once the warp has its logits in registers
+// it drops those lines from L2 without write-back.
 template <int G, int NT>
 __device__ __forceinline__ void add_scores(const Dev &d, int s, const float *lgs, int t0, int t1, int o1, int o2,
                                            int o3, const float *gM, const float *gInvL, int tid) {
+    constexpr int kPer = G >= 8 ? 4 : G >= 4 ? 8 : 16;   // x[kPer][G] fits the registers
+    const int lane = tid & 31;
     float Mh[G], Ih[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) { Mh[h] = gM[h]; Ih[h] = gInvL[h]; }
-    for (int t = t0 + tid; t < t1; t += 4 * NT) {
-        float x[4][G], sv[4];
-        float *sp[4];
+    // score row of class c, indexed by entry (class c's entries start at o_c)
+    float *const r0 = d.score[0] + (size_t)s * d.cap[0], *const r1 = d.score[1] + (size_t)s * d.cap[1] - o1;
+    float *const r2 = d.score[2] + (size_t)s * d.cap[2] - o2, *const r3 = d.score[3] + (size_t)s * d.cap[3] - o3;
+    auto srow = [&](int t) { return t >= o3 ? r3 : t >= o2 ? r2 : t >= o1 ? r1 : r0; };
+    for (int base = t0; base < t1; base += kPer * NT) {
+        float x[kPer][G], sv[kPer];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int tt = t + u * NT;
-            sp[u] = nullptr;
-            sv[u] = 0.f;
-            if (tt < t1) {
-                const float *xt = lgs + (size_t)tt * G;
+        for (int k = 0; k < kPer; ++k) {
+            const int t = base + k * NT + tid;
+            sv[k] = 0.f;
+            if (t < t1) {
+                const float *xt = lgs + (size_t)t * G;
                 if constexpr (G % 4 == 0) {
 #pragma unroll
                     for (int h = 0; h < G; h += 4) {
                         const float4 v = *reinterpret_cast<const float4 *>(xt + h);
-                        x[u][h] = v.x; x[u][h + 1] = v.y; x[u][h + 2] = v.z; x[u][h + 3] = v.w;
+                        x[k][h] = v.x; x[k][h + 1] = v.y; x[k][h + 2] = v.z; x[k][h + 3] = v.w;
                     }
                 } else {
 #pragma unroll
-                    for (int h = 0; h < G; ++h) x[u][h] = xt[h];
+                    for (int h = 0; h < G; ++h) x[k][h] = xt[h];
                 }
-                const int c = (tt >= o1) + (tt >= o2) + (tt >= o3);
-                sp[u] = d.score[c] + (size_t)s * d.cap[c] + (tt - sel4(c, 0, o1, o2, o3));
-                sv[u] = *sp[u];
+                sv[k] = srow(t)[t];
+            }
+        }
+        __syncwarp();   // the warp's logits are in registers
+        if (lane < G) {
+#pragma unroll
+            for (int k = 0; k < kPer; ++k) {
+                const int w0 = base + k * NT + (tid & ~31);   // first entry of this warp's group
+                if (w0 < t1) discard_l2_line(lgs + (size_t)w0 * G + 32 * lane);
             }
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            if (sp[u] == nullptr) continue;
+        for (int k = 0; k < kPer; ++k) {
+            const int t = base + k * NT + tid;
+            if (t >= t1) continue;
             float inc = 0.f;
 #pragma unroll
-            for (int h = 0; h < G; ++h) inc += ex2(x[u][h] - Mh[h]) * Ih[h];
-            *sp[u] = sv[u] + inc;
+            for (int h = 0; h < G; ++h) inc += ex2(x[k][h] - Mh[h]) * Ih[h];
+            srow(t)[t] = sv[k] + inc;
         }
     }
 }
