@@ -122,16 +122,17 @@ __device__ __forceinline__ void tile_compute(const uint8_t *st, int nr, int lane
         if (tig == 0 && v1) lg[g + 8] = x[2];
     }
 
-    // ---- online softmax; heads are columns, so reduce over the 8 row lanes
+    // ---- online softmax.  The reference max moves only when a tile exceeds it by more
+    //      than the slack, so the column maxima (heads are columns: a reduction over the
+    //      8 row lanes) are formed only then; the reference starts at a finite
+    //      sentinel, so p needs no -inf guard
     float t0 = fmaxf(x[0], x[2]), t1 = fmaxf(x[1], x[3]);
-#pragma unroll
-    for (int o = 4; o < 32; o <<= 1) {
-        t0 = fmaxf(t0, __shfl_xor_sync(kFull, t0, o));
-        t1 = fmaxf(t1, __shfl_xor_sync(kFull, t1, o));
-    }
-    // move the reference max only when a tile exceeds it by more than the slack;
-    // the reference starts at a finite sentinel, so p needs no -inf guard
     if (__any_sync(kFull, t0 > ws.m[0] + kRescaleSlack || t1 > ws.m[1] + kRescaleSlack)) {
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+            t0 = fmaxf(t0, __shfl_xor_sync(kFull, t0, o));
+            t1 = fmaxf(t1, __shfl_xor_sync(kFull, t1, o));
+        }
         const float mn0 = fmaxf(ws.m[0], t0), mn1 = fmaxf(ws.m[1], t1);
         const float a0 = ex2(ws.m[0] - mn0), a1 = ex2(ws.m[1] - mn1);
         ws.m[0] = mn0;
