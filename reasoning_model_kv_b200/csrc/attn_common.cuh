@@ -86,17 +86,6 @@ __device__ __forceinline__ void bulk_copy(uint32_t dst, const void *src, uint32_
         : "memory");
 }
 
-// 2-D tiled tensor copy (box of the map) into shared memory, completing on `bar`.
-// x is the byte column (a multiple of 16), y the record row.
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, int x, int y, uint32_t bar,
-                                            uint64_t policy) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint "
-        "[%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(bar), "l"(policy)
-        : "memory");
-}
-
 // Programmatic dependent launch: block until the previous kernel in the stream has
 // completed and its writes are visible (returns at once when launched without the
 // programmatic-serialisation attribute).
