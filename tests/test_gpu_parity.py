@@ -174,8 +174,11 @@ def test_budget_edge_cases(dense):
     assert (g["n"].sum(axis=1) == 17).all()
 
 
-def test_all_scores_equal_keep_lowest_positions():
-    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", ctx=500)
+@pytest.mark.parametrize("ctx", [500, 3000])
+def test_all_scores_equal_keep_lowest_positions(ctx):
+    """Equal scores: every key differs only in its position bits, so the radix
+    select runs through all score digits with every candidate still in play."""
+    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", ctx=ctx)
     views = gpu.state_views()
     for c in range(4):
         views[f"score{c}"].fill_(0.5)
