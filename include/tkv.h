@@ -212,6 +212,15 @@ TKV_API tkv_status tkv_poll_error(tkv_cache *cache, void *stream);
 TKV_API tkv_status tkv_export_state(tkv_cache *cache, void *host_dst, void *stream);
 TKV_API tkv_status tkv_import_state(tkv_cache *cache, const void *host_src, void *stream);
 
+/* Self-test of the bounded device waits; the pages have no counterpart (it checks
+ * this library's failure reporting).  Launches, on `stream`, a one-warp kernel that
+ * waits on a barrier nothing ever arrives on; after limit_cycles SM cycles (1 ..
+ * 2^31) the wait gives up and TKV_ERR_TIMEOUT is latched in the cache's device error
+ * word -- the same path a decode kernel takes when a copy never completes -- and the
+ * next tkv_poll_error reports it.  The cache's state is not touched; the context stays
+ * usable.  Returns TKV_ERR_INVALID for a NULL cache or a limit out of range. */
+TKV_API tkv_status tkv_selftest_wait_timeout(tkv_cache *cache, int64_t limit_cycles, void *stream);
+
 /* Launch counters since tkv_create (kernels this cache has launched). */
 TKV_API int64_t tkv_launch_count(const tkv_cache *cache);
 

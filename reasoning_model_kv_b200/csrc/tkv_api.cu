@@ -253,6 +253,15 @@ tkv_status tkv_import_state(tkv_cache *c, const void *host_src, void *stream) {
     return cuda_status(e, "tkv_import_state");
 }
 
+tkv_status tkv_selftest_wait_timeout(tkv_cache *c, int64_t limit_cycles, void *stream) {
+    if (!c) return fail(TKV_ERR_INVALID, "cache is NULL");
+    if (limit_cycles < 1 || limit_cycles > (1ll << 31))
+        return fail(TKV_ERR_INVALID, "limit_cycles must be in [1, 2^31]");
+    cudaError_t e = tkv::launch_wait_timeout(c->dev, (long long)limit_cycles, static_cast<cudaStream_t>(stream),
+                                             &c->launches);
+    return cuda_status(e, "tkv_selftest_wait_timeout");
+}
+
 int64_t tkv_launch_count(const tkv_cache *c) { return c ? c->launches : 0; }
 
 const char *tkv_last_error_string(void) { return g_last_error.c_str(); }

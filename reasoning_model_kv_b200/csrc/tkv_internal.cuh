@@ -53,6 +53,8 @@ cudaError_t launch_attention(const Dev &d, const void *q, float scale, float *ou
 // Dense placement: the tcgen05 kernel (attention_tc.cu).
 cudaError_t launch_attention_tc(const Dev &d, const void *q, float scale, float *out, long long live_ub,
                                 cudaStream_t st, int64_t *launches);
+// Self-test of the bounded device waits (selftest.cu).
+cudaError_t launch_wait_timeout(const Dev &d, long long limit, cudaStream_t st, int64_t *launches);
 cudaError_t launch_evict(const Dev &d, int budget, cudaStream_t st, int64_t *launches);
 
 }  // namespace tkv

@@ -45,7 +45,8 @@ class TkvLayout(ctypes.Structure):
 
 EXPORTS = ["tkv_workspace_bytes", "tkv_create", "tkv_destroy", "tkv_reset", "tkv_get_layout",
            "tkv_quantize_append", "tkv_quantize_append_noalloc", "tkv_decode_attention", "tkv_evict_compact", "tkv_poll_error",
-           "tkv_export_state", "tkv_import_state", "tkv_launch_count", "tkv_last_error_string"]
+           "tkv_export_state", "tkv_import_state", "tkv_launch_count", "tkv_last_error_string",
+           "tkv_selftest_wait_timeout"]
 
 _lib = None
 
@@ -75,6 +76,8 @@ def lib() -> ctypes.CDLL:
     L.tkv_export_state.argtypes = [vp, vp, vp]
     L.tkv_import_state.argtypes = [vp, vp, vp]
     L.tkv_launch_count.argtypes = [vp]
+    L.tkv_selftest_wait_timeout.argtypes = [vp, ctypes.c_int64, vp]
+    L.tkv_selftest_wait_timeout.restype = ctypes.c_int
     L.tkv_launch_count.restype = ctypes.c_int64
     L.tkv_last_error_string.restype = ctypes.c_char_p
     for name in ("tkv_create", "tkv_destroy", "tkv_reset", "tkv_get_layout", "tkv_quantize_append",
@@ -206,6 +209,11 @@ class TkvCache:
         if st == TKV_ERR_CUDA:
             _check(st)
         return st
+
+    def selftest_wait_timeout(self, limit_cycles: int, stream=None):
+        """Run the bounded-wait self-test (a wait that must give up); the next
+        poll_error() returns TKV_ERR_TIMEOUT."""
+        _check(lib().tkv_selftest_wait_timeout(self._h, int(limit_cycles), _stream(stream)))
 
     def launch_count(self) -> int:
         return lib().tkv_launch_count(self._h)

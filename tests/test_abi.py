@@ -92,5 +92,8 @@ def test_calls_reject_bad_arguments_without_launching():
     assert L.tkv_decode_attention(h, p, 0.1, ctypes.c_void_p((1 << 24) + 4), None) == INV
     assert L.tkv_evict_compact(h, -1, None) == INV
     assert L.tkv_evict_compact(None, 3, None) == INV
+    assert L.tkv_selftest_wait_timeout(None, 1000, None) == INV
+    assert L.tkv_selftest_wait_timeout(h, 0, None) == INV
+    assert L.tkv_selftest_wait_timeout(h, (1 << 31) + 1, None) == INV
     assert L.tkv_launch_count(h) == 0
     assert L.tkv_destroy(h) == 0
