@@ -330,12 +330,19 @@ def run_tkv(args, rank, world, dev):
                    "head_dim": 128, "context": w["ctx"], "budget": w["budget"],
                    "bf16_window": w["n_protect"], "p_RET": [w["p_r"], w["p_e"], 1 - w["p_r"] - w["p_e"]],
                    "live_kv_tokens": kv_tokens, "packed_kv_bytes": pk,
+                   # besides the packed records, the attention call reads and writes each
+                   # live entry's score (8 B), reads q (bf16) and writes out (fp32); reuse
+                   # placement also reads each entry's slot handle (4 B)
+                   "total_bytes_per_step": pk + kv_tokens * (8 + (0 if args.placement == "dense" else 4))
+                   + q.numel() * q.element_size() + out.numel() * out.element_size(),
                    "placement": args.placement, "attn_kernel": args.attn_kernel,
                    "l2": "flushed (write of %d MB) before every timed step" % (flush.numel() >> 20),
                    "parallelism": f"{world} independent replicas" if world > 1 else "single GPU"},
         "hbm_gbs_packed": gbs,
         "frac_of_8tbs": gbs / NOMINAL_HBM_GBS,
         "attention_ms": t_attn,
+        "attention_ms_median": statistics.median(attn_ms),
+        "attention_ms_min": min(attn_ms),
         "attention_timing": "attention call alone on the post-append cache (L2 flushed), CUDA events",
         "append_exposed_ms": t_step - t_attn,
         "evict_ms_untimed_step": evict_ms,
