@@ -34,11 +34,11 @@ BITS = (16, 8, 4, 2)
 def build(force: bool = False) -> Path:
     """Compile the oracle with IEEE fp32 semantics (no contraction, no fast-math)."""
     if force or not LIB.exists() or LIB.stat().st_mtime < SRC.stat().st_mtime:
+        tmp = f"{LIB}.tmp{os.getpid()}"   # per process: concurrent ranks may build at once
         cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fopenmp",
-               "-fPIC", "-shared", "-Wall", "-Wno-unused-function", str(SRC), "-o",
-               str(LIB) + ".tmp", "-lm"]
+               "-fPIC", "-shared", "-Wall", "-Wno-unused-function", str(SRC), "-o", tmp, "-lm"]
         subprocess.check_call(cmd)
-        os.replace(str(LIB) + ".tmp", LIB)
+        os.replace(tmp, LIB)
     return LIB
 
 

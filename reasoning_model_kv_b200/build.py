@@ -32,7 +32,7 @@ def _stale() -> bool:
 def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> Path:
     if not force and not _stale():
         return LIB
-    tmp = str(LIB) + ".tmp"
+    tmp = f"{LIB}.tmp{os.getpid()}"   # per process: concurrent ranks may build at once
     cmd = [NVCC, *FLAGS, *(extra or []), "-I", str(ROOT / "include"), "-I", str(CSRC),
            *[str(CSRC / s) for s in SOURCES], "-o", tmp]
     if verbose:
