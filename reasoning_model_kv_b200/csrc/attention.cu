@@ -5,17 +5,19 @@
 // on the "Back from the Future" page, problem statement).
 //
 // Work decomposition.  Stream s = (b, kv head) is processed by a cluster of C
-// CTAs of 3 warps (grid (C, S), cluster (C, 1, 1)); CTA r takes a contiguous
-// range of the stream's entries (class 0, 1, 2, 3 tables concatenated) and cuts
-// it into class-homogeneous tiles (16 records; 8 for bf16).  Warp w computes
-// tiles w, w+3, w+6, ... with its own online-softmax state.  C is picked on the
-// host so that the whole grid is resident (C = 1 for many streams).
+// CTAs of kWarps (4) warps (grid (C, S), cluster (C, 1, 1)); CTA r takes a
+// contiguous range of the stream's entries (class 0, 1, 2, 3 tables concatenated)
+// and cuts it into class-homogeneous tiles (16 records; 8 for bf16).  Warp w
+// computes tiles w, w+4, w+8, ... with its own online-softmax state, so the warps
+// of a CTA run through the class loops (and their code) together.  C is picked on
+// the host so that the whole grid is resident (C = 1 for many streams).
 //
-// Memory path.  Each warp stages its tiles in a 3-deep shared-memory ring with
-// 16-byte cp.async copies (L2 evict_first), eight lanes per record so every
-// instruction reads whole 128-byte lines; two tiles are in flight while one is
-// computed.  Tile descriptors and the record handles are read three
-// tiles ahead into a small register ring, off the critical path.
+// Memory path.  Each warp stages its tiles in a 3-deep shared-memory ring: with
+// dense placement one bulk copy per tile (the records are contiguous; completion
+// on an mbarrier), otherwise 16-byte cp.async copies, eight lanes per record so
+// every instruction reads whole 128-byte lines.  Both use the L2 evict_first
+// policy; two tiles are in flight while one is computed.  Tile descriptors and the
+// record handles are read three tiles ahead into a small register ring.
 //
 // Math path (tensor cores, mma.sync m16n8k16, f16 x f16 -> f32):
 //   S[t][h] = K[t][:] . Q[h][:]      M = 16 tokens, N = 8 heads (G used), one fp32
