@@ -83,6 +83,11 @@ def lib():
         L.orc_attend.restype = None
         L.orc_evict.argtypes = [ctypes.POINTER(_State), ctypes.c_int]
         L.orc_evict.restype = ctypes.c_int
+        L.orc_evict_segments.argtypes = [ctypes.POINTER(_State)] + [ctypes.c_void_p] * 4 + [ctypes.c_int]
+        L.orc_evict_segments.restype = ctypes.c_int
+        L.orc_tbe_schedule.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                       ctypes.c_void_p]
+        L.orc_tbe_schedule.restype = ctypes.c_int
         L.orc_num_threads.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -138,6 +143,17 @@ def unpack_record(bits: int, rec: np.ndarray, D=128, group=32):
 
 def num_threads() -> int:
     return lib().orc_num_threads()
+
+
+def tbe_schedule(labels, r0: int = 64, t_keep: int = 16) -> np.ndarray:
+    """Retention of each thought segment of one batch row (the last one open) under
+    the annealing schedule; -1 keeps the whole segment."""
+    lb = np.ascontiguousarray(np.asarray(labels, dtype=np.uint8))
+    out = np.zeros(max(len(lb), 1), dtype=np.int32)
+    rc = lib().orc_tbe_schedule(_ptr(lb) if len(lb) else 0, len(lb), int(r0), int(t_keep), _ptr(out))
+    if rc != 0:
+        raise ValueError("invalid schedule arguments")
+    return out[:len(lb)]
 
 
 # ---------------------------------------------------------------- cache model
@@ -223,6 +239,19 @@ class OracleCache:
 
     def evict(self, budget: int) -> int:
         return lib().orc_evict(ctypes.byref(self._st), int(budget))
+
+    def evict_segments(self, seg_start: np.ndarray, seg_label: np.ndarray, seg_keep: np.ndarray,
+                       nseg: np.ndarray) -> int:
+        """Segment-level eviction.  seg_start int32 / seg_label uint8 / seg_keep int32
+        [B, max_seg] (row b: the thought segments of batch row b), nseg int32 [B]."""
+        st_ = np.ascontiguousarray(seg_start, dtype=np.int32)
+        lb = np.ascontiguousarray(seg_label, dtype=np.uint8)
+        kp = np.ascontiguousarray(seg_keep, dtype=np.int32)
+        ns = np.ascontiguousarray(nseg, dtype=np.int32)
+        assert st_.ndim == 2 and st_.shape[0] == self.B and lb.shape == st_.shape == kp.shape
+        assert ns.shape == (self.B,)
+        return lib().orc_evict_segments(ctypes.byref(self._st), _ptr(st_), _ptr(lb), _ptr(kp), _ptr(ns),
+                                        st_.shape[1])
 
     # -- convenience views
     def live(self, s: int, c: int):

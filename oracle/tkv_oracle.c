@@ -28,6 +28,14 @@
  *  - Budgeted top-k eviction ("DYNTS", section 2.3, selection window: keep
  *    the k highest-scoring tokens, evict the rest) followed by a stable
  *    compaction of the block table; evicted slots go to a per-class free stack.
+ *  - Segment-level eviction ("ThinKV", section Metodologia, TBE paragraph: when
+ *    a Transition thought starts, earlier R/E segments are cut down segment by
+ *    segment on an annealing schedule, retention 64, 32, 16, ...; a few
+ *    Transition tokens are always kept).  Reading used here: a completed R/E
+ *    segment followed by k >= 1 Transition segments keeps r0 >> (k - 1) of its
+ *    tokens, a completed T segment followed by another keeps t_keep, the open
+ *    segment and bf16-labelled segments keep everything; inside a segment the
+ *    kept tokens are the first under (score desc, position asc).
  *
  * Floating point: quantisation is done in IEEE fp32 with round-to-nearest-even
  * and no contraction (build with -ffp-contract=off, no fast-math).  The
@@ -431,6 +439,8 @@ static int cand_cmp(const void *pa, const void *pb) {
  * index i to slot i, empties the free stack and sets the next never-used slot
  * to the new entry count: a class's live records stay contiguous, in table
  * order. */
+static void compact_stream(orc_state *st, int s, uint8_t *evict[4]);
+
 int orc_evict(orc_state *st, int budget) {
     if (budget < 0) return ORC_ERR_INVALID;
     const int S = n_streams(st);
@@ -454,44 +464,135 @@ int orc_evict(orc_state *st, int budget) {
             uint8_t *evict[4];
             for (int c = 0; c < 4; ++c) evict[c] = calloc(st->n[s * 4 + c] + 1, 1);
             for (int r = budget; r < nc; ++r) evict[cand[r].c][cand[r].i] = 1;
-            for (int c = 0; c < 4; ++c) {
-                int n = st->n[s * 4 + c];
-                size_t base = (size_t)s * st->cap[c];
-                int m = 0;
-                for (int i = 0; i < n; ++i) m += evict[c][i];
-                int ft0 = st->ft[s * 4 + c];
-                int w = 0, r = 0;
-                size_t rb = (size_t)orc_record_bytes(st->bits[c], st->D, st->group);
-                uint8_t *moved = st->dense ? malloc(rb * (n - m > 0 ? n - m : 1)) : NULL;
-                for (int i = 0; i < n; ++i) {
-                    if (evict[c][i]) {
-                        if (!st->dense) st->fs[c][base + ft0 + (m - 1 - r)] = st->handle[c][base + i];
-                        ++r;
-                    } else {
-                        if (st->dense)
-                            memcpy(moved + (size_t)w * rb, record_ptr(st, s, c, st->handle[c][base + i]), rb);
-                        st->handle[c][base + w] = st->handle[c][base + i];
-                        st->pos[c][base + w] = st->pos[c][base + i];
-                        st->score[c][base + w] = st->score[c][base + i];
-                        ++w;
-                    }
-                }
-                st->n[s * 4 + c] = w;
-                if (st->dense) {
-                    for (int i = 0; i < w; ++i) {
-                        memcpy(record_ptr(st, s, c, i), moved + (size_t)i * rb, rb);
-                        st->handle[c][base + i] = i;
-                    }
-                    st->hw[s * 4 + c] = w;
-                    st->ft[s * 4 + c] = 0;
-                    free(moved);
-                } else {
-                    st->ft[s * 4 + c] = ft0 + m;
-                }
-                free(evict[c]);
-            }
+            compact_stream(st, s, evict);
+            for (int c = 0; c < 4; ++c) free(evict[c]);
         }
         free(cand);
+    }
+    return ORC_OK;
+}
+
+/* Removes the entries flagged in evict[c][i] from every class list of stream s:
+ * each list keeps its surviving entries in their previous order (scores carried
+ * over); the slots of evicted entries are pushed on the class's free stack in
+ * reverse table order, so the earliest evicted entry ends on top and is reused
+ * first.  Dense placement instead moves the record of the entry that ends at
+ * table index i to slot i, empties the free stack and sets the next never-used
+ * slot to the new entry count. */
+static void compact_stream(orc_state *st, int s, uint8_t *evict[4]) {
+    for (int c = 0; c < 4; ++c) {
+        int n = st->n[s * 4 + c];
+        size_t base = (size_t)s * st->cap[c];
+        int m = 0;
+        for (int i = 0; i < n; ++i) m += evict[c][i];
+        int ft0 = st->ft[s * 4 + c];
+        int w = 0, r = 0;
+        size_t rb = (size_t)orc_record_bytes(st->bits[c], st->D, st->group);
+        uint8_t *moved = st->dense ? malloc(rb * (n - m > 0 ? n - m : 1)) : NULL;
+        for (int i = 0; i < n; ++i) {
+            if (evict[c][i]) {
+                if (!st->dense) st->fs[c][base + ft0 + (m - 1 - r)] = st->handle[c][base + i];
+                ++r;
+            } else {
+                if (st->dense)
+                    memcpy(moved + (size_t)w * rb, record_ptr(st, s, c, st->handle[c][base + i]), rb);
+                st->handle[c][base + w] = st->handle[c][base + i];
+                st->pos[c][base + w] = st->pos[c][base + i];
+                st->score[c][base + w] = st->score[c][base + i];
+                ++w;
+            }
+        }
+        st->n[s * 4 + c] = w;
+        if (st->dense) {
+            for (int i = 0; i < w; ++i) {
+                memcpy(record_ptr(st, s, c, i), moved + (size_t)i * rb, rb);
+                st->handle[c][base + i] = i;
+            }
+            st->hw[s * 4 + c] = w;
+            st->ft[s * 4 + c] = 0;
+            free(moved);
+        } else {
+            st->ft[s * 4 + c] = ft0 + m;
+        }
+    }
+}
+
+/* Thought segment of position p: the last j with seg_start[j] <= p, or -1 when p
+ * lies before the first segment (seg_start strictly increasing, nseg of them). */
+static int segment_of(const int32_t *seg_start, int nseg, int32_t p) {
+    int j = -1;
+    for (int k = 0; k < nseg && seg_start[k] <= p; ++k) j = k;
+    return j;
+}
+
+/* Segment-level eviction.  Row b of the segment arrays (stride max_seg) lists the
+ * thought segments of batch row b: segment j starts at seg_start[j] and ends where
+ * segment j + 1 starts (the last one is open), its tokens are stored in class
+ * seg_label[j], and seg_keep[j] is its retention (-1: keep all).  For every stream
+ * (b, kv head): an entry is kept when its position is below n_protect, lies before
+ * the first segment, or its class differs from its segment's label; the other
+ * entries of segment j are ranked by (score desc, position asc, table index asc)
+ * and the first seg_keep[j] of them are kept.  The tables are then compacted as
+ * by orc_evict. */
+int orc_evict_segments(orc_state *st, const int32_t *seg_start, const uint8_t *seg_label,
+                       const int32_t *seg_keep, const int32_t *nseg, int max_seg) {
+    if (max_seg < 0) return ORC_ERR_INVALID;
+    const int S = n_streams(st);
+    for (int s = 0; s < S; ++s) {
+        const int b = s / st->Hkv;
+        const int ns = nseg[b] < 0 ? 0 : (nseg[b] > max_seg ? max_seg : nseg[b]);
+        const int32_t *starts = seg_start + (size_t)b * max_seg;
+        const uint8_t *labels = seg_label + (size_t)b * max_seg;
+        const int32_t *keeps = seg_keep + (size_t)b * max_seg;
+        uint8_t *evict[4];
+        int any = 0;
+        for (int c = 0; c < 4; ++c) evict[c] = calloc(st->n[s * 4 + c] + 1, 1);
+        for (int j = 0; j < ns; ++j) {
+            if (keeps[j] < 0) continue;
+            const int c = labels[j];
+            if (c < 0 || c > 3) continue;
+            const size_t base = (size_t)s * st->cap[c];
+            const int n = st->n[s * 4 + c];
+            cand_t *cand = malloc(sizeof(cand_t) * (n > 0 ? n : 1));
+            int nc = 0;
+            for (int i = 0; i < n; ++i) {
+                const int32_t p = st->pos[c][base + i];
+                if (p < st->n_protect || segment_of(starts, ns, p) != j) continue;
+                cand[nc].skey = score_key(st->score[c][base + i]);
+                cand[nc].pos = p;
+                cand[nc].c = c;
+                cand[nc].i = i;
+                ++nc;
+            }
+            if (nc > keeps[j]) {
+                qsort(cand, nc, sizeof(cand_t), cand_cmp);
+                for (int r = keeps[j]; r < nc; ++r) evict[c][cand[r].i] = 1;
+                any = 1;
+            }
+            free(cand);
+        }
+        if (any) compact_stream(st, s, evict);
+        for (int c = 0; c < 4; ++c) free(evict[c]);
+    }
+    return ORC_OK;
+}
+
+/* Retention of each of the nseg thought segments of one batch row under the
+ * annealing schedule (labels 0 bf16, 1 R, 2 E, 3 T; the last segment is the open
+ * one).  k = number of Transition segments after segment j:
+ *   open segment, bf16 label, or k = 0          -> -1 (keep all);
+ *   R or E segment with k >= 1                   -> r0 >> (k - 1)  (64, 32, 16, ... for r0 = 64);
+ *   T segment with k >= 1                        -> t_keep (the safety net). */
+int orc_tbe_schedule(const uint8_t *label, int nseg, int r0, int t_keep, int32_t *keep) {
+    if (nseg < 0 || r0 < 0 || t_keep < 0) return ORC_ERR_INVALID;
+    for (int j = 0; j < nseg; ++j)
+        if (label[j] > 3) return ORC_ERR_INVALID;
+    for (int j = 0; j < nseg; ++j) {
+        int k = 0;
+        for (int i = j + 1; i < nseg; ++i) k += label[i] == 3;
+        if (j == nseg - 1 || label[j] == 0 || k == 0) keep[j] = -1;
+        else if (label[j] == 3) keep[j] = t_keep;
+        else keep[j] = (k - 1 >= 31) ? 0 : (r0 >> (k - 1));
     }
     return ORC_OK;
 }

@@ -33,6 +33,7 @@ per (layer, kv head) are picked by hash and their K values are multiplied by
 """
 from __future__ import annotations
 
+import numpy as np
 import torch
 
 MASK64 = (1 << 64) - 1
@@ -174,6 +175,32 @@ def class_ids(seed: int, B: int, T: int, p_r: float, p_e: float) -> torch.Tensor
             if t >= T:
                 break
     return out
+
+
+def segment_table(seed: int, B: int, upto: int, p_r: float, p_e: float, b0: int = 0,
+                  max_seg: int | None = None):
+    """Thought segments that have started by position `upto` (inclusive) in batch rows
+    b0 .. b0 + B - 1: (starts int32 [B, max_seg], labels uint8 [B, max_seg],
+    nseg int32 [B]); the last segment of a row is the open one.  Unused slots hold
+    starts past every position and label 0."""
+    rows = []
+    for b in range(b0, b0 + B):
+        labels, lengths = segment_labels(seed, b, upto + 1, p_r, p_e)
+        starts, t = [], 0
+        for ln in lengths:
+            starts.append(t)
+            t += ln
+        rows.append((starts, labels))
+    m = max_seg if max_seg is not None else max(len(r[0]) for r in rows)
+    st = np.full((B, m), np.iinfo(np.int32).max, dtype=np.int32)
+    lb = np.zeros((B, m), dtype=np.uint8)
+    ns = np.zeros(B, dtype=np.int32)
+    for i, (starts, labels) in enumerate(rows):
+        n = min(len(starts), m)
+        st[i, :n] = starts[:n]
+        lb[i, :n] = labels[:n]
+        ns[i] = n
+    return st, lb, ns
 
 
 def positions(B: int, pos0: int, T: int) -> torch.Tensor:
