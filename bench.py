@@ -58,6 +58,10 @@ def parse():
                          "tensor-memory kernel (dense placement only)")
     ap.add_argument("--evict-reps", type=int, default=5,
                     help="timed repetitions of the eviction that precedes the timed step")
+    ap.add_argument("--evict", choices=["topk", "tbe"], default="topk",
+                    help="eviction before the timed step: topk (each stream keeps its budget of "
+                         "highest-scoring tokens) or tbe (segment-level: the annealing schedule "
+                         "over the rows' thought segments, r0 64, t_keep 16)")
     ap.add_argument("--ctx", type=int, default=None,
                     help="prefill context before the eviction (default: the workload's); the "
                          "timed step is the same post-eviction step, with smaller pools")
@@ -164,10 +168,24 @@ def packed_bytes(n: np.ndarray) -> int:
 
 
 # ----------------------------------------------------------------------------
-def setup_cache(w, dev, dense, evict_reps, flush, attn_kernel=0):
-    """Prefill, one scoring step, then the eviction to the budget.  The eviction is
-    timed (CUDA events, L2 flushed) over `evict_reps` repetitions, each from a copy
-    of the pre-eviction workspace; it is not part of the timed decode step."""
+def segment_inputs(w, dev, upto):
+    """The rows' thought segments up to position `upto` and their retention under
+    the library's TBE schedule, as device tensors for tkv_evict_segments."""
+    from reasoning_model_kv_b200 import tkv
+    st, lb, ns = synth.segment_table(w["seed"], w["B"], upto, w["p_r"], w["p_e"], b0=w.get("b0", 0))
+    keep = torch.full(st.shape, -1, dtype=torch.int32)
+    for b in range(w["B"]):
+        n = int(ns[b])
+        keep[b, :n] = torch.tensor(tkv.tkv_tbe_schedule(lb[b, :n].tolist(), 64, 16), dtype=torch.int32)
+    return (torch.from_numpy(st).to(dev), torch.from_numpy(lb).to(dev), keep.to(dev),
+            torch.from_numpy(ns).to(dev))
+
+
+def setup_cache(w, dev, dense, evict_reps, flush, attn_kernel=0, evict="topk"):
+    """Prefill, one scoring step, then the eviction (to the budget, or the TBE
+    schedule at the scoring step's position).  The eviction is timed (CUDA events,
+    L2 flushed) over `evict_reps` repetitions, each from a copy of the pre-eviction
+    workspace; it is not part of the timed decode step."""
     from reasoning_model_kv_b200 import TkvCache
     gpu = TkvCache(w["B"], w["Hkv"], w["G"], w["cap"], w["n_protect"], max_append=w["ctx"], dense=dense,
                    attn_kernel=attn_kernel)
@@ -176,6 +194,7 @@ def setup_cache(w, dev, dense, evict_reps, flush, attn_kernel=0):
     k, v, c, p, q = synth.decode_inputs(w, 0, device=dev)        # untimed scoring step
     gpu.quantize_append(k, v, c, p)
     gpu.decode_attention(q, SCALE)
+    segs = segment_inputs(w, dev, w["ctx"]) if evict == "tbe" else None
     evict_ms = []
     snap = gpu.workspace.clone() if evict_reps > 0 else None
     st = torch.cuda.current_stream()
@@ -185,7 +204,10 @@ def setup_cache(w, dev, dense, evict_reps, flush, attn_kernel=0):
         flush.zero_()
         a, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(st)
-        gpu.evict_compact(w["budget"])
+        if segs is None:
+            gpu.evict_compact(w["budget"])
+        else:
+            gpu.evict_segments(*segs)
         b2.record(st)
         b2.synchronize()
         if i > 0:
@@ -202,7 +224,7 @@ def run_tkv(args, rank, world, dev):
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
     gpu, evict_ms = setup_cache(w, dev, args.placement == "dense", args.evict_reps, flush,
-                                attn_kernel=1 if args.attn_kernel == "tc" else 0)
+                                attn_kernel=1 if args.attn_kernel == "tc" else 0, evict=args.evict)
     del w["k"], w["v"]
     torch.cuda.empty_cache()
     views = gpu.state_views()
@@ -336,6 +358,8 @@ def run_tkv(args, rank, world, dev):
                    "total_bytes_per_step": pk + kv_tokens * (8 + (0 if args.placement == "dense" else 4))
                    + q.numel() * q.element_size() + out.numel() * out.element_size(),
                    "placement": args.placement, "attn_kernel": args.attn_kernel,
+                   "eviction": (f"topk, budget {w['budget']} per stream" if args.evict == "topk"
+                                else "tbe segment schedule at the scoring step (r0 64, t_keep 16)"),
                    "l2": "flushed (write of %d MB) before every timed step" % (flush.numel() >> 20),
                    "parallelism": f"{world} independent replicas" if world > 1 else "single GPU"},
         "hbm_gbs_packed": gbs,

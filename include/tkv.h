@@ -203,6 +203,41 @@ TKV_API tkv_status tkv_decode_attention(tkv_cache *cache, const void *q, float s
  */
 TKV_API tkv_status tkv_evict_compact(tkv_cache *cache, int32_t budget, void *stream);
 
+/* Segment-level eviction ("ThinKV", section Metodologia, TBE paragraph: when a
+ * Transition thought starts, tokens of earlier R/E thought segments are evicted
+ * progressively on an annealing schedule, at the granularity of segments).
+ *
+ * Row b of the segment arrays (row stride max_seg, device memory) describes batch
+ * row b: nseg[b] segments (values outside [0, max_seg] are clamped); segment j
+ * starts at position seg_start[b*max_seg + j] (strictly increasing) and ends where
+ * segment j + 1 starts, the last one is open; its tokens are stored in class
+ * seg_label[...] (0 bf16, 1 R, 2 E, 3 T); seg_keep[...] is its retention (-1 keeps
+ * the segment whole, r >= 0 keeps r tokens).  For every stream (b, kv head) an
+ * entry is kept when its position is below n_protect, lies before the first
+ * segment, or its class differs from its segment's label; the other entries of
+ * segment j are ranked by (score desc, position asc, table index asc) and the
+ * first seg_keep of them are kept.  The tables are then compacted exactly as by
+ * tkv_evict_compact.  Class tables must be ordered by position (appends in
+ * position order guarantee it).  The call uses the decode step's logits scratch
+ * (no other device memory).  Returns TKV_ERR_INVALID for a NULL cache, NULL arrays
+ * (when max_seg > 0), unaligned int32 arrays or max_seg outside [0, 4096];
+ * max_seg == 0 is a no-op. */
+TKV_API tkv_status tkv_evict_segments(tkv_cache *cache, const int32_t *seg_start, const uint8_t *seg_label,
+                                      const int32_t *seg_keep, const int32_t *nseg, int32_t max_seg,
+                                      void *stream);
+
+/* Retention of each of the nseg thought segments of one batch row (labels 0 bf16,
+ * 1 R, 2 E, 3 T, host memory; the last segment is the open one) under the TBE
+ * annealing schedule, written to keep[0..nseg) (host memory).  Reading of the
+ * page: with k the number of Transition segments after segment j, the open
+ * segment, a bf16-labelled segment and any segment with k = 0 keep everything
+ * (-1); a completed R or E segment keeps r0 >> (k - 1) tokens (64, 32, 16, ...
+ * for r0 = 64); a completed T segment with k >= 1 keeps t_keep (the safety net of
+ * Transition tokens).  Host only: no GPU, no cache.  Returns TKV_ERR_INVALID for
+ * NULL arrays (when nseg > 0), nseg < 0, r0 < 0, t_keep < 0 or a label above 3. */
+TKV_API tkv_status tkv_tbe_schedule(const uint8_t *label, int32_t nseg, int32_t r0, int32_t t_keep,
+                                    int32_t *keep);
+
 /* Synchronise `stream`, read and clear the device error word; returns the
  * first device-side status latched since the last poll (TKV_OK if none). */
 TKV_API tkv_status tkv_poll_error(tkv_cache *cache, void *stream);

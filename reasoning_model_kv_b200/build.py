@@ -10,7 +10,7 @@ PKG = Path(__file__).resolve().parent
 ROOT = PKG.parent
 CSRC = PKG / "csrc"
 LIB = PKG / "libtkv.so"
-SOURCES = ["tkv_api.cu", "append.cu", "attention.cu", "attention_tc.cu", "evict.cu", "noalloc.cu", "selftest.cu"]
+SOURCES = ["tkv_api.cu", "append.cu", "attention.cu", "attention_tc.cu", "evict.cu", "noalloc.cu", "selftest.cu", "evict_segments.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 FLAGS = [

@@ -18,65 +18,12 @@
 // so the table compacts in place.  In dense placement (handle[i] == i) the kept
 // records move the same way, from slot i to slot = new index, staged through
 // shared memory in batches.
-#include <climits>
-
-#include "tkv_internal.cuh"
+#include "compact.cuh"
 
 namespace tkv {
 namespace {
 
-constexpr int kThreads = 512;
-constexpr int kMoveBytes = 16384;   // dense placement: records staged per move batch
-constexpr int kPer = 4;             // entries per thread in flight (passes) / per chunk (compaction)
-constexpr int kWarpsE = kThreads / 32;
-constexpr unsigned kFull = 0xffffffffu;
-
-__device__ __forceinline__ uint32_t score_key(float f) {
-    const uint32_t u = __float_as_uint(f);
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-__device__ __forceinline__ uint64_t entry_key(float score, int32_t pos) {
-    const uint32_t p = ~(static_cast<uint32_t>(pos) ^ 0x80000000u);
-    return (static_cast<uint64_t>(score_key(score)) << 32) | p;
-}
-
-__device__ __forceinline__ uint64_t top_bits(uint64_t k, int nbits) {
-    return nbits == 0 ? 0ull : (k >> (64 - nbits));
-}
-
-// Exclusive block scan of v; *total receives the block sum.  scratch: >= 33 ints.
-__device__ __forceinline__ int block_scan(int v, int *total, int *scratch) {
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    int x = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(kFull, x, o);
-        if (lane >= o) x += y;
-    }
-    if (lane == 31) scratch[w] = x;
-    __syncthreads();
-    if (w == 0) {
-        int y = lane < kWarpsE ? scratch[lane] : 0;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int z = __shfl_up_sync(kFull, y, o);
-            if (lane >= o) y += z;
-        }
-        scratch[lane] = y;
-    }
-    __syncthreads();
-    const int pre = (w > 0 ? scratch[w - 1] : 0) + x - v;
-    *total = scratch[kWarpsE - 1];
-    __syncthreads();
-    return pre;
-}
-
-__device__ __forceinline__ int block_sum(int v, int *scratch) {
-    int total;
-    block_scan(v, &total, scratch);
-    return total;
-}
+using namespace evict;
 
 __global__ void __launch_bounds__(kThreads) evict_kernel(Dev d, int budget) {
     const int s = blockIdx.x;
@@ -191,7 +138,7 @@ __global__ void __launch_bounds__(kThreads) evict_kernel(Dev d, int budget) {
     //    rank in its class is its index minus the kept entries before it).  With
     //    ties, both sweeps replay the same tie order with block scans.
     const bool no_ties = done || keep_none;
-    auto keep_of = [&](int32_t p, float scv, int &tie) -> int {
+    auto keep_of = [&](int, int, int32_t p, float scv, int &tie) -> int {
         tie = 0;
         if (p < d.n_protect) return 1;
         if (keep_none) return 0;
@@ -219,7 +166,7 @@ __global__ void __launch_bounds__(kThreads) evict_kernel(Dev d, int budget) {
 #pragma unroll
                 for (int j = 0; j < kPer; ++j) {
                     int tie;
-                    if (pv[j] != INT_MIN) ev += !keep_of(pv[j], sv[j], tie);
+                    if (pv[j] != INT_MIN) ev += !keep_of(c, 0, pv[j], sv[j], tie);
                 }
             }
             evicted[c] = block_sum(ev, scratch);
@@ -228,7 +175,7 @@ __global__ void __launch_bounds__(kThreads) evict_kernel(Dev d, int budget) {
         for (int base = 0; base < n[c]; base += kThreads) {
             const int i = base + threadIdx.x;
             int keep = 1, tie = 0;
-            if (i < n[c]) keep = keep_of(pc[i], sc[i], tie);
+            if (i < n[c]) keep = keep_of(c, i, pc[i], sc[i], tie);
             int ntie;
             const int tr = block_scan(tie, &ntie, scratch) + tie_carry;
             tie_carry += ntie;
@@ -237,114 +184,7 @@ __global__ void __launch_bounds__(kThreads) evict_kernel(Dev d, int budget) {
         }
         evicted[c] = ev;
     }
-    tie_carry = 0;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        const size_t base_e = (size_t)s * d.cap[c];
-        int32_t *hc = d.handle[c] + base_e;
-        int32_t *pc = d.pos[c] + base_e;
-        float *sc = d.score[c] + base_e;
-        int32_t *fsc = d.fs[c] + base_e;
-        const int ft0 = d.ft[s * 4 + c];
-        const int m = evicted[c];
-        const int rec = d.rec[c];
-        uint8_t *pool = d.pool[c] + base_e * rec;
-        int kept_carry = 0, ev_carry = 0;
-        // chunks of kPer * kThreads entries; thread t owns kPer consecutive entries, so
-        // an exclusive block scan of per-thread counts plus a running count inside the
-        // thread gives every entry its rank in table order
-        for (int base = 0; base < n[c]; base += kPer * kThreads) {
-            const int i0 = base + kPer * threadIdx.x;
-            int32_t hd[kPer], pv[kPer];
-            float sv[kPer];
-            int keep[kPer], tie[kPer];
-#pragma unroll
-            for (int j = 0; j < kPer; ++j) {
-                const int i = i0 + j;
-                const bool valid = i < n[c];
-                hd[j] = valid ? hc[i] : 0;
-                pv[j] = valid ? pc[i] : 0;
-                sv[j] = valid ? sc[i] : 0.f;
-            }
-            int nt = 0, nk = 0, nv = 0;
-#pragma unroll
-            for (int j = 0; j < kPer; ++j) {
-                const bool valid = i0 + j < n[c];
-                keep[j] = valid ? keep_of(pv[j], sv[j], tie[j]) : 0;
-                if (!valid) tie[j] = 0;
-                nt += tie[j];
-                nv += valid;
-            }
-            if (!no_ties) {
-                int ntie;
-                int tr = block_scan(nt, &ntie, scratch) + tie_carry;
-                tie_carry += ntie;
-#pragma unroll
-                for (int j = 0; j < kPer; ++j)
-                    if (tie[j]) keep[j] = tr++ < rem0;
-            }
-#pragma unroll
-            for (int j = 0; j < kPer; ++j) nk += keep[j];
-            int nkeep;
-            int wk = block_scan(nk, &nkeep, scratch) + kept_carry;
-            int er = 0, nev = 0;
-            if (!no_ties) er = block_scan(nv - nk, &nev, scratch) + ev_carry;
-            else nev = min(kPer * kThreads, n[c] - base) - nkeep;
-            // block_scan ends with a barrier: the whole chunk has been read
-#pragma unroll
-            for (int j = 0; j < kPer; ++j) {
-                const int i = i0 + j;
-                if (i >= n[c]) continue;
-                if (keep[j]) {
-                    hc[wk] = d.dense ? wk : hd[j];
-                    pc[wk] = pv[j];
-                    sc[wk] = sv[j];
-                    if (d.dense) move_src[wk - kept_carry] = i;
-                    ++wk;
-                } else {
-                    const int r = no_ties ? i - wk : er++;   // evicted entries of this class before i
-                    if (!d.dense) fsc[ft0 + (m - 1 - r)] = hd[j];
-                }
-            }
-            if (d.dense) {
-                // move this chunk's kept records from slot i to slot wk (wk <= i), in
-                // batches staged through shared memory: a batch is read completely before
-                // any of it is written, and later batches only read slots above this one's
-                __syncthreads();
-                const int per_rec = rec / 16;
-                const int batch = kMoveBytes / rec;
-                for (int b0 = 0; b0 < nkeep; b0 += batch) {
-                    const int nb_rec = min(batch, nkeep - b0);
-                    const int pieces = nb_rec * per_rec;
-                    for (int q = threadIdx.x; q < pieces; q += kThreads) {
-                        const int k = q / per_rec, part = q - k * per_rec;
-                        move_buf[k * per_rec + part] =
-                            reinterpret_cast<const uint4 *>(pool + (size_t)move_src[b0 + k] * rec)[part];
-                    }
-                    __syncthreads();
-                    for (int q = threadIdx.x; q < pieces; q += kThreads) {
-                        const int k = q / per_rec, part = q - k * per_rec;
-                        reinterpret_cast<uint4 *>(pool + (size_t)(kept_carry + b0 + k) * rec)[part] =
-                            move_buf[k * per_rec + part];
-                    }
-                    __syncthreads();
-                }
-            }
-            kept_carry += nkeep;
-            ev_carry += nev;
-            // writes of this chunk go to indices below the next chunk's reads; the
-            // scan scratch and the move staging are protected by their own barriers
-        }
-        if (threadIdx.x == 0) {
-            d.n[s * 4 + c] = n[c] - m;
-            if (d.dense) {
-                d.ft[s * 4 + c] = 0;
-                d.hw[s * 4 + c] = n[c] - m;
-            } else {
-                d.ft[s * 4 + c] = ft0 + m;
-            }
-        }
-    }
+    compact_tables(d, s, n, evicted, keep_of, no_ties, rem0, scratch, move_src, move_buf);
 }
 
 }  // namespace

@@ -221,6 +221,37 @@ tkv_status tkv_evict_compact(tkv_cache *c, int32_t budget, void *stream) {
     return cuda_status(e, "tkv_evict_compact");
 }
 
+tkv_status tkv_evict_segments(tkv_cache *c, const int32_t *seg_start, const uint8_t *seg_label,
+                              const int32_t *seg_keep, const int32_t *nseg, int32_t max_seg, void *stream) {
+    if (!c) return fail(TKV_ERR_INVALID, "cache is NULL");
+    if (max_seg < 0 || max_seg > tkv::evict_segments_max())
+        return fail(TKV_ERR_INVALID, "max_seg must be in [0, 4096]");
+    if (max_seg == 0) return TKV_OK;
+    if (!seg_start || !seg_label || !seg_keep || !nseg) return fail(TKV_ERR_INVALID, "NULL segment array");
+    auto a4 = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; };
+    if (!a4(seg_start) || !a4(seg_keep) || !a4(nseg)) return fail(TKV_ERR_INVALID, "int32 arrays must be 4-byte aligned");
+    cudaError_t e = tkv::launch_evict_segments(c->dev, seg_start, seg_label, seg_keep, nseg, max_seg,
+                                               static_cast<cudaStream_t>(stream), &c->launches);
+    return cuda_status(e, "tkv_evict_segments");
+}
+
+tkv_status tkv_tbe_schedule(const uint8_t *label, int32_t nseg, int32_t r0, int32_t t_keep, int32_t *keep) {
+    if (nseg < 0 || r0 < 0 || t_keep < 0) return fail(TKV_ERR_INVALID, "nseg, r0 and t_keep must be >= 0");
+    if (nseg > 0 && (!label || !keep)) return fail(TKV_ERR_INVALID, "NULL array");
+    for (int32_t j = 0; j < nseg; ++j)
+        if (label[j] > 3) return fail(TKV_ERR_INVALID, "label must be 0..3");
+    // one backward sweep: `later` = Transition segments after j
+    int32_t later = 0;
+    for (int32_t j = nseg - 1; j >= 0; --j) {
+        int32_t r = -1;
+        if (j != nseg - 1 && later > 0 && label[j] != 0)
+            r = label[j] == 3 ? t_keep : (later - 1 < 31 ? (r0 >> (later - 1)) : 0);
+        keep[j] = r;
+        later += label[j] == 3;
+    }
+    return TKV_OK;
+}
+
 tkv_status tkv_poll_error(tkv_cache *c, void *stream) {
     if (!c) return fail(TKV_ERR_INVALID, "cache is NULL");
     auto st = static_cast<cudaStream_t>(stream);

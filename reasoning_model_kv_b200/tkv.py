@@ -46,7 +46,7 @@ class TkvLayout(ctypes.Structure):
 EXPORTS = ["tkv_workspace_bytes", "tkv_create", "tkv_destroy", "tkv_reset", "tkv_get_layout",
            "tkv_quantize_append", "tkv_quantize_append_noalloc", "tkv_decode_attention", "tkv_evict_compact", "tkv_poll_error",
            "tkv_export_state", "tkv_import_state", "tkv_launch_count", "tkv_last_error_string",
-           "tkv_selftest_wait_timeout"]
+           "tkv_selftest_wait_timeout", "tkv_evict_segments", "tkv_tbe_schedule"]
 
 _lib = None
 
@@ -78,6 +78,10 @@ def lib() -> ctypes.CDLL:
     L.tkv_launch_count.argtypes = [vp]
     L.tkv_selftest_wait_timeout.argtypes = [vp, ctypes.c_int64, vp]
     L.tkv_selftest_wait_timeout.restype = ctypes.c_int
+    L.tkv_evict_segments.argtypes = [vp, vp, vp, vp, vp, i32, vp]
+    L.tkv_evict_segments.restype = ctypes.c_int
+    L.tkv_tbe_schedule.argtypes = [vp, i32, i32, i32, vp]
+    L.tkv_tbe_schedule.restype = ctypes.c_int
     L.tkv_launch_count.restype = ctypes.c_int64
     L.tkv_last_error_string.restype = ctypes.c_char_p
     for name in ("tkv_create", "tkv_destroy", "tkv_reset", "tkv_get_layout", "tkv_quantize_append",
@@ -199,6 +203,23 @@ class TkvCache:
     def evict_compact(self, budget: int, stream=None):
         _check(lib().tkv_evict_compact(self._h, int(budget), _stream(stream)))
 
+    def evict_segments(self, seg_start: torch.Tensor, seg_label: torch.Tensor, seg_keep: torch.Tensor,
+                       nseg: torch.Tensor, stream=None):
+        """Segment-level eviction: seg_start int32 / seg_label uint8 / seg_keep int32
+        [B, max_seg] and nseg int32 [B], all on the device."""
+        if seg_start.dim() != 2 or seg_start.shape[0] != self.B:
+            raise TkvError(TKV_ERR_INVALID, "seg_start must be [B, max_seg]")
+        shape = tuple(seg_start.shape)
+        for t, name in ((seg_label, "seg_label"), (seg_keep, "seg_keep")):
+            if tuple(t.shape) != shape:
+                raise TkvError(TKV_ERR_INVALID, f"{name} must be [B, max_seg]")
+        if tuple(nseg.shape) != (self.B,):
+            raise TkvError(TKV_ERR_INVALID, "nseg must be [B]")
+        _check(lib().tkv_evict_segments(self._h, _dptr(seg_start, torch.int32, "seg_start"),
+                                        _dptr(seg_label, torch.uint8, "seg_label"),
+                                        _dptr(seg_keep, torch.int32, "seg_keep"),
+                                        _dptr(nseg, torch.int32, "nseg"), shape[1], _stream(stream)))
+
     # -- housekeeping
     def reset(self, stream=None):
         _check(lib().tkv_reset(self._h, _stream(stream)))
@@ -269,3 +290,17 @@ def tkv_decode_attention(cache: TkvCache, q, softmax_scale, out=None, stream=Non
 
 def tkv_evict_compact(cache: TkvCache, budget, stream=None):
     return cache.evict_compact(budget, stream)
+
+
+def tkv_evict_segments(cache: TkvCache, seg_start, seg_label, seg_keep, nseg, stream=None):
+    return cache.evict_segments(seg_start, seg_label, seg_keep, nseg, stream)
+
+
+def tkv_tbe_schedule(labels, r0: int = 64, t_keep: int = 16):
+    """Retention of each thought segment of one batch row (host computation in the
+    library): a list of ints, -1 keeps the segment whole."""
+    lab = (ctypes.c_uint8 * max(len(labels), 1))(*[int(x) for x in labels])
+    out = (ctypes.c_int32 * max(len(labels), 1))()
+    _check(lib().tkv_tbe_schedule(ctypes.addressof(lab), len(labels), int(r0), int(t_keep),
+                                  ctypes.addressof(out)))
+    return [int(out[i]) for i in range(len(labels))]

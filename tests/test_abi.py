@@ -97,3 +97,47 @@ def test_calls_reject_bad_arguments_without_launching():
     assert L.tkv_selftest_wait_timeout(h, (1 << 31) + 1, None) == INV
     assert L.tkv_launch_count(h) == 0
     assert L.tkv_destroy(h) == 0
+
+
+def test_evict_segments_rejects_bad_arguments_without_launching():
+    L = tkv.lib()
+    cfg = _cfg()
+    n = L.tkv_workspace_bytes(ctypes.byref(cfg))
+    h = ctypes.c_void_p()
+    assert L.tkv_create(ctypes.byref(cfg), ctypes.c_void_p(1 << 20), n, ctypes.byref(h)) == 0
+    p = ctypes.c_void_p(1 << 24)
+    INV = tkv.TKV_ERR_INVALID
+    assert L.tkv_evict_segments(None, p, p, p, p, 4, None) == INV
+    assert L.tkv_evict_segments(h, p, p, p, p, -1, None) == INV
+    assert L.tkv_evict_segments(h, p, p, p, p, 4097, None) == INV
+    assert L.tkv_evict_segments(h, None, p, p, p, 4, None) == INV
+    assert L.tkv_evict_segments(h, p, p, p, None, 4, None) == INV
+    assert L.tkv_evict_segments(h, ctypes.c_void_p((1 << 24) + 2), p, p, p, 4, None) == INV
+    assert L.tkv_evict_segments(h, None, None, None, None, 0, None) == tkv.TKV_OK   # no segments: no-op
+    assert L.tkv_launch_count(h) == 0
+    assert L.tkv_destroy(h) == 0
+
+
+def test_tbe_schedule_host_function_matches_the_oracle():
+    """The library's schedule (host code, one backward sweep) against the oracle's
+    (a forward count per segment) on the golden rows and random label sequences."""
+    import numpy as np
+
+    from oracle import oracle as orc
+    from tests.test_oracle_tbe import _golden_rows
+
+    for labels, expected in _golden_rows():
+        assert tkv.tkv_tbe_schedule(labels, 64, 16) == expected
+    rng = np.random.default_rng(11)
+    for _ in range(300):
+        labels = rng.integers(0, 4, size=int(rng.integers(0, 40))).tolist()
+        r0, t_keep = int(rng.integers(0, 200)), int(rng.integers(0, 40))
+        assert tkv.tkv_tbe_schedule(labels, r0, t_keep) == orc.tbe_schedule(labels, r0, t_keep).tolist()
+
+
+def test_tbe_schedule_rejects_bad_arguments():
+    for labels, r0, t_keep in (([1, 4], 64, 16), ([1, 3], -1, 16), ([1, 3], 64, -2)):
+        with pytest.raises(tkv.TkvError):
+            tkv.tkv_tbe_schedule(labels, r0, t_keep)
+    assert tkv.lib().tkv_tbe_schedule(None, -1, 64, 16, None) == tkv.TKV_ERR_INVALID
+    assert tkv.lib().tkv_tbe_schedule(None, 3, 64, 16, None) == tkv.TKV_ERR_INVALID
