@@ -13,7 +13,9 @@
 // is ordered by position, so a segment is one contiguous run).  Then a warp per
 // segment that must shrink ranks the run: every lane counts, for the entries it
 // owns, the run's keys that precede them (keys staged in shared memory 256 at a
-// time); protected entries rank first and add to the retention.  The keep flags
+// time); protected entries rank first and add to the retention.  A retention of
+// 0 needs no ranking, and a small one (about r < n / 2) is taken by r warp
+// arg-max rounds instead (O(r n / 32) rather than O(n^2 / 32)).  The keep flags
 // (a byte per entry, in the step's logits scratch, which the next decode call
 // rewrites anyway) then drive the shared table compaction.
 #include "compact.cuh"
@@ -116,6 +118,55 @@ __global__ void __launch_bounds__(kThreads) tbe_kernel(Dev d, const int32_t *__r
         const int budget = r + __reduce_add_sync(kFull, np);
         if (e - a <= budget) continue;
         shrunk = 1;
+        if (r == 0) {   // only the protected entries stay
+            for (int i = a + lane; i < e; i += 32) flags[cbase[c] + i] = pc[i] < d.n_protect;
+            continue;
+        }
+        const int cnt = e - a, per = (cnt + 31) >> 5;
+        if (cnt <= 32 * kOwn && budget * 64 < cnt * per * 32) {
+            // small retention: pick the first key under (key desc, index asc) budget
+            // times; a warp arg-max per pick
+            uint64_t ok[kOwn];
+            bool sel[kOwn];
+#pragma unroll
+            for (int m = 0; m < kOwn; ++m) {
+                const int idx = a + lane + 32 * m;
+                ok[m] = idx < e ? key_of(idx) : 0ull;
+                sel[m] = idx >= e;   // not a candidate
+            }
+            for (int it = 0; it < budget; ++it) {
+                uint64_t bk = 0ull;
+                int bi = INT_MAX, have = 0;
+#pragma unroll
+                for (int m = 0; m < kOwn; ++m) {
+                    const int idx = a + lane + 32 * m;
+                    if (!sel[m] && (!have || ok[m] > bk || (ok[m] == bk && idx < bi))) {
+                        bk = ok[m];
+                        bi = idx;
+                        have = 1;
+                    }
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    const uint64_t k2 = __shfl_xor_sync(kFull, bk, o);
+                    const int i2 = __shfl_xor_sync(kFull, bi, o), h2 = __shfl_xor_sync(kFull, have, o);
+                    if (h2 && (!have || k2 > bk || (k2 == bk && i2 < bi))) {
+                        bk = k2;
+                        bi = i2;
+                        have = 1;
+                    }
+                }
+#pragma unroll
+                for (int m = 0; m < kOwn; ++m)
+                    if (a + lane + 32 * m == bi) sel[m] = true;
+            }
+#pragma unroll
+            for (int m = 0; m < kOwn; ++m) {
+                const int idx = a + lane + 32 * m;
+                if (idx < e) flags[cbase[c] + idx] = sel[m];
+            }
+            continue;
+        }
         for (int base = a; base < e; base += 32 * kOwn) {
             uint64_t ok[kOwn];
             int rk[kOwn];
