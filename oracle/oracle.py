@@ -88,6 +88,9 @@ def lib():
         L.orc_tbe_schedule.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                        ctypes.c_void_p]
         L.orc_tbe_schedule.restype = ctypes.c_int
+        L.orc_evict_tam.argtypes = [ctypes.POINTER(_State)] + [ctypes.c_void_p] * 3 + [ctypes.c_int, ctypes.c_int,
+                                                                                      ctypes.c_double]
+        L.orc_evict_tam.restype = ctypes.c_int
         L.orc_num_threads.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -252,6 +255,17 @@ class OracleCache:
         assert ns.shape == (self.B,)
         return lib().orc_evict_segments(ctypes.byref(self._st), _ptr(st_), _ptr(lb), _ptr(kp), _ptr(ns),
                                         st_.shape[1])
+
+    def evict_tam(self, seg_start: np.ndarray, seg_label: np.ndarray, nseg: np.ndarray, budget: int,
+                  c: float) -> int:
+        """Thought-aware budgets (t_j proportional to sqrt(w_j) n_j) with pivotal tokens
+        (score >= c * mean) kept; segment arrays as for evict_segments."""
+        st_ = np.ascontiguousarray(seg_start, dtype=np.int32)
+        lb = np.ascontiguousarray(seg_label, dtype=np.uint8)
+        ns = np.ascontiguousarray(nseg, dtype=np.int32)
+        assert st_.ndim == 2 and st_.shape[0] == self.B and lb.shape == st_.shape and ns.shape == (self.B,)
+        return lib().orc_evict_tam(ctypes.byref(self._st), _ptr(st_), _ptr(lb), _ptr(ns), st_.shape[1],
+                                   int(budget), float(c))
 
     # -- convenience views
     def live(self, s: int, c: int):

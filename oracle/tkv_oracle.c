@@ -36,6 +36,12 @@
  *    tokens, a completed T segment followed by another keeps t_keep, the open
  *    segment and bf16-labelled segments keep everything; inside a segment the
  *    kept tokens are the first under (score desc, position asc).
+ *  - Thought-aware budgets with pivotal-token protection ("Compactacao de Cache KV
+ *    Consciente do Pensamento ... (TAM)", sections 2.B-2.C), as a selection policy:
+ *    segment j keeps floor(T' sqrt(w_j) n_j / sum_i sqrt(w_i) n_i) of its tokens
+ *    (w_j = mean accumulated score of its candidates), tokens scoring at least
+ *    c times the stream's mean are kept on top.  The attention-matching refit of
+ *    the kept keys that TAM performs is not specified on the page and not modelled.
  *
  * Floating point: quantisation is done in IEEE fp32 with round-to-nearest-even
  * and no contraction (build with -ffp-contract=off, no fast-math).  The
@@ -573,6 +579,110 @@ int orc_evict_segments(orc_state *st, const int32_t *seg_start, const uint8_t *s
         }
         if (any) compact_stream(st, s, evict);
         for (int c = 0; c < 4; ++c) free(evict[c]);
+    }
+    return ORC_OK;
+}
+
+/* Thought-aware budget allocation with pivotal-token protection (page "Compactacao
+ * de Cache KV Consciente do Pensamento ... (TAM)", sections 2.B and 2.C), as a
+ * selection policy over the accumulated scores.  For every stream (b, kv head), with
+ * the segments of batch row b as in orc_evict_segments (entries before the first
+ * segment, protected and foreign entries kept): the candidates of segment j are its
+ * unprotected entries in its label's class; n_j their number, w_j their mean score;
+ * a candidate is pivotal when its score >= delta = c * (mean score of all candidates
+ * of the stream) and is kept; the rest of the budget, T' = max(0, budget - pivotal),
+ * is split t_j = min(n_j - p_j, floor(T' * (a_j / D) + 1e-9)), a_j = sqrt(w_j) * n_j,
+ * D = sum_i a_i (all in fp64; segments with n_j = 0 get nothing; the 1e-9 absorbs the
+ * rounding of a share that is an exact integer), and segment j keeps its t_j first
+ * non-pivotal candidates under (score desc, position asc, table index asc). */
+int orc_evict_tam(orc_state *st, const int32_t *seg_start, const uint8_t *seg_label, const int32_t *nseg,
+                  int max_seg, int budget, double c) {
+    if (max_seg < 0 || budget < 0 || !(c >= 0.0)) return ORC_ERR_INVALID;
+    const int S = n_streams(st);
+    for (int s = 0; s < S; ++s) {
+        const int b = s / st->Hkv;
+        const int ns = nseg[b] < 0 ? 0 : (nseg[b] > max_seg ? max_seg : nseg[b]);
+        const int32_t *starts = seg_start + (size_t)b * max_seg;
+        const uint8_t *labels = seg_label + (size_t)b * max_seg;
+        if (ns == 0) continue;
+        int *cnt = calloc(ns, sizeof(int)), *piv = calloc(ns, sizeof(int));
+        double *sum = calloc(ns, sizeof(double));
+        /* 1. candidates per segment: count and score sum; the stream's mean */
+        double tot = 0.0;
+        long long ntot = 0;
+        for (int j = 0; j < ns; ++j) {
+            const int c = labels[j];
+            if (c > 3) continue;
+            const size_t base = (size_t)s * st->cap[c];
+            for (int i = 0; i < st->n[s * 4 + c]; ++i) {
+                const int32_t p = st->pos[c][base + i];
+                if (p < st->n_protect || segment_of(starts, ns, p) != j) continue;
+                cnt[j] += 1;
+                sum[j] += (double)st->score[c][base + i];
+            }
+            tot += sum[j];
+            ntot += cnt[j];
+        }
+        if (ntot == 0) { free(cnt); free(piv); free(sum); continue; }
+        const double delta = c * (tot / (double)ntot);
+        /* 2. pivotal candidates */
+        long long P = 0;
+        for (int j = 0; j < ns; ++j) {
+            const int c = labels[j];
+            if (c > 3) continue;
+            const size_t base = (size_t)s * st->cap[c];
+            for (int i = 0; i < st->n[s * 4 + c]; ++i) {
+                const int32_t p = st->pos[c][base + i];
+                if (p < st->n_protect || segment_of(starts, ns, p) != j) continue;
+                if ((double)st->score[c][base + i] >= delta) piv[j] += 1;
+            }
+            P += piv[j];
+        }
+        /* 3. budgets t_j proportional to sqrt(w_j) n_j */
+        const long long Tp = budget > P ? budget - P : 0;
+        double D = 0.0;
+        for (int j = 0; j < ns; ++j)
+            if (cnt[j] > 0) D += sqrt(sum[j] / cnt[j]) * cnt[j];
+        int32_t *keep = malloc(sizeof(int32_t) * ns);
+        for (int j = 0; j < ns; ++j) {
+            long long t = 0;
+            /* share T' a_j / D with a_j = sqrt(w_j) n_j; 1e-9 keeps a share that is an
+             * integer in exact arithmetic from flooring one below it */
+            if (cnt[j] > 0 && D > 0.0) t = (long long)floor((double)Tp * (sqrt(sum[j] / cnt[j]) * cnt[j] / D) + 1e-9);
+            if (t > cnt[j] - piv[j]) t = cnt[j] - piv[j];
+            keep[j] = (int32_t)t;
+        }
+        /* 4. selection: pivotal kept, then the t_j first of the rest */
+        uint8_t *evict[4];
+        int any = 0;
+        for (int k = 0; k < 4; ++k) evict[k] = calloc(st->n[s * 4 + k] + 1, 1);
+        for (int j = 0; j < ns; ++j) {
+            const int c = labels[j];
+            if (c > 3 || cnt[j] == 0) continue;
+            const size_t base = (size_t)s * st->cap[c];
+            const int n = st->n[s * 4 + c];
+            cand_t *cand = malloc(sizeof(cand_t) * (n > 0 ? n : 1));
+            int nc = 0;
+            for (int i = 0; i < n; ++i) {
+                const int32_t p = st->pos[c][base + i];
+                if (p < st->n_protect || segment_of(starts, ns, p) != j) continue;
+                if ((double)st->score[c][base + i] >= delta) continue;   /* pivotal: kept */
+                cand[nc].skey = score_key(st->score[c][base + i]);
+                cand[nc].pos = p;
+                cand[nc].c = c;
+                cand[nc].i = i;
+                ++nc;
+            }
+            if (nc > keep[j]) {
+                qsort(cand, nc, sizeof(cand_t), cand_cmp);
+                for (int r = keep[j]; r < nc; ++r) evict[c][cand[r].i] = 1;
+                any = 1;
+            }
+            free(cand);
+        }
+        if (any) compact_stream(st, s, evict);
+        for (int k = 0; k < 4; ++k) free(evict[k]);
+        free(keep); free(cnt); free(piv); free(sum);
     }
     return ORC_OK;
 }

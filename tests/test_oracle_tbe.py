@@ -198,3 +198,122 @@ def test_no_segments_is_a_no_op():
     assert cache.evict_segments(z, z.astype(np.uint8), z - 1, np.array([0], np.int32)) == 0
     for key in before:
         assert np.array_equal(before[key], cache.state[key])
+
+
+# --------------------------------------------------------------------------
+# thought-aware budgets with pivotal tokens (TAM page, sections 2.B-2.C)
+# --------------------------------------------------------------------------
+def _cache_with_scores(n_tok, cls, scores, n_protect=0, dense=False):
+    cache = orc.OracleCache(1, 1, 1, cap=[n_tok] * 4, n_protect=n_protect, dense=dense)
+    k = synth.normal_bf16(3, 0, synth.TID_K, 1, 1, 0, n_tok, D)
+    pos = np.arange(n_tok, dtype=np.int32).reshape(1, n_tok)
+    assert cache.append(bits_of(k), bits_of(k), cls.reshape(1, n_tok), pos) == 0
+    for c in range(4):
+        n = cache.state["n"][0, c]
+        p = cache.state[f"pos{c}"][0, :n]
+        cache.state[f"score{c}"][0, :n] = scores[p]
+    return cache
+
+
+def test_tam_budgets_follow_sqrt_w_times_n():
+    """Three R segments of 10, 20 and 30 tokens with constant scores 1, 4 and 9
+    (sqrt w = 1, 2, 3): sum sqrt(w) n = 140, so a budget of 70 gives 5, 20 and 45,
+    the last capped at its 30 tokens.  c = 10 puts delta (60) above every score."""
+    n_tok = 60
+    scores = np.array([1.0] * 10 + [4.0] * 20 + [9.0] * 30, np.float32)
+    cache = _cache_with_scores(n_tok, np.full(n_tok, 1, np.uint8), scores)
+    st = np.array([[0, 10, 30]], np.int32)
+    assert cache.evict_tam(st, np.array([[1, 1, 1]], np.uint8), np.array([3], np.int32), 70, 10.0) == 0
+    kept = cache.live(0, 1)[1].tolist()
+    # equal scores inside a segment: the earliest positions stay
+    assert kept == list(range(0, 5)) + list(range(10, 30)) + list(range(30, 60))
+
+
+def test_tam_pivotal_tokens_are_kept_and_leave_the_rest_of_the_budget():
+    """Mean score 1.0 and c = 3: the two tokens scoring 9 are pivotal and kept; the
+    remaining budget 10 - 2 = 8 splits as for scores without them."""
+    n_tok = 40
+    scores = np.full(n_tok, 0.5, np.float32)
+    scores[[7, 33]] = 9.0
+    scores[20:] = 0.5 + np.arange(20, dtype=np.float32) / 1000.0
+    scores[33] = 9.0
+    cache = _cache_with_scores(n_tok, np.full(n_tok, 2, np.uint8), scores)
+    mean = float(scores.astype(np.float64).mean())
+    assert 3 * mean < 9.0 and np.sort(scores)[-3] < 3 * mean   # exactly two pivotal tokens
+    st = np.array([[0, 20]], np.int32)
+    assert cache.evict_tam(st, np.array([[2, 2]], np.uint8), np.array([2], np.int32), 10, 3.0) == 0
+    kept = set(cache.live(0, 2)[1].tolist())
+    assert {7, 33} <= kept
+    # budgets by hand: w over each segment's candidates (pivotal included), T' = 8
+    w0 = scores[:20].astype(np.float64).mean()
+    w1 = scores[20:].astype(np.float64).mean()
+    Dn = np.sqrt(w0) * 20 + np.sqrt(w1) * 20
+    t0 = int(np.floor(8 * (np.sqrt(w0) * 20 / Dn) + 1e-9))
+    t1 = int(np.floor(8 * (np.sqrt(w1) * 20 / Dn) + 1e-9))
+    seg0 = sorted(p for p in kept if p < 20 and p != 7)
+    seg1 = sorted(p for p in kept if p >= 20 and p != 33)
+    assert seg0 == list(range(t0))                               # equal scores: earliest
+    order1 = sorted(range(20, 40), key=lambda p: (-scores[p], p))
+    assert seg1 == sorted([p for p in order1 if p != 33][:t1])
+
+
+@pytest.mark.parametrize("dense", [False, True])
+@pytest.mark.parametrize("trial", range(8))
+def test_tam_one_segment_without_pivotal_equals_token_level_eviction(trial, dense):
+    """One segment holding every candidate and no pivotal token (c huge): its budget
+    is min(n, budget), i.e. the token-level eviction."""
+    rng = np.random.default_rng(900 + trial)
+    n_tok = int(rng.integers(5, 60))
+    n_protect = int(rng.integers(0, 4))
+    c = int(rng.integers(1, 4))
+    a = _cache(rng, n_tok, n_protect, np.full(n_tok, c, np.uint8), list(rng.random(30) + 0.1), dense, Hkv=2)
+    b = orc.OracleCache(1, 2, 1, cap=a.cap, n_protect=n_protect, dense=dense)
+    b.load_state(a.copy_state())
+    r = int(rng.integers(0, n_tok + 2))
+    assert a.evict_tam(np.array([[0]], np.int32), np.array([[c]], np.uint8), np.array([1], np.int32),
+                       r, 1e30) == 0
+    assert b.evict(r) == 0
+    for key in a.state:
+        assert np.array_equal(a.state[key], b.state[key]), key
+
+
+@pytest.mark.parametrize("trial", range(20))
+def test_tam_keeps_pivotal_and_per_segment_top_t(trial):
+    rng, n_tok, n_protect, starts, labels, keeps, cls, pool = _random_case(trial)
+    cache = _cache(rng, n_tok, n_protect, cls, pool)
+    before = cache.copy_state()
+    ns = len(starts)
+    budget, cc = int(rng.integers(0, n_tok)), float(rng.choice([0.5, 1.5, 3.0]))
+    assert cache.evict_tam(starts.reshape(1, ns), labels.reshape(1, ns), np.array([ns], np.int32),
+                           budget, cc) == 0
+    kept = set()
+    for c in range(4):
+        kept |= set(cache.live(0, c)[1].tolist())
+    groups, allc = {}, []
+    for c in range(4):
+        for i in range(before["n"][0, c]):
+            p = int(before[f"pos{c}"][0, i])
+            sc = before[f"score{c}"][0, i]
+            j = _seg_of(starts, p)
+            if p < n_protect or j < 0 or labels[j] != c:
+                assert p in kept
+                continue
+            groups.setdefault(j, []).append((sc, p, c, i))
+            allc.append(float(sc))
+    if not allc:
+        return
+    delta = cc * (sum(np.float64(x) for x in allc) / len(allc))
+    nonpiv_kept = 0
+    for j, ent in groups.items():
+        piv = [e for e in ent if np.float64(e[0]) >= delta]
+        rest = [e for e in ent if np.float64(e[0]) < delta]
+        assert all(e[1] in kept for e in piv)
+        kin = [e for e in rest if e[1] in kept]
+        kout = [e for e in rest if e[1] not in kept]
+        nonpiv_kept += len(kin)
+        for a in kin:
+            for b in kout:
+                assert _order_key(*a) < _order_key(*b)
+    P = sum(1 for x in allc if np.float64(x) >= delta)
+    assert nonpiv_kept <= max(0, budget - P)
+    _check_table_invariants(cache, before)
