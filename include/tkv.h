@@ -226,6 +226,23 @@ TKV_API tkv_status tkv_evict_segments(tkv_cache *cache, const int32_t *seg_start
                                       const int32_t *seg_keep, const int32_t *nseg, int32_t max_seg,
                                       void *stream);
 
+/* Thought-aware segment budgets with pivotal-token protection (page "Compactacao de
+ * Cache KV Consciente do Pensamento para Raciocinio via Correspondencia de Atencao
+ * Adaptativa" (TAM), sections 2.B and 2.C), as a selection policy over the
+ * accumulated scores.  Segment arrays as for tkv_evict_segments (no retention
+ * array).  For every stream: the candidates of segment j are its unprotected
+ * entries in its label's class; w_j is their mean score and n_j their number; a
+ * candidate scoring at least c times the mean score of all the stream's candidates
+ * is pivotal and kept; the remaining budget T' = max(0, budget - pivotal) gives
+ * segment j t_j = min(n_j - pivotal_j, floor(T' * (a_j / D) + 1e-9)) of its other
+ * candidates, a_j = sqrt(w_j) * n_j, D = sum a_j (fp64), chosen as in
+ * tkv_evict_segments; entries outside every segment's candidates are kept.  The
+ * page's attention-matching refit of the kept keys is not performed.  Returns
+ * TKV_ERR_INVALID for a NULL cache or array (when max_seg > 0), unaligned int32
+ * arrays, max_seg outside [0, 4096], budget < 0, or c negative or not finite. */
+TKV_API tkv_status tkv_evict_tam(tkv_cache *cache, const int32_t *seg_start, const uint8_t *seg_label,
+                                 const int32_t *nseg, int32_t max_seg, int32_t budget, double c, void *stream);
+
 /* Retention of each of the nseg thought segments of one batch row (labels 0 bf16,
  * 1 R, 2 E, 3 T, host memory; the last segment is the open one) under the TBE
  * annealing schedule, written to keep[0..nseg) (host memory).  Reading of the

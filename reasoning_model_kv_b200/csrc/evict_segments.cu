@@ -18,6 +18,18 @@
 // arg-max rounds instead (O(r n / 32) rather than O(n^2 / 32)).  The keep flags
 // (a byte per entry, in the step's logits scratch, which the next decode call
 // rewrites anyway) then drive the shared table compaction.
+//
+// The same kernel, instantiated with TAM = true, serves tkv_evict_tam: the
+// thought-aware budget allocation of the TAM page (sections 2.B and 2.C) as a
+// selection policy.  After the first sweep a warp per segment counts the
+// segment's candidates (unprotected entries of its run) and sums their scores
+// (fp64); the block forms the stream's mean, delta = c * mean, the pivotal
+// candidates (score >= delta: kept, ranked first like protected entries) and the
+// budgets t_j = min(n_j - p_j, floor(T' (a_j / D) + 1e-9)) with a_j = sqrt(w_j) n_j,
+// D = sum a_j, T' = max(0, budget - pivotal), which then play the role of the
+// retentions.
+#include <cmath>
+
 #include "compact.cuh"
 
 namespace tkv {
@@ -32,12 +44,17 @@ constexpr int kOwn = 8;         // entries a lane ranks per round (32 * kOwn per
 __host__ __device__ constexpr int seg_table_bytes(int ms) {
     return (17 * ms + 15) & ~15;   // starts, keep, lo, hi (int32) and label (uint8) per segment
 }
+__host__ __device__ constexpr int tam_table_bytes(int ms) {
+    return 16 * ms;                // score sum (fp64), candidates and pivotal (int32) per segment
+}
 constexpr int kUnionBytes = kWarpsE * kStage * 8 > kMoveBytes ? kWarpsE * kStage * 8 : kMoveBytes;
 
+template <bool TAM>
 __global__ void __launch_bounds__(kThreads) tbe_kernel(Dev d, const int32_t *__restrict__ seg_start,
                                                        const uint8_t *__restrict__ seg_label,
                                                        const int32_t *__restrict__ seg_keep,
-                                                       const int32_t *__restrict__ nseg, int max_seg) {
+                                                       const int32_t *__restrict__ nseg, int max_seg,
+                                                       int budget, double cpiv) {
     extern __shared__ __align__(16) uint8_t dyn[];
     __shared__ int move_src[kPer * kThreads];
     __shared__ int scratch[33];
@@ -47,15 +64,20 @@ __global__ void __launch_bounds__(kThreads) tbe_kernel(Dev d, const int32_t *__r
     int *lo = keep + ms;
     int *hi = lo + ms;
     uint8_t *label = reinterpret_cast<uint8_t *>(hi + ms);
-    uint8_t *un = dyn + seg_table_bytes(ms);   // ranking stage, later the record move staging
+    double *ssum = reinterpret_cast<double *>(dyn + seg_table_bytes(ms));   // TAM only
+    int *scnt = reinterpret_cast<int *>(ssum + ms);
+    int *spiv = scnt + ms;
+    uint8_t *un = dyn + seg_table_bytes(ms) + (TAM ? tam_table_bytes(ms) : 0);   // ranking stage, then moves
     uint4 *move_buf = reinterpret_cast<uint4 *>(un);
+    __shared__ double red_d[kWarpsE];
+    __shared__ double sh_delta;
 
     const int s = blockIdx.x, b = s / d.Hkv;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int ns = min(max(nseg[b], 0), max_seg);
     for (int j = tid; j < ns; j += kThreads) {
         starts[j] = seg_start[(size_t)b * max_seg + j];
-        keep[j] = seg_keep[(size_t)b * max_seg + j];
+        keep[j] = TAM ? 0 : seg_keep[(size_t)b * max_seg + j];
         label[j] = seg_label[(size_t)b * max_seg + j];
         lo[j] = 0;
         hi[j] = 0;
@@ -98,6 +120,84 @@ __global__ void __launch_bounds__(kThreads) tbe_kernel(Dev d, const int32_t *__r
     }
     __syncthreads();
 
+    double delta = 0.0;   // TAM: candidates scoring at least delta are pivotal
+    if constexpr (TAM) {
+        // T1. per segment: candidates and their score sum (fp64)
+        for (int j = warp; j < ns; j += kWarpsE) {
+            const int c = label[j];
+            int n = 0;
+            double m = 0.0;
+            if (c <= 3) {
+                const int32_t *pc = d.pos[c] + (size_t)s * d.cap[c];
+                const float *sc = d.score[c] + (size_t)s * d.cap[c];
+                for (int i = lo[j] + lane; i < hi[j]; i += 32)
+                    if (pc[i] >= d.n_protect) { ++n; m += (double)sc[i]; }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                n += __shfl_xor_sync(kFull, n, o);
+                m += __shfl_xor_sync(kFull, m, o);
+            }
+            if (lane == 0) { scnt[j] = n; ssum[j] = m; }
+        }
+        __syncthreads();
+        // T2. the stream's mean score over all candidates -> delta
+        {
+            double m = 0.0;
+            int n = 0;
+            for (int j = tid; j < ns; j += kThreads) { m += ssum[j]; n += scnt[j]; }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m += __shfl_xor_sync(kFull, m, o);
+            if (lane == 0) red_d[warp] = m;
+            const int ntot = block_sum(n, scratch);   // ends with a barrier: red_d complete
+            if (tid == 0) {
+                double tot = 0.0;
+                for (int w = 0; w < kWarpsE; ++w) tot += red_d[w];
+                sh_delta = ntot > 0 ? cpiv * (tot / (double)ntot) : -1.0;
+            }
+            __syncthreads();
+            if (ntot == 0) return;   // no candidates: nothing to evict
+            delta = sh_delta;
+        }
+        // T3. pivotal candidates per segment
+        for (int j = warp; j < ns; j += kWarpsE) {
+            const int c = label[j];
+            int p = 0;
+            if (c <= 3) {
+                const int32_t *pc = d.pos[c] + (size_t)s * d.cap[c];
+                const float *sc = d.score[c] + (size_t)s * d.cap[c];
+                for (int i = lo[j] + lane; i < hi[j]; i += 32)
+                    p += pc[i] >= d.n_protect && (double)sc[i] >= delta;
+            }
+            p = __reduce_add_sync(kFull, p);
+            if (lane == 0) spiv[j] = p;
+        }
+        __syncthreads();
+        // T4. budgets: T' = max(0, budget - pivotal), t_j = min(n_j - p_j, floor(T' a_j / D + 1e-9))
+        {
+            double a = 0.0;
+            int P = 0;
+            for (int j = tid; j < ns; j += kThreads) {
+                if (scnt[j] > 0) a += sqrt(ssum[j] / scnt[j]) * scnt[j];
+                P += spiv[j];
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(kFull, a, o);
+            if (lane == 0) red_d[warp] = a;
+            const int Ptot = block_sum(P, scratch);
+            double D = 0.0;
+            for (int w = 0; w < kWarpsE; ++w) D += red_d[w];
+            const double Tp = budget > Ptot ? (double)(budget - Ptot) : 0.0;
+            for (int j = tid; j < ns; j += kThreads) {
+                long long t = 0;
+                if (scnt[j] > 0 && D > 0.0) t = (long long)floor(Tp * (sqrt(ssum[j] / scnt[j]) * scnt[j] / D) + 1e-9);
+                const int cap_j = scnt[j] - spiv[j];
+                keep[j] = (int)(t < cap_j ? t : cap_j);
+            }
+            __syncthreads();
+        }
+    }
+
     // 2. a warp per segment that must shrink: entry idx of the run is kept iff fewer
     //    than (retention + protected entries of the run) keys precede it
     uint64_t *st = reinterpret_cast<uint64_t *>(un) + warp * kStage;
@@ -109,17 +209,18 @@ __global__ void __launch_bounds__(kThreads) tbe_kernel(Dev d, const int32_t *__r
         if (e - a <= r) continue;
         const int32_t *pc = d.pos[c] + (size_t)s * d.cap[c];
         const float *sc = d.score[c] + (size_t)s * d.cap[c];
-        auto key_of = [&](int i) -> uint64_t {
-            const int32_t p = pc[i];
-            return p < d.n_protect ? ~0ull : entry_key(sc[i], p);
+        // protected (and, for TAM, pivotal) entries always stay: they rank first
+        auto fixed = [&](int i) -> bool {
+            return pc[i] < d.n_protect || (TAM && (double)sc[i] >= delta);
         };
+        auto key_of = [&](int i) -> uint64_t { return fixed(i) ? ~0ull : entry_key(sc[i], pc[i]); };
         int np = 0;
-        for (int i = a + lane; i < e; i += 32) np += pc[i] < d.n_protect;
+        for (int i = a + lane; i < e; i += 32) np += fixed(i);
         const int budget = r + __reduce_add_sync(kFull, np);
         if (e - a <= budget) continue;
         shrunk = 1;
-        if (r == 0) {   // only the protected entries stay
-            for (int i = a + lane; i < e; i += 32) flags[cbase[c] + i] = pc[i] < d.n_protect;
+        if (r == 0) {   // only the protected (pivotal) entries stay
+            for (int i = a + lane; i < e; i += 32) flags[cbase[c] + i] = fixed(i);
             continue;
         }
         const int cnt = e - a, per = (cnt + 31) >> 5;
@@ -216,24 +317,38 @@ __global__ void __launch_bounds__(kThreads) tbe_kernel(Dev d, const int32_t *__r
     compact_tables(d, s, n, evicted, keep_of, true, 0, scratch, move_src, move_buf);
 }
 
-}  // namespace
+template <bool TAM>
+cudaError_t launch_mode(const Dev &d, const int32_t *seg_start, const uint8_t *seg_label, const int32_t *seg_keep,
+                        const int32_t *nseg, int max_seg, int budget, double cpiv, cudaStream_t st,
+                        int64_t *launches) {
+    static bool configured = false;
+    const int ms = (max_seg + 3) & ~3;
+    const int smem = seg_table_bytes(ms) + (TAM ? tam_table_bytes(ms) : 0) + kUnionBytes;
+    if (!configured) {
+        const cudaError_t e = cudaFuncSetAttribute(
+            tbe_kernel<TAM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            seg_table_bytes(kMaxSeg) + (TAM ? tam_table_bytes(kMaxSeg) : 0) + kUnionBytes);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    tbe_kernel<TAM><<<d.S, kThreads, smem, st>>>(d, seg_start, seg_label, seg_keep, nseg, max_seg, budget, cpiv);
+    *launches += 1;
+    return cudaGetLastError();
+}
 
-int evict_segments_max() { return kMaxSeg; }
+}  // namespace
 
 cudaError_t launch_evict_segments(const Dev &d, const int32_t *seg_start, const uint8_t *seg_label,
                                   const int32_t *seg_keep, const int32_t *nseg, int max_seg, cudaStream_t st,
                                   int64_t *launches) {
-    static bool configured = false;
-    const int smem = seg_table_bytes((max_seg + 3) & ~3) + kUnionBytes;
-    if (!configured) {
-        const cudaError_t e = cudaFuncSetAttribute(tbe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   seg_table_bytes(kMaxSeg) + kUnionBytes);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
-    tbe_kernel<<<d.S, kThreads, smem, st>>>(d, seg_start, seg_label, seg_keep, nseg, max_seg);
-    *launches += 1;
-    return cudaGetLastError();
+    return launch_mode<false>(d, seg_start, seg_label, seg_keep, nseg, max_seg, 0, 0.0, st, launches);
 }
+
+cudaError_t launch_evict_tam(const Dev &d, const int32_t *seg_start, const uint8_t *seg_label, const int32_t *nseg,
+                             int max_seg, int budget, double c, cudaStream_t st, int64_t *launches) {
+    return launch_mode<true>(d, seg_start, seg_label, nullptr, nseg, max_seg, budget, c, st, launches);
+}
+
+int evict_segments_max() { return kMaxSeg; }
 
 }  // namespace tkv

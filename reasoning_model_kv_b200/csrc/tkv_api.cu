@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdio>
 #include <cstring>
 #include <new>
@@ -233,6 +234,22 @@ tkv_status tkv_evict_segments(tkv_cache *c, const int32_t *seg_start, const uint
     cudaError_t e = tkv::launch_evict_segments(c->dev, seg_start, seg_label, seg_keep, nseg, max_seg,
                                                static_cast<cudaStream_t>(stream), &c->launches);
     return cuda_status(e, "tkv_evict_segments");
+}
+
+tkv_status tkv_evict_tam(tkv_cache *c, const int32_t *seg_start, const uint8_t *seg_label, const int32_t *nseg,
+                         int32_t max_seg, int32_t budget, double cpiv, void *stream) {
+    if (!c) return fail(TKV_ERR_INVALID, "cache is NULL");
+    if (max_seg < 0 || max_seg > tkv::evict_segments_max())
+        return fail(TKV_ERR_INVALID, "max_seg must be in [0, 4096]");
+    if (budget < 0) return fail(TKV_ERR_INVALID, "budget must be >= 0");
+    if (!(cpiv >= 0.0) || !std::isfinite(cpiv)) return fail(TKV_ERR_INVALID, "c must be finite and >= 0");
+    if (max_seg == 0) return TKV_OK;
+    if (!seg_start || !seg_label || !nseg) return fail(TKV_ERR_INVALID, "NULL segment array");
+    auto a4 = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; };
+    if (!a4(seg_start) || !a4(nseg)) return fail(TKV_ERR_INVALID, "int32 arrays must be 4-byte aligned");
+    cudaError_t e = tkv::launch_evict_tam(c->dev, seg_start, seg_label, nseg, max_seg, budget, cpiv,
+                                          static_cast<cudaStream_t>(stream), &c->launches);
+    return cuda_status(e, "tkv_evict_tam");
 }
 
 tkv_status tkv_tbe_schedule(const uint8_t *label, int32_t nseg, int32_t r0, int32_t t_keep, int32_t *keep) {

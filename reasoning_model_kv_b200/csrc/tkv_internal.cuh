@@ -61,5 +61,8 @@ int evict_segments_max();
 cudaError_t launch_evict_segments(const Dev &d, const int32_t *seg_start, const uint8_t *seg_label,
                                   const int32_t *seg_keep, const int32_t *nseg, int max_seg, cudaStream_t st,
                                   int64_t *launches);
+// Thought-aware segment budgets with pivotal tokens (evict_segments.cu, TAM mode).
+cudaError_t launch_evict_tam(const Dev &d, const int32_t *seg_start, const uint8_t *seg_label, const int32_t *nseg,
+                             int max_seg, int budget, double c, cudaStream_t st, int64_t *launches);
 
 }  // namespace tkv

@@ -46,7 +46,8 @@ class TkvLayout(ctypes.Structure):
 EXPORTS = ["tkv_workspace_bytes", "tkv_create", "tkv_destroy", "tkv_reset", "tkv_get_layout",
            "tkv_quantize_append", "tkv_quantize_append_noalloc", "tkv_decode_attention", "tkv_evict_compact", "tkv_poll_error",
            "tkv_export_state", "tkv_import_state", "tkv_launch_count", "tkv_last_error_string",
-           "tkv_selftest_wait_timeout", "tkv_evict_segments", "tkv_tbe_schedule"]
+           "tkv_selftest_wait_timeout", "tkv_evict_segments", "tkv_tbe_schedule",
+           "tkv_evict_tam"]
 
 _lib = None
 
@@ -82,6 +83,8 @@ def lib() -> ctypes.CDLL:
     L.tkv_evict_segments.restype = ctypes.c_int
     L.tkv_tbe_schedule.argtypes = [vp, i32, i32, i32, vp]
     L.tkv_tbe_schedule.restype = ctypes.c_int
+    L.tkv_evict_tam.argtypes = [vp, vp, vp, vp, i32, i32, ctypes.c_double, vp]
+    L.tkv_evict_tam.restype = ctypes.c_int
     L.tkv_launch_count.restype = ctypes.c_int64
     L.tkv_last_error_string.restype = ctypes.c_char_p
     for name in ("tkv_create", "tkv_destroy", "tkv_reset", "tkv_get_layout", "tkv_quantize_append",
@@ -220,6 +223,18 @@ class TkvCache:
                                         _dptr(seg_keep, torch.int32, "seg_keep"),
                                         _dptr(nseg, torch.int32, "nseg"), shape[1], _stream(stream)))
 
+    def evict_tam(self, seg_start: torch.Tensor, seg_label: torch.Tensor, nseg: torch.Tensor, budget: int,
+                  c: float, stream=None):
+        """Thought-aware segment budgets with pivotal tokens (score >= c * mean) kept;
+        seg_start int32 / seg_label uint8 [B, max_seg], nseg int32 [B], on the device."""
+        if seg_start.dim() != 2 or seg_start.shape[0] != self.B or tuple(seg_label.shape) != tuple(seg_start.shape):
+            raise TkvError(TKV_ERR_INVALID, "seg_start and seg_label must be [B, max_seg]")
+        if tuple(nseg.shape) != (self.B,):
+            raise TkvError(TKV_ERR_INVALID, "nseg must be [B]")
+        _check(lib().tkv_evict_tam(self._h, _dptr(seg_start, torch.int32, "seg_start"),
+                                   _dptr(seg_label, torch.uint8, "seg_label"), _dptr(nseg, torch.int32, "nseg"),
+                                   seg_start.shape[1], int(budget), float(c), _stream(stream)))
+
     # -- housekeeping
     def reset(self, stream=None):
         _check(lib().tkv_reset(self._h, _stream(stream)))
@@ -294,6 +309,10 @@ def tkv_evict_compact(cache: TkvCache, budget, stream=None):
 
 def tkv_evict_segments(cache: TkvCache, seg_start, seg_label, seg_keep, nseg, stream=None):
     return cache.evict_segments(seg_start, seg_label, seg_keep, nseg, stream)
+
+
+def tkv_evict_tam(cache: TkvCache, seg_start, seg_label, nseg, budget, c, stream=None):
+    return cache.evict_tam(seg_start, seg_label, nseg, budget, c, stream)
 
 
 def tkv_tbe_schedule(labels, r0: int = 64, t_keep: int = 16):

@@ -141,3 +141,24 @@ def test_tbe_schedule_rejects_bad_arguments():
             tkv.tkv_tbe_schedule(labels, r0, t_keep)
     assert tkv.lib().tkv_tbe_schedule(None, -1, 64, 16, None) == tkv.TKV_ERR_INVALID
     assert tkv.lib().tkv_tbe_schedule(None, 3, 64, 16, None) == tkv.TKV_ERR_INVALID
+
+
+def test_evict_tam_rejects_bad_arguments_without_launching():
+    L = tkv.lib()
+    cfg = _cfg()
+    n = L.tkv_workspace_bytes(ctypes.byref(cfg))
+    h = ctypes.c_void_p()
+    assert L.tkv_create(ctypes.byref(cfg), ctypes.c_void_p(1 << 20), n, ctypes.byref(h)) == 0
+    p = ctypes.c_void_p(1 << 24)
+    INV = tkv.TKV_ERR_INVALID
+    assert L.tkv_evict_tam(None, p, p, p, 4, 10, 1.0, None) == INV
+    assert L.tkv_evict_tam(h, p, p, p, 4097, 10, 1.0, None) == INV
+    assert L.tkv_evict_tam(h, p, p, p, 4, -1, 1.0, None) == INV
+    assert L.tkv_evict_tam(h, p, p, p, 4, 10, -0.5, None) == INV
+    assert L.tkv_evict_tam(h, p, p, p, 4, 10, float("nan"), None) == INV
+    assert L.tkv_evict_tam(h, p, p, p, 4, 10, float("inf"), None) == INV
+    assert L.tkv_evict_tam(h, None, p, p, 4, 10, 1.0, None) == INV
+    assert L.tkv_evict_tam(h, p, p, ctypes.c_void_p((1 << 24) + 1), 4, 10, 1.0, None) == INV
+    assert L.tkv_evict_tam(h, None, None, None, 0, 10, 1.0, None) == tkv.TKV_OK   # no segments: no-op
+    assert L.tkv_launch_count(h) == 0
+    assert L.tkv_destroy(h) == 0

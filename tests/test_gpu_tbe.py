@@ -148,3 +148,79 @@ def test_segment_edge_cases(dense):
     with pytest.raises(TkvError):
         gpu.evict_segments(dev(st), dev(lb), dev(keep), dev(ns[:1]))
     assert gpu.poll_error() == tkv.TKV_OK
+
+
+# ----------------------------------------------------------------------------
+# thought-aware budgets with pivotal tokens (tkv_evict_tam)
+# ----------------------------------------------------------------------------
+def _tam_lockstep(w, gpu, o, rows, upto, budget, c):
+    st, lb, ns = synth.segment_table(w["seed"], w["B"], upto, w["p_r"], w["p_e"], b0=w.get("b0", 0))
+    sub = rows_streams(gpu, rows)
+    o.load_state(gpu.export_state(sub))
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+    gpu.evict_tam(dev(st), dev(lb), dev(ns), budget, c)
+    assert o.evict_tam(st[rows], lb[rows], ns[rows], budget, c) == 0
+    compare_states(gpu.export_state(sub), o.state, what=f"tam at {upto}")
+    assert gpu.poll_error() == tkv.TKV_OK
+
+
+@pytest.mark.parametrize("dense", [False, True], ids=["reuse", "dense"])
+def test_periodic_tam_small(dense):
+    """4 rows x 8/2 heads, 2k prefill; every 64 decode steps the thought-aware
+    budgets (512 per stream, pivotal above 3x the mean score) are applied and
+    checked against the oracle, three times (the page's periodic compaction), with
+    a checked decode step after each."""
+    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", B=4, steps=200, dense=dense)
+    ctx = w["ctx"]
+    for step in range(w["steps"]):
+        if step in (64, 128, 192):
+            _tam_lockstep(w, gpu, o, rows, ctx + step - 1, 512, 3.0)
+            _decode_step(w, gpu, o, rows, step)          # checked step on the compacted cache
+        else:
+            k, v, cls, pos, q = synth.decode_inputs(w, step, device=DEV)
+            gpu.quantize_append(k, v, cls, pos)
+            gpu.decode_attention(q, SCALE)
+    if dense:
+        _assert_dense(gpu)
+    assert gpu.poll_error() == tkv.TKV_OK
+
+
+@pytest.mark.parametrize("dense", [False, True], ids=["reuse", "dense"])
+def test_b8_ctx16k_tam_sampled_row(dense):
+    """Batch 8 x 32/8 heads, 16k prefill, 16 decode steps for scores, then budgets of
+    1638 per stream with pivotal tokens above 4x the mean; lock-step on row 6."""
+    rows = [6]
+    w = synth.prefill_inputs("b8_ctx16k_256steps", device=DEV)
+    gpu = TkvCache(w["B"], w["Hkv"], w["G"], w["cap"], w["n_protect"], max_append=w["ctx"], dense=dense)
+    gpu.quantize_append(w["k"], w["v"], w["cls"][:, :w["ctx"]].contiguous().to(DEV), w["pos"].to(DEV))
+    for step in range(16):
+        k, v, cls, pos, q = synth.decode_inputs(w, step, device=DEV)
+        gpu.quantize_append(k, v, cls, pos)
+        gpu.decode_attention(q, SCALE)
+    o = oracle_for(gpu, gpu.export_state(rows_streams(gpu, rows)), B=1)
+    before = gpu.export_state()["n"].sum()
+    _tam_lockstep(w, gpu, o, rows, w["ctx"] + 15, w["budget"], 4.0)
+    assert gpu.export_state()["n"].sum() < before
+    _decode_step(w, gpu, o, rows, 16)
+    if dense:
+        _assert_dense(gpu)
+    assert gpu.poll_error() == tkv.TKV_OK
+
+
+@pytest.mark.parametrize("dense", [False, True], ids=["reuse", "dense"])
+def test_tam_degenerate_cases(dense):
+    """c = 0 makes every candidate pivotal (nothing leaves); budget 0 with no pivotal
+    token keeps only protected, foreign and unsegmented entries."""
+    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", B=2, dense=dense, n_protect=100)
+    _decode_step(w, gpu, o, rows, 0)
+    before = gpu.export_state()
+    st, lb, ns = synth.segment_table(w["seed"], w["B"], w["ctx"], w["p_r"], w["p_e"])
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+    gpu.evict_tam(dev(st), dev(lb), dev(ns), 0, 0.0)
+    after = gpu.export_state()
+    for key in before:
+        assert np.array_equal(before[key], after[key]), key
+    _tam_lockstep(w, gpu, o, rows, w["ctx"], 0, 1e30)
+    g = gpu.export_state()
+    assert g["n"][:, 1:].sum() == 0                     # every R/E/T candidate left
+    assert (g["n"][:, 0] == 100).all()                  # the bf16 window stays
