@@ -58,10 +58,12 @@ def parse():
                          "tensor-memory kernel (dense placement only)")
     ap.add_argument("--evict-reps", type=int, default=5,
                     help="timed repetitions of the eviction that precedes the timed step")
-    ap.add_argument("--evict", choices=["topk", "tbe"], default="topk",
+    ap.add_argument("--evict", choices=["topk", "tbe", "tam"], default="topk",
                     help="eviction before the timed step: topk (each stream keeps its budget of "
-                         "highest-scoring tokens) or tbe (segment-level: the annealing schedule "
-                         "over the rows' thought segments, r0 64, t_keep 16)")
+                         "highest-scoring tokens), tbe (segment-level: the annealing schedule "
+                         "over the rows' thought segments, r0 64, t_keep 16) or tam (the budget "
+                         "split over segments in proportion to sqrt(mean score) x length, "
+                         "tokens above 3x the mean score kept)")
     ap.add_argument("--ctx", type=int, default=None,
                     help="prefill context before the eviction (default: the workload's); the "
                          "timed step is the same post-eviction step, with smaller pools")
@@ -194,7 +196,7 @@ def setup_cache(w, dev, dense, evict_reps, flush, attn_kernel=0, evict="topk"):
     k, v, c, p, q = synth.decode_inputs(w, 0, device=dev)        # untimed scoring step
     gpu.quantize_append(k, v, c, p)
     gpu.decode_attention(q, SCALE)
-    segs = segment_inputs(w, dev, w["ctx"]) if evict == "tbe" else None
+    segs = segment_inputs(w, dev, w["ctx"]) if evict in ("tbe", "tam") else None
     evict_ms = []
     snap = gpu.workspace.clone() if evict_reps > 0 else None
     st = torch.cuda.current_stream()
@@ -206,8 +208,10 @@ def setup_cache(w, dev, dense, evict_reps, flush, attn_kernel=0, evict="topk"):
         a.record(st)
         if segs is None:
             gpu.evict_compact(w["budget"])
-        else:
+        elif evict == "tbe":
             gpu.evict_segments(*segs)
+        else:
+            gpu.evict_tam(segs[0], segs[1], segs[3], w["budget"], 3.0)
         b2.record(st)
         b2.synchronize()
         if i > 0:
@@ -358,8 +362,10 @@ def run_tkv(args, rank, world, dev):
                    "total_bytes_per_step": pk + kv_tokens * (8 + (0 if args.placement == "dense" else 4))
                    + q.numel() * q.element_size() + out.numel() * out.element_size(),
                    "placement": args.placement, "attn_kernel": args.attn_kernel,
-                   "eviction": (f"topk, budget {w['budget']} per stream" if args.evict == "topk"
-                                else "tbe segment schedule at the scoring step (r0 64, t_keep 16)"),
+                   "eviction": {"topk": f"topk, budget {w['budget']} per stream",
+                                "tbe": "tbe segment schedule at the scoring step (r0 64, t_keep 16)",
+                                "tam": f"tam segment budgets, {w['budget']} per stream, pivotal above 3x "
+                                       "the mean score"}[args.evict],
                    "l2": "flushed (write of %d MB) before every timed step" % (flush.numel() >> 20),
                    "parallelism": f"{world} independent replicas" if world > 1 else "single GPU"},
         "hbm_gbs_packed": gbs,
