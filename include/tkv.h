@@ -18,6 +18,11 @@
  *   - eviction keeps, per (batch, kv head) stream, the `budget` highest-scoring
  *     unprotected tokens (DYNTS page, section 2.3, selection window: keep the
  *     top-k, evict the rest), then compacts the block table.
+ * Two segment-level policies share that compaction: tkv_evict_segments applies
+ * per-segment retentions, such as the TBE annealing schedule (ThinKV,
+ * "Metodologia", TBE) that tkv_tbe_schedule computes on the host; tkv_evict_tam
+ * splits a budget over the segments as the TAM page's allocation rule does and
+ * keeps its pivotal tokens.
  *
  * Conventions for every call:
  *   - Device pointers are plain CUDA device addresses; `stream` is a
@@ -57,7 +62,7 @@ typedef enum {
     TKV_ERR_INVALID = 1,   /* bad argument (host) or bad class id (device) */
     TKV_ERR_CAPACITY = 2,  /* a pool had no free slot: token dropped       */
     TKV_ERR_CUDA = 3,      /* a CUDA runtime call or launch failed         */
-    TKV_ERR_TIMEOUT = 4    /* reserved: a bounded device wait gave up      */
+    TKV_ERR_TIMEOUT = 4    /* a bounded device wait gave up                */
 } tkv_status;
 
 /* Thought classes.  Class 0 holds bf16 records (protected positions, or tokens
