@@ -208,6 +208,13 @@ TKV_API tkv_status tkv_decode_attention(tkv_cache *cache, const void *q, float s
  */
 TKV_API tkv_status tkv_evict_compact(tkv_cache *cache, int32_t budget, void *stream);
 
+/* tkv_evict_compact with a local window ("DYNTS", section 2.3: the most recently
+ * generated tokens are kept for local coherence): entries at positions >= keep_from
+ * are kept too and are not candidates, so `budget` applies to positions in
+ * [n_protect, keep_from) only.  keep_from = INT32_MAX is tkv_evict_compact.  Returns
+ * TKV_ERR_INVALID for a NULL cache or budget < 0. */
+TKV_API tkv_status tkv_evict_compact_window(tkv_cache *cache, int32_t budget, int32_t keep_from, void *stream);
+
 /* Segment-level eviction ("ThinKV", section Metodologia, TBE paragraph: when a
  * Transition thought starts, tokens of earlier R/E thought segments are evicted
  * progressively on an annealing schedule, at the granularity of segments).

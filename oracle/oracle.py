@@ -83,6 +83,8 @@ def lib():
         L.orc_attend.restype = None
         L.orc_evict.argtypes = [ctypes.POINTER(_State), ctypes.c_int]
         L.orc_evict.restype = ctypes.c_int
+        L.orc_evict_window.argtypes = [ctypes.POINTER(_State), ctypes.c_int, ctypes.c_int32]
+        L.orc_evict_window.restype = ctypes.c_int
         L.orc_evict_segments.argtypes = [ctypes.POINTER(_State)] + [ctypes.c_void_p] * 4 + [ctypes.c_int]
         L.orc_evict_segments.restype = ctypes.c_int
         L.orc_tbe_schedule.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -242,6 +244,11 @@ class OracleCache:
 
     def evict(self, budget: int) -> int:
         return lib().orc_evict(ctypes.byref(self._st), int(budget))
+
+    def evict_window(self, budget: int, keep_from: int) -> int:
+        """Top-k eviction whose candidates are the positions in [n_protect, keep_from):
+        the local window (positions >= keep_from) is kept as well."""
+        return lib().orc_evict_window(ctypes.byref(self._st), int(budget), int(keep_from))
 
     def evict_segments(self, seg_start: np.ndarray, seg_label: np.ndarray, seg_keep: np.ndarray,
                        nseg: np.ndarray) -> int:

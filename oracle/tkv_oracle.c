@@ -447,7 +447,15 @@ static int cand_cmp(const void *pa, const void *pb) {
  * order. */
 static void compact_stream(orc_state *st, int s, uint8_t *evict[4]);
 
-int orc_evict(orc_state *st, int budget) {
+int orc_evict_window(orc_state *st, int budget, int32_t keep_from);
+
+int orc_evict(orc_state *st, int budget) { return orc_evict_window(st, budget, INT32_MAX); }
+
+/* The same eviction with a local window ("DYNTS", section 2.3, local window: the
+ * most recently generated tokens are kept for local coherence): entries at
+ * positions >= keep_from are kept as well and are not candidates, so the budget
+ * applies to the selection window [n_protect, keep_from) only. */
+int orc_evict_window(orc_state *st, int budget, int32_t keep_from) {
     if (budget < 0) return ORC_ERR_INVALID;
     const int S = n_streams(st);
     for (int s = 0; s < S; ++s) {
@@ -458,7 +466,7 @@ int orc_evict(orc_state *st, int budget) {
         for (int c = 0; c < 4; ++c)
             for (int i = 0; i < st->n[s * 4 + c]; ++i) {
                 size_t e = (size_t)s * st->cap[c] + i;
-                if (st->pos[c][e] < st->n_protect) continue;
+                if (st->pos[c][e] < st->n_protect || st->pos[c][e] >= keep_from) continue;
                 cand[nc].skey = score_key(st->score[c][e]);
                 cand[nc].pos = st->pos[c][e];
                 cand[nc].c = c;

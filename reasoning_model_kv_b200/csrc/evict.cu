@@ -25,7 +25,9 @@ namespace {
 
 using namespace evict;
 
-__global__ void __launch_bounds__(kThreads) evict_kernel(Dev d, int budget) {
+// keep_from: positions >= keep_from (a local window of recent tokens) are kept and
+// are not candidates; INT32_MAX disables the window.
+__global__ void __launch_bounds__(kThreads) evict_kernel(Dev d, int budget, int keep_from) {
     const int s = blockIdx.x;
     __shared__ unsigned hist[256];
     __shared__ int scratch[33];
@@ -74,7 +76,7 @@ __global__ void __launch_bounds__(kThreads) evict_kernel(Dev d, int budget) {
 #pragma unroll
                 for (int j = 0; j < kPer; ++j) {
                     unsigned digit = 256u;                     // 256: lane adds nothing
-                    if (pv[j] >= d.n_protect) {
+                    if (pv[j] >= d.n_protect && pv[j] < keep_from) {
                         ++cnt;
                         const uint64_t key = entry_key(sv[j], pv[j]);
                         if (top_bits(key, 8 * pass) == want) digit = (unsigned)(key >> shift) & 255u;
@@ -140,7 +142,7 @@ __global__ void __launch_bounds__(kThreads) evict_kernel(Dev d, int budget) {
     const bool no_ties = done || keep_none;
     auto keep_of = [&](int, int, int32_t p, float scv, int &tie) -> int {
         tie = 0;
-        if (p < d.n_protect) return 1;
+        if (p < d.n_protect || p >= keep_from) return 1;
         if (keep_none) return 0;
         const uint64_t tb = top_bits(entry_key(scv, p), nb);
         tie = tb == pref && !done;
@@ -189,8 +191,8 @@ __global__ void __launch_bounds__(kThreads) evict_kernel(Dev d, int budget) {
 
 }  // namespace
 
-cudaError_t launch_evict(const Dev &d, int budget, cudaStream_t st, int64_t *launches) {
-    evict_kernel<<<d.S, kThreads, 0, st>>>(d, budget);
+cudaError_t launch_evict(const Dev &d, int budget, int keep_from, cudaStream_t st, int64_t *launches) {
+    evict_kernel<<<d.S, kThreads, 0, st>>>(d, budget, keep_from);
     *launches += 1;
     return cudaGetLastError();
 }

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <climits>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -216,10 +217,18 @@ tkv_status tkv_decode_attention(tkv_cache *c, const void *q, float softmax_scale
 tkv_status tkv_evict_compact(tkv_cache *c, int32_t budget, void *stream) {
     if (!c) return fail(TKV_ERR_INVALID, "cache is NULL");
     if (budget < 0) return fail(TKV_ERR_INVALID, "budget must be >= 0");
-    cudaError_t e = tkv::launch_evict(c->dev, budget, static_cast<cudaStream_t>(stream), &c->launches);
+    cudaError_t e = tkv::launch_evict(c->dev, budget, INT32_MAX, static_cast<cudaStream_t>(stream), &c->launches);
     const long long bound = (long long)budget + c->cfg.cap[0];
     c->live_ub = std::min(c->live_ub, bound);
     return cuda_status(e, "tkv_evict_compact");
+}
+
+tkv_status tkv_evict_compact_window(tkv_cache *c, int32_t budget, int32_t keep_from, void *stream) {
+    if (!c) return fail(TKV_ERR_INVALID, "cache is NULL");
+    if (budget < 0) return fail(TKV_ERR_INVALID, "budget must be >= 0");
+    // the window's size is not known here, so the live-entry bound stays as it is
+    cudaError_t e = tkv::launch_evict(c->dev, budget, keep_from, static_cast<cudaStream_t>(stream), &c->launches);
+    return cuda_status(e, "tkv_evict_compact_window");
 }
 
 tkv_status tkv_evict_segments(tkv_cache *c, const int32_t *seg_start, const uint8_t *seg_label,

@@ -55,7 +55,7 @@ cudaError_t launch_attention_tc(const Dev &d, const void *q, float scale, float 
                                 cudaStream_t st, int64_t *launches);
 // Self-test of the bounded device waits (selftest.cu).
 cudaError_t launch_wait_timeout(const Dev &d, long long limit, cudaStream_t st, int64_t *launches);
-cudaError_t launch_evict(const Dev &d, int budget, cudaStream_t st, int64_t *launches);
+cudaError_t launch_evict(const Dev &d, int budget, int keep_from, cudaStream_t st, int64_t *launches);
 // Segment-level eviction (evict_segments.cu); evict_segments_max() segments per row.
 int evict_segments_max();
 cudaError_t launch_evict_segments(const Dev &d, const int32_t *seg_start, const uint8_t *seg_label,

@@ -47,7 +47,7 @@ EXPORTS = ["tkv_workspace_bytes", "tkv_create", "tkv_destroy", "tkv_reset", "tkv
            "tkv_quantize_append", "tkv_quantize_append_noalloc", "tkv_decode_attention", "tkv_evict_compact", "tkv_poll_error",
            "tkv_export_state", "tkv_import_state", "tkv_launch_count", "tkv_last_error_string",
            "tkv_selftest_wait_timeout", "tkv_evict_segments", "tkv_tbe_schedule",
-           "tkv_evict_tam"]
+           "tkv_evict_tam", "tkv_evict_compact_window"]
 
 _lib = None
 
@@ -85,6 +85,8 @@ def lib() -> ctypes.CDLL:
     L.tkv_tbe_schedule.restype = ctypes.c_int
     L.tkv_evict_tam.argtypes = [vp, vp, vp, vp, i32, i32, ctypes.c_double, vp]
     L.tkv_evict_tam.restype = ctypes.c_int
+    L.tkv_evict_compact_window.argtypes = [vp, i32, i32, vp]
+    L.tkv_evict_compact_window.restype = ctypes.c_int
     L.tkv_launch_count.restype = ctypes.c_int64
     L.tkv_last_error_string.restype = ctypes.c_char_p
     for name in ("tkv_create", "tkv_destroy", "tkv_reset", "tkv_get_layout", "tkv_quantize_append",
@@ -206,6 +208,11 @@ class TkvCache:
     def evict_compact(self, budget: int, stream=None):
         _check(lib().tkv_evict_compact(self._h, int(budget), _stream(stream)))
 
+    def evict_compact_window(self, budget: int, keep_from: int, stream=None):
+        """Top-k eviction that also keeps every entry at a position >= keep_from
+        (the local window of recent tokens)."""
+        _check(lib().tkv_evict_compact_window(self._h, int(budget), int(keep_from), _stream(stream)))
+
     def evict_segments(self, seg_start: torch.Tensor, seg_label: torch.Tensor, seg_keep: torch.Tensor,
                        nseg: torch.Tensor, stream=None):
         """Segment-level eviction: seg_start int32 / seg_label uint8 / seg_keep int32
@@ -305,6 +312,10 @@ def tkv_decode_attention(cache: TkvCache, q, softmax_scale, out=None, stream=Non
 
 def tkv_evict_compact(cache: TkvCache, budget, stream=None):
     return cache.evict_compact(budget, stream)
+
+
+def tkv_evict_compact_window(cache: TkvCache, budget, keep_from, stream=None):
+    return cache.evict_compact_window(budget, keep_from, stream)
 
 
 def tkv_evict_segments(cache: TkvCache, seg_start, seg_label, seg_keep, nseg, stream=None):

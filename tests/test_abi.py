@@ -162,3 +162,15 @@ def test_evict_tam_rejects_bad_arguments_without_launching():
     assert L.tkv_evict_tam(h, None, None, None, 0, 10, 1.0, None) == tkv.TKV_OK   # no segments: no-op
     assert L.tkv_launch_count(h) == 0
     assert L.tkv_destroy(h) == 0
+
+
+def test_evict_compact_window_rejects_bad_arguments_without_launching():
+    L = tkv.lib()
+    cfg = _cfg()
+    n = L.tkv_workspace_bytes(ctypes.byref(cfg))
+    h = ctypes.c_void_p()
+    assert L.tkv_create(ctypes.byref(cfg), ctypes.c_void_p(1 << 20), n, ctypes.byref(h)) == 0
+    assert L.tkv_evict_compact_window(None, 3, 100, None) == tkv.TKV_ERR_INVALID
+    assert L.tkv_evict_compact_window(h, -1, 100, None) == tkv.TKV_ERR_INVALID
+    assert L.tkv_launch_count(h) == 0
+    assert L.tkv_destroy(h) == 0

@@ -364,3 +364,30 @@ def test_l32_b32_ctx32k_decode_loop_sampled_layers_and_steps(mode):
                         caches[layer].evict_compact(spec["budget"])
     for cache in caches:
         assert cache.poll_error() == tkv.TKV_OK
+
+
+@pytest.mark.parametrize("dense", [False, True], ids=["reuse", "dense"])
+def test_local_window_eviction(dense):
+    """Top-k with a local window of the 200 most recent positions (DYNTS 2.3): the
+    window and the protected sinks stay, the budget applies to the rest; a window
+    past every position is the plain eviction."""
+    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", B=2, dense=dense)
+    _decode_step(w, gpu, o, rows, 0)
+    keep_from = w["ctx"] + 1 - 200
+    sub = rows_streams(gpu, rows)
+    o.load_state(gpu.export_state(sub))
+    gpu.evict_compact_window(300, keep_from)
+    assert o.evict_window(300, keep_from) == 0
+    g = gpu.export_state(sub)
+    compare_states(g, o.state, what="local window")
+    assert (g["n"].sum(axis=1) == w["n_protect"] + 300 + 200).all()
+    before = gpu.export_state()
+    gpu.evict_compact_window(300, keep_from)     # the same window again: nothing to evict
+    after = gpu.export_state()
+    for key in before:
+        assert np.array_equal(before[key], after[key]), key
+    o.load_state(gpu.export_state(sub))          # window past every position: plain top-k
+    gpu.evict_compact_window(100, 1 << 30)
+    assert o.evict(100) == 0
+    compare_states(gpu.export_state(sub), o.state, what="window past every position")
+    assert gpu.poll_error() == tkv.TKV_OK

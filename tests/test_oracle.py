@@ -581,3 +581,42 @@ def test_dense_placement_matches_in_place_reuse():
                 assert dn.state["hw"][s, cc] == n and dn.state["ft"][s, cc] == 0
                 hs = ct.state[f"handle{cc}"][s, :n]
                 assert np.array_equal(dn.state[f"pool{cc}"][s, :n], ct.state[f"pool{cc}"][s, hs])
+
+
+# --------------------------------------------------------------------------
+# local window (DYNTS, section 2.3): the most recent tokens are kept
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("trial", range(20))
+def test_local_window_kept_set_equals_brute_force(trial):
+    rng = np.random.default_rng(500 + trial)
+    n_tok = int(rng.integers(3, 11))
+    n_protect = int(rng.integers(0, 3))
+    tie_pool = [0.0, 0.25, 0.5, 1.0, 1.0] if trial % 2 else list(rng.random(20))
+    cache = _tiny_cache_with_scores(rng, n_tok, n_protect, tie_pool)
+    before = cache.copy_state()
+    keep_from = int(rng.integers(0, n_tok + 2))
+    entries = []
+    for c in range(4):
+        for i in range(before["n"][0, c]):
+            p = before[f"pos{c}"][0, i]
+            if n_protect <= p < keep_from:
+                entries.append((before[f"score{c}"][0, i], p, c, i))
+    budget = int(rng.integers(0, n_tok + 1))
+    assert cache.evict_window(budget, keep_from) == 0
+    kept_pos = set()
+    for c in range(4):
+        kept_pos |= set(cache.live(0, c)[1].tolist())
+    expect = set(range(len(entries))) if budget >= len(entries) else _brute_force_kept(entries, budget)
+    fixed = {p for p in range(n_tok) if p < n_protect or p >= keep_from}
+    assert kept_pos == {int(entries[j][1]) for j in expect} | fixed
+    _check_table_invariants(cache, before)
+
+
+def test_local_window_past_every_position_is_plain_eviction():
+    rng = np.random.default_rng(77)
+    a = _tiny_cache_with_scores(rng, 10, 2, list(rng.random(10)))
+    b = orc.OracleCache(1, 1, 1, cap=a.cap, n_protect=2)
+    b.load_state(a.copy_state())
+    assert a.evict_window(4, 1 << 30) == 0 and b.evict(4) == 0
+    for key in a.state:
+        assert np.array_equal(a.state[key], b.state[key]), key
