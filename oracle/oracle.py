@@ -94,6 +94,19 @@ def lib():
                                                                                       ctypes.c_double]
         L.orc_evict_tam.restype = ctypes.c_int
         L.orc_num_threads.restype = ctypes.c_int
+        L.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
+        L.orc_e4m3_decode.restype = ctypes.c_double
+        L.orc_e4m3_encode.argtypes = [ctypes.c_float]
+        L.orc_e4m3_encode.restype = ctypes.c_uint8
+        L.orc_e4m3_round_up.argtypes = [ctypes.c_float]
+        L.orc_e4m3_round_up.restype = ctypes.c_uint8
+        L.orc_e2m1_decode.argtypes = [ctypes.c_uint8]
+        L.orc_e2m1_decode.restype = ctypes.c_double
+        L.orc_e2m1_encode.argtypes = [ctypes.c_float]
+        L.orc_e2m1_encode.restype = ctypes.c_uint8
+        for name in ("orc_quantize_group_fp8", "orc_quantize_group_ternary", "orc_quantize_block_nvfp4"):
+            getattr(L, name).argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
+            getattr(L, name).restype = None
         _lib = L
     return _lib
 
@@ -148,6 +161,50 @@ def unpack_record(bits: int, rec: np.ndarray, D=128, group=32):
 
 def num_threads() -> int:
     return lib().orc_num_threads()
+
+
+# ---------------------------------------------------------------- floating-point class codecs
+def e4m3_decode(code: int) -> float:
+    return lib().orc_e4m3_decode(int(code) & 0xFF)
+
+
+def e4m3_encode(x: float) -> int:
+    return lib().orc_e4m3_encode(float(np.float32(x)))
+
+
+def e4m3_round_up(x: float) -> int:
+    return lib().orc_e4m3_round_up(float(np.float32(x)))
+
+
+def e2m1_decode(code: int) -> float:
+    return lib().orc_e2m1_decode(int(code) & 0xF)
+
+
+def e2m1_encode(x: float) -> int:
+    return lib().orc_e2m1_encode(float(np.float32(x)))
+
+
+def _quantize_scaled(fn, x, scale_dtype):
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    sc = np.zeros(1, dtype=scale_dtype)
+    codes = np.zeros(len(x), dtype=np.uint8)
+    fn(_ptr(x), len(x), _ptr(sc), _ptr(codes))
+    return sc[0], codes
+
+
+def quantize_group_fp8(x):
+    """FP8 (E4M3) class group -> (fp16 scale bits, E4M3 codes)."""
+    return _quantize_scaled(lib().orc_quantize_group_fp8, x, np.uint16)
+
+
+def quantize_block_nvfp4(x):
+    """NVFP4 block of 16 -> (E4M3 scale code, E2M1 codes)."""
+    return _quantize_scaled(lib().orc_quantize_block_nvfp4, x, np.uint8)
+
+
+def quantize_group_ternary(x):
+    """Ternary group -> (fp16 scale bits, codes 0 / 1 (+1) / 3 (-1))."""
+    return _quantize_scaled(lib().orc_quantize_group_ternary, x, np.uint16)
 
 
 def tbe_schedule(labels, r0: int = 64, t_keep: int = 16) -> np.ndarray:

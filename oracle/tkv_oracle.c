@@ -152,6 +152,129 @@ uint16_t orc_f32_to_f16_ru(float xf) {
 /* ------------------------------------------------------------------ */
 /* Group quantisation and record packing                               */
 /* ------------------------------------------------------------------ */
+/* ------------------------------------------------------------------ */
+/* Floating-point class codecs (the ThinKV page, Metodologia, TBQ: FP8 or NVFP4 */
+/* for Reasoning tokens, ternary for Transition tokens).  Oracle only: the CUDA  */
+/* path does not implement these formats yet.                                   */
+/* ------------------------------------------------------------------ */
+
+/* FP8 E4M3 in its "fn" form (OCP 8-bit floating point): sign, 4 exponent bits
+ * (bias 7), 3 mantissa bits, no infinities, S.1111.111 is NaN, largest finite
+ * value 1.75 * 2^8 = 448, subnormals m/8 * 2^-6. */
+double orc_e4m3_decode(uint8_t code) {
+    const int sg = code >> 7, e = (code >> 3) & 15, m = code & 7;
+    if (e == 15 && m == 7) return NAN;
+    const double v = e == 0 ? ldexp(m / 8.0, -6) : ldexp(1.0 + m / 8.0, e - 7);
+    return sg ? -v : v;
+}
+
+/* Nearest E4M3 value, ties to an even mantissa; magnitudes at or above 448
+ * saturate to 448 (the format has no infinity); NaN encodes as 0x7F. */
+uint8_t orc_e4m3_encode(float xf) {
+    if (isnan(xf)) return 0x7F;
+    const uint8_t sg = signbit(xf) ? 0x80 : 0x00;
+    const double a = fabs((double)xf);
+    if (a >= 448.0) return sg | 0x7E;
+    if (a == 0.0) return sg;
+    int E;
+    frexp(a, &E);                                  /* a = f 2^E, f in [0.5, 1) */
+    const int ex = a < ldexp(1.0, -6) ? -6 : E - 1;   /* binade (subnormals: -6) */
+    const double q = ldexp(1.0, ex - 3);           /* spacing of the binade */
+    const double r = a / q, fl = floor(r), fr = r - fl;
+    const double n = (fr > 0.5 || (fr == 0.5 && fmod(fl, 2.0) != 0.0)) ? fl + 1.0 : fl;
+    const double v = n * q;                        /* <= 448: a < 448 and 448 is on the grid */
+    if (v == 0.0) return sg;
+    int E2;
+    frexp(v, &E2);
+    const int e2 = E2 - 1;
+    if (e2 < -6) return sg | (uint8_t)(v / ldexp(1.0, -9));          /* subnormal */
+    const int m = (int)((v / ldexp(1.0, e2) - 1.0) * 8.0);
+    return sg | (uint8_t)(((e2 + 7) << 3) | m);
+}
+
+/* Smallest E4M3 value >= y > 0 (saturated at 448). */
+uint8_t orc_e4m3_round_up(float y) {
+    if (!(y > 0.0f)) return 0x00;
+    if ((double)y >= 448.0) return 0x7E;
+    uint8_t c = orc_e4m3_encode(y);
+    if (orc_e4m3_decode(c) < (double)y) c = (uint8_t)(c + 1);   /* positive codes are ordered */
+    return c;
+}
+
+/* FP4 E2M1 (the element type of NVFP4): bit 3 sign, magnitudes of codes 0..7. */
+static const double k_e2m1[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+double orc_e2m1_decode(uint8_t code) {
+    const double v = k_e2m1[code & 7];
+    return (code & 8) ? -v : v;
+}
+
+/* Nearest E2M1 value, ties to the even code (even mantissa); saturates at 6. */
+uint8_t orc_e2m1_encode(float xf) {
+    const uint8_t sg = signbit(xf) ? 8 : 0;
+    const double a = fabs((double)xf);
+    int k = 7;
+    for (int j = 0; j < 7; ++j) {
+        const double mid = 0.5 * (k_e2m1[j] + k_e2m1[j + 1]);
+        if (a < mid) { k = j; break; }
+        if (a == mid) { k = (j % 2 == 0) ? j : j + 1; break; }
+    }
+    return sg | (uint8_t)k;
+}
+
+/* fp16 nearest (ties to even) of an fp32 value, from the directed roundings. */
+static uint16_t f16_rn(float x);
+
+/* FP8 class group: scale = smallest fp16 >= amax / 448 (fp32 division); code =
+ * E4M3 nearest of x / scale (fp32 division); all codes 0 when amax == 0.  The
+ * group's x_hat = decode(code) * scale. */
+void orc_quantize_group_fp8(const float *x, int n, uint16_t *scale_h, uint8_t *codes) {
+    float amax = 0.0f;
+    for (int i = 0; i < n; ++i) amax = fmaxf(amax, fabsf(x[i]));
+    const uint16_t sh = orc_f32_to_f16_ru(amax / 448.0f);
+    const float sf = (float)orc_f16_to_f64(sh);
+    *scale_h = sh;
+    for (int i = 0; i < n; ++i) codes[i] = sf == 0.0f ? 0 : orc_e4m3_encode(x[i] / sf);
+}
+
+/* NVFP4 block (16 values): scale = smallest E4M3 >= amax / 6 (fp32 division,
+ * saturated at 448); code = E2M1 nearest of x / scale (fp32 division); all codes 0
+ * when amax == 0. */
+void orc_quantize_block_nvfp4(const float *x, int n, uint8_t *scale_e4m3, uint8_t *codes) {
+    float amax = 0.0f;
+    for (int i = 0; i < n; ++i) amax = fmaxf(amax, fabsf(x[i]));
+    const uint8_t sc = orc_e4m3_round_up(amax / 6.0f);
+    const float sf = (float)orc_e4m3_decode(sc);
+    *scale_e4m3 = sc;
+    for (int i = 0; i < n; ++i) codes[i] = sf == 0.0f ? 0 : orc_e2m1_encode(x[i] / sf);
+}
+
+/* Ternary group (threshold ternarisation): delta = 0.7 * mean |x|, alpha = mean of
+ * |x| over the elements with |x| > delta, scale = fp16 nearest of alpha; code 1 for
+ * x > delta, 3 (-1 in two bits) for x < -delta, else 0 (all fp32, sums left to
+ * right).  x_hat = {0, +scale, -scale}. */
+void orc_quantize_group_ternary(const float *x, int n, uint16_t *scale_h, uint8_t *codes) {
+    float sa = 0.0f;
+    for (int i = 0; i < n; ++i) sa += fabsf(x[i]);
+    const float delta = 0.7f * (sa / (float)n);
+    float sb = 0.0f;
+    int cnt = 0;
+    for (int i = 0; i < n; ++i)
+        if (fabsf(x[i]) > delta) { sb += fabsf(x[i]); ++cnt; }
+    const float alpha = cnt ? sb / (float)cnt : 0.0f;
+    *scale_h = f16_rn(alpha);
+    for (int i = 0; i < n; ++i) codes[i] = x[i] > delta ? 1 : (x[i] < -delta ? 3 : 0);
+}
+
+static uint16_t f16_rn(float x) {
+    const uint16_t lo = orc_f32_to_f16_rd(x), hi = orc_f32_to_f16_ru(x);
+    if (lo == hi) return lo;
+    const double dl = (double)x - orc_f16_to_f64(lo), dh = orc_f16_to_f64(hi) - (double)x;
+    if (dl < dh) return lo;
+    if (dh < dl) return hi;
+    return (lo & 1) ? hi : lo;   /* tie: the even fp16 */
+}
+
 int orc_record_bytes(int bits, int D, int group) {
     if (bits == 16) return 2 * D * 2;
     int ngroups = D / group;

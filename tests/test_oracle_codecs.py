@@ -1,0 +1,136 @@
+"""Pins of the oracle's floating-point class codecs (ThinKV page, Metodologia, TBQ:
+FP8 or NVFP4 for Reasoning tokens, ternary for Transition tokens).  These are oracle
+groundwork for a later CUDA path; CPU only.
+
+FP8 E4M3 is pinned against torch's float8_e4m3fn conversions (a library routine:
+every code's value, round-to-nearest-even on random and half-way inputs); E2M1
+against the OCP table of its eight magnitudes and a brute-force nearest search;
+the group quantisers against their error bounds, exact round trips and hand cases."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as orc
+
+# OCP MX: the magnitudes of the E2M1 codes 0..7 (bit 3 is the sign)
+E2M1_TABLE = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def test_e4m3_decode_matches_torch_for_every_code():
+    ref = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).float().numpy()
+    for c in range(256):
+        got = orc.e4m3_decode(c)
+        if np.isnan(ref[c]):
+            assert np.isnan(got), c
+        else:
+            assert got == ref[c] and np.signbit(got) == np.signbit(ref[c]), c
+
+
+def _torch_e4m3_code(x):
+    return int(torch.tensor([x], dtype=torch.float32).to(torch.float8_e4m3fn).view(torch.uint8)[0])
+
+
+def test_e4m3_encode_matches_torch_round_to_nearest_even():
+    rng = np.random.default_rng(0)
+    xs = np.concatenate([rng.uniform(-440, 440, 3000), rng.normal(0, 1, 3000),
+                         rng.uniform(-2 ** -6, 2 ** -6, 1000), rng.normal(0, 1e-3, 500)]).astype(np.float32)
+    # every half-way point between neighbouring finite codes (ties go to the even code)
+    vals = sorted({orc.e4m3_decode(c) for c in range(0x7F)})
+    mids = np.array([(a + b) / 2 for a, b in zip(vals, vals[1:])], np.float32)
+    for x in np.concatenate([xs, mids, -mids]):
+        assert orc.e4m3_encode(x) == _torch_e4m3_code(float(x)), x
+
+
+def test_e4m3_saturates_and_rounds_up():
+    assert orc.e4m3_encode(448.0) == 0x7E and orc.e4m3_encode(1e9) == 0x7E and orc.e4m3_encode(-500) == 0xFE
+    assert np.isnan(orc.e4m3_decode(orc.e4m3_encode(float("nan"))))
+    rng = np.random.default_rng(1)
+    for y in np.concatenate([rng.uniform(1e-4, 440, 2000), [2 ** -9, 1.0, 448.0]]).astype(np.float32):
+        c = orc.e4m3_round_up(y)
+        v = orc.e4m3_decode(c)
+        assert v >= y and (c == 0 or orc.e4m3_decode(c - 1) < y), y
+
+
+def test_e2m1_table_and_brute_force_nearest():
+    for c in range(16):
+        mag = E2M1_TABLE[c & 7]
+        assert orc.e2m1_decode(c) == (-mag if c & 8 else mag)
+    rng = np.random.default_rng(2)
+    mids = [(a + b) / 2 for a, b in zip(E2M1_TABLE, E2M1_TABLE[1:])]
+    xs = np.concatenate([rng.uniform(-6.5, 6.5, 4000), mids, [-m for m in mids], [7.0, -100.0]])
+    for x in xs.astype(np.float32):
+        a = min(abs(float(x)), 6.0)
+        best = min(range(8), key=lambda k: (abs(E2M1_TABLE[k] - a), k % 2))   # nearest, then even
+        assert orc.e2m1_encode(x) & 7 == best, x
+        assert (orc.e2m1_encode(x) >> 3) == (1 if np.signbit(x) else 0)
+
+
+def _e4m3_half_gap(a):
+    """Half the E4M3 spacing at magnitude a (the largest rounding error there)."""
+    ex = -6 if a < 2 ** -6 else int(np.floor(np.log2(a)))
+    return 2.0 ** (ex - 3) / 2
+
+
+@pytest.mark.parametrize("scale", [1.0, 0.01, 37.0])
+def test_fp8_group_error_bound_and_range(scale):
+    rng = np.random.default_rng(3)
+    for _ in range(200):
+        x = (rng.normal(0, 1, 32) * scale).astype(np.float32)
+        sh, codes = orc.quantize_group_fp8(x)
+        s = orc.f16_value(sh)
+        amax = float(np.max(np.abs(x)))
+        assert s >= amax / 448 and s > 0
+        for xi, c in zip(x, codes):
+            r = np.float32(xi) / np.float32(s)
+            assert abs(float(r)) <= 448
+            xh = orc.e4m3_decode(int(c)) * s
+            assert abs(xh - float(xi)) <= (_e4m3_half_gap(abs(float(r))) + 2 ** -20 * abs(float(r))) * s
+
+
+def test_fp8_group_round_trip_of_representable_values():
+    s_bits = orc.f16_rd(0.25)
+    s = orc.f16_value(s_bits)
+    codes = np.array([0x38, 0x39, 0x3F, 0x01, 0x7E, 0xB8, 0x00, 0x10] * 4, np.uint8)
+    x = np.array([orc.e4m3_decode(int(c)) * s for c in codes], np.float32)
+    sh, got = orc.quantize_group_fp8(x)
+    assert orc.f16_value(sh) == s          # amax = 448 s, so the scale is s itself
+    assert np.array_equal(got, codes)
+
+
+def test_nvfp4_block_error_bound():
+    rng = np.random.default_rng(4)
+    for _ in range(300):
+        x = (rng.normal(0, 1, 16) * rng.choice([0.01, 1.0, 30.0])).astype(np.float32)
+        sc, codes = orc.quantize_block_nvfp4(x)
+        s = orc.e4m3_decode(int(sc))
+        amax = float(np.max(np.abs(x)))
+        assert s >= amax / 6 and (sc == 0 or orc.e4m3_decode(int(sc) - 1) < np.float32(amax) / np.float32(6))
+        for xi, c in zip(x, codes):
+            r = abs(float(np.float32(xi) / np.float32(s)))
+            assert r <= 6.0 + 1e-6
+            gap = 0.5 if r <= 2 else (1.0 if r <= 4 else 2.0)
+            xh = orc.e2m1_decode(int(c)) * s
+            assert abs(xh - float(xi)) <= (gap / 2 + 1e-6) * s
+
+
+def test_ternary_hand_cases():
+    x = np.array([3.0, -3.0] + [0.25] * 30, np.float32)      # mean |x| = 0.421875, delta = 0.2953125
+    sh, codes = orc.quantize_group_ternary(x)
+    assert orc.f16_value(sh) == 3.0
+    assert codes.tolist() == [1, 3] + [0] * 30
+    x = np.full(32, -2.0, np.float32)                          # every element beyond delta = 1.4
+    sh, codes = orc.quantize_group_ternary(x)
+    assert orc.f16_value(sh) == 2.0 and codes.tolist() == [3] * 32
+    sh, codes = orc.quantize_group_ternary(np.zeros(32, np.float32))
+    assert orc.f16_value(sh) == 0.0 and codes.tolist() == [0] * 32
+
+
+def test_ternary_scale_is_the_mean_magnitude_above_the_threshold():
+    rng = np.random.default_rng(5)
+    for _ in range(200):
+        x = rng.normal(0, 1, 32).astype(np.float32)
+        sh, codes = orc.quantize_group_ternary(x)
+        delta = np.float32(0.7) * (np.float32(np.sum(np.abs(x), dtype=np.float32)) / np.float32(32))
+        big = np.abs(x) > delta
+        assert codes.tolist() == [1 if v > delta else (3 if v < -delta else 0) for v in x]
+        assert abs(orc.f16_value(sh) - float(np.abs(x[big]).mean())) <= 2 ** -10 * float(np.abs(x[big]).mean()) + 1e-6
