@@ -51,6 +51,7 @@ class _State(ctypes.Structure):
         ("n", ctypes.c_void_p), ("ft", ctypes.c_void_p), ("hw", ctypes.c_void_p),
         ("handle", ctypes.c_void_p * 4), ("pos", ctypes.c_void_p * 4),
         ("fs", ctypes.c_void_p * 4), ("score", ctypes.c_void_p * 4),
+        ("codec", ctypes.c_int32),
     ]
 
 
@@ -69,6 +70,12 @@ def lib():
         L.orc_f16_to_f64.restype = ctypes.c_double
         L.orc_record_bytes.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int]
         L.orc_record_bytes.restype = ctypes.c_int
+        L.orc_record_bytes_fmt.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int]
+        L.orc_record_bytes_fmt.restype = ctypes.c_int
+        L.orc_pack_record_fmt.argtypes = [ctypes.c_int] * 3 + [ctypes.c_void_p] * 3
+        L.orc_pack_record_fmt.restype = None
+        L.orc_unpack_record_fmt.argtypes = [ctypes.c_int] * 3 + [ctypes.c_void_p] * 3
+        L.orc_unpack_record_fmt.restype = None
         L.orc_quantize_group.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
                                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
         L.orc_quantize_group.restype = None
@@ -131,6 +138,35 @@ def f16_value(h: int) -> float:
 
 def record_bytes(bits: int, D: int = 128, group: int = 32) -> int:
     return lib().orc_record_bytes(bits, D, group)
+
+
+FMT_FP8, FMT_NVFP4, FMT_TERNARY = 108, 104, 102   # floating-point class record formats
+
+
+def record_bytes_fmt(fmt: int, D: int = 128, group: int = 32) -> int:
+    return lib().orc_record_bytes_fmt(fmt, D, group)
+
+
+def class_format(bits: int, codec: int) -> int:
+    """Record format of a class: bf16 (16), integer codes (8/4/2), or with codec = 1
+    the FP codecs (FP8 for 8, NVFP4 for 4, ternary for 2)."""
+    return 100 + bits if codec and bits < 16 else bits
+
+
+def pack_record_fmt(fmt: int, k_bf16: np.ndarray, v_bf16: np.ndarray, D: int = 128, group: int = 32):
+    k = np.ascontiguousarray(k_bf16, dtype=np.uint16)
+    v = np.ascontiguousarray(v_bf16, dtype=np.uint16)
+    rec = np.zeros(record_bytes_fmt(fmt, D, group), dtype=np.uint8)
+    lib().orc_pack_record_fmt(fmt, D, group, _ptr(k), _ptr(v), _ptr(rec))
+    return rec
+
+
+def unpack_record_fmt(fmt: int, rec: np.ndarray, D: int = 128, group: int = 32):
+    rec = np.ascontiguousarray(rec, dtype=np.uint8)
+    kh = np.zeros(D, dtype=np.float64)
+    vh = np.zeros(D, dtype=np.float64)
+    lib().orc_unpack_record_fmt(fmt, D, group, _ptr(rec), _ptr(kh), _ptr(vh))
+    return kh, vh
 
 
 def quantize_group(x, bits: int):
@@ -222,9 +258,10 @@ def tbe_schedule(labels, r0: int = 64, t_keep: int = 16) -> np.ndarray:
 class OracleCache:
     """Host-side model of one layer's compressed cache."""
 
-    def __init__(self, B, Hkv, G, cap, n_protect, D=128, group=32, bits=BITS, dense=False):
+    def __init__(self, B, Hkv, G, cap, n_protect, D=128, group=32, bits=BITS, dense=False, codec=0):
         self.B, self.Hkv, self.G, self.D, self.group = B, Hkv, G, D, group
         self.dense = bool(dense)
+        self.codec = int(codec)
         self.n_protect = n_protect
         self.bits = tuple(bits)
         self.cap = tuple(int(c) for c in cap)
@@ -238,18 +275,19 @@ class OracleCache:
             self.state[f"pos{c}"] = np.zeros((S, cc), np.int32)
             self.state[f"score{c}"] = np.zeros((S, cc), np.float32)
             self.state[f"fs{c}"] = np.zeros((S, cc), np.int32)
-            self.state[f"pool{c}"] = np.zeros((S, cc, record_bytes(self.bits[c], D, group)),
-                                              np.uint8)
+            self.state[f"pool{c}"] = np.zeros(
+                (S, cc, record_bytes_fmt(class_format(self.bits[c], self.codec), D, group)), np.uint8)
         self._sync_struct()
 
     def rec_bytes(self, c):
-        return record_bytes(self.bits[c], self.D, self.group)
+        return record_bytes_fmt(class_format(self.bits[c], self.codec), self.D, self.group)
 
     def _sync_struct(self):
         st = _State()
         st.B, st.Hkv, st.G, st.D, st.group = self.B, self.Hkv, self.G, self.D, self.group
         st.n_protect = self.n_protect
         st.dense = int(self.dense)
+        st.codec = self.codec
         for c in range(4):
             st.bits[c] = self.bits[c]
             st.cap[c] = self.cap[c]

@@ -70,6 +70,7 @@ typedef struct {
     int32_t *n, *ft, *hw;          /* [S][4] */
     int32_t *handle[4], *pos[4], *fs[4];  /* [S][cap[c]] */
     float *score[4];               /* [S][cap[c]] */
+    int32_t codec;     /* 0: integer codes; 1: FP codes for classes 1-3 (FP8, NVFP4, ternary) */
 } orc_state;
 
 /* ------------------------------------------------------------------ */
@@ -411,13 +412,100 @@ void orc_unpack_record(int bits, int D, int group, const uint8_t *rec, double *k
     }
 }
 
+/* Record formats: 16 bf16, 8 / 4 / 2 integer codes (above), and the floating-point
+ * class codecs 108 FP8 (E4M3), 104 NVFP4 (E2M1, blocks of 16), 102 ternary.  FP
+ * records keep the codes in head-dim order:
+ *   108: [K codes: D bytes][V codes: D bytes][K scale x ngroups][V scale x ngroups] (fp16)
+ *   104: [K codes: D/2 bytes, element i in the low nibble of byte i/2 when i is even]
+ *        [V codes][K block scales: D/16 bytes (E4M3)][V block scales]
+ *   102: [K codes: D/4 bytes, element i at bit 2(i%4) of byte i/4; 1 = +1, 3 = -1]
+ *        [V codes][K scale x ngroups][V scale x ngroups] (fp16) */
+int orc_record_bytes_fmt(int fmt, int D, int group) {
+    const int ng = D / group;
+    switch (fmt) {
+        case 108: return 2 * D + 4 * ng;
+        case 104: return D + 2 * (D / 16);
+        case 102: return D / 2 + 4 * ng;
+        default: return orc_record_bytes(fmt, D, group);
+    }
+}
+
+static int class_fmt(const orc_state *st, int c) {
+    return (st->codec && st->bits[c] < 16) ? 100 + st->bits[c] : st->bits[c];
+}
+
+void orc_pack_record_fmt(int fmt, int D, int group, const uint16_t *k, const uint16_t *v, uint8_t *rec) {
+    if (fmt < 100) {
+        orc_pack_record(fmt, D, group, k, v, rec);
+        return;
+    }
+    const int ng = D / group;
+    float x[512];
+    uint8_t codes[512];
+    for (int which = 0; which < 2; ++which) {
+        const uint16_t *src = which == 0 ? k : v;
+        for (int i = 0; i < D; ++i) x[i] = bf16_to_f32(src[i]);
+        if (fmt == 108) {
+            for (int g = 0; g < ng; ++g) {
+                uint16_t sh;
+                orc_quantize_group_fp8(x + g * group, group, &sh, codes + g * group);
+                put_u16(rec + 2 * D + (which * ng + g) * 2, sh);
+            }
+            memcpy(rec + which * D, codes, D);
+        } else if (fmt == 104) {
+            for (int blk = 0; blk < D / 16; ++blk) {
+                uint8_t sc;
+                orc_quantize_block_nvfp4(x + blk * 16, 16, &sc, codes + blk * 16);
+                rec[D + which * (D / 16) + blk] = sc;
+            }
+            uint8_t *dst = rec + which * (D / 2);
+            for (int i = 0; i < D; i += 2) dst[i / 2] = (uint8_t)((codes[i] & 15) | ((codes[i + 1] & 15) << 4));
+        } else {   /* 102 */
+            for (int g = 0; g < ng; ++g) {
+                uint16_t sh;
+                orc_quantize_group_ternary(x + g * group, group, &sh, codes + g * group);
+                put_u16(rec + D / 2 + (which * ng + g) * 2, sh);
+            }
+            uint8_t *dst = rec + which * (D / 4);
+            for (int i = 0; i < D; i += 4)
+                dst[i / 4] = (uint8_t)(codes[i] | (codes[i + 1] << 2) | (codes[i + 2] << 4) | (codes[i + 3] << 6));
+        }
+    }
+}
+
+/* Dequantise a record of any format, in fp64. */
+void orc_unpack_record_fmt(int fmt, int D, int group, const uint8_t *rec, double *k_hat, double *v_hat) {
+    if (fmt < 100) {
+        orc_unpack_record(fmt, D, group, rec, k_hat, v_hat);
+        return;
+    }
+    for (int which = 0; which < 2; ++which) {
+        double *dst = which == 0 ? k_hat : v_hat;
+        for (int d = 0; d < D; ++d) {
+            const int g = d / group;
+            if (fmt == 108) {
+                const double sc = orc_f16_to_f64(get_u16(rec + 2 * D + (which * (D / group) + g) * 2));
+                dst[d] = orc_e4m3_decode(rec[which * D + d]) * sc;
+            } else if (fmt == 104) {
+                const uint8_t byte = rec[which * (D / 2) + d / 2];
+                const uint8_t code = (d & 1) ? (byte >> 4) : (byte & 15);
+                dst[d] = orc_e2m1_decode(code) * orc_e4m3_decode(rec[D + which * (D / 16) + d / 16]);
+            } else {
+                const uint8_t code = (rec[which * (D / 4) + d / 4] >> (2 * (d % 4))) & 3;
+                const double sc = orc_f16_to_f64(get_u16(rec + D / 2 + (which * (D / group) + g) * 2));
+                dst[d] = code == 1 ? sc : (code == 3 ? -sc : 0.0);
+            }
+        }
+    }
+}
+
 /* ------------------------------------------------------------------ */
 /* Cache operations                                                    */
 /* ------------------------------------------------------------------ */
 static int n_streams(const orc_state *st) { return st->B * st->Hkv; }
 
 static uint8_t *record_ptr(const orc_state *st, int s, int c, int slot) {
-    size_t rb = (size_t)orc_record_bytes(st->bits[c], st->D, st->group);
+    size_t rb = (size_t)orc_record_bytes_fmt(class_fmt(st, c), st->D, st->group);
     return st->pool[c] + ((size_t)s * st->cap[c] + slot) * rb;
 }
 
@@ -460,8 +548,8 @@ int orc_append(orc_state *st, const uint16_t *k, const uint16_t *v, const uint8_
                 st->pos[c][e] = p;
                 st->score[c][e] = 0.0f;
                 size_t off = (((size_t)b * st->Hkv + h) * T + t) * D;
-                orc_pack_record(st->bits[c], D, st->group, k + off, v + off,
-                                record_ptr(st, s, c, slot));
+                orc_pack_record_fmt(class_fmt(st, c), D, st->group, k + off, v + off,
+                                    record_ptr(st, s, c, slot));
             }
         }
     return status;
@@ -496,8 +584,8 @@ void orc_attend(orc_state *st, const uint16_t *q, float softmax_scale, float *ou
         for (int c = 0; c < 4; ++c)
             for (int i = 0; i < st->n[s * 4 + c]; ++i, ++t) {
                 size_t e = (size_t)s * st->cap[c] + i;
-                orc_unpack_record(st->bits[c], D, st->group,
-                                  record_ptr(st, s, c, st->handle[c][e]), kh, vh + (size_t)t * D);
+                orc_unpack_record_fmt(class_fmt(st, c), D, st->group,
+                                      record_ptr(st, s, c, st->handle[c][e]), kh, vh + (size_t)t * D);
                 sc[t] = &st->score[c][e];
                 for (int j = 0; j < G; ++j) {
                     double acc = 0;
@@ -624,7 +712,7 @@ static void compact_stream(orc_state *st, int s, uint8_t *evict[4]) {
         for (int i = 0; i < n; ++i) m += evict[c][i];
         int ft0 = st->ft[s * 4 + c];
         int w = 0, r = 0;
-        size_t rb = (size_t)orc_record_bytes(st->bits[c], st->D, st->group);
+        size_t rb = (size_t)orc_record_bytes_fmt(class_fmt(st, c), st->D, st->group);
         uint8_t *moved = st->dense ? malloc(rb * (n - m > 0 ? n - m : 1)) : NULL;
         for (int i = 0; i < n; ++i) {
             if (evict[c][i]) {

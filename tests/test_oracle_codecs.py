@@ -5,12 +5,16 @@ groundwork for a later CUDA path; CPU only.
 FP8 E4M3 is pinned against torch's float8_e4m3fn conversions (a library routine:
 every code's value, round-to-nearest-even on random and half-way inputs); E2M1
 against the OCP table of its eight magnitudes and a brute-force nearest search;
-the group quantisers against their error bounds, exact round trips and hand cases."""
+the group quantisers against their error bounds, exact round trips and hand cases;
+the FP-class records against an independent numpy/torch reading of their layout, and
+attention over an FP-class cache against softmax attention over the decoded records."""
 import numpy as np
 import pytest
 import torch
 
+import synth
 from oracle import oracle as orc
+from tests.helpers import bits_of
 
 # OCP MX: the magnitudes of the E2M1 codes 0..7 (bit 3 is the sign)
 E2M1_TABLE = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
@@ -134,3 +138,110 @@ def test_ternary_scale_is_the_mean_magnitude_above_the_threshold():
         big = np.abs(x) > delta
         assert codes.tolist() == [1 if v > delta else (3 if v < -delta else 0) for v in x]
         assert abs(orc.f16_value(sh) - float(np.abs(x[big]).mean())) <= 2 ** -10 * float(np.abs(x[big]).mean()) + 1e-6
+
+
+# --------------------------------------------------------------------------
+# FP-class records in the cache (codec = 1: classes 1/2/3 = FP8 / NVFP4 / ternary)
+# --------------------------------------------------------------------------
+D = 128
+
+
+def _np_decode_record(fmt, rec):
+    """Independent reading of the documented FP record layouts (numpy + torch)."""
+    rec = np.asarray(rec, np.uint8)
+    out = []
+    for which in range(2):
+        if fmt == orc.FMT_FP8:
+            codes = torch.from_numpy(rec[which * D:(which + 1) * D].copy()).view(torch.float8_e4m3fn).double().numpy()
+            sc = rec[2 * D:2 * D + 16].view(np.float16).astype(np.float64)[which * 4:(which + 1) * 4]
+            out.append(codes * np.repeat(sc, 32))
+        elif fmt == orc.FMT_NVFP4:
+            b = rec[which * 64:(which + 1) * 64]
+            nib = np.stack([b & 15, b >> 4], axis=1).reshape(-1)
+            mag = np.array(E2M1_TABLE)[nib & 7] * np.where(nib & 8, -1.0, 1.0)
+            sc = torch.from_numpy(rec[D + which * 8:D + (which + 1) * 8].copy()).view(torch.float8_e4m3fn).double().numpy()
+            out.append(mag * np.repeat(sc, 16))
+        else:
+            b = rec[which * 32:(which + 1) * 32]
+            codes = np.stack([(b >> (2 * j)) & 3 for j in range(4)], axis=1).reshape(-1)
+            sc = rec[64:80].view(np.float16).astype(np.float64)[which * 4:(which + 1) * 4]
+            out.append(np.select([codes == 1, codes == 3], [1.0, -1.0], 0.0) * np.repeat(sc, 32))
+    return out
+
+
+def test_fp_record_sizes():
+    assert [orc.record_bytes_fmt(f) for f in (orc.FMT_FP8, orc.FMT_NVFP4, orc.FMT_TERNARY)] == [272, 144, 80]
+
+
+@pytest.mark.parametrize("fmt", [108, 104, 102])
+def test_fp_records_decode_as_documented(fmt):
+    for t in range(20):
+        k = synth.normal_bf16(t, 0, synth.TID_K, 1, 1, 0, 1, D)[0, 0, 0] * (1 + 5 * (t % 3))
+        v = synth.normal_bf16(t, 0, synth.TID_V, 1, 1, 0, 1, D)[0, 0, 0]
+        rec = orc.pack_record_fmt(fmt, bits_of(k), bits_of(v))
+        kh, vh = orc.unpack_record_fmt(fmt, rec)
+        nk, nv = _np_decode_record(fmt, rec)
+        assert np.array_equal(kh, nk) and np.array_equal(vh, nv)
+        # codes of each element are those of its own group / block quantiser
+        x = k.float().numpy()
+        if fmt == orc.FMT_FP8:
+            sh, codes = orc.quantize_group_fp8(x[:32])
+            assert np.array_equal(rec[:32], codes)
+        elif fmt == orc.FMT_NVFP4:
+            sc, codes = orc.quantize_block_nvfp4(x[:16])
+            assert rec[D] == sc and np.array_equal(rec[:8], (codes[0::2] & 15) | ((codes[1::2] & 15) << 4))
+
+
+def test_attention_over_fp_class_records_equals_softmax_over_the_decoded_records():
+    B, Hkv, G, ctx = 1, 2, 4, 400
+    cls = synth.class_ids(6, B, ctx, 0.4, 0.4)
+    caps = [ctx] * 4
+    cache = orc.OracleCache(B, Hkv, G, cap=caps, n_protect=4, codec=1)
+    k = synth.normal_bf16(6, 0, synth.TID_K, B, Hkv, 0, ctx, D)
+    v = synth.normal_bf16(6, 0, synth.TID_V, B, Hkv, 0, ctx, D)
+    assert cache.append(bits_of(k), bits_of(v), cls.numpy(), synth.positions(B, 0, ctx).numpy()) == 0
+    q = synth.normal_bf16(6, 0, synth.TID_Q, B, Hkv * G, ctx, 1, D)[:, :, 0]
+    out = cache.attend(bits_of(q), 1 / np.sqrt(D))
+    for s in range(Hkv):
+        K, V = [], []
+        for c in range(4):
+            fmt = orc.class_format(orc.BITS[c], 1)
+            for h in cache.live(s, c)[0]:
+                rec = cache.state[f"pool{c}"][s, h]
+                if fmt == 16:
+                    kh, vh = orc.unpack_record_fmt(16, rec)
+                else:
+                    kh, vh = _np_decode_record(fmt, rec)
+                K.append(kh)
+                V.append(vh)
+        K, V = np.array(K), np.array(V)
+        qd = q[0, s * G:(s + 1) * G].double().numpy()
+        sl = (qd @ K.T) / np.sqrt(D)
+        p = np.exp(sl - sl.max(axis=1, keepdims=True))
+        p /= p.sum(axis=1, keepdims=True)
+        ref = p @ V
+        assert np.max(np.abs(out[0, s * G:(s + 1) * G] - ref)) < 1e-6
+
+
+def test_fp_class_cache_dense_matches_reuse_after_eviction():
+    B, Hkv, G, ctx = 1, 1, 4, 300
+    cls = synth.class_ids(7, B, ctx, 0.4, 0.4)
+    k = synth.normal_bf16(7, 0, synth.TID_K, B, Hkv, 0, ctx, D)
+    v = synth.normal_bf16(7, 0, synth.TID_V, B, Hkv, 0, ctx, D)
+    q = synth.normal_bf16(7, 0, synth.TID_Q, B, Hkv * G, ctx, 1, D)[:, :, 0]
+    caches = []
+    for dense in (False, True):
+        c = orc.OracleCache(B, Hkv, G, cap=[ctx] * 4, n_protect=4, dense=dense, codec=1)
+        assert c.append(bits_of(k), bits_of(v), cls.numpy(), synth.positions(B, 0, ctx).numpy()) == 0
+        c.attend(bits_of(q), 1 / np.sqrt(D))
+        assert c.evict(60) == 0
+        caches.append(c)
+    ct, dn = caches
+    for c in range(4):
+        n = ct.state["n"][0, c]
+        assert dn.state["n"][0, c] == n
+        for i, h in enumerate(ct.state[f"handle{c}"][0, :n]):
+            assert np.array_equal(dn.state[f"pool{c}"][0, i], ct.state[f"pool{c}"][0, h])
+    out_ct = ct.attend(bits_of(q), 1 / np.sqrt(D))
+    out_dn = dn.attend(bits_of(q), 1 / np.sqrt(D))
+    assert np.array_equal(out_ct, out_dn)
