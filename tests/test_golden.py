@@ -1,5 +1,4 @@
 """Golden fixtures: hand-derived record bytes, and a regression snapshot of the oracle."""
-import hashlib
 import json
 import os
 

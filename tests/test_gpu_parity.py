@@ -14,7 +14,7 @@ from oracle import oracle as orc
 from reasoning_model_kv_b200 import TkvCache, TkvError, tkv
 from tests.conftest import gpu_available
 from tests.gpu_harness import (MODES, OUT_ATOL, build_pair, compare_states, np_bits, oracle_for,
-                               rows_streams, score_error)
+                               rows_streams)
 
 pytestmark = [pytest.mark.gpu,
               pytest.mark.skipif(not gpu_available(), reason="needs a CUDA device")]

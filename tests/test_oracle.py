@@ -9,7 +9,6 @@ from itertools import combinations
 
 import numpy as np
 import pytest
-import torch
 
 import synth
 from oracle import oracle as orc
