@@ -101,6 +101,11 @@ def lib():
                                                                                       ctypes.c_double]
         L.orc_evict_tam.restype = ctypes.c_int
         L.orc_num_threads.restype = ctypes.c_int
+        L.orc_attention_sparsity.argtypes = [ctypes.POINTER(_State), ctypes.c_void_p, ctypes.c_float,
+                                             ctypes.c_void_p]
+        L.orc_attention_sparsity.restype = None
+        L.orc_classify_sparsity.argtypes = [ctypes.c_double] * 3
+        L.orc_classify_sparsity.restype = ctypes.c_int
         L.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
         L.orc_e4m3_decode.restype = ctypes.c_double
         L.orc_e4m3_encode.argtypes = [ctypes.c_float]
@@ -243,6 +248,11 @@ def quantize_group_ternary(x):
     return _quantize_scaled(lib().orc_quantize_group_ternary, x, np.uint16)
 
 
+def classify_sparsity(s: float, th_r: float, th_t: float) -> int:
+    """Thought type (3 T, 1 R, 2 E) of a sparsity value under thresholds th_r <= th_t."""
+    return lib().orc_classify_sparsity(float(s), float(th_r), float(th_t))
+
+
 def tbe_schedule(labels, r0: int = 64, t_keep: int = 16) -> np.ndarray:
     """Retention of each thought segment of one batch row (the last one open) under
     the annealing schedule; -1 keeps the whole segment."""
@@ -336,6 +346,14 @@ class OracleCache:
         lib().orc_attend(ctypes.byref(self._st), _ptr(q), float(softmax_scale), _ptr(out),
                          int(s_dbg), pp)
         return (out, p) if s_dbg >= 0 else out
+
+    def attention_sparsity(self, q_bf16: np.ndarray, softmax_scale: float) -> np.ndarray:
+        """1 - H(p) / ln N per stream and query head for the step's query -> [S, G]."""
+        q = np.ascontiguousarray(q_bf16, dtype=np.uint16)
+        assert q.shape == (self.B, self.Hkv * self.G, self.D)
+        out = np.zeros((self.S, self.G), dtype=np.float64)
+        lib().orc_attention_sparsity(ctypes.byref(self._st), _ptr(q), float(softmax_scale), _ptr(out))
+        return out
 
     def evict(self, budget: int) -> int:
         return lib().orc_evict(ctypes.byref(self._st), int(budget))

@@ -926,6 +926,62 @@ int orc_tbe_schedule(const uint8_t *label, int nseg, int r0, int t_keep, int32_t
     return ORC_OK;
 }
 
+/* Attention sparsity of one decode step (the ThinKV page, Metodologia: thought
+ * types differ in the sparsity of their attention weights -- Transition the
+ * sparsest, then Reasoning, Execution the least).  The page gives no measure;
+ * reading used here: for every stream s and query head j, with p the step's
+ * softmax over the stream's N live tokens (as orc_attend computes it, scores not
+ * touched), sparsity = 1 - H(p) / ln N with H(p) = -sum p ln p (fp64): 0 for
+ * uniform attention, 1 for attention on one token; 0 when N < 2.
+ * out: [S][G]. */
+void orc_attention_sparsity(orc_state *st, const uint16_t *q, float softmax_scale, double *out) {
+    const int D = st->D, G = st->G, S = n_streams(st);
+    const int Hq = st->Hkv * G;
+    for (int s = 0; s < S; ++s) {
+        const int b = s / st->Hkv, kvh = s % st->Hkv;
+        int N = 0;
+        for (int c = 0; c < 4; ++c) N += st->n[s * 4 + c];
+        if (N < 2) {
+            for (int j = 0; j < G; ++j) out[(size_t)s * G + j] = 0.0;
+            continue;
+        }
+        double *logit = malloc(sizeof(double) * (size_t)G * N);
+        double *kh = malloc(sizeof(double) * D), *vh = malloc(sizeof(double) * D);
+        int t = 0;
+        for (int c = 0; c < 4; ++c)
+            for (int i = 0; i < st->n[s * 4 + c]; ++i, ++t) {
+                const size_t e = (size_t)s * st->cap[c] + i;
+                orc_unpack_record_fmt(class_fmt(st, c), D, st->group, record_ptr(st, s, c, st->handle[c][e]),
+                                      kh, vh);
+                for (int j = 0; j < G; ++j) {
+                    double acc = 0.0;
+                    for (int d = 0; d < D; ++d)
+                        acc += (double)bf16_to_f32(q[((size_t)b * Hq + kvh * G + j) * D + d]) * kh[d];
+                    logit[(size_t)j * N + t] = acc * (double)softmax_scale;
+                }
+            }
+        for (int j = 0; j < G; ++j) {
+            const double *x = logit + (size_t)j * N;
+            double m = x[0];
+            for (int u = 1; u < N; ++u) m = x[u] > m ? x[u] : m;
+            double z = 0.0;
+            for (int u = 0; u < N; ++u) z += exp(x[u] - m);
+            double h = 0.0;   /* H = ln z - sum p (x - m) */
+            for (int u = 0; u < N; ++u) h -= exp(x[u] - m) / z * (x[u] - m);
+            h += log(z);
+            out[(size_t)s * G + j] = 1.0 - h / log((double)N);
+        }
+        free(logit); free(kh); free(vh);
+    }
+}
+
+/* Thought type from a sparsity value with thresholds th_r <= th_t (parameters: the
+ * page gives none): 3 (Transition) when s >= th_t, 1 (Reasoning) when s >= th_r,
+ * else 2 (Execution). */
+int orc_classify_sparsity(double s, double th_r, double th_t) {
+    return s >= th_t ? 3 : (s >= th_r ? 1 : 2);
+}
+
 int orc_num_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();

@@ -245,3 +245,46 @@ def test_fp_class_cache_dense_matches_reuse_after_eviction():
     out_ct = ct.attend(bits_of(q), 1 / np.sqrt(D))
     out_dn = dn.attend(bits_of(q), 1 / np.sqrt(D))
     assert np.array_equal(out_ct, out_dn)
+
+
+# --------------------------------------------------------------------------
+# attention sparsity of a step (ThinKV, Metodologia: thought types differ in the
+# sparsity of their attention); measure 1 - H(p) / ln N
+# --------------------------------------------------------------------------
+def _bf16_cache_with_key_column(col0):
+    """All-bf16 cache whose keys are zero except dimension 0 = col0 (exact in bf16)."""
+    N = len(col0)
+    cache = orc.OracleCache(1, 1, 1, cap=[N, 0, 0, 0], n_protect=N)
+    k = torch.zeros((1, 1, N, D), dtype=torch.bfloat16)
+    k[0, 0, :, 0] = torch.tensor(col0, dtype=torch.float32).to(torch.bfloat16)
+    v = torch.zeros_like(k)
+    assert cache.append(bits_of(k), bits_of(v), np.ones((1, N), np.uint8),
+                        np.arange(N, dtype=np.int32).reshape(1, N)) == 0
+    q = torch.zeros((1, 1, D), dtype=torch.bfloat16)
+    q[0, 0, 0] = 1.0
+    return cache, bits_of(q)
+
+
+def test_sparsity_uniform_attention_is_zero():
+    cache, q = _bf16_cache_with_key_column([2.0] * 50)
+    assert abs(cache.attention_sparsity(q, 1.0)[0, 0]) < 1e-12
+
+
+@pytest.mark.parametrize("m,N,a,b", [(1, 10, 3.0, 0.0), (5, 40, 1.0, -2.0), (30, 64, 0.5, 0.25)])
+def test_sparsity_two_level_closed_form(m, N, a, b):
+    cache, q = _bf16_cache_with_key_column([a] * m + [b] * (N - m))
+    z = m * np.exp(a) + (N - m) * np.exp(b)
+    ph, pl = np.exp(a) / z, np.exp(b) / z
+    H = -(m * ph * np.log(ph) + (N - m) * pl * np.log(pl))
+    assert abs(cache.attention_sparsity(q, 1.0)[0, 0] - (1 - H / np.log(N))) < 1e-12
+
+
+def test_sparsity_one_dominant_token_and_degenerate_sizes():
+    cache, q = _bf16_cache_with_key_column([40.0] + [0.0] * 99)
+    assert cache.attention_sparsity(q, 1.0)[0, 0] > 0.99
+    cache, q = _bf16_cache_with_key_column([1.0])
+    assert cache.attention_sparsity(q, 1.0)[0, 0] == 0.0
+
+
+def test_sparsity_classification_thresholds():
+    assert [orc.classify_sparsity(s, 0.3, 0.6) for s in (0.0, 0.29, 0.3, 0.59, 0.6, 1.0)] == [2, 2, 1, 1, 3, 3]
