@@ -107,10 +107,20 @@ typedef struct tkv_cache tkv_cache;
  *   score_c[s*cap_c + i]            float: accumulated attention mass of entry i
  *   fs_c[s*cap_c + j]               int32: free stack of slots (j < ft; top = j = ft-1)
  *   pool_c[(s*cap_c + slot)*rec_bytes_c]  packed record of a slot:
- *     bf16 class: [K: D bf16][V: D bf16]                                 (512 bytes)
+ *     bf16 class: [K block: D bf16][V block: D bf16]                     (512 bytes)
  *     b-bit class: [K codes D*b/8][V codes D*b/8][K scale x4][K zero x4]
  *                  [V scale x4][V zero x4]  (fp16, little-endian)        (288/160/96 bytes)
- *     element i of a code block sits at bit b*(i % (8/b)) of byte i*b/8.
+ *     Scale and zero of group g (head dims 32g..32g+31) are entry g of their x4.
+ *   Element order inside a K or V block (b = 16 for bf16, else the class's bits):
+ *   the block is four quarters of 4*b bytes (quarter q = bytes [4bq, 4b(q+1)));
+ *   a quarter is b little-endian 32-bit words; word w of a quarter holds the
+ *   16/b head-dim pairs p = w*(16/b) + j, j = 0 .. 16/b - 1, with the pair's first
+ *   member in bits [b*j, b*j + b) and its second member 16 bits higher, in bits
+ *   [b*j + 16, b*j + 16 + b).  Pair p of quarter q holds head dims
+ *     K block: 32*(p/4) + 8*q + 2*(p%4) + {0, 1}
+ *     V block: 8*p + 2*q + {0, 1}
+ *   (first member = the even dim).  Example (K, b = 8): byte 0 of the block holds
+ *   dim 0, byte 1 dim 2, byte 2 dim 1, byte 3 dim 3, byte 4 dim 4, byte 8 dim 32.
  * The state region [0, state_bytes) holds all of the above; the rest of the
  * workspace is scratch. */
 typedef struct {
@@ -172,7 +182,9 @@ TKV_API tkv_status tkv_quantize_append(tkv_cache *cache, const void *k, const vo
  *   Limit: B * (T + 4) <= 524288 when T > 1 (T == 1 needs no scratch);
  *          larger appends return TKV_ERR_INVALID and launch nothing.
  *   The first call on each device looks up the array's device address (with
- *   that device current); make that first call before any stream capture.
+ *   that device current) and keeps it for that device's current context; make
+ *   that first call before any stream capture, and do not use this entry point
+ *   after cudaDeviceReset in the same process.
  *   All calls share the one array and each call rewrites what it uses, so calls
  *   that overlap on the GPU (two streams, or two caches at once) race.
  */
@@ -272,7 +284,12 @@ TKV_API tkv_status tkv_tbe_schedule(const uint8_t *label, int32_t nseg, int32_t 
 TKV_API tkv_status tkv_poll_error(tkv_cache *cache, void *stream);
 
 /* Copy the state region (see tkv_layout) to / from a host buffer of
- * state_bytes bytes.  Both synchronise `stream`. */
+ * state_bytes bytes (the buffer is the caller's; the state is the cache's
+ * checkpoint: counters, tables, scores, free stacks and records).  Both
+ * synchronise `stream`.  Import also derives the host-side launch bound (the
+ * largest stream's entry count) from the imported counters, so a cache restored
+ * from a checkpoint launches exactly as the cache it was taken from would after
+ * the same import.  Returns TKV_ERR_INVALID for NULL arguments. */
 TKV_API tkv_status tkv_export_state(tkv_cache *cache, void *host_dst, void *stream);
 TKV_API tkv_status tkv_import_state(tkv_cache *cache, const void *host_src, void *stream);
 

@@ -545,30 +545,20 @@ __global__ void __launch_bounds__(kThreads, TKV_ATTN_MIN_BLOCKS) attn_kernel(con
     if (C > 1) cluster_sync();   // peers may still be reading this CTA's shared memory
 }
 
-int g_blocks_per_sm[2][kMaxG + 1] = {};
-int g_sms = 0;
+int g_blocks_per_sm[2][kMaxG + 1][kMaxDevices] = {};   // per placement, G and device
 
 template <int G, bool DENSE>
 cudaError_t launch_g(const Dev &d, const void *q, float scale, float *out, long long live_ub,
                      cudaStream_t st, int64_t *launches) {
-    if (g_sms == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&g_sms, cudaDevAttrMultiProcessorCount, dev);
-    }
-    int &bps = g_blocks_per_sm[DENSE][G];
-    if (bps == 0) {
-        cudaError_t e = cudaFuncSetAttribute(attn_kernel<G, DENSE>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, kRingBytes);
-        if (e != cudaSuccess) return e;
-        int nb = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, attn_kernel<G, DENSE>, kThreads, kRingBytes);
-        if (e != cudaSuccess) return e;
-        bps = nb > 0 ? nb : 1;
-    }
+    int sms = 0, bps = 0;
+    cudaError_t e0 = device_sm_count(&sms);
+    if (e0 != cudaSuccess) return e0;
+    e0 = cached_blocks_per_sm(g_blocks_per_sm[DENSE][G], reinterpret_cast<const void *>(attn_kernel<G, DENSE>),
+                              kThreads, kRingBytes, &bps);
+    if (e0 != cudaSuccess) return e0;
     // Largest cluster (<= 8) whose grid is fully resident, never splitting a stream
     // below ~128 tokens per CTA; one CTA per stream when the streams fill the GPU.
-    const long long slots = (long long)bps * g_sms;
+    const long long slots = (long long)bps * sms;
     long long C = slots / d.S;
     if (C > kMaxCluster) C = kMaxCluster;
     if (C > live_ub / 128) C = live_ub / 128;

@@ -15,7 +15,10 @@
 // library holds it until the process exits.  Host code must not use the array's
 // name as a device address: the first call on each device looks the address up
 // with cudaGetSymbolAddress (with that device current) and caches it, so that
-// first call should be made before any stream capture begins.
+// first call should be made before any stream capture begins.  The cached address
+// is valid only for the device context that was current at that first call: a
+// process that calls cudaDeviceReset (or otherwise tears the primary context down
+// and creates it again) must not use this entry point afterwards.
 #include <cuda_runtime.h>
 
 #include <mutex>

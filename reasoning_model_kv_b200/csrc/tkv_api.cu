@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
+#include <mutex>
 #include <climits>
 #include <cmath>
 #include <cstdio>
@@ -133,6 +135,49 @@ void note_append(tkv_cache *c, int64_t launches, int T) {
     c->live_ub = std::min<long long>(c->dev.ncap, c->live_ub + T);
 }
 tkv_status api_fail(tkv_status st, const std::string &msg) { return fail(st, msg); }
+
+namespace {
+std::atomic<int> g_sm_count[kMaxDevices];
+std::mutex g_occ_mu;
+}  // namespace
+
+cudaError_t device_sm_count(int *sms) {
+    *sms = 0;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    int v = g_sm_count[dev].load(std::memory_order_relaxed);
+    if (v == 0) {
+        e = cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        g_sm_count[dev].store(v, std::memory_order_relaxed);
+    }
+    *sms = v;
+    return cudaSuccess;
+}
+
+cudaError_t cached_blocks_per_sm(int *slot_per_device, const void *kernel, int threads, size_t smem,
+                                 int *blocks) {
+    *blocks = 0;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_occ_mu);
+    if (slot_per_device[dev] == 0) {
+        if (smem > 48 * 1024) {
+            e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+        }
+        int nb = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kernel, threads, smem);
+        if (e != cudaSuccess) return e;
+        slot_per_device[dev] = nb > 0 ? nb : 1;
+    }
+    *blocks = slot_per_device[dev];
+    return cudaSuccess;
+}
 }  // namespace tkv
 
 extern "C" {
@@ -306,7 +351,15 @@ tkv_status tkv_import_state(tkv_cache *c, const void *host_src, void *stream) {
     auto st = static_cast<cudaStream_t>(stream);
     cudaError_t e = cudaMemcpyAsync(c->base, host_src, c->lay.state_bytes, cudaMemcpyHostToDevice, st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
-    c->live_ub = c->dev.ncap;
+    // the live-entry bound from the imported counters: the largest stream's entry count
+    const int32_t *n = reinterpret_cast<const int32_t *>(static_cast<const uint8_t *>(host_src) + c->lay.n);
+    long long ub = 0;
+    for (int s = 0; s < c->dev.S; ++s) {
+        long long tot = 0;
+        for (int k = 0; k < 4; ++k) tot += std::max<int32_t>(0, std::min(n[s * 4 + k], c->cfg.cap[k]));
+        ub = std::max(ub, tot);
+    }
+    c->live_ub = ub;
     return cuda_status(e, "tkv_import_state");
 }
 

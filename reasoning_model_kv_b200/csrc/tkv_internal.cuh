@@ -44,6 +44,16 @@ __device__ __forceinline__ void raise_error(uint32_t *err, uint32_t code, uint32
     atomicAdd(err + 1, 1u);
 }
 
+// Host-side per-device facts, looked up once per device and thread-safe (racing
+// first calls compute and store the same value).
+constexpr int kMaxDevices = 64;
+// SM count of the current device; 0 (and the CUDA error) if it cannot be read.
+cudaError_t device_sm_count(int *sms);
+// Resident CTAs per SM of `kernel` with `threads` threads and `smem` dynamic shared
+// bytes on the current device, cached in slot[device] (0 means "not yet known").
+cudaError_t cached_blocks_per_sm(int *slot_per_device, const void *kernel, int threads, size_t smem,
+                                 int *blocks);
+
 // Launchers (each returns the CUDA error of its launches and adds the number
 // of kernels it launched to *launches).
 cudaError_t launch_append(const Dev &d, const void *k, const void *v, const uint8_t *cls,

@@ -10,6 +10,7 @@ from __future__ import annotations
 import ctypes
 from pathlib import Path
 
+import numpy as np
 import torch
 
 LIB_PATH = Path(__file__).resolve().parent / "libtkv.so"
@@ -284,21 +285,58 @@ class TkvCache:
             out[f"pool{c}"] = ws[L.pool[c]:L.pool[c] + S * cc * rb].view(S, cc, rb)
         return out
 
+    def _state_arrays(self, buf: np.ndarray) -> dict:
+        """Numpy views of the state arrays inside a host copy of the state region
+        (the tkv_layout offsets; same keys and shapes as state_views)."""
+        L = self.layout
+        S = self.S
+
+        def view(off, count, dtype, shape):
+            nbytes = count * np.dtype(dtype).itemsize
+            return buf[off:off + nbytes].view(dtype).reshape(shape)
+
+        out = {"n": view(L.n, S * 4, np.int32, (S, 4)),
+               "ft": view(L.ft, S * 4, np.int32, (S, 4)),
+               "hw": view(L.hw, S * 4, np.int32, (S, 4))}
+        for c in range(4):
+            cc = self.cap[c]
+            out[f"handle{c}"] = view(L.handle[c], S * cc, np.int32, (S, cc))
+            out[f"pos{c}"] = view(L.pos[c], S * cc, np.int32, (S, cc))
+            out[f"score{c}"] = view(L.score[c], S * cc, np.float32, (S, cc))
+            out[f"fs{c}"] = view(L.fs[c], S * cc, np.int32, (S, cc))
+            rb = L.rec_bytes[c]
+            out[f"pool{c}"] = view(L.pool[c], S * cc * rb, np.uint8, (S, cc, rb))
+        return out
+
     def export_state(self, streams=None) -> dict:
-        """Host (numpy) copy of the state, optionally of a subset of streams."""
+        """Host (numpy) copy of the state.  The whole state goes through the C ABI's
+        tkv_export_state (one copy of the state region); a subset of streams is read
+        through device views of the workspace instead, which avoids copying every
+        stream of a large cache to the host."""
+        if streams is None:
+            buf = np.empty(self.layout.state_bytes, dtype=np.uint8)
+            _check(lib().tkv_export_state(self._h, buf.ctypes.data, _stream()))
+            return self._state_arrays(buf)
         torch.cuda.current_stream().synchronize()
         v = self.state_views()
-        if streams is None:
-            return {k: t.cpu().numpy() for k, t in v.items()}
         idx = torch.as_tensor(list(streams), device=self.workspace.device)
         return {k: t.index_select(0, idx).cpu().numpy() for k, t in v.items()}
 
     def import_state(self, state: dict):
-        v = self.state_views()
+        """Load state arrays (all streams; keys as export_state returns them) through
+        the C ABI's tkv_import_state.  Keys that are absent keep their current
+        contents."""
+        buf = np.empty(self.layout.state_bytes, dtype=np.uint8)
+        _check(lib().tkv_export_state(self._h, buf.ctypes.data, _stream()))
+        arrs = self._state_arrays(buf)
         for k, arr in state.items():
-            if k in v:
-                v[k].copy_(torch.as_tensor(arr).view(v[k].dtype).reshape(v[k].shape))
-        torch.cuda.current_stream().synchronize()
+            if k not in arrs:
+                raise TkvError(TKV_ERR_INVALID, f"unknown state array {k}")
+            a = np.asarray(arr)
+            if a.shape != arrs[k].shape:
+                raise TkvError(TKV_ERR_INVALID, f"{k} must have shape {arrs[k].shape}, got {a.shape}")
+            arrs[k][...] = a.view(arrs[k].dtype) if a.dtype.itemsize == arrs[k].dtype.itemsize else a
+        _check(lib().tkv_import_state(self._h, buf.ctypes.data, _stream()))
 
 
 # Module-level aliases with the C ABI's names.
