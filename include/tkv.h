@@ -89,11 +89,13 @@ typedef struct {
                             i) and decode reads them as whole blocks.  Results
                             are identical in both modes.                      */
     int32_t attn_kernel; /* decode-attention kernel: 0 = warp-tile kernel
-                            (mma.sync fragments, either placement; the
-                            default); 1 = tensor-memory kernel (tcgen05 MMAs
-                            with accumulators in tensor memory, one thread per
-                            token row; dense placement only).  Both compute the
-                            same result within the stated tolerances.         */
+                            (mma.sync fragments, either placement);
+                            1 = tensor-core kernel (tcgen05 MMAs with integer
+                            operands: exact code products, accumulators in
+                            tensor memory; persistent, one CTA per SM with the
+                            step's bytes split evenly; dense placement only).
+                            Both compute the same result within the stated
+                            tolerances.                                       */
 } tkv_config;
 
 typedef struct tkv_cache tkv_cache;
@@ -203,6 +205,26 @@ TKV_API tkv_status tkv_quantize_append_noalloc(tkv_cache *cache, const void *k, 
  */
 TKV_API tkv_status tkv_decode_attention(tkv_cache *cache, const void *q, float softmax_scale,
                                 float *out, void *stream);
+
+/*
+ * tkv_decode_attention plus, per (stream, query head), the attention sparsity of
+ * this step and the thought type it indicates (ThinKV page, "Metodologia": the
+ * thought types differ in how sparse their attention is -- Transition the most,
+ * Execution the least).  The page gives no measure and no thresholds; this library
+ * uses the normalised entropy of the step's softmax over the stream's N live tokens:
+ *   sparsity = 1 - H(p) / ln N,   H(p) = -sum_t p_t ln p_t   (0 when N < 2),
+ * which is 0 for uniform attention and 1 for attention on one token, and the class
+ *   3 (Transition) if sparsity >= th_t, else 1 (Reasoning) if sparsity >= th_r,
+ *   else 2 (Execution).
+ *   sparsity  device fp32 [B][Hkv*G]  (required)
+ *   thought   device uint8 [B][Hkv*G] (may be NULL)
+ * Requires dense placement with attn_kernel = 1 (the statistic is formed by that
+ * kernel's softmax); returns TKV_ERR_INVALID otherwise, for NULL q / out / sparsity,
+ * unaligned pointers, or thresholds that are not finite with th_r <= th_t.
+ */
+TKV_API tkv_status tkv_decode_attention_sparsity(tkv_cache *cache, const void *q, float softmax_scale,
+                                                 float *out, float *sparsity, uint8_t *thought, float th_r,
+                                                 float th_t, void *stream);
 
 /*
  * Budgeted top-k eviction and table compaction, per stream.

@@ -21,7 +21,7 @@ ROOT = PKG.parent
 CSRC = PKG / "csrc"
 LIB = PKG / "libtkv.so"
 LIB_DEBUG = PKG / "libtkv_debug.so"
-SOURCES = ["tkv_api.cu", "append.cu", "attention.cu", "attention_tc.cu", "evict.cu", "noalloc.cu", "selftest.cu",
+SOURCES = ["tkv_api.cu", "append.cu", "attention.cu", "attention_i8.cu", "evict.cu", "noalloc.cu", "selftest.cu",
            "evict_segments.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 

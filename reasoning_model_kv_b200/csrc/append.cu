@@ -218,9 +218,13 @@ __global__ void __launch_bounds__(256) append_pack_kernel(
     const int sc = s * 4 + c;
     const int cap = d.cap[c];
     const int ft = pick4(ft4, c), hw = pick4(hw4, c), n = pick4(n4, c);
+    if (!dcheck(d.err, n >= 0 && n + r < cap && ft >= 0 && ft <= cap && hw >= 0 && hw <= cap && r >= 0,
+                kDbgAppend + c))
+        return;
     int slot;
     if (r < ft) {
         slot = d.fs[c][(size_t)s * cap + ft - 1 - r];
+        if (!dcheck(d.err, slot >= 0 && slot < cap, kDbgAppend + 0x10 + c)) return;
     } else {
         slot = hw + (r - ft);
         if (slot >= cap) {

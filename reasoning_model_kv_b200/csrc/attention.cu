@@ -26,7 +26,9 @@
 //   O[d][h] += V^T[d][t] . (P * vscale)[t][h]   M = 16 dims, N = 8 heads, K = 16
 //            tokens, plus sum_t p * vzero per group (fp32, outside the MMA).
 // Integer codes are exact in f16 (magic-number conversion, 1-2 ALU ops per pair);
-// bf16 keys/values and queries convert exactly to f16 in its normal range.  The
+// the query is f16 too, each (group, head) scaled by a power of two into f16's range
+// when needed.  bf16 tiles use bf16 MMAs on the raw keys, values and query (P as a
+// bf16 high part plus the bf16 of the remainder), so nothing is narrowed.  The
 // record storage order puts each lane's operand pairs 16 bits apart in one word,
 // so a row's quarter loads with one or two 16-byte shared-memory reads; the V
 // operand and P are transposed in registers with movmatrix.  The running max is
@@ -74,7 +76,8 @@ struct WarpState {
 // are masked to -inf, so they contribute p = 0 everywhere.
 template <int BITS, int ROWS, int STRIDE, int G, bool SWZ>
 __device__ __forceinline__ void tile_compute(const uint8_t *st, int nr, int lane,
-                                             const uint32_t (&qb)[4][2][2], const float (&qs)[2][4],
+                                             const uint32_t (&qb)[4][2][2], const uint32_t (&qbb)[4][2][2],
+                                             const float (&qs)[2][4], const float (&qinv)[2][4], bool qscaled,
                                              float xscale, WarpState &ws, float *lg, uint32_t magic) {
     const int g = lane >> 2, tig = lane & 3;
     constexpr int QB = 4 * BITS;     // bytes of one quarter of a code block
@@ -105,10 +108,10 @@ __device__ __forceinline__ void tile_compute(const uint8_t *st, int nr, int lane
             load_meta(r0 + km_off0, km0);
             load_meta(r1 + km_off1, km1);
         }
-        qk_group<BITS, 0>(x, k0, k1, qb, qs, km0, km1, magic);
-        qk_group<BITS, 1>(x, k0, k1, qb, qs, km0, km1, magic);
-        qk_group<BITS, 2>(x, k0, k1, qb, qs, km0, km1, magic);
-        qk_group<BITS, 3>(x, k0, k1, qb, qs, km0, km1, magic);
+        qk_group<BITS, 0>(x, k0, k1, qb, qbb, qs, qinv, qscaled, km0, km1, magic);
+        qk_group<BITS, 1>(x, k0, k1, qb, qbb, qs, qinv, qscaled, km0, km1, magic);
+        qk_group<BITS, 2>(x, k0, k1, qb, qbb, qs, qinv, qscaled, km0, km1, magic);
+        qk_group<BITS, 3>(x, k0, k1, qb, qbb, qs, qinv, qscaled, km0, km1, magic);
     }
     const bool h0 = 2 * tig < G, h1 = 2 * tig + 1 < G;
     x[0] = (v0 && h0) ? x[0] * xscale : -INFINITY;
@@ -156,11 +159,24 @@ __device__ __forceinline__ void tile_compute(const uint8_t *st, int nr, int lane
     ws.l[0] += p[0] + p[2];
     ws.l[1] += p[1] + p[3];
 
-    // ---- phase 2: O += V^T . (P * vscale) per group; zero term accumulated apart
+    // ---- phase 2: O += V^T . (P * vscale) per group; zero term accumulated apart.
+    //      bf16 values: bf16 MMAs with P split into a bf16 high part and the bf16 of
+    //      the remainder (two MMAs), so P keeps ~16 bits and V is never narrowed
     uint32_t bfr[4][2];
+    uint32_t blo0 = 0u, blo1 = 0u;
     if constexpr (BITS == 16) {
-        const uint32_t b0 = transpose8x8(f32x2_to_f16x2(p[0], p[1]));
-        const uint32_t b1 = ROWS == 16 ? transpose8x8(f32x2_to_f16x2(p[2], p[3])) : 0u;
+        const uint32_t h01 = f32x2_to_bf16x2(p[0], p[1]);
+        const uint32_t l01 = f32x2_to_bf16x2(p[0] - __uint_as_float(h01 << 16), p[1] - __uint_as_float(h01 & 0xffff0000u));
+        const uint32_t b0 = transpose8x8(h01);
+        blo0 = transpose8x8(l01);
+        uint32_t b1 = 0u;
+        if constexpr (ROWS == 16) {
+            const uint32_t h23 = f32x2_to_bf16x2(p[2], p[3]);
+            const uint32_t l23 =
+                f32x2_to_bf16x2(p[2] - __uint_as_float(h23 << 16), p[3] - __uint_as_float(h23 & 0xffff0000u));
+            b1 = transpose8x8(h23);
+            blo1 = transpose8x8(l23);
+        }
 #pragma unroll
         for (int grp = 0; grp < 4; ++grp) { bfr[grp][0] = b0; bfr[grp][1] = b1; }
     } else {
@@ -189,7 +205,12 @@ __device__ __forceinline__ void tile_compute(const uint8_t *st, int nr, int lane
         const uint32_t e1 = transpose8x8(quarter_pair<BITS, 2 * (MT) + 1>(w0, magic));                   \
         const uint32_t e2 = ROWS == 16 ? transpose8x8(quarter_pair<BITS, 2 * (MT)>(w1, magic)) : 0u;     \
         const uint32_t e3 = ROWS == 16 ? transpose8x8(quarter_pair<BITS, 2 * (MT) + 1>(w1, magic)) : 0u; \
-        mma16816(ws.o[MT], e0, e1, e2, e3, bfr[(MT) >> 1][0], bfr[(MT) >> 1][1]);                 \
+        if constexpr (BITS == 16) {                                                               \
+            mma16816_bf16(ws.o[MT], e0, e1, e2, e3, bfr[(MT) >> 1][0], bfr[(MT) >> 1][1]);        \
+            mma16816_bf16(ws.o[MT], e0, e1, e2, e3, blo0, blo1);                                  \
+        } else {                                                                                  \
+            mma16816(ws.o[MT], e0, e1, e2, e3, bfr[(MT) >> 1][0], bfr[(MT) >> 1][1]);             \
+        }                                                                                         \
     }
     TKV_VMMA(0) TKV_VMMA(1) TKV_VMMA(2) TKV_VMMA(3) TKV_VMMA(4) TKV_VMMA(5) TKV_VMMA(6) TKV_VMMA(7)
 #undef TKV_VMMA
@@ -267,40 +288,76 @@ __global__ void __launch_bounds__(kThreads, TKV_ATTN_MIN_BLOCKS) attn_kernel(con
     const int b = s / d.Hkv, kvh = s - b * d.Hkv;
 
     // ---- query operand (B of S = K Q^T; independent of the previous kernel, so it is
-    //      loaded before the dependency wait): head g, dims 32grp + 8tig + 4hh + 0..3
-    uint32_t qb[4][2][2];
-    float qs[2][4];
+    //      loaded before the dependency wait): head g, dims 32grp + 8tig + 4hh + 0..3.
+    //      qbb: the raw bf16 pairs (bf16 keys); qb: f16 pairs for the integer codes,
+    //      each (group, head) scaled by a power of two when its largest |q| lies
+    //      outside [2^-10, 2^14) so that f16 neither overflows nor goes subnormal on
+    //      it; qinv holds the inverse scale of heads 2tig, 2tig+1 per group.
+    uint32_t qb[4][2][2], qbb[4][2][2];
+    float qs[2][4], qinv[2][4];
+    bool qscaled;
     {
-        float qsg[4];
+        float qsg[4], qsc[4];
         const __nv_bfloat16 *qr = q + ((size_t)b * d.Hkv * G + (size_t)kvh * G + (g < G ? g : 0)) * kD;
+        uint2 raw[4][2];
 #pragma unroll
-        for (int grp = 0; grp < 4; ++grp) {
-            float sum = 0.f;
+        for (int grp = 0; grp < 4; ++grp)
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
-                uint2 raw = make_uint2(0u, 0u);
-                if (g < G) raw = *reinterpret_cast<const uint2 *>(qr + 32 * grp + 8 * tig + 4 * hh);
-                const float f0 = __uint_as_float(raw.x << 16), f1 = __uint_as_float(raw.x & 0xffff0000u);
-                const float f2 = __uint_as_float(raw.y << 16), f3 = __uint_as_float(raw.y & 0xffff0000u);
-                qb[grp][hh][0] = f32x2_to_f16x2(f0, f1);
-                qb[grp][hh][1] = f32x2_to_f16x2(f2, f3);
+                raw[grp][hh] = make_uint2(0u, 0u);
+                if (g < G) raw[grp][hh] = *reinterpret_cast<const uint2 *>(qr + 32 * grp + 8 * tig + 4 * hh);
+            }
+        bool any = false;
+#pragma unroll
+        for (int grp = 0; grp < 4; ++grp) {
+            float sum = 0.f, mx = 0.f;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const uint2 r2 = raw[grp][hh];
+                const float f0 = __uint_as_float(r2.x << 16), f1 = __uint_as_float(r2.x & 0xffff0000u);
+                const float f2 = __uint_as_float(r2.y << 16), f3 = __uint_as_float(r2.y & 0xffff0000u);
                 sum += (f0 + f1) + (f2 + f3);
+                mx = fmaxf(mx, fmaxf(fmaxf(fabsf(f0), fabsf(f1)), fmaxf(fabsf(f2), fabsf(f3))));
             }
             sum += __shfl_xor_sync(kFull, sum, 1);
             sum += __shfl_xor_sync(kFull, sum, 2);
+            mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
             qsg[grp] = sum;                              // sum over group grp of q[head g]
+            // scale 2^(13 - floor(log2 mx)) puts the largest |q| in [2^13, 2^14)
+            float sc = 1.f;
+            if (mx >= 16384.f || (mx > 0.f && mx < 0.0009765625f)) {
+                const int e = (int)((__float_as_uint(mx) >> 23) & 0xff) - 127;
+                sc = __uint_as_float((uint32_t)(127 + 13 - e) << 23);
+                any = true;
+            }
+            qsc[grp] = sc;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const uint2 r2 = raw[grp][hh];
+                qbb[grp][hh][0] = r2.x;
+                qbb[grp][hh][1] = r2.y;
+                qb[grp][hh][0] = f32x2_to_f16x2(__uint_as_float(r2.x << 16) * sc, __uint_as_float(r2.x & 0xffff0000u) * sc);
+                qb[grp][hh][1] = f32x2_to_f16x2(__uint_as_float(r2.y << 16) * sc, __uint_as_float(r2.y & 0xffff0000u) * sc);
+            }
         }
 #pragma unroll
         for (int grp = 0; grp < 4; ++grp) {
             qs[0][grp] = __shfl_sync(kFull, qsg[grp], (2 * tig) * 4);
             qs[1][grp] = __shfl_sync(kFull, qsg[grp], (2 * tig + 1) * 4);
+            qinv[0][grp] = 1.f / __shfl_sync(kFull, qsc[grp], (2 * tig) * 4);
+            qinv[1][grp] = 1.f / __shfl_sync(kFull, qsc[grp], (2 * tig + 1) * 4);
         }
+        qscaled = __any_sync(kFull, any);
     }
 
     grid_dependency_wait();   // the append's counters and records are visible from here
 
     // ---- this CTA's entry range and its tiles (class by class)
-    const int n0 = d.n[s * 4 + 0], n1 = d.n[s * 4 + 1], n2 = d.n[s * 4 + 2], n3 = d.n[s * 4 + 3];
+    const int n0 = dclamp(d.err, d.n[s * 4 + 0], d.cap[0], kDbgAttention + 0);
+    const int n1 = dclamp(d.err, d.n[s * 4 + 1], d.cap[1], kDbgAttention + 1);
+    const int n2 = dclamp(d.err, d.n[s * 4 + 2], d.cap[2], kDbgAttention + 2);
+    const int n3 = dclamp(d.err, d.n[s * 4 + 3], d.cap[3], kDbgAttention + 3);
     const int o1 = n0, o2 = o1 + n1, o3 = o2 + n2, N = o3 + n3;
     const int chunk = ((N + C - 1) / C + 31) & ~31;
     const int t0 = min(N, rank * chunk), t1 = min(N, t0 + chunk);
@@ -352,7 +409,8 @@ __global__ void __launch_bounds__(kThreads, TKV_ATTN_MIN_BLOCKS) attn_kernel(con
         } else {
             if (dsc < 0) return 0;
             const int e = dsc & 0xffffff, nr = (dsc >> 24) & 31, c = dsc >> 29;
-            return d.handle[c][(size_t)s * d.cap[c] + e + min(lane, nr - 1)];
+            const int h = d.handle[c][(size_t)s * d.cap[c] + e + min(lane, nr - 1)];
+            return dclamp(d.err, h, d.cap[c] - 1, kDbgAttention + 0x10 + c);
         }
     };
     auto issue = [&](int dsc, int stage, int hd) {
@@ -421,7 +479,7 @@ __global__ void __launch_bounds__(kThreads, TKV_ATTN_MIN_BLOCKS) attn_kernel(con
         const int e = (LO) + (T - (PLO)) * (ROWS);                                            \
         const int nr = min((ROWS), (HI) - e);                                                 \
         tile_compute<BITS, ROWS, STRIDE, G, !DENSE>(ring + (warp * kStages + stage) * kStageBytes, \
-                                                    nr, lane, qb, qs, xscale, ws,             \
+                                                    nr, lane, qb, qbb, qs, qinv, qscaled, xscale, ws, \
                                                     lgs + (size_t)((OFF) + e) * G, magic);    \
         __syncwarp();                                                                         \
         stage = stage == 2 ? 0 : stage + 1;                                                   \
@@ -588,7 +646,8 @@ cudaError_t launch_g(const Dev &d, const void *q, float scale, float *out, long 
 
 cudaError_t launch_attention(const Dev &d, const void *q, float scale, float *out, long long live_ub,
                              cudaStream_t st, int64_t *launches) {
-    if (d.dense && d.attn_kernel == 1) return launch_attention_tc(d, q, scale, out, live_ub, st, launches);
+    if (d.dense && d.attn_kernel == 1)
+        return launch_attention_i8(d, q, scale, out, nullptr, nullptr, 0.f, 0.f, live_ub, st, launches);
     if (d.dense) {
         switch (d.G) {
             case 1: return launch_g<1, true>(d, q, scale, out, live_ub, st, launches);

@@ -80,6 +80,27 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
     return mbar_wait_for(bar, parity, kWaitCycles);
 }
 
+// The same bounded wait, but each probe lets the hardware suspend the warp until the
+// phase completes (or a 10 ms hint runs out), so a waiting warp takes no issue slots
+// from the warps that work on the same scheduler.
+__device__ __forceinline__ uint32_t mbar_try_wait_suspend(uint32_t bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, 10000000;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return done;
+}
+__device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity) {
+    if (mbar_try_wait_suspend(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait_suspend(bar, parity))
+        if (clock64() - t0 > kWaitCycles) return false;
+    return true;
+}
+
 __device__ __forceinline__ void bulk_copy(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar,
                                           uint64_t policy) {
     asm volatile(
@@ -133,6 +154,17 @@ __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// bf16 x bf16 -> f32 (the operands of bf16-class tiles: raw bf16 keys / values and
+// the query, no conversion and no narrowing).
+__device__ __forceinline__ void mma16816_bf16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                              uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 __device__ __forceinline__ uint32_t transpose8x8(uint32_t x) {
     uint32_t y;
     asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
@@ -146,11 +178,17 @@ __device__ __forceinline__ uint32_t f32x2_to_f16x2(float lo, float hi) {
     return h2_as_u32(__floats2half2_rn(lo, hi));
 }
 
+__device__ __forceinline__ uint32_t f32x2_to_bf16x2(float lo, float hi) {
+    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&v);
+}
+
 __device__ __forceinline__ int sel4(int c, int a0, int a1, int a2, int a3) {
     return c == 0 ? a0 : c == 1 ? a1 : c == 2 ? a2 : a3;
 }
 
 // ------------------------------------------------- code pair -> f16x2 operand
+// (BITS == 16: the raw bf16 pair, the operand of a bf16 MMA.)
 // A 32-bit word of a BITS-bit code block holds 16/BITS dim pairs; pair s has its
 // members at bits BITS*s and BITS*s + 16.  OR-ing the masked word into 0x6400
 // (f16 1024) gives 1024 + m*code in each half (m = 2^(BITS*s') after an optional
@@ -166,7 +204,7 @@ __device__ __forceinline__ uint32_t magic_f16() {
 template <int BITS, int S>
 __device__ __forceinline__ uint32_t code_pair(uint32_t word, uint32_t magic) {
     if constexpr (BITS == 16) {
-        return f32x2_to_f16x2(__uint_as_float(word << 16), __uint_as_float(word & 0xffff0000u));
+        return word;
     } else if constexpr (BITS == 8) {
         const uint32_t x = __byte_perm(word, 0x64646464u, S == 0 ? 0x4240 : 0x4341);
         return h2_as_u32(__hsub2(u32_as_h2(x), u32_as_h2(0x64006400u)));
@@ -222,24 +260,36 @@ __device__ __forceinline__ void load_quarter(const uint8_t *row, int off, int od
 
 // S += K . Q^T over head-dim group GRP (32 dims = 2 k-steps).  Pair p = 4*GRP + 2*hh
 // of a quarter carries k-indices 2tig, 2tig+1 of k-step hh; pair p + 1 carries
-// 2tig+8, 2tig+9.  The group's K scale multiplies the fp32 result and its zero adds
-// zero * sum_group(q).
+// 2tig+8, 2tig+9.  Codes: f16 MMA against the f16 query qb (each head's group scaled
+// by a power of two into f16's range when its magnitudes need it; qinv undoes the
+// scale on the fp32 product); the group's K scale multiplies the fp32 result and its
+// zero adds zero * sum_group(q).  bf16 keys: bf16 MMA against the raw bf16 query qbb.
 template <int BITS, int GRP>
 __device__ __forceinline__ void qk_group(float (&x)[4], const uint32_t (&k0)[BITS],
                                          const uint32_t (&k1)[BITS], const uint32_t (&qb)[4][2][2],
-                                         const float (&qs)[2][4], const float2 (&km0)[4],
+                                         const uint32_t (&qbb)[4][2][2], const float (&qs)[2][4],
+                                         const float (&qinv)[2][4], bool qscaled, const float2 (&km0)[4],
                                          const float2 (&km1)[4], uint32_t magic) {
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    mma16816(acc, quarter_pair<BITS, 4 * GRP>(k0, magic), quarter_pair<BITS, 4 * GRP>(k1, magic),
-             quarter_pair<BITS, 4 * GRP + 1>(k0, magic), quarter_pair<BITS, 4 * GRP + 1>(k1, magic),
-             qb[GRP][0][0], qb[GRP][0][1]);
-    mma16816(acc, quarter_pair<BITS, 4 * GRP + 2>(k0, magic), quarter_pair<BITS, 4 * GRP + 2>(k1, magic),
-             quarter_pair<BITS, 4 * GRP + 3>(k0, magic), quarter_pair<BITS, 4 * GRP + 3>(k1, magic),
-             qb[GRP][1][0], qb[GRP][1][1]);
     if constexpr (BITS == 16) {
+        mma16816_bf16(acc, quarter_pair<BITS, 4 * GRP>(k0, magic), quarter_pair<BITS, 4 * GRP>(k1, magic),
+                      quarter_pair<BITS, 4 * GRP + 1>(k0, magic), quarter_pair<BITS, 4 * GRP + 1>(k1, magic),
+                      qbb[GRP][0][0], qbb[GRP][0][1]);
+        mma16816_bf16(acc, quarter_pair<BITS, 4 * GRP + 2>(k0, magic), quarter_pair<BITS, 4 * GRP + 2>(k1, magic),
+                      quarter_pair<BITS, 4 * GRP + 3>(k0, magic), quarter_pair<BITS, 4 * GRP + 3>(k1, magic),
+                      qbb[GRP][1][0], qbb[GRP][1][1]);
 #pragma unroll
         for (int i = 0; i < 4; ++i) x[i] += acc[i];
     } else {
+        mma16816(acc, quarter_pair<BITS, 4 * GRP>(k0, magic), quarter_pair<BITS, 4 * GRP>(k1, magic),
+                 quarter_pair<BITS, 4 * GRP + 1>(k0, magic), quarter_pair<BITS, 4 * GRP + 1>(k1, magic),
+                 qb[GRP][0][0], qb[GRP][0][1]);
+        mma16816(acc, quarter_pair<BITS, 4 * GRP + 2>(k0, magic), quarter_pair<BITS, 4 * GRP + 2>(k1, magic),
+                 quarter_pair<BITS, 4 * GRP + 3>(k0, magic), quarter_pair<BITS, 4 * GRP + 3>(k1, magic),
+                 qb[GRP][1][0], qb[GRP][1][1]);
+        if (qscaled) {
+            acc[0] *= qinv[0][GRP]; acc[1] *= qinv[1][GRP]; acc[2] *= qinv[0][GRP]; acc[3] *= qinv[1][GRP];
+        }
         // km = (scale, zero) of the group for row g (0) and row g + 8 (1)
         x[0] = fmaf(km0[GRP].x, acc[0], fmaf(km0[GRP].y, qs[0][GRP], x[0]));
         x[1] = fmaf(km0[GRP].x, acc[1], fmaf(km0[GRP].y, qs[1][GRP], x[1]));
@@ -313,7 +363,7 @@ __device__ __forceinline__ void add_scores(const Dev &d, int s, const float *lgs
             if (t >= t1) continue;
             float inc = 0.f;
 #pragma unroll
-            for (int h = 0; h < G; ++h) inc += ex2(x[k][h] - Mh[h]) * Ih[h];
+            for (int h = 0; h < G; ++h) inc += exp2f(x[k][h] - Mh[h]) * Ih[h];   // full-precision exp2
             srow(t)[t] = sv[k] + inc;
         }
     }

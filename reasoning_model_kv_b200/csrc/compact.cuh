@@ -85,8 +85,8 @@ __device__ __forceinline__ void compact_tables(const Dev &d, int s, const int (&
         int32_t *pc = d.pos[c] + base_e;
         float *sc = d.score[c] + base_e;
         int32_t *fsc = d.fs[c] + base_e;
-        const int ft0 = d.ft[s * 4 + c];
         const int m = evicted[c];
+        const int ft0 = dclamp(d.err, d.ft[s * 4 + c], d.cap[c] - m, kDbgEvict + 0x10 + c);
         const int rec = d.rec[c];
         uint8_t *pool = d.pool[c] + base_e * rec;
         int kept_carry = 0, ev_carry = 0;

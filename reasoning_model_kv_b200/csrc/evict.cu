@@ -38,7 +38,7 @@ __global__ void __launch_bounds__(kThreads) evict_kernel(Dev d, int budget, int 
 
     int n[4];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) n[c] = d.n[s * 4 + c];
+    for (int c = 0; c < 4; ++c) n[c] = dclamp(d.err, d.n[s * 4 + c], d.cap[c], kDbgEvict + c);
 
     // 1+2. radix select of the budget-th largest key (budget == 0: nothing kept);
     //      pass 0 also counts the unprotected entries

@@ -87,7 +87,7 @@ __global__ void __launch_bounds__(kThreads) tbe_kernel(Dev d, const int32_t *__r
         int acc = 0;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-            n[c] = d.n[s * 4 + c];
+            n[c] = dclamp(d.err, d.n[s * 4 + c], d.cap[c], kDbgSegments + c);
             cbase[c] = acc;   // the flags of class c start here
             acc += d.cap[c];
         }

@@ -90,6 +90,9 @@ void make_layout(const tkv_config &c, tkv_layout *lay, tkv::Dev *dev, uint8_t *b
     const size_t o_rank = take((size_t)c.B * c.max_append * sizeof(int32_t));
     const size_t o_tot = take((size_t)c.B * 4 * sizeof(int32_t));
     const size_t o_lg = take(S * (size_t)ncap * c.G * sizeof(float));
+    const size_t o_part = take((S + tkv::kNctaMax) * (size_t)tkv::part_floats(c.G) * sizeof(float));
+    const size_t o_seglo = take(S * sizeof(int32_t));
+    const size_t o_seghi = take(S * sizeof(int32_t));
     lay->total_bytes = off;
     if (!dev) return;
     dev->B = c.B; dev->Hkv = c.Hkv; dev->G = c.G; dev->S = (int)S;
@@ -113,6 +116,10 @@ void make_layout(const tkv_config &c, tkv_layout *lay, tkv::Dev *dev, uint8_t *b
     dev->totals = reinterpret_cast<int32_t *>(base + o_tot);
     dev->logits = reinterpret_cast<float *>(base + o_lg);
     dev->ncap = ncap;
+    dev->part = reinterpret_cast<float *>(base + o_part);
+    dev->seg_lo = reinterpret_cast<int32_t *>(base + o_seglo);
+    dev->seg_hi = reinterpret_cast<int32_t *>(base + o_seghi);
+    dev->ncta_max = tkv::kNctaMax;
 }
 
 tkv_status cuda_status(cudaError_t e, const char *what) {
@@ -257,6 +264,22 @@ tkv_status tkv_decode_attention(tkv_cache *c, const void *q, float softmax_scale
     cudaError_t e = tkv::launch_attention(c->dev, q, softmax_scale, out, ub,
                                           static_cast<cudaStream_t>(stream), &c->launches);
     return cuda_status(e, "tkv_decode_attention");
+}
+
+tkv_status tkv_decode_attention_sparsity(tkv_cache *c, const void *q, float softmax_scale, float *out,
+                                         float *sparsity, uint8_t *thought, float th_r, float th_t, void *stream) {
+    if (!c) return fail(TKV_ERR_INVALID, "cache is NULL");
+    if (!q || !out || !sparsity) return fail(TKV_ERR_INVALID, "NULL q, out or sparsity");
+    if (!aligned16(q) || !aligned16(out)) return fail(TKV_ERR_INVALID, "q and out must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(sparsity) & 3u) != 0) return fail(TKV_ERR_INVALID, "sparsity must be 4-byte aligned");
+    if (!(th_r <= th_t) || !std::isfinite(th_r) || !std::isfinite(th_t))
+        return fail(TKV_ERR_INVALID, "thresholds must be finite with th_r <= th_t");
+    if (!(c->cfg.dense == 1 && c->cfg.attn_kernel == 1))
+        return fail(TKV_ERR_INVALID, "the sparsity statistic needs dense placement and attn_kernel 1");
+    const long long ub = std::max(1ll, c->live_ub);
+    cudaError_t e = tkv::launch_attention_i8(c->dev, q, softmax_scale, out, sparsity, thought, th_r, th_t, ub,
+                                             static_cast<cudaStream_t>(stream), &c->launches);
+    return cuda_status(e, "tkv_decode_attention_sparsity");
 }
 
 tkv_status tkv_evict_compact(tkv_cache *c, int32_t budget, void *stream) {

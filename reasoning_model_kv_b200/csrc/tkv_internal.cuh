@@ -35,7 +35,18 @@ struct Dev {
     int32_t *totals;   // [B][4] tokens per class in the current append
     float *logits;     // [S][ncap][G] raw logits (log2 domain) of the current step
     int ncap;          // sum of cap[c], rounded up to a multiple of 32
+    // tensor-core decode attention (attention_i8.cu): per (stream, CTA) partial
+    // results, slot s + cta, part_floats(G) floats each, and the first / last CTA of
+    // every stream
+    float *part;       // [S + ncta_max][part_floats(G)]
+    int32_t *seg_lo, *seg_hi;   // [S]
+    int ncta_max;
 };
+
+// Floats of one partial result of the tensor-core decode attention: running max,
+// sum and sum p*(x - m) per head, then the unnormalised O [G][D].
+__host__ __device__ constexpr int part_floats(int G) { return G * (3 + kD); }
+constexpr int kNctaMax = 1024;   // upper bound on the persistent grid (one CTA per SM)
 
 enum : uint32_t { kErrInvalid = 1, kErrCapacity = 2, kErrTimeout = 4 };
 
@@ -43,6 +54,30 @@ __device__ __forceinline__ void raise_error(uint32_t *err, uint32_t code, uint32
     if (atomicCAS(err, 0u, code) == 0u) err[2] = detail;
     atomicAdd(err + 1, 1u);
 }
+
+// Bounds checks of the TKV_DEBUG build (libtkv_debug.so; the pages' pipeline has no
+// counterpart: it stands in for a memory checker).  Before a table or pool access the
+// kernels check the counters and slot handles they index with against the cache's
+// capacities; a failed check latches TKV_ERR_INVALID with the check's id as detail
+// (kDbg* below, + class) and the access is skipped or its index clamped into range.
+// Release builds compile every check to `true` / the unchanged value.
+enum : uint32_t { kDbgAppend = 0x100, kDbgAttention = 0x200, kDbgEvict = 0x300, kDbgSegments = 0x400 };
+#ifdef TKV_DEBUG
+__device__ __forceinline__ bool dcheck(uint32_t *err, bool ok, uint32_t id) {
+    if (!ok) raise_error(err, kErrInvalid, id);
+    return ok;
+}
+__device__ __forceinline__ int dclamp(uint32_t *err, int v, int hi, uint32_t id) {
+    if (v < 0 || v > hi) {
+        raise_error(err, kErrInvalid, id);
+        return v < 0 ? 0 : hi;
+    }
+    return v;
+}
+#else
+__device__ __forceinline__ bool dcheck(uint32_t *, bool, uint32_t) { return true; }
+__device__ __forceinline__ int dclamp(uint32_t *, int v, int, uint32_t) { return v; }
+#endif
 
 // Host-side per-device facts, looked up once per device and thread-safe (racing
 // first calls compute and store the same value).
@@ -60,9 +95,12 @@ cudaError_t launch_append(const Dev &d, const void *k, const void *v, const uint
                           const int32_t *pos, int T, cudaStream_t st, int64_t *launches);
 cudaError_t launch_attention(const Dev &d, const void *q, float scale, float *out,
                              long long live_ub, cudaStream_t st, int64_t *launches);
-// Dense placement: the tcgen05 kernel (attention_tc.cu).
-cudaError_t launch_attention_tc(const Dev &d, const void *q, float scale, float *out, long long live_ub,
-                                cudaStream_t st, int64_t *launches);
+// Dense placement: the tensor-core kernel with integer operands (attention_i8.cu).  With
+// sparsity / thought non-NULL it also writes, per (stream, query head), the attention
+// sparsity 1 - H(p) / ln N and its thought class under the thresholds th_r <= th_t.
+cudaError_t launch_attention_i8(const Dev &d, const void *q, float scale, float *out, float *sparsity,
+                                uint8_t *thought, float th_r, float th_t, long long live_ub, cudaStream_t st,
+                                int64_t *launches);
 // Self-test of the bounded device waits (selftest.cu).
 cudaError_t launch_wait_timeout(const Dev &d, long long limit, cudaStream_t st, int64_t *launches);
 cudaError_t launch_evict(const Dev &d, int budget, int keep_from, cudaStream_t st, int64_t *launches);

@@ -8,12 +8,15 @@ the calls raise.
 from __future__ import annotations
 
 import ctypes
+import os
 from pathlib import Path
 
 import numpy as np
 import torch
 
-LIB_PATH = Path(__file__).resolve().parent / "libtkv.so"
+# TKV_LIBRARY selects another build of the library (e.g. libtkv_debug.so, the
+# bounds-checking build) for the whole process; by default the release build.
+LIB_PATH = Path(os.environ.get("TKV_LIBRARY") or (Path(__file__).resolve().parent / "libtkv.so"))
 
 TKV_OK, TKV_ERR_INVALID, TKV_ERR_CAPACITY, TKV_ERR_CUDA, TKV_ERR_TIMEOUT = range(5)
 STATUS_NAMES = {0: "TKV_OK", 1: "TKV_ERR_INVALID", 2: "TKV_ERR_CAPACITY", 3: "TKV_ERR_CUDA",
@@ -48,7 +51,7 @@ EXPORTS = ["tkv_workspace_bytes", "tkv_create", "tkv_destroy", "tkv_reset", "tkv
            "tkv_quantize_append", "tkv_quantize_append_noalloc", "tkv_decode_attention", "tkv_evict_compact", "tkv_poll_error",
            "tkv_export_state", "tkv_import_state", "tkv_launch_count", "tkv_last_error_string",
            "tkv_selftest_wait_timeout", "tkv_evict_segments", "tkv_tbe_schedule",
-           "tkv_evict_tam", "tkv_evict_compact_window"]
+           "tkv_evict_tam", "tkv_evict_compact_window", "tkv_decode_attention_sparsity"]
 
 _lib = None
 
@@ -73,6 +76,9 @@ def lib() -> ctypes.CDLL:
     L.tkv_quantize_append.argtypes = [vp, vp, vp, vp, vp, i32, vp]
     L.tkv_quantize_append_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, vp]
     L.tkv_decode_attention.argtypes = [vp, vp, ctypes.c_float, vp, vp]
+    L.tkv_decode_attention_sparsity.argtypes = [vp, vp, ctypes.c_float, vp, vp, vp, ctypes.c_float,
+                                                ctypes.c_float, vp]
+    L.tkv_decode_attention_sparsity.restype = ctypes.c_int
     L.tkv_evict_compact.argtypes = [vp, i32, vp]
     L.tkv_poll_error.argtypes = [vp, vp]
     L.tkv_export_state.argtypes = [vp, vp, vp]
@@ -205,6 +211,24 @@ class TkvCache:
                                           float(softmax_scale), _dptr(out, torch.float32, "out"),
                                           _stream(stream)))
         return out
+
+    def decode_attention_sparsity(self, q: torch.Tensor, softmax_scale: float, th_r: float = 0.5,
+                                  th_t: float = 0.7, out: torch.Tensor | None = None, stream=None):
+        """decode_attention plus the per-(stream, head) attention sparsity 1 - H(p)/ln N
+        and its thought class (3 T if >= th_t, 1 R if >= th_r, else 2 E); returns
+        (out, sparsity [B, Hkv*G] fp32, thought class [B, Hkv*G] uint8)."""
+        if q.shape != (self.B, self.Hkv * self.G, 128):
+            raise TkvError(TKV_ERR_INVALID, f"q must be [B, Hkv*G, 128], got {tuple(q.shape)}")
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+        sp = torch.empty(q.shape[:2], dtype=torch.float32, device=q.device)
+        cls = torch.empty(q.shape[:2], dtype=torch.uint8, device=q.device)
+        _check(lib().tkv_decode_attention_sparsity(self._h, _dptr(q, torch.bfloat16, "q"), float(softmax_scale),
+                                                   _dptr(out, torch.float32, "out"),
+                                                   _dptr(sp, torch.float32, "sparsity"),
+                                                   _dptr(cls, torch.uint8, "thought"), float(th_r), float(th_t),
+                                                   _stream(stream)))
+        return out, sp, cls
 
     def evict_compact(self, budget: int, stream=None):
         _check(lib().tkv_evict_compact(self._h, int(budget), _stream(stream)))

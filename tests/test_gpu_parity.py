@@ -391,3 +391,42 @@ def test_local_window_eviction(dense):
     assert o.evict(100) == 0
     compare_states(gpu.export_state(sub), o.state, what="window past every position")
     assert gpu.poll_error() == tkv.TKV_OK
+
+
+def _scaled_case(mode, k_scale, v_scale, q_fn):
+    """The 709-token two-row workload with its 4 bf16 sink tokens' K / V scaled by
+    k_scale / v_scale (exactly, in bf16) and the query transformed by q_fn."""
+    w = synth.prefill_inputs("tiny_b1_ctx2k", B=2, Hq=8, Hkv=2, ctx=709, n_protect=4, steps=2)
+    w["k"][:, :, :4] = (w["k"][:, :, :4].float() * k_scale).to(torch.bfloat16)
+    w["v"][:, :, :4] = (w["v"][:, :, :4].float() * v_scale).to(torch.bfloat16)
+    gpu = TkvCache(w["B"], w["Hkv"], w["G"], w["cap"], w["n_protect"], max_append=w["ctx"], **MODES[mode])
+    gpu.quantize_append(w["k"].to(DEV), w["v"].to(DEV), w["cls"][:, :w["ctx"]].contiguous().to(DEV),
+                        w["pos"].to(DEV))
+    o = oracle_for(gpu, gpu.export_state())
+    q = q_fn(synth.decode_inputs(w, 0)[4].float()).to(torch.bfloat16)
+    out = gpu.decode_attention(q.to(DEV), SCALE).cpu().numpy()
+    ref = o.attend(np_bits(q), SCALE)
+    assert np.isfinite(out).all(), "non-finite output"
+    # an fp32 output of magnitude |ref| >> 1 cannot be closer than its own rounding, so
+    # the 2e-3 bound applies to max(1, |ref|)
+    err = np.abs(out.astype(np.float64) - ref) / np.maximum(1.0, np.abs(ref))
+    assert float(err.max()) <= OUT_ATOL, float(err.max())
+    assert gpu.poll_error() == tkv.TKV_OK
+    return float(err.max())
+
+
+@pytest.mark.parametrize("mode", list(MODES))
+def test_extreme_magnitudes_sinks_and_query(mode):
+    """bf16 sink keys / values around 1e5 (beyond f16's range), query entries around
+    +-1e5 in one dim per head, and a query scaled below 2^-14 (f16-subnormal) against
+    sink keys scaled up by 2^20: every path keeps bf16 values and the query without
+    narrowing them (ThinKV, TBQ: protected tokens stay at full precision)."""
+    _scaled_case(mode, 1e5, 1e5, lambda q: q)
+
+    def spike(q):
+        q = q.clone()
+        q[:, :, 17] = 1e5
+        q[:, ::2, 90] = -1e5
+        return q
+    _scaled_case(mode, 1.0, 1.0, spike)
+    _scaled_case(mode, 2.0 ** 20, 8.0, lambda q: q * 2.0 ** -20)

@@ -32,8 +32,8 @@ def test_export_import_round_trip_continues_bit_identically(mode):
     fresh = TkvCache(gpu.B, gpu.Hkv, gpu.G, gpu.cap, gpu.n_protect, max_append=gpu.max_append, **MODES[mode])
     fresh.import_state(st)
     back = fresh.export_state()
-    for key, arr in st.items():
-        assert np.array_equal(back[key], arr), key
+    for key, arr in st.items():   # bytes: unused slots may hold NaN patterns
+        assert np.array_equal(back[key].view(np.uint8), arr.view(np.uint8)), key
     gpu.import_state(st)           # both caches restored from the same checkpoint
     outs, states = [], []
     for step in (1, 2):
@@ -45,7 +45,7 @@ def test_export_import_round_trip_continues_bit_identically(mode):
         assert torch.equal(pair[0], pair[1]), f"step {step}: outputs differ"
     a, b = gpu.export_state(), fresh.export_state()
     for key in a:
-        assert np.array_equal(a[key], b[key]), key
+        assert np.array_equal(a[key].view(np.uint8), b[key].view(np.uint8)), key
     o.load_state(b)
     k, v, cls, pos, q = synth.decode_inputs(w, 2)
     ref = o.attend(np_bits(q), SCALE)          # the restored state still matches the oracle
