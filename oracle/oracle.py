@@ -101,6 +101,8 @@ def lib():
                                                                                       ctypes.c_double]
         L.orc_evict_tam.restype = ctypes.c_int
         L.orc_num_threads.restype = ctypes.c_int
+        L.orc_sum_f32_exact.argtypes = [ctypes.c_void_p, ctypes.c_int]
+        L.orc_sum_f32_exact.restype = ctypes.c_double
         L.orc_attention_sparsity.argtypes = [ctypes.POINTER(_State), ctypes.c_void_p, ctypes.c_float,
                                              ctypes.c_void_p]
         L.orc_attention_sparsity.restype = None
@@ -198,6 +200,13 @@ def unpack_record(bits: int, rec: np.ndarray, D=128, group=32):
     vh = np.zeros(D, dtype=np.float64)
     lib().orc_unpack_record(bits, D, group, _ptr(rec), _ptr(kh), _ptr(vh))
     return kh, vh
+
+
+def sum_f32_exact(v) -> float:
+    """The exact sum of fp32 values (negative and non-finite ones count as 0), rounded
+    to the nearest double: the score sums of the TAM budgets."""
+    a = np.ascontiguousarray(np.asarray(v, dtype=np.float32))
+    return lib().orc_sum_f32_exact(_ptr(a) if a.size else None, int(a.size))
 
 
 def num_threads() -> int:

@@ -744,6 +744,63 @@ static void compact_stream(orc_state *st, int s, uint8_t *evict[4]) {
 
 /* Thought segment of position p: the last j with seg_start[j] <= p, or -1 when p
  * lies before the first segment (seg_start strictly increasing, nseg of them). */
+/* Exact sums of fp32 scores (TAM page, sections 2.B-2.C: w_j is the mean attention
+ * score of segment j and delta = c times the stream's mean score; the means are taken
+ * of the exact sums).  A finite non-negative fp32 value is m * 2^(b - 149) with m < 2^24
+ * and 0 <= b <= 253, so the exact sum of up to 2^32 of them is a 288-bit integer times
+ * 2^-149: nine 32-bit digits.  Negative and non-finite values (attention mass never is
+ * either) count as 0.  The sum is then rounded to the nearest double (ties to even). */
+typedef struct { uint64_t d[9]; } exact_sum;
+
+static void exact_add(exact_sum *a, float v) {
+    uint32_t u;
+    memcpy(&u, &v, 4);
+    const uint32_t eb = u >> 23;                  /* sign bit set: eb >= 256 */
+    if (u == 0 || eb >= 255) return;
+    const uint64_t m = eb ? (uint64_t)((u & 0x7FFFFFu) | 0x800000u) : (uint64_t)(u & 0x7FFFFFu);
+    const int b = eb ? (int)eb - 1 : 0;           /* bit of m's lowest bit above 2^-149 */
+    const uint64_t x = m << (b % 32);
+    a->d[b / 32] += x & 0xFFFFFFFFull;
+    a->d[b / 32 + 1] += x >> 32;                  /* b / 32 <= 7 */
+}
+
+static void exact_merge(exact_sum *a, const exact_sum *b) {
+    for (int i = 0; i < 9; ++i) a->d[i] += b->d[i];
+}
+
+static double exact_value(const exact_sum *a) {
+    uint32_t dig[11];
+    uint64_t carry = 0;
+    for (int i = 0; i < 9; ++i) {
+        const uint64_t t = a->d[i] + carry;       /* digits below 2^64 - 2^32: no overflow */
+        dig[i] = (uint32_t)t;
+        carry = t >> 32;
+    }
+    dig[9] = (uint32_t)carry;
+    dig[10] = (uint32_t)(carry >> 32);
+    int top = 10;
+    while (top >= 0 && dig[top] == 0) --top;
+    if (top < 0) return 0.0;
+    /* the 64 bits below the leading one of the 96-bit window dig[top..top-2], the bits
+     * under them folded into bit 0 (sticky), converted with one rounding */
+    const uint64_t w2 = dig[top], w1 = top >= 1 ? dig[top - 1] : 0, w0 = top >= 2 ? dig[top - 2] : 0;
+    int sticky = 0;
+    for (int i = 0; i < top - 2; ++i) sticky |= dig[i] != 0;
+    int lz = 0;
+    while (!((w2 << lz) & 0x80000000ull)) ++lz;
+    uint64_t t = ((w2 << 32) | w1) << lz;
+    if (lz) t |= w0 >> (32 - lz);
+    if (((w0 << lz) & 0xFFFFFFFFull) != 0 || sticky) t |= 1;
+    return ldexp((double)t, 32 - lz + 32 * (top - 2) - 149);
+}
+
+double orc_sum_f32_exact(const float *v, int n) {
+    exact_sum a;
+    memset(&a, 0, sizeof(a));
+    for (int i = 0; i < n; ++i) exact_add(&a, v[i]);
+    return exact_value(&a);
+}
+
 static int segment_of(const int32_t *seg_start, int nseg, int32_t p) {
     int j = -1;
     for (int k = 0; k < nseg && seg_start[k] <= p; ++k) j = k;
@@ -826,23 +883,28 @@ int orc_evict_tam(orc_state *st, const int32_t *seg_start, const uint8_t *seg_la
         if (ns == 0) continue;
         int *cnt = calloc(ns, sizeof(int)), *piv = calloc(ns, sizeof(int));
         double *sum = calloc(ns, sizeof(double));
-        /* 1. candidates per segment: count and score sum; the stream's mean */
-        double tot = 0.0;
+        /* 1. candidates per segment: count and exact score sum; the stream's mean */
+        exact_sum tot_x;
+        memset(&tot_x, 0, sizeof(tot_x));
         long long ntot = 0;
         for (int j = 0; j < ns; ++j) {
             const int c = labels[j];
             if (c > 3) continue;
             const size_t base = (size_t)s * st->cap[c];
+            exact_sum seg;
+            memset(&seg, 0, sizeof(seg));
             for (int i = 0; i < st->n[s * 4 + c]; ++i) {
                 const int32_t p = st->pos[c][base + i];
                 if (p < st->n_protect || segment_of(starts, ns, p) != j) continue;
                 cnt[j] += 1;
-                sum[j] += (double)st->score[c][base + i];
+                exact_add(&seg, st->score[c][base + i]);
             }
-            tot += sum[j];
+            sum[j] = exact_value(&seg);
+            exact_merge(&tot_x, &seg);
             ntot += cnt[j];
         }
         if (ntot == 0) { free(cnt); free(piv); free(sum); continue; }
+        const double tot = exact_value(&tot_x);
         const double delta = c * (tot / (double)ntot);
         /* 2. pivotal candidates */
         long long P = 0;

@@ -317,3 +317,64 @@ def test_tam_keeps_pivotal_and_per_segment_top_t(trial):
     P = sum(1 for x in allc if np.float64(x) >= delta)
     assert nonpiv_kept <= max(0, budget - P)
     _check_table_invariants(cache, before)
+
+
+# --------------------------------------------------------------------------
+# exact score sums behind the TAM means (TAM page, sections 2.B-2.C)
+# --------------------------------------------------------------------------
+def _wide_f32(rng, n):
+    """fp32 values spread over the whole exponent range, subnormals and zeros included."""
+    e = rng.integers(-149, 128, n)
+    m = rng.random(n) + 0.5
+    v = np.ldexp(m, e).astype(np.float32)          # overflow to inf is dropped below
+    v[rng.random(n) < 0.1] = 0.0
+    v[rng.random(n) < 0.1] = np.float32(1e-45) * rng.integers(1, 1 << 23, 1).astype(np.float32)
+    return v[np.isfinite(v)]
+
+
+@pytest.mark.parametrize("trial", range(12))
+def test_exact_sum_is_the_correctly_rounded_sum(trial):
+    """math.fsum returns the exact sum of its (double) inputs rounded once; every fp32
+    is a double, so the two must agree bit for bit, in any order of the terms."""
+    import math
+    rng = np.random.default_rng(4400 + trial)
+    n = int(rng.integers(0, 3000))
+    v = _wide_f32(rng, n) if trial % 2 else (rng.random(n) * 3).astype(np.float32)
+    want = math.fsum(float(x) for x in v)
+    assert orc.sum_f32_exact(v) == want
+    assert orc.sum_f32_exact(v[rng.permutation(len(v))]) == want
+
+
+def test_exact_sum_cancellation_free_cases():
+    """Closed forms: 2^24 + 1 + 1 (a naive fp32 loop returns 2^24), 2^k tails far below
+    the leading term, the largest and smallest fp32, and the rule for negative and
+    non-finite terms (they count as 0)."""
+    big = np.float32(2.0 ** 24)
+    assert orc.sum_f32_exact(np.array([big, 1, 1], np.float32)) == 2.0 ** 24 + 2
+    tiny = np.float32(2.0 ** -149)
+    assert orc.sum_f32_exact(np.array([tiny] * 3, np.float32)) == 3 * 2.0 ** -149
+    v = np.array([2.0 ** 100, 2.0 ** -100], np.float32)
+    assert orc.sum_f32_exact(v) == 2.0 ** 100                      # 2^-200 relative: rounds away
+    v = np.array([2.0 ** 20, 2.0 ** -33, 2.0 ** -33], np.float32)   # exactly 2^20 + 2^-32: one ulp up
+    assert orc.sum_f32_exact(v) == 2.0 ** 20 + 2.0 ** -32
+    fmax = float(np.finfo(np.float32).max)
+    assert orc.sum_f32_exact(np.array([fmax] * 5, np.float32)) == 5 * fmax
+    assert orc.sum_f32_exact(np.array([1.5, -7.0, np.inf, np.nan, 2.5], np.float32)) == 4.0
+    assert orc.sum_f32_exact(np.zeros(0, np.float32)) == 0.0
+    # 2^60 + 2^-60 + 2^-60: one rounding of the exact sum (ties to even are not reached)
+    v = np.array([2.0 ** 60, 2.0 ** -60, 2.0 ** -60], np.float32)
+    assert orc.sum_f32_exact(v) == 2.0 ** 60
+
+
+def test_tam_delta_is_the_exact_mean():
+    """Scores 2^24 then 2^24 ones: the exact mean is (2^24 + n) / (n + 1), which a
+    running fp32 sum would lose; c = 1 then makes exactly the first token pivotal."""
+    n_tok = 33
+    scores = np.ones(n_tok, np.float32)
+    scores[0] = np.float32(2.0 ** 24)
+    cache = _cache_with_scores(n_tok, np.full(n_tok, 1, np.uint8), scores)
+    st = np.array([[0]], np.int32)
+    assert cache.evict_tam(st, np.array([[1]], np.uint8), np.array([1], np.int32), 4, 1.0) == 0
+    kept = cache.live(0, 1)[1].tolist()
+    # pivotal: position 0 (2^24 >= mean); T' = 3; t = min(32, floor(3 * 1 + 1e-9)) = 3
+    assert kept == [0, 1, 2, 3]
