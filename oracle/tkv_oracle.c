@@ -155,8 +155,7 @@ uint16_t orc_f32_to_f16_ru(float xf) {
 /* ------------------------------------------------------------------ */
 /* ------------------------------------------------------------------ */
 /* Floating-point class codecs (the ThinKV page, Metodologia, TBQ: FP8 or NVFP4 */
-/* for Reasoning tokens, ternary for Transition tokens).  Oracle only: the CUDA  */
-/* path does not implement these formats yet.                                   */
+/* for Reasoning tokens, ternary for Transition tokens).                          */
 /* ------------------------------------------------------------------ */
 
 /* FP8 E4M3 in its "fn" form (OCP 8-bit floating point): sign, 4 exponent bits
@@ -414,12 +413,13 @@ void orc_unpack_record(int bits, int D, int group, const uint8_t *rec, double *k
 
 /* Record formats: 16 bf16, 8 / 4 / 2 integer codes (above), and the floating-point
  * class codecs 108 FP8 (E4M3), 104 NVFP4 (E2M1, blocks of 16), 102 ternary.  FP
- * records keep the codes in head-dim order:
+ * records place their 8-, 4- and 2-bit codes in the storage order of the integer
+ * records of the same width (storage_dim / pack_codes above):
  *   108: [K codes: D bytes][V codes: D bytes][K scale x ngroups][V scale x ngroups] (fp16)
- *   104: [K codes: D/2 bytes, element i in the low nibble of byte i/2 when i is even]
- *        [V codes][K block scales: D/16 bytes (E4M3)][V block scales]
- *   102: [K codes: D/4 bytes, element i at bit 2(i%4) of byte i/4; 1 = +1, 3 = -1]
- *        [V codes][K scale x ngroups][V scale x ngroups] (fp16) */
+ *   104: [K codes: D/2 bytes, 4-bit E2M1 fields][V codes]
+ *        [K block scales: D/16 bytes (E4M3), block j = dims 16j..16j+15][V block scales]
+ *   102: [K codes: D/4 bytes, 2-bit fields: 1 = +1, 3 = -1, 0 = 0][V codes]
+ *        [K scale x ngroups][V scale x ngroups] (fp16) */
 int orc_record_bytes_fmt(int fmt, int D, int group) {
     const int ng = D / group;
     switch (fmt) {
@@ -451,24 +451,21 @@ void orc_pack_record_fmt(int fmt, int D, int group, const uint16_t *k, const uin
                 orc_quantize_group_fp8(x + g * group, group, &sh, codes + g * group);
                 put_u16(rec + 2 * D + (which * ng + g) * 2, sh);
             }
-            memcpy(rec + which * D, codes, D);
+            pack_codes(codes, D, 8, which, rec + which * D);
         } else if (fmt == 104) {
             for (int blk = 0; blk < D / 16; ++blk) {
                 uint8_t sc;
                 orc_quantize_block_nvfp4(x + blk * 16, 16, &sc, codes + blk * 16);
                 rec[D + which * (D / 16) + blk] = sc;
             }
-            uint8_t *dst = rec + which * (D / 2);
-            for (int i = 0; i < D; i += 2) dst[i / 2] = (uint8_t)((codes[i] & 15) | ((codes[i + 1] & 15) << 4));
+            pack_codes(codes, D, 4, which, rec + which * (D / 2));
         } else {   /* 102 */
             for (int g = 0; g < ng; ++g) {
                 uint16_t sh;
                 orc_quantize_group_ternary(x + g * group, group, &sh, codes + g * group);
                 put_u16(rec + D / 2 + (which * ng + g) * 2, sh);
             }
-            uint8_t *dst = rec + which * (D / 4);
-            for (int i = 0; i < D; i += 4)
-                dst[i / 4] = (uint8_t)(codes[i] | (codes[i + 1] << 2) | (codes[i + 2] << 4) | (codes[i + 3] << 6));
+            pack_codes(codes, D, 2, which, rec + which * (D / 4));
         }
     }
 }
@@ -479,21 +476,22 @@ void orc_unpack_record_fmt(int fmt, int D, int group, const uint8_t *rec, double
         orc_unpack_record(fmt, D, group, rec, k_hat, v_hat);
         return;
     }
+    uint8_t codes[512];
     for (int which = 0; which < 2; ++which) {
         double *dst = which == 0 ? k_hat : v_hat;
+        if (fmt == 108) unpack_codes(rec + which * D, D, 8, which, codes);
+        else if (fmt == 104) unpack_codes(rec + which * (D / 2), D, 4, which, codes);
+        else unpack_codes(rec + which * (D / 4), D, 2, which, codes);
         for (int d = 0; d < D; ++d) {
             const int g = d / group;
             if (fmt == 108) {
                 const double sc = orc_f16_to_f64(get_u16(rec + 2 * D + (which * (D / group) + g) * 2));
-                dst[d] = orc_e4m3_decode(rec[which * D + d]) * sc;
+                dst[d] = orc_e4m3_decode(codes[d]) * sc;
             } else if (fmt == 104) {
-                const uint8_t byte = rec[which * (D / 2) + d / 2];
-                const uint8_t code = (d & 1) ? (byte >> 4) : (byte & 15);
-                dst[d] = orc_e2m1_decode(code) * orc_e4m3_decode(rec[D + which * (D / 16) + d / 16]);
+                dst[d] = orc_e2m1_decode(codes[d]) * orc_e4m3_decode(rec[D + which * (D / 16) + d / 16]);
             } else {
-                const uint8_t code = (rec[which * (D / 4) + d / 4] >> (2 * (d % 4))) & 3;
                 const double sc = orc_f16_to_f64(get_u16(rec + D / 2 + (which * (D / group) + g) * 2));
-                dst[d] = code == 1 ? sc : (code == 3 ? -sc : 0.0);
+                dst[d] = codes[d] == 1 ? sc : (codes[d] == 3 ? -sc : 0.0);
             }
         }
     }

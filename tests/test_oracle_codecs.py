@@ -1,6 +1,5 @@
 """Pins of the oracle's floating-point class codecs (ThinKV page, Metodologia, TBQ:
-FP8 or NVFP4 for Reasoning tokens, ternary for Transition tokens).  These are oracle
-groundwork for a later CUDA path; CPU only.
+FP8 or NVFP4 for Reasoning tokens, ternary for Transition tokens); CPU only.
 
 FP8 E4M3 is pinned against torch's float8_e4m3fn conversions (a library routine:
 every code's value, round-to-nearest-even on random and half-way inputs); E2M1
@@ -15,6 +14,7 @@ import torch
 import synth
 from oracle import oracle as orc
 from tests.helpers import bits_of
+from tests.test_record_layout import header_position
 
 # OCP MX: the magnitudes of the E2M1 codes 0..7 (bit 3 is the sign)
 E2M1_TABLE = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
@@ -146,24 +146,34 @@ def test_ternary_scale_is_the_mean_magnitude_above_the_threshold():
 D = 128
 
 
+def _codes_by_dim(block, bits, is_v):
+    """Codes of a K or V block read at the positions the header's element order gives
+    (the same order as the integer records of that width)."""
+    out = np.zeros(D, np.int64)
+    for dim in range(D):
+        byte, bit = header_position(bits, is_v, dim)
+        word = int.from_bytes(bytes(block[byte:byte + 4]), "little")
+        out[dim] = (word >> bit) & ((1 << bits) - 1)
+    return out
+
+
 def _np_decode_record(fmt, rec):
     """Independent reading of the documented FP record layouts (numpy + torch)."""
     rec = np.asarray(rec, np.uint8)
     out = []
     for which in range(2):
         if fmt == orc.FMT_FP8:
-            codes = torch.from_numpy(rec[which * D:(which + 1) * D].copy()).view(torch.float8_e4m3fn).double().numpy()
+            c = _codes_by_dim(rec[which * D:(which + 1) * D], 8, which == 1).astype(np.uint8)
+            codes = torch.from_numpy(c).view(torch.float8_e4m3fn).double().numpy()
             sc = rec[2 * D:2 * D + 16].view(np.float16).astype(np.float64)[which * 4:(which + 1) * 4]
             out.append(codes * np.repeat(sc, 32))
         elif fmt == orc.FMT_NVFP4:
-            b = rec[which * 64:(which + 1) * 64]
-            nib = np.stack([b & 15, b >> 4], axis=1).reshape(-1)
+            nib = _codes_by_dim(rec[which * 64:(which + 1) * 64], 4, which == 1)
             mag = np.array(E2M1_TABLE)[nib & 7] * np.where(nib & 8, -1.0, 1.0)
             sc = torch.from_numpy(rec[D + which * 8:D + (which + 1) * 8].copy()).view(torch.float8_e4m3fn).double().numpy()
             out.append(mag * np.repeat(sc, 16))
         else:
-            b = rec[which * 32:(which + 1) * 32]
-            codes = np.stack([(b >> (2 * j)) & 3 for j in range(4)], axis=1).reshape(-1)
+            codes = _codes_by_dim(rec[which * 32:(which + 1) * 32], 2, which == 1)
             sc = rec[64:80].view(np.float16).astype(np.float64)[which * 4:(which + 1) * 4]
             out.append(np.select([codes == 1, codes == 3], [1.0, -1.0], 0.0) * np.repeat(sc, 32))
     return out
@@ -186,10 +196,13 @@ def test_fp_records_decode_as_documented(fmt):
         x = k.float().numpy()
         if fmt == orc.FMT_FP8:
             sh, codes = orc.quantize_group_fp8(x[:32])
-            assert np.array_equal(rec[:32], codes)
+            assert np.array_equal(_codes_by_dim(rec[:D], 8, False)[:32], codes)
         elif fmt == orc.FMT_NVFP4:
             sc, codes = orc.quantize_block_nvfp4(x[:16])
-            assert rec[D] == sc and np.array_equal(rec[:8], (codes[0::2] & 15) | ((codes[1::2] & 15) << 4))
+            assert rec[D] == sc and np.array_equal(_codes_by_dim(rec[:64], 4, False)[:16], codes & 15)
+        else:
+            sh, codes = orc.quantize_group_ternary(x[:32])
+            assert np.array_equal(_codes_by_dim(rec[:32], 2, False)[:32], codes)
 
 
 def test_attention_over_fp_class_records_equals_softmax_over_the_decoded_records():
