@@ -64,6 +64,9 @@ def parse():
                          "over the rows' thought segments, r0 64, t_keep 16) or tam (the budget "
                          "split over segments in proportion to sqrt(mean score) x length, "
                          "tokens above 3x the mean score kept)")
+    ap.add_argument("--full-reps", type=int, default=3,
+                    help="timed attention calls on the full prefill context before the eviction "
+                         "(the full-context phase; 0 skips it)")
     ap.add_argument("--ctx", type=int, default=None,
                     help="prefill context before the eviction (default: the workload's); the "
                          "timed step is the same post-eviction step, with smaller pools")
@@ -186,7 +189,7 @@ def segment_inputs(w, dev, upto):
             torch.from_numpy(ns).to(dev))
 
 
-def setup_cache(w, dev, dense, evict_reps, flush, attn_kernel=0, evict="topk"):
+def setup_cache(w, dev, dense, evict_reps, flush, attn_kernel=0, evict="topk", full_reps=0):
     """Prefill, one scoring step, then the eviction (to the budget, or the TBE
     schedule at the scoring step's position).  The eviction is timed (CUDA events,
     L2 flushed) over `evict_reps` repetitions, each from a copy of the pre-eviction
@@ -199,6 +202,29 @@ def setup_cache(w, dev, dense, evict_reps, flush, attn_kernel=0, evict="topk"):
     k, v, c, p, q = synth.decode_inputs(w, 0, device=dev)        # untimed scoring step
     gpu.quantize_append(k, v, c, p)
     gpu.decode_attention(q, SCALE)
+    full = None
+    if full_reps > 0:
+        # the full-context phase (before any eviction): the attention call alone, L2
+        # flushed, on the whole prefill; it adds to the scores, which the eviction reads
+        # anyway (a second scoring step)
+        out = torch.empty((w["B"], w["Hq"], 128), dtype=torch.float32, device=dev)
+        n_full = gpu.state_views()["n"].cpu().numpy()
+        ms = []
+        st0 = torch.cuda.current_stream()
+        for i in range(full_reps + 1):
+            flush.zero_()
+            a, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(st0)
+            gpu.decode_attention(q, SCALE, out)
+            b2.record(st0)
+            b2.synchronize()
+            if i > 0:
+                ms.append(a.elapsed_time(b2))
+        t = sum(ms) / len(ms)
+        pkf = packed_bytes(n_full)
+        full = {"live_kv_tokens": int(n_full.sum()), "packed_kv_bytes": pkf, "attention_ms": t,
+                "hbm_gbs_packed": pkf / (t * 1e-3) / 1e9, "kv_tokens_per_s": int(n_full.sum()) / (t * 1e-3),
+                "reps": full_reps}
     segs = segment_inputs(w, dev, w["ctx"]) if evict in ("tbe", "tam") else None
     evict_ms = []
     snap = gpu.workspace.clone() if evict_reps > 0 else None
@@ -222,7 +248,7 @@ def setup_cache(w, dev, dense, evict_reps, flush, attn_kernel=0, evict="topk"):
     del snap
     torch.cuda.synchronize()
     assert gpu.poll_error() == 0
-    return gpu, (statistics.median(evict_ms) if evict_ms else None)
+    return gpu, (statistics.median(evict_ms) if evict_ms else None), full
 
 
 def run_tkv(args, rank, world, dev):
@@ -230,8 +256,9 @@ def run_tkv(args, rank, world, dev):
     w = synth.prefill_inputs(args.workload, seed=rank, device=dev, steps=2, **over)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
-    gpu, evict_ms = setup_cache(w, dev, args.placement == "dense", args.evict_reps, flush,
-                                attn_kernel=1 if args.attn_kernel == "tc" else 0, evict=args.evict)
+    gpu, evict_ms, full = setup_cache(w, dev, args.placement == "dense", args.evict_reps, flush,
+                                      attn_kernel=1 if args.attn_kernel == "tc" else 0, evict=args.evict,
+                                      full_reps=args.full_reps)
     del w["k"], w["v"]
     torch.cuda.empty_cache()
     views = gpu.state_views()
@@ -379,6 +406,7 @@ def run_tkv(args, rank, world, dev):
         "attention_timing": "attention call alone on the post-append cache (L2 flushed), CUDA events",
         "append_exposed_ms": t_step - t_attn,
         "evict_ms_untimed_step": evict_ms,
+        "full_context_phase": full,
         "kv_tokens_per_s": world * kv_tokens / (t_attn * 1e-3),
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
                      "frac": gbs / peak, "traffic": None, "peak_source": peak_src,

@@ -96,6 +96,13 @@ typedef struct {
                             step's bytes split evenly; dense placement only).
                             Both compute the same result within the stated
                             tolerances.                                       */
+    int32_t codec;       /* class record formats: 0 = integer codes (classes
+                            1/2/3: 8/4/2-bit asymmetric, fp16 scale and zero
+                            per group); 1 = floating-point codes (class 1 FP8
+                            E4M3, class 2 NVFP4: E2M1 with an E4M3 scale per
+                            16 dims, class 3 ternary {0, +1, -1}; FP8 and
+                            ternary with an fp16 scale per group).  Codec 1
+                            needs attn_kernel 0.                              */
 } tkv_config;
 
 typedef struct tkv_cache tkv_cache;
@@ -113,6 +120,12 @@ typedef struct tkv_cache tkv_cache;
  *     b-bit class: [K codes D*b/8][V codes D*b/8][K scale x4][K zero x4]
  *                  [V scale x4][V zero x4]  (fp16, little-endian)        (288/160/96 bytes)
  *     Scale and zero of group g (head dims 32g..32g+31) are entry g of their x4.
+ *     codec 1 (floating-point codes, same element order as the b-bit classes):
+ *       class 1 FP8:    [K E4M3 codes D][V codes D][K scale x4][V scale x4] (fp16)  (272 bytes)
+ *       class 2 NVFP4:  [K E2M1 codes D/2][V codes D/2][K scale x8][V scale x8]
+ *                       (E4M3; scale j covers head dims 16j..16j+15)       (144 bytes)
+ *       class 3 ternary:[K codes D/4][V codes D/4][K scale x4][V scale x4] (fp16; code
+ *                       1 = +scale, 3 = -scale, 0 = 0)                     (80 bytes)
  *   Element order inside a K or V block (b = 16 for bf16, else the class's bits):
  *   the block is four quarters of 4*b bytes (quarter q = bytes [4bq, 4b(q+1)));
  *   a quarter is b little-endian 32-bit words; word w of a quarter holds the

@@ -140,6 +140,103 @@ __device__ __forceinline__ void quantize_row(const float (&x)[4], int lane, uint
     }
 }
 
+// ---- floating-point class codes (codec 1; ThinKV page, Metodologia, TBQ: FP8 or
+//      NVFP4 for Reasoning tokens, ternary for Transition tokens).  Every step is a
+//      correctly rounded fp32 operation or a hardware conversion with round-to-nearest-
+//      even and saturation to the format's largest finite value, so the codes and
+//      scales are bit-exact with any IEEE implementation of the same definition.
+// E4M3 code of x: nearest, ties to even, |x| >= 448 saturating to 448, NaN -> 0x7F
+// (both halves of the packed conversion get x, so the byte order does not matter).
+__device__ __forceinline__ uint32_t e4m3_rn(float x) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %1;" : "=h"(r) : "f"(x));
+    return r & 0xFFu;
+}
+// E2M1 code of x: nearest, ties to the even code, saturating at 6.
+__device__ __forceinline__ uint32_t e2m1_rn(float x) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %1;\n\tcvt.u32.u8 %0, t;\n\t}"
+        : "=r"(r)
+        : "f"(x));
+    return r & 0xFu;
+}
+// Value of a positive E4M3 code (exact in fp32).
+__device__ __forceinline__ float e4m3_value(uint32_t code) {
+    const uint32_t e = (code >> 3) & 15u, m = code & 7u;
+    return e == 0 ? (float)m * 0.001953125f                                   // m/8 * 2^-6
+                  : __uint_as_float(((e + 120u) << 23) | (m << 20));         // (1 + m/8) * 2^(e-7)
+}
+// Smallest E4M3 value >= y > 0, saturated at 448 (y <= 0: code 0).
+__device__ __forceinline__ uint32_t e4m3_round_up(float y) {
+    if (!(y > 0.f)) return 0u;
+    if (y >= 448.f) return 0x7Eu;
+    uint32_t c = e4m3_rn(y);
+    if (e4m3_value(c) < y) ++c;   // positive codes are ordered
+    return c;
+}
+
+// Codes (by head dim, into the warp's stage) and scales of one 128-element row under
+// codec 1.  BITS 8: FP8 per 32-dim group, scale = fp16 round-up of amax / 448, code =
+// E4M3 of x / scale.  BITS 4: NVFP4 per 16-dim block, scale = E4M3 round-up of amax / 6,
+// code = E2M1 of x / scale.  BITS 2: ternary per group, delta = 0.7 * mean |x|, scale =
+// fp16 nearest of the mean |x| over |x| > delta, code 1 / 3 / 0 for x > delta /
+// x < -delta / else (sums in head-dim order).  Lane l holds dims 4l .. 4l+3.
+template <int BITS>
+__device__ __forceinline__ void quantize_row_fp(const float (&x)[4], int lane, uint8_t *scales, uint8_t *stage) {
+    uint32_t packed = 0;
+    if constexpr (BITS == 8 || BITS == 4) {
+        float amax = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+        constexpr int span = BITS == 8 ? 8 : 4;   // lanes of a group / block
+#pragma unroll
+        for (int o = 1; o < span; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
+        float sf;
+        if constexpr (BITS == 8) {
+            const __half sh = __float2half_ru(__fdiv_rn(amax, 448.f));
+            sf = __half2float(sh);
+            if ((lane & 7) == 0) reinterpret_cast<__half *>(scales)[lane >> 3] = sh;
+        } else {
+            const uint32_t sc = e4m3_round_up(__fdiv_rn(amax, 6.f));
+            sf = e4m3_value(sc);
+            if ((lane & 3) == 0) scales[lane >> 2] = (uint8_t)sc;
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            uint32_t c = 0;
+            if (sf != 0.f) c = BITS == 8 ? e4m3_rn(__fdiv_rn(x[i], sf)) : e2m1_rn(__fdiv_rn(x[i], sf));
+            packed |= c << (8 * i);
+        }
+    } else {
+        // the group's 32 values in head-dim order, gathered from its 8 lanes
+        const int base = lane & ~7;
+        float sa = 0.f;
+        for (int j = 0; j < 8; ++j)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) sa = __fadd_rn(sa, fabsf(__shfl_sync(kFull, x[i], base + j)));
+        const float delta = __fmul_rn(0.7f, __fdiv_rn(sa, 32.f));
+        float sb = 0.f;
+        int cnt = 0;
+        for (int j = 0; j < 8; ++j)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float a = fabsf(__shfl_sync(kFull, x[i], base + j));
+                if (a > delta) { sb = __fadd_rn(sb, a); ++cnt; }
+            }
+        const float alpha = cnt ? __fdiv_rn(sb, (float)cnt) : 0.f;
+        // fp16 nearest; a finite value above the largest finite fp16 takes that value (65504)
+        const bool big = alpha >= 65520.f && alpha <= 3.402823466e38f;
+        const __half sh = big ? __ushort_as_half((unsigned short)0x7BFFu) : __float2half_rn(alpha);
+        if ((lane & 7) == 0) reinterpret_cast<__half *>(scales)[lane >> 3] = sh;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t c = x[i] > delta ? 1u : (x[i] < -delta ? 3u : 0u);
+            packed |= c << (8 * i);
+        }
+    }
+    __syncwarp();
+    reinterpret_cast<uint32_t *>(stage)[lane] = packed;   // codes by head dim
+    __syncwarp();
+}
+
 __device__ __forceinline__ void row_floats(const uint2 &raw, float (&x)[4]) {
     x[0] = __uint_as_float(raw.x << 16);
     x[1] = __uint_as_float(raw.x & 0xffff0000u);
@@ -161,6 +258,21 @@ __device__ __forceinline__ void store_bf16_row(const uint2 &raw, int lane, uint8
         const uint32_t hi = stage[stored_dim<16, IS_V>(q, w, 1)];
         reinterpret_cast<uint32_t *>(dst)[word] = lo | (hi << 16);
     }
+}
+
+// Codec 1 record of BITS-bit codes: [K codes][V codes][K scales][V scales].
+template <int BITS>
+__device__ __forceinline__ void pack_record_fp(const uint2 &rk, const uint2 &rv, uint8_t *rec, int lane,
+                                               uint8_t *stage) {
+    constexpr int cb = kD * BITS / 8;
+    constexpr int sb = BITS == 4 ? kD / 16 : 2 * kNG;   // scale bytes of one block
+    float x[4];
+    row_floats(rk, x);
+    quantize_row_fp<BITS>(x, lane, rec + 2 * cb, stage);
+    if (lane < 4 * BITS) reinterpret_cast<uint32_t *>(rec)[lane] = code_word<BITS, false>(stage, lane);
+    row_floats(rv, x);
+    quantize_row_fp<BITS>(x, lane, rec + 2 * cb + sb, stage);
+    if (lane < 4 * BITS) reinterpret_cast<uint32_t *>(rec + cb)[lane] = code_word<BITS, true>(stage, lane);
 }
 
 // Packs one record from this lane's 4 elements of the K and V rows (raw bf16 pairs).
@@ -240,11 +352,19 @@ __global__ void __launch_bounds__(256) append_pack_kernel(
     }
     uint8_t *rec = d.pool[c] + ((size_t)s * cap + slot) * d.rec[c];
     uint8_t *stage = stage_all + (threadIdx.x >> 5) * 2 * kD;
-    switch (c) {
-        case 0: pack_record<16>(rk, rv, rec, lane, stage); break;
-        case 1: pack_record<8>(rk, rv, rec, lane, stage); break;
-        case 2: pack_record<4>(rk, rv, rec, lane, stage); break;
-        default: pack_record<2>(rk, rv, rec, lane, stage); break;
+    if (d.codec == 0 || c == 0) {
+        switch (c) {
+            case 0: pack_record<16>(rk, rv, rec, lane, stage); break;
+            case 1: pack_record<8>(rk, rv, rec, lane, stage); break;
+            case 2: pack_record<4>(rk, rv, rec, lane, stage); break;
+            default: pack_record<2>(rk, rv, rec, lane, stage); break;
+        }
+    } else {
+        switch (c) {
+            case 1: pack_record_fp<8>(rk, rv, rec, lane, stage); break;
+            case 2: pack_record_fp<4>(rk, rv, rec, lane, stage); break;
+            default: pack_record_fp<2>(rk, rv, rec, lane, stage); break;
+        }
     }
     __syncwarp();  // every lane has read the pre-call counters
     if (kSingle && lane == 0) {

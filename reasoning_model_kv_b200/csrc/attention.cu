@@ -44,6 +44,8 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <type_traits>
+
 #include "attn_common.cuh"
 
 namespace tkv {
@@ -74,7 +76,7 @@ struct WarpState {
 // STRIDE; int8 odd rows chunk-swizzled when SWZ).  Lane (g, tig) owns rows g and
 // g + 8.  Rows at or beyond nr hold zeros (the copy zero-fills them); their logits
 // are masked to -inf, so they contribute p = 0 everywhere.
-template <int BITS, int ROWS, int STRIDE, int G, bool SWZ>
+template <int BITS, int ROWS, int STRIDE, int G, bool SWZ, int FMT = 0>
 __device__ __forceinline__ void tile_compute(const uint8_t *st, int nr, int lane,
                                              const uint32_t (&qb)[4][2][2], const uint32_t (&qbb)[4][2][2],
                                              const float (&qs)[2][4], const float (&qinv)[2][4], bool qscaled,
@@ -104,14 +106,24 @@ __device__ __forceinline__ void tile_compute(const uint8_t *st, int nr, int lane
 #pragma unroll
             for (int i = 0; i < BITS; ++i) k1[i] = 0u;
         }
-        if constexpr (BITS < 16) {
-            load_meta(r0 + km_off0, km0);
-            load_meta(r1 + km_off1, km1);
+        if constexpr (FMT == 1) {
+            // scales: fp16 per group (FP8, ternary) or E4M3 per 16 dims (NVFP4) at 2 CB
+            const uint2 ka = *reinterpret_cast<const uint2 *>(r0 + 2 * CB);
+            const uint2 kc = *reinterpret_cast<const uint2 *>(r1 + 2 * CB);
+            qk_group_fp<BITS, 0>(x, k0, k1, qb, qinv, qscaled, ka, kc, tig);
+            qk_group_fp<BITS, 1>(x, k0, k1, qb, qinv, qscaled, ka, kc, tig);
+            qk_group_fp<BITS, 2>(x, k0, k1, qb, qinv, qscaled, ka, kc, tig);
+            qk_group_fp<BITS, 3>(x, k0, k1, qb, qinv, qscaled, ka, kc, tig);
+        } else {
+            if constexpr (BITS < 16) {
+                load_meta(r0 + km_off0, km0);
+                load_meta(r1 + km_off1, km1);
+            }
+            qk_group<BITS, 0>(x, k0, k1, qb, qbb, qs, qinv, qscaled, km0, km1, magic);
+            qk_group<BITS, 1>(x, k0, k1, qb, qbb, qs, qinv, qscaled, km0, km1, magic);
+            qk_group<BITS, 2>(x, k0, k1, qb, qbb, qs, qinv, qscaled, km0, km1, magic);
+            qk_group<BITS, 3>(x, k0, k1, qb, qbb, qs, qinv, qscaled, km0, km1, magic);
         }
-        qk_group<BITS, 0>(x, k0, k1, qb, qbb, qs, qinv, qscaled, km0, km1, magic);
-        qk_group<BITS, 1>(x, k0, k1, qb, qbb, qs, qinv, qscaled, km0, km1, magic);
-        qk_group<BITS, 2>(x, k0, k1, qb, qbb, qs, qinv, qscaled, km0, km1, magic);
-        qk_group<BITS, 3>(x, k0, k1, qb, qbb, qs, qinv, qscaled, km0, km1, magic);
     }
     const bool h0 = 2 * tig < G, h1 = 2 * tig + 1 < G;
     x[0] = (v0 && h0) ? x[0] * xscale : -INFINITY;
@@ -179,6 +191,24 @@ __device__ __forceinline__ void tile_compute(const uint8_t *st, int nr, int lane
         }
 #pragma unroll
         for (int grp = 0; grp < 4; ++grp) { bfr[grp][0] = b0; bfr[grp][1] = b1; }
+    } else if constexpr (FMT == 1 && BITS == 4) {
+        // NVFP4 values are dequantised exactly in f16 (scale folded into V): P alone
+        const uint32_t b0 = transpose8x8(f32x2_to_f16x2(p[0], p[1]));
+        const uint32_t b1 = transpose8x8(f32x2_to_f16x2(p[2], p[3]));
+#pragma unroll
+        for (int grp = 0; grp < 4; ++grp) { bfr[grp][0] = b0; bfr[grp][1] = b1; }
+    } else if constexpr (FMT == 1) {
+        // FP8 / ternary: the group's fp16 scale folds into P; no zero term
+        const uint2 va = *reinterpret_cast<const uint2 *>(r0 + 2 * CB + 8);
+        const uint2 vc = *reinterpret_cast<const uint2 *>(r1 + 2 * CB + 8);
+        const float2 a01 = __half22float2(u32_as_h2(va.x)), a23 = __half22float2(u32_as_h2(va.y));
+        const float2 c01 = __half22float2(u32_as_h2(vc.x)), c23 = __half22float2(u32_as_h2(vc.y));
+        const float s0[4] = {a01.x, a01.y, a23.x, a23.y}, s1[4] = {c01.x, c01.y, c23.x, c23.y};
+#pragma unroll
+        for (int grp = 0; grp < 4; ++grp) {
+            bfr[grp][0] = transpose8x8(f32x2_to_f16x2(p[0] * s0[grp], p[1] * s0[grp]));
+            bfr[grp][1] = transpose8x8(f32x2_to_f16x2(p[2] * s1[grp], p[3] * s1[grp]));
+        }
     } else {
         float2 vm0[4], vm1[4];
         load_meta(r0 + vm_off0, vm0);
@@ -199,12 +229,31 @@ __device__ __forceinline__ void tile_compute(const uint8_t *st, int nr, int lane
 #pragma unroll
         for (int i = 0; i < BITS; ++i) w1[i] = 0u;
     }
+    // NVFP4: each row's E4M3 scale of block MT (dims 16 MT .. 16 MT + 15) as f16x2
+    uint2 vb0 = make_uint2(0u, 0u), vb1 = make_uint2(0u, 0u);
+    if constexpr (FMT == 1 && BITS == 4) {
+        vb0 = *reinterpret_cast<const uint2 *>(r0 + 2 * CB + 8);
+        vb1 = *reinterpret_cast<const uint2 *>(r1 + 2 * CB + 8);
+    }
+    auto vpair = [&](auto pc, const uint32_t (&w)[BITS], const uint2 &vb) -> uint32_t {
+        constexpr int P = decltype(pc)::value;
+        if constexpr (FMT == 1 && BITS == 4) {
+            const uint32_t code = ((P / 2 < 4 ? vb.x : vb.y) >> (8 * ((P / 2) & 3))) & 0xFFu;
+            return hmul2_u32(quarter_pair_fp<BITS, P>(w), e4m3_h2(code));
+        } else if constexpr (FMT == 1) {
+            return quarter_pair_fp<BITS, P>(w);
+        } else {
+            return quarter_pair<BITS, P>(w, magic);
+        }
+    };
 #define TKV_VMMA(MT)                                                                              \
     {                                                                                             \
-        const uint32_t e0 = transpose8x8(quarter_pair<BITS, 2 * (MT)>(w0, magic));                       \
-        const uint32_t e1 = transpose8x8(quarter_pair<BITS, 2 * (MT) + 1>(w0, magic));                   \
-        const uint32_t e2 = ROWS == 16 ? transpose8x8(quarter_pair<BITS, 2 * (MT)>(w1, magic)) : 0u;     \
-        const uint32_t e3 = ROWS == 16 ? transpose8x8(quarter_pair<BITS, 2 * (MT) + 1>(w1, magic)) : 0u; \
+        using P0 = std::integral_constant<int, 2 * (MT)>;                                         \
+        using P1 = std::integral_constant<int, 2 * (MT) + 1>;                                     \
+        const uint32_t e0 = transpose8x8(vpair(P0{}, w0, vb0));                                   \
+        const uint32_t e1 = transpose8x8(vpair(P1{}, w0, vb0));                                   \
+        const uint32_t e2 = ROWS == 16 ? transpose8x8(vpair(P0{}, w1, vb1)) : 0u;                 \
+        const uint32_t e3 = ROWS == 16 ? transpose8x8(vpair(P1{}, w1, vb1)) : 0u;                 \
         if constexpr (BITS == 16) {                                                               \
             mma16816_bf16(ws.o[MT], e0, e1, e2, e3, bfr[(MT) >> 1][0], bfr[(MT) >> 1][1]);        \
             mma16816_bf16(ws.o[MT], e0, e1, e2, e3, blo0, blo1);                                  \
@@ -216,6 +265,18 @@ __device__ __forceinline__ void tile_compute(const uint8_t *st, int nr, int lane
 #undef TKV_VMMA
 }
 
+// Record bytes, reuse-placement stage row stride and rows per tile of class C_ under
+// codec CODEC.  Int8 rows (codec 0) are unpadded and chunk-swizzled on odd rows (SWZ);
+// the other strides make a quad's row reads fall in distinct banks.
+template <int C_, int CODEC>
+struct ClassShape {
+    static constexpr int REC = C_ == 0 ? 512 : CODEC == 0 ? (C_ == 1 ? 288 : C_ == 2 ? 160 : 96)
+                                                          : (C_ == 1 ? 272 : C_ == 2 ? 144 : 80);
+    static constexpr int STRIDE = C_ == 0 ? 528 : (CODEC == 0 && C_ == 2) ? 192 : REC;
+    static constexpr int ROWS = C_ == 0 ? 8 : 16;
+    static constexpr bool SWZ = CODEC == 0 && C_ == 1;
+};
+
 // Copy a tile of class C_ into a stage with coalesced 16-byte cp.async: eight
 // consecutive lanes cover 128 contiguous bytes of one record, so one instruction
 // reads four whole 128-byte lines (records r = lane/8 + 4i).  `hd` holds, in lane
@@ -223,12 +284,11 @@ __device__ __forceinline__ void tile_compute(const uint8_t *st, int nr, int lane
 // or beyond nr are zero-filled without reading memory, so the copy has no
 // branches and the compute reads zeros (finite) there.  Int8 rows are unpadded and
 // odd rows store 16-byte chunk k at k ^ 1.
-template <int C_>
+template <int C_, int CODEC>
 __device__ __forceinline__ void issue_tile(uint32_t stage, const uint8_t *pool, int hd, int nr,
                                            int lane, uint64_t pol) {
-    constexpr int REC = C_ == 0 ? 512 : C_ == 1 ? 288 : C_ == 2 ? 160 : 96;
-    constexpr int STRIDE = C_ == 0 ? 528 : C_ == 1 ? 288 : C_ == 2 ? 192 : 96;
-    constexpr int ROWS = C_ == 0 ? 8 : 16;
+    using CS = ClassShape<C_, CODEC>;
+    constexpr int REC = CS::REC, STRIDE = CS::STRIDE, ROWS = CS::ROWS;
     constexpr int NCH = REC / 16;                  // 16-byte chunks per record
     constexpr int NBLK = (NCH + 7) / 8;            // 8-chunk blocks per record
     const int sub = lane & 7;
@@ -239,7 +299,7 @@ __device__ __forceinline__ void issue_tile(uint32_t stage, const uint8_t *pool, 
         const uint32_t bytes = r < nr ? 16u : 0u;
         const uint8_t *src = pool + (size_t)slot * REC + 16 * sub;
         int dpos = 16 * sub;
-        if constexpr (C_ == 1) dpos += (r & 1) ? ((sub & 1) ? -16 : 16) : 0;   // k ^ 1 on odd rows
+        if constexpr (CS::SWZ) dpos += (r & 1) ? ((sub & 1) ? -16 : 16) : 0;   // k ^ 1 on odd rows
         const uint32_t dst = stage + r * STRIDE + dpos;
 #pragma unroll
         for (int j = 0; j < NBLK; ++j)
@@ -251,11 +311,10 @@ __device__ __forceinline__ void issue_tile(uint32_t stage, const uint8_t *pool, 
 // copied by one bulk copy into an unpadded stage (row stride REC).  Rows nr..ROWS-1
 // of the stage are zeroed first by the warp (generic stores, then a proxy fence so
 // they are ordered before later bulk writes of the stage).
-template <int C_>
+template <int C_, int CODEC>
 __device__ __forceinline__ void issue_tile_dense(uint8_t *stage_ptr, uint32_t stage, const uint8_t *src,
                                                  int nr, int lane, uint32_t bar, uint64_t pol) {
-    constexpr int REC = C_ == 0 ? 512 : C_ == 1 ? 288 : C_ == 2 ? 160 : 96;
-    constexpr int ROWS = C_ == 0 ? 8 : 16;
+    constexpr int REC = ClassShape<C_, CODEC>::REC, ROWS = ClassShape<C_, CODEC>::ROWS;
     if (nr < ROWS) {
         uint4 *z = reinterpret_cast<uint4 *>(stage_ptr + nr * REC);
         const int nz = (ROWS - nr) * (REC / 16);
@@ -270,7 +329,7 @@ __device__ __forceinline__ void issue_tile_dense(uint8_t *stage_ptr, uint32_t st
     }
 }
 
-template <int G, bool DENSE>
+template <int G, bool DENSE, int CODEC>
 __global__ void __launch_bounds__(kThreads, TKV_ATTN_MIN_BLOCKS) attn_kernel(const __grid_constant__ Dev d,
                                                            const __nv_bfloat16 *__restrict__ q,
                                                            float xscale, float *__restrict__ out,
@@ -422,17 +481,23 @@ __global__ void __launch_bounds__(kThreads, TKV_ATTN_MIN_BLOCKS) attn_kernel(con
             uint8_t *sp = ring_w + stage * kStageBytes;
             const uint32_t bar = bar0 + 8 * stage;
             switch (c) {
-                case 0: issue_tile_dense<0>(sp, st, pool + (size_t)e * 512, nr, lane, bar, pol); break;
-                case 1: issue_tile_dense<1>(sp, st, pool + (size_t)e * 288, nr, lane, bar, pol); break;
-                case 2: issue_tile_dense<2>(sp, st, pool + (size_t)e * 160, nr, lane, bar, pol); break;
-                default: issue_tile_dense<3>(sp, st, pool + (size_t)e * 96, nr, lane, bar, pol); break;
+                case 0: issue_tile_dense<0, CODEC>(sp, st, pool + (size_t)e * 512, nr, lane, bar, pol); break;
+                case 1:
+                    issue_tile_dense<1, CODEC>(sp, st, pool + (size_t)e * ClassShape<1, CODEC>::REC, nr, lane, bar, pol);
+                    break;
+                case 2:
+                    issue_tile_dense<2, CODEC>(sp, st, pool + (size_t)e * ClassShape<2, CODEC>::REC, nr, lane, bar, pol);
+                    break;
+                default:
+                    issue_tile_dense<3, CODEC>(sp, st, pool + (size_t)e * ClassShape<3, CODEC>::REC, nr, lane, bar, pol);
+                    break;
             }
         } else {
             switch (c) {
-                case 0: issue_tile<0>(st, pool, hd, nr, lane, pol); break;
-                case 1: issue_tile<1>(st, pool, hd, nr, lane, pol); break;
-                case 2: issue_tile<2>(st, pool, hd, nr, lane, pol); break;
-                default: issue_tile<3>(st, pool, hd, nr, lane, pol); break;
+                case 0: issue_tile<0, CODEC>(st, pool, hd, nr, lane, pol); break;
+                case 1: issue_tile<1, CODEC>(st, pool, hd, nr, lane, pol); break;
+                case 2: issue_tile<2, CODEC>(st, pool, hd, nr, lane, pol); break;
+                default: issue_tile<3, CODEC>(st, pool, hd, nr, lane, pol); break;
             }
         }
     };
@@ -473,28 +538,23 @@ __global__ void __launch_bounds__(kThreads, TKV_ATTN_MIN_BLOCKS) attn_kernel(con
         hr2 = handle_of(dr2);
         arrive_wait(stage);
     };
-#define TKV_CONSUME(CLS, BITS, ROWS, STRIDE, PLO, PHI, LO, HI, OFF)                               \
+#define TKV_CONSUME(CLS, BITS, PLO, PHI, LO, HI, OFF)                                             \
     for (; T < (PHI); T += kWarps) {                                                          \
+        using CS = ClassShape<CLS, CODEC>;                                                    \
         produce();                                                                            \
-        const int e = (LO) + (T - (PLO)) * (ROWS);                                            \
-        const int nr = min((ROWS), (HI) - e);                                                 \
-        tile_compute<BITS, ROWS, STRIDE, G, !DENSE>(ring + (warp * kStages + stage) * kStageBytes, \
-                                                    nr, lane, qb, qbb, qs, qinv, qscaled, xscale, ws, \
-                                                    lgs + (size_t)((OFF) + e) * G, magic);    \
+        const int e = (LO) + (T - (PLO)) * CS::ROWS;                                          \
+        const int nr = min(CS::ROWS, (HI) - e);                                               \
+        tile_compute<BITS, CS::ROWS, (DENSE ? CS::REC : CS::STRIDE), G, (!DENSE && CS::SWZ),  \
+                     ((CLS) > 0 ? CODEC : 0)>(ring + (warp * kStages + stage) * kStageBytes,  \
+                                            nr, lane, qb, qbb, qs, qinv, qscaled, xscale, ws, \
+                                            lgs + (size_t)((OFF) + e) * G, magic);            \
         __syncwarp();                                                                         \
         stage = stage == 2 ? 0 : stage + 1;                                                   \
     }
-    if constexpr (DENSE) {
-        TKV_CONSUME(0, 16, 8, 512, 0, p1, lo0, hi0, 0)
-        TKV_CONSUME(1, 8, 16, 288, p1, p2, lo1, hi1, o1)
-        TKV_CONSUME(2, 4, 16, 160, p2, p3, lo2, hi2, o2)
-        TKV_CONSUME(3, 2, 16, 96, p3, p4, lo3, hi3, o3)
-    } else {
-        TKV_CONSUME(0, 16, 8, 528, 0, p1, lo0, hi0, 0)
-        TKV_CONSUME(1, 8, 16, 288, p1, p2, lo1, hi1, o1)
-        TKV_CONSUME(2, 4, 16, 192, p2, p3, lo2, hi2, o2)
-        TKV_CONSUME(3, 2, 16, 96, p3, p4, lo3, hi3, o3)
-    }
+    TKV_CONSUME(0, 16, 0, p1, lo0, hi0, 0)
+    TKV_CONSUME(1, 8, p1, p2, lo1, hi1, o1)
+    TKV_CONSUME(2, 4, p2, p3, lo2, hi2, o2)
+    TKV_CONSUME(3, 2, p3, p4, lo3, hi3, o3)
 #undef TKV_CONSUME
     if constexpr (!DENSE) cp_async_wait_0();
 
@@ -603,15 +663,15 @@ __global__ void __launch_bounds__(kThreads, TKV_ATTN_MIN_BLOCKS) attn_kernel(con
     if (C > 1) cluster_sync();   // peers may still be reading this CTA's shared memory
 }
 
-int g_blocks_per_sm[2][kMaxG + 1][kMaxDevices] = {};   // per placement, G and device
+int g_blocks_per_sm[2][2][kMaxG + 1][kMaxDevices] = {};   // per codec, placement, G and device
 
-template <int G, bool DENSE>
+template <int G, bool DENSE, int CODEC>
 cudaError_t launch_g(const Dev &d, const void *q, float scale, float *out, long long live_ub,
                      cudaStream_t st, int64_t *launches) {
     int sms = 0, bps = 0;
     cudaError_t e0 = device_sm_count(&sms);
     if (e0 != cudaSuccess) return e0;
-    e0 = cached_blocks_per_sm(g_blocks_per_sm[DENSE][G], reinterpret_cast<const void *>(attn_kernel<G, DENSE>),
+    e0 = cached_blocks_per_sm(g_blocks_per_sm[CODEC][DENSE][G], reinterpret_cast<const void *>(attn_kernel<G, DENSE, CODEC>),
                               kThreads, kRingBytes, &bps);
     if (e0 != cudaSuccess) return e0;
     // Largest cluster (<= 8) whose grid is fully resident, never splitting a stream
@@ -636,7 +696,7 @@ cudaError_t launch_g(const Dev &d, const void *q, float scale, float *out, long 
     cfg.attrs = attr;
     cfg.numAttrs = 2;
     const float xscale = scale * 1.4426950408889634f;   // logits in the log2 domain
-    cudaError_t e = cudaLaunchKernelEx(&cfg, attn_kernel<G, DENSE>, d, static_cast<const __nv_bfloat16 *>(q),
+    cudaError_t e = cudaLaunchKernelEx(&cfg, attn_kernel<G, DENSE, CODEC>, d, static_cast<const __nv_bfloat16 *>(q),
                                        xscale, out, (int)C);
     *launches += 1;
     return e;
@@ -646,24 +706,22 @@ cudaError_t launch_g(const Dev &d, const void *q, float scale, float *out, long 
 
 cudaError_t launch_attention(const Dev &d, const void *q, float scale, float *out, long long live_ub,
                              cudaStream_t st, int64_t *launches) {
-    if (d.dense && d.attn_kernel == 1)
-        return launch_attention_i8(d, q, scale, out, nullptr, nullptr, 0.f, 0.f, live_ub, st, launches);
-    if (d.dense) {
-        switch (d.G) {
-            case 1: return launch_g<1, true>(d, q, scale, out, live_ub, st, launches);
-            case 2: return launch_g<2, true>(d, q, scale, out, live_ub, st, launches);
-            case 4: return launch_g<4, true>(d, q, scale, out, live_ub, st, launches);
-            case 8: return launch_g<8, true>(d, q, scale, out, live_ub, st, launches);
-            default: return cudaErrorInvalidValue;
-        }
+    if (d.dense && d.attn_kernel == 1) return cudaErrorInvalidValue;   // launch_attention_i8's
+#define TKV_G_CASES(DN, CD)                                                           \
+    switch (d.G) {                                                                    \
+        case 1: return launch_g<1, DN, CD>(d, q, scale, out, live_ub, st, launches);  \
+        case 2: return launch_g<2, DN, CD>(d, q, scale, out, live_ub, st, launches);  \
+        case 4: return launch_g<4, DN, CD>(d, q, scale, out, live_ub, st, launches);  \
+        case 8: return launch_g<8, DN, CD>(d, q, scale, out, live_ub, st, launches);  \
+        default: return cudaErrorInvalidValue;                                        \
     }
-    switch (d.G) {
-        case 1: return launch_g<1, false>(d, q, scale, out, live_ub, st, launches);
-        case 2: return launch_g<2, false>(d, q, scale, out, live_ub, st, launches);
-        case 4: return launch_g<4, false>(d, q, scale, out, live_ub, st, launches);
-        case 8: return launch_g<8, false>(d, q, scale, out, live_ub, st, launches);
-        default: return cudaErrorInvalidValue;
+    if (d.codec == 0) {
+        if (d.dense) TKV_G_CASES(true, 0)
+        TKV_G_CASES(false, 0)
     }
+    if (d.dense) TKV_G_CASES(true, 1)
+    TKV_G_CASES(false, 1)
+#undef TKV_G_CASES
 }
 
 }  // namespace tkv

@@ -7,46 +7,53 @@
 // statement).
 //
 // Two kernels.  attn_i8_kernel runs one persistent CTA per SM.  The work of the
-// whole step -- every stream's class tables cut into class-homogeneous tiles
-// (64 records for bf16, 112 for int8, 128 for int4 / int2) -- is laid on one line
-// weighted by bytes (+ a fixed cost per tile), and CTA c takes the tiles that
-// start in the c-th equal share, so every SM streams the same number of bytes
-// whatever the streams' lengths and class mixes.  A stream split over several
-// CTAs leaves one partial (running max m, sum l, O) per CTA; attn_finalize_kernel
-// merges the partials of each stream, writes the output and adds p to the scores
-// (from the raw logits the first kernel left in an L2-resident scratch).
+// whole step -- every stream's class tables cut into class-homogeneous tiles (64
+// records for bf16, 128 for int8 / int4 / int2) -- is laid on one line weighted by
+// bytes (+ a fixed cost per tile), and CTA c takes the tiles that start in the c-th
+// equal share, so every SM streams the same number of bytes whatever the streams'
+// lengths and class mixes.  Each (stream, CTA, warpgroup) leaves one partial
+// (running max m, sum l, sum p*(x - m), O); attn_finalize_kernel merges the
+// partials of each stream, writes the output and adds p to the scores (from the raw
+// logits the first kernel left in an L2-resident scratch).
 //
-// Roles inside a CTA (320 threads):
-//   warp 0      producer: one bulk copy per tile into a 3-deep ring of raw stages;
-//   warp 1      tensor-memory owner and MMA issuer (one thread);
-//   warps 2-5   stager: thread r takes record r of the tile, puts its K and V
-//               codes in head-dim order into the MMA operand layouts in shared
-//               memory (int4 / int2 codes widened to one byte each), copies the
-//               scale / zero block, and builds the query operands per stream;
-//   warps 6-9   softmax: thread r owns row r of the tile's accumulators in tensor
-//               memory (token r for QK, head dim r for PV).
+// Memory path.  A tile arrives by TMA in 2-3 boxes whose 32- to 128-byte rows are
+// the records' K codes, V codes and scale / zero block, written with the matching
+// hardware swizzle: int8 K and V then ARE the MMA operands (K-major and MN-major
+// layouts with 128-byte swizzle), with no copy through registers.  int4 / int2 codes
+// are widened to bytes in the int8 records' element order: K into tensor memory (the
+// A operand of QK), V into a swizzled shared buffer; bf16 keys are the A operand as
+// they arrive, bf16 values are regathered into the same element order.
 //
-// Math (per tile; exact integer products, no per-element dequantisation):
-//   QK  q is written once per stream as three signed 8-bit digits per element,
-//       q = (d0 * 2^14 + d1 * 2^7 + d2) * 2^(E_gh - 146), E_gh the exponent of the
-//       largest |q| of head h in group g (exact for every bf16 within 2^12 of that
-//       largest value), so for each 32-dim group g one kind::i8 MMA (A = the
-//       tile's codes, u8; B = the digits, s8; M 128, K 32) gives
-//       c_s = sum_d code_d * digit_s,d exactly in s32.  Thread t folds
+// Roles (320 threads): warp 0 issues the TMA boxes and publishes each tile's
+// descriptor; warp 1 owns tensor memory and issues the MMAs (one thread); warps 2-5
+// and 6-9 are two compute warpgroups taking alternate tiles: thread r widens row r,
+// owns row r of the QK accumulators (token r) and of the PV accumulators (head dim
+// r of the int8 element order), forms logits, softmax and the PV operand.
+//
+// Math (per tile):
+//   QK  q is written once per stream and warpgroup as three signed 8-bit digits per
+//       element, q = (d0 * 2^14 + d1 * 2^7 + d2) * 2^(E_gh - 146), E_gh the exponent
+//       of the largest |q| of head h in 32-dim group g (exact for every bf16 within
+//       2^12 of that largest value); one kind::i8 MMA chain (A = codes, u8; B = the
+//       digits, s8, zero outside the column's group; M 128, K 128) gives
+//       c_s = sum_{d in g} code_d * digit_s,d exactly in s32.  Thread t folds
 //       x_h = sum_g kscale_g * 2^(E_gh-146) * (c0 2^14 + c1 2^7 + c2) + kzero_g * sum_g(q_h).
 //   PV  W_t,(g,h) = p_h,t * vscale_g,t becomes an unsigned integer below 2^22 under a
-//       per-tile power-of-two scale; its three bytes are three u8 columns, so one
-//       kind::i8 MMA chain (A = V codes, MN-major, M = 128 head dims; B = W,
-//       MN-major; K = the tile's tokens) gives exact s32 byte sums, which thread
-//       d scales back into its fp32 O; the zero term sum_t p * vzero_g is
-//       accumulated by the token threads in fp32.
-//   bf16 tiles (protected tokens) use kind::f16 with bf16 operands: q exact, P
-//   split into a bf16 high and low part (two columns), so nothing is narrowed.
+//       per-tile power-of-two scale; its bytes are u8 columns, so one kind::i8 MMA
+//       chain (A = V codes, M = 128 head dims; B = W; K = the tile's tokens) gives
+//       exact s32 byte sums, which thread d scales back into its fp32 O; the zero
+//       term sum_t p * vzero_g is accumulated by the token threads in fp32.
+//   bf16 tiles (protected tokens) use kind::f16 with bf16 operands: q exact, P split
+//   into a bf16 high and low part (two columns), so nothing is narrowed.
 // The running max only moves (and l, O are rescaled) when a tile exceeds it by
 // more than 2^8.
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstring>
 
 #include "attn_common.cuh"
 
@@ -56,39 +63,43 @@ namespace {
 using namespace attn;
 
 constexpr int kThreads = 320;
-constexpr int kRawStages = 3;
-constexpr int kRawBytes = 32768;      // >= rows * record bytes of every class
-constexpr int kStgBytes = 32768;      // staged K (16 KB) + V (16 KB)
-constexpr int kStgV = 16384;
-constexpr int kMetaBytes = 5120;      // 128 rows x 32 B of fp16 scale / zero + vmax header (4 warps x 4)
-constexpr int kMetaHdr = 4096;
+constexpr int kRawBytes = 36864;      // a tile's boxes: int8 128 x (128 K + 128 V + 32 meta)
+constexpr int kStgV = 16384;          // widened V of one tile (128 rows x 128 B)
 constexpr int kTileOverhead = 4096;   // cost of a tile beyond its bytes, for the work split
 constexpr int kTmemCols = 512;
 constexpr int kMaxStreamTable = 64;   // streams whose counts a CTA keeps in shared memory
 
-__host__ __device__ constexpr int rows_of(int c) { return c == 0 ? 64 : c == 1 ? 112 : 128; }
+__host__ __device__ constexpr int raw_stages(int G) { return G <= 4 ? 4 : 3; }
+__host__ __device__ constexpr int rows_of(int c) { return c == 0 ? 64 : 128; }
 __host__ __device__ constexpr int rec_of(int c) { return c == 0 ? 512 : c == 1 ? 288 : c == 2 ? 160 : 96; }
-__host__ __device__ constexpr int ng_of(int G) { return 3 * G <= 16 ? 16 : 32; }   // QK columns per group
-__host__ __device__ constexpr int gs_of(int G) { return 4 * G < 16 ? 16 : 4 * G; }  // PV columns per group
+// box layout inside a raw stage: K, V and meta offsets and the bytes a tile's boxes bring
+__host__ __device__ constexpr int v_off(int c) { return c == 0 ? 16384 : c == 1 ? 16384 : c == 2 ? 8192 : 4096; }
+__host__ __device__ constexpr int meta_off(int c) { return c == 1 ? 32768 : c == 2 ? 16384 : 8192; }
+__host__ __device__ constexpr int tile_bytes(int c) { return c == 0 ? 32768 : c == 1 ? 36864 : c == 2 ? 20480 : 12288; }
+__host__ __device__ constexpr int code_box_bytes(int c) { return c <= 1 ? 128 : c == 2 ? 64 : 32; }
+__host__ __device__ constexpr int ns_of(int G) { return (12 * G + 15) / 16 * 16; }   // QK columns (i8 tiles)
+__host__ __device__ constexpr int gs_of(int G) { return 4 * G < 16 ? 16 : 4 * G; }   // PV columns per group
 __host__ __device__ constexpr int no_of(int G) { return 4 * gs_of(G); }              // PV columns (i8 tiles)
 __host__ __device__ constexpr int w_bytes(int G) { return 128 * no_of(G); }
-__host__ __device__ constexpr int qi8_bytes(int G) { return 4 * 32 * ng_of(G); }
+constexpr uint32_t kSw128 = 2;        // shared-memory descriptor layout: 128-byte swizzle
+__host__ __device__ constexpr int qi8_bytes(int G) { return 128 * ns_of(G); }
 constexpr int kQbfBytes = 16 * 128 * 2;
 __host__ __device__ constexpr int align1k(int x) { return (x + 1023) & ~1023; }
 __host__ __device__ constexpr int q_bytes(int G) { return align1k(qi8_bytes(G) + kQbfBytes + 2 * 4 * kMaxG * 4); }
-// dynamic shared memory layout (from a 1024-byte aligned base)
+// dynamic shared memory layout (from a 1024-byte aligned base); per warpgroup wg: the
+// widened V, the PV operand W and the query operands
 constexpr int kOffRaw = 0;
-constexpr int kOffStg = kOffRaw + kRawStages * kRawBytes;
-constexpr int kOffMeta = kOffStg + 2 * kStgBytes;
-constexpr int kOffW = kOffMeta + 2 * kMetaBytes;
-__host__ __device__ constexpr int off_q(int G) { return kOffW + 2 * w_bytes(G); }
+__host__ __device__ constexpr int off_stg(int G) { return kOffRaw + raw_stages(G) * kRawBytes; }
+__host__ __device__ constexpr int off_w(int G) { return off_stg(G) + 2 * kStgV; }
+__host__ __device__ constexpr int off_q(int G) { return off_w(G) + 2 * w_bytes(G); }
 __host__ __device__ constexpr int smem_bytes(int G) { return 1024 + off_q(G) + 2 * q_bytes(G); }
-// tensor memory: buffer b holds the QK accumulators at column 256b and the PV
-// accumulators at column 256b + 128
-__host__ __device__ constexpr uint32_t col_s(int b) { return 256u * b; }
-__host__ __device__ constexpr uint32_t col_o(int b) { return 256u * b + 128u; }
+// tensor memory of warpgroup wg: widened K at 256 wg, QK accumulators at 256 wg + 32,
+// PV accumulators at 256 wg + 128
+__host__ __device__ constexpr uint32_t col_a(int wg) { return 256u * wg; }
+__host__ __device__ constexpr uint32_t col_s(int wg) { return 256u * wg + 32u; }
+__host__ __device__ constexpr uint32_t col_o(int wg) { return 256u * wg + 128u; }
 
-// ------------------------------------------------------------ tcgen05 wrappers
+// ------------------------------------------------------------ tcgen05 / TMA wrappers
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t cols) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(cols)
                  : "memory");
@@ -100,12 +111,12 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t cols) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-// Shared-memory matrix descriptor without swizzle: lbo = byte stride between core
-// matrices along K, sbo = along M / N (both multiples of 16).
-__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+// Shared-memory matrix descriptor: lbo / sbo in bytes, layout 0 = no swizzle, 2 = 128B swizzle.
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo, uint32_t layout = 0) {
     return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
-           ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46);
+           ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46) | ((uint64_t)layout << 61);
 }
 // Instruction descriptor: accumulator format (1 f32, 2 s32), A / B formats (kind::i8:
 // 0 u8, 1 s8; kind::f16: 1 bf16), A / B major (0 K, 1 MN), N, M = 128.
@@ -116,6 +127,13 @@ __host__ __device__ constexpr uint32_t idesc(uint32_t cfmt, uint32_t afmt, uint3
 __device__ __forceinline__ void mma_i8(uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
     asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
                  "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d), "l"(a), "l"(b), "r"(id),
+                 "r"(acc)
+                 : "memory");
+}
+// A in tensor memory
+__device__ __forceinline__ void mma_i8_tmem(uint32_t d, uint32_t a, uint64_t b, uint32_t id, uint32_t acc) {
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d), "r"(a), "l"(b), "r"(id),
                  "r"(acc)
                  : "memory");
 }
@@ -138,6 +156,14 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 __device__ __forceinline__ void named_sync(int id, int n) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar,
+                                            uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+        "[%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(policy)
+        : "memory");
+}
 
 #define TKV_LD_REGS16(r) "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), \
     "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
@@ -149,6 +175,27 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t *r) {
         : "memory");
 }
 #undef TKV_LD_REGS16
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t *r) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_ld4(uint32_t taddr, uint32_t *r) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(taddr)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
 
 // ------------------------------------------------------------ the work split
 struct Counts {
@@ -295,12 +342,12 @@ struct TileIter {
 };
 
 // The producer walks the tile sequence once and publishes each tile to the other roles
-// through a small ring in shared memory (written before the tile's copy is issued, so
-// a role that has waited for the tile's copy -- directly or through the stager's
-// barriers -- reads a complete descriptor).  No role lags the producer by more than
-// kDescRing - 4 tiles: the producer needs the raw stage of tile k - 3, which the stager
-// releases only after staging it, which needs tile k - 5's PV complete, which needs its
-// softmax done.
+// through a small ring in shared memory (written before the tile's copies are issued,
+// so a role that has waited for the tile's copies -- directly or through a warpgroup's
+// barrier -- reads a complete descriptor).  No role lags the producer by more than a
+// few tiles: the producer reuses the stage of tile k - R only after that tile's PV has
+// completed, and the MMA issuer takes tiles in order, so neither warpgroup can run more
+// than two tiles ahead of the other.
 constexpr int kDescRing = 16;
 struct __align__(16) TileDesc {
     int32_t s;       // stream
@@ -372,170 +419,125 @@ __device__ void plan_work(const Dev &d, SharedPlan &pl, int cta, int ncta) {
     __syncthreads();
 }
 
-// ------------------------------------------------------------ staging (code order)
-// Head-dim ("natural") order for the MMA operands.  Word layouts of the records:
-// see stored_dim in append.cu.  Each function writes the 16-byte chunk kc of the
-// row's natural-order codes as 4 words (K: K-major rows; V: MN-major columns --
-// the same byte formula for both: chunk kc at kc*2048 + (r/8)*128 + (r%8)*16).
 
+
+// ------------------------------------------------------------ widening to the int8 element order
+// All classes are brought to the element order of the int8 records (tkv.h: quarters of
+// 32-bit words, word w of quarter q at byte 32q + 4w, pairs 16 bits apart), so one query
+// operand serves every integer class and the PV accumulator rows (= V byte positions)
+// mean the same head dim for every class.
+//   int4 word (q, w) of a code block (nibbles n0..n7) -> int8 words (q, 2w), (q, 2w+1):
+//     lo = nibbles 0,2,4,6; hi = nibbles 1,3,5,7; (q,2w) = [lo0 hi0 lo2 hi2], (q,2w+1) = [lo1 hi1 lo3 hi3]
+//   int2 word (q, w) (fields f0..f15) -> int8 words (q, 4w + m): e_k = field bytes k, k+4, k+8, k+12;
+//     m = 0: [e0.0 e1.0 e0.2 e1.2], 1: [e2.0 e3.0 e2.2 e3.2], 2: [e0.1 e1.1 e0.3 e1.3], 3: [e2.1 e3.1 e2.3 e3.3]
+// (the same for K and V blocks: both formats store head-dim pair p of quarter q in the
+// same place, only the pair -> dim maps of K and V differ, and those are shared).
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) { return __byte_perm(a, b, sel); }
 __device__ __forceinline__ void sts128(uint8_t *p, uint32_t a, uint32_t b, uint32_t c, uint32_t dd) {
     *reinterpret_cast<uint4 *>(p) = make_uint4(a, b, c, dd);
 }
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) { return __byte_perm(a, b, sel); }
 
-// int8: K word (q, w) holds dims base + {0, 2, 1, 3}, base = 32(w/2) + 8q + 4(w%2);
-// V word (q, w) holds dims 16w + 2q + {0, 8, 1, 9}.
-__device__ __forceinline__ void stage_row_i8(const uint8_t *rec, uint8_t *k_dst, uint8_t *v_dst) {
-    uint32_t kw[4][8], vw[4][8];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const uint4 a = *reinterpret_cast<const uint4 *>(rec + 32 * q);
-        const uint4 b = *reinterpret_cast<const uint4 *>(rec + 32 * q + 16);
-        kw[q][0] = a.x; kw[q][1] = a.y; kw[q][2] = a.z; kw[q][3] = a.w;
-        kw[q][4] = b.x; kw[q][5] = b.y; kw[q][6] = b.z; kw[q][7] = b.w;
-        const uint4 c = *reinterpret_cast<const uint4 *>(rec + 128 + 32 * q);
-        const uint4 e = *reinterpret_cast<const uint4 *>(rec + 128 + 32 * q + 16);
-        vw[q][0] = c.x; vw[q][1] = c.y; vw[q][2] = c.z; vw[q][3] = c.w;
-        vw[q][4] = e.x; vw[q][5] = e.y; vw[q][6] = e.z; vw[q][7] = e.w;
-    }
-    // K chunk kc = 2(w/2) + q/2, position 2(q%2) + w%2
-#pragma unroll
-    for (int kc = 0; kc < 8; ++kc) {
-        const int w0 = 2 * (kc / 2), q0 = 2 * (kc % 2);
-        sts128(k_dst + kc * 2048, prmt(kw[q0][w0], 0, 0x3120), prmt(kw[q0][w0 + 1], 0, 0x3120),
-               prmt(kw[q0 + 1][w0], 0, 0x3120), prmt(kw[q0 + 1][w0 + 1], 0, 0x3120));
-    }
-    // V chunk w: [p(0,1,0x6420), p(2,3,0x6420), p(0,1,0x7531), p(2,3,0x7531)]
-#pragma unroll
-    for (int w = 0; w < 8; ++w)
-        sts128(v_dst + w * 2048, prmt(vw[0][w], vw[1][w], 0x6420), prmt(vw[2][w], vw[3][w], 0x6420),
-               prmt(vw[0][w], vw[1][w], 0x7531), prmt(vw[2][w], vw[3][w], 0x7531));
+// Row r of a [row][64 B] box with 64-byte swizzle: the 16-byte chunk j of the row.
+__device__ __forceinline__ uint4 ld_sw64(const uint8_t *base, int r, int j) {
+    return *reinterpret_cast<const uint4 *>(base + r * 64 + 16 * (j ^ ((r >> 1) & 3)));
+}
+// Row r of a [row][32 B] box with 32-byte swizzle.
+__device__ __forceinline__ uint4 ld_sw32(const uint8_t *base, int r, int j) {
+    return *reinterpret_cast<const uint4 *>(base + r * 32 + 16 * (j ^ ((r >> 2) & 1)));
+}
+// Row r of a [row][128 B] box with 128-byte swizzle.
+__device__ __forceinline__ uint4 ld_sw128(const uint8_t *base, int r, int j) {
+    return *reinterpret_cast<const uint4 *>(base + r * 128 + 16 * (j ^ (r & 7)));
+}
+__device__ __forceinline__ void st_sw128(uint8_t *base, int r, int j, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    *reinterpret_cast<uint4 *>(base + r * 128 + 16 * (j ^ (r & 7))) = make_uint4(a, b, c, d);
 }
 
-// int4: K word (q, w) = group w, dims 32w + 8q + {0..7}, nibble e at offset
-// 2(e%4) + e/4; V word (q, w) nibble e = dim 32w + 8(e%4) + 2q + e/4.
-__device__ __forceinline__ void stage_row_i4(const uint8_t *rec, uint8_t *k_dst, uint8_t *v_dst) {
-    uint32_t kw[4][4], vw[4][4];
+// 32 int8-order words (128 bytes) of an int4 code block held as row r of a 64B-swizzled box.
+__device__ __forceinline__ void widen_i4(const uint8_t *box, int r, uint32_t (&o)[32]) {
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-        const uint4 a = *reinterpret_cast<const uint4 *>(rec + 16 * q);
-        kw[q][0] = a.x; kw[q][1] = a.y; kw[q][2] = a.z; kw[q][3] = a.w;
-        const uint4 b = *reinterpret_cast<const uint4 *>(rec + 64 + 16 * q);
-        vw[q][0] = b.x; vw[q][1] = b.y; vw[q][2] = b.z; vw[q][3] = b.w;
-    }
-    // K: natural words 8w + 2q + {0,1} = (prmt(lo,hi,0x6420), prmt(lo,hi,0x7531)); chunk 2w + q/2
+        const uint4 v = ld_sw64(box, r, q);
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
-        uint32_t nat[8];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const uint32_t lo = kw[q][w] & 0x0F0F0F0Fu, hi = (kw[q][w] >> 4) & 0x0F0F0F0Fu;
-            nat[2 * q] = prmt(lo, hi, 0x6420);
-            nat[2 * q + 1] = prmt(lo, hi, 0x7531);
+        for (int w = 0; w < 4; ++w) {
+            const uint32_t lo = w4[w] & 0x0F0F0F0Fu, hi = (w4[w] >> 4) & 0x0F0F0F0Fu;
+            o[8 * q + 2 * w] = prmt(lo, hi, 0x6240);
+            o[8 * q + 2 * w + 1] = prmt(lo, hi, 0x7351);
         }
-        sts128(k_dst + (2 * w) * 2048, nat[0], nat[1], nat[2], nat[3]);
-        sts128(k_dst + (2 * w + 1) * 2048, nat[4], nat[5], nat[6], nat[7]);
-    }
-    // V: natural word 8w + 2m + r from A = (2r, w), B = (2r+1, w); chunk 2w + m/2,
-    // position 2(m%2) + r
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-        uint32_t nat[8];
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            const uint32_t alo = vw[2 * r][w] & 0x0F0F0F0Fu, ahi = (vw[2 * r][w] >> 4) & 0x0F0F0F0Fu;
-            const uint32_t blo = vw[2 * r + 1][w] & 0x0F0F0F0Fu, bhi = (vw[2 * r + 1][w] >> 4) & 0x0F0F0F0Fu;
-            nat[2 * 0 + r] = prmt(alo, blo, 0x6420);   // m = 0
-            nat[2 * 1 + r] = prmt(ahi, bhi, 0x6420);   // m = 1
-            nat[2 * 2 + r] = prmt(alo, blo, 0x7531);   // m = 2
-            nat[2 * 3 + r] = prmt(ahi, bhi, 0x7531);   // m = 3
-        }
-        sts128(v_dst + (2 * w) * 2048, nat[0], nat[1], nat[2], nat[3]);
-        sts128(v_dst + (2 * w + 1) * 2048, nat[4], nat[5], nat[6], nat[7]);
     }
 }
-
-// int2: K word (q, w) field e = dim 32(2w + (e%8)/4) + 8q + 2(e%4) + e/8;
-// V word (q, w) field e = dim 64w + 8(e%8) + 2q + e/8.
-__device__ __forceinline__ void stage_row_i2(const uint8_t *rec, uint8_t *k_dst, uint8_t *v_dst) {
-    uint32_t kw[4][2], vw[4][2];
-    {
-        const uint4 a = *reinterpret_cast<const uint4 *>(rec);
-        const uint4 b = *reinterpret_cast<const uint4 *>(rec + 16);
-        kw[0][0] = a.x; kw[0][1] = a.y; kw[1][0] = a.z; kw[1][1] = a.w;
-        kw[2][0] = b.x; kw[2][1] = b.y; kw[3][0] = b.z; kw[3][1] = b.w;
-        const uint4 c = *reinterpret_cast<const uint4 *>(rec + 32);
-        const uint4 e = *reinterpret_cast<const uint4 *>(rec + 48);
-        vw[0][0] = c.x; vw[0][1] = c.y; vw[1][0] = c.z; vw[1][1] = c.w;
-        vw[2][0] = e.x; vw[2][1] = e.y; vw[3][0] = e.z; vw[3][1] = e.w;
-    }
-    // K: group 2w + gg, dims 8q + {0..3} = prmt(e0, e1, sel(gg)), 8q + {4..7} = prmt(e2, e3, sel(gg));
-    // natural word 16w + 8gg + 2q + {0,1}: chunk 4w + 2gg + q/2, position 2(q%2) + {0,1}
+// 32 int8-order words of an int2 code block held as row r of a 32B-swizzled box.
+__device__ __forceinline__ void widen_i2(const uint8_t *box, int r, uint32_t (&o)[32]) {
 #pragma unroll
-    for (int w = 0; w < 2; ++w) {
-        uint32_t nat[2][8];   // [gg][2q + half]
+    for (int j = 0; j < 2; ++j) {
+        const uint4 v = ld_sw32(box, r, j);   // quarters 2j (words x, y) and 2j + 1 (z, w)
+        const uint32_t w2[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const uint32_t x = kw[q][w];
+        for (int i = 0; i < 4; ++i) {
+            const int q = 2 * j + i / 2, w = i % 2;
+            const uint32_t x = w2[i];
             const uint32_t e0 = x & 0x03030303u, e1 = (x >> 2) & 0x03030303u;
             const uint32_t e2 = (x >> 4) & 0x03030303u, e3 = (x >> 6) & 0x03030303u;
-            nat[0][2 * q] = prmt(e0, e1, 0x6420);
-            nat[0][2 * q + 1] = prmt(e2, e3, 0x6420);
-            nat[1][2 * q] = prmt(e0, e1, 0x7531);
-            nat[1][2 * q + 1] = prmt(e2, e3, 0x7531);
-        }
-#pragma unroll
-        for (int gg = 0; gg < 2; ++gg) {
-            sts128(k_dst + (4 * w + 2 * gg) * 2048, nat[gg][0], nat[gg][1], nat[gg][2], nat[gg][3]);
-            sts128(k_dst + (4 * w + 2 * gg + 1) * 2048, nat[gg][4], nat[gg][5], nat[gg][6], nat[gg][7]);
-        }
-    }
-    // V: natural word 16w + 2m + r = prmt(A.e_{m%4}, B.e_{m%4}, m/4 ? 0x7531 : 0x6420), A = (2r, w),
-    // B = (2r+1, w); chunk 4w + m/2, position 2(m%2) + r
-#pragma unroll
-    for (int w = 0; w < 2; ++w) {
-        uint32_t nat[16];
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            const uint32_t A = vw[2 * r][w], Bw = vw[2 * r + 1][w];
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const uint32_t ea = (A >> (2 * kk)) & 0x03030303u, eb = (Bw >> (2 * kk)) & 0x03030303u;
-                nat[2 * kk + r] = prmt(ea, eb, 0x6420);         // m = kk
-                nat[2 * (kk + 4) + r] = prmt(ea, eb, 0x7531);   // m = kk + 4
-            }
-        }
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch)
-            sts128(v_dst + (4 * w + ch) * 2048, nat[4 * ch], nat[4 * ch + 1], nat[4 * ch + 2], nat[4 * ch + 3]);
-    }
-}
-
-// bf16: K word (q, w) = dims 32(w/4) + 8q + 2(w%4) + {0,1}: chunk kc (dims 8kc..8kc+7)
-// is the 16 bytes at 64(kc%4) + 16(kc/4); V word (q, w) = dims 8w + 2q + {0,1}: chunk
-// kc = words (q, kc) for q = 0..3.  Layout: chunk kc at kc*1024 + (r/8)*128 + (r%8)*16.
-__device__ __forceinline__ void stage_row_bf16(const uint8_t *rec, uint8_t *dst, bool is_v, int rot) {
-    // rows are 512 bytes apart, so every row starts on the same bank: each thread walks
-    // the chunks from a different starting chunk (rot = row) to spread a phase's loads
-    if (!is_v) {
-#pragma unroll 4
-        for (int i = 0; i < 16; ++i) {
-            const int kc = (i + rot) & 15;
-            *reinterpret_cast<uint4 *>(dst + kc * 1024) =
-                *reinterpret_cast<const uint4 *>(rec + 64 * (kc % 4) + 16 * (kc / 4));
-        }
-    } else {
-#pragma unroll 4
-        for (int i = 0; i < 16; ++i) {
-            const int kc = (i + rot) & 15;
-            const uint32_t *src = reinterpret_cast<const uint32_t *>(rec + 256 + 4 * kc);
-            sts128(dst + kc * 1024, src[0], src[16], src[32], src[48]);
+            o[8 * q + 4 * w + 0] = prmt(e0, e1, 0x6240);
+            o[8 * q + 4 * w + 1] = prmt(e2, e3, 0x6240);
+            o[8 * q + 4 * w + 2] = prmt(e0, e1, 0x7351);
+            o[8 * q + 4 * w + 3] = prmt(e2, e3, 0x7351);
         }
     }
 }
+// 32 int8-order words -> row r of a [row][128 B] 128B-swizzled buffer (chunk j = words 4j..4j+3)
+__device__ __forceinline__ void store_row_sw128(uint8_t *buf, int r, const uint32_t (&o)[32]) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) st_sw128(buf, r, j, o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+}
+// bf16 V of row r (two 128B-swizzled atoms of 64 rows) regathered into the int8 element
+// order, half `a` (positions 64a .. 64a + 63): output word u (positions 2u, 2u + 1) of
+// quarter q = u / 16, word w8 = (u % 16) / 2 takes the low (u even) or high (u odd)
+// halves of bf16 words (q, 2 w8) and (q, 2 w8 + 1) (bf16 word (q, w) sits at byte
+// 64 q + 4 w of the value block).  Output chunk c (8 positions) of atom a of the
+// staged buffer: row r, chunk c ^ (r % 8).
+__device__ __forceinline__ void regather_bf16_v(const uint8_t *vbox, uint8_t *stg, int r, int a) {
+    // the atom a of the value block holds quarters 2a, 2a + 1 (bytes 128 a .. 128 a + 127)
+    uint32_t w[2][16];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const uint4 v = ld_sw128(vbox + a * 8192, r, j);   // bytes 16 j.. of the atom: quarter 2a + j/4
+        w[j / 4][4 * (j % 4)] = v.x; w[j / 4][4 * (j % 4) + 1] = v.y;
+        w[j / 4][4 * (j % 4) + 2] = v.z; w[j / 4][4 * (j % 4) + 3] = v.w;
+    }
+    uint8_t *dst = stg + a * 8192;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {   // output chunk c holds words u = 32a + 4c .. + 3
+        uint32_t ow[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int u = 32 * a + 4 * c + i;
+            const int ql = (u / 16) - 2 * a, w8 = (u % 16) / 2;
+            ow[i] = prmt(w[ql][2 * w8], w[ql][2 * w8 + 1], (u & 1) ? 0x7632 : 0x5410);
+        }
+        st_sw128(dst, r, c, ow[0], ow[1], ow[2], ow[3]);
+    }
+}
 
-__device__ __forceinline__ void zero_row(uint8_t *dst, int nchunks, int stride) {
-    for (int i = 0; i < nchunks; ++i) *reinterpret_cast<uint4 *>(dst + i * stride) = make_uint4(0u, 0u, 0u, 0u);
+// Head dim of position m (0..127) of an int8 K / V block (tkv.h element order).
+__device__ __forceinline__ int dim_of_k8(int m) {
+    const int q = m >> 5, w = (m & 31) >> 2, e = m & 3;
+    return 32 * (w >> 1) + 8 * q + 4 * (w & 1) + ((e & 1) << 1) + (e >> 1);
+}
+__device__ __forceinline__ int dim_of_v8(int m) {
+    const int q = m >> 5, w = (m & 31) >> 2, e = m & 3;
+    return 16 * w + 8 * (e & 1) + 2 * q + (e >> 1);
+}
+// Position of head dim d in an int8 K block (inverse of dim_of_k8) and of bf16 K.
+__device__ __forceinline__ int pos_k8(int d) {
+    const int g = d >> 5, q = (d >> 3) & 3, o = d & 7;
+    const int w = 2 * g + (o >> 2), e = ((o & 1) << 1) | ((o >> 1) & 1);
+    return 32 * q + 4 * w + e;
+}
+__device__ __forceinline__ int pos_kbf(int d) {
+    const int g = d >> 5, q = (d >> 3) & 3, o = d & 7;
+    return 32 * q + 8 * g + o;
 }
 
 // Order-preserving uint32 image of a float (for max reductions with redux).
@@ -557,7 +559,6 @@ __device__ __forceinline__ float inv_pow2_ceil(float x, int &e_out) {
 __device__ __forceinline__ float pow2f(int e) {   // 2^e for -126 <= e <= 127
     return __uint_as_float((uint32_t)(e + 127) << 23);
 }
-__device__ __forceinline__ float i2f_exact(int32_t c) { return __int2float_rn(c); }
 
 template <int G>
 struct QConst {   // per-stream constants of the query operand, in shared memory
@@ -565,22 +566,49 @@ struct QConst {   // per-stream constants of the query operand, in shared memory
     float qsum[4][kMaxG];   // sum over group g of head h's (digit-exact) query
 };
 
+
 // ------------------------------------------------------------ the attention kernel
+__device__ __forceinline__ bool wg_any(int id, bool pred) {   // OR of pred over the 128 threads of a warpgroup
+    uint32_t r;
+    asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, %2, 128, p;\n\t"
+                 "selp.u32 %0, 1, 0, q;\n\t}"
+                 : "=r"(r)
+                 : "r"((uint32_t)pred), "r"(id)
+                 : "memory");
+    return r != 0;
+}
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+template <int N>
+__device__ __forceinline__ void tmem_ldn(uint32_t taddr, uint32_t *r) {
+    if constexpr (N >= 16) {
+#pragma unroll
+        for (int i = 0; i < N; i += 16) tmem_ld16(taddr + i, r + i);
+    } else if constexpr (N == 8) {
+        tmem_ld8(taddr, r);
+    } else {
+        static_assert(N == 4, "column count");
+        tmem_ld4(taddr, r);
+    }
+}
+
 template <int G, bool STATS>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_i8_kernel(const __grid_constant__ Dev d, const __nv_bfloat16 *__restrict__ q, float xscale) {
-    constexpr int NG = ng_of(G);
+    attn_i8_kernel(const __grid_constant__ Dev d, const __grid_constant__ I8Maps maps,
+                   const __nv_bfloat16 *__restrict__ q, float xscale) {
+    constexpr int NS = ns_of(G);
     constexpr int NO = no_of(G);
+    constexpr int GS = gs_of(G);
+    constexpr int R = raw_stages(G);
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
-    __shared__ __align__(8) uint64_t bar_raw_full[kRawStages], bar_raw_empty[kRawStages];
-    __shared__ __align__(8) uint64_t bar_stg_full[2], bar_stg_empty[2], bar_meta_full[2], bar_meta_empty[2];
-    __shared__ __align__(8) uint64_t bar_s_full[2], bar_w_full[2], bar_o_full[2];
+    __shared__ __align__(8) uint64_t bar_raw_full[R], bar_raw_empty[R];
+    __shared__ __align__(8) uint64_t bar_kready[2], bar_s_full[2], bar_w_full[2], bar_o_full[2], bar_mma_done;
     __shared__ uint32_t tmem_base;
     __shared__ SharedPlan pl;
-    __shared__ uint32_t xred[2][4][kMaxG];      // tile max keys per softmax warp (double-buffered)
-    __shared__ float fred[4][6 * kMaxG];        // segment flush reductions
-    __shared__ float zsum[4][kMaxG];            // reduced zero-term sums of the segment being flushed
+    __shared__ uint32_t xred[2][2][4][kMaxG + 4];   // [wg][parity][warp]: tile max keys per head, v-scale max keys
+    __shared__ float fred[2][4][6 * kMaxG];         // segment flush reductions
+    __shared__ float zsum[2][4][kMaxG];             // reduced zero-term sums of the segment being flushed
     __shared__ uint32_t err_timeout;
     __shared__ TileDesc desc[kDescRing];
 
@@ -590,26 +618,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- set-up (independent of the append, so before the dependency wait)
     if (warp == 1) tmem_alloc(smem_addr(&tmem_base), kTmemCols);
     if (tid == 0) {
-        for (int i = 0; i < kRawStages; ++i) {
+        for (int i = 0; i < R; ++i) {
             mbar_init_n(smem_addr(&bar_raw_full[i]), 1);
-            mbar_init_n(smem_addr(&bar_raw_empty[i]), 4);
+            mbar_init_n(smem_addr(&bar_raw_empty[i]), 1);
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init_n(smem_addr(&bar_stg_full[i]), 4);
-            mbar_init_n(smem_addr(&bar_stg_empty[i]), 1);
-            mbar_init_n(smem_addr(&bar_meta_full[i]), 4);
-            mbar_init_n(smem_addr(&bar_meta_empty[i]), 4);
+            mbar_init_n(smem_addr(&bar_kready[i]), 4);
             mbar_init_n(smem_addr(&bar_s_full[i]), 1);
             mbar_init_n(smem_addr(&bar_w_full[i]), 4);
             mbar_init_n(smem_addr(&bar_o_full[i]), 1);
         }
+        mbar_init_n(smem_addr(&bar_mma_done), 1);
         err_timeout = 0;
         mbar_init_fence();
     }
-    // query operand buffers: padding rows and columns stay zero
+    if (warp == 0 && lane == 0) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int z = 0; z < 2; ++z) asm volatile("prefetch.tensormap [%0];" ::"l"(&maps.m[i][j][z]) : "memory");
+    }
+    // query operand buffers: the block-diagonal zeros and padding columns stay zero
     for (int i = tid; i < 2 * q_bytes(G) / 16; i += kThreads)
         reinterpret_cast<uint4 *>(sm + off_q(G))[i] = make_uint4(0u, 0u, 0u, 0u);
-    fence_proxy_async_smem();
+    fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -627,233 +661,197 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t pol = policy_evict_first();
             TileIter it;
             it.begin(d, pl);
+            int last_copy[R];
+            bool landed[R];
+#pragma unroll
+            for (int i = 0; i < R; ++i) { last_copy[i] = -1; landed[i] = true; }
             int k = 0;
-            for (;; ++k) {
-                const int slot = k % kRawStages;
-                if (k >= kRawStages && ok)
-                    ok = mbar_wait_sleep(smem_addr(&bar_raw_empty[slot]), (uint32_t)((k / kRawStages - 1) & 1));
-                const uint32_t bar = smem_addr(&bar_raw_full[slot]);
-                if (!it.valid()) {
-                    TileDesc td;
-                    td.s = -1; td.e = 0; td.oc = 0; td.meta = 1u << 31;
-                    desc[k % kDescRing] = td;
-                    mbar_arrive(bar);   // completes the stage's phase without a copy: "no more tiles"
-                    break;
+            for (; ok; ++k) {
+                const int slot = k % R;
+                if (k >= R) {
+                    ok = mbar_wait_sleep(smem_addr(&bar_raw_empty[slot]), (uint32_t)((k / R - 1) & 1));
+                    if (!ok) break;
+                    landed[slot] = true;   // its previous copy was consumed
                 }
+                if (!it.valid()) break;
                 const Tile t = it.tile();
                 TileDesc td;
                 td.s = t.s; td.e = t.e; td.oc = t.oc;
                 td.meta = (uint32_t)t.c | ((uint32_t)t.nr << 2) | ((uint32_t)t.first << 11) | ((uint32_t)t.last << 12);
                 desc[k % kDescRing] = td;
-                const uint32_t bytes = (uint32_t)(t.nr * rec_of(t.c));
-                const uint8_t *src = d.pool[t.c] + ((size_t)t.s * d.cap[t.c] + t.e) * rec_of(t.c);
-                mbar_expect_tx(bar, bytes);
-                bulk_copy(smb + kOffRaw + slot * kRawBytes, src, bytes, bar, pol);
+                const bool full = t.nr == rows_of(t.c);
+                const int nb = full ? 1 : (t.nr + 15) >> 4;                 // 16-row boxes of a tail tile
+                const int rows = full ? rows_of(t.c) : 16 * nb;
+                const uint32_t bar = smem_addr(&bar_raw_full[slot]);
+                mbar_expect_tx(bar, (uint32_t)(rows * rec_of(t.c)));
+                const uint32_t dst = smb + kOffRaw + slot * kRawBytes;
+                const int y0 = t.s * d.cap[t.c] + t.e;
+                const int nbox = t.c == 0 ? 4 : 3;
+                const int cw = code_box_bytes(t.c);
+                for (int bx = 0; bx < nbox; ++bx) {
+                    const bool is_meta = t.c != 0 && bx == 2;
+                    const int wbytes = is_meta ? 32 : cw;
+                    const int x = bx * cw;
+                    const uint32_t bdst = dst + (uint32_t)(bx * rows_of(t.c) * cw);
+                    const CUtensorMap *mp = &maps.m[t.c][is_meta ? 1 : 0][full ? 0 : 1];
+                    for (int j = 0; j < nb; ++j)
+                        tma_load_2d(bdst + (uint32_t)(j * 16 * wbytes), mp, x, y0 + 16 * j, bar, pol);
+                }
+                last_copy[slot] = k;
+                landed[slot] = false;
                 it.advance(d, pl);
             }
-            // every copy this CTA issued (tiles 0 .. k-1) has landed before the CTA may exit;
-            // the stage of tile k ended with the "no more tiles" arrival
-            for (int i = 0; i < kRawStages; ++i) {
-                if (k < 1 || i == k % kRawStages) continue;
-                const int kl = k - 1 - ((k - 1 - i) % kRawStages);   // last tile copied into stage i
-                if (kl < 0) continue;
-                if (!mbar_wait_sleep(smem_addr(&bar_raw_full[i]), (uint32_t)((kl / kRawStages) & 1))) ok = false;
+            // "no more tiles" for the next tile of each warpgroup (slot free: waited above or unused)
+            if (ok) {
+                for (int u = 0; u < 2; ++u) {
+                    const int kk = k + u, slot = kk % R;
+                    if (u == 1 && kk >= R) {
+                        ok = mbar_wait_sleep(smem_addr(&bar_raw_empty[slot]), (uint32_t)((kk / R - 1) & 1));
+                        if (!ok) break;
+                        landed[slot] = true;
+                    }
+                    TileDesc td;
+                    td.s = -1; td.e = 0; td.oc = 0; td.meta = 1u << 31;
+                    desc[kk % kDescRing] = td;
+                    mbar_arrive(smem_addr(&bar_raw_full[slot]));
+                }
+            }
+            // every copy still unconsumed lands before the CTA may exit (each slot holds at most one)
+            for (int i = 0; i < R; ++i) {
+                if (landed[i] || last_copy[i] < 0) continue;
+                if (!mbar_wait_sleep(smem_addr(&bar_raw_full[i]), (uint32_t)((last_copy[i] / R) & 1))) ok = false;
             }
         }
     } else if (warp == 1) {
         // ================================================= MMA issuer
         if (lane == 0) {
-            int k = 0, prev_c = -1, seg = -1, prev_s = -1;
-            auto issue_pv = [&](int kp, int cp) {
-                const int b = kp & 1;
-                if (ok) ok = mbar_wait_sleep(smem_addr(&bar_w_full[b]), (uint32_t)((kp >> 1) & 1));
+            int k = 0;
+            TileDesc prev;
+            prev.meta = 0;
+            auto issue_pv = [&](int kp, const TileDesc &tp) {
+                const int wg = kp & 1, cp = td_c(tp);
+                ok = mbar_wait_sleep(smem_addr(&bar_w_full[wg]), (uint32_t)((kp >> 1) & 1));
+                if (!ok) return;
                 tc_fence_after();
-                const uint32_t av = smb + kOffStg + b * kStgBytes + kStgV;
-                const uint32_t bw = smb + kOffW + b * w_bytes(G);
+                const uint32_t raw = smb + kOffRaw + (kp % R) * kRawBytes;
+                const uint32_t stg = smb + off_stg(G) + wg * kStgV;
+                const uint32_t bw = smb + off_w(G) + wg * w_bytes(G);
+                const uint32_t dcol = tb + col_o(wg);
                 if (cp == 0) {
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
-                        mma_f16(tb + col_o(b), sdesc(av + ks * 256, 128, 1024), sdesc(bw + ks * 256, 128, 1024),
+                        mma_f16(dcol, sdesc(stg + ks * 2048, 8192, 1024, kSw128), sdesc(bw + ks * 256, 128, 1024),
                                 idesc(1, 1, 1, 1, 1, 16), ks > 0);
                 } else {
+                    const uint32_t av = cp == 1 ? raw + v_off(1) : stg;
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
-                        mma_i8(tb + col_o(b), sdesc(av + ks * 512, 128, 2048), sdesc(bw + ks * 512, 128, 2048),
+                        mma_i8(dcol, sdesc(av + ks * 4096, 16, 1024, kSw128), sdesc(bw + ks * 512, 128, 2048),
                                idesc(2, 0, 0, 1, 1, NO), ks > 0);
                 }
-                mma_commit(smem_addr(&bar_o_full[b]));
-                mma_commit(smem_addr(&bar_stg_empty[b]));
+                mma_commit(smem_addr(&bar_o_full[wg]));
+                mma_commit(smem_addr(&bar_raw_empty[kp % R]));
             };
-            for (;; ++k) {
-                const int b = k & 1;
-                if (ok) ok = mbar_wait_sleep(smem_addr(&bar_stg_full[b]), (uint32_t)((k >> 1) & 1));
+            for (; ok; ++k) {
+                const int wg = k & 1;
+                ok = mbar_wait_sleep(smem_addr(&bar_kready[wg]), (uint32_t)((k >> 1) & 1));
+                if (!ok) break;
                 const TileDesc td = desc[k % kDescRing];
                 if (td_end(td)) break;
-                const int tc = td_c(td);
-                if (td.s != prev_s) { ++seg; prev_s = td.s; }
                 tc_fence_after();
-                const uint32_t ak = smb + kOffStg + b * kStgBytes;
-                const uint32_t qb = smb + off_q(G) + (seg & 1) * q_bytes(G);
+                const int tc = td_c(td);
+                const uint32_t raw = smb + kOffRaw + (k % R) * kRawBytes;
+                const uint32_t qb = smb + off_q(G) + wg * q_bytes(G);
+                const uint32_t dcol = tb + col_s(wg);
                 if (tc == 0) {
                     const uint32_t bq = qb + qi8_bytes(G);
 #pragma unroll
                     for (int ks = 0; ks < 8; ++ks)
-                        mma_f16(tb + col_s(b), sdesc(ak + ks * 2048, 1024, 128), sdesc(bq + ks * 512, 256, 128),
-                                idesc(1, 1, 1, 0, 0, 16), ks > 0);
+                        mma_f16(dcol, sdesc(raw + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kSw128),
+                                sdesc(bq + ks * 512, 256, 128), idesc(1, 1, 1, 0, 0, 16), ks > 0);
+                } else if (tc == 1) {
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_i8(dcol, sdesc(raw + ks * 32, 16, 1024, kSw128), sdesc(qb + ks * 32 * NS, NS * 16, 128),
+                               idesc(2, 0, 1, 0, 0, NS), ks > 0);
                 } else {
 #pragma unroll
-                    for (int g = 0; g < 4; ++g)
-                        mma_i8(tb + col_s(b) + g * NG, sdesc(ak + 2 * g * 2048, 2048, 128),
-                               sdesc(qb + g * 32 * NG, NG * 16, 128), idesc(2, 0, 1, 0, 0, NG), 0u);
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_i8_tmem(dcol, tb + col_a(wg) + 8 * ks, sdesc(qb + ks * 32 * NS, NS * 16, 128),
+                                    idesc(2, 0, 1, 0, 0, NS), ks > 0);
                 }
-                mma_commit(smem_addr(&bar_s_full[b]));
-                if (k > 0) issue_pv(k - 1, prev_c);
-                prev_c = tc;
+                mma_commit(smem_addr(&bar_s_full[wg]));
+                if (k > 0) issue_pv(k - 1, prev);
+                prev = td;
             }
-            if (k > 0) issue_pv(k - 1, prev_c);
-        }
-    } else if (warp < 6) {
-        // ================================================= stager
-        const int r = tid - 64;            // row of the tile, also head dim for the query operand
-        const int sw = warp - 2;           // stager warp = query group it builds
-        int k = 0, seg = -1, prev_s = -1;
-        for (;; ++k) {
-            const int b = k & 1, slot = k % kRawStages;
-            if (k >= 2) {
-                if (ok) ok = mbar_wait_sleep(smem_addr(&bar_stg_empty[b]), (uint32_t)(((k - 2) >> 1) & 1));
-                if (ok) ok = mbar_wait_sleep(smem_addr(&bar_meta_empty[b]), (uint32_t)(((k - 2) >> 1) & 1));
-            }
-            if (ok) ok = mbar_wait_sleep(smem_addr(&bar_raw_full[slot]), (uint32_t)((k / kRawStages) & 1));
-            const TileDesc td = desc[k % kDescRing];
-            if (td_end(td)) {
-                // pass "no more tiles" on to the MMA issuer and the softmax warps
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(smem_addr(&bar_stg_full[b]));
-                    mbar_arrive(smem_addr(&bar_meta_full[b]));
-                }
-                break;
-            }
-            Tile t;
-            t.s = td.s; t.c = td_c(td); t.e = td.e; t.nr = td_nr(td); t.oc = td.oc;
-            t.first = td_first(td); t.last = td_last(td);
-            if (t.s != prev_s) {
-                // ---- query operands of stream t.s: thread r takes head dim r
-                ++seg;
-                prev_s = t.s;
-                uint8_t *qbuf = sm + off_q(G) + (seg & 1) * q_bytes(G);
-                QConst<G> *qc = reinterpret_cast<QConst<G> *>(qbuf + qi8_bytes(G) + kQbfBytes);
-                const int bb = t.s / d.Hkv, kvh = t.s - bb * d.Hkv;
-                const uint16_t *qrow =
-                    reinterpret_cast<const uint16_t *>(q) + ((size_t)bb * d.Hkv * G + (size_t)kvh * G) * kD;
-                const int g = sw, kk = r & 31;
-#pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    const uint32_t bits = qrow[h * kD + r];
-                    // bf16 operand: element (n = h, k = r), K-major
-                    *reinterpret_cast<uint16_t *>(qbuf + qi8_bytes(G) + (r / 8) * 256 + (h / 8) * 128 + (h % 8) * 16 +
-                                                  (r % 8) * 2) = (uint16_t)bits;
-                    // digits: q = v * 2^(Emax - 146) with v = m * 2^(e - Emax + 12) (rounded)
-                    const int ex = (int)((bits >> 7) & 0xff);
-                    const int m = ex == 0 ? (int)(bits & 0x7f) : (int)((bits & 0x7f) | 0x80);
-                    const int e_eff = ex == 0 ? 1 : ex;
-                    const int emax = (int)__reduce_max_sync(kFull, (unsigned)e_eff);
-                    const int sh = e_eff - emax + 12;
-                    int v;
-                    if (sh >= 0) v = m << sh;
-                    else if (sh > -9) v = (m + (1 << (-sh - 1))) >> (-sh);
-                    else v = 0;
-                    if (bits & 0x8000) v = -v;
-                    const int d2 = ((v + 64) & 127) - 64;
-                    const int v1 = (v - d2) >> 7;
-                    const int d1 = ((v1 + 64) & 127) - 64;
-                    const int d0 = (v1 - d1) >> 7;
-                    uint8_t *gb = qbuf + g * 32 * NG;
-                    const int n0 = 0 * G + h, n1 = 1 * G + h, n2 = 2 * G + h;
-                    const int ko = (kk / 16) * (NG * 16) + kk % 16;
-                    gb[ko + (n0 / 8) * 128 + (n0 % 8) * 16] = (uint8_t)(int8_t)d0;
-                    gb[ko + (n1 / 8) * 128 + (n1 % 8) * 16] = (uint8_t)(int8_t)d1;
-                    gb[ko + (n2 / 8) * 128 + (n2 % 8) * 16] = (uint8_t)(int8_t)d2;
-                    const int vsum = __reduce_add_sync(kFull, v);
-                    if (lane == 0) {
-                        const int ea = emax - 146;
-                        const float a = ea >= -126 ? pow2f(ea) : pow2f(ea + 64) * 5.421010862427522e-20f;   // 2^-64
-                        qc->a[g][h] = a;
-                        qc->qsum[g][h] = (float)vsum * a;
-                    }
-                }
-            }
-            // ---- the tile
-            const uint8_t *raw = sm + kOffRaw + slot * kRawBytes;
-            uint8_t *stg = sm + kOffStg + b * kStgBytes;
-            uint8_t *meta = sm + kOffMeta + b * kMetaBytes;
-            const int R = rec_of(t.c);
-            if (t.c == 0) {
-                // 64 rows: threads 0..63 take K, 64..127 take V of row r % 64
-                const int rr = r & 63;
-                const bool is_v = r >= 64;
-                uint8_t *dst = stg + (is_v ? kStgV : 0) + (rr / 8) * 128 + (rr % 8) * 16;
-                if (rr < t.nr) stage_row_bf16(raw + rr * R, dst, is_v, rr);
-                else zero_row(dst, 16, 1024);
-            } else {
-                uint8_t *kd = stg + (r / 8) * 128 + (r % 8) * 16;
-                uint8_t *vd = kd + kStgV;
-                uint32_t vkey[4] = {0u, 0u, 0u, 0u};
-                if (r < t.nr) {
-                    const uint8_t *rec = raw + r * R;
-                    if (t.c == 1) stage_row_i8(rec, kd, vd);
-                    else if (t.c == 2) stage_row_i4(rec, kd, vd);
-                    else stage_row_i2(rec, kd, vd);
-                    const int cb = R == 288 ? 128 : R == 160 ? 64 : 32;
-                    const uint4 km = *reinterpret_cast<const uint4 *>(rec + 2 * cb);
-                    const uint4 vm = *reinterpret_cast<const uint4 *>(rec + 2 * cb + 16);
-                    *reinterpret_cast<uint4 *>(meta + r * 32) = km;
-                    *reinterpret_cast<uint4 *>(meta + r * 32 + 16) = vm;
-                    // v scales are >= 0: their fp16 bits order as integers
-                    vkey[0] = vm.x & 0xffffu; vkey[1] = vm.x >> 16; vkey[2] = vm.y & 0xffffu; vkey[3] = vm.y >> 16;
-                } else {
-                    zero_row(kd, 8, 2048);
-                    zero_row(vd, 8, 2048);
-                    *reinterpret_cast<uint4 *>(meta + r * 32) = make_uint4(0u, 0u, 0u, 0u);
-                    *reinterpret_cast<uint4 *>(meta + r * 32 + 16) = make_uint4(0u, 0u, 0u, 0u);
-                }
-#pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    const uint32_t mx = __reduce_max_sync(kFull, vkey[g]);
-                    if (lane == 0) reinterpret_cast<uint32_t *>(meta + kMetaHdr)[sw * 4 + g] = mx;
-                }
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(smem_addr(&bar_stg_full[b]));
-                mbar_arrive(smem_addr(&bar_meta_full[b]));
-                mbar_arrive(smem_addr(&bar_raw_empty[slot]));
-            }
+            if (ok && k > 0) issue_pv(k - 1, prev);
+            // every MMA issued has completed before tensor memory is released
+            mma_commit(smem_addr(&bar_mma_done));
+            if (!mbar_wait_sleep(smem_addr(&bar_mma_done), 0u)) ok = false;
         }
     } else {
-        // ================================================= softmax / epilogue
-        const int wq = warp & 3;                 // lane quarter of tensor memory
-        const int r = 32 * wq + lane;            // token row (QK) and head dim (PV)
-        const int gr = r >> 5;                   // group of head dim r
+        // ================================================= compute warpgroups (warps 2-5, 6-9)
+        const int wg = (warp - 2) >> 2;
+        const int wq = warp & 3;                         // lane quarter of tensor memory
+        const int r = 32 * wq + lane;                    // token row (QK), element m of the V order (PV), dim (q)
+        const int gr = (r & 31) >> 3;                    // group of the head dim at V position r
+        const int bid = 1 + wg;                          // named barrier of the warpgroup
         const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
+        uint8_t *qbuf = sm + off_q(G) + wg * q_bytes(G);
+        QConst<G> *qc = reinterpret_cast<QConst<G> *>(qbuf + qi8_bytes(G) + kQbfBytes);
+        uint8_t *stg = sm + off_stg(G) + wg * kStgV;
+        uint8_t *wbuf = sm + off_w(G) + wg * w_bytes(G);
         float m[G], l[G], e[G], z[4][G], oacc[G];
         float alpha_prev[G], bp_prev[G], bv_prev = 1.f;
-        int c_prev = 0;
 #pragma unroll
         for (int h = 0; h < G; ++h) {
             m[h] = kNoMax; l[h] = 0.f; e[h] = 0.f; oacc[h] = 0.f; alpha_prev[h] = 1.f; bp_prev[h] = 1.f;
 #pragma unroll
             for (int g = 0; g < 4; ++g) z[g][h] = 0.f;
         }
-        int k = 0, seg = -1, prev_s = -1;
-        Tile tp;                                 // previous tile
-        tp.s = -1; tp.first = false; tp.last = false;
-        int seg_first_cta_tile = 0;              // the current segment began with the stream's first tile
+        int cur_s = -1, c_prev = 0, kp = -1;
+        bool cta_empty = false;
+        // an empty partial (l = 0: the merge skips it) in this warpgroup's slot of stream s
+        auto write_empty = [&](int s) {
+            float *part = d.part + (size_t)(2 * (s + cta) + wg) * part_floats(G);
+            part[r] = kNoMax;
+            part[G + r] = 0.f;
+            part[2 * G + r] = 0.f;
+        };
 
-        // reduce the per-thread partial sums of the softmax warps; thread 0..: write the
-        // segment's (m, l, e) and keep the zero-term sums in shared memory
-        auto flush_softmax_side = [&](int s_old, bool first_flag) {
+        // add the PV result of own tile kp (class cp) to O
+        auto o_accumulate = [&](int kpp, int cp) {
+            if (ok) ok = mbar_wait_sleep(smem_addr(&bar_o_full[wg]), (uint32_t)((kpp >> 1) & 1));
+            tc_fence_after();
+            if (cp == 0) {
+                uint32_t dv[16];
+                tmem_ld16(tb + lane_off + col_o(wg), dv);
+                tc_wait_ld();
+#pragma unroll
+                for (int h = 0; h < G; ++h)
+                    oacc[h] = fmaf(oacc[h], alpha_prev[h], __uint_as_float(dv[h]) + __uint_as_float(dv[G + h]));
+            } else {
+                uint32_t sel[4 * G];
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    uint32_t dv[4 * G];
+                    tmem_ldn<4 * G>(tb + lane_off + col_o(wg) + g * GS, dv);
+                    tc_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 4 * G; ++i) sel[i] = g == gr ? dv[i] : (g == 0 ? 0u : sel[i]);
+                }
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    const float v = fmaf(__int2float_rn((int32_t)sel[4 * h + 2]), 65536.f,
+                                         fmaf(__int2float_rn((int32_t)sel[4 * h + 1]), 256.f,
+                                              __int2float_rn((int32_t)sel[4 * h])));
+                    oacc[h] = fmaf(oacc[h], alpha_prev[h], v * bp_prev[h] * bv_prev);
+                }
+            }
+            tc_fence_before();
+        };
+        // write the partial of segment s_old: (m, l, e) per head and O + zero term
+        auto flush = [&](int s_old) {
 #pragma unroll
             for (int h = 0; h < G; ++h) {
                 float vl = l[h], ve = e[h];
@@ -862,79 +860,126 @@ __global__ void __launch_bounds__(kThreads, 1)
                     vl += __shfl_xor_sync(kFull, vl, o);
                     if (STATS) ve += __shfl_xor_sync(kFull, ve, o);
                 }
-                if (lane == 0) { fred[wq][h] = vl; fred[wq][G + h] = ve; }
+                if (lane == 0) { fred[wg][wq][h] = vl; fred[wg][wq][G + h] = ve; }
 #pragma unroll
                 for (int g = 0; g < 4; ++g) {
                     float vz = z[g][h];
 #pragma unroll
                     for (int o = 16; o > 0; o >>= 1) vz += __shfl_xor_sync(kFull, vz, o);
-                    if (lane == 0) fred[wq][2 * G + g * G + h] = vz;
+                    if (lane == 0) fred[wg][wq][2 * G + g * G + h] = vz;
                 }
             }
-            named_sync(1, 128);
-            float *part = d.part + (size_t)(s_old + cta) * part_floats(G);
+            named_sync(bid, 128);
+            float *part = d.part + (size_t)(2 * (s_old + cta) + wg) * part_floats(G);
             if (r < 6 * G) {
-                const float v = fred[0][r] + fred[1][r] + fred[2][r] + fred[3][r];
-                if (r < G) part[G + r] = v;                        // l
-                else if (r < 2 * G) part[2 * G + (r - G)] = v;     // e
-                else zsum[(r - 2 * G) / G][(r - 2 * G) % G] = v;   // zero term
+                const float v = fred[wg][0][r] + fred[wg][1][r] + fred[wg][2][r] + fred[wg][3][r];
+                if (r < G) part[G + r] = v;                                 // l
+                else if (r < 2 * G) part[2 * G + (r - G)] = v;              // e
+                else zsum[wg][(r - 2 * G) / G][(r - 2 * G) % G] = v;        // zero term
             }
             if (r == 0) {
 #pragma unroll
                 for (int h = 0; h < G; ++h) part[h] = m[h];
-                if (first_flag) d.seg_lo[s_old] = cta;
             }
-            named_sync(1, 128);
-        };
-        auto flush_o_side = [&](int s_old, bool last_flag) {
-            float *part = d.part + (size_t)(s_old + cta) * part_floats(G);
+            named_sync(bid, 128);
+            const int dim = dim_of_v8(r);
 #pragma unroll
-            for (int h = 0; h < G; ++h) part[3 * G + h * kD + r] = oacc[h] + zsum[gr][h];
-            if (r == 0 && last_flag) d.seg_hi[s_old] = cta;
-        };
-        // add the PV result of own tile kp (class cp) to O
-        auto o_accumulate = [&](int kp, int cp) {
-            const int b = kp & 1;
-            if (ok) ok = mbar_wait_sleep(smem_addr(&bar_o_full[b]), (uint32_t)((kp >> 1) & 1));
-            tc_fence_after();
-            if (cp == 0) {
-                uint32_t dv[16];
-                tmem_ld16(tb + lane_off + col_o(b), dv);
-                tc_wait_ld();
-#pragma unroll
-                for (int h = 0; h < G; ++h)
-                    oacc[h] = fmaf(oacc[h], alpha_prev[h], __uint_as_float(dv[h]) + __uint_as_float(dv[G + h]));
-            } else {
-                uint32_t dv[gs_of(G)];
-#pragma unroll
-                for (int i = 0; i < gs_of(G); i += 16) tmem_ld16(tb + lane_off + col_o(b) + gr * gs_of(G) + i, dv + i);
-                tc_wait_ld();
-#pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    const float v = fmaf(i2f_exact((int32_t)dv[4 * h + 2]), 65536.f,
-                                         fmaf(i2f_exact((int32_t)dv[4 * h + 1]), 256.f,
-                                              i2f_exact((int32_t)dv[4 * h])));
-                    oacc[h] = fmaf(oacc[h], alpha_prev[h], v * bp_prev[h] * bv_prev);
-                }
-            }
-            tc_fence_before();
+            for (int h = 0; h < G; ++h) part[3 * G + h * kD + dim] = oacc[h] + zsum[wg][gr][h];
         };
 
-        float *lgs_base = d.logits;
-        for (;; ++k) {
-            const int b = k & 1;
-            if (ok) ok = mbar_wait_sleep(smem_addr(&bar_meta_full[b]), (uint32_t)((k >> 1) & 1));
+        for (int k = wg;; k += 2) {
+            const int slot = k % R;
+            if (ok) ok = mbar_wait_sleep(smem_addr(&bar_raw_full[slot]), (uint32_t)((k / R) & 1));
             const TileDesc td = desc[k % kDescRing];
-            if (td_end(td)) break;
-            Tile t;
-            t.s = td.s; t.c = td_c(td); t.e = td.e; t.nr = td_nr(td); t.oc = td.oc;
-            t.first = td_first(td); t.last = td_last(td);
-            const bool newseg = t.s != prev_s;
-            if (newseg && k > 0) flush_softmax_side(prev_s, seg_first_cta_tile != 0);
+            const bool end = td_end(td);
+            if (k == wg) cta_empty = end && (wg == 0 || td_end(desc[0]));
+            // a stream whose tiles in this CTA all went to the other warpgroup (the tile
+            // between this warpgroup's previous tile and this one) gets an empty partial
+            if (ok && k >= 1 && r < G) {
+                const TileDesc to = desc[(k - 1) % kDescRing];
+                if (!td_end(to) && to.s != cur_s && (end || to.s != td.s)) write_empty(to.s);
+            }
+            if (wg_any(bid, end || !ok)) {
+                if (end && ok) {   // let the MMA issuer see the end
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_addr(&bar_kready[wg]));
+                }
+                break;
+            }
+            const int tcls = td_c(td), nr = td_nr(td);
+            const uint8_t *raw = sm + kOffRaw + slot * kRawBytes;
+            const bool newseg = td.s != cur_s;
             if (newseg) {
-                ++seg;
-                prev_s = t.s;
-                seg_first_cta_tile = t.first ? 1 : 0;
+                // ---- query operands of stream td.s: thread r takes head dim r (group wq)
+                const int bb = td.s / d.Hkv, kvh = td.s - bb * d.Hkv;
+                const uint16_t *qrow =
+                    reinterpret_cast<const uint16_t *>(q) + ((size_t)bb * d.Hkv * G + (size_t)kvh * G) * kD;
+                const int kb = pos_kbf(r), m8 = pos_k8(r);
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    const uint32_t bits = qrow[h * kD + r];
+                    *reinterpret_cast<uint16_t *>(qbuf + qi8_bytes(G) + (kb / 8) * 256 + (h / 8) * 128 + (h % 8) * 16 +
+                                                  (kb % 8) * 2) = (uint16_t)bits;
+                    // digits: q = v * 2^(Emax - 146) with v = m * 2^(e - Emax + 12) (rounded)
+                    const int ex = (int)((bits >> 7) & 0xff);
+                    const int mant = ex == 0 ? (int)(bits & 0x7f) : (int)((bits & 0x7f) | 0x80);
+                    const int e_eff = ex == 0 ? 1 : ex;
+                    const int emax = (int)__reduce_max_sync(kFull, (unsigned)e_eff);
+                    const int sh = e_eff - emax + 12;
+                    int v;
+                    if (sh >= 0) v = mant << sh;
+                    else if (sh > -9) v = (mant + (1 << (-sh - 1))) >> (-sh);
+                    else v = 0;
+                    if (bits & 0x8000) v = -v;
+                    const int d2 = ((v + 64) & 127) - 64;
+                    const int v1 = (v - d2) >> 7;
+                    const int d1 = ((v1 + 64) & 127) - 64;
+                    const int d0 = (v1 - d1) >> 7;
+                    const int dg[3] = {d0, d1, d2};
+#pragma unroll
+                    for (int s3 = 0; s3 < 3; ++s3) {
+                        const int n = wq * 3 * G + s3 * G + h;
+                        qbuf[(m8 / 16) * (NS * 16) + (n / 8) * 128 + (n % 8) * 16 + (m8 % 16)] = (uint8_t)(int8_t)dg[s3];
+                    }
+                    const int vsum = __reduce_add_sync(kFull, v);
+                    if (lane == 0) {
+                        const int ea = emax - 146;
+                        const float a = ea >= -126 ? pow2f(ea) : pow2f(ea + 64) * 5.421010862427522e-20f;   // 2^-64
+                        qc->a[wq][h] = a;
+                        qc->qsum[wq][h] = (float)vsum * a;
+                    }
+                }
+            }
+            // ---- keys of int4 / int2 tiles: widened into tensor memory (row r = token r)
+            if (tcls >= 2) {
+                uint32_t o[32];
+                if (tcls == 2) widen_i4(raw, r, o);
+                else widen_i2(raw, r, o);
+                tmem_st16(tb + lane_off + col_a(wg), o);
+                tmem_st16(tb + lane_off + col_a(wg) + 16, o + 16);
+                tc_wait_st();
+            }
+            fence_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&bar_kready[wg]));
+            if (r == 0) {
+                if (td_first(td)) d.seg_lo[td.s] = cta;
+                if (td_last(td)) d.seg_hi[td.s] = cta;
+            }
+
+            // ---- O of the previous own tile; the segment's partial when the stream changes
+            if (kp >= 0) {
+                o_accumulate(kp, c_prev);
+                if (newseg) {
+                    flush(cur_s);
+#pragma unroll
+                    for (int h = 0; h < G; ++h) oacc[h] = 0.f;
+                }
+            }
+            if (newseg) {
+                cur_s = td.s;
 #pragma unroll
                 for (int h = 0; h < G; ++h) {
                     m[h] = kNoMax; l[h] = 0.f; e[h] = 0.f;
@@ -942,67 +987,104 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int g = 0; g < 4; ++g) z[g][h] = 0.f;
                 }
             }
-            const QConst<G> *qc =
-                reinterpret_cast<const QConst<G> *>(sm + off_q(G) + (seg & 1) * q_bytes(G) + qi8_bytes(G) + kQbfBytes);
-            if (ok) ok = mbar_wait_sleep(smem_addr(&bar_s_full[b]), (uint32_t)((k >> 1) & 1));
+
+            // ---- values of int4 / int2 / bf16 tiles: widened / regathered into the staged buffer
+            if (tcls >= 2) {
+                uint32_t o[32];
+                if (tcls == 2) widen_i4(raw + v_off(2), r, o);
+                else widen_i2(raw + v_off(3), r, o);
+                store_row_sw128(stg, r, o);
+            } else if (tcls == 0) {
+                const int t = r & 63, a = r >> 6;
+                if (t < nr) {
+                    regather_bf16_v(raw + 16384, stg, t, a);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) st_sw128(stg + a * 8192, t, j, 0u, 0u, 0u, 0u);
+                }
+            }
+
+            // ---- logits
+            if (ok) ok = mbar_wait_sleep(smem_addr(&bar_s_full[wg]), (uint32_t)((k >> 1) & 1));
             tc_fence_after();
-            const bool valid = r < t.nr;
+            const bool valid = r < nr;
             float x[G];
             float vsc[4] = {0.f, 0.f, 0.f, 0.f}, vze[4] = {0.f, 0.f, 0.f, 0.f};
-            if (t.c == 0) {
+            uint32_t vkey[4] = {0u, 0u, 0u, 0u};
+            if (tcls == 0) {
                 uint32_t sv[16];
-                tmem_ld16(tb + lane_off + col_s(b), sv);
+                tmem_ld16(tb + lane_off + col_s(wg), sv);
                 tc_wait_ld();
 #pragma unroll
                 for (int h = 0; h < G; ++h) x[h] = valid ? __uint_as_float(sv[h]) * xscale : -INFINITY;
             } else {
-                const uint8_t *meta = sm + kOffMeta + b * kMetaBytes;
-                const uint4 km = *reinterpret_cast<const uint4 *>(meta + r * 32);
-                const uint4 vm = *reinterpret_cast<const uint4 *>(meta + r * 32 + 16);
+                const uint8_t *meta = raw + meta_off(tcls) + 32 * r;
+                const uint4 km = *reinterpret_cast<const uint4 *>(meta);
+                const uint4 vm = *reinterpret_cast<const uint4 *>(meta + 16);
                 const float2 ks01 = __half22float2(u32_as_h2(km.x)), ks23 = __half22float2(u32_as_h2(km.y));
                 const float2 kz01 = __half22float2(u32_as_h2(km.z)), kz23 = __half22float2(u32_as_h2(km.w));
                 const float2 vs01 = __half22float2(u32_as_h2(vm.x)), vs23 = __half22float2(u32_as_h2(vm.y));
                 const float2 vz01 = __half22float2(u32_as_h2(vm.z)), vz23 = __half22float2(u32_as_h2(vm.w));
                 const float ks[4] = {ks01.x, ks01.y, ks23.x, ks23.y}, kz[4] = {kz01.x, kz01.y, kz23.x, kz23.y};
-                vsc[0] = vs01.x; vsc[1] = vs01.y; vsc[2] = vs23.x; vsc[3] = vs23.y;
-                vze[0] = vz01.x; vze[1] = vz01.y; vze[2] = vz23.x; vze[3] = vz23.y;
+                if (valid) {
+                    vsc[0] = vs01.x; vsc[1] = vs01.y; vsc[2] = vs23.x; vsc[3] = vs23.y;
+                    vze[0] = vz01.x; vze[1] = vz01.y; vze[2] = vz23.x; vze[3] = vz23.y;
+                    // v scales are >= 0: their fp16 bits order as integers
+                    vkey[0] = vm.x & 0xffffu; vkey[1] = vm.x >> 16; vkey[2] = vm.y & 0xffffu; vkey[3] = vm.y >> 16;
+                }
 #pragma unroll
                 for (int h = 0; h < G; ++h) x[h] = 0.f;
+                constexpr int GPL = G == 8 ? 2 : 4;                       // groups per accumulator load
+                constexpr int NL = (GPL * 3 * G + 15) / 16 * 16;
 #pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    uint32_t sv[NG];
-#pragma unroll
-                    for (int i = 0; i < NG; i += 16) tmem_ld16(tb + lane_off + col_s(b) + g * NG + i, sv + i);
+                for (int g0 = 0; g0 < 4; g0 += GPL) {
+                    uint32_t sv[NL];
+                    tmem_ldn<NL>(tb + lane_off + col_s(wg) + g0 * 3 * G, sv);
                     tc_wait_ld();
 #pragma unroll
-                    for (int h = 0; h < G; ++h) {
-                        const float tsum = fmaf(i2f_exact((int32_t)sv[h]), 16384.f,
-                                                fmaf(i2f_exact((int32_t)sv[G + h]), 128.f,
-                                                     i2f_exact((int32_t)sv[2 * G + h])));
-                        x[h] = fmaf(ks[g] * qc->a[g][h], tsum, fmaf(kz[g], qc->qsum[g][h], x[h]));
+                    for (int gi = 0; gi < GPL; ++gi) {
+                        const int g = g0 + gi;
+#pragma unroll
+                        for (int h = 0; h < G; ++h) {
+                            const float tsum = fmaf(__int2float_rn((int32_t)sv[gi * 3 * G + h]), 16384.f,
+                                                    fmaf(__int2float_rn((int32_t)sv[gi * 3 * G + G + h]), 128.f,
+                                                         __int2float_rn((int32_t)sv[gi * 3 * G + 2 * G + h])));
+                            x[h] = fmaf(ks[g] * qc->a[g][h], tsum, fmaf(kz[g], qc->qsum[g][h], x[h]));
+                        }
                     }
                 }
 #pragma unroll
                 for (int h = 0; h < G; ++h) x[h] = valid ? x[h] * xscale : -INFINITY;
             }
+            tc_fence_before();
             // raw logits for the score pass (entry order of the stream)
             if (valid) {
-                float *lg = lgs_base + ((size_t)t.s * d.ncap + t.oc + t.e + r) * G;
+                float *lg = d.logits + ((size_t)td.s * d.ncap + td.oc + td.e + r) * G;
+                if constexpr (G == 4) {
+                    *reinterpret_cast<float4 *>(lg) = make_float4(x[0], x[1], x[2], x[3]);
+                } else {
 #pragma unroll
-                for (int h = 0; h < G; ++h) lg[h] = x[h];
+                    for (int h = 0; h < G; ++h) lg[h] = x[h];
+                }
             }
-            // tile max per head (and the stager's v-scale maxima) across the softmax warps
-            const int par = k & 1;
+            // tile max per head and v-scale max per group across the warpgroup
+            const int par = (k >> 1) & 1;
 #pragma unroll
             for (int h = 0; h < G; ++h) {
                 const uint32_t mk = __reduce_max_sync(kFull, fkey(x[h]));
-                if (lane == 0) xred[par][wq][h] = mk;
+                if (lane == 0) xred[wg][par][wq][h] = mk;
             }
-            named_sync(1, 128);
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                const uint32_t mx = __reduce_max_sync(kFull, vkey[g]);
+                if (lane == 0) xred[wg][par][wq][kMaxG + g] = mx;
+            }
+            named_sync(bid, 128);
             float alpha[G], tmax[G];
 #pragma unroll
             for (int h = 0; h < G; ++h) {
-                const uint32_t mk = max(max(xred[par][0][h], xred[par][1][h]), max(xred[par][2][h], xred[par][3][h]));
+                const uint32_t mk = max(max(xred[wg][par][0][h], xred[wg][par][1][h]),
+                                        max(xred[wg][par][2][h], xred[wg][par][3][h]));
                 tmax[h] = fkey_inv(mk);
                 alpha[h] = 1.f;
                 if (tmax[h] > m[h] + kRescaleSlack) {
@@ -1022,9 +1104,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (STATS) e[h] = fmaf(p[h], valid ? x[h] - m[h] : 0.f, e[h]);
             }
             // ---- W (the B operand of PV) for row r
-            uint8_t *wbuf = sm + kOffW + b * w_bytes(G);
             float bp_cur[G], bv_cur = 1.f;
-            if (t.c == 0) {
+            if (tcls == 0) {
                 if (r < 64) {
                     uint32_t pw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};   // 16 bf16 columns: hi then lo
 #pragma unroll
@@ -1043,12 +1124,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int h = 0; h < G; ++h) bp_cur[h] = 1.f;
             } else {
-                const uint32_t *hdr = reinterpret_cast<const uint32_t *>(sm + kOffMeta + b * kMetaBytes + kMetaHdr);
                 float iv[4], ip[G];
                 int ev[4], ep[G];
 #pragma unroll
                 for (int g = 0; g < 4; ++g) {
-                    const uint32_t vk = max(max(hdr[0 * 4 + g], hdr[1 * 4 + g]), max(hdr[2 * 4 + g], hdr[3 * 4 + g]));
+                    const uint32_t vk = max(max(xred[wg][par][0][kMaxG + g], xred[wg][par][1][kMaxG + g]),
+                                            max(xred[wg][par][2][kMaxG + g], xred[wg][par][3][kMaxG + g]));
                     const float vmax = __half2float(__ushort_as_half((unsigned short)vk));
                     if (vmax > 0.f) {
                         iv[g] = inv_pow2_ceil(vmax, ev[g]) * 4194304.f;   // 2^(22 - ceil log2 vmax)
@@ -1066,23 +1147,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     bp_cur[h] = pow2f(ep[h]);
                 }
-                bv_cur = pow2f(ev[gr] - 22);
+                const int evr = gr == 0 ? ev[0] : gr == 1 ? ev[1] : gr == 2 ? ev[2] : ev[3];
+                bv_cur = pow2f(evr - 22);
                 uint32_t wv[4 * G];
 #pragma unroll
                 for (int g = 0; g < 4; ++g) {
                     const float vv = vsc[g] * iv[g];
 #pragma unroll
                     for (int h = 0; h < G; ++h) {
-                        const float pv = p[h] * ip[h];
-                        const float wf = pv * vv;   // in [0, 2^22)
+                        const float wf = (p[h] * ip[h]) * vv;   // in [0, 2^22)
                         wv[g * G + h] = __float_as_uint(wf + 12582912.f) - 0x4B400000u;
                         z[g][h] = fmaf(p[h], vze[g], z[g][h]);
                     }
                 }
-                // row r: group g's columns start at g * gs_of(G); column 4h + byte of a group is
-                // byte `byte` of wv[g*G + h]; 16-column chunks 2048 B apart
+                // row r: group g's columns start at g * GS; column 4h + byte of a group is byte
+                // `byte` of wv[g*G + h]; 16-column chunks 2048 B apart
                 uint8_t *dst = wbuf + (r / 8) * 128 + (r % 8) * 16;
-                constexpr int CPG = gs_of(G) / 16;   // chunks per group
+                constexpr int CPG = GS / 16;   // chunks per group
 #pragma unroll
                 for (int g = 0; g < 4; ++g)
 #pragma unroll
@@ -1093,36 +1174,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                         sts128(dst + (g * CPG + i) * 2048, a4[0], a4[1], a4[2], a4[3]);
                     }
             }
-            fence_proxy_async_smem();
+            fence_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(smem_addr(&bar_w_full[b]));
-                mbar_arrive(smem_addr(&bar_meta_empty[b]));
-            }
-            // ---- O of the previous tile
-            if (k > 0) {
-                o_accumulate(k - 1, c_prev);
-                if (newseg) {
-                    flush_o_side(tp.s, tp.last);
-#pragma unroll
-                    for (int h = 0; h < G; ++h) oacc[h] = 0.f;
-                }
-            }
+            if (lane == 0) mbar_arrive(smem_addr(&bar_w_full[wg]));
 #pragma unroll
             for (int h = 0; h < G; ++h) { alpha_prev[h] = alpha[h]; bp_prev[h] = bp_cur[h]; }
             bv_prev = bv_cur;
-            c_prev = t.c;
-            tp = t;
+            c_prev = tcls;
+            kp = k;
         }
-        if (k > 0) {
-            flush_softmax_side(prev_s, seg_first_cta_tile != 0);
-            o_accumulate(k - 1, c_prev);
-            flush_o_side(tp.s, tp.last);
-        } else if (pl.s0 < d.S && r < G) {
-            // no tile starts in this CTA's share, which lies inside stream s0 between two
-            // tiles: the merge reads this slot, so mark it empty
-            d.part[(size_t)(pl.s0 + cta) * part_floats(G) + G + r] = 0.f;
+        if (!wg_any(bid, !ok)) {
+            if (kp >= 0) {
+                o_accumulate(kp, c_prev);
+                flush(cur_s);
+            } else if (cta_empty && pl.s0 < d.S && r < G) {
+                // no tile starts in this CTA's share, which lies inside stream s0 between
+                // two tiles: the merge reads this CTA's slots of s0
+                write_empty(pl.s0);
+            }
         }
     }
 
@@ -1138,6 +1208,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ------------------------------------------------------------ merge + score pass
+// One CTA row per stream: merges the stream's partials (slots 2 (s + c) + w for the CTAs
+// c of its first .. last tile and both warpgroups w; empty ones have l = 0), writes O and
+// the sparsity statistic, then adds p = 2^(x - M) / L to the scores of its slice.
 template <int G, bool STATS>
 __global__ void __launch_bounds__(256) attn_finalize_kernel(const __grid_constant__ Dev d, float *__restrict__ out,
                                                             float *__restrict__ sparsity,
@@ -1167,16 +1240,17 @@ __global__ void __launch_bounds__(256) attn_finalize_kernel(const __grid_constan
         if (tid == 0 && split == 0) raise_error(d.err, kErrInvalid, (uint32_t)s);
         return;
     }
-    const int nparts = c_hi - c_lo + 1;
+    const int nparts = 2 * (c_hi - c_lo + 1);
+    const float *part0 = d.part + (size_t)2 * (s + c_lo) * part_floats(G);
     if (tid < G) {
         float M = kNoMax;
         for (int j = 0; j < nparts; ++j) {
-            const float *pp = d.part + (size_t)(s + c_lo + j) * part_floats(G);
+            const float *pp = part0 + (size_t)j * part_floats(G);
             if (pp[G + tid] > 0.f) M = fmaxf(M, pp[tid]);
         }
         float L = 0.f, E = 0.f;
         for (int j = 0; j < nparts; ++j) {
-            const float *pp = d.part + (size_t)(s + c_lo + j) * part_floats(G);
+            const float *pp = part0 + (size_t)j * part_floats(G);
             const float lj = pp[G + tid];
             const float f = lj > 0.f ? ex2(pp[tid] - M) : 0.f;
             if (j < 64) fac[j][tid] = f;
@@ -1197,7 +1271,7 @@ __global__ void __launch_bounds__(256) attn_finalize_kernel(const __grid_constan
             const int h = i / kD;
             float acc = 0.f;
             for (int j = 0; j < nparts; ++j) {
-                const float *pp = d.part + (size_t)(s + c_lo + j) * part_floats(G);
+                const float *pp = part0 + (size_t)j * part_floats(G);
                 const float f = j < 64 ? fac[j][h] : (pp[G + h] > 0.f ? ex2(pp[h] - gM[h]) : 0.f);
                 if (f > 0.f) acc = fmaf(f, pp[3 * G + i], acc);
             }
@@ -1217,8 +1291,9 @@ __global__ void __launch_bounds__(256) attn_finalize_kernel(const __grid_constan
 int g_bps_i8[kMaxG + 1][2][kMaxDevices] = {};
 
 template <int G, bool STATS>
-cudaError_t launch_i8_g(const Dev &d, const void *q, float scale, float *out, float *sparsity, uint8_t *thought,
-                        float th_r, float th_t, long long live_ub, cudaStream_t st, int64_t *launches) {
+cudaError_t launch_i8_g(const Dev &d, const I8Maps &maps, const void *q, float scale, float *out, float *sparsity,
+                        uint8_t *thought, float th_r, float th_t, long long live_ub, cudaStream_t st,
+                        int64_t *launches) {
     constexpr int smem = smem_bytes(G);
     int sms = 0, bps = 0;
     cudaError_t e = device_sm_count(&sms);
@@ -1240,7 +1315,7 @@ cudaError_t launch_i8_g(const Dev &d, const void *q, float scale, float *out, fl
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     const float xscale = scale * 1.4426950408889634f;   // logits in the log2 domain
-    e = cudaLaunchKernelEx(&cfg, attn_i8_kernel<G, STATS>, d, static_cast<const __nv_bfloat16 *>(q), xscale);
+    e = cudaLaunchKernelEx(&cfg, attn_i8_kernel<G, STATS>, d, maps, static_cast<const __nv_bfloat16 *>(q), xscale);
     *launches += 1;
     if (e != cudaSuccess) return e;
     // the merge + score pass: one CTA per stream, more for long streams
@@ -1257,23 +1332,65 @@ cudaError_t launch_i8_g(const Dev &d, const void *q, float scale, float *out, fl
     return e;
 }
 
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
 }  // namespace
 
-cudaError_t launch_attention_i8(const Dev &d, const void *q, float scale, float *out, float *sparsity,
-                                uint8_t *thought, float th_r, float th_t, long long live_ub, cudaStream_t st,
-                                int64_t *launches) {
+cudaError_t make_i8_maps(const Dev &d, I8Maps *maps) {
+    std::memset(maps, 0, sizeof(*maps));
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &qr);
+    if (e != cudaSuccess) return e;
+    if (fn == nullptr || qr != cudaDriverEntryPointSuccess) return cudaErrorNotSupported;
+    const auto encode = reinterpret_cast<EncodeTiledFn>(fn);
+    for (int c = 0; c < 4; ++c) {
+        const long long rows = (long long)d.S * d.cap[c];
+        if (rows == 0) continue;   // the class holds no records: no tile ever reads it
+        if (rows + 128 > (long long)INT32_MAX) return cudaErrorInvalidValue;
+        const int rec = rec_of(c);
+        if (d.rec[c] != rec) return cudaErrorInvalidValue;
+        const cuuint64_t gdim[2] = {(cuuint64_t)rec, (cuuint64_t)rows};
+        const cuuint64_t gstride[1] = {(cuuint64_t)rec};
+        const cuuint32_t es[2] = {1, 1};
+        const CUtensorMapSwizzle sw = c <= 1 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                             : c == 2 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+        for (int kind = 0; kind < (c == 0 ? 1 : 2); ++kind)
+            for (int small = 0; small < 2; ++small) {
+                const cuuint32_t box[2] = {(cuuint32_t)(kind == 0 ? code_box_bytes(c) : 32),
+                                           (cuuint32_t)(small ? 16 : rows_of(c))};
+                const CUresult r = encode(&maps->m[c][kind][small], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, d.pool[c], gdim,
+                                          gstride, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                          kind == 0 ? sw : CU_TENSOR_MAP_SWIZZLE_NONE,
+                                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+            }
+    }
+    return cudaSuccess;
+}
+
+size_t i8_part_bytes(int S, int G) { return (size_t)2 * (S + kNctaMax) * part_floats(G) * sizeof(float); }
+
+cudaError_t launch_attention_i8(const Dev &d, const I8Maps &maps, const void *q, float scale, float *out,
+                                float *sparsity, uint8_t *thought, float th_r, float th_t, long long live_ub,
+                                cudaStream_t st, int64_t *launches) {
     const bool stats = sparsity != nullptr || thought != nullptr;
+#define TKV_I8_CASE(GG)                                                                                             \
+    case GG:                                                                                                        \
+        return stats ? launch_i8_g<GG, true>(d, maps, q, scale, out, sparsity, thought, th_r, th_t, live_ub, st,   \
+                                             launches)                                                              \
+                     : launch_i8_g<GG, false>(d, maps, q, scale, out, sparsity, thought, th_r, th_t, live_ub, st,  \
+                                              launches);
     switch (d.G) {
-        case 1: return stats ? launch_i8_g<1, true>(d, q, scale, out, sparsity, thought, th_r, th_t, live_ub, st, launches)
-                             : launch_i8_g<1, false>(d, q, scale, out, sparsity, thought, th_r, th_t, live_ub, st, launches);
-        case 2: return stats ? launch_i8_g<2, true>(d, q, scale, out, sparsity, thought, th_r, th_t, live_ub, st, launches)
-                             : launch_i8_g<2, false>(d, q, scale, out, sparsity, thought, th_r, th_t, live_ub, st, launches);
-        case 4: return stats ? launch_i8_g<4, true>(d, q, scale, out, sparsity, thought, th_r, th_t, live_ub, st, launches)
-                             : launch_i8_g<4, false>(d, q, scale, out, sparsity, thought, th_r, th_t, live_ub, st, launches);
-        case 8: return stats ? launch_i8_g<8, true>(d, q, scale, out, sparsity, thought, th_r, th_t, live_ub, st, launches)
-                             : launch_i8_g<8, false>(d, q, scale, out, sparsity, thought, th_r, th_t, live_ub, st, launches);
+        TKV_I8_CASE(1)
+        TKV_I8_CASE(2)
+        TKV_I8_CASE(4)
+        TKV_I8_CASE(8)
         default: return cudaErrorInvalidValue;
     }
+#undef TKV_I8_CASE
 }
 
 }  // namespace tkv

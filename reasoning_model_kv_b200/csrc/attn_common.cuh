@@ -5,6 +5,8 @@
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp4.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
 #include "tkv_internal.cuh"
@@ -233,6 +235,41 @@ __device__ __forceinline__ uint32_t quarter_pair(const uint32_t (&w)[BITS], uint
     return code_pair<BITS, P % ppw>(w[P / ppw], magic);
 }
 
+// ------------------------------------------------- floating-point code pair -> f16x2
+// (codec 1; same storage order as the integer codes: pair S at elements S and
+// S + 16/BITS, i.e. 16 bits apart.)  8: E4M3 and 4: E2M1 through the hardware
+// conversions (every value is exact in f16); 2: ternary 1 -> +1, 3 -> -1, 0 -> 0.
+template <int BITS, int S>
+__device__ __forceinline__ uint32_t code_pair_fp(uint32_t word) {
+    if constexpr (BITS == 8) {
+        const uint32_t b2 = __byte_perm(word, 0u, S == 0 ? 0x0020u : 0x0031u);   // bytes S, S + 2
+        const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)b2, __NV_E4M3);
+        return (uint32_t)h.x | ((uint32_t)h.y << 16);
+    } else if constexpr (BITS == 4) {
+        const uint32_t b = ((word >> (4 * S)) & 0xFu) | ((word >> (4 * S + 12)) & 0xF0u);   // nibbles S, S + 4
+        const __half2_raw h = __nv_cvt_fp4x2_to_halfraw2((__nv_fp4x2_storage_t)b, __NV_E2M1);
+        return (uint32_t)h.x | ((uint32_t)h.y << 16);
+    } else {
+        const uint32_t c = (word >> (2 * S)) & 0x00030003u;
+        return (c & 0x00010001u) * 0x3C00u | ((c & 0x00020002u) << 14);
+    }
+}
+
+template <int BITS, int P>
+__device__ __forceinline__ uint32_t quarter_pair_fp(const uint32_t (&w)[BITS]) {
+    constexpr int ppw = 16 / BITS;
+    return code_pair_fp<BITS, P % ppw>(w[P / ppw]);
+}
+
+// f16x2 with both halves the value of E4M3 code `code` (exact).
+__device__ __forceinline__ uint32_t e4m3_h2(uint32_t code) {
+    const __half_raw h = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)code, __NV_E4M3);
+    return (uint32_t)h.x * 0x00010001u;
+}
+__device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
+    return h2_as_u32(__hmul2(u32_as_h2(a), u32_as_h2(b)));
+}
+
 // One row's quarter (4*BITS bytes at byte offset `off` of the record).  Int8 tiles keep
 // rows unpadded (288 bytes) and store odd rows with 16-byte chunks k and k ^ 1
 // swapped, which spreads the two rows a load phase touches over all 32 banks.
@@ -296,6 +333,45 @@ __device__ __forceinline__ void qk_group(float (&x)[4], const uint32_t (&k0)[BIT
         x[2] = fmaf(km1[GRP].x, acc[2], fmaf(km1[GRP].y, qs[0][GRP], x[2]));
         x[3] = fmaf(km1[GRP].x, acc[3], fmaf(km1[GRP].y, qs[1][GRP], x[3]));
     }
+}
+
+// S += K . Q^T over head-dim group GRP for floating-point codes (codec 1), pairs as in
+// qk_group.  FP8 / ternary: the code values against the f16 query, times the group's
+// fp16 scale (ka / kc: the four K scales of rows g / g + 8); no zero term.  NVFP4: each
+// code times its 16-dim block's E4M3 scale (ka / kc: the eight block scales) is exact
+// in f16, so the products need no scale afterwards.  Lane tig holds quarter tig, whose
+// dims of group GRP lie in block 2 GRP + tig / 2.
+template <int BITS, int GRP>
+__device__ __forceinline__ void qk_group_fp(float (&x)[4], const uint32_t (&k0)[BITS], const uint32_t (&k1)[BITS],
+                                            const uint32_t (&qb)[4][2][2], const float (&qinv)[2][4], bool qscaled,
+                                            const uint2 &ka, const uint2 &kc, int tig) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    uint32_t a[4][2];   // pairs 4 GRP + j of rows g (0) and g + 8 (1)
+    a[0][0] = quarter_pair_fp<BITS, 4 * GRP>(k0); a[0][1] = quarter_pair_fp<BITS, 4 * GRP>(k1);
+    a[1][0] = quarter_pair_fp<BITS, 4 * GRP + 1>(k0); a[1][1] = quarter_pair_fp<BITS, 4 * GRP + 1>(k1);
+    a[2][0] = quarter_pair_fp<BITS, 4 * GRP + 2>(k0); a[2][1] = quarter_pair_fp<BITS, 4 * GRP + 2>(k1);
+    a[3][0] = quarter_pair_fp<BITS, 4 * GRP + 3>(k0); a[3][1] = quarter_pair_fp<BITS, 4 * GRP + 3>(k1);
+    float s0 = 1.f, s1 = 1.f;
+    if constexpr (BITS == 4) {
+        const int sh = 8 * ((2 * GRP + (tig >> 1)) & 3);
+        const uint32_t b0 = e4m3_h2(((GRP < 2 ? ka.x : ka.y) >> sh) & 0xFFu);
+        const uint32_t b1 = e4m3_h2(((GRP < 2 ? kc.x : kc.y) >> sh) & 0xFFu);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) { a[j][0] = hmul2_u32(a[j][0], b0); a[j][1] = hmul2_u32(a[j][1], b1); }
+    } else {
+        const int sh = 16 * (GRP & 1);
+        s0 = __half2float(__ushort_as_half((unsigned short)(((GRP < 2 ? ka.x : ka.y) >> sh) & 0xFFFFu)));
+        s1 = __half2float(__ushort_as_half((unsigned short)(((GRP < 2 ? kc.x : kc.y) >> sh) & 0xFFFFu)));
+    }
+    mma16816(acc, a[0][0], a[0][1], a[1][0], a[1][1], qb[GRP][0][0], qb[GRP][0][1]);
+    mma16816(acc, a[2][0], a[2][1], a[3][0], a[3][1], qb[GRP][1][0], qb[GRP][1][1]);
+    if (qscaled) {
+        acc[0] *= qinv[0][GRP]; acc[1] *= qinv[1][GRP]; acc[2] *= qinv[0][GRP]; acc[3] *= qinv[1][GRP];
+    }
+    x[0] = fmaf(s0, acc[0], x[0]);
+    x[1] = fmaf(s0, acc[1], x[1]);
+    x[2] = fmaf(s1, acc[2], x[2]);
+    x[3] = fmaf(s1, acc[3], x[3]);
 }
 
 // (scale, zero) pairs of the 4 groups from half of a record's meta block.

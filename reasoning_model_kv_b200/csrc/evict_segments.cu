@@ -23,7 +23,7 @@
 // thought-aware budget allocation of the TAM page (sections 2.B and 2.C) as a
 // selection policy.  After the first sweep a warp per segment counts the
 // segment's candidates (unprotected entries of its run) and sums their scores
-// (fp64); the block forms the stream's mean, delta = c * mean, the pivotal
+// exactly (integer digits: the same sum in any order); the block forms the stream's mean, delta = c * mean, the pivotal
 // candidates (score >= delta: kept, ranked first like protected entries) and the
 // budgets t_j = min(n_j - p_j, floor(T' (a_j / D) + 1e-9)) with a_j = sqrt(w_j) n_j,
 // D = sum a_j, T' = max(0, budget - pivotal), which then play the role of the
@@ -49,6 +49,53 @@ __host__ __device__ constexpr int tam_table_bytes(int ms) {
 }
 constexpr int kUnionBytes = kWarpsE * kStage * 8 > kMoveBytes ? kWarpsE * kStage * 8 : kMoveBytes;
 
+// Exact sums of fp32 scores for the TAM means.  A finite non-negative fp32 is
+// m * 2^(b - 149) (m < 2^24, 0 <= b <= 253), so a sum of them is an integer times
+// 2^-149 held in nine 32-bit digits, each in a 64-bit counter with room for the
+// carries of 2^32 terms: integer adds, so every summation order gives the same sum.
+// Negative and non-finite scores (attention mass is neither) count as 0.
+constexpr int kDig = 9;
+__device__ __forceinline__ void xsum_add(unsigned long long (&a)[kDig], float v) {
+    const uint32_t u = __float_as_uint(v);
+    const uint32_t eb = u >> 23;
+    if (u == 0u || eb >= 255u) return;
+    const unsigned long long m = eb ? ((u & 0x7FFFFFu) | 0x800000u) : (u & 0x7FFFFFu);
+    const int b = eb ? (int)eb - 1 : 0;
+    const unsigned long long x = m << (b & 31);
+    const int i = b >> 5;
+#pragma unroll
+    for (int k = 0; k < kDig; ++k) {   // register-resident digits: no indexed access
+        if (k == i) a[k] += x & 0xFFFFFFFFull;
+        if (k == i + 1) a[k] += x >> 32;
+    }
+}
+// The sum rounded to the nearest double (ties to even): the leading 64 bits, with every
+// bit below them folded into the lowest (sticky), converted once and scaled by 2^e.
+__device__ double xsum_value(const unsigned long long (&a)[kDig]) {
+    uint32_t dig[kDig + 2];
+    unsigned long long carry = 0;
+#pragma unroll
+    for (int k = 0; k < kDig; ++k) {
+        const unsigned long long t = a[k] + carry;
+        dig[k] = (uint32_t)t;
+        carry = t >> 32;
+    }
+    dig[kDig] = (uint32_t)carry;
+    dig[kDig + 1] = (uint32_t)(carry >> 32);
+    int top = kDig + 1;
+    while (top >= 0 && dig[top] == 0u) --top;
+    if (top < 0) return 0.0;
+    const unsigned long long w2 = dig[top], w1 = top >= 1 ? dig[top - 1] : 0u, w0 = top >= 2 ? dig[top - 2] : 0u;
+    bool sticky = false;
+    for (int k = 0; k < top - 2; ++k) sticky |= dig[k] != 0u;
+    const int lz = __clz((int)(uint32_t)w2);
+    unsigned long long t = ((w2 << 32) | w1) << lz;
+    if (lz) t |= w0 >> (32 - lz);
+    if (((w0 << lz) & 0xFFFFFFFFull) != 0ull || sticky) t |= 1ull;
+    const int e = 32 - lz + 32 * (top - 2) - 149;   // in [-212, 202]: 2^e is a normal double
+    return __dmul_rn(__ull2double_rn(t), __longlong_as_double((long long)(1023 + e) << 52));
+}
+
 template <bool TAM>
 __global__ void __launch_bounds__(kThreads) tbe_kernel(Dev d, const int32_t *__restrict__ seg_start,
                                                        const uint8_t *__restrict__ seg_label,
@@ -64,13 +111,13 @@ __global__ void __launch_bounds__(kThreads) tbe_kernel(Dev d, const int32_t *__r
     int *lo = keep + ms;
     int *hi = lo + ms;
     uint8_t *label = reinterpret_cast<uint8_t *>(hi + ms);
-    double *ssum = reinterpret_cast<double *>(dyn + seg_table_bytes(ms));   // TAM only
+    double *ssum = reinterpret_cast<double *>(dyn + seg_table_bytes(ms));   // TAM only: w_j n_j, then a_j
     int *scnt = reinterpret_cast<int *>(ssum + ms);
     int *spiv = scnt + ms;
     uint8_t *un = dyn + seg_table_bytes(ms) + (TAM ? tam_table_bytes(ms) : 0);   // ranking stage, then moves
     uint4 *move_buf = reinterpret_cast<uint4 *>(un);
-    __shared__ double red_d[kWarpsE];
-    __shared__ double sh_delta;
+    __shared__ double sh_delta, sh_D;
+    __shared__ unsigned long long tot_dig[kDig];   // TAM: exact sum of every candidate's score
 
     const int s = blockIdx.x, b = s / d.Hkv;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -122,38 +169,44 @@ __global__ void __launch_bounds__(kThreads) tbe_kernel(Dev d, const int32_t *__r
 
     double delta = 0.0;   // TAM: candidates scoring at least delta are pivotal
     if constexpr (TAM) {
-        // T1. per segment: candidates and their score sum (fp64)
+        if (tid < kDig) tot_dig[tid] = 0ull;
+        __syncthreads();
+        // T1. per segment: candidates and the exact sum of their scores
         for (int j = warp; j < ns; j += kWarpsE) {
             const int c = label[j];
             int n = 0;
-            double m = 0.0;
+            unsigned long long a[kDig];
+#pragma unroll
+            for (int k = 0; k < kDig; ++k) a[k] = 0ull;
             if (c <= 3) {
                 const int32_t *pc = d.pos[c] + (size_t)s * d.cap[c];
                 const float *sc = d.score[c] + (size_t)s * d.cap[c];
                 for (int i = lo[j] + lane; i < hi[j]; i += 32)
-                    if (pc[i] >= d.n_protect) { ++n; m += (double)sc[i]; }
+                    if (pc[i] >= d.n_protect) { ++n; xsum_add(a, sc[i]); }
             }
+            n = __reduce_add_sync(kFull, n);
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                n += __shfl_xor_sync(kFull, n, o);
-                m += __shfl_xor_sync(kFull, m, o);
+            for (int k = 0; k < kDig; ++k)
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) a[k] += __shfl_xor_sync(kFull, a[k], o);
+            if (lane == 0) {
+                scnt[j] = n;
+                ssum[j] = xsum_value(a);
+#pragma unroll
+                for (int k = 0; k < kDig; ++k)
+                    if (a[k]) atomicAdd(&tot_dig[k], a[k]);
             }
-            if (lane == 0) { scnt[j] = n; ssum[j] = m; }
         }
-        __syncthreads();
         // T2. the stream's mean score over all candidates -> delta
         {
-            double m = 0.0;
             int n = 0;
-            for (int j = tid; j < ns; j += kThreads) { m += ssum[j]; n += scnt[j]; }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) m += __shfl_xor_sync(kFull, m, o);
-            if (lane == 0) red_d[warp] = m;
-            const int ntot = block_sum(n, scratch);   // ends with a barrier: red_d complete
+            for (int j = tid; j < ns; j += kThreads) n += scnt[j];
+            const int ntot = block_sum(n, scratch);   // ends with a barrier: tot_dig complete
             if (tid == 0) {
-                double tot = 0.0;
-                for (int w = 0; w < kWarpsE; ++w) tot += red_d[w];
-                sh_delta = ntot > 0 ? cpiv * (tot / (double)ntot) : -1.0;
+                unsigned long long t[kDig];
+#pragma unroll
+                for (int k = 0; k < kDig; ++k) t[k] = tot_dig[k];
+                sh_delta = ntot > 0 ? __dmul_rn(cpiv, __ddiv_rn(xsum_value(t), (double)ntot)) : -1.0;
             }
             __syncthreads();
             if (ntot == 0) return;   // no candidates: nothing to evict
@@ -173,24 +226,30 @@ __global__ void __launch_bounds__(kThreads) tbe_kernel(Dev d, const int32_t *__r
             if (lane == 0) spiv[j] = p;
         }
         __syncthreads();
-        // T4. budgets: T' = max(0, budget - pivotal), t_j = min(n_j - p_j, floor(T' a_j / D + 1e-9))
+        // T4. budgets: T' = max(0, budget - pivotal), t_j = min(n_j - p_j, floor(T' a_j / D + 1e-9)),
+        // a_j = sqrt(w_j) n_j and D = sum a_j in segment order (every operation rounded once,
+        // no fused multiply-add: the same doubles as a plain sequential evaluation)
         {
-            double a = 0.0;
             int P = 0;
             for (int j = tid; j < ns; j += kThreads) {
-                if (scnt[j] > 0) a += sqrt(ssum[j] / scnt[j]) * scnt[j];
+                const int n = scnt[j];
+                ssum[j] = n > 0 ? __dmul_rn(__dsqrt_rn(__ddiv_rn(ssum[j], (double)n)), (double)n) : 0.0;
                 P += spiv[j];
             }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(kFull, a, o);
-            if (lane == 0) red_d[warp] = a;
-            const int Ptot = block_sum(P, scratch);
-            double D = 0.0;
-            for (int w = 0; w < kWarpsE; ++w) D += red_d[w];
+            const int Ptot = block_sum(P, scratch);   // ends with a barrier: every a_j written
+            if (tid == 0) {
+                double D = 0.0;
+                for (int j = 0; j < ns; ++j)
+                    if (scnt[j] > 0) D = __dadd_rn(D, ssum[j]);
+                sh_D = D;
+            }
+            __syncthreads();
+            const double D = sh_D;
             const double Tp = budget > Ptot ? (double)(budget - Ptot) : 0.0;
             for (int j = tid; j < ns; j += kThreads) {
                 long long t = 0;
-                if (scnt[j] > 0 && D > 0.0) t = (long long)floor(Tp * (sqrt(ssum[j] / scnt[j]) * scnt[j] / D) + 1e-9);
+                if (scnt[j] > 0 && D > 0.0)
+                    t = (long long)floor(__dadd_rn(__dmul_rn(Tp, __ddiv_rn(ssum[j], D)), 1e-9));
                 const int cap_j = scnt[j] - spiv[j];
                 keep[j] = (int)(t < cap_j ? t : cap_j);
             }

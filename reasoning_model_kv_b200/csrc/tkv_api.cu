@@ -23,6 +23,8 @@ struct tkv_cache {
     uint8_t *base;
     long long live_ub;   // host-side upper bound of live entries in any stream
     int64_t launches;
+    tkv::I8Maps maps;    // TMA descriptors of the pools (tensor-core attention), made on first use
+    bool maps_ready;
 };
 
 namespace {
@@ -59,6 +61,8 @@ bool valid_config(const tkv_config *c, std::string *why) {
     if (c->dense != 0 && c->dense != 1) { *why = "dense must be 0 or 1"; return false; }
     if (c->attn_kernel != 0 && c->attn_kernel != 1) { *why = "attn_kernel must be 0 or 1"; return false; }
     if (c->attn_kernel == 1 && c->dense != 1) { *why = "attn_kernel 1 needs dense placement"; return false; }
+    if (c->codec != 0 && c->codec != 1) { *why = "codec must be 0 or 1"; return false; }
+    if (c->codec == 1 && c->attn_kernel != 0) { *why = "codec 1 needs attn_kernel 0"; return false; }
     for (int i = 0; i < 4; ++i)
         if (c->cap[i] >= (1 << 24)) { *why = "cap[c] must be < 2^24"; return false; }
     return true;
@@ -81,7 +85,7 @@ void make_layout(const tkv_config &c, tkv_layout *lay, tkv::Dev *dev, uint8_t *b
         lay->fs[k] = take(e * sizeof(int32_t));
     }
     for (int k = 0; k < 4; ++k) {
-        lay->rec_bytes[k] = tkv::record_bytes(c.bits[k]);
+        lay->rec_bytes[k] = tkv::record_bytes(c.bits[k], c.codec);
         lay->pool[k] = take(S * (size_t)c.cap[k] * lay->rec_bytes[k]);
     }
     lay->state_bytes = off;
@@ -90,7 +94,7 @@ void make_layout(const tkv_config &c, tkv_layout *lay, tkv::Dev *dev, uint8_t *b
     const size_t o_rank = take((size_t)c.B * c.max_append * sizeof(int32_t));
     const size_t o_tot = take((size_t)c.B * 4 * sizeof(int32_t));
     const size_t o_lg = take(S * (size_t)ncap * c.G * sizeof(float));
-    const size_t o_part = take((S + tkv::kNctaMax) * (size_t)tkv::part_floats(c.G) * sizeof(float));
+    const size_t o_part = take(tkv::part_bytes(S, c.G));
     const size_t o_seglo = take(S * sizeof(int32_t));
     const size_t o_seghi = take(S * sizeof(int32_t));
     lay->total_bytes = off;
@@ -99,6 +103,7 @@ void make_layout(const tkv_config &c, tkv_layout *lay, tkv::Dev *dev, uint8_t *b
     dev->n_protect = c.n_protect; dev->max_append = c.max_append;
     dev->dense = c.dense;
     dev->attn_kernel = c.attn_kernel;
+    dev->codec = c.codec;
     dev->n = reinterpret_cast<int32_t *>(base + lay->n);
     dev->ft = reinterpret_cast<int32_t *>(base + lay->ft);
     dev->hw = reinterpret_cast<int32_t *>(base + lay->hw);
@@ -216,6 +221,7 @@ tkv_status tkv_create(const tkv_config *cfg, void *d_workspace, size_t workspace
     make_layout(*cfg, &c->lay, &c->dev, c->base);
     c->live_ub = 0;
     c->launches = 0;
+    c->maps_ready = false;
     *out = c;
     return TKV_OK;
 }
@@ -255,14 +261,33 @@ tkv_status tkv_quantize_append(tkv_cache *c, const void *k, const void *v, const
     return cuda_status(e, "tkv_quantize_append");
 }
 
+namespace {
+// The pools' TMA descriptors, encoded once per cache (the pools never move).
+tkv_status ensure_maps(tkv_cache *c) {
+    if (c->maps_ready) return TKV_OK;
+    cudaError_t e = tkv::make_i8_maps(c->dev, &c->maps);
+    if (e != cudaSuccess) return cuda_status(e, "encoding the pools' TMA descriptors");
+    c->maps_ready = true;
+    return TKV_OK;
+}
+}  // namespace
+
 tkv_status tkv_decode_attention(tkv_cache *c, const void *q, float softmax_scale, float *out,
                                 void *stream) {
     if (!c) return fail(TKV_ERR_INVALID, "cache is NULL");
     if (!q || !out) return fail(TKV_ERR_INVALID, "NULL q or out");
     if (!aligned16(q) || !aligned16(out)) return fail(TKV_ERR_INVALID, "q and out must be 16-byte aligned");
     const long long ub = std::max(1ll, c->live_ub);
-    cudaError_t e = tkv::launch_attention(c->dev, q, softmax_scale, out, ub,
-                                          static_cast<cudaStream_t>(stream), &c->launches);
+    cudaError_t e;
+    if (c->cfg.dense == 1 && c->cfg.attn_kernel == 1) {
+        const tkv_status ms = ensure_maps(c);
+        if (ms != TKV_OK) return ms;
+        e = tkv::launch_attention_i8(c->dev, c->maps, q, softmax_scale, out, nullptr, nullptr, 0.f, 0.f, ub,
+                                     static_cast<cudaStream_t>(stream), &c->launches);
+    } else {
+        e = tkv::launch_attention(c->dev, q, softmax_scale, out, ub, static_cast<cudaStream_t>(stream),
+                                  &c->launches);
+    }
     return cuda_status(e, "tkv_decode_attention");
 }
 
@@ -276,9 +301,11 @@ tkv_status tkv_decode_attention_sparsity(tkv_cache *c, const void *q, float soft
         return fail(TKV_ERR_INVALID, "thresholds must be finite with th_r <= th_t");
     if (!(c->cfg.dense == 1 && c->cfg.attn_kernel == 1))
         return fail(TKV_ERR_INVALID, "the sparsity statistic needs dense placement and attn_kernel 1");
+    const tkv_status ms = ensure_maps(c);
+    if (ms != TKV_OK) return ms;
     const long long ub = std::max(1ll, c->live_ub);
-    cudaError_t e = tkv::launch_attention_i8(c->dev, q, softmax_scale, out, sparsity, thought, th_r, th_t, ub,
-                                             static_cast<cudaStream_t>(stream), &c->launches);
+    cudaError_t e = tkv::launch_attention_i8(c->dev, c->maps, q, softmax_scale, out, sparsity, thought, th_r, th_t,
+                                             ub, static_cast<cudaStream_t>(stream), &c->launches);
     return cuda_status(e, "tkv_decode_attention_sparsity");
 }
 

@@ -2,6 +2,7 @@
 // of the sm_100a kernels.  Internal to libtkv (the C ABI is include/tkv.h).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstddef>
 #include <cstdint>
@@ -13,9 +14,14 @@ constexpr int kGroup = 32;    // quantisation group along head dim
 constexpr int kNG = kD / kGroup;
 constexpr int kMaxG = 8;      // query heads per kv head supported
 
-// Record bytes of a class with `bits` bits per element (bits == 16: bf16).
-__host__ __device__ constexpr int record_bytes(int bits) {
-    return bits == 16 ? 4 * kD : 2 * (kD * bits / 8) + 4 * kNG * 2;
+// Record bytes of a class with `bits` bits per element (bits == 16: bf16) under codec 0
+// (integer codes, fp16 scale + zero per group) or codec 1 (floating-point codes: FP8
+// and ternary with an fp16 scale per group, NVFP4 with an E4M3 scale per 16 dims).
+__host__ __device__ constexpr int record_bytes(int bits, int codec = 0) {
+    return bits == 16 ? 4 * kD
+           : codec == 0 ? 2 * (kD * bits / 8) + 4 * kNG * 2
+           : bits == 4 ? 2 * (kD / 2) + 2 * (kD / 16)
+                       : 2 * (kD * bits / 8) + 2 * kNG * 2;
 }
 
 // Everything a kernel needs to address one cache.  Passed by value.
@@ -23,6 +29,7 @@ struct Dev {
     int B, Hkv, G, S, n_protect, max_append;
     int dense;              // 1: live records contiguous in table order (handle[i] == i)
     int attn_kernel;        // 0: warp-tile (mma.sync) kernel, 1: tensor-memory (tcgen05) kernel
+    int codec;              // 0: integer class records, 1: FP8 / NVFP4 / ternary class records
     int cap[4];
     int rec[4];
     int32_t *n, *ft, *hw;   // [S][4]
@@ -35,10 +42,10 @@ struct Dev {
     int32_t *totals;   // [B][4] tokens per class in the current append
     float *logits;     // [S][ncap][G] raw logits (log2 domain) of the current step
     int ncap;          // sum of cap[c], rounded up to a multiple of 32
-    // tensor-core decode attention (attention_i8.cu): per (stream, CTA) partial
-    // results, slot s + cta, part_floats(G) floats each, and the first / last CTA of
-    // every stream
-    float *part;       // [S + ncta_max][part_floats(G)]
+    // tensor-core decode attention (attention_i8.cu): per (stream, CTA, warpgroup)
+    // partial results, slot 2 (s + cta) + warpgroup, part_floats(G) floats each, and
+    // the first / last CTA of every stream
+    float *part;       // [2 (S + ncta_max)][part_floats(G)]
     int32_t *seg_lo, *seg_hi;   // [S]
     int ncta_max;
 };
@@ -47,6 +54,15 @@ struct Dev {
 // sum and sum p*(x - m) per head, then the unnormalised O [G][D].
 __host__ __device__ constexpr int part_floats(int G) { return G * (3 + kD); }
 constexpr int kNctaMax = 1024;   // upper bound on the persistent grid (one CTA per SM)
+__host__ __device__ constexpr size_t part_bytes(size_t S, int G) {
+    return 2 * (S + kNctaMax) * (size_t)part_floats(G) * sizeof(float);
+}
+
+// TMA descriptors of the record pools for the tensor-core decode attention:
+// m[class][0 = code boxes, 1 = scale / zero box][0 = a whole tile's rows, 1 = 16 rows].
+struct I8Maps {
+    CUtensorMap m[4][2][2];
+};
 
 enum : uint32_t { kErrInvalid = 1, kErrCapacity = 2, kErrTimeout = 4 };
 
@@ -98,9 +114,11 @@ cudaError_t launch_attention(const Dev &d, const void *q, float scale, float *ou
 // Dense placement: the tensor-core kernel with integer operands (attention_i8.cu).  With
 // sparsity / thought non-NULL it also writes, per (stream, query head), the attention
 // sparsity 1 - H(p) / ln N and its thought class under the thresholds th_r <= th_t.
-cudaError_t launch_attention_i8(const Dev &d, const void *q, float scale, float *out, float *sparsity,
-                                uint8_t *thought, float th_r, float th_t, long long live_ub, cudaStream_t st,
-                                int64_t *launches);
+cudaError_t launch_attention_i8(const Dev &d, const I8Maps &maps, const void *q, float scale, float *out,
+                                float *sparsity, uint8_t *thought, float th_r, float th_t, long long live_ub,
+                                cudaStream_t st, int64_t *launches);
+// Encodes the TMA descriptors of d's pools (host only; needs the CUDA driver).
+cudaError_t make_i8_maps(const Dev &d, I8Maps *maps);
 // Self-test of the bounded device waits (selftest.cu).
 cudaError_t launch_wait_timeout(const Dev &d, long long limit, cudaStream_t st, int64_t *launches);
 cudaError_t launch_evict(const Dev &d, int budget, int keep_from, cudaStream_t st, int64_t *launches);

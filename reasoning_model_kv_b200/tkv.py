@@ -35,7 +35,7 @@ class TkvConfig(ctypes.Structure):
                 ("D", ctypes.c_int32), ("group", ctypes.c_int32), ("bits", ctypes.c_int32 * 4),
                 ("n_protect", ctypes.c_int32), ("cap", ctypes.c_int32 * 4),
                 ("max_append", ctypes.c_int32), ("dense", ctypes.c_int32),
-                ("attn_kernel", ctypes.c_int32)]
+                ("attn_kernel", ctypes.c_int32), ("codec", ctypes.c_int32)]
 
 
 class TkvLayout(ctypes.Structure):
@@ -111,7 +111,7 @@ def _check(status: int):
 
 
 def make_config(B, Hkv, G, cap, n_protect, max_append=1, D=128, group=32, dense=False,
-                attn_kernel=0) -> TkvConfig:
+                attn_kernel=0, codec=0) -> TkvConfig:
     cfg = TkvConfig()
     cfg.B, cfg.Hkv, cfg.G, cfg.D, cfg.group = B, Hkv, G, D, group
     for i in range(4):
@@ -121,6 +121,7 @@ def make_config(B, Hkv, G, cap, n_protect, max_append=1, D=128, group=32, dense=
     cfg.max_append = max_append
     cfg.dense = int(bool(dense))
     cfg.attn_kernel = int(attn_kernel)
+    cfg.codec = int(codec)
     return cfg
 
 
@@ -148,10 +149,13 @@ class TkvCache:
     """One layer's compressed KV cache: a device workspace owned by torch plus the
     library's cache object.  Methods mirror the C ABI names."""
 
-    def __init__(self, B, Hkv, G, cap, n_protect, max_append=1, device="cuda", dense=False, attn_kernel=0):
-        self.cfg = make_config(B, Hkv, G, cap, n_protect, max_append, dense=dense, attn_kernel=attn_kernel)
+    def __init__(self, B, Hkv, G, cap, n_protect, max_append=1, device="cuda", dense=False, attn_kernel=0,
+                 codec=0):
+        self.cfg = make_config(B, Hkv, G, cap, n_protect, max_append, dense=dense, attn_kernel=attn_kernel,
+                               codec=codec)
         self.dense = bool(dense)
         self.attn_kernel = int(attn_kernel)
+        self.codec = int(codec)
         self.B, self.Hkv, self.G, self.S = B, Hkv, G, B * Hkv
         self.cap = tuple(int(c) for c in cap)
         self.n_protect, self.max_append = n_protect, max_append

@@ -27,7 +27,8 @@ def oracle_for(gpu: TkvCache, state: dict, B: int | None = None) -> orc.OracleCa
     """An oracle cache holding `state` (exported from `gpu`, possibly a subset of
     whole batch rows: B rows x Hkv streams)."""
     Bn = B if B is not None else gpu.B
-    o = orc.OracleCache(Bn, gpu.Hkv, gpu.G, cap=gpu.cap, n_protect=gpu.n_protect, dense=gpu.dense)
+    o = orc.OracleCache(Bn, gpu.Hkv, gpu.G, cap=gpu.cap, n_protect=gpu.n_protect, dense=gpu.dense,
+                        codec=gpu.codec)
     o.load_state(state)
     return o
 
@@ -84,20 +85,21 @@ MODES = {"reuse": dict(dense=False), "dense": dict(dense=True),
          "dense_tc": dict(dense=True, attn_kernel=1)}
 
 
-def build_pair(name: str, device="cuda", rows=None, dense=False, attn_kernel=0, **over):
+def build_pair(name: str, device="cuda", rows=None, dense=False, attn_kernel=0, codec=0, **over):
     """Prefill a GPU cache with a workload, and an oracle cache with the same
     inputs for batch rows `rows` (default: all); `dense` selects dense placement
     on both sides, `attn_kernel` the GPU's decode-attention kernel.  Returns
     (w, gpu, oracle, rows)."""
     w = synth.prefill_inputs(name, **over)
     gpu = TkvCache(w["B"], w["Hkv"], w["G"], w["cap"], w["n_protect"], max_append=w["ctx"], dense=dense,
-                   attn_kernel=attn_kernel)
+                   attn_kernel=attn_kernel, codec=codec)
     k, v = w["k"].to(device), w["v"].to(device)
     cls = w["cls"][:, :w["ctx"]].contiguous().to(device)
     pos = w["pos"].to(device)
     gpu.quantize_append(k, v, cls, pos)
     rows = list(range(w["B"])) if rows is None else list(rows)
-    o = orc.OracleCache(len(rows), w["Hkv"], w["G"], cap=w["cap"], n_protect=w["n_protect"], dense=dense)
+    o = orc.OracleCache(len(rows), w["Hkv"], w["G"], cap=w["cap"], n_protect=w["n_protect"], dense=dense,
+                        codec=codec)
     st = o.append(np_bits(w["k"][rows]), np_bits(w["v"][rows]), w["cls"][rows, :w["ctx"]].numpy(),
                   w["pos"][rows].numpy())
     assert st == orc.ORC_OK

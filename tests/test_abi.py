@@ -184,12 +184,31 @@ def test_every_config_rule_is_enforced_on_the_host():
     for kw in (dict(Hkv=0), dict(G=16), dict(n_protect=-1), dict(max_append=(1 << 24) + 1),
                dict(B=256, Hkv=256),                  # B * Hkv above 65535
                dict(cap=[0, 1 << 24, 0, 0]),          # a class capacity of 2^24
-               dict(attn_kernel=1)):                  # the tensor-memory kernel needs dense placement
+               dict(attn_kernel=1),                   # the tensor-memory kernel needs dense placement
+               dict(dense=True, attn_kernel=1, codec=1)):   # FP codes: the warp-tile kernel only
         assert tkv.tkv_workspace_bytes(_cfg(**kw)) == 0, kw
-    for field, value in (("group", 16), ("dense", 2), ("attn_kernel", 2)):
+    for field, value in (("group", 16), ("dense", 2), ("attn_kernel", 2), ("codec", 2)):
         cfg = _cfg()
         setattr(cfg, field, value)
         assert tkv.tkv_workspace_bytes(cfg) == 0, field
     cfg = _cfg()
     cfg.bits[0] = 8
     assert tkv.tkv_workspace_bytes(cfg) == 0
+
+
+def test_fp_codec_record_sizes_in_the_layout():
+    """codec 1: class records of 272 (FP8), 144 (NVFP4) and 80 (ternary) bytes, as the
+    header documents and the oracle packs them; codec 0 keeps 288 / 160 / 96."""
+    from oracle import oracle as orc
+    for codec, want in ((0, [512, 288, 160, 96]), (1, [512, 272, 144, 80])):
+        cfg = _cfg(codec=codec)
+        n = tkv.tkv_workspace_bytes(cfg)
+        assert n > 0
+        L = tkv.lib()
+        h = ctypes.c_void_p()
+        assert L.tkv_create(ctypes.byref(cfg), ctypes.c_void_p(1 << 20), n, ctypes.byref(h)) == 0
+        lay = tkv.TkvLayout()
+        assert L.tkv_get_layout(h, ctypes.byref(lay)) == 0
+        assert list(lay.rec_bytes) == want
+        assert want[1:] == [orc.record_bytes_fmt(orc.class_format(b, codec)) for b in (8, 4, 2)]
+        assert L.tkv_destroy(h) == 0

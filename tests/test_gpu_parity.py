@@ -286,7 +286,7 @@ def test_b8_ctx16k_decode_loop_sampled_steps(mode):
     assert gpu.poll_error() == tkv.TKV_OK
 
 
-@pytest.mark.parametrize("mode", ["reuse", "dense"])
+@pytest.mark.parametrize("mode", list(MODES))
 def test_b1_ctx131k_long_decode_sampled_steps(mode):
     """Batch 1 x 64/8 heads (G = 8), 131k context, transition-heavy segments,
     eviction to 4096 every 64 steps; lock-step at steps 0, 63, 64 and 200."""
@@ -310,7 +310,7 @@ def test_b1_ctx131k_long_decode_sampled_steps(mode):
     assert gpu.poll_error() == tkv.TKV_OK
 
 
-@pytest.mark.parametrize("mode", ["reuse", "dense"])
+@pytest.mark.parametrize("mode", list(MODES))
 def test_l32_b32_ctx32k_decode_loop_sampled_layers_and_steps(mode):
     """32 layers x batch 32 x 32/8 heads, 32k context with K outliers and a 128-token
     bf16 window, 1024 decode steps with eviction to 1638 every 64 steps.  Every layer
@@ -430,3 +430,47 @@ def test_extreme_magnitudes_sinks_and_query(mode):
         return q
     _scaled_case(mode, 1.0, 1.0, spike)
     _scaled_case(mode, 2.0 ** 20, 8.0, lambda q: q * 2.0 ** -20)
+
+
+SPARSITY_ATOL = 2e-5
+
+
+@pytest.mark.parametrize("G,ctx,n_protect", [(4, 2000, 128), (8, 709, 4), (1, 3000, 0)])
+def test_attention_sparsity_statistic(G, ctx, n_protect):
+    """tkv_decode_attention_sparsity: the step's output and scores as in a plain decode
+    call, plus per (stream, head) 1 - H(p) / ln N against the oracle's fp64 value and
+    the thought class under the thresholds (ThinKV, Metodologia: thought types differ in
+    the sparsity of their attention)."""
+    rows = [0, 1]
+    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", rows=rows, B=2, Hq=2 * G, Hkv=2, ctx=ctx, n_protect=n_protect,
+                                 steps=2, dense=True, attn_kernel=1)
+    k, v, cls, pos, q = synth.decode_inputs(w, 0)
+    sub = rows_streams(gpu, rows)
+    o.load_state(gpu.export_state(sub))
+    gpu.quantize_append(k.to(DEV), v.to(DEV), cls.to(DEV), pos.to(DEV))
+    assert o.append(np_bits(k[rows]), np_bits(v[rows]), cls[rows].numpy(), pos[rows].numpy()) == 0
+    ref_sp = o.attention_sparsity(np_bits(q[rows]), SCALE).reshape(len(rows), -1)
+    th_r, th_t = float(np.quantile(ref_sp, 0.3)), float(np.quantile(ref_sp, 0.7))
+    out, sp, thought = gpu.decode_attention_sparsity(q.to(DEV), SCALE, th_r, th_t)
+    ref = o.attend(np_bits(q[rows]), SCALE)
+    assert float(np.max(np.abs(out[rows].cpu().numpy() - ref))) <= OUT_ATOL
+    compare_states(gpu.export_state(sub), o.state, scores="tol", what="sparsity step")
+    got = sp[rows].cpu().numpy().astype(np.float64)
+    assert float(np.max(np.abs(got - ref_sp))) <= SPARSITY_ATOL
+    th = thought[rows].cpu().numpy()
+    for i in np.ndindex(ref_sp.shape):
+        near = min(abs(ref_sp[i] - th_r), abs(ref_sp[i] - th_t)) <= SPARSITY_ATOL
+        if not near:
+            assert th[i] == orc.classify_sparsity(ref_sp[i], th_r, th_t), i
+    assert gpu.poll_error() == tkv.TKV_OK
+
+
+def test_attention_sparsity_needs_the_tensor_core_kernel():
+    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", B=1, dense=True)
+    q = synth.decode_inputs(w, 0)[4].to(DEV)
+    with pytest.raises(TkvError):
+        gpu.decode_attention_sparsity(q, SCALE)
+    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", B=1, dense=True, attn_kernel=1)
+    q = synth.decode_inputs(w, 0)[4].to(DEV)
+    with pytest.raises(TkvError):
+        gpu.decode_attention_sparsity(q, SCALE, 0.8, 0.2)   # th_r > th_t

@@ -12,7 +12,7 @@ import synth
 from oracle import oracle as orc
 from reasoning_model_kv_b200 import TkvCache, TkvError, tkv
 from tests.conftest import gpu_available
-from tests.gpu_harness import build_pair, compare_states, oracle_for, rows_streams
+from tests.gpu_harness import MODES, build_pair, compare_states, oracle_for, rows_streams
 from tests.test_gpu_parity import _assert_dense, _decode_step
 
 pytestmark = [pytest.mark.gpu,
@@ -56,12 +56,12 @@ def _transition_starts(w, lo, hi):
     return sorted(out)
 
 
-@pytest.mark.parametrize("dense", [False, True], ids=["reuse", "dense"])
-def test_small_decode_loop_with_segment_eviction_at_every_transition(dense):
+@pytest.mark.parametrize("mode", list(MODES))
+def test_small_decode_loop_with_segment_eviction_at_every_transition(mode):
     """4 rows x 8/2 heads, 2k prefill, 800 decode steps (R/E/T 0.25/0.25/0.5);
     whenever a row starts a Transition segment the schedule is applied (lock-step
     state check), and the decode step that follows is checked against the oracle."""
-    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", B=4, steps=800, p_r=0.25, p_e=0.25, dense=dense)
+    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", B=4, steps=800, p_r=0.25, p_e=0.25, **MODES[mode])
     ctx = w["ctx"]
     _tbe_lockstep(w, gpu, o, rows, ctx - 1)            # after the prefill (scores all 0)
     _decode_step(w, gpu, o, rows, 0)
@@ -81,19 +81,19 @@ def test_small_decode_loop_with_segment_eviction_at_every_transition(dense):
             if step % 50 == 0:
                 o.load_state(gpu.export_state(rows_streams(gpu, rows)))
     assert checked >= 3
-    if dense:
+    if MODES[mode]["dense"]:
         _assert_dense(gpu)
     assert gpu.poll_error() == tkv.TKV_OK
 
 
-@pytest.mark.parametrize("dense", [False, True], ids=["reuse", "dense"])
-def test_b8_ctx16k_segment_eviction_sampled_row(dense):
+@pytest.mark.parametrize("mode", list(MODES))
+def test_b8_ctx16k_segment_eviction_sampled_row(mode):
     """Batch 8 x 32/8 heads, 16k prefill and a scoring step, then the schedule at the
     first transitions of the decode loop; lock-step on row 3 (about 110 segments,
     most R/E segments cut to 64/32/16 at the first call)."""
     rows = [3]
     w = synth.prefill_inputs("b8_ctx16k_256steps", device=DEV)
-    gpu = TkvCache(w["B"], w["Hkv"], w["G"], w["cap"], w["n_protect"], max_append=w["ctx"], dense=dense)
+    gpu = TkvCache(w["B"], w["Hkv"], w["G"], w["cap"], w["n_protect"], max_append=w["ctx"], **MODES[mode])
     gpu.quantize_append(w["k"], w["v"], w["cls"][:, :w["ctx"]].contiguous().to(DEV), w["pos"].to(DEV))
     o = oracle_for(gpu, gpu.export_state(rows_streams(gpu, rows)), B=1)
     trig = _transition_starts(w, w["ctx"], w["ctx"] + w["steps"])
@@ -111,17 +111,17 @@ def test_b8_ctx16k_segment_eviction_sampled_row(dense):
             gpu.decode_attention(q, SCALE)
     assert done >= 1
     assert gpu.export_state()["n"].sum() < before      # the schedule did evict
-    if dense:
+    if MODES[mode]["dense"]:
         _assert_dense(gpu)
     assert gpu.poll_error() == tkv.TKV_OK
 
 
-@pytest.mark.parametrize("dense", [False, True], ids=["reuse", "dense"])
-def test_segment_edge_cases(dense):
+@pytest.mark.parametrize("mode", list(MODES))
+def test_segment_edge_cases(mode):
     """Retention 0 and whole-segment keeps, segments starting inside the protected
     window (those tokens are bf16, foreign to the segment's label: kept), a row
     with no segments, and a call with no segment columns (no-op)."""
-    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", B=2, dense=dense, n_protect=100)
+    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", B=2, **MODES[mode], n_protect=100)
     _decode_step(w, gpu, o, rows, 0)
     ctx = w["ctx"]
     st, lb, ns = synth.segment_table(w["seed"], w["B"], ctx, w["p_r"], w["p_e"])
@@ -164,13 +164,13 @@ def _tam_lockstep(w, gpu, o, rows, upto, budget, c):
     assert gpu.poll_error() == tkv.TKV_OK
 
 
-@pytest.mark.parametrize("dense", [False, True], ids=["reuse", "dense"])
-def test_periodic_tam_small(dense):
+@pytest.mark.parametrize("mode", list(MODES))
+def test_periodic_tam_small(mode):
     """4 rows x 8/2 heads, 2k prefill; every 64 decode steps the thought-aware
     budgets (512 per stream, pivotal above 3x the mean score) are applied and
     checked against the oracle, three times (the page's periodic compaction), with
     a checked decode step after each."""
-    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", B=4, steps=200, dense=dense)
+    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", B=4, steps=200, **MODES[mode])
     ctx = w["ctx"]
     for step in range(w["steps"]):
         if step in (64, 128, 192):
@@ -180,18 +180,18 @@ def test_periodic_tam_small(dense):
             k, v, cls, pos, q = synth.decode_inputs(w, step, device=DEV)
             gpu.quantize_append(k, v, cls, pos)
             gpu.decode_attention(q, SCALE)
-    if dense:
+    if MODES[mode]["dense"]:
         _assert_dense(gpu)
     assert gpu.poll_error() == tkv.TKV_OK
 
 
-@pytest.mark.parametrize("dense", [False, True], ids=["reuse", "dense"])
-def test_b8_ctx16k_tam_sampled_row(dense):
+@pytest.mark.parametrize("mode", list(MODES))
+def test_b8_ctx16k_tam_sampled_row(mode):
     """Batch 8 x 32/8 heads, 16k prefill, 16 decode steps for scores, then budgets of
     1638 per stream with pivotal tokens above 4x the mean; lock-step on row 6."""
     rows = [6]
     w = synth.prefill_inputs("b8_ctx16k_256steps", device=DEV)
-    gpu = TkvCache(w["B"], w["Hkv"], w["G"], w["cap"], w["n_protect"], max_append=w["ctx"], dense=dense)
+    gpu = TkvCache(w["B"], w["Hkv"], w["G"], w["cap"], w["n_protect"], max_append=w["ctx"], **MODES[mode])
     gpu.quantize_append(w["k"], w["v"], w["cls"][:, :w["ctx"]].contiguous().to(DEV), w["pos"].to(DEV))
     for step in range(16):
         k, v, cls, pos, q = synth.decode_inputs(w, step, device=DEV)
@@ -202,16 +202,16 @@ def test_b8_ctx16k_tam_sampled_row(dense):
     _tam_lockstep(w, gpu, o, rows, w["ctx"] + 15, w["budget"], 4.0)
     assert gpu.export_state()["n"].sum() < before
     _decode_step(w, gpu, o, rows, 16)
-    if dense:
+    if MODES[mode]["dense"]:
         _assert_dense(gpu)
     assert gpu.poll_error() == tkv.TKV_OK
 
 
-@pytest.mark.parametrize("dense", [False, True], ids=["reuse", "dense"])
-def test_tam_degenerate_cases(dense):
+@pytest.mark.parametrize("mode", list(MODES))
+def test_tam_degenerate_cases(mode):
     """c = 0 makes every candidate pivotal (nothing leaves); budget 0 with no pivotal
     token keeps only protected, foreign and unsegmented entries."""
-    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", B=2, dense=dense, n_protect=100)
+    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", B=2, **MODES[mode], n_protect=100)
     _decode_step(w, gpu, o, rows, 0)
     before = gpu.export_state()
     st, lb, ns = synth.segment_table(w["seed"], w["B"], w["ctx"], w["p_r"], w["p_e"])
@@ -224,3 +224,21 @@ def test_tam_degenerate_cases(dense):
     g = gpu.export_state()
     assert g["n"][:, 1:].sum() == 0                     # every R/E/T candidate left
     assert (g["n"][:, 0] == 100).all()                  # the bf16 window stays
+
+
+@pytest.mark.parametrize("mode", list(MODES))
+def test_tam_wide_scores_bit_exact(mode):
+    """Scores spread over 2^-40 .. 2^30: fp64 sums taken in different orders would round
+    differently here; the exact sums make the budgets, and so the kept sets, bit-exact
+    with the oracle (both sides start from the same state)."""
+    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", B=2, **MODES[mode])
+    _decode_step(w, gpu, o, rows, 0)
+    state = gpu.export_state()
+    rng = np.random.default_rng(77)
+    for c in range(4):
+        sc = state[f"score{c}"]
+        sc[...] = np.ldexp(rng.random(sc.shape) + 0.5, rng.integers(-40, 31, sc.shape)).astype(np.float32)
+    gpu.import_state(state)
+    for budget, c in ((300, 2.0), (120, 0.7), (700, 5.0)):
+        _tam_lockstep(w, gpu, o, rows, w["ctx"], budget, c)
+    assert gpu.poll_error() == tkv.TKV_OK
