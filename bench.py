@@ -64,6 +64,9 @@ def parse():
                          "over the rows' thought segments, r0 64, t_keep 16) or tam (the budget "
                          "split over segments in proportion to sqrt(mean score) x length, "
                          "tokens above 3x the mean score kept)")
+    ap.add_argument("--codec", choices=["int", "fp"], default="int",
+                    help="class record formats: int (8/4/2-bit integer codes) or fp (FP8 E4M3 / NVFP4 / "
+                         "ternary; warp-tile kernel)")
     ap.add_argument("--full-reps", type=int, default=3,
                     help="timed attention calls on the full prefill context before the eviction "
                          "(the full-context phase; 0 skips it)")
@@ -171,8 +174,8 @@ def reduce_max(vals, world: int, device) -> list:
     return t.tolist()
 
 
-def packed_bytes(n: np.ndarray) -> int:
-    return int(sum(int(n[:, c].sum()) * REC_BYTES[c] for c in range(4)))
+def packed_bytes(n: np.ndarray, rec=REC_BYTES) -> int:
+    return int(sum(int(n[:, c].sum()) * rec[c] for c in range(4)))
 
 
 # ----------------------------------------------------------------------------
@@ -189,14 +192,14 @@ def segment_inputs(w, dev, upto):
             torch.from_numpy(ns).to(dev))
 
 
-def setup_cache(w, dev, dense, evict_reps, flush, attn_kernel=0, evict="topk", full_reps=0):
+def setup_cache(w, dev, dense, evict_reps, flush, attn_kernel=0, evict="topk", full_reps=0, codec=0):
     """Prefill, one scoring step, then the eviction (to the budget, or the TBE
     schedule at the scoring step's position).  The eviction is timed (CUDA events,
     L2 flushed) over `evict_reps` repetitions, each from a copy of the pre-eviction
     workspace; it is not part of the timed decode step."""
     from reasoning_model_kv_b200 import TkvCache
     gpu = TkvCache(w["B"], w["Hkv"], w["G"], w["cap"], w["n_protect"], max_append=w["ctx"], dense=dense,
-                   attn_kernel=attn_kernel)
+                   attn_kernel=attn_kernel, codec=codec)
     cls = w["cls"][:, :w["ctx"]].contiguous().to(dev)
     gpu.quantize_append(w["k"], w["v"], cls, w["pos"].to(dev))
     k, v, c, p, q = synth.decode_inputs(w, 0, device=dev)        # untimed scoring step
@@ -221,7 +224,7 @@ def setup_cache(w, dev, dense, evict_reps, flush, attn_kernel=0, evict="topk", f
             if i > 0:
                 ms.append(a.elapsed_time(b2))
         t = sum(ms) / len(ms)
-        pkf = packed_bytes(n_full)
+        pkf = packed_bytes(n_full, list(gpu.layout.rec_bytes))
         full = {"live_kv_tokens": int(n_full.sum()), "packed_kv_bytes": pkf, "attention_ms": t,
                 "hbm_gbs_packed": pkf / (t * 1e-3) / 1e9, "kv_tokens_per_s": int(n_full.sum()) / (t * 1e-3),
                 "reps": full_reps}
@@ -258,7 +261,7 @@ def run_tkv(args, rank, world, dev):
     flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
     gpu, evict_ms, full = setup_cache(w, dev, args.placement == "dense", args.evict_reps, flush,
                                       attn_kernel=1 if args.attn_kernel == "tc" else 0, evict=args.evict,
-                                      full_reps=args.full_reps)
+                                      full_reps=args.full_reps, codec=1 if args.codec == "fp" else 0)
     del w["k"], w["v"]
     torch.cuda.empty_cache()
     views = gpu.state_views()
@@ -279,7 +282,7 @@ def run_tkv(args, rank, world, dev):
     step()
     torch.cuda.synchronize()
     n_after = views["n"].cpu().numpy()
-    pk = packed_bytes(n_after)
+    pk = packed_bytes(n_after, list(gpu.layout.rec_bytes))
     kv_tokens = int(n_after.sum())
     saved_post = {key: views[key].clone() for key in ("n", "ft", "hw")}
 
@@ -391,7 +394,7 @@ def run_tkv(args, rank, world, dev):
                    # placement also reads each entry's slot handle (4 B)
                    "total_bytes_per_step": pk + kv_tokens * (8 + (0 if args.placement == "dense" else 4))
                    + q.numel() * q.element_size() + out.numel() * out.element_size(),
-                   "placement": args.placement, "attn_kernel": args.attn_kernel,
+                   "placement": args.placement, "attn_kernel": args.attn_kernel, "codec": args.codec,
                    "eviction": {"topk": f"topk, budget {w['budget']} per stream",
                                 "tbe": "tbe segment schedule at the scoring step (r0 64, t_keep 16)",
                                 "tam": f"tam segment budgets, {w['budget']} per stream, pivotal above 3x "

@@ -202,7 +202,8 @@ struct Counts {
     int n[4];
 };
 
-__device__ __forceinline__ int ntiles(int n, int c) { return (n + rows_of(c) - 1) / rows_of(c); }
+// tiles of class c holding n records (64-row bf16 tiles, 128-row code tiles)
+__device__ __forceinline__ int ntiles(int n, int c) { return c == 0 ? (n + 63) >> 6 : (n + 127) >> 7; }
 __device__ __forceinline__ unsigned long long class_cost(int n, int c) {
     return (unsigned long long)n * rec_of(c) + (unsigned long long)ntiles(n, c) * kTileOverhead;
 }
@@ -249,94 +250,89 @@ struct Tile {
     bool last;      // last tile of the stream
 };
 
-// Iterator over the tiles a CTA owns (the same sequence in every role).
+// Iterator over the tiles a CTA owns.  The current stream's counts live in scalars
+// (no indexed register arrays, which would go to local memory) and each step costs a
+// few integer operations: the iterator runs on a single producer thread whose every
+// instruction is on the tile pipeline's critical path.
+__device__ __forceinline__ int pick(int c, int a0, int a1, int a2, int a3) {
+    return c == 0 ? a0 : c == 1 ? a1 : c == 2 ? a2 : a3;
+}
 struct TileIter {
-    int s, c, j;
-    Counts k;
-    unsigned long long sbase, cbase, start, cend;
-    int S;
+    int S, s, c, j;
+    int n0, n1, n2, n3, mask;        // the stream's counts, classes holding records (bit c)
+    int n, nt, oc;                   // current class: records, tiles, entries before it
+    unsigned long long start, cend, cls_end, full;   // costs: current tile, share end, class end, per tile
 
     __device__ __forceinline__ void load(const Dev &d, const SharedPlan &pl, int stream) {
         const int i = stream - pl.s0;
         if (i >= 0 && i < pl.nst) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) k.n[q] = pl.cnt[i][q];
+            n0 = pl.cnt[i][0]; n1 = pl.cnt[i][1]; n2 = pl.cnt[i][2]; n3 = pl.cnt[i][3];
         } else {
-            k = load_counts(d, stream);
+            const Counts k = load_counts(d, stream);
+            n0 = k.n[0]; n1 = k.n[1]; n2 = k.n[2]; n3 = k.n[3];
         }
+        mask = (n0 > 0) | ((n1 > 0) << 1) | ((n2 > 0) << 2) | ((n3 > 0) << 3);
     }
-    // first class >= c0 with entries, 4 if none; cbase advanced over skipped classes
-    __device__ __forceinline__ int next_class(int c0) {
-        int cc = c0;
-        while (cc < 4 && k.n[cc] == 0) ++cc;
-        return cc;
+    // enter class cc of the current stream; its region starts at cost `at`
+    __device__ __forceinline__ void enter(int cc, unsigned long long at) {
+        c = cc;
+        n = pick(cc, n0, n1, n2, n3);
+        nt = ntiles(n, cc);
+        oc = pick(cc, 0, n0, n0 + n1, n0 + n1 + n2);
+        full = tile_cost_full(cc);
+        start = at;
+        cls_end = at + class_cost(n, cc);
+        j = 0;
     }
-    __device__ __forceinline__ bool valid() const { return s < S && start < cend; }
-    __device__ __forceinline__ void settle(const Dev &d, const SharedPlan &pl) {
-        // move to the next tile that exists (possibly in a later stream)
-        while (s < S) {
-            if (c < 4 && j < ntiles(k.n[c], c)) {
-                start = cbase + (unsigned long long)j * tile_cost_full(c);
-                return;
-            }
-            if (c < 4) {
-                cbase += class_cost(k.n[c], c);
-                c = next_class(c + 1);
-                j = 0;
-                continue;
-            }
-            sbase += stream_cost(k);
-            ++s;
-            if (s >= S) break;
+    // first class of the next stream holding records (streams without records cost 0)
+    __device__ __forceinline__ void next_stream(const Dev &d, const SharedPlan &pl, unsigned long long at) {
+        for (++s; s < S; ++s) {
             load(d, pl, s);
-            c = next_class(0);
-            cbase = sbase;
-            j = 0;
+            if (mask) { enter(__ffs(mask) - 1, at); return; }
         }
         start = ~0ull;
     }
+    __device__ __forceinline__ bool valid() const { return s < S && start < cend; }
     __device__ __forceinline__ void begin(const Dev &d, const SharedPlan &pl) {
         S = d.S;
         cend = pl.cend;
         s = pl.s0;
-        if (s >= S) { start = ~0ull; return; }
+        start = ~0ull;
+        if (s >= S) return;
         load(d, pl, s);
-        sbase = pl.p0;
-        cbase = sbase;
-        c = next_class(0);
-        j = 0;
+        if (!mask) { next_stream(d, pl, pl.p0); return; }
+        enter(__ffs(mask) - 1, pl.p0);
         // skip the tiles of s0 that start before cstart
-        while (c < 4) {
-            const unsigned long long span = class_cost(k.n[c], c);
-            if (cbase + span <= pl.cstart) {
-                cbase += span;
-                c = next_class(c + 1);
-                continue;
-            }
-            const unsigned long long full = tile_cost_full(c);
-            j = pl.cstart > cbase ? (int)((pl.cstart - cbase + full - 1) / full) : 0;
-            break;
+        while (cls_end <= pl.cstart) {
+            const int rest = mask & ~((2 << c) - 1);
+            if (!rest) { next_stream(d, pl, cls_end); return; }
+            enter(__ffs(rest) - 1, cls_end);
         }
-        settle(d, pl);
+        if (pl.cstart > start) {
+            j = (int)((pl.cstart - start + full - 1) / full);
+            start += (unsigned long long)j * full;
+            if (j >= nt) advance_class(d, pl);
+        }
+    }
+    __device__ __forceinline__ void advance_class(const Dev &d, const SharedPlan &pl) {
+        const int rest = mask & ~((2 << c) - 1);
+        if (rest) enter(__ffs(rest) - 1, cls_end);
+        else next_stream(d, pl, cls_end);
     }
     __device__ __forceinline__ void advance(const Dev &d, const SharedPlan &pl) {
         ++j;
-        settle(d, pl);
+        start += full;
+        if (j >= nt) advance_class(d, pl);
     }
     __device__ __forceinline__ Tile tile() const {
         Tile t;
         t.s = s;
         t.c = c;
-        t.e = j * rows_of(c);
-        t.nr = min(rows_of(c), k.n[c] - t.e);
-        t.oc = 0;
-        for (int q = 0; q < c; ++q) t.oc += k.n[q];
-        int cf = 0;
-        while (cf < 4 && k.n[cf] == 0) ++cf;
-        int cl = 3;
-        while (cl >= 0 && k.n[cl] == 0) --cl;
-        t.first = (c == cf && j == 0);
-        t.last = (c == cl && j == ntiles(k.n[c], c) - 1);
+        t.e = j << (c == 0 ? 6 : 7);
+        t.nr = min(c == 0 ? 64 : 128, n - t.e);
+        t.oc = oc;
+        t.first = j == 0 && c == __ffs(mask) - 1;
+        t.last = j == nt - 1 && c == 31 - __clz(mask);
         return t;
     }
 };
@@ -578,6 +574,16 @@ __device__ __forceinline__ bool wg_any(int id, bool pred) {   // OR of pred over
     return r != 0;
 }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+// Non-blocking probe of phase `parity` of a barrier.
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile("{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(done)
+                 : "r"(bar), "r"(parity)
+                 : "memory");
+    return done != 0;
+}
 
 template <int N>
 __device__ __forceinline__ void tmem_ldn(uint32_t taddr, uint32_t *r) {
@@ -661,17 +667,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t pol = policy_evict_first();
             TileIter it;
             it.begin(d, pl);
-            int last_copy[R];
-            bool landed[R];
-#pragma unroll
-            for (int i = 0; i < R; ++i) { last_copy[i] = -1; landed[i] = true; }
-            int k = 0;
+            uint32_t pending = 0;   // bit i: stage i holds a copy not yet seen consumed
+            int k = 0, ncopied = 0; // tiles copied: stage i last received tile ncopied-1-((ncopied-1-i) mod R)
             for (; ok; ++k) {
                 const int slot = k % R;
                 if (k >= R) {
                     ok = mbar_wait_sleep(smem_addr(&bar_raw_empty[slot]), (uint32_t)((k / R - 1) & 1));
                     if (!ok) break;
-                    landed[slot] = true;   // its previous copy was consumed
+                    pending &= ~(1u << slot);   // its previous copy was consumed
                 }
                 if (!it.valid()) break;
                 const Tile t = it.tile();
@@ -697,8 +700,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int j = 0; j < nb; ++j)
                         tma_load_2d(bdst + (uint32_t)(j * 16 * wbytes), mp, x, y0 + 16 * j, bar, pol);
                 }
-                last_copy[slot] = k;
-                landed[slot] = false;
+                pending |= 1u << slot;
+                ncopied = k + 1;
                 it.advance(d, pl);
             }
             // "no more tiles" for the next tile of each warpgroup (slot free: waited above or unused)
@@ -708,7 +711,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (u == 1 && kk >= R) {
                         ok = mbar_wait_sleep(smem_addr(&bar_raw_empty[slot]), (uint32_t)((kk / R - 1) & 1));
                         if (!ok) break;
-                        landed[slot] = true;
+                        pending &= ~(1u << slot);
                     }
                     TileDesc td;
                     td.s = -1; td.e = 0; td.oc = 0; td.meta = 1u << 31;
@@ -718,73 +721,97 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             // every copy still unconsumed lands before the CTA may exit (each slot holds at most one)
             for (int i = 0; i < R; ++i) {
-                if (landed[i] || last_copy[i] < 0) continue;
-                if (!mbar_wait_sleep(smem_addr(&bar_raw_full[i]), (uint32_t)((last_copy[i] / R) & 1))) ok = false;
+                if (!((pending >> i) & 1u)) continue;
+                const int kl = ncopied - 1 - ((ncopied - 1 - i) % R);   // >= 0: stage i received a copy
+                if (!mbar_wait_sleep(smem_addr(&bar_raw_full[i]), (uint32_t)((kl / R) & 1))) ok = false;
             }
         }
     } else if (warp == 1) {
         // ================================================= MMA issuer
+        // Two independent in-order streams: QK(kq) once its warpgroup has the tile ready,
+        // PV(kpv) once that warpgroup has written W; whichever is ready is issued, so
+        // neither warpgroup waits on the other's progress.  QK(k) always precedes PV(k)
+        // (W needs the logits).  Descriptors stay in the ring until the tile's PV is
+        // issued (the producer reuses a ring slot only 16 tiles later, after the PV of
+        // an even later tile).
         if (lane == 0) {
-            int k = 0;
-            TileDesc prev;
-            prev.meta = 0;
-            auto issue_pv = [&](int kp, const TileDesc &tp) {
-                const int wg = kp & 1, cp = td_c(tp);
-                ok = mbar_wait_sleep(smem_addr(&bar_w_full[wg]), (uint32_t)((kp >> 1) & 1));
-                if (!ok) return;
-                tc_fence_after();
-                const uint32_t raw = smb + kOffRaw + (kp % R) * kRawBytes;
-                const uint32_t stg = smb + off_stg(G) + wg * kStgV;
-                const uint32_t bw = smb + off_w(G) + wg * w_bytes(G);
-                const uint32_t dcol = tb + col_o(wg);
-                if (cp == 0) {
+            // descriptor templates (start address 0): a descriptor is template | (address >> 4)
+            const uint64_t dA = sdesc(0, 16, 1024, kSw128);     // tiles and staged values, 128B swizzle
+            const uint64_t dVb = sdesc(0, 8192, 1024, kSw128);  // staged bf16 values (two 64-dim atoms)
+            const uint64_t dQi = sdesc(0, NS * 16, 128);        // query digits
+            const uint64_t dQb = sdesc(0, 256, 128);            // bf16 query
+            const uint64_t dWi = sdesc(0, 128, 2048);           // W, integer columns
+            const uint64_t dWb = sdesc(0, 128, 1024);           // W, bf16 columns
+            auto at = [](uint64_t t, uint32_t addr) { return t | (uint64_t)(addr >> 4); };
+            int kq = 0, kpv = 0;
+            bool q_done = false;
+            long long t_idle = 0;
+            while (ok) {
+                bool progress = false;
+                if (!q_done && mbar_test(smem_addr(&bar_kready[kq & 1]), (uint32_t)((kq >> 1) & 1))) {
+                    const TileDesc td = desc[kq % kDescRing];
+                    progress = true;
+                    if (td_end(td)) {
+                        q_done = true;
+                    } else {
+                        tc_fence_after();
+                        const int wg = kq & 1, tc = td_c(td);
+                        const uint32_t raw = smb + kOffRaw + (kq % R) * kRawBytes;
+                        const uint32_t qb = smb + off_q(G) + wg * q_bytes(G);
+                        const uint32_t dcol = tb + col_s(wg);
+                        if (tc == 0) {
+                            const uint32_t bq = qb + qi8_bytes(G);
 #pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_f16(dcol, sdesc(stg + ks * 2048, 8192, 1024, kSw128), sdesc(bw + ks * 256, 128, 1024),
-                                idesc(1, 1, 1, 1, 1, 16), ks > 0);
-                } else {
-                    const uint32_t av = cp == 1 ? raw + v_off(1) : stg;
+                            for (int ks = 0; ks < 8; ++ks)
+                                mma_f16(dcol, at(dA, raw + (ks >> 2) * 8192 + (ks & 3) * 32), at(dQb, bq + ks * 512),
+                                        idesc(1, 1, 1, 0, 0, 16), ks > 0);
+                        } else if (tc == 1) {
 #pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_i8(dcol, sdesc(av + ks * 4096, 16, 1024, kSw128), sdesc(bw + ks * 512, 128, 2048),
-                               idesc(2, 0, 0, 1, 1, NO), ks > 0);
+                            for (int ks = 0; ks < 4; ++ks)
+                                mma_i8(dcol, at(dA, raw + ks * 32), at(dQi, qb + ks * 32 * NS), idesc(2, 0, 1, 0, 0, NS), ks > 0);
+                        } else {
+#pragma unroll
+                            for (int ks = 0; ks < 4; ++ks)
+                                mma_i8_tmem(dcol, tb + col_a(wg) + 8 * ks, at(dQi, qb + ks * 32 * NS), idesc(2, 0, 1, 0, 0, NS),
+                                            ks > 0);
+                        }
+                        mma_commit(smem_addr(&bar_s_full[wg]));
+                        ++kq;
+                    }
                 }
-                mma_commit(smem_addr(&bar_o_full[wg]));
-                mma_commit(smem_addr(&bar_raw_empty[kp % R]));
-            };
-            for (; ok; ++k) {
-                const int wg = k & 1;
-                ok = mbar_wait_sleep(smem_addr(&bar_kready[wg]), (uint32_t)((k >> 1) & 1));
-                if (!ok) break;
-                const TileDesc td = desc[k % kDescRing];
-                if (td_end(td)) break;
-                tc_fence_after();
-                const int tc = td_c(td);
-                const uint32_t raw = smb + kOffRaw + (k % R) * kRawBytes;
-                const uint32_t qb = smb + off_q(G) + wg * q_bytes(G);
-                const uint32_t dcol = tb + col_s(wg);
-                if (tc == 0) {
-                    const uint32_t bq = qb + qi8_bytes(G);
+                if (kpv < kq && mbar_test(smem_addr(&bar_w_full[kpv & 1]), (uint32_t)((kpv >> 1) & 1))) {
+                    tc_fence_after();
+                    const TileDesc tp = desc[kpv % kDescRing];
+                    const int wg = kpv & 1, cp = td_c(tp);
+                    const uint32_t raw = smb + kOffRaw + (kpv % R) * kRawBytes;
+                    const uint32_t stg = smb + off_stg(G) + wg * kStgV;
+                    const uint32_t bw = smb + off_w(G) + wg * w_bytes(G);
+                    const uint32_t dcol = tb + col_o(wg);
+                    if (cp == 0) {
 #pragma unroll
-                    for (int ks = 0; ks < 8; ++ks)
-                        mma_f16(dcol, sdesc(raw + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kSw128),
-                                sdesc(bq + ks * 512, 256, 128), idesc(1, 1, 1, 0, 0, 16), ks > 0);
-                } else if (tc == 1) {
+                        for (int ks = 0; ks < 4; ++ks)
+                            mma_f16(dcol, at(dVb, stg + ks * 2048), at(dWb, bw + ks * 256), idesc(1, 1, 1, 1, 1, 16), ks > 0);
+                    } else {
+                        const uint32_t av = cp == 1 ? raw + v_off(1) : stg;
 #pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_i8(dcol, sdesc(raw + ks * 32, 16, 1024, kSw128), sdesc(qb + ks * 32 * NS, NS * 16, 128),
-                               idesc(2, 0, 1, 0, 0, NS), ks > 0);
-                } else {
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_i8_tmem(dcol, tb + col_a(wg) + 8 * ks, sdesc(qb + ks * 32 * NS, NS * 16, 128),
-                                    idesc(2, 0, 1, 0, 0, NS), ks > 0);
+                        for (int ks = 0; ks < 4; ++ks)
+                            mma_i8(dcol, at(dA, av + ks * 4096), at(dWi, bw + ks * 512), idesc(2, 0, 0, 1, 1, NO), ks > 0);
+                    }
+                    mma_commit(smem_addr(&bar_o_full[wg]));
+                    mma_commit(smem_addr(&bar_raw_empty[kpv % R]));
+                    ++kpv;
+                    progress = true;
                 }
-                mma_commit(smem_addr(&bar_s_full[wg]));
-                if (k > 0) issue_pv(k - 1, prev);
-                prev = td;
+                if (q_done && kpv == kq) break;
+                if (progress) {
+                    t_idle = 0;
+                } else {
+                    // bounded: a second without a ready operand is a timeout
+                    const long long now = clock64();
+                    if (t_idle == 0) t_idle = now;
+                    else if (now - t_idle > kWaitCycles) ok = false;
+                }
             }
-            if (ok && k > 0) issue_pv(k - 1, prev);
             // every MMA issued has completed before tensor memory is released
             mma_commit(smem_addr(&bar_mma_done));
             if (!mbar_wait_sleep(smem_addr(&bar_mma_done), 0u)) ok = false;
@@ -916,9 +943,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint16_t *qrow =
                     reinterpret_cast<const uint16_t *>(q) + ((size_t)bb * d.Hkv * G + (size_t)kvh * G) * kD;
                 const int kb = pos_kbf(r), m8 = pos_k8(r);
+                uint32_t qraw[G];
+#pragma unroll
+                for (int h = 0; h < G; ++h) qraw[h] = qrow[h * kD + r];   // every load in flight at once
 #pragma unroll
                 for (int h = 0; h < G; ++h) {
-                    const uint32_t bits = qrow[h * kD + r];
+                    const uint32_t bits = qraw[h];
                     *reinterpret_cast<uint16_t *>(qbuf + qi8_bytes(G) + (kb / 8) * 256 + (h / 8) * 128 + (h % 8) * 16 +
                                                   (kb % 8) * 2) = (uint16_t)bits;
                     // digits: q = v * 2^(Emax - 146) with v = m * 2^(e - Emax + 12) (rounded)
@@ -969,15 +999,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (td_last(td)) d.seg_hi[td.s] = cta;
             }
 
-            // ---- O of the previous own tile; the segment's partial when the stream changes
-            if (kp >= 0) {
+            // ---- O of the previous own tile: at a stream change now (the segment's partial
+            //      is written); otherwise after this tile's logits, so that the PV of the
+            //      previous tile runs meanwhile.  Its values (staged) and W must be read
+            //      before this tile overwrites them.
+            const bool o_late = kp >= 0 && !newseg;
+            if (kp >= 0 && newseg) {
                 o_accumulate(kp, c_prev);
-                if (newseg) {
-                    flush(cur_s);
+                flush(cur_s);
 #pragma unroll
-                    for (int h = 0; h < G; ++h) oacc[h] = 0.f;
-                }
+                for (int h = 0; h < G; ++h) oacc[h] = 0.f;
             }
+            if (o_late && tcls != 1 && ok)
+                ok = mbar_wait_sleep(smem_addr(&bar_o_full[wg]), (uint32_t)((kp >> 1) & 1));
             if (newseg) {
                 cur_s = td.s;
 #pragma unroll
@@ -1103,6 +1137,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 l[h] += p[h];
                 if (STATS) e[h] = fmaf(p[h], valid ? x[h] - m[h] : 0.f, e[h]);
             }
+            if (o_late) o_accumulate(kp, c_prev);
             // ---- W (the B operand of PV) for row r
             float bp_cur[G], bv_cur = 1.f;
             if (tcls == 0) {
@@ -1216,8 +1251,10 @@ __global__ void __launch_bounds__(256) attn_finalize_kernel(const __grid_constan
                                                             float *__restrict__ sparsity,
                                                             uint8_t *__restrict__ thought, float th_r, float th_t,
                                                             int ncta) {
+    constexpr int kParts = 64;   // partials staged in shared memory (more are read from global)
     __shared__ float gM[kMaxG], gInvL[kMaxG], gH[kMaxG];
-    __shared__ float fac[64][kMaxG];
+    __shared__ float fac[kParts][kMaxG];
+    __shared__ float hm[kParts][kMaxG], hl[kParts][kMaxG], he[kParts][kMaxG];
     grid_dependency_wait();
     const int s = blockIdx.x, split = blockIdx.y, nsplit = gridDim.y;
     const int tid = threadIdx.x;
@@ -1242,20 +1279,30 @@ __global__ void __launch_bounds__(256) attn_finalize_kernel(const __grid_constan
     }
     const int nparts = 2 * (c_hi - c_lo + 1);
     const float *part0 = d.part + (size_t)2 * (s + c_lo) * part_floats(G);
+    // (m, l, e) of the first kParts partials, loaded by all threads at once
+    const int nstage = min(nparts, kParts);
+    for (int i = tid; i < nstage * G; i += 256) {
+        const int j = i / G, h = i - j * G;
+        const float *pp = part0 + (size_t)j * part_floats(G);
+        hm[j][h] = pp[h];
+        hl[j][h] = pp[G + h];
+        if (STATS) he[j][h] = pp[2 * G + h];
+    }
+    __syncthreads();
+    auto pm = [&](int j, int h) { return j < kParts ? hm[j][h] : part0[(size_t)j * part_floats(G) + h]; };
+    auto pl_ = [&](int j, int h) { return j < kParts ? hl[j][h] : part0[(size_t)j * part_floats(G) + G + h]; };
+    auto pe = [&](int j, int h) { return j < kParts ? he[j][h] : part0[(size_t)j * part_floats(G) + 2 * G + h]; };
     if (tid < G) {
         float M = kNoMax;
-        for (int j = 0; j < nparts; ++j) {
-            const float *pp = part0 + (size_t)j * part_floats(G);
-            if (pp[G + tid] > 0.f) M = fmaxf(M, pp[tid]);
-        }
+        for (int j = 0; j < nparts; ++j)
+            if (pl_(j, tid) > 0.f) M = fmaxf(M, pm(j, tid));
         float L = 0.f, E = 0.f;
         for (int j = 0; j < nparts; ++j) {
-            const float *pp = part0 + (size_t)j * part_floats(G);
-            const float lj = pp[G + tid];
-            const float f = lj > 0.f ? ex2(pp[tid] - M) : 0.f;
-            if (j < 64) fac[j][tid] = f;
+            const float lj = pl_(j, tid), mj = pm(j, tid);
+            const float f = lj > 0.f ? ex2(mj - M) : 0.f;
+            if (j < kParts) fac[j][tid] = f;
             L += f * lj;
-            if (STATS && lj > 0.f) E += f * (pp[2 * G + tid] + (pp[tid] - M) * lj);
+            if (STATS && lj > 0.f) E += f * (pe(j, tid) + (mj - M) * lj);
         }
         gM[tid] = M;
         gInvL[tid] = L > 0.f ? 1.f / L : 0.f;
@@ -1272,7 +1319,7 @@ __global__ void __launch_bounds__(256) attn_finalize_kernel(const __grid_constan
             float acc = 0.f;
             for (int j = 0; j < nparts; ++j) {
                 const float *pp = part0 + (size_t)j * part_floats(G);
-                const float f = j < 64 ? fac[j][h] : (pp[G + h] > 0.f ? ex2(pp[h] - gM[h]) : 0.f);
+                const float f = j < kParts ? fac[j][h] : (pp[G + h] > 0.f ? ex2(pp[h] - gM[h]) : 0.f);
                 if (f > 0.f) acc = fmaf(f, pp[3 * G + i], acc);
             }
             orow[i] = acc * gInvL[h];
