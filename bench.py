@@ -53,9 +53,10 @@ def parse():
     ap.add_argument("--placement", choices=["dense", "reuse"], default="dense",
                     help="record placement: dense (eviction moves kept records together, appends "
                          "go after them) or reuse (records stay put, evicted slots are reused)")
-    ap.add_argument("--attn-kernel", choices=["warp", "tc"], default="warp",
-                    help="decode-attention kernel: warp-tile mma.sync (default) or the tcgen05 "
-                         "tensor-memory kernel (dense placement only)")
+    ap.add_argument("--attn-kernel", choices=["warp", "tc", "ws"], default="warp",
+                    help="decode-attention kernel: warp-tile mma.sync (default), the tcgen05 "
+                         "tensor-memory kernel, or the warp-tile math on a persistent TMA pipeline "
+                         "(the last two: dense placement only)")
     ap.add_argument("--evict-reps", type=int, default=5,
                     help="timed repetitions of the eviction that precedes the timed step")
     ap.add_argument("--evict", choices=["topk", "tbe", "tam"], default="topk",
@@ -70,6 +71,11 @@ def parse():
     ap.add_argument("--full-reps", type=int, default=3,
                     help="timed attention calls on the full prefill context before the eviction "
                          "(the full-context phase; 0 skips it)")
+    ap.add_argument("--decode-loop", action="store_true",
+                    help="time the workload's whole decode loop instead of one step: every layer, "
+                         "every step (append + attention), the periodic eviction, CUDA events "
+                         "around each 64-step chunk (inputs are generated outside the timed chunks)")
+    ap.add_argument("--loop-steps", type=int, default=None, help="decode steps of --decode-loop (default: the workload's)")
     ap.add_argument("--ctx", type=int, default=None,
                     help="prefill context before the eviction (default: the workload's); the "
                          "timed step is the same post-eviction step, with smaller pools")
@@ -260,7 +266,7 @@ def run_tkv(args, rank, world, dev):
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
     gpu, evict_ms, full = setup_cache(w, dev, args.placement == "dense", args.evict_reps, flush,
-                                      attn_kernel=1 if args.attn_kernel == "tc" else 0, evict=args.evict,
+                                      attn_kernel={"warp": 0, "tc": 1, "ws": 2}[args.attn_kernel], evict=args.evict,
                                       full_reps=args.full_reps, codec=1 if args.codec == "fp" else 0)
     del w["k"], w["v"]
     torch.cuda.empty_cache()
@@ -509,6 +515,82 @@ def run_reference(args, rank, world):
             "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_loop(args, dev):
+    """The workload's decode loop on one GPU: prefill every layer's cache, then `steps`
+    decode steps of append + attention on every layer with the eviction to the budget
+    every `evict_every` steps (ThinKV / TAM periodic compaction).  Per 64-step chunk the
+    inputs are generated first (untimed), then the chunk runs between two CUDA events."""
+    from reasoning_model_kv_b200 import TkvCache
+    spec = synth.WORKLOADS[args.workload]
+    L, E = spec.get("layers", 1), spec["evict_every"]
+    steps = args.loop_steps or spec["steps"]
+    B, Hkv, Hq, D, ctx = spec["B"], spec["Hkv"], spec["Hq"], spec["D"], spec["ctx"]
+    kern = {"warp": 0, "tc": 1, "ws": 2}[args.attn_kernel]
+    caches, ws = [], []
+    t0 = time.time()
+    for layer in range(L):
+        w = synth.prefill_inputs(args.workload, layer=layer, device=dev, steps=steps)
+        g = TkvCache(w["B"], w["Hkv"], w["G"], w["cap"], w["n_protect"], max_append=w["ctx"],
+                     dense=args.placement == "dense", attn_kernel=kern, codec=1 if args.codec == "fp" else 0)
+        g.quantize_append(w["k"], w["v"], w["cls"][:, :w["ctx"]].contiguous().to(dev), w["pos"].to(dev))
+        del w["k"], w["v"]
+        caches.append(g)
+        ws.append(w)
+    torch.cuda.synchronize()
+    prefill_s = time.time() - t0
+    cls_dev = ws[0]["cls"][:, ctx:ctx + steps].contiguous().to(dev)
+    out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+    st = torch.cuda.current_stream()
+    chunk_ms, n_evict = [], 0
+    for c0 in range(0, steps, 64):
+        n = min(64, steps - c0)
+        chunk = []
+        for layer in range(L):
+            seed = ws[layer]["seed"]
+            k = synth.normal_bf16(seed, layer, synth.TID_K, B, Hkv, ctx + c0, n, D, dev)
+            if spec["outliers"]:
+                k = synth.apply_k_outliers(k, seed, layer)
+            v = synth.normal_bf16(seed, layer, synth.TID_V, B, Hkv, ctx + c0, n, D, dev)
+            q = synth.normal_bf16(seed, layer, synth.TID_Q, B, Hq, ctx + c0, n, D, dev)
+            chunk.append(([k[:, :, j:j + 1].contiguous() for j in range(n)], [v[:, :, j:j + 1].contiguous() for j in range(n)],
+                          [q[:, :, j].contiguous() for j in range(n)]))
+        pos = [torch.full((B, 1), ctx + c0 + j, dtype=torch.int32, device=dev) for j in range(n)]
+        cls = [cls_dev[:, c0 + j:c0 + j + 1].contiguous() for j in range(n)]
+        torch.cuda.synchronize()
+        a, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        for j in range(n):
+            for layer in range(L):
+                kk, vv, qq = chunk[layer]
+                caches[layer].quantize_append(kk[j], vv[j], cls[j], pos[j])
+                caches[layer].decode_attention(qq[j], SCALE, out)
+            if E and (c0 + j + 1) % E == 0:
+                for layer in range(L):
+                    caches[layer].evict_compact(spec["budget"])
+                n_evict += 1
+        b2.record(st)
+        b2.synchronize()
+        chunk_ms.append(a.elapsed_time(b2))
+        del chunk
+    for g in caches:
+        assert g.poll_error() == 0
+    total_ms = sum(chunk_ms)
+    return {
+        "metric": "decode loop wall time (all layers, append + attention + periodic eviction)",
+        "value": total_ms, "unit": "ms", "higher_is_better": False,
+        "n_gpus": 1, "steps": steps, "layers": L,
+        "decode_tokens_per_s": B * steps / (total_ms * 1e-3),
+        "us_per_step_all_layers": total_ms * 1e3 / steps,
+        "chunk_ms_64_steps": chunk_ms,
+        "first_chunk_note": "steps 0-63 run on the full prefill context (no eviction before step 63)",
+        "evictions": n_evict, "prefill_s_untimed": prefill_s,
+        "config": {"workload": args.workload, "batch": B, "q_heads": Hq, "kv_heads": Hkv, "context": ctx,
+                   "budget": spec["budget"], "evict_every": E, "placement": args.placement,
+                   "attn_kernel": args.attn_kernel, "codec": args.codec},
+        "data": "synthetic (seeded counter-hash N(0,1) bf16)",
+    }
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -529,6 +611,12 @@ def main():
                                              device_id=torch.device(dev))
     from reasoning_model_kv_b200 import build as b
     b.build()
+    if args.decode_loop:
+        if rank == 0:
+            print(json.dumps(run_loop(args, dev)), flush=True)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
     res, gpu, w = run_tkv(args, rank, world, dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(gpu, w, rows=list(range(SAMPLE_ROWS)))

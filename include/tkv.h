@@ -93,9 +93,11 @@ typedef struct {
                             1 = tensor-core kernel (tcgen05 MMAs with integer
                             operands: exact code products, accumulators in
                             tensor memory; persistent, one CTA per SM with the
-                            step's bytes split evenly; dense placement only).
-                            Both compute the same result within the stated
-                            tolerances.                                       */
+                            step's bytes split evenly; dense placement only);
+                            2 = the warp-tile math fed by a persistent TMA
+                            pipeline (two CTAs per SM, the step's bytes split
+                            evenly; dense placement only).  All compute the
+                            same result within the stated tolerances.       */
     int32_t codec;       /* class record formats: 0 = integer codes (classes
                             1/2/3: 8/4/2-bit asymmetric, fp16 scale and zero
                             per group); 1 = floating-point codes (class 1 FP8

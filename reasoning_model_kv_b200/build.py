@@ -21,8 +21,8 @@ ROOT = PKG.parent
 CSRC = PKG / "csrc"
 LIB = PKG / "libtkv.so"
 LIB_DEBUG = PKG / "libtkv_debug.so"
-SOURCES = ["tkv_api.cu", "append.cu", "attention.cu", "attention_i8.cu", "evict.cu", "noalloc.cu", "selftest.cu",
-           "evict_segments.cu"]
+SOURCES = ["tkv_api.cu", "append.cu", "attention.cu", "attention_i8.cu", "attention_ws.cu", "evict.cu", "noalloc.cu",
+           "selftest.cu", "evict_segments.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 FLAGS = [

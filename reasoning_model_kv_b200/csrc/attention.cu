@@ -44,9 +44,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
-#include <type_traits>
-
-#include "attn_common.cuh"
+#include "attn_tile.cuh"
 
 namespace tkv {
 namespace {
@@ -65,205 +63,6 @@ constexpr int kThreads = 32 * kWarps;
 constexpr int kStages = 3;
 constexpr int kStageBytes = 16 * 288;   // the largest tile: 16 int8 records (rows unpadded, swizzled)
 constexpr int kRingBytes = kWarps * kStages * kStageBytes;
-
-struct WarpState {
-    float m[2], l[2];   // reference max / (lane-partial) sum for heads 2*tig, 2*tig+1
-    float o[8][4];      // O^T fragments: dims 16*mt + g (+8), heads 2*tig, 2*tig+1
-    float z[2][4];      // lane-partial sum_t p * vzero per (head, group)
-};
-
-// One tile: up to ROWS records of one class, resident in shared memory (row stride
-// STRIDE; int8 odd rows chunk-swizzled when SWZ).  Lane (g, tig) owns rows g and
-// g + 8.  Rows at or beyond nr hold zeros (the copy zero-fills them); their logits
-// are masked to -inf, so they contribute p = 0 everywhere.
-template <int BITS, int ROWS, int STRIDE, int G, bool SWZ, int FMT = 0>
-__device__ __forceinline__ void tile_compute(const uint8_t *st, int nr, int lane,
-                                             const uint32_t (&qb)[4][2][2], const uint32_t (&qbb)[4][2][2],
-                                             const float (&qs)[2][4], const float (&qinv)[2][4], bool qscaled,
-                                             float xscale, WarpState &ws, float *lg, uint32_t magic) {
-    const int g = lane >> 2, tig = lane & 3;
-    constexpr int QB = 4 * BITS;     // bytes of one quarter of a code block
-    constexpr int CB = 16 * BITS;    // bytes of a code block
-    const bool v0 = g < nr;
-    const bool v1 = ROWS == 16 && g + 8 < nr;
-    const int i0 = g, i1 = g + 8;
-    const uint8_t *r0 = st + i0 * STRIDE;
-    const uint8_t *r1 = st + i1 * STRIDE;
-    const int odd0 = (BITS == 8 && SWZ) ? (i0 & 1) : 0, odd1 = (BITS == 8 && SWZ) ? (i1 & 1) : 0;
-    // meta chunk positions (int8 rows: chunks 16 and 17 swap on odd rows)
-    const int km_off0 = 2 * CB + 16 * odd0, vm_off0 = 2 * CB + 16 - 16 * odd0;
-    const int km_off1 = 2 * CB + 16 * odd1, vm_off1 = 2 * CB + 16 - 16 * odd1;
-
-    // ---- phase 1: S = K . Q^T
-    float x[4] = {0.f, 0.f, 0.f, 0.f};   // (row g, head 2tig), (g, 2tig+1), (g+8, 2tig), (g+8, 2tig+1)
-    {
-        uint32_t k0[BITS], k1[BITS];
-        float2 km0[4], km1[4];
-        load_quarter<BITS>(r0, QB * tig, odd0, k0);
-        if constexpr (ROWS == 16) {
-            load_quarter<BITS>(r1, QB * tig, odd1, k1);
-        } else {
-#pragma unroll
-            for (int i = 0; i < BITS; ++i) k1[i] = 0u;
-        }
-        if constexpr (FMT == 1) {
-            // scales: fp16 per group (FP8, ternary) or E4M3 per 16 dims (NVFP4) at 2 CB
-            const uint2 ka = *reinterpret_cast<const uint2 *>(r0 + 2 * CB);
-            const uint2 kc = *reinterpret_cast<const uint2 *>(r1 + 2 * CB);
-            qk_group_fp<BITS, 0>(x, k0, k1, qb, qinv, qscaled, ka, kc, tig);
-            qk_group_fp<BITS, 1>(x, k0, k1, qb, qinv, qscaled, ka, kc, tig);
-            qk_group_fp<BITS, 2>(x, k0, k1, qb, qinv, qscaled, ka, kc, tig);
-            qk_group_fp<BITS, 3>(x, k0, k1, qb, qinv, qscaled, ka, kc, tig);
-        } else {
-            if constexpr (BITS < 16) {
-                load_meta(r0 + km_off0, km0);
-                load_meta(r1 + km_off1, km1);
-            }
-            qk_group<BITS, 0>(x, k0, k1, qb, qbb, qs, qinv, qscaled, km0, km1, magic);
-            qk_group<BITS, 1>(x, k0, k1, qb, qbb, qs, qinv, qscaled, km0, km1, magic);
-            qk_group<BITS, 2>(x, k0, k1, qb, qbb, qs, qinv, qscaled, km0, km1, magic);
-            qk_group<BITS, 3>(x, k0, k1, qb, qbb, qs, qinv, qscaled, km0, km1, magic);
-        }
-    }
-    const bool h0 = 2 * tig < G, h1 = 2 * tig + 1 < G;
-    x[0] = (v0 && h0) ? x[0] * xscale : -INFINITY;
-    x[1] = (v0 && h1) ? x[1] * xscale : -INFINITY;
-    x[2] = (v1 && h0) ? x[2] * xscale : -INFINITY;
-    x[3] = (v1 && h1) ? x[3] * xscale : -INFINITY;
-    // raw logits (log2 domain) for the score pass
-    if constexpr (G >= 2) {
-        if (h0 && v0) *reinterpret_cast<float2 *>(lg + g * G + 2 * tig) = make_float2(x[0], x[1]);
-        if (h0 && v1) *reinterpret_cast<float2 *>(lg + (g + 8) * G + 2 * tig) = make_float2(x[2], x[3]);
-    } else {
-        if (tig == 0 && v0) lg[g] = x[0];
-        if (tig == 0 && v1) lg[g + 8] = x[2];
-    }
-
-    // ---- online softmax.  The reference max moves only when a tile exceeds it by more
-    //      than the slack, so the column maxima (heads are columns: a reduction over the
-    //      8 row lanes) are formed only then; the reference starts at a finite
-    //      sentinel, so p needs no -inf guard
-    float t0 = fmaxf(x[0], x[2]), t1 = fmaxf(x[1], x[3]);
-    if (__any_sync(kFull, t0 > ws.m[0] + kRescaleSlack || t1 > ws.m[1] + kRescaleSlack)) {
-#pragma unroll
-        for (int o = 4; o < 32; o <<= 1) {
-            t0 = fmaxf(t0, __shfl_xor_sync(kFull, t0, o));
-            t1 = fmaxf(t1, __shfl_xor_sync(kFull, t1, o));
-        }
-        const float mn0 = fmaxf(ws.m[0], t0), mn1 = fmaxf(ws.m[1], t1);
-        const float a0 = ex2(ws.m[0] - mn0), a1 = ex2(ws.m[1] - mn1);
-        ws.m[0] = mn0;
-        ws.m[1] = mn1;
-        ws.l[0] *= a0;
-        ws.l[1] *= a1;
-#pragma unroll
-        for (int mt = 0; mt < 8; ++mt) {
-            ws.o[mt][0] *= a0; ws.o[mt][1] *= a1; ws.o[mt][2] *= a0; ws.o[mt][3] *= a1;
-        }
-#pragma unroll
-        for (int grp = 0; grp < 4; ++grp) { ws.z[0][grp] *= a0; ws.z[1][grp] *= a1; }
-    }
-    float p[4];
-    p[0] = ex2(x[0] - ws.m[0]);
-    p[2] = ex2(x[2] - ws.m[0]);
-    p[1] = ex2(x[1] - ws.m[1]);
-    p[3] = ex2(x[3] - ws.m[1]);
-    ws.l[0] += p[0] + p[2];
-    ws.l[1] += p[1] + p[3];
-
-    // ---- phase 2: O += V^T . (P * vscale) per group; zero term accumulated apart.
-    //      bf16 values: bf16 MMAs with P split into a bf16 high part and the bf16 of
-    //      the remainder (two MMAs), so P keeps ~16 bits and V is never narrowed
-    uint32_t bfr[4][2];
-    uint32_t blo0 = 0u, blo1 = 0u;
-    if constexpr (BITS == 16) {
-        const uint32_t h01 = f32x2_to_bf16x2(p[0], p[1]);
-        const uint32_t l01 = f32x2_to_bf16x2(p[0] - __uint_as_float(h01 << 16), p[1] - __uint_as_float(h01 & 0xffff0000u));
-        const uint32_t b0 = transpose8x8(h01);
-        blo0 = transpose8x8(l01);
-        uint32_t b1 = 0u;
-        if constexpr (ROWS == 16) {
-            const uint32_t h23 = f32x2_to_bf16x2(p[2], p[3]);
-            const uint32_t l23 =
-                f32x2_to_bf16x2(p[2] - __uint_as_float(h23 << 16), p[3] - __uint_as_float(h23 & 0xffff0000u));
-            b1 = transpose8x8(h23);
-            blo1 = transpose8x8(l23);
-        }
-#pragma unroll
-        for (int grp = 0; grp < 4; ++grp) { bfr[grp][0] = b0; bfr[grp][1] = b1; }
-    } else if constexpr (FMT == 1 && BITS == 4) {
-        // NVFP4 values are dequantised exactly in f16 (scale folded into V): P alone
-        const uint32_t b0 = transpose8x8(f32x2_to_f16x2(p[0], p[1]));
-        const uint32_t b1 = transpose8x8(f32x2_to_f16x2(p[2], p[3]));
-#pragma unroll
-        for (int grp = 0; grp < 4; ++grp) { bfr[grp][0] = b0; bfr[grp][1] = b1; }
-    } else if constexpr (FMT == 1) {
-        // FP8 / ternary: the group's fp16 scale folds into P; no zero term
-        const uint2 va = *reinterpret_cast<const uint2 *>(r0 + 2 * CB + 8);
-        const uint2 vc = *reinterpret_cast<const uint2 *>(r1 + 2 * CB + 8);
-        const float2 a01 = __half22float2(u32_as_h2(va.x)), a23 = __half22float2(u32_as_h2(va.y));
-        const float2 c01 = __half22float2(u32_as_h2(vc.x)), c23 = __half22float2(u32_as_h2(vc.y));
-        const float s0[4] = {a01.x, a01.y, a23.x, a23.y}, s1[4] = {c01.x, c01.y, c23.x, c23.y};
-#pragma unroll
-        for (int grp = 0; grp < 4; ++grp) {
-            bfr[grp][0] = transpose8x8(f32x2_to_f16x2(p[0] * s0[grp], p[1] * s0[grp]));
-            bfr[grp][1] = transpose8x8(f32x2_to_f16x2(p[2] * s1[grp], p[3] * s1[grp]));
-        }
-    } else {
-        float2 vm0[4], vm1[4];
-        load_meta(r0 + vm_off0, vm0);
-        load_meta(r1 + vm_off1, vm1);
-#pragma unroll
-        for (int grp = 0; grp < 4; ++grp) {
-            ws.z[0][grp] = fmaf(p[2], vm1[grp].y, fmaf(p[0], vm0[grp].y, ws.z[0][grp]));
-            ws.z[1][grp] = fmaf(p[3], vm1[grp].y, fmaf(p[1], vm0[grp].y, ws.z[1][grp]));
-            bfr[grp][0] = transpose8x8(f32x2_to_f16x2(p[0] * vm0[grp].x, p[1] * vm0[grp].x));
-            bfr[grp][1] = transpose8x8(f32x2_to_f16x2(p[2] * vm1[grp].x, p[3] * vm1[grp].x));
-        }
-    }
-    uint32_t w0[BITS], w1[BITS];
-    load_quarter<BITS>(r0, CB + QB * tig, odd0, w0);
-    if constexpr (ROWS == 16) {
-        load_quarter<BITS>(r1, CB + QB * tig, odd1, w1);
-    } else {
-#pragma unroll
-        for (int i = 0; i < BITS; ++i) w1[i] = 0u;
-    }
-    // NVFP4: each row's E4M3 scale of block MT (dims 16 MT .. 16 MT + 15) as f16x2
-    uint2 vb0 = make_uint2(0u, 0u), vb1 = make_uint2(0u, 0u);
-    if constexpr (FMT == 1 && BITS == 4) {
-        vb0 = *reinterpret_cast<const uint2 *>(r0 + 2 * CB + 8);
-        vb1 = *reinterpret_cast<const uint2 *>(r1 + 2 * CB + 8);
-    }
-    auto vpair = [&](auto pc, const uint32_t (&w)[BITS], const uint2 &vb) -> uint32_t {
-        constexpr int P = decltype(pc)::value;
-        if constexpr (FMT == 1 && BITS == 4) {
-            const uint32_t code = ((P / 2 < 4 ? vb.x : vb.y) >> (8 * ((P / 2) & 3))) & 0xFFu;
-            return hmul2_u32(quarter_pair_fp<BITS, P>(w), e4m3_h2(code));
-        } else if constexpr (FMT == 1) {
-            return quarter_pair_fp<BITS, P>(w);
-        } else {
-            return quarter_pair<BITS, P>(w, magic);
-        }
-    };
-#define TKV_VMMA(MT)                                                                              \
-    {                                                                                             \
-        using P0 = std::integral_constant<int, 2 * (MT)>;                                         \
-        using P1 = std::integral_constant<int, 2 * (MT) + 1>;                                     \
-        const uint32_t e0 = transpose8x8(vpair(P0{}, w0, vb0));                                   \
-        const uint32_t e1 = transpose8x8(vpair(P1{}, w0, vb0));                                   \
-        const uint32_t e2 = ROWS == 16 ? transpose8x8(vpair(P0{}, w1, vb1)) : 0u;                 \
-        const uint32_t e3 = ROWS == 16 ? transpose8x8(vpair(P1{}, w1, vb1)) : 0u;                 \
-        if constexpr (BITS == 16) {                                                               \
-            mma16816_bf16(ws.o[MT], e0, e1, e2, e3, bfr[(MT) >> 1][0], bfr[(MT) >> 1][1]);        \
-            mma16816_bf16(ws.o[MT], e0, e1, e2, e3, blo0, blo1);                                  \
-        } else {                                                                                  \
-            mma16816(ws.o[MT], e0, e1, e2, e3, bfr[(MT) >> 1][0], bfr[(MT) >> 1][1]);             \
-        }                                                                                         \
-    }
-    TKV_VMMA(0) TKV_VMMA(1) TKV_VMMA(2) TKV_VMMA(3) TKV_VMMA(4) TKV_VMMA(5) TKV_VMMA(6) TKV_VMMA(7)
-#undef TKV_VMMA
-}
 
 // Record bytes, reuse-placement stage row stride and rows per tile of class C_ under
 // codec CODEC.  Int8 rows (codec 0) are unpadded and chunk-swizzled on odd rows (SWZ);
@@ -355,60 +154,7 @@ __global__ void __launch_bounds__(kThreads, TKV_ATTN_MIN_BLOCKS) attn_kernel(con
     uint32_t qb[4][2][2], qbb[4][2][2];
     float qs[2][4], qinv[2][4];
     bool qscaled;
-    {
-        float qsg[4], qsc[4];
-        const __nv_bfloat16 *qr = q + ((size_t)b * d.Hkv * G + (size_t)kvh * G + (g < G ? g : 0)) * kD;
-        uint2 raw[4][2];
-#pragma unroll
-        for (int grp = 0; grp < 4; ++grp)
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                raw[grp][hh] = make_uint2(0u, 0u);
-                if (g < G) raw[grp][hh] = *reinterpret_cast<const uint2 *>(qr + 32 * grp + 8 * tig + 4 * hh);
-            }
-        bool any = false;
-#pragma unroll
-        for (int grp = 0; grp < 4; ++grp) {
-            float sum = 0.f, mx = 0.f;
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const uint2 r2 = raw[grp][hh];
-                const float f0 = __uint_as_float(r2.x << 16), f1 = __uint_as_float(r2.x & 0xffff0000u);
-                const float f2 = __uint_as_float(r2.y << 16), f3 = __uint_as_float(r2.y & 0xffff0000u);
-                sum += (f0 + f1) + (f2 + f3);
-                mx = fmaxf(mx, fmaxf(fmaxf(fabsf(f0), fabsf(f1)), fmaxf(fabsf(f2), fabsf(f3))));
-            }
-            sum += __shfl_xor_sync(kFull, sum, 1);
-            sum += __shfl_xor_sync(kFull, sum, 2);
-            mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
-            mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
-            qsg[grp] = sum;                              // sum over group grp of q[head g]
-            // scale 2^(13 - floor(log2 mx)) puts the largest |q| in [2^13, 2^14)
-            float sc = 1.f;
-            if (mx >= 16384.f || (mx > 0.f && mx < 0.0009765625f)) {
-                const int e = (int)((__float_as_uint(mx) >> 23) & 0xff) - 127;
-                sc = __uint_as_float((uint32_t)(127 + 13 - e) << 23);
-                any = true;
-            }
-            qsc[grp] = sc;
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const uint2 r2 = raw[grp][hh];
-                qbb[grp][hh][0] = r2.x;
-                qbb[grp][hh][1] = r2.y;
-                qb[grp][hh][0] = f32x2_to_f16x2(__uint_as_float(r2.x << 16) * sc, __uint_as_float(r2.x & 0xffff0000u) * sc);
-                qb[grp][hh][1] = f32x2_to_f16x2(__uint_as_float(r2.y << 16) * sc, __uint_as_float(r2.y & 0xffff0000u) * sc);
-            }
-        }
-#pragma unroll
-        for (int grp = 0; grp < 4; ++grp) {
-            qs[0][grp] = __shfl_sync(kFull, qsg[grp], (2 * tig) * 4);
-            qs[1][grp] = __shfl_sync(kFull, qsg[grp], (2 * tig + 1) * 4);
-            qinv[0][grp] = 1.f / __shfl_sync(kFull, qsc[grp], (2 * tig) * 4);
-            qinv[1][grp] = 1.f / __shfl_sync(kFull, qsc[grp], (2 * tig + 1) * 4);
-        }
-        qscaled = __any_sync(kFull, any);
-    }
+    query_frags<G>(q + ((size_t)b * d.Hkv * G + (size_t)kvh * G) * kD, lane, qb, qbb, qs, qinv, qscaled);
 
     grid_dependency_wait();   // the append's counters and records are visible from here
 
@@ -544,10 +290,11 @@ __global__ void __launch_bounds__(kThreads, TKV_ATTN_MIN_BLOCKS) attn_kernel(con
         produce();                                                                            \
         const int e = (LO) + (T - (PLO)) * CS::ROWS;                                          \
         const int nr = min(CS::ROWS, (HI) - e);                                               \
-        tile_compute<BITS, CS::ROWS, (DENSE ? CS::REC : CS::STRIDE), G, (!DENSE && CS::SWZ),  \
-                     ((CLS) > 0 ? CODEC : 0)>(ring + (warp * kStages + stage) * kStageBytes,  \
-                                            nr, lane, qb, qbb, qs, qinv, qscaled, xscale, ws, \
-                                            lgs + (size_t)((OFF) + e) * G, magic);            \
+        constexpr int FMT_ = (CLS) > 0 ? CODEC : 0;                                          \
+        const RowLoader<BITS, (DENSE ? CS::REC : CS::STRIDE), (!DENSE && CS::SWZ), FMT_> ldr(   \
+            ring + (warp * kStages + stage) * kStageBytes, lane >> 2);                        \
+        tile_compute<BITS, CS::ROWS, G, FMT_>(ldr, nr, lane, qb, qbb, qs, qinv, qscaled, xscale, ws, \
+                                              lgs + (size_t)((OFF) + e) * G, magic);          \
         __syncwarp();                                                                         \
         stage = stage == 2 ? 0 : stage + 1;                                                   \
     }
@@ -706,7 +453,7 @@ cudaError_t launch_g(const Dev &d, const void *q, float scale, float *out, long 
 
 cudaError_t launch_attention(const Dev &d, const void *q, float scale, float *out, long long live_ub,
                              cudaStream_t st, int64_t *launches) {
-    if (d.dense && d.attn_kernel == 1) return cudaErrorInvalidValue;   // launch_attention_i8's
+    if (d.dense && d.attn_kernel != 0) return cudaErrorInvalidValue;   // the persistent kernels'
 #define TKV_G_CASES(DN, CD)                                                           \
     switch (d.G) {                                                                    \
         case 1: return launch_g<1, DN, CD>(d, q, scale, out, live_ub, st, launches);  \

@@ -59,8 +59,8 @@ bool valid_config(const tkv_config *c, std::string *why) {
     if (c->max_append < 1 || c->max_append > (1 << 24)) { *why = "max_append must be in [1, 2^24]"; return false; }
     if ((long long)c->B * c->Hkv > 65535) { *why = "B * Hkv must be <= 65535"; return false; }
     if (c->dense != 0 && c->dense != 1) { *why = "dense must be 0 or 1"; return false; }
-    if (c->attn_kernel != 0 && c->attn_kernel != 1) { *why = "attn_kernel must be 0 or 1"; return false; }
-    if (c->attn_kernel == 1 && c->dense != 1) { *why = "attn_kernel 1 needs dense placement"; return false; }
+    if (c->attn_kernel < 0 || c->attn_kernel > 2) { *why = "attn_kernel must be 0, 1 or 2"; return false; }
+    if (c->attn_kernel != 0 && c->dense != 1) { *why = "attn_kernel 1 and 2 need dense placement"; return false; }
     if (c->codec != 0 && c->codec != 1) { *why = "codec must be 0 or 1"; return false; }
     if (c->codec == 1 && c->attn_kernel != 0) { *why = "codec 1 needs attn_kernel 0"; return false; }
     for (int i = 0; i < 4; ++i)
@@ -279,11 +279,15 @@ tkv_status tkv_decode_attention(tkv_cache *c, const void *q, float softmax_scale
     if (!aligned16(q) || !aligned16(out)) return fail(TKV_ERR_INVALID, "q and out must be 16-byte aligned");
     const long long ub = std::max(1ll, c->live_ub);
     cudaError_t e;
-    if (c->cfg.dense == 1 && c->cfg.attn_kernel == 1) {
+    if (c->cfg.dense == 1 && c->cfg.attn_kernel != 0) {
         const tkv_status ms = ensure_maps(c);
         if (ms != TKV_OK) return ms;
-        e = tkv::launch_attention_i8(c->dev, c->maps, q, softmax_scale, out, nullptr, nullptr, 0.f, 0.f, ub,
-                                     static_cast<cudaStream_t>(stream), &c->launches);
+        if (c->cfg.attn_kernel == 1)
+            e = tkv::launch_attention_i8(c->dev, c->maps, q, softmax_scale, out, nullptr, nullptr, 0.f, 0.f, ub,
+                                         static_cast<cudaStream_t>(stream), &c->launches);
+        else
+            e = tkv::launch_attention_ws(c->dev, c->maps, q, softmax_scale, out, ub, static_cast<cudaStream_t>(stream),
+                                         &c->launches);
     } else {
         e = tkv::launch_attention(c->dev, q, softmax_scale, out, ub, static_cast<cudaStream_t>(stream),
                                   &c->launches);

@@ -28,7 +28,7 @@ __host__ __device__ constexpr int record_bytes(int bits, int codec = 0) {
 struct Dev {
     int B, Hkv, G, S, n_protect, max_append;
     int dense;              // 1: live records contiguous in table order (handle[i] == i)
-    int attn_kernel;        // 0: warp-tile (mma.sync) kernel, 1: tensor-memory (tcgen05) kernel
+    int attn_kernel;        // 0: warp-tile kernel, 1: tensor-memory (tcgen05) kernel, 2: warp-tile on a TMA pipeline
     int codec;              // 0: integer class records, 1: FP8 / NVFP4 / ternary class records
     int cap[4];
     int rec[4];
@@ -119,6 +119,10 @@ cudaError_t launch_attention_i8(const Dev &d, const I8Maps &maps, const void *q,
                                 cudaStream_t st, int64_t *launches);
 // Encodes the TMA descriptors of d's pools (host only; needs the CUDA driver).
 cudaError_t make_i8_maps(const Dev &d, I8Maps *maps);
+// Dense placement, attn_kernel 2: the warp-tile math fed by a persistent TMA pipeline
+// (attention_ws.cu).
+cudaError_t launch_attention_ws(const Dev &d, const I8Maps &maps, const void *q, float scale, float *out,
+                                long long live_ub, cudaStream_t st, int64_t *launches);
 // Self-test of the bounded device waits (selftest.cu).
 cudaError_t launch_wait_timeout(const Dev &d, long long limit, cudaStream_t st, int64_t *launches);
 cudaError_t launch_evict(const Dev &d, int budget, int keep_from, cudaStream_t st, int64_t *launches);

@@ -82,7 +82,7 @@ def np_bits(t: torch.Tensor) -> np.ndarray:
 
 # Cache modes the parity tests run in: placement and decode-attention kernel.
 MODES = {"reuse": dict(dense=False), "dense": dict(dense=True),
-         "dense_tc": dict(dense=True, attn_kernel=1)}
+         "dense_tc": dict(dense=True, attn_kernel=1), "dense_ws": dict(dense=True, attn_kernel=2)}
 
 
 def build_pair(name: str, device="cuda", rows=None, dense=False, attn_kernel=0, codec=0, **over):

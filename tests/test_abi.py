@@ -180,14 +180,16 @@ def test_every_config_rule_is_enforced_on_the_host():
     """Each rule of the configuration check, one violation at a time (no device needed)."""
     assert tkv.tkv_workspace_bytes(_cfg(dense=True)) > 0
     assert tkv.tkv_workspace_bytes(_cfg(dense=True, attn_kernel=1)) > 0
+    assert tkv.tkv_workspace_bytes(_cfg(dense=True, attn_kernel=2)) > 0
     assert tkv.tkv_workspace_bytes(_cfg(cap=[(1 << 24) - 1] * 4)) > 0      # largest legal capacities
     for kw in (dict(Hkv=0), dict(G=16), dict(n_protect=-1), dict(max_append=(1 << 24) + 1),
                dict(B=256, Hkv=256),                  # B * Hkv above 65535
                dict(cap=[0, 1 << 24, 0, 0]),          # a class capacity of 2^24
                dict(attn_kernel=1),                   # the tensor-memory kernel needs dense placement
+               dict(attn_kernel=2),                   # so does the persistent warp-tile kernel
                dict(dense=True, attn_kernel=1, codec=1)):   # FP codes: the warp-tile kernel only
         assert tkv.tkv_workspace_bytes(_cfg(**kw)) == 0, kw
-    for field, value in (("group", 16), ("dense", 2), ("attn_kernel", 2), ("codec", 2)):
+    for field, value in (("group", 16), ("dense", 2), ("attn_kernel", 3), ("codec", 2)):
         cfg = _cfg()
         setattr(cfg, field, value)
         assert tkv.tkv_workspace_bytes(cfg) == 0, field
