@@ -536,7 +536,19 @@ def run_loop(args, dev):
         del w["k"], w["v"]
         caches.append(g)
         ws.append(w)
+    # every kernel of the loop launched once before timing (module loading, launch
+    # attributes), on a small cache of the same shape class
+    wu = synth.prefill_inputs("tiny_b1_ctx2k", device=dev, B=1, Hq=Hq // Hkv, Hkv=1, ctx=512,
+                              n_protect=spec["n_protect"], steps=2)
+    gw = TkvCache(1, 1, wu["G"], wu["cap"], wu["n_protect"], max_append=wu["ctx"], dense=args.placement == "dense",
+                  attn_kernel=kern, codec=1 if args.codec == "fp" else 0)
+    gw.quantize_append(wu["k"], wu["v"], wu["cls"][:, :wu["ctx"]].contiguous().to(dev), wu["pos"].to(dev))
+    kw, vw, cw, pw, qw = synth.decode_inputs(wu, 0, device=dev)
+    gw.quantize_append(kw, vw, cw, pw)
+    gw.decode_attention(qw, SCALE)
+    gw.evict_compact(128)
     torch.cuda.synchronize()
+    del gw
     prefill_s = time.time() - t0
     cls_dev = ws[0]["cls"][:, ctx:ctx + steps].contiguous().to(dev)
     out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)

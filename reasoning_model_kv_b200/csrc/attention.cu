@@ -451,6 +451,17 @@ cudaError_t launch_g(const Dev &d, const void *q, float scale, float *out, long 
 
 }  // namespace
 
+bool warp_tile_underfills(const Dev &d, long long live_ub) {
+    // the warp-tile kernel gives a stream at most kMaxCluster CTAs; with few long streams
+    // that leaves most of the GPU idle, where the persistent pipeline (every SM, an equal
+    // share of the bytes) is faster: fewer CTAs than two per SM and at least 32k entries
+    // in the longest stream
+    if (live_ub < 32768) return false;
+    int sms = 0;
+    if (device_sm_count(&sms) != cudaSuccess || sms <= 0) return false;
+    return (long long)d.S * kMaxCluster < 2ll * sms;
+}
+
 cudaError_t launch_attention(const Dev &d, const void *q, float scale, float *out, long long live_ub,
                              cudaStream_t st, int64_t *launches) {
     if (d.dense && d.attn_kernel != 0) return cudaErrorInvalidValue;   // the persistent kernels'

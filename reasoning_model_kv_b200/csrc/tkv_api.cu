@@ -279,7 +279,9 @@ tkv_status tkv_decode_attention(tkv_cache *c, const void *q, float softmax_scale
     if (!aligned16(q) || !aligned16(out)) return fail(TKV_ERR_INVALID, "q and out must be 16-byte aligned");
     const long long ub = std::max(1ll, c->live_ub);
     cudaError_t e;
-    if (c->cfg.dense == 1 && c->cfg.attn_kernel != 0) {
+    const bool persistent = c->cfg.dense == 1 &&
+                            (c->cfg.attn_kernel != 0 || (c->cfg.codec == 0 && tkv::warp_tile_underfills(c->dev, ub)));
+    if (persistent) {
         const tkv_status ms = ensure_maps(c);
         if (ms != TKV_OK) return ms;
         if (c->cfg.attn_kernel == 1)
