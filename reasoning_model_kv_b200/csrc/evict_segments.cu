@@ -197,6 +197,7 @@ __global__ void __launch_bounds__(kThreads) tbe_kernel(Dev d, const int32_t *__r
                     if (a[k]) atomicAdd(&tot_dig[k], a[k]);
             }
         }
+        __syncthreads();   // every segment's count and sum written
         // T2. the stream's mean score over all candidates -> delta
         {
             int n = 0;
