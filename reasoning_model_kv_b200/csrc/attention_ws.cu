@@ -56,17 +56,6 @@ struct QFrag {
     uint32_t pad;
 };
 
-// OR of pred over the warps of a consumer group (its barrier, with a reduction).
-__device__ __forceinline__ bool group_any(int bar, bool pred) {
-    uint32_t r;
-    asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, %2, %3, p;\n\t"
-                 "selp.u32 %0, 1, 0, q;\n\t}"
-                 : "=r"(r)
-                 : "r"((uint32_t)pred), "r"(bar), "r"(32 * kConsumers)
-                 : "memory");
-    return r != 0;
-}
-
 template <int G>
 __global__ void __launch_bounds__(kThreadsWS, kCtasPerSm)
     attn_ws_kernel(const __grid_constant__ Dev d, const __grid_constant__ I8Maps maps,
@@ -75,6 +64,10 @@ __global__ void __launch_bounds__(kThreadsWS, kCtasPerSm)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);   // stages: 1024-aligned
     __shared__ __align__(8) uint64_t bar_full[R], bar_empty[R];
+    // per group: its warps' partials written / read (the two halves of a merge), and the
+    // stream's query operands published; bounded waits, so a warp that gave up on a
+    // timeout never leaves the others stuck at a barrier
+    __shared__ __align__(8) uint64_t bar_written[kGroups], bar_read[kGroups], bar_query[kGroups];
     __shared__ SharedPlan pl;
     __shared__ TileDesc desc[kDescRing];
     __shared__ float wm[kGroups][kConsumers][kMaxG], wl[kGroups][kConsumers][kMaxG];
@@ -88,6 +81,11 @@ __global__ void __launch_bounds__(kThreadsWS, kCtasPerSm)
         for (int i = 0; i < R; ++i) {
             mbar_init_n(smem_addr(&bar_full[i]), 1);
             mbar_init_n(smem_addr(&bar_empty[i]), kConsumers);
+        }
+        for (int i = 0; i < kGroups; ++i) {
+            mbar_init_n(smem_addr(&bar_written[i]), kConsumers);
+            mbar_init_n(smem_addr(&bar_read[i]), kConsumers);
+            mbar_init_n(smem_addr(&bar_query[i]), 1);
         }
         err_timeout = 0;
         mbar_init_fence();
@@ -106,8 +104,16 @@ __global__ void __launch_bounds__(kThreadsWS, kCtasPerSm)
     } else {
         // ================================================= consumer group grp, warp cw of it
         const int grp = warp / kConsumers, cw = warp - grp * kConsumers;
-        const int gbar = 1 + grp;                       // the group's named barrier
         const int gt = tid - grp * 32 * kConsumers;     // thread index inside the group
+        int nmerge = 0, nquery = 0;                     // phases used of bar_written / bar_read, bar_query
+        // every warp of the group at a merge point (lane 0 arrives after the warp's writes)
+        auto group_sync = [&](uint64_t *bar, int &uses) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(bar));
+            if (ok) ok = mbar_wait(smem_addr(bar), (uint32_t)(uses & 1));
+            ok = __all_sync(kFull, ok);
+            ++uses;
+        };
         const int g = lane >> 2, tig = lane & 3;
         const uint32_t magic = magic_f16();
         float *wo = reinterpret_cast<float *>(sm + R * kRawBytes + grp * ws_merge_bytes(G));   // [cw][G][kD]
@@ -131,9 +137,9 @@ __global__ void __launch_bounds__(kThreadsWS, kCtasPerSm)
                 ws.l[0] += __shfl_xor_sync(kFull, ws.l[0], o);
                 ws.l[1] += __shfl_xor_sync(kFull, ws.l[1], o);
 #pragma unroll
-                for (int grp = 0; grp < 4; ++grp) {
-                    ws.z[0][grp] += __shfl_xor_sync(kFull, ws.z[0][grp], o);
-                    ws.z[1][grp] += __shfl_xor_sync(kFull, ws.z[1][grp], o);
+                for (int zg = 0; zg < 4; ++zg) {
+                    ws.z[0][zg] += __shfl_xor_sync(kFull, ws.z[0][zg], o);
+                    ws.z[1][zg] += __shfl_xor_sync(kFull, ws.z[1][zg], o);
                 }
             }
             if (g == 0) {
@@ -143,17 +149,18 @@ __global__ void __launch_bounds__(kThreadsWS, kCtasPerSm)
             float *w = wo + cw * G * kD;
 #pragma unroll
             for (int mt = 0; mt < 8; ++mt) {
-                const int d0 = 16 * mt + g, grp = mt >> 1;
+                const int d0 = 16 * mt + g, zg = mt >> 1;
                 if (2 * tig < G) {
-                    w[(2 * tig) * kD + d0] = ws.o[mt][0] + ws.z[0][grp];
-                    w[(2 * tig) * kD + d0 + 8] = ws.o[mt][2] + ws.z[0][grp];
+                    w[(2 * tig) * kD + d0] = ws.o[mt][0] + ws.z[0][zg];
+                    w[(2 * tig) * kD + d0 + 8] = ws.o[mt][2] + ws.z[0][zg];
                 }
                 if (2 * tig + 1 < G) {
-                    w[(2 * tig + 1) * kD + d0] = ws.o[mt][1] + ws.z[1][grp];
-                    w[(2 * tig + 1) * kD + d0 + 8] = ws.o[mt][3] + ws.z[1][grp];
+                    w[(2 * tig + 1) * kD + d0] = ws.o[mt][1] + ws.z[1][zg];
+                    w[(2 * tig + 1) * kD + d0 + 8] = ws.o[mt][3] + ws.z[1][zg];
                 }
             }
-            named_sync(gbar, 32 * kConsumers);
+            int u = nmerge;
+            group_sync(&bar_written[grp], u);
             float *part = d.part + (size_t)(kGroups * (s_old + cta) + grp) * part_floats(G);
             for (int i = gt; i < G * kD; i += 32 * kConsumers) {
                 const int h = i / kD;
@@ -175,7 +182,9 @@ __global__ void __launch_bounds__(kThreadsWS, kCtasPerSm)
                     part[2 * G + h] = 0.f;
                 }
             }
-            named_sync(gbar, 32 * kConsumers);   // wm / wl / wo free again
+            u = nmerge;
+            group_sync(&bar_read[grp], u);   // wm / wl / wo free again
+            ++nmerge;
         };
         // an empty partial (l = 0: the merge skips it) in this group's slot of stream s
         auto write_empty = [&](int s) {
@@ -200,9 +209,8 @@ __global__ void __launch_bounds__(kThreadsWS, kCtasPerSm)
                 const TileDesc to = desc[(k - 1) % kDescRing];
                 if (!td_end(to) && to.s != cur_s && (end || to.s != td.s)) write_empty(to.s);
             }
-            // one decision for all warps of the group, so that they leave together and the
-            // merge barriers are always met by all of them
-            if (group_any(gbar, !ok || end)) break;
+            const bool wok = __all_sync(kFull, ok);
+            if (end || !wok) { ok = wok; break; }
             if (td.s != cur_s) {
                 if (cur_s >= 0) flush(cur_s);
                 cur_s = td.s;
@@ -214,8 +222,12 @@ __global__ void __launch_bounds__(kThreadsWS, kCtasPerSm)
                                    f.qinv, sc);
                     qf[grp][lane] = f;
                     if (lane == 0) qscaled_sh[grp] = sc;
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_addr(&bar_query[grp]));
                 }
-                named_sync(gbar, 32 * kConsumers);   // the stream's query operands are in place
+                if (ok) ok = mbar_wait(smem_addr(&bar_query[grp]), (uint32_t)(nquery & 1));   // operands in place
+                ok = __all_sync(kFull, ok);
+                ++nquery;
                 qscaled = qscaled_sh[grp] != 0;
                 reset();
             }
@@ -252,9 +264,9 @@ __global__ void __launch_bounds__(kThreadsWS, kCtasPerSm)
                 if (td_last(td)) d.seg_hi[td.s] = cta;
             }
         }
-        // every warp of the group left the loop at the same tile, so the merge barriers
-        // below are met by all eight (or, after a timeout, by none)
-        if (!group_any(gbar, !ok)) {
+        // every warp of the group left the loop at its end tile (or gave up on a timeout,
+        // in which case the bounded merge waits of the others run out as well)
+        if (ok) {
             if (cur_s >= 0) {
                 flush(cur_s);
             } else if (cta_empty && pl.s0 < d.S) {
