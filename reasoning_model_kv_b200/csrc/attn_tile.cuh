@@ -151,10 +151,12 @@ __device__ __forceinline__ void tile_compute(const Loader &ld, int nr, int lane,
         float2 vm0[4], vm1[4];
         load_meta(ld.v_meta(0), vm0);
         load_meta(ld.v_meta(1), vm1);
+        if constexpr (!Loader::kZeroFilled) {
 #pragma unroll
-        for (int grp = 0; grp < 4; ++grp) {
-            vm0[grp] = v0 ? vm0[grp] : make_float2(0.f, 0.f);
-            vm1[grp] = v1 ? vm1[grp] : make_float2(0.f, 0.f);
+            for (int grp = 0; grp < 4; ++grp) {
+                vm0[grp] = v0 ? vm0[grp] : make_float2(0.f, 0.f);
+                vm1[grp] = v1 ? vm1[grp] : make_float2(0.f, 0.f);
+            }
         }
 #pragma unroll
         for (int grp = 0; grp < 4; ++grp) {
@@ -173,11 +175,14 @@ __device__ __forceinline__ void tile_compute(const Loader &ld, int nr, int lane,
         for (int i = 0; i < BITS; ++i) w1[i] = 0u;
     }
     // rows past the tile's records may hold anything (a TMA box's trailing rows): their
-    // values must not reach the MMA, where 0 * inf would poison the sums
+    // values must not reach the MMA, where 0 * inf would poison the sums (a staging ring
+    // zero-fills them already)
+    if constexpr (!Loader::kZeroFilled) {
 #pragma unroll
-    for (int i = 0; i < BITS; ++i) {
-        w0[i] = v0 ? w0[i] : 0u;
-        w1[i] = v1 ? w1[i] : 0u;
+        for (int i = 0; i < BITS; ++i) {
+            w0[i] = v0 ? w0[i] : 0u;
+            w1[i] = v1 ? w1[i] : 0u;
+        }
     }
     // NVFP4: each row's E4M3 scale of block MT (dims 16 MT .. 16 MT + 15) as f16x2
     uint2 vb0 = make_uint2(0u, 0u), vb1 = make_uint2(0u, 0u);
@@ -288,6 +293,7 @@ __device__ __forceinline__ void query_frags(const __nv_bfloat16 *__restrict__ qh
 // (SWZ); meta (codec 0: scale x4 + zero x4 per block; codec 1: scales) after the codes.
 template <int BITS, int STRIDE, bool SWZ, int FMT>
 struct RowLoader {
+    static constexpr bool kZeroFilled = true;   // the copies zero-fill rows past the tile
     static constexpr int QB = 4 * BITS, CB = 16 * BITS;
     const uint8_t *r[2];
     int odd[2];
@@ -318,6 +324,7 @@ struct RowLoader {
 // 0-127, 128-255, then V).  Rows r0 + g and r0 + g + 8 of the tile.
 template <int BITS>
 struct TmaLoader {
+    static constexpr bool kZeroFilled = false;  // trailing rows hold what the pool or an earlier tile left
     static constexpr int W = BITS == 16 ? 128 : 16 * BITS;   // box row bytes
     static constexpr int KOFF = 0;
     static constexpr int VOFF = BITS == 16 ? 16384 : BITS == 8 ? 16384 : BITS == 4 ? 8192 : 4096;

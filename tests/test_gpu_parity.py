@@ -142,8 +142,9 @@ def test_multi_token_append_after_eviction_reuses_slots_in_order(dense):
     compare_states(gpu.export_state(), o.state, what="append T=77 after eviction")
 
 
-def test_empty_cache_and_single_token():
-    gpu = TkvCache(1, 2, 4, cap=[4, 4, 4, 4], n_protect=0)
+@pytest.mark.parametrize("mode", list(MODES))
+def test_empty_cache_and_single_token(mode):
+    gpu = TkvCache(1, 2, 4, cap=[4, 4, 4, 4], n_protect=0, **MODES[mode])
     q = synth.normal_bf16(0, 0, synth.TID_Q, 1, 8, 0, 1, 128)[:, :, 0].contiguous()
     out = gpu.decode_attention(q.to(DEV), SCALE)
     assert not out.any()
@@ -151,7 +152,7 @@ def test_empty_cache_and_single_token():
     cls = torch.tensor([[3]], dtype=torch.uint8)
     pos = torch.zeros((1, 1), dtype=torch.int32)
     gpu.quantize_append(k.to(DEV), k.to(DEV), cls.to(DEV), pos.to(DEV))
-    o = orc.OracleCache(1, 2, 4, cap=[4, 4, 4, 4], n_protect=0)
+    o = orc.OracleCache(1, 2, 4, cap=[4, 4, 4, 4], n_protect=0, dense=MODES[mode]["dense"])
     o.append(np_bits(k), np_bits(k), cls.numpy(), pos.numpy())
     out = gpu.decode_attention(q.to(DEV), SCALE).cpu().numpy()
     ref = o.attend(np_bits(q), SCALE)
@@ -160,9 +161,9 @@ def test_empty_cache_and_single_token():
     assert abs(g["score3"][0, 0] - 4.0) < 1e-6 and abs(g["score3"][1, 0] - 4.0) < 1e-6
 
 
-@pytest.mark.parametrize("dense", [False, True], ids=["reuse", "dense"])
-def test_budget_edge_cases(dense):
-    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", ctx=300, n_protect=17, dense=dense)
+@pytest.mark.parametrize("mode", list(MODES))
+def test_budget_edge_cases(mode):
+    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", ctx=300, n_protect=17, **MODES[mode])
     gpu.decode_attention(synth.decode_inputs(w, 0)[4].to(DEV), SCALE)
     before = gpu.export_state()
     gpu.evict_compact(300)                     # budget >= candidates: untouched
@@ -474,3 +475,30 @@ def test_attention_sparsity_needs_the_tensor_core_kernel():
     q = synth.decode_inputs(w, 0)[4].to(DEV)
     with pytest.raises(TkvError):
         gpu.decode_attention_sparsity(q, SCALE, 0.8, 0.2)   # th_r > th_t
+
+
+
+@pytest.mark.parametrize("mode", ["dense", "dense_tc", "dense_ws"])
+@pytest.mark.parametrize("seed", [0, 1])
+def test_ragged_streams_with_empty_classes_and_streams(mode, seed):
+    """Dense caches whose streams hold very different numbers of entries per class --
+    empty classes, empty streams, single entries, full tiles plus a ragged tail -- so the
+    persistent kernels' byte-balanced split puts several streams in one CTA, one stream
+    over several CTAs, and leaves CTAs with no tile at all."""
+    rng = np.random.default_rng(900 + seed)
+    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", B=6, Hq=16, Hkv=4, ctx=700, n_protect=5, steps=2,
+                                 **MODES[mode])
+    st = gpu.export_state()
+    for s_ in range(gpu.S):
+        for c in range(4):
+            n = int(st["n"][s_, c])
+            pick = rng.choice([0, 1, n // 3, n, max(n - 1, 0), int(rng.integers(0, n + 1))])
+            st["n"][s_, c] = min(n, pick)
+            st["hw"][s_, c] = st["n"][s_, c]
+    st["n"][3] = 0                     # one empty stream
+    st["hw"][3] = 0
+    gpu.import_state(st)
+    o.load_state(gpu.export_state(rows_streams(gpu, rows)))
+    for step in range(2):
+        _decode_step(w, gpu, o, rows, step)
+    assert gpu.poll_error() == tkv.TKV_OK
