@@ -298,7 +298,10 @@ __device__ __forceinline__ int pick4(const int4 &v, int c) {
     return c == 0 ? v.x : c == 1 ? v.y : c == 2 ? v.z : v.w;
 }
 
-template <bool kSingle>
+// kCodec: the class record formats (0 integer codes, 1 FP codes), a template argument so
+// that each instantiation holds only its own quantiser (the T = 1 append overlaps the
+// decode attention launched after it, and a leaner kernel leaves it more room).
+template <bool kSingle, int kCodec>
 __global__ void __launch_bounds__(256) append_pack_kernel(
     Dev d, const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ v,
     const uint8_t *__restrict__ cls, const int32_t *__restrict__ pos, int T) {
@@ -352,7 +355,7 @@ __global__ void __launch_bounds__(256) append_pack_kernel(
     }
     uint8_t *rec = d.pool[c] + ((size_t)s * cap + slot) * d.rec[c];
     uint8_t *stage = stage_all + (threadIdx.x >> 5) * 2 * kD;
-    if (d.codec == 0 || c == 0) {
+    if constexpr (kCodec == 0) {
         switch (c) {
             case 0: pack_record<16>(rk, rv, rec, lane, stage); break;
             case 1: pack_record<8>(rk, rv, rec, lane, stage); break;
@@ -361,6 +364,7 @@ __global__ void __launch_bounds__(256) append_pack_kernel(
         }
     } else {
         switch (c) {
+            case 0: pack_record<16>(rk, rv, rec, lane, stage); break;
             case 1: pack_record_fp<8>(rk, rv, rec, lane, stage); break;
             case 2: pack_record_fp<4>(rk, rv, rec, lane, stage); break;
             default: pack_record_fp<2>(rk, rv, rec, lane, stage); break;
@@ -397,12 +401,14 @@ cudaError_t launch_append(const Dev &d, const void *k, const void *v, const uint
     const int threads = 256;
     const unsigned blocks = (unsigned)((warps * 32 + threads - 1) / threads);
     if (T == 1) {
-        append_pack_kernel<true><<<blocks, threads, 0, st>>>(d, kk, vv, cls, pos, T);
+        if (d.codec == 0) append_pack_kernel<true, 0><<<blocks, threads, 0, st>>>(d, kk, vv, cls, pos, T);
+        else append_pack_kernel<true, 1><<<blocks, threads, 0, st>>>(d, kk, vv, cls, pos, T);
         *launches += 1;
         return cudaGetLastError();
     }
     append_rank_kernel<<<d.B, 1024, 0, st>>>(d, cls, pos, T);
-    append_pack_kernel<false><<<blocks, threads, 0, st>>>(d, kk, vv, cls, pos, T);
+    if (d.codec == 0) append_pack_kernel<false, 0><<<blocks, threads, 0, st>>>(d, kk, vv, cls, pos, T);
+    else append_pack_kernel<false, 1><<<blocks, threads, 0, st>>>(d, kk, vv, cls, pos, T);
     append_finalize_kernel<<<(d.S * 4 + 255) / 256, 256, 0, st>>>(d);
     *launches += 3;
     return cudaGetLastError();
