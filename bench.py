@@ -5,8 +5,10 @@ context with x10 K outlier channels, R/E/T = 0.35/0.35/0.30 segments, a 128-toke
 bf16 question window, eviction to 1638 tokens, then the timed step: quantize-append
 of the new token + decode attention with score accumulation.
 
-One timed step = tkv_quantize_append + tkv_decode_attention on every stream.  The
-cache counters are restored (untimed) before each step so every step sees the same
+One timed step = the new token's quantize-append + decode attention on every stream:
+one tkv_decode_step call (default), or tkv_quantize_append then tkv_decode_attention
+with --step-call separate (the same two launches).  The cache
+counters are restored (untimed) before each step so every step sees the same
 post-eviction cache, and the L2 is flushed (untimed) before each step.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl tkv|reference]
@@ -71,6 +73,9 @@ def parse():
     ap.add_argument("--full-reps", type=int, default=3,
                     help="timed attention calls on the full prefill context before the eviction "
                          "(the full-context phase; 0 skips it)")
+    ap.add_argument("--step-call", choices=["step", "separate"], default="step",
+                    help="the calls a step makes: step (tkv_decode_step, one call) or separate "
+                         "(tkv_quantize_append, then tkv_decode_attention)")
     ap.add_argument("--decode-loop", action="store_true",
                     help="time the workload's whole decode loop instead of one step: every layer, "
                          "every step (append + attention), the periodic eviction, CUDA events "
@@ -279,9 +284,15 @@ def run_tkv(args, rank, world, dev):
         for key in ("n", "ft", "hw"):
             views[key].copy_(saved[key])
 
+    def call_step(kk, vv, cc, pp, qq):
+        if args.step_call == "step":
+            gpu.decode_step(kk[:, :, 0], vv[:, :, 0], cc[:, 0], pp[:, 0], qq, SCALE, out)
+        else:
+            gpu.quantize_append(kk, vv, cc, pp)
+            gpu.decode_attention(qq, SCALE, out)
+
     def step():
-        gpu.quantize_append(k, v, c, p)
-        gpu.decode_attention(q, SCALE, out)
+        call_step(k, v, c, p, q)
 
     # packed bytes read by the timed attention: every live entry after the append
     restore()
@@ -304,8 +315,9 @@ def run_tkv(args, rank, world, dev):
     if world > 1:
         torch.distributed.barrier()
     st = torch.cuda.current_stream()
-    # (1) the step: append + attention back to back (no event between them, so the
-    #     attention launch may overlap the append as it does in a decode loop)
+    # (1) the step: append + attention back to back, through tkv_decode_step or the two
+    #     calls (no event between them: the attention launch overlaps the append as it
+    #     does in a decode loop)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
     # (2) the attention call alone, on the post-append cache: the kernel the roofline
@@ -320,8 +332,7 @@ def run_tkv(args, rank, world, dev):
             restore()
             flush.zero_()
             ev[i][0].record(st)
-            gpu.quantize_append(k, v, c, p)
-            gpu.decode_attention(q, SCALE, out)
+            call_step(k, v, c, p, q)
             ev[i][1].record(st)
         torch.cuda.synchronize()
         launches = gpu.launch_count() - launches0
@@ -364,8 +375,7 @@ def run_tkv(args, rank, world, dev):
         a, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(st)
         dbuf.copy_(hbuf, non_blocking=True)
-        gpu.quantize_append(dk, dv, dc, dp)
-        gpu.decode_attention(dq, SCALE, out)
+        call_step(dk, dv, dc, dp, dq)
         hout.copy_(out, non_blocking=True)
         b2.record(st)
         b2.synchronize()
@@ -401,6 +411,8 @@ def run_tkv(args, rank, world, dev):
                    "total_bytes_per_step": pk + kv_tokens * (8 + (0 if args.placement == "dense" else 4))
                    + q.numel() * q.element_size() + out.numel() * out.element_size(),
                    "placement": args.placement, "attn_kernel": args.attn_kernel, "codec": args.codec,
+                   "step_call": {"step": "tkv_decode_step",
+                                 "separate": "tkv_quantize_append + tkv_decode_attention"}[args.step_call],
                    "eviction": {"topk": f"topk, budget {w['budget']} per stream",
                                 "tbe": "tbe segment schedule at the scoring step (r0 64, t_keep 16)",
                                 "tam": f"tam segment budgets, {w['budget']} per stream, pivotal above 3x "
@@ -413,7 +425,7 @@ def run_tkv(args, rank, world, dev):
         "attention_ms_median": statistics.median(attn_ms),
         "attention_ms_min": min(attn_ms),
         "attention_timing": "attention call alone on the post-append cache (L2 flushed), CUDA events",
-        "append_exposed_ms": t_step - t_attn,
+        "append_exposed_ms": t_step - t_attn,   # step minus the attention call timed alone
         "evict_ms_untimed_step": evict_ms,
         "full_context_phase": full,
         "kv_tokens_per_s": world * kv_tokens / (t_attn * 1e-3),
@@ -546,6 +558,7 @@ def run_loop(args, dev):
     kw, vw, cw, pw, qw = synth.decode_inputs(wu, 0, device=dev)
     gw.quantize_append(kw, vw, cw, pw)
     gw.decode_attention(qw, SCALE)
+    gw.decode_step(kw[:, :, 0], vw[:, :, 0], cw[:, 0], pw[:, 0], qw, SCALE)
     gw.evict_compact(128)
     torch.cuda.synchronize()
     del gw
@@ -574,8 +587,12 @@ def run_loop(args, dev):
         for j in range(n):
             for layer in range(L):
                 kk, vv, qq = chunk[layer]
-                caches[layer].quantize_append(kk[j], vv[j], cls[j], pos[j])
-                caches[layer].decode_attention(qq[j], SCALE, out)
+                if args.step_call == "step":
+                    caches[layer].decode_step(kk[j][:, :, 0], vv[j][:, :, 0], cls[j][:, 0], pos[j][:, 0], qq[j],
+                                              SCALE, out)
+                else:
+                    caches[layer].quantize_append(kk[j], vv[j], cls[j], pos[j])
+                    caches[layer].decode_attention(qq[j], SCALE, out)
             if E and (c0 + j + 1) % E == 0:
                 for layer in range(L):
                     caches[layer].evict_compact(spec["budget"])
@@ -598,7 +615,7 @@ def run_loop(args, dev):
         "evictions": n_evict, "prefill_s_untimed": prefill_s,
         "config": {"workload": args.workload, "batch": B, "q_heads": Hq, "kv_heads": Hkv, "context": ctx,
                    "budget": spec["budget"], "evict_every": E, "placement": args.placement,
-                   "attn_kernel": args.attn_kernel, "codec": args.codec},
+                   "attn_kernel": args.attn_kernel, "codec": args.codec, "step_call": args.step_call},
         "data": "synthetic (seeded counter-hash N(0,1) bf16)",
     }
 

@@ -225,6 +225,22 @@ TKV_API tkv_status tkv_decode_attention(tkv_cache *cache, const void *q, float s
                                 float *out, void *stream);
 
 /*
+ * One decode step with its new token: exactly tkv_quantize_append with T = 1
+ * (k, v, cls, pos as there: k, v device bf16 [B][Hkv][D], cls uint8 [B], pos
+ * int32 [B]) followed by tkv_decode_attention (q, softmax_scale, out as there),
+ * so the step attends over the new token too, in one call: the two launches go
+ * back to back, the attention's launch overlapping the append (programmatic
+ * dependent launch).  Results, device errors and the cache state are those of the
+ * two calls.  The ThinKV page's decode loop (Implementacao do Sistema) writes each
+ * new token into the block table the same step reads.
+ * Returns TKV_ERR_INVALID (launching nothing) for a NULL pointer or k, v, pos, q,
+ * out not 16-byte aligned.
+ */
+TKV_API tkv_status tkv_decode_step(tkv_cache *cache, const void *k, const void *v, const uint8_t *cls,
+                                   const int32_t *pos, const void *q, float softmax_scale, float *out,
+                                   void *stream);
+
+/*
  * tkv_decode_attention plus, per (stream, query head), the attention sparsity of
  * this step and the thought type it indicates (ThinKV page, "Metodologia": the
  * thought types differ in how sparse their attention is -- Transition the most,

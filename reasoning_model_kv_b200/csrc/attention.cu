@@ -145,8 +145,12 @@ __global__ void __launch_bounds__(kThreads, TKV_ATTN_MIN_BLOCKS) attn_kernel(con
     const int s = blockIdx.y;
     const int b = s / d.Hkv, kvh = s - b * d.Hkv;
 
-    // ---- query operand (B of S = K Q^T; independent of the previous kernel, so it is
-    //      loaded before the dependency wait): head g, dims 32grp + 8tig + 4hh + 0..3.
+    // the previous kernel's writes (an append's counters and records, or the caller's
+    // query) are visible from here: nothing is read before it, since this kernel may
+    // launch while the previous one still runs (programmatic dependent launch)
+    grid_dependency_wait();
+
+    // ---- query operand (B of S = K Q^T): head g, dims 32grp + 8tig + 4hh + 0..3.
     //      qbb: the raw bf16 pairs (bf16 keys); qb: f16 pairs for the integer codes,
     //      each (group, head) scaled by a power of two when its largest |q| lies
     //      outside [2^-10, 2^14) so that f16 neither overflows nor goes subnormal on
@@ -155,8 +159,6 @@ __global__ void __launch_bounds__(kThreads, TKV_ATTN_MIN_BLOCKS) attn_kernel(con
     float qs[2][4], qinv[2][4];
     bool qscaled;
     query_frags<G>(q + ((size_t)b * d.Hkv * G + (size_t)kvh * G) * kD, lane, qb, qbb, qs, qinv, qscaled);
-
-    grid_dependency_wait();   // the append's counters and records are visible from here
 
     // ---- this CTA's entry range and its tiles (class by class)
     const int n0 = dclamp(d.err, d.n[s * 4 + 0], d.cap[0], kDbgAttention + 0);
@@ -438,7 +440,7 @@ cudaError_t launch_g(const Dev &d, const void *q, float scale, float *out, long 
     attr[0].val.clusterDim.x = (unsigned)C;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // overlap the launch with the append
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // overlap the launch with the kernel before
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;

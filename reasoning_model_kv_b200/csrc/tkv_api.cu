@@ -272,12 +272,10 @@ tkv_status ensure_maps(tkv_cache *c) {
 }
 }  // namespace
 
-tkv_status tkv_decode_attention(tkv_cache *c, const void *q, float softmax_scale, float *out,
-                                void *stream) {
-    if (!c) return fail(TKV_ERR_INVALID, "cache is NULL");
-    if (!q || !out) return fail(TKV_ERR_INVALID, "NULL q or out");
-    if (!aligned16(q) || !aligned16(out)) return fail(TKV_ERR_INVALID, "q and out must be 16-byte aligned");
-    const long long ub = std::max(1ll, c->live_ub);
+namespace {
+// Decode attention over the cache with `ub` bounding every stream's live entries.
+tkv_status launch_decode(tkv_cache *c, const void *q, float softmax_scale, float *out, long long ub,
+                         cudaStream_t st, const char *what) {
     cudaError_t e;
     const bool persistent = c->cfg.dense == 1 &&
                             (c->cfg.attn_kernel != 0 || (c->cfg.codec == 0 && tkv::warp_tile_underfills(c->dev, ub)));
@@ -285,16 +283,42 @@ tkv_status tkv_decode_attention(tkv_cache *c, const void *q, float softmax_scale
         const tkv_status ms = ensure_maps(c);
         if (ms != TKV_OK) return ms;
         if (c->cfg.attn_kernel == 1)
-            e = tkv::launch_attention_i8(c->dev, c->maps, q, softmax_scale, out, nullptr, nullptr, 0.f, 0.f, ub,
-                                         static_cast<cudaStream_t>(stream), &c->launches);
-        else
-            e = tkv::launch_attention_ws(c->dev, c->maps, q, softmax_scale, out, ub, static_cast<cudaStream_t>(stream),
+            e = tkv::launch_attention_i8(c->dev, c->maps, q, softmax_scale, out, nullptr, nullptr, 0.f, 0.f, ub, st,
                                          &c->launches);
+        else
+            e = tkv::launch_attention_ws(c->dev, c->maps, q, softmax_scale, out, ub, st, &c->launches);
     } else {
-        e = tkv::launch_attention(c->dev, q, softmax_scale, out, ub, static_cast<cudaStream_t>(stream),
-                                  &c->launches);
+        e = tkv::launch_attention(c->dev, q, softmax_scale, out, ub, st, &c->launches);
     }
-    return cuda_status(e, "tkv_decode_attention");
+    return cuda_status(e, what);
+}
+}  // namespace
+
+tkv_status tkv_decode_attention(tkv_cache *c, const void *q, float softmax_scale, float *out,
+                                void *stream) {
+    if (!c) return fail(TKV_ERR_INVALID, "cache is NULL");
+    if (!q || !out) return fail(TKV_ERR_INVALID, "NULL q or out");
+    if (!aligned16(q) || !aligned16(out)) return fail(TKV_ERR_INVALID, "q and out must be 16-byte aligned");
+    const long long ub = std::max(1ll, c->live_ub);
+    return launch_decode(c, q, softmax_scale, out, ub, static_cast<cudaStream_t>(stream), "tkv_decode_attention");
+}
+
+tkv_status tkv_decode_step(tkv_cache *c, const void *k, const void *v, const uint8_t *cls, const int32_t *pos,
+                           const void *q, float softmax_scale, float *out, void *stream) {
+    if (!c) return fail(TKV_ERR_INVALID, "cache is NULL");
+    if (!k || !v || !cls || !pos) return fail(TKV_ERR_INVALID, "NULL input pointer");
+    if (!q || !out) return fail(TKV_ERR_INVALID, "NULL q or out");
+    if (!aligned16(k) || !aligned16(v)) return fail(TKV_ERR_INVALID, "k and v must be 16-byte aligned");
+    if (!aligned16(pos)) return fail(TKV_ERR_INVALID, "pos must be 16-byte aligned");
+    if (!aligned16(q) || !aligned16(out)) return fail(TKV_ERR_INVALID, "q and out must be 16-byte aligned");
+    // the append, then the attention, whose launch overlaps the append's (programmatic
+    // dependent launch); one launch with the append inside the attention kernel measured
+    // slower in every arrangement tried
+    auto st = static_cast<cudaStream_t>(stream);
+    const cudaError_t e = tkv::launch_append(c->dev, k, v, cls, pos, 1, st, &c->launches);
+    c->live_ub = std::min<long long>(c->dev.ncap, c->live_ub + 1);
+    if (e != cudaSuccess) return cuda_status(e, "tkv_decode_step");
+    return launch_decode(c, q, softmax_scale, out, std::max(1ll, c->live_ub), st, "tkv_decode_step");
 }
 
 tkv_status tkv_decode_attention_sparsity(tkv_cache *c, const void *q, float softmax_scale, float *out,

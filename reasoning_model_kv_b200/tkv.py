@@ -51,7 +51,7 @@ EXPORTS = ["tkv_workspace_bytes", "tkv_create", "tkv_destroy", "tkv_reset", "tkv
            "tkv_quantize_append", "tkv_quantize_append_noalloc", "tkv_decode_attention", "tkv_evict_compact", "tkv_poll_error",
            "tkv_export_state", "tkv_import_state", "tkv_launch_count", "tkv_last_error_string",
            "tkv_selftest_wait_timeout", "tkv_evict_segments", "tkv_tbe_schedule",
-           "tkv_evict_tam", "tkv_evict_compact_window", "tkv_decode_attention_sparsity"]
+           "tkv_evict_tam", "tkv_evict_compact_window", "tkv_decode_attention_sparsity", "tkv_decode_step"]
 
 _lib = None
 
@@ -76,6 +76,7 @@ def lib() -> ctypes.CDLL:
     L.tkv_quantize_append.argtypes = [vp, vp, vp, vp, vp, i32, vp]
     L.tkv_quantize_append_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, vp]
     L.tkv_decode_attention.argtypes = [vp, vp, ctypes.c_float, vp, vp]
+    L.tkv_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp]
     L.tkv_decode_attention_sparsity.argtypes = [vp, vp, ctypes.c_float, vp, vp, vp, ctypes.c_float,
                                                 ctypes.c_float, vp]
     L.tkv_decode_attention_sparsity.restype = ctypes.c_int
@@ -98,7 +99,7 @@ def lib() -> ctypes.CDLL:
     L.tkv_last_error_string.restype = ctypes.c_char_p
     for name in ("tkv_create", "tkv_destroy", "tkv_reset", "tkv_get_layout", "tkv_quantize_append",
                  "tkv_quantize_append_noalloc",
-                 "tkv_decode_attention", "tkv_evict_compact", "tkv_poll_error", "tkv_export_state",
+                 "tkv_decode_attention", "tkv_decode_step", "tkv_evict_compact", "tkv_poll_error", "tkv_export_state",
                  "tkv_import_state"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
@@ -214,6 +215,25 @@ class TkvCache:
         _check(lib().tkv_decode_attention(self._h, _dptr(q, torch.bfloat16, "q"),
                                           float(softmax_scale), _dptr(out, torch.float32, "out"),
                                           _stream(stream)))
+        return out
+
+    def decode_step(self, k: torch.Tensor, v: torch.Tensor, cls: torch.Tensor, pos: torch.Tensor,
+                    q: torch.Tensor, softmax_scale: float, out: torch.Tensor | None = None,
+                    stream=None) -> torch.Tensor:
+        """One decode step with its new token: quantize_append of k, v [B, Hkv, 128] (cls,
+        pos [B]) followed by decode_attention of q, in one call."""
+        if k.shape != (self.B, self.Hkv, 128) or v.shape != k.shape:
+            raise TkvError(TKV_ERR_INVALID, f"k/v must be [B, Hkv, 128], got {tuple(k.shape)}")
+        if cls.shape != (self.B,) or pos.shape != (self.B,):
+            raise TkvError(TKV_ERR_INVALID, "cls/pos must be [B]")
+        if q.shape != (self.B, self.Hkv * self.G, 128):
+            raise TkvError(TKV_ERR_INVALID, f"q must be [B, Hkv*G, 128], got {tuple(q.shape)}")
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+        _check(lib().tkv_decode_step(self._h, _dptr(k, torch.bfloat16, "k"), _dptr(v, torch.bfloat16, "v"),
+                                     _dptr(cls, torch.uint8, "cls"), _dptr(pos, torch.int32, "pos"),
+                                     _dptr(q, torch.bfloat16, "q"), float(softmax_scale),
+                                     _dptr(out, torch.float32, "out"), _stream(stream)))
         return out
 
     def decode_attention_sparsity(self, q: torch.Tensor, softmax_scale: float, th_r: float = 0.5,
@@ -374,6 +394,10 @@ def tkv_quantize_append(cache: TkvCache, k, v, cls, pos, stream=None):
 
 def tkv_decode_attention(cache: TkvCache, q, softmax_scale, out=None, stream=None):
     return cache.decode_attention(q, softmax_scale, out, stream)
+
+
+def tkv_decode_step(cache: TkvCache, k, v, cls, pos, q, softmax_scale, out=None, stream=None):
+    return cache.decode_step(k, v, cls, pos, q, softmax_scale, out, stream)
 
 
 def tkv_evict_compact(cache: TkvCache, budget, stream=None):

@@ -90,6 +90,16 @@ def test_calls_reject_bad_arguments_without_launching():
     assert L.tkv_quantize_append(h, ctypes.c_void_p((1 << 24) + 8), p, p, p, 1, None) == INV
     assert L.tkv_decode_attention(h, None, 0.1, p, None) == INV
     assert L.tkv_decode_attention(h, p, 0.1, ctypes.c_void_p((1 << 24) + 4), None) == INV
+    odd = ctypes.c_void_p((1 << 24) + 8)
+    assert L.tkv_decode_step(None, p, p, p, p, p, 0.1, p, None) == INV
+    for i in range(6):                                   # each NULL pointer, in argument order
+        args = [p] * 6
+        args[i] = None
+        assert L.tkv_decode_step(h, *args[:5], 0.1, args[5], None) == INV, i
+    for i in (0, 1, 3, 4, 5):                            # k, v, pos, q, out must be 16-byte aligned
+        args = [p] * 6
+        args[i] = odd
+        assert L.tkv_decode_step(h, *args[:5], 0.1, args[5], None) == INV, i
     assert L.tkv_evict_compact(h, -1, None) == INV
     assert L.tkv_evict_compact(None, 3, None) == INV
     assert L.tkv_selftest_wait_timeout(None, 1000, None) == INV
