@@ -89,10 +89,9 @@ typedef struct {
                             i) and decode reads them as whole blocks.  Results
                             are identical in both modes.                      */
     int32_t attn_kernel; /* decode-attention kernel: 0 = warp-tile kernel
-                            (mma.sync fragments, either placement; with dense
-                            placement and few long streams -- fewer than 2
-                            CTAs per SM at 8 per stream, 32k+ entries -- it
-                            runs on the persistent pipeline of 2);
+                            (mma.sync fragments, either placement; a few long
+                            streams are each split over more CTAs than a
+                            cluster holds and merged by a second pass);
                             1 = tensor-core kernel (tcgen05 MMAs with integer
                             operands: exact code products, accumulators in
                             tensor memory; persistent, one CTA per SM with the

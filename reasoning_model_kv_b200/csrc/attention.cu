@@ -10,7 +10,11 @@
 // and cuts it into class-homogeneous tiles (16 records; 8 for bf16).  Warp w
 // computes tiles w, w+4, w+8, ... with its own online-softmax state, so the warps
 // of a CTA run through the class loops (and their code) together.  C is picked on
-// the host so that the whole grid is resident (C = 1 for many streams).
+// the host so that the whole grid is resident (C = 1 for many streams).  When even
+// clusters of 8 would leave SMs idle (a few long streams), a stream gets as many CTAs
+// as fill the grid (at least 1024 entries each, and 16 or more) without a cluster: each
+// writes its partial (m, l, O) and the merge + score pass of the persistent kernels
+// finishes.
 //
 // Memory path.  Each warp stages its tiles in a 3-deep shared-memory ring: with
 // dense placement one bulk copy per tile (the records are contiguous; completion
@@ -44,7 +48,10 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
+
 #include "attn_tile.cuh"
+#include "persist.cuh"
 
 namespace tkv {
 namespace {
@@ -63,6 +70,7 @@ constexpr int kThreads = 32 * kWarps;
 constexpr int kStages = 3;
 constexpr int kStageBytes = 16 * 288;   // the largest tile: 16 int8 records (rows unpadded, swizzled)
 constexpr int kRingBytes = kWarps * kStages * kStageBytes;
+constexpr int kSplitTokens = 1024;   // fewest entries per CTA of a stream split beyond a cluster
 
 // Record bytes, reuse-placement stage row stride and rows per tile of class C_ under
 // codec CODEC.  Int8 rows (codec 0) are unpadded and chunk-swizzled on odd rows (SWZ);
@@ -128,11 +136,14 @@ __device__ __forceinline__ void issue_tile_dense(uint8_t *stage_ptr, uint32_t st
     }
 }
 
+// split: C CTAs per stream without a cluster (more than one holds); each writes its
+// partial (m, l, O) to slot s C + rank and the merge + score pass of the persistent
+// kernels (attn_finalize_kernel) completes the stream.
 template <int G, bool DENSE, int CODEC>
 __global__ void __launch_bounds__(kThreads, TKV_ATTN_MIN_BLOCKS) attn_kernel(const __grid_constant__ Dev d,
                                                            const __nv_bfloat16 *__restrict__ q,
                                                            float xscale, float *__restrict__ out,
-                                                           int C) {
+                                                           int C, int split) {
     extern __shared__ __align__(128) uint8_t ring[];   // kRingBytes, dynamic
     __shared__ float cta_m[kMaxG], cta_l[kMaxG];
     __shared__ float fac[kMaxCluster][kMaxG];     // exp2(m_j - M) per warp / peer rank and head
@@ -368,6 +379,22 @@ __global__ void __launch_bounds__(kThreads, TKV_ATTN_MIN_BLOCKS) attn_kernel(con
     }
     __syncthreads();
 
+    // ---- split: this CTA's partial of the stream for the merge + score pass
+    if (split) {
+        float *pp = d.part + (size_t)(s * C + rank) * part_floats(G);
+        if (tid < G) {
+            pp[tid] = cta_m[tid];
+            pp[G + tid] = cta_l[tid];
+            pp[2 * G + tid] = 0.f;
+        }
+        for (int idx = tid; idx < G * kD; idx += kThreads) pp[3 * G + idx] = co[idx];
+        if (rank == 0 && tid == 0) {   // the stream's partial slots: s + c_lo .. s + c_hi
+            d.seg_lo[s] = s * (C - 1);
+            d.seg_hi[s] = s * (C - 1) + C - 1;
+        }
+        return;
+    }
+
     // ---- cluster merge: global (M, L) per head; this rank writes its output slice
     float *orow = out + ((size_t)b * d.Hkv * G + (size_t)kvh * G) * kD;
     if (C == 1) {
@@ -425,44 +452,43 @@ cudaError_t launch_g(const Dev &d, const void *q, float scale, float *out, long 
     if (e0 != cudaSuccess) return e0;
     // Largest cluster (<= 8) whose grid is fully resident, never splitting a stream
     // below ~128 tokens per CTA; one CTA per stream when the streams fill the GPU.
+    // Few long streams (the clusters would leave SMs idle): as many CTAs per stream as
+    // fill the resident grid, at least kSplitTokens entries each, merged by a second pass,
+    // once that is at least twice a cluster.
     const long long slots = (long long)bps * sms;
     long long C = slots / d.S;
-    if (C > kMaxCluster) C = kMaxCluster;
-    if (C > live_ub / 128) C = live_ub / 128;
-    if (C < 1) C = 1;
+    const long long c_split = std::min<long long>({C, live_ub / kSplitTokens, 2ll * (d.S + kNctaMax) / d.S});
+    const bool split = c_split >= 2 * kMaxCluster;   // (a few more CTAs do not pay for the second pass)
+    if (split) {
+        C = c_split;
+    } else {
+        if (C > kMaxCluster) C = kMaxCluster;
+        if (C > live_ub / 128) C = live_ub / 128;
+        if (C < 1) C = 1;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)C, (unsigned)d.S, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = kRingBytes;
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)C;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // overlap the launch with the kernel before
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // overlap the launch with the kernel before
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = (unsigned)C;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 2;
+    cfg.numAttrs = split ? 1 : 2;
     const float xscale = scale * 1.4426950408889634f;   // logits in the log2 domain
     cudaError_t e = cudaLaunchKernelEx(&cfg, attn_kernel<G, DENSE, CODEC>, d, static_cast<const __nv_bfloat16 *>(q),
-                                       xscale, out, (int)C);
+                                       xscale, out, (int)C, (int)split);
     *launches += 1;
-    return e;
+    if (e != cudaSuccess || !split) return e;
+    return launch_finalize<G, false, 1>(d, out, nullptr, nullptr, 0.f, 0.f, (int)(d.S * C), live_ub, st, launches);
 }
 
 }  // namespace
-
-bool warp_tile_underfills(const Dev &d, long long live_ub) {
-    // the warp-tile kernel gives a stream at most kMaxCluster CTAs; with few long streams
-    // that leaves most of the GPU idle, where the persistent pipeline (every SM, an equal
-    // share of the bytes) is faster: fewer CTAs than two per SM and at least 32k entries
-    // in the longest stream
-    if (live_ub < 32768) return false;
-    int sms = 0;
-    if (device_sm_count(&sms) != cudaSuccess || sms <= 0) return false;
-    return (long long)d.S * kMaxCluster < 2ll * sms;
-}
 
 cudaError_t launch_attention(const Dev &d, const void *q, float scale, float *out, long long live_ub,
                              cudaStream_t st, int64_t *launches) {

@@ -431,17 +431,31 @@ __global__ void __launch_bounds__(256) attn_finalize_kernel(const __grid_constan
         }
     }
     __syncthreads();
-    if (split == 0) {
-        for (int i = tid; i < G * kD; i += 256) {
-            const int h = i / kD;
+    // the output: the stream's G x 128 elements spread over its nsplit CTAs, each element's
+    // partials summed by kSub threads (partials sub, sub + kSub, ...) and then reduced over
+    // those threads (a fixed order, so the result does not depend on timing)
+    {
+        constexpr int kSub = 16;
+        const int E = G * kD, per = (E + nsplit - 1) / nsplit;
+        const int e_lo = split * per, e_hi = min(E, e_lo + per);
+        const int sub = tid % kSub;
+        for (int base = e_lo; base < e_hi; base += 256 / kSub) {
+            const int i = base + tid / kSub;
+            const int h = (i < e_hi ? i : e_lo) / kD;
             float acc = 0.f;
-            for (int j = 0; j < nparts; ++j) {
-                const float *pp = part0 + (size_t)j * part_floats(G);
-                const float f = j < kParts ? fac[j][h] : (pp[G + h] > 0.f ? ex2(pp[h] - gM[h]) : 0.f);
-                if (f > 0.f) acc = fmaf(f, pp[3 * G + i], acc);
+            if (i < e_hi) {
+                for (int j = sub; j < nparts; j += kSub) {
+                    const float *pp = part0 + (size_t)j * part_floats(G);
+                    const float f = j < kParts ? fac[j][h] : (pp[G + h] > 0.f ? ex2(pp[h] - gM[h]) : 0.f);
+                    if (f > 0.f) acc = fmaf(f, pp[3 * G + i], acc);
+                }
             }
-            orow[i] = acc * gInvL[h];
+#pragma unroll
+            for (int o = kSub / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
+            if (sub == 0 && i < e_hi) orow[i] = acc * gInvL[h];
         }
+    }
+    if (split == 0) {
         if (STATS && tid < G) {
             if (sparsity) sparsity[(size_t)s * G + tid] = gH[tid];
             if (thought) thought[(size_t)s * G + tid] = (uint8_t)(gH[tid] >= th_t ? 3 : gH[tid] >= th_r ? 1 : 2);

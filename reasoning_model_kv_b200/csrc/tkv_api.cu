@@ -277,9 +277,7 @@ namespace {
 tkv_status launch_decode(tkv_cache *c, const void *q, float softmax_scale, float *out, long long ub,
                          cudaStream_t st, const char *what) {
     cudaError_t e;
-    const bool persistent = c->cfg.dense == 1 &&
-                            (c->cfg.attn_kernel != 0 || (c->cfg.codec == 0 && tkv::warp_tile_underfills(c->dev, ub)));
-    if (persistent) {
+    if (c->cfg.attn_kernel != 0) {   // the persistent kernels (dense placement)
         const tkv_status ms = ensure_maps(c);
         if (ms != TKV_OK) return ms;
         if (c->cfg.attn_kernel == 1)

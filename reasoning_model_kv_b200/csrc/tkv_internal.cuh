@@ -111,10 +111,6 @@ cudaError_t launch_append(const Dev &d, const void *k, const void *v, const uint
                           const int32_t *pos, int T, cudaStream_t st, int64_t *launches);
 cudaError_t launch_attention(const Dev &d, const void *q, float scale, float *out,
                              long long live_ub, cudaStream_t st, int64_t *launches);
-// True when the warp-tile kernel's per-stream clusters would leave most SMs idle (few
-// long streams): dense integer-code caches with attn_kernel 0 then run the same tile math
-// on the persistent pipeline (launch_attention_ws).
-bool warp_tile_underfills(const Dev &d, long long live_ub);
 // Dense placement: the tensor-core kernel with integer operands (attention_i8.cu).  With
 // sparsity / thought non-NULL it also writes, per (stream, query head), the attention
 // sparsity 1 - H(p) / ln N and its thought class under the thresholds th_r <= th_t.

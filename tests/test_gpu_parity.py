@@ -125,6 +125,20 @@ def test_gqa_widths_and_windows(G, n_protect, outliers, mode):
     _decode_step(w, gpu, o, rows, 1)
 
 
+@pytest.mark.parametrize("mode,codec", [("reuse", 0), ("dense", 0), ("reuse", 1), ("dense", 1)])
+@pytest.mark.parametrize("G", [4, 8])
+def test_few_long_streams_split_beyond_a_cluster(G, mode, codec):
+    """Two 24k-token streams: the warp-tile kernel gives each stream more CTAs than a
+    cluster holds (23 here) and a second pass merges their partials and adds the scores;
+    a ragged tail (24000 + 1 entries) and a step after an eviction to 3000 (8 CTAs: the
+    cluster path again)."""
+    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", B=1, Hq=2 * G, Hkv=2, ctx=24000, n_protect=4,
+                                 outliers=True, steps=2, codec=codec, **MODES[mode])
+    _decode_step(w, gpu, o, rows, 0)
+    _evict_lockstep(gpu, o, rows, 3000)
+    _decode_step(w, gpu, o, rows, 1)
+
+
 @pytest.mark.parametrize("dense", [False, True], ids=["reuse", "dense"])
 def test_multi_token_append_after_eviction_reuses_slots_in_order(dense):
     w, gpu, o, rows = build_pair("tiny_b1_ctx2k", ctx=600, steps=80, dense=dense)
