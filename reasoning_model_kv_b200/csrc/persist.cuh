@@ -473,6 +473,8 @@ __global__ void __launch_bounds__(256) attn_finalize_kernel(const __grid_constan
 template <int G, bool STATS, int SPC>
 cudaError_t launch_finalize(const Dev &d, float *out, float *sparsity, uint8_t *thought, float th_r, float th_t,
                             int ncta, long long live_ub, cudaStream_t st, int64_t *launches) {
+    // about 4096 entries per CTA of the score pass, at most 64 CTAs per stream (more CTAs
+    // than one resident wave measured slower: each is bound by its own latencies)
     const int nsplit = (int)(live_ub < 4096 ? 1 : live_ub >= 64ll * 4096 ? 64 : (live_ub + 4095) / 4096);
     cudaLaunchConfig_t cf = {};
     cf.gridDim = dim3((unsigned)d.S, (unsigned)nsplit, 1);
