@@ -365,7 +365,7 @@ __device__ __forceinline__ void prefetch_maps(const I8Maps &maps) {
 // l = 0), writes O and the sparsity statistic, then adds p = 2^(x - M) / L to the scores
 // of its slice.
 template <int G, bool STATS, int SPC>
-__global__ void __launch_bounds__(256) attn_finalize_kernel(const __grid_constant__ Dev d, float *__restrict__ out,
+__global__ void __launch_bounds__(256, 4) attn_finalize_kernel(const __grid_constant__ Dev d, float *__restrict__ out,
                                                             float *__restrict__ sparsity,
                                                             uint8_t *__restrict__ thought, float th_r, float th_t,
                                                             int ncta) {
@@ -432,27 +432,28 @@ __global__ void __launch_bounds__(256) attn_finalize_kernel(const __grid_constan
     }
     __syncthreads();
     // the output: the stream's G x 128 elements spread over its nsplit CTAs, each element's
-    // partials summed by kSub threads (partials sub, sub + kSub, ...) and then reduced over
-    // those threads (a fixed order, so the result does not depend on timing)
+    // partials summed by sub threads (partials j, j + sub, ...; sub = the power of two that
+    // leaves each thread at most 4, up to 16) and then reduced over those threads (a fixed
+    // order, so the result does not depend on timing)
     {
-        constexpr int kSub = 16;
+        int sub = 1;
+        while (sub < 16 && sub * 4 < nparts) sub *= 2;
         const int E = G * kD, per = (E + nsplit - 1) / nsplit;
         const int e_lo = split * per, e_hi = min(E, e_lo + per);
-        const int sub = tid % kSub;
-        for (int base = e_lo; base < e_hi; base += 256 / kSub) {
-            const int i = base + tid / kSub;
+        const int k = tid % sub;
+        for (int base = e_lo; base < e_hi; base += 256 / sub) {
+            const int i = base + tid / sub;
             const int h = (i < e_hi ? i : e_lo) / kD;
             float acc = 0.f;
             if (i < e_hi) {
-                for (int j = sub; j < nparts; j += kSub) {
+                for (int j = k; j < nparts; j += sub) {
                     const float *pp = part0 + (size_t)j * part_floats(G);
                     const float f = j < kParts ? fac[j][h] : (pp[G + h] > 0.f ? ex2(pp[h] - gM[h]) : 0.f);
                     if (f > 0.f) acc = fmaf(f, pp[3 * G + i], acc);
                 }
             }
-#pragma unroll
-            for (int o = kSub / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
-            if (sub == 0 && i < e_hi) orow[i] = acc * gInvL[h];
+            for (int o = sub / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
+            if (k == 0 && i < e_hi) orow[i] = acc * gInvL[h];
         }
     }
     if (split == 0) {
@@ -473,9 +474,10 @@ __global__ void __launch_bounds__(256) attn_finalize_kernel(const __grid_constan
 template <int G, bool STATS, int SPC>
 cudaError_t launch_finalize(const Dev &d, float *out, float *sparsity, uint8_t *thought, float th_r, float th_t,
                             int ncta, long long live_ub, cudaStream_t st, int64_t *launches) {
-    // about 4096 entries per CTA of the score pass, at most 64 CTAs per stream (more CTAs
-    // than one resident wave measured slower: each is bound by its own latencies)
-    const int nsplit = (int)(live_ub < 4096 ? 1 : live_ub >= 64ll * 4096 ? 64 : (live_ub + 4095) / 4096);
+    // about 2048 entries per CTA of the score pass, at most 64 CTAs per stream (four
+    // resident per SM; more CTAs than one resident wave measured slower: each is bound by
+    // its own latencies)
+    const int nsplit = (int)(live_ub < 2048 ? 1 : live_ub >= 64ll * 2048 ? 64 : (live_ub + 2047) / 2048);
     cudaLaunchConfig_t cf = {};
     cf.gridDim = dim3((unsigned)d.S, (unsigned)nsplit, 1);
     cf.blockDim = dim3(256, 1, 1);
