@@ -343,8 +343,20 @@ def run_tkv(args, rank, world, dev):
             gpu.decode_attention(q, SCALE, out)
             ea[i][1].record(st)
         torch.cuda.synchronize()
+        # (3) the same call with the attention-sparsity statistic (its cost over (2); the
+        #     persistent warp-tile pipeline does not form it)
+        es = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(n_attn if args.attn_kernel != "ws" else 0)]
+        for i in range(len(es)):
+            restore_post()
+            flush.zero_()
+            es[i][0].record(st)
+            gpu.decode_attention_sparsity(q, SCALE, 0.5, 0.7, out=out)
+            es[i][1].record(st)
+        torch.cuda.synchronize()
     step_ms = [a.elapsed_time(b2) for a, b2 in ev]
     attn_ms = [a.elapsed_time(b2) for a, b2 in ea]
+    sp_ms = [a.elapsed_time(b2) for a, b2 in es]
     t_step = sum(step_ms) / len(step_ms)
     t_attn = sum(attn_ms) / len(attn_ms)
     t_step, t_attn = reduce_max([t_step, t_attn], world, dev)
@@ -425,6 +437,8 @@ def run_tkv(args, rank, world, dev):
         "attention_ms_median": statistics.median(attn_ms),
         "attention_ms_min": min(attn_ms),
         "attention_timing": "attention call alone on the post-append cache (L2 flushed), CUDA events",
+        "sparsity_call_ms": statistics.median(sp_ms) if sp_ms else None,
+        "sparsity_overhead": statistics.median(sp_ms) / statistics.median(attn_ms) - 1.0 if sp_ms else None,
         "append_exposed_ms": t_step - t_attn,   # step minus the attention call timed alone
         "evict_ms_untimed_step": evict_ms,
         "full_context_phase": full,

@@ -251,9 +251,10 @@ TKV_API tkv_status tkv_decode_step(tkv_cache *cache, const void *k, const void *
  *   else 2 (Execution).
  *   sparsity  device fp32 [B][Hkv*G]  (required)
  *   thought   device uint8 [B][Hkv*G] (may be NULL)
- * Requires dense placement with attn_kernel = 1 (the statistic is formed by that
- * kernel's softmax); returns TKV_ERR_INVALID otherwise, for NULL q / out / sparsity,
- * unaligned pointers, or thresholds that are not finite with th_r <= th_t.
+ * Requires attn_kernel 0 (either placement; the score pass forms the statistic from the
+ * exp2(x - M) it computes anyway) or 1; returns TKV_ERR_INVALID with attn_kernel 2, for
+ * NULL q / out / sparsity, unaligned pointers, or thresholds that are not finite with
+ * th_r <= th_t.
  */
 TKV_API tkv_status tkv_decode_attention_sparsity(tkv_cache *cache, const void *q, float softmax_scale,
                                                  float *out, float *sparsity, uint8_t *thought, float th_r,

@@ -139,16 +139,20 @@ __device__ __forceinline__ void issue_tile_dense(uint8_t *stage_ptr, uint32_t st
 // split: C CTAs per stream without a cluster (more than one holds); each writes its
 // partial (m, l, O) to slot s C + rank and the merge + score pass of the persistent
 // kernels (attn_finalize_kernel) completes the stream.
-template <int G, bool DENSE, int CODEC>
+// STATS: also the attention sparsity 1 - H(p) / ln N of every (stream, query head) and its
+// thought class (tkv_decode_attention_sparsity), from the score pass's exp2(x - M).
+template <int G, bool DENSE, int CODEC, bool STATS>
 __global__ void __launch_bounds__(kThreads, TKV_ATTN_MIN_BLOCKS) attn_kernel(const __grid_constant__ Dev d,
                                                            const __nv_bfloat16 *__restrict__ q,
                                                            float xscale, float *__restrict__ out,
-                                                           int C, int split) {
+                                                           int C, int split, float *__restrict__ sparsity,
+                                                           uint8_t *__restrict__ thought, float th_r, float th_t) {
     extern __shared__ __align__(128) uint8_t ring[];   // kRingBytes, dynamic
     __shared__ float cta_m[kMaxG], cta_l[kMaxG];
     __shared__ float fac[kMaxCluster][kMaxG];     // exp2(m_j - M) per warp / peer rank and head
     __shared__ float gM[kMaxG], gInvL[kMaxG];
     __shared__ __align__(8) uint64_t bars[kWarps][kStages];   // dense placement only
+    __shared__ float se[kWarps][kMaxG], ce[kMaxG];   // STATS: entropy terms per warp, per CTA
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, tig = lane & 3;
@@ -379,13 +383,45 @@ __global__ void __launch_bounds__(kThreads, TKV_ATTN_MIN_BLOCKS) attn_kernel(con
     }
     __syncthreads();
 
+    // per-warp slots -> ce[h] (a fixed order): the CTA's sum of this thread's e[h], written
+    // by thread h (which alone reads it afterwards, or its peers after a cluster barrier)
+    auto cta_sum = [&](const float (&e)[G]) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            float v = e[h];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+            if (lane == 0) se[warp][h] = v;
+        }
+        __syncthreads();
+        if (tid < G) {
+            float v = 0.f;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) v += se[w][tid];
+            ce[tid] = v;
+        }
+    };
+
     // ---- split: this CTA's partial of the stream for the merge + score pass
     if (split) {
+        if constexpr (STATS) {
+            // e relative to this CTA's reference max, from the raw logits of its entries
+            float e[G];
+#pragma unroll
+            for (int h = 0; h < G; ++h) e[h] = 0.f;
+            for (int t = t0 + tid; t < t1; t += kThreads)
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    const float x = lgs[(size_t)t * G + h];
+                    e[h] = fmaf(exp2f(x - cta_m[h]), x - cta_m[h], e[h]);
+                }
+            cta_sum(e);
+        }
         float *pp = d.part + (size_t)(s * C + rank) * part_floats(G);
         if (tid < G) {
             pp[tid] = cta_m[tid];
             pp[G + tid] = cta_l[tid];
-            pp[2 * G + tid] = 0.f;
+            pp[2 * G + tid] = STATS ? ce[tid] : 0.f;
         }
         for (int idx = tid; idx < G * kD; idx += kThreads) pp[3 * G + idx] = co[idx];
         if (rank == 0 && tid == 0) {   // the stream's partial slots: s + c_lo .. s + c_hi
@@ -432,23 +468,40 @@ __global__ void __launch_bounds__(kThreads, TKV_ATTN_MIN_BLOCKS) attn_kernel(con
     }
 
     // ---- scores of this CTA's tokens: += sum_h exp2(x - M_h) / L_h (none if the stream is empty)
-    if (N > 0) {
-        add_scores<G, kThreads>(d, s, lgs, t0, t1, o1, o2, o3, gM, gInvL, tid);
-
+    float e[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) e[h] = 0.f;
+    if (N > 0) add_scores<G, kThreads, STATS>(d, s, lgs, t0, t1, o1, o2, o3, gM, gInvL, tid, e);
+    if constexpr (STATS) {
+        // the stream's entropy term: this CTA's, plus its peers' over DSMEM (rank 0 writes)
+        cta_sum(e);
+        if (C > 1) cluster_sync();
+        if (rank == 0 && tid < G) {
+            float E = 0.f;
+            if (C == 1) E = ce[tid];
+            else
+                for (int j = 0; j < C; ++j) E += dsmem_ld(dsmem_addr(ce + tid, (uint32_t)j));
+            const float L = gInvL[tid] > 0.f ? 1.f / gInvL[tid] : 0.f;
+            const float sp = sparsity_of(L, E, N);
+            sparsity[(size_t)s * G + tid] = sp;
+            if (thought) thought[(size_t)s * G + tid] = thought_of(sp, th_r, th_t);
+        }
     }
     if (C > 1) cluster_sync();   // peers may still be reading this CTA's shared memory
 }
 
-int g_blocks_per_sm[2][2][kMaxG + 1][kMaxDevices] = {};   // per codec, placement, G and device
+int g_blocks_per_sm[2][2][2][kMaxG + 1][kMaxDevices] = {};   // per codec, placement, stats, G and device
 
-template <int G, bool DENSE, int CODEC>
+template <int G, bool DENSE, int CODEC, bool STATS>
 cudaError_t launch_g(const Dev &d, const void *q, float scale, float *out, long long live_ub,
-                     cudaStream_t st, int64_t *launches) {
+                     cudaStream_t st, int64_t *launches, float *sparsity, uint8_t *thought, float th_r,
+                     float th_t) {
     int sms = 0, bps = 0;
     cudaError_t e0 = device_sm_count(&sms);
     if (e0 != cudaSuccess) return e0;
-    e0 = cached_blocks_per_sm(g_blocks_per_sm[CODEC][DENSE][G], reinterpret_cast<const void *>(attn_kernel<G, DENSE, CODEC>),
-                              kThreads, kRingBytes, &bps);
+    e0 = cached_blocks_per_sm(g_blocks_per_sm[CODEC][DENSE][STATS][G],
+                              reinterpret_cast<const void *>(attn_kernel<G, DENSE, CODEC, STATS>), kThreads, kRingBytes,
+                              &bps);
     if (e0 != cudaSuccess) return e0;
     // Largest cluster (<= 8) whose grid is fully resident, never splitting a stream
     // below ~128 tokens per CTA; one CTA per stream when the streams fill the GPU.
@@ -481,32 +534,41 @@ cudaError_t launch_g(const Dev &d, const void *q, float scale, float *out, long 
     cfg.attrs = attr;
     cfg.numAttrs = split ? 1 : 2;
     const float xscale = scale * 1.4426950408889634f;   // logits in the log2 domain
-    cudaError_t e = cudaLaunchKernelEx(&cfg, attn_kernel<G, DENSE, CODEC>, d, static_cast<const __nv_bfloat16 *>(q),
-                                       xscale, out, (int)C, (int)split);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, attn_kernel<G, DENSE, CODEC, STATS>, d,
+                                       static_cast<const __nv_bfloat16 *>(q), xscale, out, (int)C, (int)split,
+                                       sparsity, thought, th_r, th_t);
     *launches += 1;
     if (e != cudaSuccess || !split) return e;
-    return launch_finalize<G, false, 1>(d, out, nullptr, nullptr, 0.f, 0.f, (int)(d.S * C), live_ub, st, launches);
+    return launch_finalize<G, STATS, 1>(d, out, sparsity, thought, th_r, th_t, (int)(d.S * C), live_ub, st, launches);
 }
 
 }  // namespace
 
 cudaError_t launch_attention(const Dev &d, const void *q, float scale, float *out, long long live_ub,
-                             cudaStream_t st, int64_t *launches) {
+                             cudaStream_t st, int64_t *launches, float *sparsity, uint8_t *thought, float th_r,
+                             float th_t) {
     if (d.dense && d.attn_kernel != 0) return cudaErrorInvalidValue;   // the persistent kernels'
-#define TKV_G_CASES(DN, CD)                                                           \
-    switch (d.G) {                                                                    \
-        case 1: return launch_g<1, DN, CD>(d, q, scale, out, live_ub, st, launches);  \
-        case 2: return launch_g<2, DN, CD>(d, q, scale, out, live_ub, st, launches);  \
-        case 4: return launch_g<4, DN, CD>(d, q, scale, out, live_ub, st, launches);  \
-        case 8: return launch_g<8, DN, CD>(d, q, scale, out, live_ub, st, launches);  \
-        default: return cudaErrorInvalidValue;                                        \
+#define TKV_G_CASES(DN, CD, ST)                                                                              \
+    switch (d.G) {                                                                                           \
+        case 1: return launch_g<1, DN, CD, ST>(d, q, scale, out, live_ub, st, launches, sparsity, thought, th_r, th_t); \
+        case 2: return launch_g<2, DN, CD, ST>(d, q, scale, out, live_ub, st, launches, sparsity, thought, th_r, th_t); \
+        case 4: return launch_g<4, DN, CD, ST>(d, q, scale, out, live_ub, st, launches, sparsity, thought, th_r, th_t); \
+        case 8: return launch_g<8, DN, CD, ST>(d, q, scale, out, live_ub, st, launches, sparsity, thought, th_r, th_t); \
+        default: return cudaErrorInvalidValue;                                                               \
+    }
+    // one compound statement per (placement, codec): both switches return
+#define TKV_ST_CASES(DN, CD)                     \
+    {                                            \
+        if (sparsity) TKV_G_CASES(DN, CD, true)  \
+        TKV_G_CASES(DN, CD, false)               \
     }
     if (d.codec == 0) {
-        if (d.dense) TKV_G_CASES(true, 0)
-        TKV_G_CASES(false, 0)
+        if (d.dense) TKV_ST_CASES(true, 0)
+        TKV_ST_CASES(false, 0)
     }
-    if (d.dense) TKV_G_CASES(true, 1)
-    TKV_G_CASES(false, 1)
+    if (d.dense) TKV_ST_CASES(true, 1)
+    TKV_ST_CASES(false, 1)
+#undef TKV_ST_CASES
 #undef TKV_G_CASES
 }
 

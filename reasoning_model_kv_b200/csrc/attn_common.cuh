@@ -391,6 +391,18 @@ __device__ __forceinline__ void load_meta(const uint8_t *meta, float2 (&out)[4])
     out[3] = make_float2(s23.y, z23.y);
 }
 
+// The attention sparsity 1 - H(p) / ln N of one head (0 when N < 2) from the softmax sum
+// L = sum_t exp2(x_t - M) and e = sum_t exp2(x_t - M) (x_t - M) (x, M in log2 units):
+// H = ln L - ln 2 * e / L.  Its thought class: 3 (Transition) at or above th_t, else 1
+// (Reasoning) at or above th_r, else 2 (Execution).
+__device__ __forceinline__ float sparsity_of(float L, float e, int N) {
+    const float Hh = L > 0.f ? logf(L) - 0.6931471805599453f * e / L : 0.f;
+    return N > 1 ? 1.f - Hh / logf((float)N) : 0.f;
+}
+__device__ __forceinline__ uint8_t thought_of(float sp, float th_r, float th_t) {
+    return (uint8_t)(sp >= th_t ? 3 : sp >= th_r ? 1 : 2);
+}
+
 // Scores of this CTA's entries [t0, t1) of stream s: score += sum_h exp2(x_h - M_h) *
 // invL_h, x the step's raw logits (log2 domain, entry order, from the L2 scratch).
 // Entry t0 + k*NT + tid belongs to thread tid (coalesced), kPer of them per round
@@ -398,9 +410,12 @@ __device__ __forceinline__ void load_meta(const uint8_t *meta, float2 (&out)[4])
 // warp's 32 consecutive entries fill exactly G whole 128-byte scratch lines (a CTA's
 // range starts on a 32-entry boundary), so once the warp has its logits in registers
 // it drops those lines from L2 without write-back.
-template <int G, int NT>
+// STATS: e[h] (this thread's share) also accumulates sum_t exp2(x_t - M_h) (x_t - M_h), the
+// attention-entropy term H(p) = ln L - ln 2 * e / L of the sparsity statistic.
+template <int G, int NT, bool STATS = false>
 __device__ __forceinline__ void add_scores(const Dev &d, int s, const float *lgs, int t0, int t1, int o1, int o2,
-                                           int o3, const float *gM, const float *gInvL, int tid) {
+                                           int o3, const float *gM, const float *gInvL, int tid,
+                                           float *e = nullptr) {
     constexpr int kPer = G >= 8 ? 4 : G >= 4 ? 8 : 16;   // x[kPer][G] fits the registers
     const int lane = tid & 31;
     float Mh[G], Ih[G];
@@ -445,7 +460,11 @@ __device__ __forceinline__ void add_scores(const Dev &d, int s, const float *lgs
             if (t >= t1) continue;
             float inc = 0.f;
 #pragma unroll
-            for (int h = 0; h < G; ++h) inc += exp2f(x[k][h] - Mh[h]) * Ih[h];   // full-precision exp2
+            for (int h = 0; h < G; ++h) {
+                const float ex = exp2f(x[k][h] - Mh[h]);   // full-precision exp2
+                inc += ex * Ih[h];
+                if constexpr (STATS) e[h] = fmaf(ex, x[k][h] - Mh[h], e[h]);
+            }
             srow(t)[t] = sv[k] + inc;
         }
     }

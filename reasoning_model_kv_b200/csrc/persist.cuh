@@ -385,7 +385,7 @@ __global__ void __launch_bounds__(256, 4) attn_finalize_kernel(const __grid_cons
             for (int i = tid; i < G * kD; i += 256) orow[i] = 0.f;
             if (STATS && tid < G) {
                 if (sparsity) sparsity[(size_t)s * G + tid] = 0.f;
-                if (thought) thought[(size_t)s * G + tid] = (uint8_t)(0.f >= th_t ? 3 : 0.f >= th_r ? 1 : 2);
+                if (thought) thought[(size_t)s * G + tid] = thought_of(0.f, th_r, th_t);
             }
         }
         return;
@@ -425,9 +425,7 @@ __global__ void __launch_bounds__(256, 4) attn_finalize_kernel(const __grid_cons
         gM[tid] = M;
         gInvL[tid] = L > 0.f ? 1.f / L : 0.f;
         if (STATS) {
-            // H = ln L - ln 2 * sum p (x - M) / L  (x, M in log2 units)
-            const float Hh = L > 0.f ? logf(L) - 0.6931471805599453f * E / L : 0.f;
-            gH[tid] = N > 1 ? 1.f - Hh / logf((float)N) : 0.f;
+            gH[tid] = sparsity_of(L, E, N);
         }
     }
     __syncthreads();
@@ -459,7 +457,7 @@ __global__ void __launch_bounds__(256, 4) attn_finalize_kernel(const __grid_cons
     if (split == 0) {
         if (STATS && tid < G) {
             if (sparsity) sparsity[(size_t)s * G + tid] = gH[tid];
-            if (thought) thought[(size_t)s * G + tid] = (uint8_t)(gH[tid] >= th_t ? 3 : gH[tid] >= th_r ? 1 : 2);
+            if (thought) thought[(size_t)s * G + tid] = thought_of(gH[tid], th_r, th_t);
         }
     }
     // scores of this CTA's slice of the stream (slices start on 32-entry boundaries)

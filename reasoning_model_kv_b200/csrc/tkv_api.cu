@@ -327,13 +327,19 @@ tkv_status tkv_decode_attention_sparsity(tkv_cache *c, const void *q, float soft
     if ((reinterpret_cast<uintptr_t>(sparsity) & 3u) != 0) return fail(TKV_ERR_INVALID, "sparsity must be 4-byte aligned");
     if (!(th_r <= th_t) || !std::isfinite(th_r) || !std::isfinite(th_t))
         return fail(TKV_ERR_INVALID, "thresholds must be finite with th_r <= th_t");
-    if (!(c->cfg.dense == 1 && c->cfg.attn_kernel == 1))
-        return fail(TKV_ERR_INVALID, "the sparsity statistic needs dense placement and attn_kernel 1");
-    const tkv_status ms = ensure_maps(c);
-    if (ms != TKV_OK) return ms;
+    if (c->cfg.attn_kernel == 2)
+        return fail(TKV_ERR_INVALID, "the sparsity statistic needs attn_kernel 0 or 1");
     const long long ub = std::max(1ll, c->live_ub);
-    cudaError_t e = tkv::launch_attention_i8(c->dev, c->maps, q, softmax_scale, out, sparsity, thought, th_r, th_t,
-                                             ub, static_cast<cudaStream_t>(stream), &c->launches);
+    auto st = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (c->cfg.attn_kernel == 1) {
+        const tkv_status ms = ensure_maps(c);
+        if (ms != TKV_OK) return ms;
+        e = tkv::launch_attention_i8(c->dev, c->maps, q, softmax_scale, out, sparsity, thought, th_r, th_t, ub, st,
+                                     &c->launches);
+    } else {
+        e = tkv::launch_attention(c->dev, q, softmax_scale, out, ub, st, &c->launches, sparsity, thought, th_r, th_t);
+    }
     return cuda_status(e, "tkv_decode_attention_sparsity");
 }
 

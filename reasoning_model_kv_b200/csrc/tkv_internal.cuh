@@ -109,8 +109,11 @@ cudaError_t cached_blocks_per_sm(int *slot_per_device, const void *kernel, int t
 // of kernels it launched to *launches).
 cudaError_t launch_append(const Dev &d, const void *k, const void *v, const uint8_t *cls,
                           const int32_t *pos, int T, cudaStream_t st, int64_t *launches);
+// Warp-tile decode attention; with `sparsity` non-NULL it also writes, per (stream, query
+// head), the attention sparsity and (thought non-NULL) its thought class.
 cudaError_t launch_attention(const Dev &d, const void *q, float scale, float *out,
-                             long long live_ub, cudaStream_t st, int64_t *launches);
+                             long long live_ub, cudaStream_t st, int64_t *launches, float *sparsity = nullptr,
+                             uint8_t *thought = nullptr, float th_r = 0.f, float th_t = 0.f);
 // Dense placement: the tensor-core kernel with integer operands (attention_i8.cu).  With
 // sparsity / thought non-NULL it also writes, per (stream, query head), the attention
 // sparsity 1 - H(p) / ln N and its thought class under the thresholds th_r <= th_t.

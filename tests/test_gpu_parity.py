@@ -450,15 +450,23 @@ def test_extreme_magnitudes_sinks_and_query(mode):
 SPARSITY_ATOL = 2e-5
 
 
-@pytest.mark.parametrize("G,ctx,n_protect", [(4, 2000, 128), (8, 709, 4), (1, 3000, 0)])
-def test_attention_sparsity_statistic(G, ctx, n_protect):
+SPARSITY_MODES = {"warp_dense": dict(dense=True), "warp_reuse": dict(dense=False),
+                  "tc": dict(dense=True, attn_kernel=1)}
+
+
+@pytest.mark.parametrize("mode", list(SPARSITY_MODES))
+@pytest.mark.parametrize("G,ctx,n_protect,B,Hkv", [(4, 2000, 128, 2, 2), (8, 709, 4, 2, 2), (1, 3000, 0, 2, 2),
+                                                   (4, 24000, 4, 1, 2), (4, 300, 4, 40, 8)])
+def test_attention_sparsity_statistic(G, ctx, n_protect, B, Hkv, mode):
     """tkv_decode_attention_sparsity: the step's output and scores as in a plain decode
     call, plus per (stream, head) 1 - H(p) / ln N against the oracle's fp64 value and
     the thought class under the thresholds (ThinKV, Metodologia: thought types differ in
-    the sparsity of their attention)."""
-    rows = [0, 1]
-    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", rows=rows, B=2, Hq=2 * G, Hkv=2, ctx=ctx, n_protect=n_protect,
-                                 steps=2, dense=True, attn_kernel=1)
+    the sparsity of their attention).  The warp-tile kernel's three layouts: clusters
+    (4 streams), the split with the merge pass (2 streams of 24k) and one CTA per stream
+    (320 streams)."""
+    rows = [0, 1] if B > 1 else [0]
+    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", rows=rows, B=B, Hq=Hkv * G, Hkv=Hkv, ctx=ctx,
+                                 n_protect=n_protect, steps=2, **SPARSITY_MODES[mode])
     k, v, cls, pos, q = synth.decode_inputs(w, 0)
     sub = rows_streams(gpu, rows)
     o.load_state(gpu.export_state(sub))
@@ -480,15 +488,16 @@ def test_attention_sparsity_statistic(G, ctx, n_protect):
     assert gpu.poll_error() == tkv.TKV_OK
 
 
-def test_attention_sparsity_needs_the_tensor_core_kernel():
-    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", B=1, dense=True)
+def test_attention_sparsity_rejects_the_persistent_pipeline_and_bad_thresholds():
+    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", B=1, dense=True, attn_kernel=2)
     q = synth.decode_inputs(w, 0)[4].to(DEV)
     with pytest.raises(TkvError):
         gpu.decode_attention_sparsity(q, SCALE)
-    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", B=1, dense=True, attn_kernel=1)
-    q = synth.decode_inputs(w, 0)[4].to(DEV)
-    with pytest.raises(TkvError):
-        gpu.decode_attention_sparsity(q, SCALE, 0.8, 0.2)   # th_r > th_t
+    for kernel in (0, 1):
+        w, gpu, o, rows = build_pair("tiny_b1_ctx2k", B=1, dense=True, attn_kernel=kernel)
+        q = synth.decode_inputs(w, 0)[4].to(DEV)
+        with pytest.raises(TkvError):
+            gpu.decode_attention_sparsity(q, SCALE, 0.8, 0.2)   # th_r > th_t
 
 
 
