@@ -170,10 +170,17 @@ __global__ void __launch_bounds__(kThreads, TKV_ATTN_MIN_BLOCKS) attn_kernel(con
     //      each (group, head) scaled by a power of two when its largest |q| lies
     //      outside [2^-10, 2^14) so that f16 neither overflows nor goes subnormal on
     //      it; qinv holds the inverse scale of heads 2tig, 2tig+1 per group.
-    uint32_t qb[4][2][2], qbb[4][2][2];
+    //      One copy lives through the tile loops: qf holds the raw pairs while the bf16
+    //      tiles (the first class loop) run, then the scaled f16 pairs.
+    uint32_t qf[4][2][2];
     float qs[2][4], qinv[2][4];
     bool qscaled;
-    query_frags<G>(q + ((size_t)b * d.Hkv * G + (size_t)kvh * G) * kD, lane, qb, qbb, qs, qinv, qscaled);
+    uint32_t scexp;
+    {
+        uint32_t qb_unused[4][2][2];
+        query_frags<G>(q + ((size_t)b * d.Hkv * G + (size_t)kvh * G) * kD, lane, qb_unused, qf, qs, qinv, qscaled,
+                       &scexp);
+    }
 
     // ---- this CTA's entry range and its tiles (class by class)
     const int n0 = dclamp(d.err, d.n[s * 4 + 0], d.cap[0], kDbgAttention + 0);
@@ -310,12 +317,13 @@ __global__ void __launch_bounds__(kThreads, TKV_ATTN_MIN_BLOCKS) attn_kernel(con
         constexpr int FMT_ = (CLS) > 0 ? CODEC : 0;                                          \
         const RowLoader<BITS, (DENSE ? CS::REC : CS::STRIDE), (!DENSE && CS::SWZ), FMT_> ldr(   \
             ring + (warp * kStages + stage) * kStageBytes, lane >> 2);                        \
-        tile_compute<BITS, CS::ROWS, G, FMT_>(ldr, nr, lane, qb, qbb, qs, qinv, qscaled, xscale, ws, \
+        tile_compute<BITS, CS::ROWS, G, FMT_>(ldr, nr, lane, qf, qf, qs, qinv, qscaled, xscale, ws, \
                                               lgs + (size_t)((OFF) + e) * G, magic);          \
         __syncwarp();                                                                         \
         stage = stage == 2 ? 0 : stage + 1;                                                   \
     }
     TKV_CONSUME(0, 16, 0, p1, lo0, hi0, 0)
+    query_to_f16(qf, scexp);   // the code classes take the scaled f16 query
     TKV_CONSUME(1, 8, p1, p2, lo1, hi1, o1)
     TKV_CONSUME(2, 4, p2, p3, lo2, hi2, o2)
     TKV_CONSUME(3, 2, p3, p4, lo3, hi3, o3)

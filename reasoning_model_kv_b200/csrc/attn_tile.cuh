@@ -227,10 +227,12 @@ __device__ __forceinline__ void tile_compute(const Loader &ld, int nr, int lane,
 // when its largest |q| lies outside [2^-10, 2^14), so that f16 neither overflows nor goes
 // subnormal on it; qinv: the inverse scales of heads 2 tig, 2 tig + 1 per group; qs: the
 // group sums of q (for the zero term); qscaled: any scale differs from 1.
+// scexp (optional): the biased exponents of this lane's own four group scales (head g),
+// one byte per group, for query_to_f16 below.
 template <int G>
 __device__ __forceinline__ void query_frags(const __nv_bfloat16 *__restrict__ qh, int lane, uint32_t (&qb)[4][2][2],
                                             uint32_t (&qbb)[4][2][2], float (&qs)[2][4], float (&qinv)[2][4],
-                                            bool &qscaled) {
+                                            bool &qscaled, uint32_t *scexp = nullptr) {
     const int g = lane >> 2, tig = lane & 3;
     {
         float qsg[4], qsc[4];
@@ -268,6 +270,7 @@ __device__ __forceinline__ void query_frags(const __nv_bfloat16 *__restrict__ qh
                 any = true;
             }
             qsc[grp] = sc;
+            if (scexp) *scexp = (grp == 0 ? 0u : *scexp) | (((__float_as_uint(sc) >> 23) & 0xFFu) << (8 * grp));
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 const uint2 r2 = raw[grp][hh];
@@ -285,6 +288,23 @@ __device__ __forceinline__ void query_frags(const __nv_bfloat16 *__restrict__ qh
             qinv[1][grp] = 1.f / __shfl_sync(kFull, qsc[grp], (2 * tig + 1) * 4);
         }
         qscaled = __any_sync(kFull, any);
+    }
+}
+
+// The raw bf16 query pairs (qbb of query_frags) turned, in place, into the scaled f16 pairs
+// (its qb) -- the same arithmetic -- from the lane's scale exponents (scexp): a kernel that
+// runs its bf16 tiles first keeps one copy of the query through the tile loops.
+__device__ __forceinline__ void query_to_f16(uint32_t (&qf)[4][2][2], uint32_t scexp) {
+#pragma unroll
+    for (int grp = 0; grp < 4; ++grp) {
+        const float sc = __uint_as_float(((scexp >> (8 * grp)) & 0xFFu) << 23);
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const uint32_t r = qf[grp][hh][k];
+                qf[grp][hh][k] = f32x2_to_f16x2(__uint_as_float(r << 16) * sc, __uint_as_float(r & 0xffff0000u) * sc);
+            }
     }
 }
 
