@@ -260,14 +260,14 @@ __device__ __forceinline__ int pick4(const int4 &v, int c) {
 // counters before the call (n4 entries, ft4 free slots, hw4 slots ever used per class);
 // r is its rank among the new tokens of its class in its batch row.  Returns its class
 // and *slot, or -1 when it is dropped: an invalid class id (TKV_ERR_INVALID) or a class
-// with neither a free nor a fresh slot (TKV_ERR_CAPACITY).  Statuses are latched only
-// with kReport (one lane of the warp reports).
-template <bool kReport>
+// with neither a free nor a fresh slot (TKV_ERR_CAPACITY), latched when `report` (one
+// lane of the warp reports).
 __device__ __forceinline__ int append_decide(const Dev &d, int s, uint8_t craw, int32_t p, int r, const int4 &n4,
-                                             const int4 &ft4, const int4 &hw4, uint32_t detail, int *slot) {
+                                             const int4 &ft4, const int4 &hw4, uint32_t detail, bool report,
+                                             int *slot) {
     auto check = [&](bool ok, uint32_t id) {   // the debug build's range checks
 #ifdef TKV_DEBUG
-        if (!ok && kReport) raise_error(d.err, kErrInvalid, id);
+        if (!ok && report) raise_error(d.err, kErrInvalid, id);
         return ok;
 #else
         (void)ok;
@@ -277,7 +277,7 @@ __device__ __forceinline__ int append_decide(const Dev &d, int s, uint8_t craw, 
     };
     const int c = token_class(d, craw, p);
     if (c < 0) {
-        if (kReport) raise_error(d.err, kErrInvalid, detail);
+        if (report) raise_error(d.err, kErrInvalid, detail);
         return -1;
     }
     const int cap = d.cap[c];
@@ -290,22 +290,11 @@ __device__ __forceinline__ int append_decide(const Dev &d, int s, uint8_t craw, 
     } else {
         *slot = hw + (r - ft);
         if (*slot >= cap) {
-            if (kReport) raise_error(d.err, kErrCapacity, (uint32_t)(s * 4 + c));
+            if (report) raise_error(d.err, kErrCapacity, (uint32_t)(s * 4 + c));
             return -1;
         }
     }
     return c;
-}
-
-// The stream counters after a T = 1 append of class c (-1: dropped) to counters n4, ft4,
-// hw4: one more entry, from the free stack if it was not empty, else a fresh slot.
-__device__ __forceinline__ void counters_after(int c, int4 &n4, int4 &ft4, int4 &hw4) {
-    if (c < 0) return;
-    auto bump = [c](int4 &v, int delta) {   // component c, without indexing (registers only)
-        if (c == 0) v.x += delta; else if (c == 1) v.y += delta; else if (c == 2) v.z += delta; else v.w += delta;
-    };
-    if (pick4(ft4, c) > 0) bump(ft4, -1); else bump(hw4, 1);
-    bump(n4, 1);
 }
 
 // One warp appends token t of stream s, gw = s * T + t, from the callers' K / V rows
@@ -332,8 +321,7 @@ __device__ __forceinline__ void append_token(const Dev &d, const __nv_bfloat16 *
     const int4 hw4 = *reinterpret_cast<const int4 *>(d.hw + s * 4);
     const int r = kSingle ? 0 : d.rank[(size_t)b * d.max_append + t];
     int slot = 0;
-    const int c = lane == 0 ? append_decide<true>(d, s, craw, p, r, n4, ft4, hw4, (uint32_t)gw, &slot)
-                            : append_decide<false>(d, s, craw, p, r, n4, ft4, hw4, (uint32_t)gw, &slot);
+    const int c = append_decide(d, s, craw, p, r, n4, ft4, hw4, (uint32_t)gw, lane == 0, &slot);
     if (c < 0) return;
     const int cap = d.cap[c];
     const size_t e = (size_t)s * cap + pick4(n4, c) + r;
@@ -361,12 +349,9 @@ __device__ __forceinline__ void append_token(const Dev &d, const __nv_bfloat16 *
     if constexpr (kSingle) {
         __syncwarp();  // every lane has read the pre-call counters
         if (lane == 0) {
-            int4 n1 = n4, ft1 = ft4, hw1 = hw4;
-            counters_after(c, n1, ft1, hw1);
-            const int sc = s * 4 + c;
-            d.ft[sc] = pick4(ft1, c);
-            d.hw[sc] = pick4(hw1, c);
-            d.n[sc] = pick4(n1, c);
+            const int sc = s * 4 + c, ft = pick4(ft4, c);
+            if (ft > 0) d.ft[sc] = ft - 1; else d.hw[sc] = pick4(hw4, c) + 1;   // popped, or a fresh slot
+            d.n[sc] = pick4(n4, c) + 1;
         }
     }
 }
