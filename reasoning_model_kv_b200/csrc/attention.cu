@@ -153,6 +153,7 @@ __global__ void __launch_bounds__(kThreads, TKV_ATTN_MIN_BLOCKS) attn_kernel(con
     __shared__ float gM[kMaxG], gInvL[kMaxG];
     __shared__ __align__(8) uint64_t bars[kWarps][kStages];   // dense placement only
     __shared__ float se[kWarps][kMaxG], ce[kMaxG];   // STATS: entropy terms per warp, per CTA
+    __shared__ float sqinv[kWarps][4][2][4];          // query inverse scales per warp and tig (rarely read)
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, tig = lane & 3;
@@ -172,15 +173,26 @@ __global__ void __launch_bounds__(kThreads, TKV_ATTN_MIN_BLOCKS) attn_kernel(con
     //      it; qinv holds the inverse scale of heads 2tig, 2tig+1 per group.
     //      One copy lives through the tile loops: qf holds the raw pairs while the bf16
     //      tiles (the first class loop) run, then the scaled f16 pairs.
+    //      The inverse scales (used only by queries that needed a scale) wait in shared
+    //      memory, one copy per warp and tig, rather than in registers.
     uint32_t qf[4][2][2];
-    float qs[2][4], qinv[2][4];
+    float qs[2][4];
     bool qscaled;
     uint32_t scexp;
     {
         uint32_t qb_unused[4][2][2];
+        float qinv[2][4];
         query_frags<G>(q + ((size_t)b * d.Hkv * G + (size_t)kvh * G) * kD, lane, qb_unused, qf, qs, qinv, qscaled,
                        &scexp);
+        if (g == 0) {
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                for (int grp = 0; grp < 4; ++grp) sqinv[warp][tig][hh][grp] = qinv[hh][grp];
+        }
+        __syncwarp();
     }
+    const float (&qinv)[2][4] = sqinv[warp][tig];
 
     // ---- this CTA's entry range and its tiles (class by class)
     const int n0 = dclamp(d.err, d.n[s * 4 + 0], d.cap[0], kDbgAttention + 0);

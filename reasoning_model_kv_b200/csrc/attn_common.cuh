@@ -341,6 +341,21 @@ __device__ __forceinline__ void qk_group(float (&x)[4], const uint32_t (&k0)[BIT
     }
 }
 
+// The two MMAs of qk_group for integer codes alone: acc = codes . q over group GRP (the
+// f16 query as scaled), with no scale, zero or inverse query scale applied yet.  Used
+// when a tile's four groups are formed first and folded together (see tile_compute).
+template <int BITS, int GRP>
+__device__ __forceinline__ void qk_acc(float (&acc)[4], const uint32_t (&k0)[BITS], const uint32_t (&k1)[BITS],
+                                       const uint32_t (&qb)[4][2][2], uint32_t magic) {
+    acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+    mma16816(acc, quarter_pair<BITS, 4 * GRP>(k0, magic), quarter_pair<BITS, 4 * GRP>(k1, magic),
+             quarter_pair<BITS, 4 * GRP + 1>(k0, magic), quarter_pair<BITS, 4 * GRP + 1>(k1, magic),
+             qb[GRP][0][0], qb[GRP][0][1]);
+    mma16816(acc, quarter_pair<BITS, 4 * GRP + 2>(k0, magic), quarter_pair<BITS, 4 * GRP + 2>(k1, magic),
+             quarter_pair<BITS, 4 * GRP + 3>(k0, magic), quarter_pair<BITS, 4 * GRP + 3>(k1, magic),
+             qb[GRP][1][0], qb[GRP][1][1]);
+}
+
 // S += K . Q^T over head-dim group GRP for floating-point codes (codec 1), pairs as in
 // qk_group.  FP8 / ternary: the code values against the f16 query, times the group's
 // fp16 scale (ka / kc: the four K scales of rows g / g + 8); no zero term.  NVFP4: each

@@ -51,11 +51,31 @@ __device__ __forceinline__ void tile_compute(const Loader &ld, int nr, int lane,
             qk_group_fp<BITS, 1>(x, k0, k1, qb, qinv, qscaled, ka, kc, tig);
             qk_group_fp<BITS, 2>(x, k0, k1, qb, qinv, qscaled, ka, kc, tig);
             qk_group_fp<BITS, 3>(x, k0, k1, qb, qinv, qscaled, ka, kc, tig);
-        } else {
-            if constexpr (BITS < 16) {
-                load_meta(ld.k_meta(0), km0);
-                load_meta(ld.k_meta(1), km1);
+        } else if constexpr (BITS < 16) {
+            // the four groups' products first, one branch for the (rare) query scale, then
+            // the folds in group order (the same arithmetic as qk_group, group by group)
+            load_meta(ld.k_meta(0), km0);
+            load_meta(ld.k_meta(1), km1);
+            float acc[4][4];
+            qk_acc<BITS, 0>(acc[0], k0, k1, qb, magic);
+            qk_acc<BITS, 1>(acc[1], k0, k1, qb, magic);
+            qk_acc<BITS, 2>(acc[2], k0, k1, qb, magic);
+            qk_acc<BITS, 3>(acc[3], k0, k1, qb, magic);
+            if (qscaled) {
+#pragma unroll
+                for (int grp = 0; grp < 4; ++grp) {
+                    acc[grp][0] *= qinv[0][grp]; acc[grp][1] *= qinv[1][grp];
+                    acc[grp][2] *= qinv[0][grp]; acc[grp][3] *= qinv[1][grp];
+                }
             }
+#pragma unroll
+            for (int grp = 0; grp < 4; ++grp) {
+                x[0] = fmaf(km0[grp].x, acc[grp][0], fmaf(km0[grp].y, qs[0][grp], x[0]));
+                x[1] = fmaf(km0[grp].x, acc[grp][1], fmaf(km0[grp].y, qs[1][grp], x[1]));
+                x[2] = fmaf(km1[grp].x, acc[grp][2], fmaf(km1[grp].y, qs[0][grp], x[2]));
+                x[3] = fmaf(km1[grp].x, acc[grp][3], fmaf(km1[grp].y, qs[1][grp], x[3]));
+            }
+        } else {
             qk_group<BITS, 0>(x, k0, k1, qb, qbb, qs, qinv, qscaled, km0, km1, magic);
             qk_group<BITS, 1>(x, k0, k1, qb, qbb, qs, qinv, qscaled, km0, km1, magic);
             qk_group<BITS, 2>(x, k0, k1, qb, qbb, qs, qinv, qscaled, km0, km1, magic);
