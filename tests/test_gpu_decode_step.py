@@ -83,6 +83,19 @@ def test_decode_step_equals_append_then_attention_and_the_oracle(mode, codec):
             _same_state(gpu, twin, "eviction")
 
 
+@pytest.mark.parametrize("dense", [False, True], ids=["reuse", "dense"])
+def test_decode_step_few_long_streams(dense):
+    """Two 24k-token streams: the attention splits each over more CTAs than a cluster holds
+    and merges them in a second pass; two steps against the two calls, bit for bit."""
+    w = synth.prefill_inputs("tiny_b1_ctx2k", B=1, Hkv=2, Hq=8, ctx=24000, n_protect=4, steps=2)
+    gpu = TkvCache(w["B"], w["Hkv"], w["G"], w["cap"], w["n_protect"], max_append=w["ctx"], dense=dense)
+    gpu.quantize_append(w["k"].to(DEV), w["v"].to(DEV), w["cls"][:, :w["ctx"]].contiguous().to(DEV),
+                        w["pos"].to(DEV))
+    twin = _twin(gpu)
+    for step in range(2):
+        _step_and_twin(gpu, twin, *_step_inputs(w, step), f"long streams step {step}")
+
+
 @pytest.mark.parametrize("G", [1, 2, 8])
 def test_decode_step_gqa_widths(G):
     """Other GQA group widths (one CTA per stream at 8 streams)."""
