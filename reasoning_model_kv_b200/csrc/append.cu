@@ -2,7 +2,7 @@
 // tokens (ThinKV, Metodologia / TBQ) into paged per-precision pools with
 // in-place reuse of evicted slots (ThinKV, Implementacao do Sistema /
 // Continuous Thinking).  The per-token work (one warp per (stream, token)) is in
-// append_token.cuh, shared with the fused decode step.
+// append_token.cuh.
 //
 // Slot allocation needs, per (stream, class), the rank of each new token among
 // the new tokens of its class.  For T == 1 that rank is 0 and the packing warp

@@ -2,8 +2,8 @@
 // group quantisation of one new token's K/V row (ThinKV, Metodologia / TBQ) into its
 // class record, slot allocation in the per-precision pool with in-place reuse of
 // evicted slots (ThinKV, Implementacao do Sistema / Continuous Thinking), and the
-// table / counter updates.  One warp per token; used by the append kernels and by the
-// fused decode step (append + attention in one launch).  Internal to libtkv.
+// table / counter updates.  One warp per token; the append kernels' device code.
+// Internal to libtkv.
 //
 // Lane l owns head-dim elements [4l, 4l+4), so a 32-element group is 8 lanes and its
 // min/max is a 3-step xor-shuffle reduction.  Codes are then re-gathered through shared
