@@ -218,38 +218,29 @@ __device__ __forceinline__ void store_bf16_row(const uint2 &raw, int lane, uint8
     }
 }
 
-// Codec 1 record of BITS-bit codes: [K codes][V codes][K scales][V scales].
-template <int BITS>
-__device__ __forceinline__ void pack_record_fp(const uint2 &rk, const uint2 &rv, uint8_t *rec, int lane,
-                                               uint8_t *stage) {
-    constexpr int cb = kD * BITS / 8;
-    constexpr int sb = BITS == 4 ? kD / 16 : 2 * kNG;   // scale bytes of one block
-    float x[4];
-    row_floats(rk, x);
-    quantize_row_fp<BITS>(x, lane, rec + 2 * cb, stage);
-    if (lane < 4 * BITS) reinterpret_cast<uint32_t *>(rec)[lane] = code_word<BITS, false>(stage, lane);
-    row_floats(rv, x);
-    quantize_row_fp<BITS>(x, lane, rec + 2 * cb + sb, stage);
-    if (lane < 4 * BITS) reinterpret_cast<uint32_t *>(rec + cb)[lane] = code_word<BITS, true>(stage, lane);
-}
-
-// Packs one record from this lane's 4 elements of the K and V rows (raw bf16 pairs).
-template <int BITS>
-__device__ __forceinline__ void pack_record(const uint2 &rk, const uint2 &rv, uint8_t *rec, int lane,
-                                            uint8_t *stage) {
+// One half of a record -- the K (IS_V false) or the V row -- from this lane's 4 elements
+// of that row (raw bf16 pairs).  Codec 0 record: [K codes][V codes][K meta][V meta] (bf16
+// rows for class 0); codec 1: [K codes][V codes][K scales][V scales].
+template <int BITS, bool IS_V>
+__device__ __forceinline__ void pack_half(const uint2 &raw, uint8_t *rec, int lane, uint8_t *stage) {
     if constexpr (BITS == 16) {
-        uint16_t *st16 = reinterpret_cast<uint16_t *>(stage);
-        store_bf16_row<false>(rk, lane, rec, st16);
-        store_bf16_row<true>(rv, lane, rec + 2 * kD, st16);
+        store_bf16_row<IS_V>(raw, lane, rec + (IS_V ? 2 * kD : 0), reinterpret_cast<uint16_t *>(stage));
     } else {
         constexpr int cb = kD * BITS / 8;
         __half *meta = reinterpret_cast<__half *>(rec + 2 * cb);
         float x[4];
-        row_floats(rk, x);
-        quantize_row<BITS, false>(x, lane, rec, meta, stage);
-        row_floats(rv, x);
-        quantize_row<BITS, true>(x, lane, rec + cb, meta + 2 * kNG, stage);
+        row_floats(raw, x);
+        quantize_row<BITS, IS_V>(x, lane, rec + (IS_V ? cb : 0), meta + (IS_V ? 2 * kNG : 0), stage);
     }
+}
+template <int BITS, bool IS_V>
+__device__ __forceinline__ void pack_half_fp(const uint2 &raw, uint8_t *rec, int lane, uint8_t *stage) {
+    constexpr int cb = kD * BITS / 8;
+    constexpr int sb = BITS == 4 ? kD / 16 : 2 * kNG;   // scale bytes of one block
+    float x[4];
+    row_floats(raw, x);
+    quantize_row_fp<BITS>(x, lane, rec + 2 * cb + (IS_V ? sb : 0), stage);
+    if (lane < 4 * BITS) reinterpret_cast<uint32_t *>(rec + (IS_V ? cb : 0))[lane] = code_word<BITS, IS_V>(stage, lane);
 }
 
 __device__ __forceinline__ int pick4(const int4 &v, int c) {
@@ -297,23 +288,25 @@ __device__ __forceinline__ int append_decide(const Dev &d, int s, uint8_t craw, 
     return c;
 }
 
-// One warp appends token t of stream s, gw = s * T + t, from the callers' K / V rows
-// (bf16, [S][T][128]), class ids and positions ([B][T]).  r is the token's rank among the
-// new tokens of its class in its batch row: 0 when T == 1, and then the warp also
-// advances the stream's counters; for T > 1 the ranks come from the scan kernel and a
-// finalize kernel advances the counters.  `stage`: 256 bytes of this warp's shared memory.
+// Two warps append token t of stream s, tok = s * T + t, from the callers' K / V rows
+// (bf16, [S][T][128]), class ids and positions ([B][T]): `half` 0 packs the K row and
+// writes the table entry, half 1 packs the V row (both reach the same slot decision from
+// the same inputs).  r is the token's rank among the new tokens of its class in its batch
+// row: 0 when T == 1, and then the pair meets at named barrier `pair_bar` (64 threads)
+// once both have read the stream's counters, and half 0 advances them; for T > 1 the
+// ranks come from the scan kernel and a finalize kernel advances the counters.  `stage`:
+// 256 bytes of this warp's shared memory.
 template <bool kSingle, int kCodec>
 __device__ __forceinline__ void append_token(const Dev &d, const __nv_bfloat16 *__restrict__ k,
                                              const __nv_bfloat16 *__restrict__ v, const uint8_t *__restrict__ cls,
-                                             const int32_t *__restrict__ pos, int T, int gw, int lane,
-                                             uint8_t *stage) {
-    const int s = gw / T, t = gw - s * T;
+                                             const int32_t *__restrict__ pos, int T, int tok, int half, int lane,
+                                             uint8_t *stage, int pair_bar) {
+    const int s = tok / T, t = tok - s * T;
     const int b = s / d.Hkv;
-    // every independent load first (one round trip): the K/V rows, the token's
+    // every independent load first (one round trip): this half's row, the token's
     // position and class, and the stream's counters of all four classes
     const size_t row = ((size_t)s * T + t) * kD;
-    const uint2 rk = reinterpret_cast<const uint2 *>(k + row)[lane];
-    const uint2 rv = reinterpret_cast<const uint2 *>(v + row)[lane];
+    const uint2 raw = reinterpret_cast<const uint2 *>((half ? v : k) + row)[lane];
     const int32_t p = pos[(size_t)b * T + t];
     const uint8_t craw = cls[(size_t)b * T + t];
     const int4 n4 = *reinterpret_cast<const int4 *>(d.n + s * 4);
@@ -321,34 +314,41 @@ __device__ __forceinline__ void append_token(const Dev &d, const __nv_bfloat16 *
     const int4 hw4 = *reinterpret_cast<const int4 *>(d.hw + s * 4);
     const int r = kSingle ? 0 : d.rank[(size_t)b * d.max_append + t];
     int slot = 0;
-    const int c = append_decide(d, s, craw, p, r, n4, ft4, hw4, (uint32_t)gw, lane == 0, &slot);
-    if (c < 0) return;
+    const int c = append_decide(d, s, craw, p, r, n4, ft4, hw4, (uint32_t)tok, half == 0 && lane == 0, &slot);
+    if (c < 0) return;   // (both warps of the pair)
     const int cap = d.cap[c];
     const size_t e = (size_t)s * cap + pick4(n4, c) + r;
-    if (lane == 0) {
+    if (half == 0 && lane == 0) {
         d.handle[c][e] = slot;
         d.pos[c][e] = p;
         d.score[c][e] = 0.0f;
     }
     uint8_t *rec = d.pool[c] + ((size_t)s * cap + slot) * d.rec[c];
+#define TKV_PACK_HALF(FN, BITS)                                      \
+    {                                                                \
+        if (half) FN<BITS, true>(raw, rec, lane, stage);             \
+        else FN<BITS, false>(raw, rec, lane, stage);                 \
+    }
     if constexpr (kCodec == 0) {
         switch (c) {
-            case 0: pack_record<16>(rk, rv, rec, lane, stage); break;
-            case 1: pack_record<8>(rk, rv, rec, lane, stage); break;
-            case 2: pack_record<4>(rk, rv, rec, lane, stage); break;
-            default: pack_record<2>(rk, rv, rec, lane, stage); break;
+            case 0: TKV_PACK_HALF(pack_half, 16) break;
+            case 1: TKV_PACK_HALF(pack_half, 8) break;
+            case 2: TKV_PACK_HALF(pack_half, 4) break;
+            default: TKV_PACK_HALF(pack_half, 2) break;
         }
     } else {
         switch (c) {
-            case 0: pack_record<16>(rk, rv, rec, lane, stage); break;
-            case 1: pack_record_fp<8>(rk, rv, rec, lane, stage); break;
-            case 2: pack_record_fp<4>(rk, rv, rec, lane, stage); break;
-            default: pack_record_fp<2>(rk, rv, rec, lane, stage); break;
+            case 0: TKV_PACK_HALF(pack_half, 16) break;
+            case 1: TKV_PACK_HALF(pack_half_fp, 8) break;
+            case 2: TKV_PACK_HALF(pack_half_fp, 4) break;
+            default: TKV_PACK_HALF(pack_half_fp, 2) break;
         }
     }
+#undef TKV_PACK_HALF
     if constexpr (kSingle) {
-        __syncwarp();  // every lane has read the pre-call counters
-        if (lane == 0) {
+        // both warps of the pair have read the pre-call counters
+        asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
+        if (half == 0 && lane == 0) {
             const int sc = s * 4 + c, ft = pick4(ft4, c);
             if (ft > 0) d.ft[sc] = ft - 1; else d.hw[sc] = pick4(hw4, c) + 1;   // popped, or a fresh slot
             d.n[sc] = pick4(n4, c) + 1;

@@ -146,7 +146,8 @@ __global__ void __launch_bounds__(kThreads, TKV_ATTN_MIN_BLOCKS) attn_kernel(con
                                                            const __nv_bfloat16 *__restrict__ q,
                                                            float xscale, float *__restrict__ out,
                                                            int C, int split, float *__restrict__ sparsity,
-                                                           uint8_t *__restrict__ thought, float th_r, float th_t) {
+                                                           uint8_t *__restrict__ thought, float th_r, float th_t,
+                                                           int q_ready) {
     extern __shared__ __align__(128) uint8_t ring[];   // kRingBytes, dynamic
     __shared__ float cta_m[kMaxG], cta_l[kMaxG];
     __shared__ float fac[kMaxCluster][kMaxG];     // exp2(m_j - M) per warp / peer rank and head
@@ -162,9 +163,12 @@ __global__ void __launch_bounds__(kThreads, TKV_ATTN_MIN_BLOCKS) attn_kernel(con
     const int b = s / d.Hkv, kvh = s - b * d.Hkv;
 
     // the previous kernel's writes (an append's counters and records, or the caller's
-    // query) are visible from here: nothing is read before it, since this kernel may
-    // launch while the previous one still runs (programmatic dependent launch)
-    grid_dependency_wait();
+    // query) are visible from here: nothing it may write is read before it, since this
+    // kernel may launch while the previous one still runs (programmatic dependent
+    // launch).  q_ready: the previous kernel is this library's append, itself launched
+    // in plain stream order (so the query was complete before it started), and the
+    // query is read while the append still runs.
+    if (!q_ready) grid_dependency_wait();
 
     // ---- query operand (B of S = K Q^T): head g, dims 32grp + 8tig + 4hh + 0..3.
     //      qbb: the raw bf16 pairs (bf16 keys); qb: f16 pairs for the integer codes,
@@ -193,6 +197,7 @@ __global__ void __launch_bounds__(kThreads, TKV_ATTN_MIN_BLOCKS) attn_kernel(con
         __syncwarp();
     }
     const float (&qinv)[2][4] = sqinv[warp][tig];
+    if (q_ready) grid_dependency_wait();
 
     // ---- this CTA's entry range and its tiles (class by class)
     const int n0 = dclamp(d.err, d.n[s * 4 + 0], d.cap[0], kDbgAttention + 0);
@@ -515,7 +520,7 @@ int g_blocks_per_sm[2][2][2][kMaxG + 1][kMaxDevices] = {};   // per codec, place
 template <int G, bool DENSE, int CODEC, bool STATS>
 cudaError_t launch_g(const Dev &d, const void *q, float scale, float *out, long long live_ub,
                      cudaStream_t st, int64_t *launches, float *sparsity, uint8_t *thought, float th_r,
-                     float th_t) {
+                     float th_t, bool q_ready) {
     int sms = 0, bps = 0;
     cudaError_t e0 = device_sm_count(&sms);
     if (e0 != cudaSuccess) return e0;
@@ -556,7 +561,7 @@ cudaError_t launch_g(const Dev &d, const void *q, float scale, float *out, long 
     const float xscale = scale * 1.4426950408889634f;   // logits in the log2 domain
     cudaError_t e = cudaLaunchKernelEx(&cfg, attn_kernel<G, DENSE, CODEC, STATS>, d,
                                        static_cast<const __nv_bfloat16 *>(q), xscale, out, (int)C, (int)split,
-                                       sparsity, thought, th_r, th_t);
+                                       sparsity, thought, th_r, th_t, (int)q_ready);
     *launches += 1;
     if (e != cudaSuccess || !split) return e;
     return launch_finalize<G, STATS, 1>(d, out, sparsity, thought, th_r, th_t, (int)(d.S * C), live_ub, st, launches);
@@ -566,14 +571,14 @@ cudaError_t launch_g(const Dev &d, const void *q, float scale, float *out, long 
 
 cudaError_t launch_attention(const Dev &d, const void *q, float scale, float *out, long long live_ub,
                              cudaStream_t st, int64_t *launches, float *sparsity, uint8_t *thought, float th_r,
-                             float th_t) {
+                             float th_t, bool q_ready) {
     if (d.dense && d.attn_kernel != 0) return cudaErrorInvalidValue;   // the persistent kernels'
 #define TKV_G_CASES(DN, CD, ST)                                                                              \
     switch (d.G) {                                                                                           \
-        case 1: return launch_g<1, DN, CD, ST>(d, q, scale, out, live_ub, st, launches, sparsity, thought, th_r, th_t); \
-        case 2: return launch_g<2, DN, CD, ST>(d, q, scale, out, live_ub, st, launches, sparsity, thought, th_r, th_t); \
-        case 4: return launch_g<4, DN, CD, ST>(d, q, scale, out, live_ub, st, launches, sparsity, thought, th_r, th_t); \
-        case 8: return launch_g<8, DN, CD, ST>(d, q, scale, out, live_ub, st, launches, sparsity, thought, th_r, th_t); \
+        case 1: return launch_g<1, DN, CD, ST>(d, q, scale, out, live_ub, st, launches, sparsity, thought, th_r, th_t, q_ready); \
+        case 2: return launch_g<2, DN, CD, ST>(d, q, scale, out, live_ub, st, launches, sparsity, thought, th_r, th_t, q_ready); \
+        case 4: return launch_g<4, DN, CD, ST>(d, q, scale, out, live_ub, st, launches, sparsity, thought, th_r, th_t, q_ready); \
+        case 8: return launch_g<8, DN, CD, ST>(d, q, scale, out, live_ub, st, launches, sparsity, thought, th_r, th_t, q_ready); \
         default: return cudaErrorInvalidValue;                                                               \
     }
     // one compound statement per (placement, codec): both switches return

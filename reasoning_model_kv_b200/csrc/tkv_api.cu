@@ -274,8 +274,9 @@ tkv_status ensure_maps(tkv_cache *c) {
 
 namespace {
 // Decode attention over the cache with `ub` bounding every stream's live entries.
+// q_ready: the append was the last launch on `st` (see launch_attention).
 tkv_status launch_decode(tkv_cache *c, const void *q, float softmax_scale, float *out, long long ub,
-                         cudaStream_t st, const char *what) {
+                         cudaStream_t st, const char *what, bool q_ready = false) {
     cudaError_t e;
     if (c->cfg.attn_kernel != 0) {   // the persistent kernels (dense placement)
         const tkv_status ms = ensure_maps(c);
@@ -286,7 +287,8 @@ tkv_status launch_decode(tkv_cache *c, const void *q, float softmax_scale, float
         else
             e = tkv::launch_attention_ws(c->dev, c->maps, q, softmax_scale, out, ub, st, &c->launches);
     } else {
-        e = tkv::launch_attention(c->dev, q, softmax_scale, out, ub, st, &c->launches);
+        e = tkv::launch_attention(c->dev, q, softmax_scale, out, ub, st, &c->launches, nullptr, nullptr, 0.f, 0.f,
+                                  q_ready);
     }
     return cuda_status(e, what);
 }
@@ -316,7 +318,7 @@ tkv_status tkv_decode_step(tkv_cache *c, const void *k, const void *v, const uin
     const cudaError_t e = tkv::launch_append(c->dev, k, v, cls, pos, 1, st, &c->launches);
     c->live_ub = std::min<long long>(c->dev.ncap, c->live_ub + 1);
     if (e != cudaSuccess) return cuda_status(e, "tkv_decode_step");
-    return launch_decode(c, q, softmax_scale, out, std::max(1ll, c->live_ub), st, "tkv_decode_step");
+    return launch_decode(c, q, softmax_scale, out, std::max(1ll, c->live_ub), st, "tkv_decode_step", true);
 }
 
 tkv_status tkv_decode_attention_sparsity(tkv_cache *c, const void *q, float softmax_scale, float *out,

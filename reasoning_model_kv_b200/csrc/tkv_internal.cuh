@@ -110,10 +110,12 @@ cudaError_t cached_blocks_per_sm(int *slot_per_device, const void *kernel, int t
 cudaError_t launch_append(const Dev &d, const void *k, const void *v, const uint8_t *cls,
                           const int32_t *pos, int T, cudaStream_t st, int64_t *launches);
 // Warp-tile decode attention; with `sparsity` non-NULL it also writes, per (stream, query
-// head), the attention sparsity and (thought non-NULL) its thought class.
+// head), the attention sparsity and (thought non-NULL) its thought class.  q_ready: the
+// kernel before it on `st` is launch_append's (launched in plain stream order), so the
+// query may be read before that kernel completes.
 cudaError_t launch_attention(const Dev &d, const void *q, float scale, float *out,
                              long long live_ub, cudaStream_t st, int64_t *launches, float *sparsity = nullptr,
-                             uint8_t *thought = nullptr, float th_r = 0.f, float th_t = 0.f);
+                             uint8_t *thought = nullptr, float th_r = 0.f, float th_t = 0.f, bool q_ready = false);
 // Dense placement: the tensor-core kernel with integer operands (attention_i8.cu).  With
 // sparsity / thought non-NULL it also writes, per (stream, query head), the attention
 // sparsity 1 - H(p) / ln N and its thought class under the thresholds th_r <= th_t.
