@@ -516,6 +516,7 @@ __global__ void __launch_bounds__(kThreads, TKV_ATTN_MIN_BLOCKS) attn_kernel(con
 }
 
 int g_blocks_per_sm[2][2][2][kMaxG + 1][kMaxDevices] = {};   // per codec, placement, stats, G and device
+int g_max_clusters[2][2][2][kMaxG + 1][kMaxCluster + 1][kMaxDevices] = {};   // ... and cluster size
 
 template <int G, bool DENSE, int CODEC, bool STATS>
 cudaError_t launch_g(const Dev &d, const void *q, float scale, float *out, long long live_ub,
@@ -543,6 +544,18 @@ cudaError_t launch_g(const Dev &d, const void *q, float scale, float *out, long 
         if (C > kMaxCluster) C = kMaxCluster;
         if (C > live_ub / 128) C = live_ub / 128;
         if (C < 1) C = 1;
+        // clusters are placed within one GPC, where a few SMs' slots can stay unusable for
+        // a cluster size: shrink it until every stream's cluster is resident at once (a
+        // second wave would double the call)
+        while (C > 1) {
+            int fit = 0;
+            e0 = cached_max_clusters(g_max_clusters[CODEC][DENSE][STATS][G][C],
+                                     reinterpret_cast<const void *>(attn_kernel<G, DENSE, CODEC, STATS>), kThreads,
+                                     kRingBytes, (int)C, &fit);
+            if (e0 != cudaSuccess) return e0;
+            if (fit >= d.S) break;
+            --C;
+        }
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)C, (unsigned)d.S, 1);

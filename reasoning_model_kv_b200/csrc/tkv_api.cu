@@ -190,6 +190,35 @@ cudaError_t cached_blocks_per_sm(int *slot_per_device, const void *kernel, int t
     *blocks = slot_per_device[dev];
     return cudaSuccess;
 }
+
+cudaError_t cached_max_clusters(int *slot_per_device, const void *kernel, int threads, size_t smem, int C,
+                                int *clusters) {
+    *clusters = 0;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_occ_mu);
+    if (slot_per_device[dev] == 0) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)C, 1, 1);
+        cfg.blockDim = dim3((unsigned)threads, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)C;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        e = cudaOccupancyMaxActiveClusters(&n, kernel, &cfg);
+        if (e != cudaSuccess) return e;
+        slot_per_device[dev] = n > 0 ? n : 1;
+    }
+    *clusters = slot_per_device[dev];
+    return cudaSuccess;
+}
 }  // namespace tkv
 
 extern "C" {

@@ -104,6 +104,12 @@ cudaError_t device_sm_count(int *sms);
 // bytes on the current device, cached in slot[device] (0 means "not yet known").
 cudaError_t cached_blocks_per_sm(int *slot_per_device, const void *kernel, int threads, size_t smem,
                                  int *blocks);
+// Clusters of C CTAs of `kernel` (threads per CTA, dynamic shared memory smem, already set
+// up by cached_blocks_per_sm) that the current device holds at once, cached per device in
+// slot_per_device.  A cluster lives within one GPC, so on a part whose GPCs hold an odd
+// number of SMs this is below blocks-per-SM x SMs / C.
+cudaError_t cached_max_clusters(int *slot_per_device, const void *kernel, int threads, size_t smem, int C,
+                                int *clusters);
 
 // Launchers (each returns the CUDA error of its launches and adds the number
 // of kernels it launched to *launches).

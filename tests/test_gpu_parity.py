@@ -139,6 +139,19 @@ def test_few_long_streams_split_beyond_a_cluster(G, mode, codec):
     _decode_step(w, gpu, o, rows, 1)
 
 
+@pytest.mark.parametrize("mode", list(MODES))
+def test_clusters_shrunk_to_one_wave(mode):
+    """72 streams of 2048 entries: eight CTAs per stream would fill the SMs' slots, but
+    clusters live within one GPC and a B200 holds only 71 clusters of eight such CTAs, so
+    the launcher takes the largest cluster size that keeps every stream resident at once
+    (seven here: a size that is not a power of two), compared on three sampled rows."""
+    w, gpu, o, rows = build_pair("tiny_b1_ctx2k", B=9, Hq=32, Hkv=8, ctx=2048, n_protect=4, outliers=True,
+                                 steps=2, rows=[0, 4, 8], **MODES[mode])
+    _decode_step(w, gpu, o, rows, 0)
+    _evict_lockstep(gpu, o, rows, 1200)
+    _decode_step(w, gpu, o, rows, 1)
+
+
 @pytest.mark.parametrize("dense", [False, True], ids=["reuse", "dense"])
 def test_multi_token_append_after_eviction_reuses_slots_in_order(dense):
     w, gpu, o, rows = build_pair("tiny_b1_ctx2k", ctx=600, steps=80, dense=dense)
