@@ -1,8 +1,9 @@
 // append.cu -- tkv_quantize_append: thought-adaptive group quantisation of new
 // tokens (ThinKV, Metodologia / TBQ) into paged per-precision pools with
 // in-place reuse of evicted slots (ThinKV, Implementacao do Sistema /
-// Continuous Thinking).  The per-token work (two warps per (stream, token): one
-// quantises the K row, the other the V row) is in append_token.cuh.
+// Continuous Thinking).  The per-token work (for T == 1 two warps per (stream, token),
+// one quantising the K row and the other the V row; for T > 1 one warp per (stream,
+// token)) is in append_token.cuh.
 //
 // Slot allocation needs, per (stream, class), the rank of each new token among
 // the new tokens of its class.  For T == 1 that rank is 0 and the packing warp
@@ -70,11 +71,13 @@ __global__ void __launch_bounds__(256) append_pack_kernel(
     // let the next kernel in the stream (decode attention) launch now; it waits for
     // this grid's completion before it reads the cache
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    // two warps per (stream, token): warps 2i (K) and 2i + 1 (V) of the grid
+    // T == 1: two warps per (stream, token), warps 2i (K) and 2i + 1 (V) of the grid;
+    // T > 1: one warp per (stream, token)
+    constexpr int kShift = kSingle ? 1 : 0;
     const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
-    if ((gw >> 1) >= d.S * T) return;   // (both warps of a pair)
-    app::append_token<kSingle, kCodec>(d, k, v, cls, pos, T, gw >> 1, gw & 1, lane,
+    if ((gw >> kShift) >= d.S * T) return;   // (both warps of a pair)
+    app::append_token<kSingle, kCodec>(d, k, v, cls, pos, T, gw >> kShift, gw & 1, lane,
                                        stage_all + (threadIdx.x >> 5) * 2 * kD, 1 + ((threadIdx.x >> 5) >> 1));
 }
 
@@ -98,7 +101,8 @@ cudaError_t launch_append(const Dev &d, const void *k, const void *v, const uint
                           const int32_t *pos, int T, cudaStream_t st, int64_t *launches) {
     const auto *kk = static_cast<const __nv_bfloat16 *>(k);
     const auto *vv = static_cast<const __nv_bfloat16 *>(v);
-    const long long warps = 2ll * d.S * T;   // a K warp and a V warp per (stream, token)
+    // T == 1: a K warp and a V warp per (stream, token); T > 1: one warp per (stream, token)
+    const long long warps = (T == 1 ? 2ll : 1ll) * d.S * T;
     const int threads = 256;
     const unsigned blocks = (unsigned)((warps * 32 + threads - 1) / threads);
     if (T == 1) {

@@ -288,46 +288,21 @@ __device__ __forceinline__ int append_decide(const Dev &d, int s, uint8_t craw, 
     return c;
 }
 
-// Two warps append token t of stream s, tok = s * T + t, from the callers' K / V rows
-// (bf16, [S][T][128]), class ids and positions ([B][T]): `half` 0 packs the K row and
-// writes the table entry, half 1 packs the V row (both reach the same slot decision from
-// the same inputs).  r is the token's rank among the new tokens of its class in its batch
-// row: 0 when T == 1, and then the pair meets at named barrier `pair_bar` (64 threads)
-// once both have read the stream's counters, and half 0 advances them; for T > 1 the
-// ranks come from the scan kernel and a finalize kernel advances the counters.  `stage`:
-// 256 bytes of this warp's shared memory.
-template <bool kSingle, int kCodec>
-__device__ __forceinline__ void append_token(const Dev &d, const __nv_bfloat16 *__restrict__ k,
-                                             const __nv_bfloat16 *__restrict__ v, const uint8_t *__restrict__ cls,
-                                             const int32_t *__restrict__ pos, int T, int tok, int half, int lane,
-                                             uint8_t *stage, int pair_bar) {
-    const int s = tok / T, t = tok - s * T;
-    const int b = s / d.Hkv;
-    // every independent load first (one round trip): this half's row, the token's
-    // position and class, and the stream's counters of all four classes
-    const size_t row = ((size_t)s * T + t) * kD;
-    const uint2 raw = reinterpret_cast<const uint2 *>((half ? v : k) + row)[lane];
-    const int32_t p = pos[(size_t)b * T + t];
-    const uint8_t craw = cls[(size_t)b * T + t];
-    const int4 n4 = *reinterpret_cast<const int4 *>(d.n + s * 4);
-    const int4 ft4 = *reinterpret_cast<const int4 *>(d.ft + s * 4);
-    const int4 hw4 = *reinterpret_cast<const int4 *>(d.hw + s * 4);
-    const int r = kSingle ? 0 : d.rank[(size_t)b * d.max_append + t];
-    int slot = 0;
-    const int c = append_decide(d, s, craw, p, r, n4, ft4, hw4, (uint32_t)tok, half == 0 && lane == 0, &slot);
-    if (c < 0) return;   // (both warps of the pair)
-    const int cap = d.cap[c];
-    const size_t e = (size_t)s * cap + pick4(n4, c) + r;
-    if (half == 0 && lane == 0) {
-        d.handle[c][e] = slot;
-        d.pos[c][e] = p;
-        d.score[c][e] = 0.0f;
-    }
-    uint8_t *rec = d.pool[c] + ((size_t)s * cap + slot) * d.rec[c];
+// A record of class c from this warp's rows: kBoth, the K row `raw` and the V row `rawv`;
+// otherwise the K row (half 0) or the V row (half 1) in `raw`.
+template <int kCodec, bool kBoth>
+__device__ __forceinline__ void pack_row(int c, int half, const uint2 &raw, const uint2 &rawv, uint8_t *rec, int lane,
+                                         uint8_t *stage) {
 #define TKV_PACK_HALF(FN, BITS)                                      \
     {                                                                \
-        if (half) FN<BITS, true>(raw, rec, lane, stage);             \
-        else FN<BITS, false>(raw, rec, lane, stage);                 \
+        if (kBoth) {                                                 \
+            FN<BITS, false>(raw, rec, lane, stage);                  \
+            FN<BITS, true>(rawv, rec, lane, stage);                  \
+        } else if (half) {                                           \
+            FN<BITS, true>(raw, rec, lane, stage);                   \
+        } else {                                                     \
+            FN<BITS, false>(raw, rec, lane, stage);                  \
+        }                                                            \
     }
     if constexpr (kCodec == 0) {
         switch (c) {
@@ -345,6 +320,50 @@ __device__ __forceinline__ void append_token(const Dev &d, const __nv_bfloat16 *
         }
     }
 #undef TKV_PACK_HALF
+}
+
+// Appends token t of stream s, tok = s * T + t, from the callers' K / V rows (bf16,
+// [S][T][128]), class ids and positions ([B][T]).
+// kSingle (T == 1, a decode step): two warps share the token, `half` 0 packing the K row
+// and writing the table entry, half 1 the V row (both reach the same slot decision from
+// the same inputs); the token's rank r among the new tokens of its class is 0, and the
+// pair meets at named barrier `pair_bar` (64 threads) once both have read the stream's
+// counters, before half 0 advances them.  Otherwise (a prefill, where throughput rather
+// than one token's latency counts) one warp packs both rows (`half` unused), the ranks
+// come from the scan kernel and a finalize kernel advances the counters.
+// `stage`: 256 bytes of this warp's shared memory.
+template <bool kSingle, int kCodec>
+__device__ __forceinline__ void append_token(const Dev &d, const __nv_bfloat16 *__restrict__ k,
+                                             const __nv_bfloat16 *__restrict__ v, const uint8_t *__restrict__ cls,
+                                             const int32_t *__restrict__ pos, int T, int tok, int half, int lane,
+                                             uint8_t *stage, int pair_bar) {
+    if constexpr (!kSingle) half = 0;
+    const int s = tok / T, t = tok - s * T;
+    const int b = s / d.Hkv;
+    // every independent load first (one round trip): the row(s), the token's position
+    // and class, and the stream's counters of all four classes
+    const size_t row = ((size_t)s * T + t) * kD;
+    const uint2 raw = reinterpret_cast<const uint2 *>((half ? v : k) + row)[lane];
+    uint2 rawv = make_uint2(0u, 0u);
+    if constexpr (!kSingle) rawv = reinterpret_cast<const uint2 *>(v + row)[lane];
+    const int32_t p = pos[(size_t)b * T + t];
+    const uint8_t craw = cls[(size_t)b * T + t];
+    const int4 n4 = *reinterpret_cast<const int4 *>(d.n + s * 4);
+    const int4 ft4 = *reinterpret_cast<const int4 *>(d.ft + s * 4);
+    const int4 hw4 = *reinterpret_cast<const int4 *>(d.hw + s * 4);
+    const int r = kSingle ? 0 : d.rank[(size_t)b * d.max_append + t];
+    int slot = 0;
+    const int c = append_decide(d, s, craw, p, r, n4, ft4, hw4, (uint32_t)tok, half == 0 && lane == 0, &slot);
+    if (c < 0) return;   // (both warps of a pair)
+    const int cap = d.cap[c];
+    const size_t e = (size_t)s * cap + pick4(n4, c) + r;
+    if (half == 0 && lane == 0) {
+        d.handle[c][e] = slot;
+        d.pos[c][e] = p;
+        d.score[c][e] = 0.0f;
+    }
+    uint8_t *rec = d.pool[c] + ((size_t)s * cap + slot) * d.rec[c];
+    pack_row<kCodec, !kSingle>(c, half, raw, rawv, rec, lane, stage);
     if constexpr (kSingle) {
         // both warps of the pair have read the pre-call counters
         asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");

@@ -240,19 +240,19 @@ __global__ void __launch_bounds__(kThreadsWS, kCtasPerSm)
                 float *lg = d.logits + ((size_t)td.s * d.ncap + td.oc + td.e + r0) * G;
                 switch (tcls) {
                     case 0:
-                        tile_compute<16, 8, G, 0>(TmaLoader<16>(stage, r0, g), nw, lane, Q.qb, Q.qbb, Q.qs, Q.qinv,
+                        tile_compute<16, 8, G, 0, false>(TmaLoader<16>(stage, r0, g), nw, lane, Q.qb, Q.qbb, Q.qs, Q.qinv,
                                                   qscaled, xscale, ws, lg, magic);
                         break;
                     case 1:
-                        tile_compute<8, 16, G, 0>(TmaLoader<8>(stage, r0, g), nw, lane, Q.qb, Q.qbb, Q.qs, Q.qinv,
+                        tile_compute<8, 16, G, 0, false>(TmaLoader<8>(stage, r0, g), nw, lane, Q.qb, Q.qbb, Q.qs, Q.qinv,
                                                   qscaled, xscale, ws, lg, magic);
                         break;
                     case 2:
-                        tile_compute<4, 16, G, 0>(TmaLoader<4>(stage, r0, g), nw, lane, Q.qb, Q.qbb, Q.qs, Q.qinv,
+                        tile_compute<4, 16, G, 0, false>(TmaLoader<4>(stage, r0, g), nw, lane, Q.qb, Q.qbb, Q.qs, Q.qinv,
                                                   qscaled, xscale, ws, lg, magic);
                         break;
                     default:
-                        tile_compute<2, 16, G, 0>(TmaLoader<2>(stage, r0, g), nw, lane, Q.qb, Q.qbb, Q.qs, Q.qinv,
+                        tile_compute<2, 16, G, 0, false>(TmaLoader<2>(stage, r0, g), nw, lane, Q.qb, Q.qbb, Q.qs, Q.qinv,
                                                   qscaled, xscale, ws, lg, magic);
                         break;
                 }

@@ -22,7 +22,11 @@ struct WarpState {
 // STRIDE; int8 odd rows chunk-swizzled when SWZ).  Lane (g, tig) owns rows g and
 // g + 8.  Rows at or beyond nr hold zeros (the copy zero-fills them); their logits
 // are masked to -inf, so they contribute p = 0 everywhere.
-template <int BITS, int ROWS, int G, int FMT, class Loader>
+// FOLD4 (integer codes): the four groups' products are formed before one query-scaling
+// branch and then folded (the warp-tile kernel); otherwise group by group, each with its
+// own branch (the persistent pipeline, whose register budget favours it).  Both give the
+// same arithmetic.
+template <int BITS, int ROWS, int G, int FMT, bool FOLD4 = true, class Loader>
 __device__ __forceinline__ void tile_compute(const Loader &ld, int nr, int lane,
                                              const uint32_t (&qb)[4][2][2], const uint32_t (&qbb)[4][2][2],
                                              const float (&qs)[2][4], const float (&qinv)[2][4], bool qscaled,
@@ -51,7 +55,7 @@ __device__ __forceinline__ void tile_compute(const Loader &ld, int nr, int lane,
             qk_group_fp<BITS, 1>(x, k0, k1, qb, qinv, qscaled, ka, kc, tig);
             qk_group_fp<BITS, 2>(x, k0, k1, qb, qinv, qscaled, ka, kc, tig);
             qk_group_fp<BITS, 3>(x, k0, k1, qb, qinv, qscaled, ka, kc, tig);
-        } else if constexpr (BITS < 16) {
+        } else if constexpr (BITS < 16 && FOLD4) {
             // the four groups' products first, one branch for the (rare) query scale, then
             // the folds in group order (the same arithmetic as qk_group, group by group)
             load_meta(ld.k_meta(0), km0);
@@ -76,6 +80,10 @@ __device__ __forceinline__ void tile_compute(const Loader &ld, int nr, int lane,
                 x[3] = fmaf(km1[grp].x, acc[grp][3], fmaf(km1[grp].y, qs[1][grp], x[3]));
             }
         } else {
+            if constexpr (BITS < 16) {
+                load_meta(ld.k_meta(0), km0);
+                load_meta(ld.k_meta(1), km1);
+            }
             qk_group<BITS, 0>(x, k0, k1, qb, qbb, qs, qinv, qscaled, km0, km1, magic);
             qk_group<BITS, 1>(x, k0, k1, qb, qbb, qs, qinv, qscaled, km0, km1, magic);
             qk_group<BITS, 2>(x, k0, k1, qb, qbb, qs, qinv, qscaled, km0, km1, magic);
