@@ -229,8 +229,10 @@ TKV_API tkv_status tkv_decode_attention(tkv_cache *cache, const void *q, float s
  * int32 [B]) followed by tkv_decode_attention (q, softmax_scale, out as there),
  * so the step attends over the new token too, in one call: the two launches go
  * back to back, the attention's launch overlapping the append (programmatic
- * dependent launch).  Results, device errors and the cache state are those of the
- * two calls.  The ThinKV page's decode loop (Implementacao do Sistema) writes each
+ * dependent launch; the attention reads q while the append runs, which is safe for
+ * any q the caller's earlier work on `stream` produced, since the append starts
+ * only after that work).  Results, device errors and the cache state are those of
+ * the two calls.  The ThinKV page's decode loop (Implementacao do Sistema) writes each
  * new token into the block table the same step reads.
  * Returns TKV_ERR_INVALID (launching nothing) for a NULL pointer or k, v, pos, q,
  * out not 16-byte aligned.
